@@ -1,0 +1,213 @@
+/*
+ * stca.h - C ABI of libstca: forward pass of stacked target-to-history cross
+ * attention (STCA) and two related target-attention forms, on one NVIDIA B200.
+ *
+ * Sources for what is computed (page title, section / equation):
+ *   [notes]   "超长序列建模 —— STCA 精读笔记" (wln20.github.io): problem statement,
+ *             sections "STCA" and "Request Level Batching（RLB）".
+ *   [review]  "Make It Long, Keep It Fast" paper review (xllm-io.github.io):
+ *             §三 核心公式 and the architecture tree; §四 table (SwiGLU FFN, time gap).
+ *   [wechat]  "视频号推荐超长序列技术演进" (dingyadong.top): §1.1 distributed TA
+ *             (local attention, then merge) and the low-memory TA operator (lookup
+ *             fused with attention); §1.2 element-wise ReLU scores.
+ *   [hyformer] "HyFormer：重新审视序列建模和特征交互在 CTR 预测中的作用"
+ *             (gitcode.csdn.net): §3.4-3.7, eq (7)-(16).
+ *
+ * Conventions for every entry point:
+ *   - All tensors are row-major and dense.  Weight matrices are [in, out] and act as
+ *     y = x W ([review] 核心公式 writes q W_Q and X~ W_K).  Head h of a d-wide
+ *     projection is columns [h*d/H, (h+1)*d/H).
+ *   - "dtype" tensors are float32 for STCA_FP32 and bfloat16 for STCA_BF16.  LayerNorm
+ *     gamma/beta are always float32.  Outputs are always float32.
+ *   - Pointers are DEVICE pointers unless the entry point's name ends in _host.  The
+ *     caller owns every buffer; the library never frees or keeps them past the call.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream) and
+ *     is asynchronous.  Argument errors are detected on the host before anything is
+ *     launched and returned synchronously.  Errors the GPU detects (an item id outside
+ *     [0, n_items), lengths that do not add up, a bounded wait that ran out) are
+ *     recorded in the handle's device error word; the kernels never trap and keep
+ *     going, and outputs are then undefined.  stca_sync_status() reads and clears it.
+ *   - A handle is not thread-safe; use one handle per host thread or serialise calls.
+ */
+#ifndef STCA_H
+#define STCA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define STCA_MAX_LAYERS 8
+#define STCA_MAX_QUERY_TOKENS 64
+
+enum stca_status {
+  STCA_OK = 0,
+  STCA_ERR_INVALID_ARG = 1,      /* null pointer, bad size, inconsistent counts */
+  STCA_ERR_UNSUPPORTED = 2,      /* configuration outside what the kernels implement */
+  STCA_ERR_CAPACITY = 3,         /* a size above the handle's max_* limits */
+  STCA_ERR_CUDA = 4,             /* a CUDA runtime/driver call failed */
+  STCA_ERR_ID_OUT_OF_RANGE = 5,  /* device: an item id outside [0, n_items) (row read as 0) */
+  STCA_ERR_TIMEOUT = 6,          /* device: a bounded wait ran out */
+  STCA_ERR_BAD_LENGTHS = 7       /* device: negative lengths or a sum != n_tok / t_tot */
+};
+
+enum stca_dtype { STCA_FP32 = 0, STCA_BF16 = 1 };
+/* Which entry point a handle serves; stca_create sizes the workspace for it. */
+enum stca_mode { STCA_MODE_STCA = 0, STCA_MODE_POINTWISE = 1, STCA_MODE_HYFORMER = 2 };
+enum stca_score { STCA_SOFTMAX = 0, STCA_RELU = 1 };
+
+/* Model shape and capacity.  mode: enum stca_mode.  M layers (or HyFormer blocks), model width d, H heads (d_h = d/H, which must be
+ * 32 for STCA_FP32 or 64 for STCA_BF16 in this build), SwiGLU hidden width `hidden`.
+ * time_buckets: 0, or 16 for the time-difference feature of [review] §四.
+ * max_users / max_tokens / max_targets bound B, n_tok and t_tot of every later call;
+ * stca_create sizes all device workspace from them, and later calls allocate nothing. */
+typedef struct {
+  int mode;         /* enum stca_mode */
+  int M, d, H, hidden;
+  int dtype;        /* enum stca_dtype */
+  int score;        /* enum stca_score */
+  int time_buckets; /* 0 or 16 */
+  int max_users, max_tokens, max_targets;
+  float ln_eps;     /* LayerNorm epsilon (biased variance) */
+} stca_config;
+
+/* One SwiGLU FFN, SwiGLU(x) = (SiLU(x W1) * (x W3)) W2 (the "dimension-preserving"
+ * SwiGLU FFN of [review] §四), optionally followed by LayerNorm.
+ * W1, W3: [d, hidden] dtype;  W2: [hidden, d] dtype;  gamma, beta: [d] float32 or NULL
+ * where the block has no LayerNorm. */
+typedef struct {
+  const void* W1;
+  const void* W3;
+  const void* W2;
+  const float* gamma;
+  const float* beta;
+} stca_ffn;
+
+/* STCA weights ([notes] STCA, [review] 核心公式).  Layer index i = 0..M-1.
+ *   table    E [n_items, d] dtype              item embedding table
+ *   dt_table T [16, d] dtype or NULL           time-difference bucket embeddings
+ *   hist[i]  history SwiGLU + LN of layer i (X~^(i) from the ORIGINAL X)
+ *   WQ/WK/WV/WO[i] [d, d] dtype
+ *   tgt      target-side SwiGLU + LN of layer 1 (q^(1) = LN(SwiGLU(x_t)))
+ *   WC[i]    for i = 1..M-1: [(i+1) d, d] dtype, fusion input of layer i+1
+ *            (rows [0, i*d) multiply o^(1..i), rows [i*d, (i+1)d) multiply x_t)
+ *   fuse[i]  for i = 1..M-1: SwiGLU + LN of the fusion into q^(i+1)
+ *   WZ       [(M+1) d, d] dtype;  zffn: SwiGLU without LN, z = SwiGLU_Z([o|x_t] WZ) */
+typedef struct {
+  const void* table;
+  int64_t n_items;
+  const void* dt_table;
+  stca_ffn hist[STCA_MAX_LAYERS];
+  const void* WQ[STCA_MAX_LAYERS];
+  const void* WK[STCA_MAX_LAYERS];
+  const void* WV[STCA_MAX_LAYERS];
+  const void* WO[STCA_MAX_LAYERS];
+  stca_ffn tgt;
+  const void* WC[STCA_MAX_LAYERS];
+  stca_ffn fuse[STCA_MAX_LAYERS];
+  const void* WZ;
+  stca_ffn zffn;
+} stca_weights;
+
+typedef struct stca_handle stca_handle;
+
+/* Validates the configuration and allocates every device buffer later calls need
+ * (workspace, error word).  Returns STCA_ERR_UNSUPPORTED for shapes the kernels do not
+ * implement (bf16: d in {256, 512} with d_h = 64 and hidden a multiple of 128 up to
+ * 1024; fp32: d_h = 32, d <= 1024), STCA_ERR_CUDA if allocation fails.  On error *out
+ * is set to NULL and nothing is leaked. */
+int stca_create(const stca_config* cfg, stca_handle** out);
+
+/* STCA forward for B users and their targets (Request-Level Batching, [notes] RLB:
+ * each user's per-layer K/V is computed once and serves all of that user's targets).
+ *   hist_ids         [n_tok] int32   item ids of all histories, user after user
+ *   hist_lengths     [B] int32       L_u >= 0; sum = n_tok
+ *   hist_dt          [n_tok] int32   time differences >= 0 (seconds), or NULL when the
+ *                                    handle has time_buckets == 0 (must be non-NULL
+ *                                    otherwise)
+ *   target_emb       [t_tot, d] dtype  x_t of every target, user after user
+ *   targets_per_user [B] int32       m_u >= 0; sum = t_tot
+ *   z_out            [t_tot, d] float32  z of every target
+ *   o_out            [M, t_tot, d] float32 per-layer o^(i), or NULL
+ * A user with L_u = 0 gets o_h = 0 in every head.  Device-side checks: ids in range,
+ * lengths non-negative and summing to n_tok / t_tot. */
+int stca_forward(stca_handle* h, const int32_t* hist_ids, const int32_t* hist_lengths,
+                 const int32_t* hist_dt, const void* target_emb, const int32_t* targets_per_user,
+                 int B, int n_tok, int t_tot, const stca_weights* w, float* z_out, float* o_out,
+                 void* stream);
+
+/* stca_forward with the per-request inputs and the output in HOST memory (pinned memory
+ * makes the copies asynchronous): the library copies the inputs into its workspace,
+ * runs the forward on `stream` and copies z back.  Weights and the table stay device
+ * pointers.  Returns after enqueueing; synchronise `stream` before reading z_out_host. */
+int stca_forward_host(stca_handle* h, const int32_t* hist_ids_host, const int32_t* hist_lengths_host,
+                      const int32_t* hist_dt_host, const void* target_emb_host,
+                      const int32_t* targets_per_user_host, int B, int n_tok, int t_tot,
+                      const stca_weights* w, float* z_out_host, void* stream);
+
+/* Pointwise ReLU target attention with fused lookup ([wechat] §1.1 low-memory TA
+ * operator, §1.2 ReLU scores): for each sample b,
+ *   out[b] = sum_{j < L_b} relu(q_b . e_j / sqrt(D)) e_j,   e_j = table[ids_b[j]]
+ * Keys and values are the looked-up rows themselves; the gathered [B, L, D] matrix is
+ * never written.  Handle: dtype STCA_BF16, d = D = 128 (the only width in this build),
+ * max_users >= B, max_tokens >= n_tok.
+ *   ids [n_tok] int32, lengths [B] int32, q [B, D] bf16, table [n_items, D] bf16,
+ *   out [B, D] float32. */
+int stca_pointwise_forward(stca_handle* h, const int32_t* ids, const int32_t* lengths, const void* q,
+                           const void* table, int64_t n_items, int B, int n_tok, float* out,
+                           void* stream);
+
+/* Multi-query multi-sequence decode ([hyformer] §3.4-3.7).  Two sequences per user
+ * (s = 0 "feed", s = 1 "search"), each with n_query query tokens.  Per block l and
+ * sequence s: H = SwiGLU_{l,s}(X_s) (eq 7), K,V = H W_K, H W_V (eq 8), decoded queries
+ * = multi-head CrossAttn(Q_s W_Q, K, V) W_O (eq 9/16).  Then Q = [Q^_0; Q^_1]
+ * (T = 2 n_query tokens, eq 10), token mixing (eq 11-13), a per-token SwiGLU per token
+ * index (eq 14) and the residual Q + Q~ (eq 15) give the next block's queries.
+ * Handle: dtype STCA_BF16, d = 512, H = 8, hidden = 1024 in this build; M = number of
+ * blocks; max_users >= B; max_tokens >= max(n_feed, n_search); max_targets >=
+ * B * 2 * n_query.  T must divide d. */
+typedef struct {
+  stca_ffn ffn; /* W1, W3, W2 only (no LayerNorm, eq 7) */
+  const void* WQ;
+  const void* WK;
+  const void* WV;
+  const void* WO;
+} hyf_seq_weights;
+
+typedef struct {
+  hyf_seq_weights seq[2];
+  stca_ffn tok[STCA_MAX_QUERY_TOKENS]; /* per-token SwiGLU, token index 0..T-1 */
+} hyf_block_weights;
+
+typedef struct {
+  const void* table;
+  int64_t n_items;
+  int blocks;
+  hyf_block_weights blk[STCA_MAX_LAYERS];
+} hyf_weights;
+
+/*   ids_feed [n_feed] int32, len_feed [B] int32, ids_search [n_search], len_search [B],
+ *   q0 [B, 2*n_query, d] bf16 (rows 0..n_query-1 query sequence 0), out [B, 2*n_query, d]
+ *   float32. */
+int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len_feed, int n_feed,
+                     const int32_t* ids_search, const int32_t* len_search, int n_search,
+                     const void* q0, int B, int n_query, const hyf_weights* w, float* out,
+                     void* stream);
+
+/* Synchronises the stream of the handle's last call, then returns and clears the device
+ * error word (STCA_OK if no error was recorded), or STCA_ERR_CUDA. */
+int stca_sync_status(stca_handle* h);
+
+/* Static description of a status code. */
+const char* stca_strerror(int code);
+
+/* Frees the handle's device memory.  NULL is a no-op. */
+void stca_destroy(stca_handle* h);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STCA_H */

@@ -1,0 +1,60 @@
+/*
+ * stca_kernels.h - kernel-level entry points of libstca.  Each runs one step of the
+ * forward passes declared in stca.h, on caller-provided device buffers, so that a step
+ * can be checked on its own.  The same conventions hold (row-major, device pointers,
+ * asynchronous on `stream`, int status, device-detected errors recorded in `err`, a
+ * device int32 the caller zeroes and reads).  Nothing here allocates.
+ */
+#ifndef STCA_KERNELS_H
+#define STCA_KERNELS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Ragged layout ([notes] problem statement: one history of length L_u per user; RLB:
+ * targets grouped per user).  offsets[0] = 0, offsets[i+1] = offsets[i] + lengths[i]
+ * ([B+1] int32); records STCA_ERR_BAD_LENGTHS in err for a negative length or a total
+ * different from `expected`. */
+int stca_k_offsets(const int32_t* lengths, int B, int32_t* offsets, int expected, int32_t* err, void* stream);
+
+/* Packs a bf16 weight W [K, N] (row-major, y = x W) into the K-major operand layout of
+ * the tensor-core GEMMs: mode 0 writes column n to row row_offset + n of dst [rows, K];
+ * modes 1 / 2 write W1 / W3 of a SwiGLU into the gate / up halves of 256-row groups
+ * (row (n/128)*256 + n%128, plus 128 for mode 2). */
+int stca_k_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_offset, void* stream);
+
+/* Tensor-core GEMM with A resident in shared memory (K = 256 or 512), bf16 in, fp32
+ * accumulate, bf16 out C [M, ldc]:
+ *   amode 0: A dense [M, K];  amode 1: A row r = table[ids[r]] (+ dt_table[b(dt[r])]),
+ *   b(x) = min(15, floor(log2(x + 1))): the fused embedding gather ([wechat] §1.1
+ *   "lookup while computing"; time feature of [review] §四).
+ *   epi 0: C = A Wp^T (Wp packed mode 0, [Nout, K], Nout % 256 == 0)
+ *   epi 1: C = SiLU(A W1) * (A W3) (Wp packed modes 1+2, [2 Nout, K], Nout % 128 == 0).
+ * An id outside [0, n_items) reads as a zero row and records STCA_ERR_ID_OUT_OF_RANGE. */
+int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, const int32_t* dt, const void* table,
+                         const void* dt_table, int64_t n_items, int M, int K, const void* Wp, int Nout, void* C,
+                         int ldc, int32_t* err, void* stream);
+
+/* Tensor-core GEMM with A streamed (K % 64 == 0) and the full output row (N = 256 or
+ * 512) in tensor memory: epi 0 plain, epi 2 LayerNorm(gamma, beta, eps) of each row
+ * ([notes] STCA: X~ = LN(SwiGLU(X))).  C [M, ldc] bf16. */
+int stca_k_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
+                        const float* beta, float eps, void* C, int ldc, int32_t* err, void* stream);
+
+/* Split-L cross attention plus merge ([review] 核心公式; [wechat] §1.1 local attention,
+ * then merge; §1.2 ReLU scores).  Q [T, d] fp32 projected queries, KV [N, 2d] (K in
+ * columns [0, d), V in [d, 2d)) bf16 when kv_bf16 else fp32, hoff/toff [B+1] offsets of
+ * the users' keys and queries.  score 0 softmax, 1 relu.  part_acc [splits, T, d] and
+ * part_ml [splits, T, H, 2] float32 scratch; out [T, d] float32. */
+int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B,
+                     int T, int d, int H, int splits, int score, float* part_acc, float* part_ml, float* out,
+                     int32_t* err, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STCA_KERNELS_H */

@@ -1,0 +1,202 @@
+"""ctypes binding of libstca (include/stca.h, include/stca_kernels.h).
+
+Argument marshalling only: every computation runs inside libstca's CUDA kernels.  The
+functions keep the C names and take torch tensors (device pointers) plus a CUDA stream;
+they return the C status code.  Loading fails loudly when libstca.so is missing: there
+is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libstca.so")
+
+MAX_LAYERS = 8
+MAX_QUERY_TOKENS = 64
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_ID_OUT_OF_RANGE, ERR_TIMEOUT, \
+    ERR_BAD_LENGTHS = range(8)
+FP32, BF16 = 0, 1
+SOFTMAX, RELU = 0, 1
+MODE_STCA, MODE_POINTWISE, MODE_HYFORMER = 0, 1, 2
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int
+_i64 = ctypes.c_int64
+
+
+class StcaConfig(ctypes.Structure):
+    _fields_ = [("mode", _i32), ("M", _i32), ("d", _i32), ("H", _i32), ("hidden", _i32),
+                ("dtype", _i32), ("score", _i32), ("time_buckets", _i32), ("max_users", _i32),
+                ("max_tokens", _i32), ("max_targets", _i32), ("ln_eps", ctypes.c_float)]
+
+
+class StcaFfn(ctypes.Structure):
+    _fields_ = [("W1", _vp), ("W3", _vp), ("W2", _vp), ("gamma", _vp), ("beta", _vp)]
+
+
+class StcaWeights(ctypes.Structure):
+    _fields_ = [("table", _vp), ("n_items", _i64), ("dt_table", _vp),
+                ("hist", StcaFfn * MAX_LAYERS), ("WQ", _vp * MAX_LAYERS), ("WK", _vp * MAX_LAYERS),
+                ("WV", _vp * MAX_LAYERS), ("WO", _vp * MAX_LAYERS), ("tgt", StcaFfn),
+                ("WC", _vp * MAX_LAYERS), ("fuse", StcaFfn * MAX_LAYERS), ("WZ", _vp), ("zffn", StcaFfn)]
+
+
+class HyfSeqWeights(ctypes.Structure):
+    _fields_ = [("ffn", StcaFfn), ("WQ", _vp), ("WK", _vp), ("WV", _vp), ("WO", _vp)]
+
+
+class HyfBlockWeights(ctypes.Structure):
+    _fields_ = [("seq", HyfSeqWeights * 2), ("tok", StcaFfn * MAX_QUERY_TOKENS)]
+
+
+class HyfWeights(ctypes.Structure):
+    _fields_ = [("table", _vp), ("n_items", _i64), ("blocks", _i32),
+                ("blk", HyfBlockWeights * MAX_LAYERS)]
+
+
+class StcaError(RuntimeError):
+    def __init__(self, code, what=""):
+        self.code = code
+        super().__init__(f"{what}: libstca status {code} ({strerror(code)})")
+
+
+_LIB = None
+
+# (name, restype, argtypes)
+_SIGS = [
+    ("stca_create", _i32, [ctypes.POINTER(StcaConfig), ctypes.POINTER(_vp)]),
+    ("stca_destroy", None, [_vp]),
+    ("stca_forward", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.POINTER(StcaWeights), _vp, _vp,
+                            _vp]),
+    ("stca_forward_host", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.POINTER(StcaWeights), _vp,
+                                 _vp]),
+    ("stca_pointwise_forward", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp]),
+    ("hyformer_forward", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, ctypes.POINTER(HyfWeights),
+                                _vp, _vp]),
+    ("stca_sync_status", _i32, [_vp]),
+    ("stca_strerror", ctypes.c_char_p, [_i32]),
+    ("stca_k_offsets", _i32, [_vp, _i32, _vp, _i32, _vp, _vp]),
+    ("stca_k_pack_weight", _i32, [_vp, _i32, _i32, _vp, _i32, _i32, _vp]),
+    ("stca_k_gemm_resident", _i32, [_i32, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _i32, _vp, _i32, _vp,
+                                    _vp]),
+    ("stca_k_gemm_rowwise", _i32, [_i32, _vp, _i32, _i32, _vp, _i32, _vp, _vp, ctypes.c_float, _vp, _i32, _vp, _vp]),
+    ("stca_k_attention", _i32, [_i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
+                                _vp]),
+]
+
+EXPORTED = [s[0] for s in _SIGS]
+
+
+def lib():
+    """The loaded libstca (built in-tree by ``target_attention_b200.build``)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libstca.so is not built ({LIB_PATH}); run "
+                               "`python -m target_attention_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, res, args in _SIGS:
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def strerror(code: int) -> str:
+    try:
+        return lib().stca_strerror(code).decode()
+    except RuntimeError:
+        return "?"
+
+
+def ptr(t):
+    """Device (or host) address of a tensor, or None."""
+    return None if t is None else t.data_ptr()
+
+
+def stream_ptr(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def check(rc, what=""):
+    if rc != OK:
+        raise StcaError(rc, what)
+    return rc
+
+
+# --------------------------------------------------------------------------- handles
+
+
+def stca_create(cfg: StcaConfig):
+    h = _vp()
+    check(lib().stca_create(ctypes.byref(cfg), ctypes.byref(h)), "stca_create")
+    return h
+
+
+def stca_destroy(h):
+    lib().stca_destroy(h)
+
+
+def stca_sync_status(h) -> int:
+    return lib().stca_sync_status(h)
+
+
+# --------------------------------------------------------------------------- forwards
+
+
+def stca_forward(h, ids, lengths, dt, x_t, tpu, B, n_tok, t_tot, weights: StcaWeights, z_out, o_out=None,
+                 stream=None) -> int:
+    return lib().stca_forward(h, ptr(ids), ptr(lengths), ptr(dt), ptr(x_t), ptr(tpu), B, n_tok, t_tot,
+                              ctypes.byref(weights), ptr(z_out), ptr(o_out), stream_ptr(stream))
+
+
+def stca_forward_host(h, ids, lengths, dt, x_t, tpu, B, n_tok, t_tot, weights: StcaWeights, z_out,
+                      stream=None) -> int:
+    return lib().stca_forward_host(h, ptr(ids), ptr(lengths), ptr(dt), ptr(x_t), ptr(tpu), B, n_tok, t_tot,
+                                   ctypes.byref(weights), ptr(z_out), stream_ptr(stream))
+
+
+def stca_pointwise_forward(h, ids, lengths, q, table, n_items, B, n_tok, out, stream=None) -> int:
+    return lib().stca_pointwise_forward(h, ptr(ids), ptr(lengths), ptr(q), ptr(table), n_items, B, n_tok, ptr(out),
+                                        stream_ptr(stream))
+
+
+def hyformer_forward(h, ids_feed, len_feed, n_feed, ids_search, len_search, n_search, q0, B, n_query,
+                     weights: HyfWeights, out, stream=None) -> int:
+    return lib().hyformer_forward(h, ptr(ids_feed), ptr(len_feed), n_feed, ptr(ids_search), ptr(len_search),
+                                  n_search, ptr(q0), B, n_query, ctypes.byref(weights), ptr(out),
+                                  stream_ptr(stream))
+
+
+# --------------------------------------------------------------------------- kernel-level
+
+
+def stca_k_offsets(lengths, B, offsets, expected, err, stream=None) -> int:
+    return lib().stca_k_offsets(ptr(lengths), B, ptr(offsets), expected, ptr(err), stream_ptr(stream))
+
+
+def stca_k_pack_weight(W, K, N, dst, mode, row_offset, stream=None) -> int:
+    return lib().stca_k_pack_weight(ptr(W), K, N, ptr(dst), mode, row_offset, stream_ptr(stream))
+
+
+def stca_k_gemm_resident(amode, epi, A, ids, dt, table, dt_table, n_items, M, K, Wp, Nout, C, ldc, err,
+                         stream=None) -> int:
+    return lib().stca_k_gemm_resident(amode, epi, ptr(A), ptr(ids), ptr(dt), ptr(table), ptr(dt_table), n_items, M,
+                                      K, ptr(Wp), Nout, ptr(C), ldc, ptr(err), stream_ptr(stream))
+
+
+def stca_k_gemm_rowwise(epi, A, M, K, Wp, N, gamma, beta, eps, C, ldc, err, stream=None) -> int:
+    return lib().stca_k_gemm_rowwise(epi, ptr(A), M, K, ptr(Wp), N, ptr(gamma), ptr(beta), eps, ptr(C), ldc,
+                                     ptr(err), stream_ptr(stream))
+
+
+def stca_k_attention(kv_bf16, Q, KV, hoff, toff, B, T, d, H, splits, score, part_acc, part_ml, out, err,
+                     stream=None) -> int:
+    return lib().stca_k_attention(kv_bf16, ptr(Q), ptr(KV), ptr(hoff), ptr(toff), B, T, d, H, splits, score,
+                                  ptr(part_acc), ptr(part_ml), ptr(out), ptr(err), stream_ptr(stream))

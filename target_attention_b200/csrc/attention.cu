@@ -1,0 +1,472 @@
+// Split-L few-query cross attention with Request-Level Batching.
+//
+// For one user u, one head h and one slice c of the user's keys, every target of u
+// (all m_u queries at once, so each K/V row is read once for all of them: RLB, STCA
+// notes "Request Level Batching") produces a local state over the slice:
+//   softmax: mx = max_j s_j, l = sum_j 2^(s_j - mx), acc = sum_j 2^(s_j - mx) v_j
+//   relu:    acc = sum_j relu(s_j) v_j
+// with s_j = q.k_j / sqrt(d_h) (scores kept in log2 units for the softmax form).
+// The merge kernel combines the slices (WeChat TA article §1.1: items of a sequence do
+// not interact, so local attention results can be merged):
+//   softmax: M = max_c mx_c, o = sum_c 2^(mx_c - M) acc_c / sum_c 2^(mx_c - M) l_c
+//   relu:    o = sum_c acc_c
+// An empty key set gives o = 0.
+#include "common.cuh"
+#include "internal.h"
+
+namespace stca {
+
+namespace {
+
+constexpr float LOG2E = 1.4426950408889634f;
+
+__device__ __forceinline__ void slice_bounds(const AttnArgs& a, int u, int s, int64_t& k0, int& nk, int& t0, int& m) {
+  const int h0 = a.hoff[u], h1 = a.hoff[u + 1];
+  const int64_t L = h1 - h0;
+  k0 = h0 + (L * s) / a.splits;
+  const int64_t k1 = h0 + (L * (s + 1)) / a.splits;
+  nk = int(k1 - k0);
+  t0 = a.toff[u];
+  m = a.toff[u + 1] - t0;
+}
+
+// ------------------------------------------------------------------------------------
+// bf16 K/V, d_h = 64, tensor-core (mma.sync m16n8k16) scores and P V.
+
+constexpr int DH = 64;
+constexpr int KT = 32;                    // keys per warp tile
+constexpr int TILE_BYTES = KT * DH * 2;   // 4 KB for K (same for V)
+constexpr int WARP_STAGE = 2 * TILE_BYTES;
+constexpr int WARP_BYTES = 2 * WARP_STAGE;   // double-buffered K+V: 16 KB
+constexpr int ATTN_SMEM = 4 * WARP_BYTES;    // 64 KB per CTA
+
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+// Issues the cp.async copies of K and V rows [key0, key0+32) of head h into one stage.
+__device__ __forceinline__ void load_kv_tile(uint8_t* stage, const bf16* KV, int64_t ld, int64_t row0, int valid,
+                                             int hcol, int d, int lane) {
+  uint8_t* sK = stage;
+  uint8_t* sV = stage + TILE_BYTES;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int idx = i * 32 + lane;
+    const int key = idx >> 3, ch = idx & 7;
+    const bool ok = key < valid;
+    const bf16* src = KV + (ok ? (row0 + key) * ld : 0) + hcol + ch * 8;
+    const int off = key * 128 + ((ch ^ (key & 7)) << 4);
+    cp_async_16(sK + off, src, ok ? 16u : 0u);
+    cp_async_16(sV + off, src + d, ok ? 16u : 0u);
+  }
+}
+
+template <int SCORE>
+__global__ void __launch_bounds__(128, 2) attn_bf16_kernel(AttnArgs a) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int u = blockIdx.x / a.splits, s = blockIdx.x % a.splits, h = blockIdx.y;
+  int64_t k0;
+  int nk, t0, m;
+  slice_bounds(a, u, s, k0, nk, t0, m);
+  if (m <= 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, tq = lane & 3;
+  const int d = a.d;
+  const int64_t ld = 2 * int64_t(d);
+  const int hcol = h * DH;
+  const bf16* KV = reinterpret_cast<const bf16*>(a.KV);
+  uint8_t* wbuf = smem + warp * WARP_BYTES;
+  const float qscale = (SCORE == 0 ? LOG2E : 1.0f) * rsqrtf(float(DH));
+  const int n_tiles = (nk + KT - 1) / KT;
+
+  for (int qp = 0; qp < m; qp += 32) {
+    const int mq = min(32, m - qp);
+    const int groups = mq > 16 ? 2 : 1;
+    // ---- query fragments (A operand), scaled, bf16
+    uint32_t qa[2][4][4];
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int row = gi * 16 + g + ((e & 1) ? 8 : 0);
+          const int col = kk * 16 + 2 * tq + ((e & 2) ? 8 : 0);
+          float x0 = 0.f, x1 = 0.f;
+          if (row < mq) {
+            const float* qrow = a.Q + int64_t(t0 + qp + row) * d + hcol + col;
+            x0 = qrow[0] * qscale;
+            x1 = qrow[1] * qscale;
+          }
+          qa[gi][kk][e] = pack_bf16x2(x0, x1);
+        }
+    float o[2][8][4];
+    float mrow[2][2], lrow[2][2];
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[gi][nt][e] = 0.f;
+      mrow[gi][0] = mrow[gi][1] = -INFINITY;
+      lrow[gi][0] = lrow[gi][1] = 0.f;
+    }
+
+    // ---- stream this warp's tiles: warp w takes tiles w, w+4, ...
+    int stage = 0;
+    int tile = warp;
+    if (tile < n_tiles) load_kv_tile(wbuf, KV, ld, k0 + int64_t(tile) * KT, min(KT, nk - tile * KT), hcol, d, lane);
+    cp_async_commit();
+    for (; tile < n_tiles; tile += 4) {
+      const int next = tile + 4;
+      if (next < n_tiles)
+        load_kv_tile(wbuf + (stage ^ 1) * WARP_STAGE, KV, ld, k0 + int64_t(next) * KT, min(KT, nk - next * KT),
+                     hcol, d, lane);
+      cp_async_commit();
+      cp_async_wait<1>();
+      __syncwarp();
+      const uint32_t sK = smem_u32(wbuf + stage * WARP_STAGE);
+      const uint32_t sV = sK + TILE_BYTES;
+      const int valid = min(KT, nk - tile * KT);
+
+      // S = Q K^T for 32 keys (4 n-tiles of 8)
+      float sacc[2][4][4];
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sacc[gi][j][e] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          const int key = j * 8 + (lane & 7);
+          const int ch = 4 * p + (lane >> 3);
+          uint32_t kb[4];
+          ldsm_x4(sK + key * 128 + ((ch ^ (key & 7)) << 4), kb);
+          mma_bf16_16816(sacc[0][j], qa[0][2 * p], kb[0], kb[1]);
+          mma_bf16_16816(sacc[0][j], qa[0][2 * p + 1], kb[2], kb[3]);
+          if (groups > 1) {
+            mma_bf16_16816(sacc[1][j], qa[1][2 * p], kb[0], kb[1]);
+            mma_bf16_16816(sacc[1][j], qa[1][2 * p + 1], kb[2], kb[3]);
+          }
+        }
+      }
+      // mask keys past the slice end, then scores -> weights
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int kidx = j * 8 + 2 * tq + (e & 1);
+            if (kidx >= valid) sacc[gi][j][e] = (SCORE == 0) ? -INFINITY : 0.f;
+          }
+        if (SCORE == 0) {
+#pragma unroll
+          for (int hr = 0; hr < 2; ++hr) {
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) mx = fmaxf(mx, fmaxf(sacc[gi][j][2 * hr], sacc[gi][j][2 * hr + 1]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float mnew = fmaxf(mrow[gi][hr], mx);
+            const float muse = (mnew == -INFINITY) ? 0.f : mnew;
+            const float corr = exp2f(mrow[gi][hr] - muse);
+            mrow[gi][hr] = mnew;
+            float sum = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float p0 = exp2f(sacc[gi][j][2 * hr] - muse);
+              const float p1 = exp2f(sacc[gi][j][2 * hr + 1] - muse);
+              sacc[gi][j][2 * hr] = p0;
+              sacc[gi][j][2 * hr + 1] = p1;
+              sum += p0 + p1;
+            }
+            lrow[gi][hr] = lrow[gi][hr] * corr + sum;
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+              o[gi][nt][2 * hr] *= corr;
+              o[gi][nt][2 * hr + 1] *= corr;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sacc[gi][j][e] = fmaxf(sacc[gi][j][e], 0.f);
+        }
+      }
+      // O += P V   (P as A fragments straight from the score accumulators)
+#pragma unroll
+      for (int kb = 0; kb < 2; ++kb) {
+        uint32_t pa[2][4];
+#pragma unroll
+        for (int gi = 0; gi < 2; ++gi) {
+          pa[gi][0] = pack_bf16x2(sacc[gi][2 * kb][0], sacc[gi][2 * kb][1]);
+          pa[gi][1] = pack_bf16x2(sacc[gi][2 * kb][2], sacc[gi][2 * kb][3]);
+          pa[gi][2] = pack_bf16x2(sacc[gi][2 * kb + 1][0], sacc[gi][2 * kb + 1][1]);
+          pa[gi][3] = pack_bf16x2(sacc[gi][2 * kb + 1][2], sacc[gi][2 * kb + 1][3]);
+        }
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          const int key = kb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int ch = 2 * np + (lane >> 4);
+          uint32_t vb[4];
+          ldsm_x4_t(sV + key * 128 + ((ch ^ (key & 7)) << 4), vb);
+          mma_bf16_16816(o[0][2 * np], pa[0], vb[0], vb[1]);
+          mma_bf16_16816(o[0][2 * np + 1], pa[0], vb[2], vb[3]);
+          if (groups > 1) {
+            mma_bf16_16816(o[1][2 * np], pa[1], vb[0], vb[1]);
+            mma_bf16_16816(o[1][2 * np + 1], pa[1], vb[2], vb[3]);
+          }
+        }
+      }
+      __syncwarp();
+      stage ^= 1;
+    }
+    cp_async_wait_all();
+
+    // ---- combine the four warps' states through shared memory
+    if (SCORE == 0) {
+#pragma unroll
+      for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          lrow[gi][hr] += __shfl_xor_sync(0xffffffffu, lrow[gi][hr], 1);
+          lrow[gi][hr] += __shfl_xor_sync(0xffffffffu, lrow[gi][hr], 2);
+        }
+    }
+    __syncthreads();
+    float* comb = reinterpret_cast<float*>(smem);        // [4 warps][32 rows][64]
+    float* cm = comb + 4 * 32 * DH;                        // [4][32]
+    float* cl = cm + 4 * 32;                               // [4][32]
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int row = gi * 16 + g + hr * 8;
+        float* dst = comb + (warp * 32 + row) * DH;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          dst[nt * 8 + 2 * tq] = o[gi][nt][2 * hr];
+          dst[nt * 8 + 2 * tq + 1] = o[gi][nt][2 * hr + 1];
+        }
+        if (tq == 0) {
+          cm[warp * 32 + row] = mrow[gi][hr];
+          cl[warp * 32 + row] = lrow[gi][hr];
+        }
+      }
+    __syncthreads();
+    {
+      const int row = threadIdx.x >> 2, seg = threadIdx.x & 3;
+      if (row < mq) {
+        const int t = t0 + qp + row;
+        float wgt[4];
+        float M = -INFINITY, Lsum = 0.f;
+        if (SCORE == 0) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) M = fmaxf(M, cm[w * 32 + row]);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const float mw = cm[w * 32 + row];
+            wgt[w] = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+            Lsum += wgt[w] * cl[w * 32 + row];
+          }
+        } else {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) wgt[w] = 1.f;
+        }
+        float* pacc = a.part_acc + (int64_t(s) * a.T + t) * d + hcol + seg * 16;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          float v = 0.f;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) v += wgt[w] * comb[(w * 32 + row) * DH + seg * 16 + c];
+          pacc[c] = v;
+        }
+        if (SCORE == 0 && seg == 0) {
+          float* pml = a.part_ml + ((int64_t(s) * a.T + t) * a.H + h) * 2;
+          pml[0] = M;
+          pml[1] = Lsum;
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// fp32 K/V (the fp32 configuration), SIMT; lane c holds dims c, c+32, ... of the head.
+
+template <int DPL, int SCORE>
+__global__ void __launch_bounds__(128) attn_f32_kernel(AttnArgs a) {
+  __shared__ float comb[4][DPL * 32 + 2];
+  const int u = blockIdx.x / a.splits, s = blockIdx.x % a.splits, h = blockIdx.y;
+  int64_t k0;
+  int nk, t0, m;
+  slice_bounds(a, u, s, k0, nk, t0, m);
+  if (m <= 0) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = a.d, dh = DPL * 32;
+  const int64_t ld = 2 * int64_t(d);
+  const float* KV = reinterpret_cast<const float*>(a.KV);
+  const float scale = (SCORE == 0 ? LOG2E : 1.0f) / sqrtf(float(dh));
+  for (int ti = 0; ti < m; ++ti) {
+    const int t = t0 + ti;
+    float q[DPL], acc[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      q[i] = a.Q[int64_t(t) * d + h * dh + lane + 32 * i] * scale;
+      acc[i] = 0.f;
+    }
+    float mx = -INFINITY, l = 0.f;
+    for (int j = warp; j < nk; j += 4) {
+      const float* krow = KV + (k0 + j) * ld + h * dh;
+      float sc = 0.f;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) sc += q[i] * krow[lane + 32 * i];
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) sc += __shfl_xor_sync(0xffffffffu, sc, off);
+      const float* vrow = krow + d;
+      if (SCORE == 0) {
+        const float mnew = fmaxf(mx, sc);
+        const float corr = exp2f(mx - mnew);
+        const float p = exp2f(sc - mnew);
+        l = l * corr + p;
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) acc[i] = acc[i] * corr + p * vrow[lane + 32 * i];
+        mx = mnew;
+      } else {
+        const float p = fmaxf(sc, 0.f);
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) acc[i] += p * vrow[lane + 32 * i];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) comb[warp][lane + 32 * i] = acc[i];
+    if (lane == 0) {
+      comb[warp][dh] = mx;
+      comb[warp][dh + 1] = l;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      float M = -INFINITY, wgt[4], Lsum = 0.f;
+      if (SCORE == 0) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, comb[w][dh]);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          wgt[w] = comb[w][dh] == -INFINITY ? 0.f : exp2f(comb[w][dh] - M);
+          Lsum += wgt[w] * comb[w][dh + 1];
+        }
+      } else {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) wgt[w] = 1.f;
+      }
+      float* pacc = a.part_acc + (int64_t(s) * a.T + t) * d + h * dh;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) v += wgt[w] * comb[w][lane + 32 * i];
+        pacc[lane + 32 * i] = v;
+      }
+      if (SCORE == 0 && lane == 0) {
+        float* pml = a.part_ml + ((int64_t(s) * a.T + t) * a.H + h) * 2;
+        pml[0] = M;
+        pml[1] = Lsum;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// merge of the per-slice states; one warp per (target, head)
+
+template <int SCORE>
+__global__ void attn_merge_kernel(AttnArgs a) {
+  const int64_t wid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= int64_t(a.T) * a.H) return;
+  const int t = int(wid / a.H), h = int(wid % a.H);
+  const int dh = a.d / a.H;
+  float M = -INFINITY;
+  if (SCORE == 0)
+    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[((int64_t(s) * a.T + t) * a.H + h) * 2]);
+  float Lsum = 0.f;
+  for (int c = lane; c < dh; c += 32) {
+    float v = 0.f;
+    Lsum = 0.f;
+    for (int s = 0; s < a.splits; ++s) {
+      float w = 1.f;
+      if (SCORE == 0) {
+        const float* ml = a.part_ml + ((int64_t(s) * a.T + t) * a.H + h) * 2;
+        w = (ml[0] == -INFINITY) ? 0.f : exp2f(ml[0] - M);
+        Lsum += w * ml[1];
+      }
+      v += w * a.part_acc[(int64_t(s) * a.T + t) * a.d + h * dh + c];
+    }
+    if (SCORE == 0) v = Lsum > 0.f ? v / Lsum : 0.f;
+    a.out[int64_t(t) * a.d + h * dh + c] = v;
+  }
+}
+
+}  // namespace
+
+int attention_bf16(const AttnArgs& a, cudaStream_t s) {
+  if (a.B == 0 || a.T == 0) return 0;
+  if (a.d / a.H != DH || a.d % a.H != 0) return STCA_ERR_UNSUPPORTED;
+  dim3 grid(a.B * a.splits, a.H);
+  if (a.score == 0) {
+    cudaFuncSetAttribute(attn_bf16_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_SMEM);
+    attn_bf16_kernel<0><<<grid, 128, ATTN_SMEM, s>>>(a);
+  } else {
+    cudaFuncSetAttribute(attn_bf16_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_SMEM);
+    attn_bf16_kernel<1><<<grid, 128, ATTN_SMEM, s>>>(a);
+  }
+  return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
+}
+
+int attention_f32(const AttnArgs& a, cudaStream_t s) {
+  if (a.B == 0 || a.T == 0) return 0;
+  const int dh = a.d / a.H;
+  dim3 grid(a.B * a.splits, a.H);
+#define STCA_F32(DPL)                                                    \
+  (a.score == 0 ? (attn_f32_kernel<DPL, 0><<<grid, 128, 0, s>>>(a), 0) \
+                : (attn_f32_kernel<DPL, 1><<<grid, 128, 0, s>>>(a), 0))
+  if (dh == 32) STCA_F32(1);
+  else if (dh == 64) STCA_F32(2);
+  else if (dh == 128) STCA_F32(4);
+  else return STCA_ERR_UNSUPPORTED;
+#undef STCA_F32
+  return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
+}
+
+int attention_merge(const AttnArgs& a, cudaStream_t s) {
+  if (a.T == 0) return 0;
+  const int64_t warps = int64_t(a.T) * a.H;
+  const int blocks = int((warps * 32 + 255) / 256);
+  if (a.score == 0) attn_merge_kernel<0><<<blocks, 256, 0, s>>>(a);
+  else attn_merge_kernel<1><<<blocks, 256, 0, s>>>(a);
+  return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
+}
+
+}  // namespace stca

@@ -1,0 +1,122 @@
+// Host-side launchers shared between the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace stca {
+
+// Rows of A read straight from an embedding table by item id ("lookup while
+// computing"): row r of A is table[ids[r]] (+ dt_table[bucket(dt[r])]).
+struct GatherSrc {
+  const int32_t* ids;
+  const int32_t* dt;      // may be null
+  const void* table;      // [n_items, K] (bf16 or fp32, the kernel's type)
+  const void* dt_table;   // [16, K] or null
+  int64_t n_items;
+};
+
+enum AMode { A_TMA = 0, A_GATHER = 1 };
+enum Epi { EPI_PLAIN = 0, EPI_SWIGLU = 1, EPI_LN = 2 };
+
+// ---------------------------------------------------------------- tcgen05 GEMMs (bf16)
+
+// Packs a [K, N] row-major bf16 weight into the K-major [rows, K] operand layout.
+// mode 0: dst row (row_offset + n)        <- column n
+// mode 1: SwiGLU gate half:  dst row (n/128)*256 + n%128       <- column n of W1
+// mode 2: SwiGLU up half:    dst row (n/128)*256 + 128 + n%128 <- column n of W3
+int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_offset, cudaStream_t s);
+
+// C[M, Nout] (bf16, row stride ldc) from A (resident in shared memory, K in {256, 512}):
+//   amode A_TMA: A is a dense bf16 [M, K] matrix; A_GATHER: rows gathered via `g`.
+//   epi EPI_PLAIN:  C = A Wp^T, Wp packed [N, K], N a multiple of 256, Nout = N
+//   epi EPI_SWIGLU: Wp packed gate/up interleaved [2*Nout, K], C = SiLU(A W1) * (A W3)
+int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int K, const void* Wp,
+                     int Nout, void* C, int ldc, int32_t* err, cudaStream_t s);
+
+// C[M, N] (bf16) = epi(A Wp^T), A dense bf16 [M, K] streamed (K a multiple of 64),
+// N in {256, 512}; epi EPI_LN applies LayerNorm (gamma, beta, eps) over the full row.
+int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
+                    const float* beta, float eps, void* C, int ldc, int32_t* err, cudaStream_t s);
+
+// ---------------------------------------------------------------- SIMT fp32 GEMMs
+
+constexpr int MAX_BATCH_PTRS = 64;
+
+template <typename TA, typename TB>
+struct SimtGemmArgs {
+  int M, N, K;
+  // A: logical row r lives at physical row ra = remap(r, a_grp, a_gstride, a_goff) with
+  // remap(r, g, s, o) = g ? (r / g) * s + o + r % g : r; column k at
+  // A[ra*lda + (k < ksplit ? k : k + kshift)].  When gather.ids != null, row r is
+  // table[ids[r]*K + k] (+ dt_table[bucket(dt[r])*K + k]) instead.
+  const TA* A;
+  int64_t lda;
+  int ksplit, kshift;
+  int a_grp, a_gstride, a_goff;
+  GatherSrc gather;
+  const TB* B;   // [K, N] row-major (ldb = N)
+  const TB* B2;  // second operand for the SwiGLU form SiLU(A B) * (A B2), or null
+  // per-batch operands (batch z uses Bz[z] / B2z[z] when Bz[0] != null)
+  const TB* Bz[MAX_BATCH_PTRS];
+  const TB* B2z[MAX_BATCH_PTRS];
+  float* C;      // logical row r at physical row remap(r, c_grp, c_gstride, c_goff)
+  int64_t ldc;
+  int c_grp, c_gstride, c_goff;
+  const float* R;  // residual added to the result, row m at R[m*ldr], or null
+  int64_t ldr;
+  // batch (grid z): element offsets of A, C and R per batch; B per batch via bsB or Bz
+  int64_t bsA, bsB, bsC, bsR;
+  int batch;
+  int32_t* err;
+};
+
+template <typename TA, typename TB>
+int simt_gemm(const SimtGemmArgs<TA, TB>& a, cudaStream_t s);
+
+// y = LayerNorm(x) row-wise over d columns, fp32; x and y may alias.
+int layer_norm_f32(const float* x, int64_t ldx, float* y, int64_t ldy, int rows, int d, const float* gamma,
+                   const float* beta, float eps, cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+
+struct AttnArgs {
+  const float* Q;       // [T, d] fp32 (projected queries)
+  const void* KV;       // [N, 2d]: K in columns [0, d), V in [d, 2d); bf16 or fp32
+  const int32_t* hoff;  // [B+1] history offsets
+  const int32_t* toff;  // [B+1] target offsets
+  int B, T, d, H, splits;
+  int score;            // 0 softmax, 1 relu
+  float* part_acc;      // [splits, T, d]
+  float* part_ml;       // [splits, T, H, 2]
+  float* out;           // [T, d]
+  int32_t* err;
+};
+int attention_bf16(const AttnArgs& a, cudaStream_t s);
+int attention_f32(const AttnArgs& a, cudaStream_t s);
+int attention_merge(const AttnArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- small kernels
+
+// offsets[0] = 0, offsets[i+1] = offsets[i] + lengths[i]; checks lengths >= 0 and the
+// total against `expected` (records STCA_ERR_BAD_LENGTHS otherwise).
+int exclusive_offsets(const int32_t* lengths, int B, int32_t* offsets, int expected, int32_t* err,
+                      cudaStream_t s);
+// dst[r, col0 + c] = float(src[r, c]) for c < d (src bf16 or fp32 by `src_bf16`).
+int copy_rows_to_f32(const void* src, int src_bf16, int rows, int d, float* dst, int64_t ldd, int col0,
+                     cudaStream_t s);
+
+// ---------------------------------------------------------------- pointwise ReLU TA
+
+int pointwise_relu_ta(const int32_t* ids, const int32_t* offsets, const void* q, const void* table,
+                      int64_t n_items, int B, int D, int splits, float* partials, float* out, int32_t* err,
+                      cudaStream_t s);
+
+// ---------------------------------------------------------------- query boosting
+
+// mixed[b, h, t*sub + j] = Q[b, t, h*sub + j], sub = d / T
+int token_mix(const float* Q, int B, int T, int d, float* mixed, cudaStream_t s);
+// out[i] = i * step for i in [0, n)
+int fill_arange(int32_t* out, int n, int step, cudaStream_t s);
+
+}  // namespace stca

@@ -1,0 +1,76 @@
+// Kernel-level C entry points (include/stca_kernels.h): thin wrappers over the launchers.
+#include <cstring>
+
+#include "../../include/stca_kernels.h"
+#include "common.cuh"
+#include "internal.h"
+
+using namespace stca;
+
+extern "C" {
+
+int stca_k_offsets(const int32_t* lengths, int B, int32_t* offsets, int expected, int32_t* err, void* stream) {
+  if (B < 0 || !offsets || (B > 0 && !lengths)) return STCA_ERR_INVALID_ARG;
+  return exclusive_offsets(lengths, B, offsets, expected, err, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int stca_k_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_offset, void* stream) {
+  if (!W || !dst || mode < 0 || mode > 2) return STCA_ERR_INVALID_ARG;
+  return tc_pack_weight(W, K, N, dst, mode, row_offset, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, const int32_t* dt, const void* table,
+                         const void* dt_table, int64_t n_items, int M, int K, const void* Wp, int Nout, void* C,
+                         int ldc, int32_t* err, void* stream) {
+  if (M < 0 || !Wp || (M > 0 && !C)) return STCA_ERR_INVALID_ARG;
+  if (epi != EPI_PLAIN && epi != EPI_SWIGLU) return STCA_ERR_INVALID_ARG;
+  GatherSrc g;
+  memset(&g, 0, sizeof(g));
+  if (amode == A_GATHER) {
+    if (M > 0 && (!ids || !table || n_items <= 0)) return STCA_ERR_INVALID_ARG;
+    g.ids = ids;
+    g.dt = dt_table ? dt : nullptr;
+    g.table = table;
+    g.dt_table = dt ? dt_table : nullptr;
+    g.n_items = n_items;
+  } else if (amode != A_TMA || (M > 0 && !A)) {
+    return STCA_ERR_INVALID_ARG;
+  }
+  return tc_gemm_resident(amode, epi, A, g, M, K, Wp, Nout, C, ldc, err, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int stca_k_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
+                        const float* beta, float eps, void* C, int ldc, int32_t* err, void* stream) {
+  if (M < 0 || (M > 0 && (!A || !C)) || !Wp) return STCA_ERR_INVALID_ARG;
+  if (epi != EPI_PLAIN && epi != EPI_LN) return STCA_ERR_INVALID_ARG;
+  return tc_gemm_rowwise(epi, A, M, K, Wp, N, gamma, beta, eps, C, ldc, err, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B,
+                     int T, int d, int H, int splits, int score, float* part_acc, float* part_ml, float* out,
+                     int32_t* err, void* stream) {
+  if (B < 0 || T < 0 || d <= 0 || H <= 0 || d % H != 0 || splits < 1 || (score != 0 && score != 1))
+    return STCA_ERR_INVALID_ARG;
+  if (B > 0 && T > 0 && (!Q || !KV || !hoff || !toff || !part_acc || !part_ml || !out)) return STCA_ERR_INVALID_ARG;
+  AttnArgs a;
+  a.Q = Q;
+  a.KV = KV;
+  a.hoff = hoff;
+  a.toff = toff;
+  a.B = B;
+  a.T = T;
+  a.d = d;
+  a.H = H;
+  a.splits = splits;
+  a.score = score;
+  a.part_acc = part_acc;
+  a.part_ml = part_ml;
+  a.out = out;
+  a.err = err;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int rc = kv_bf16 ? attention_bf16(a, s) : attention_f32(a, s);
+  if (rc != STCA_OK) return rc;
+  return attention_merge(a, s);
+}
+
+}  // extern "C"

@@ -1,0 +1,523 @@
+// C ABI of libstca: argument checks, the workspace, and the launch sequence of each
+// forward pass.  Every step of the path runs in this library's kernels; PyTorch (or any
+// other caller) only provides device memory and the stream.
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+using namespace stca;
+
+namespace {
+
+constexpr int MAX_SPLITS = 16;
+
+}  // namespace
+
+struct stca_handle {
+  stca_config cfg;
+  int device = 0;
+  cudaStream_t last_stream = nullptr;
+  std::vector<void*> allocs;
+  int32_t* err = nullptr;
+  int32_t *hoff = nullptr, *toff = nullptr, *hoff2 = nullptr;
+  // history side
+  void* wpack = nullptr;
+  size_t wpack_layer = 0;  // elements per layer (per sequence for the decode variant)
+  void *hidden = nullptr, *xt = nullptr, *kv = nullptr;
+  // query side
+  float *cat = nullptr, *qbuf = nullptr, *qproj = nullptr, *attn = nullptr, *tmp_h = nullptr, *tmp_d = nullptr;
+  float *part_acc = nullptr, *part_ml = nullptr;
+  float *hq = nullptr, *hqhat = nullptr, *hmix = nullptr;
+  // staging for the host-buffer entry point
+  int32_t *in_ids = nullptr, *in_len = nullptr, *in_dt = nullptr, *in_tpu = nullptr;
+  void* in_xt = nullptr;
+  float* out_z = nullptr;
+};
+
+namespace {
+
+#define CK(x)                      \
+  do {                             \
+    const int _rc = (x);           \
+    if (_rc != STCA_OK) return _rc; \
+  } while (0)
+
+template <typename T>
+bool dalloc(stca_handle* h, T** p, size_t bytes) {
+  void* q = nullptr;
+  if (bytes == 0) bytes = 16;
+  if (cudaMalloc(&q, bytes) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  h->allocs.push_back(q);
+  *p = reinterpret_cast<T*>(q);
+  return true;
+}
+
+void free_all(stca_handle* h) {
+  for (void* p : h->allocs) cudaFree(p);
+  h->allocs.clear();
+}
+
+int choose_splits(int64_t n_tok, int B, int per_split) {
+  if (B <= 0) return 1;
+  const int64_t avg = n_tok / B;
+  int64_t s = (avg + per_split - 1) / per_split;
+  if (s < 1) s = 1;
+  if (s > MAX_SPLITS) s = MAX_SPLITS;
+  return int(s);
+}
+
+int esize(const stca_config& c) { return c.dtype == STCA_BF16 ? 2 : 4; }
+
+int validate_config(const stca_config& c) {
+  if (c.M < 1 || c.M > STCA_MAX_LAYERS || c.d <= 0 || c.H <= 0 || c.max_users < 0 || c.max_tokens < 0 ||
+      c.max_targets < 0 || !(c.ln_eps >= 0.f))
+    return STCA_ERR_INVALID_ARG;
+  if (c.dtype != STCA_FP32 && c.dtype != STCA_BF16) return STCA_ERR_INVALID_ARG;
+  if (c.score != STCA_SOFTMAX && c.score != STCA_RELU) return STCA_ERR_INVALID_ARG;
+  if (c.time_buckets != 0 && c.time_buckets != 16) return STCA_ERR_UNSUPPORTED;
+  if (c.mode == STCA_MODE_POINTWISE) {
+    if (c.dtype != STCA_BF16 || c.d != 128) return STCA_ERR_UNSUPPORTED;
+    return STCA_OK;
+  }
+  if (c.hidden <= 0 || c.d % c.H != 0) return STCA_ERR_INVALID_ARG;
+  const int dh = c.d / c.H;
+  if (c.mode == STCA_MODE_HYFORMER) {
+    if (c.dtype != STCA_BF16 || c.score != STCA_SOFTMAX || c.d != 512 || dh != 64 || c.hidden % 128 != 0)
+      return STCA_ERR_UNSUPPORTED;
+    return STCA_OK;
+  }
+  if (c.mode != STCA_MODE_STCA) return STCA_ERR_INVALID_ARG;
+  if (c.dtype == STCA_BF16) {
+    if ((c.d != 256 && c.d != 512) || dh != 64 || c.hidden % 128 != 0) return STCA_ERR_UNSUPPORTED;
+  } else {
+    if ((dh != 32 && dh != 64 && dh != 128) || c.d > 1024) return STCA_ERR_UNSUPPORTED;
+  }
+  return STCA_OK;
+}
+
+int allocate(stca_handle* h) {
+  const stca_config& c = h->cfg;
+  const size_t U = size_t(c.max_users) + 1, N = size_t(c.max_tokens), T = size_t(c.max_targets);
+  const size_t d = size_t(c.d), hd = size_t(c.hidden);
+  bool ok = dalloc(h, &h->err, 4) && dalloc(h, &h->hoff, U * 4) && dalloc(h, &h->toff, U * 4);
+  if (!ok) return STCA_ERR_CUDA;
+  if (c.mode == STCA_MODE_POINTWISE) {
+    ok = dalloc(h, &h->part_acc, size_t(MAX_SPLITS) * c.max_users * d * 4);
+    return ok ? STCA_OK : STCA_ERR_CUDA;
+  }
+  const size_t E = esize(c);
+  const int nseq = c.mode == STCA_MODE_HYFORMER ? 2 : 1;
+  if (c.dtype == STCA_BF16) {
+    h->wpack_layer = 2 * hd * d + d * hd + 2 * d * d;
+    ok = ok && dalloc(h, &h->wpack, size_t(c.M) * nseq * h->wpack_layer * 2);
+  }
+  ok = ok && dalloc(h, &h->hidden, N * hd * E) && dalloc(h, &h->xt, N * d * E) && dalloc(h, &h->kv, N * 2 * d * E);
+  ok = ok && dalloc(h, &h->qproj, T * d * 4) && dalloc(h, &h->attn, T * d * 4) && dalloc(h, &h->tmp_h, T * hd * 4) &&
+       dalloc(h, &h->tmp_d, T * d * 4);
+  ok = ok && dalloc(h, &h->part_acc, size_t(MAX_SPLITS) * T * d * 4) &&
+       dalloc(h, &h->part_ml, size_t(MAX_SPLITS) * T * c.H * 2 * 4);
+  if (c.mode == STCA_MODE_STCA) {
+    ok = ok && dalloc(h, &h->cat, T * (c.M + 1) * d * 4) && dalloc(h, &h->qbuf, T * d * 4);
+    ok = ok && dalloc(h, &h->in_ids, N * 4) && dalloc(h, &h->in_len, U * 4) && dalloc(h, &h->in_tpu, U * 4) &&
+         dalloc(h, &h->in_xt, T * d * E) && dalloc(h, &h->out_z, T * d * 4);
+    if (c.time_buckets) ok = ok && dalloc(h, &h->in_dt, N * 4);
+  } else {
+    ok = ok && dalloc(h, &h->hoff2, U * 4) && dalloc(h, &h->hq, T * d * 4) && dalloc(h, &h->hqhat, T * d * 4) &&
+         dalloc(h, &h->hmix, T * d * 4);
+  }
+  return ok ? STCA_OK : STCA_ERR_CUDA;
+}
+
+template <typename TB>
+SimtGemmArgs<float, TB> gemm_args(int M, int N, int K, const float* A, int64_t lda, const void* B, float* C,
+                                  int64_t ldc, int32_t* err) {
+  SimtGemmArgs<float, TB> a;
+  memset(&a, 0, sizeof(a));
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.A = A;
+  a.lda = lda;
+  a.ksplit = K;
+  a.B = reinterpret_cast<const TB*>(B);
+  a.C = C;
+  a.ldc = ldc;
+  a.batch = 1;
+  a.err = err;
+  return a;
+}
+
+// out[rows, d] = SwiGLU(A) (then LayerNorm when ffn.gamma != null); A [rows, K=d] fp32.
+template <typename TB>
+int query_ffn(stca_handle* h, const float* A, int64_t lda, int rows, const stca_ffn& f, float* out, int64_t ldo,
+              cudaStream_t s) {
+  const int d = h->cfg.d, hd = h->cfg.hidden;
+  auto g = gemm_args<TB>(rows, hd, d, A, lda, f.W1, h->tmp_h, hd, h->err);
+  g.B2 = reinterpret_cast<const TB*>(f.W3);
+  CK(simt_gemm(g, s));
+  auto g2 = gemm_args<TB>(rows, d, hd, h->tmp_h, hd, f.W2, out, ldo, h->err);
+  CK(simt_gemm(g2, s));
+  if (f.gamma) CK(layer_norm_f32(out, ldo, out, ldo, rows, d, f.gamma, f.beta, h->cfg.ln_eps, s));
+  return STCA_OK;
+}
+
+bool ffn_ok(const stca_ffn& f, bool ln) { return f.W1 && f.W3 && f.W2 && (!ln || (f.gamma && f.beta)); }
+
+int check_weights(const stca_config& c, const stca_weights* w) {
+  if (!w || !w->table || w->n_items <= 0) return STCA_ERR_INVALID_ARG;
+  if (c.time_buckets && !w->dt_table) return STCA_ERR_INVALID_ARG;
+  if (!ffn_ok(w->tgt, true) || !w->WZ || !ffn_ok(w->zffn, false)) return STCA_ERR_INVALID_ARG;
+  for (int i = 0; i < c.M; ++i) {
+    if (!ffn_ok(w->hist[i], true) || !w->WQ[i] || !w->WK[i] || !w->WV[i] || !w->WO[i]) return STCA_ERR_INVALID_ARG;
+    if (i > 0 && (!w->WC[i] || !ffn_ok(w->fuse[i], true))) return STCA_ERR_INVALID_ARG;
+  }
+  return STCA_OK;
+}
+
+// Packs one layer's history weights into K-major operand order (bf16).
+int pack_layer(stca_handle* h, size_t slot, const stca_ffn& f, const void* WK, const void* WV, cudaStream_t s) {
+  const int d = h->cfg.d, hd = h->cfg.hidden;
+  bf16* base = reinterpret_cast<bf16*>(h->wpack) + slot * h->wpack_layer;
+  bf16* wp1 = base;                          // [2 hd, d]  gate/up interleaved
+  bf16* wp2 = base + size_t(2) * hd * d;     // [d, hd]
+  bf16* wp3 = wp2 + size_t(d) * hd;          // [2 d, d]   K rows then V rows
+  CK(tc_pack_weight(f.W1, d, hd, wp1, 1, 0, s));
+  CK(tc_pack_weight(f.W3, d, hd, wp1, 2, 0, s));
+  CK(tc_pack_weight(f.W2, hd, d, wp2, 0, 0, s));
+  CK(tc_pack_weight(WK, d, d, wp3, 0, 0, s));
+  CK(tc_pack_weight(WV, d, d, wp3, 0, d, s));
+  return STCA_OK;
+}
+
+// K/V of every history token for one layer: bf16 tensor-core path.
+int history_bf16(stca_handle* h, size_t slot, const GatherSrc& g, int n_tok, const float* gamma, const float* beta,
+                 cudaStream_t s) {
+  const int d = h->cfg.d, hd = h->cfg.hidden;
+  const bf16* base = reinterpret_cast<const bf16*>(h->wpack) + slot * h->wpack_layer;
+  const bf16* wp1 = base;
+  const bf16* wp2 = base + size_t(2) * hd * d;
+  const bf16* wp3 = wp2 + size_t(d) * hd;
+  GatherSrc none;
+  memset(&none, 0, sizeof(none));
+  CK(tc_gemm_resident(A_GATHER, EPI_SWIGLU, nullptr, g, n_tok, d, wp1, hd, h->hidden, hd, h->err, s));
+  CK(tc_gemm_rowwise(gamma ? EPI_LN : EPI_PLAIN, h->hidden, n_tok, hd, wp2, d, gamma, beta, h->cfg.ln_eps, h->xt, d,
+                     h->err, s));
+  CK(tc_gemm_resident(A_TMA, EPI_PLAIN, h->xt, none, n_tok, d, wp3, 2 * d, h->kv, 2 * d, h->err, s));
+  return STCA_OK;
+}
+
+// K/V of every history token for one layer: fp32 SIMT path.
+int history_f32(stca_handle* h, const GatherSrc& g, int n_tok, const stca_ffn& f, const void* WK, const void* WV,
+                cudaStream_t s) {
+  const int d = h->cfg.d, hd = h->cfg.hidden;
+  float* hid = reinterpret_cast<float*>(h->hidden);
+  float* xt = reinterpret_cast<float*>(h->xt);
+  float* kv = reinterpret_cast<float*>(h->kv);
+  auto a = gemm_args<float>(n_tok, hd, d, nullptr, d, f.W1, hid, hd, h->err);
+  a.B2 = reinterpret_cast<const float*>(f.W3);
+  a.gather = g;
+  CK(simt_gemm(a, s));
+  CK(simt_gemm(gemm_args<float>(n_tok, d, hd, hid, hd, f.W2, xt, d, h->err), s));
+  CK(layer_norm_f32(xt, d, xt, d, n_tok, d, f.gamma, f.beta, h->cfg.ln_eps, s));
+  CK(simt_gemm(gemm_args<float>(n_tok, d, d, xt, d, WK, kv, 2 * d, h->err), s));
+  CK(simt_gemm(gemm_args<float>(n_tok, d, d, xt, d, WV, kv + d, 2 * d, h->err), s));
+  return STCA_OK;
+}
+
+int run_attention(stca_handle* h, const float* Q, const int32_t* hoff, const int32_t* toff, int B, int T,
+                  int splits, int score, cudaStream_t s) {
+  AttnArgs a;
+  a.Q = Q;
+  a.KV = h->kv;
+  a.hoff = hoff;
+  a.toff = toff;
+  a.B = B;
+  a.T = T;
+  a.d = h->cfg.d;
+  a.H = h->cfg.H;
+  a.splits = splits;
+  a.score = score;
+  a.part_acc = h->part_acc;
+  a.part_ml = h->part_ml;
+  a.out = h->attn;
+  a.err = h->err;
+  CK(h->cfg.dtype == STCA_BF16 ? attention_bf16(a, s) : attention_f32(a, s));
+  CK(attention_merge(a, s));
+  return STCA_OK;
+}
+
+template <typename TB>
+int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int32_t* dt, const void* x_t,
+             const int32_t* tpu, int B, int n_tok, int t_tot, const stca_weights* w, float* z_out, float* o_out,
+             cudaStream_t s) {
+  const stca_config& c = h->cfg;
+  const int d = c.d, M = c.M;
+  const bool bf = c.dtype == STCA_BF16;
+  const int64_t ldcat = int64_t(M + 1) * d;
+  CK(exclusive_offsets(lens, B, h->hoff, n_tok, h->err, s));
+  CK(exclusive_offsets(tpu, B, h->toff, t_tot, h->err, s));
+  CK(copy_rows_to_f32(x_t, bf, t_tot, d, h->cat, ldcat, M * d, s));
+  if (bf)
+    for (int i = 0; i < M; ++i) CK(pack_layer(h, i, w->hist[i], w->WK[i], w->WV[i], s));
+  const float* xcol = h->cat + int64_t(M) * d;
+  // q^(1) = LN(SwiGLU_t(x_t))
+  CK(query_ffn<TB>(h, xcol, ldcat, t_tot, w->tgt, h->qbuf, d, s));
+  GatherSrc g;
+  g.ids = ids;
+  g.dt = c.time_buckets ? dt : nullptr;
+  g.table = w->table;
+  g.dt_table = c.time_buckets ? w->dt_table : nullptr;
+  g.n_items = w->n_items;
+  const int splits = choose_splits(n_tok, B, 1024);
+  for (int i = 0; i < M; ++i) {
+    if (bf) CK(history_bf16(h, i, g, n_tok, w->hist[i].gamma, w->hist[i].beta, s));
+    else CK(history_f32(h, g, n_tok, w->hist[i], w->WK[i], w->WV[i], s));
+    CK(simt_gemm(gemm_args<TB>(t_tot, d, d, h->qbuf, d, w->WQ[i], h->qproj, d, h->err), s));
+    CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, splits, c.score, s));
+    CK(simt_gemm(gemm_args<TB>(t_tot, d, d, h->attn, d, w->WO[i], h->cat + int64_t(i) * d, ldcat, h->err), s));
+    if (i + 1 < M) {
+      // q^(i+2) = LN(SwiGLU([o^(1) .. o^(i+1) | x_t] W_C))
+      const int K = (i + 2) * d;
+      auto a = gemm_args<TB>(t_tot, d, K, h->cat, ldcat, w->WC[i + 1], h->tmp_d, d, h->err);
+      a.ksplit = (i + 1) * d;
+      a.kshift = (M - (i + 1)) * d;
+      CK(simt_gemm(a, s));
+      CK(query_ffn<TB>(h, h->tmp_d, d, t_tot, w->fuse[i + 1], h->qbuf, d, s));
+    }
+  }
+  // z = SwiGLU_Z([o^(1) .. o^(M) | x_t] W_Z)
+  CK(simt_gemm(gemm_args<TB>(t_tot, d, int(ldcat), h->cat, ldcat, w->WZ, h->tmp_d, d, h->err), s));
+  CK(query_ffn<TB>(h, h->tmp_d, d, t_tot, w->zffn, z_out, d, s));
+  if (o_out && t_tot > 0) {
+    for (int i = 0; i < M; ++i)
+      if (cudaMemcpy2DAsync(o_out + int64_t(i) * t_tot * d, size_t(d) * 4, h->cat + int64_t(i) * d, size_t(ldcat) * 4,
+                            size_t(d) * 4, t_tot, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return STCA_ERR_CUDA;
+  }
+  return STCA_OK;
+}
+
+int check_forward_args(stca_handle* h, const int32_t* ids, const int32_t* lens, const int32_t* dt, const void* x_t,
+                       const int32_t* tpu, int B, int n_tok, int t_tot, const stca_weights* w, const float* z) {
+  if (!h) return STCA_ERR_INVALID_ARG;
+  const stca_config& c = h->cfg;
+  if (c.mode != STCA_MODE_STCA) return STCA_ERR_INVALID_ARG;
+  if (B < 0 || n_tok < 0 || t_tot < 0) return STCA_ERR_INVALID_ARG;
+  if (B > c.max_users || n_tok > c.max_tokens || t_tot > c.max_targets) return STCA_ERR_CAPACITY;
+  if ((B > 0 && (!lens || !tpu)) || (n_tok > 0 && !ids) || (t_tot > 0 && (!x_t || !z))) return STCA_ERR_INVALID_ARG;
+  if (c.time_buckets && n_tok > 0 && !dt) return STCA_ERR_INVALID_ARG;
+  return check_weights(c, w);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* stca_strerror(int code) {
+  switch (code) {
+    case STCA_OK: return "ok";
+    case STCA_ERR_INVALID_ARG: return "invalid argument";
+    case STCA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case STCA_ERR_CAPACITY: return "size exceeds the handle's capacity";
+    case STCA_ERR_CUDA: return "CUDA error";
+    case STCA_ERR_ID_OUT_OF_RANGE: return "item id out of range";
+    case STCA_ERR_TIMEOUT: return "a bounded device wait timed out";
+    case STCA_ERR_BAD_LENGTHS: return "lengths negative or inconsistent with the totals";
+    default: return "unknown status";
+  }
+}
+
+int stca_create(const stca_config* cfg, stca_handle** out) {
+  if (!out) return STCA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg) return STCA_ERR_INVALID_ARG;
+  CK(validate_config(*cfg));
+  stca_handle* h = new (std::nothrow) stca_handle();
+  if (!h) return STCA_ERR_CUDA;
+  h->cfg = *cfg;
+  if (cudaGetDevice(&h->device) != cudaSuccess) {
+    delete h;
+    return STCA_ERR_CUDA;
+  }
+  const int rc = allocate(h);
+  if (rc != STCA_OK || cudaMemset(h->err, 0, 4) != cudaSuccess) {
+    free_all(h);
+    delete h;
+    return rc != STCA_OK ? rc : STCA_ERR_CUDA;
+  }
+  *out = h;
+  return STCA_OK;
+}
+
+void stca_destroy(stca_handle* h) {
+  if (!h) return;
+  cudaSetDevice(h->device);
+  free_all(h);
+  delete h;
+}
+
+int stca_forward(stca_handle* h, const int32_t* hist_ids, const int32_t* hist_lengths, const int32_t* hist_dt,
+                 const void* target_emb, const int32_t* targets_per_user, int B, int n_tok, int t_tot,
+                 const stca_weights* w, float* z_out, float* o_out, void* stream) {
+  CK(check_forward_args(h, hist_ids, hist_lengths, hist_dt, target_emb, targets_per_user, B, n_tok, t_tot, w, z_out));
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  if (B == 0) return STCA_OK;
+  return h->cfg.dtype == STCA_BF16
+             ? run_stca<bf16>(h, hist_ids, hist_lengths, hist_dt, target_emb, targets_per_user, B, n_tok, t_tot, w,
+                              z_out, o_out, s)
+             : run_stca<float>(h, hist_ids, hist_lengths, hist_dt, target_emb, targets_per_user, B, n_tok, t_tot, w,
+                               z_out, o_out, s);
+}
+
+int stca_forward_host(stca_handle* h, const int32_t* ids, const int32_t* lens, const int32_t* dt, const void* x_t,
+                      const int32_t* tpu, int B, int n_tok, int t_tot, const stca_weights* w, float* z_host,
+                      void* stream) {
+  CK(check_forward_args(h, ids, lens, dt, x_t, tpu, B, n_tok, t_tot, w, z_host));
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  if (B == 0) return STCA_OK;
+  const size_t E = esize(h->cfg);
+  const size_t d = size_t(h->cfg.d);
+  bool ok = cudaMemcpyAsync(h->in_len, lens, size_t(B) * 4, cudaMemcpyHostToDevice, s) == cudaSuccess &&
+            cudaMemcpyAsync(h->in_tpu, tpu, size_t(B) * 4, cudaMemcpyHostToDevice, s) == cudaSuccess;
+  if (n_tok > 0) ok = ok && cudaMemcpyAsync(h->in_ids, ids, size_t(n_tok) * 4, cudaMemcpyHostToDevice, s) == cudaSuccess;
+  if (n_tok > 0 && h->cfg.time_buckets)
+    ok = ok && cudaMemcpyAsync(h->in_dt, dt, size_t(n_tok) * 4, cudaMemcpyHostToDevice, s) == cudaSuccess;
+  if (t_tot > 0) ok = ok && cudaMemcpyAsync(h->in_xt, x_t, size_t(t_tot) * d * E, cudaMemcpyHostToDevice, s) == cudaSuccess;
+  if (!ok) return STCA_ERR_CUDA;
+  const int rc = h->cfg.dtype == STCA_BF16
+                     ? run_stca<bf16>(h, h->in_ids, h->in_len, h->in_dt, h->in_xt, h->in_tpu, B, n_tok, t_tot, w,
+                                      h->out_z, nullptr, s)
+                     : run_stca<float>(h, h->in_ids, h->in_len, h->in_dt, h->in_xt, h->in_tpu, B, n_tok, t_tot, w,
+                                       h->out_z, nullptr, s);
+  CK(rc);
+  if (t_tot > 0 && cudaMemcpyAsync(z_host, h->out_z, size_t(t_tot) * d * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return STCA_ERR_CUDA;
+  return STCA_OK;
+}
+
+int stca_pointwise_forward(stca_handle* h, const int32_t* ids, const int32_t* lengths, const void* q, const void* table,
+                           int64_t n_items, int B, int n_tok, float* out, void* stream) {
+  if (!h || h->cfg.mode != STCA_MODE_POINTWISE) return STCA_ERR_INVALID_ARG;
+  if (B < 0 || n_tok < 0 || n_items <= 0) return STCA_ERR_INVALID_ARG;
+  if (B > h->cfg.max_users || n_tok > h->cfg.max_tokens) return STCA_ERR_CAPACITY;
+  if (B > 0 && (!lengths || !q || !table || !out)) return STCA_ERR_INVALID_ARG;
+  if (n_tok > 0 && !ids) return STCA_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  if (B == 0) return STCA_OK;
+  CK(exclusive_offsets(lengths, B, h->hoff, n_tok, h->err, s));
+  const int splits = choose_splits(n_tok, B, 2048);
+  return pointwise_relu_ta(ids, h->hoff, q, table, n_items, B, h->cfg.d, splits, h->part_acc, out, h->err, s);
+}
+
+int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len_feed, int n_feed,
+                     const int32_t* ids_search, const int32_t* len_search, int n_search, const void* q0, int B,
+                     int n_query, const hyf_weights* w, float* out, void* stream) {
+  if (!h || h->cfg.mode != STCA_MODE_HYFORMER || !w) return STCA_ERR_INVALID_ARG;
+  const stca_config& c = h->cfg;
+  const int d = c.d, hd = c.hidden;
+  const int T = 2 * n_query;
+  if (B < 0 || n_feed < 0 || n_search < 0 || n_query <= 0 || T > STCA_MAX_QUERY_TOKENS || d % T != 0)
+    return STCA_ERR_INVALID_ARG;
+  if (w->blocks != c.M || !w->table || w->n_items <= 0) return STCA_ERR_INVALID_ARG;
+  if (B > c.max_users || n_feed > c.max_tokens || n_search > c.max_tokens || int64_t(B) * T > c.max_targets)
+    return STCA_ERR_CAPACITY;
+  if (B > 0 && (!len_feed || !len_search || !q0 || !out)) return STCA_ERR_INVALID_ARG;
+  if ((n_feed > 0 && !ids_feed) || (n_search > 0 && !ids_search)) return STCA_ERR_INVALID_ARG;
+  for (int l = 0; l < c.M; ++l) {
+    for (int sq = 0; sq < 2; ++sq) {
+      const hyf_seq_weights& f = w->blk[l].seq[sq];
+      if (!ffn_ok(f.ffn, false) || !f.WQ || !f.WK || !f.WV || !f.WO) return STCA_ERR_INVALID_ARG;
+    }
+    for (int t = 0; t < T; ++t)
+      if (!ffn_ok(w->blk[l].tok[t], false)) return STCA_ERR_INVALID_ARG;
+  }
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  if (B == 0) return STCA_OK;
+  const int rows = B * T, rows_s = B * n_query;
+  CK(exclusive_offsets(len_feed, B, h->hoff, n_feed, h->err, s));
+  CK(exclusive_offsets(len_search, B, h->hoff2, n_search, h->err, s));
+  CK(fill_arange(h->toff, B + 1, n_query, s));
+  CK(copy_rows_to_f32(q0, 1, rows, d, h->hq, d, 0, s));
+  for (int l = 0; l < c.M; ++l)
+    for (int sq = 0; sq < 2; ++sq) {
+      const hyf_seq_weights& f = w->blk[l].seq[sq];
+      CK(pack_layer(h, size_t(l) * 2 + sq, f.ffn, f.WK, f.WV, s));
+    }
+  const int32_t* ids[2] = {ids_feed, ids_search};
+  const int32_t* offs[2] = {h->hoff, h->hoff2};
+  const int ntok[2] = {n_feed, n_search};
+  for (int l = 0; l < c.M; ++l) {
+    for (int sq = 0; sq < 2; ++sq) {
+      const hyf_seq_weights& f = w->blk[l].seq[sq];
+      GatherSrc g;
+      memset(&g, 0, sizeof(g));
+      g.ids = ids[sq];
+      g.table = w->table;
+      g.n_items = w->n_items;
+      // H = SwiGLU(X_s) (eq 7), K/V = H W_K, H W_V (eq 8)
+      CK(history_bf16(h, size_t(l) * 2 + sq, g, ntok[sq], nullptr, nullptr, s));
+      // queries of sequence sq: rows b*T + sq*n_query + n
+      auto qa = gemm_args<bf16>(rows_s, d, d, h->hq, d, f.WQ, h->qproj, d, h->err);
+      qa.a_grp = n_query;
+      qa.a_gstride = T;
+      qa.a_goff = sq * n_query;
+      CK(simt_gemm(qa, s));
+      CK(run_attention(h, h->qproj, offs[sq], h->toff, B, rows_s, choose_splits(ntok[sq], B, 1024), STCA_SOFTMAX, s));
+      auto oa = gemm_args<bf16>(rows_s, d, d, h->attn, d, f.WO, h->hqhat, d, h->err);
+      oa.c_grp = n_query;
+      oa.c_gstride = T;
+      oa.c_goff = sq * n_query;
+      CK(simt_gemm(oa, s));
+    }
+    // query boosting: token mix (eq 11-13), per-token SwiGLU (eq 14), residual (eq 15)
+    CK(token_mix(h->hqhat, B, T, d, h->hmix, s));
+    auto a1 = gemm_args<bf16>(B, hd, d, h->hmix, int64_t(T) * d, nullptr, h->tmp_h, int64_t(T) * hd, h->err);
+    a1.batch = T;
+    a1.bsA = d;
+    a1.bsC = hd;
+    for (int t = 0; t < T; ++t) {
+      a1.Bz[t] = reinterpret_cast<const bf16*>(w->blk[l].tok[t].W1);
+      a1.B2z[t] = reinterpret_cast<const bf16*>(w->blk[l].tok[t].W3);
+    }
+    a1.B2 = a1.B2z[0];
+    CK(simt_gemm(a1, s));
+    float* dst = (l + 1 == c.M) ? out : h->hq;
+    auto a2 = gemm_args<bf16>(B, d, hd, h->tmp_h, int64_t(T) * hd, nullptr, dst, int64_t(T) * d, h->err);
+    a2.batch = T;
+    a2.bsA = hd;
+    a2.bsC = d;
+    a2.R = h->hqhat;
+    a2.ldr = int64_t(T) * d;
+    a2.bsR = d;
+    for (int t = 0; t < T; ++t) a2.Bz[t] = reinterpret_cast<const bf16*>(w->blk[l].tok[t].W2);
+    CK(simt_gemm(a2, s));
+  }
+  return STCA_OK;
+}
+
+int stca_sync_status(stca_handle* h) {
+  if (!h) return STCA_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return STCA_ERR_CUDA;
+  int32_t e = 0;
+  if (cudaMemcpy(&e, h->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return STCA_ERR_CUDA;
+  if (e != 0 && cudaMemset(h->err, 0, 4) != cudaSuccess) return STCA_ERR_CUDA;
+  return e;
+}
+
+}  // extern "C"

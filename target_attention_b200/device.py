@@ -1,0 +1,175 @@
+"""Device-side holders for the three entry points: upload a workload's weights and
+inputs (numpy arrays in the storage formats of ``workloads``) to torch tensors, fill the
+ctypes weight structs, own the libstca handle.  Marshalling only."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+
+def to_device(arr, device="cuda", pin=False):
+    """numpy (float32, int32, or bf16 bit patterns in uint16) -> torch tensor."""
+    if arr is None:
+        return None
+    a = np.ascontiguousarray(arr)
+    if a.dtype == np.uint16:
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(a)
+    if pin:
+        return t.pin_memory()
+    return t.to(device, non_blocking=False)
+
+
+class _Holder:
+    def __init__(self, device):
+        self.device = device
+        self.keep = []
+
+    def up(self, arr):
+        t = to_device(arr, self.device)
+        if t is not None:
+            self.keep.append(t)
+        return t
+
+    def p(self, arr):
+        t = self.up(arr)
+        return None if t is None else t.data_ptr()
+
+    def ffn(self, f, ln=True):
+        s = B.StcaFfn()
+        s.W1, s.W3, s.W2 = self.p(f["W1"]), self.p(f["W3"]), self.p(f["W2"])
+        if ln and "gamma" in f:
+            s.gamma, s.beta = self.p(f["gamma"]), self.p(f["beta"])
+        return s
+
+
+class StcaModel(_Holder):
+    """Weights of an STCA workload on the device plus a handle sized for it."""
+
+    def __init__(self, wl, device="cuda", max_users=None, max_tokens=None, max_targets=None):
+        super().__init__(device)
+        c = wl["cfg"]
+        self.cfg = c
+        self.config = B.StcaConfig(
+            mode=B.MODE_STCA, M=c["M"], d=c["d"], H=c["H"], hidden=c["hidden"],
+            dtype=B.BF16 if c["dtype"] == "bf16" else B.FP32,
+            score=B.RELU if c["score"] == "relu" else B.SOFTMAX, time_buckets=c["time_buckets"],
+            max_users=max_users or len(wl["lengths"]), max_tokens=max_tokens or int(wl["lengths"].sum()),
+            max_targets=max_targets or int(wl["targets_per_user"].sum()), ln_eps=c.get("ln_eps", 1e-5))
+        w = wl["weights"]
+        ws = B.StcaWeights()
+        ws.table = self.p(wl["table"])
+        ws.n_items = wl["table"].shape[0]
+        ws.dt_table = self.p(wl["dt_table"])
+        for i in range(c["M"]):
+            ws.hist[i] = self.ffn(w["hist"][i])
+            ws.WQ[i], ws.WK[i] = self.p(w["WQ"][i]), self.p(w["WK"][i])
+            ws.WV[i], ws.WO[i] = self.p(w["WV"][i]), self.p(w["WO"][i])
+            if i > 0:
+                ws.WC[i] = self.p(w["WC"][i])
+                ws.fuse[i] = self.ffn(w["fuse"][i])
+        ws.tgt = self.ffn(w["tgt"])
+        ws.WZ = self.p(w["WZ"])
+        ws.zffn = self.ffn(w["zffn"], ln=False)
+        self.weights = ws
+        self.handle = B.stca_create(self.config)
+
+    def inputs(self, wl):
+        d = {k: to_device(wl[k], self.device) for k in ("ids", "lengths", "dt", "x_t", "targets_per_user")}
+        d["B"] = len(wl["lengths"])
+        d["n_tok"] = int(wl["lengths"].sum())
+        d["t_tot"] = int(wl["targets_per_user"].sum())
+        return d
+
+    def forward(self, x, z_out, o_out=None, stream=None):
+        return B.stca_forward(self.handle, x["ids"], x["lengths"], x["dt"], x["x_t"], x["targets_per_user"],
+                              x["B"], x["n_tok"], x["t_tot"], self.weights, z_out, o_out, stream)
+
+    def forward_host(self, x, z_out, stream=None):
+        return B.stca_forward_host(self.handle, x["ids"], x["lengths"], x["dt"], x["x_t"], x["targets_per_user"],
+                                   x["B"], x["n_tok"], x["t_tot"], self.weights, z_out, stream)
+
+    def close(self):
+        if getattr(self, "handle", None) is not None:
+            B.stca_destroy(self.handle)
+            self.handle = None
+
+    __del__ = close
+
+
+class PointwiseModel(_Holder):
+    def __init__(self, wl, device="cuda", max_users=None, max_tokens=None):
+        super().__init__(device)
+        c = wl["cfg"]
+        self.cfg = c
+        self.config = B.StcaConfig(mode=B.MODE_POINTWISE, M=1, d=c["d"], H=1, hidden=c["d"], dtype=B.BF16,
+                                   score=B.RELU, time_buckets=0, max_users=max_users or len(wl["lengths"]),
+                                   max_tokens=max_tokens or int(wl["lengths"].sum()), max_targets=0, ln_eps=1e-5)
+        self.table = self.up(wl["table"])
+        self.handle = B.stca_create(self.config)
+
+    def inputs(self, wl):
+        return dict(ids=to_device(wl["ids"], self.device), lengths=to_device(wl["lengths"], self.device),
+                    q=to_device(wl["q"], self.device), B=len(wl["lengths"]), n_tok=int(wl["lengths"].sum()))
+
+    def forward(self, x, out, stream=None):
+        return B.stca_pointwise_forward(self.handle, x["ids"], x["lengths"], x["q"], self.table, self.table.shape[0],
+                                        x["B"], x["n_tok"], out, stream)
+
+    def close(self):
+        if getattr(self, "handle", None) is not None:
+            B.stca_destroy(self.handle)
+            self.handle = None
+
+    __del__ = close
+
+
+class HyformerModel(_Holder):
+    def __init__(self, wl, device="cuda", max_users=None, max_tokens=None):
+        super().__init__(device)
+        c = wl["cfg"]
+        self.cfg = c
+        nq = c["n_query"]
+        Bu = len(wl["lengths"][0])
+        self.config = B.StcaConfig(
+            mode=B.MODE_HYFORMER, M=c["blocks"], d=c["d"], H=c["H"], hidden=c["hidden"], dtype=B.BF16,
+            score=B.SOFTMAX, time_buckets=0, max_users=max_users or Bu,
+            max_tokens=max_tokens or int(max(wl["lengths"][0].sum(), wl["lengths"][1].sum())),
+            max_targets=(max_users or Bu) * 2 * nq, ln_eps=1e-5)
+        ws = B.HyfWeights()
+        ws.table = self.p(wl["table"])
+        ws.n_items = wl["table"].shape[0]
+        ws.blocks = c["blocks"]
+        for l, blk in enumerate(wl["weights"]["blocks"]):
+            for s in range(2):
+                f = blk["seq"][s]
+                sw = B.HyfSeqWeights()
+                sw.ffn = self.ffn(f, ln=False)
+                sw.WQ, sw.WK, sw.WV, sw.WO = (self.p(f[k]) for k in ("WQ", "WK", "WV", "WO"))
+                ws.blk[l].seq[s] = sw
+            for t, f in enumerate(blk["tok"]):
+                ws.blk[l].tok[t] = self.ffn(f, ln=False)
+        self.weights = ws
+        self.handle = B.stca_create(self.config)
+
+    def inputs(self, wl):
+        return dict(ids_feed=to_device(wl["ids"][0], self.device), len_feed=to_device(wl["lengths"][0], self.device),
+                    ids_search=to_device(wl["ids"][1], self.device),
+                    len_search=to_device(wl["lengths"][1], self.device), q0=to_device(wl["q0"], self.device),
+                    B=len(wl["lengths"][0]), n_feed=int(wl["lengths"][0].sum()),
+                    n_search=int(wl["lengths"][1].sum()), n_query=self.cfg["n_query"])
+
+    def forward(self, x, out, stream=None):
+        return B.hyformer_forward(self.handle, x["ids_feed"], x["len_feed"], x["n_feed"], x["ids_search"],
+                                  x["len_search"], x["n_search"], x["q0"], x["B"], x["n_query"], self.weights, out,
+                                  stream)
+
+    def close(self):
+        if getattr(self, "handle", None) is not None:
+            B.stca_destroy(self.handle)
+            self.handle = None
+
+    __del__ = close

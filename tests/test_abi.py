@@ -1,0 +1,100 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function the headers
+declare, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import target_attention_b200 as tab
+from target_attention_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for hdr in ("stca.h", "stca_kernels.h"):
+        text = open(os.path.join(ROOT, "include", hdr)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_library_exports_every_declared_function():
+    L = tab.lib()
+    declared = _declared_functions()
+    assert {"stca_create", "stca_forward", "stca_pointwise_forward", "hyformer_forward"} <= declared
+    missing = [n for n in declared if not hasattr(L, n)]
+    assert not missing, missing
+    assert declared == set(B.EXPORTED), declared ^ set(B.EXPORTED)
+
+
+def test_struct_layouts_match_c():
+    # sizes computed by the C compiler from include/stca.h
+    assert ctypes.sizeof(B.StcaConfig) == 48
+    assert ctypes.sizeof(B.StcaWeights) == 1072
+    assert ctypes.sizeof(B.HyfWeights) == 21656
+
+
+def test_strerror_covers_all_codes():
+    for c in range(8):
+        assert B.strerror(c) not in ("?", "unknown status")
+    assert B.strerror(99) == "unknown status"
+
+
+def _cfg(**kw):
+    base = dict(mode=B.MODE_STCA, M=2, d=256, H=4, hidden=512, dtype=B.BF16, score=B.SOFTMAX, time_buckets=0,
+                max_users=4, max_tokens=100, max_targets=8, ln_eps=1e-5)
+    base.update(kw)
+    return B.StcaConfig(**base)
+
+
+@pytest.mark.parametrize("kw, code", [
+    (dict(M=0), B.ERR_INVALID_ARG),
+    (dict(M=9), B.ERR_INVALID_ARG),
+    (dict(d=384, H=6), B.ERR_UNSUPPORTED),        # bf16 needs d in {256, 512}
+    (dict(H=8), B.ERR_UNSUPPORTED),               # d_h = 32 with bf16
+    (dict(hidden=200), B.ERR_UNSUPPORTED),        # hidden % 128
+    (dict(time_buckets=8), B.ERR_UNSUPPORTED),
+    (dict(dtype=7), B.ERR_INVALID_ARG),
+    (dict(score=3), B.ERR_INVALID_ARG),
+    (dict(max_tokens=-1), B.ERR_INVALID_ARG),
+    (dict(mode=B.MODE_POINTWISE, d=256), B.ERR_UNSUPPORTED),
+    (dict(mode=B.MODE_HYFORMER, d=256), B.ERR_UNSUPPORTED),
+    (dict(mode=5), B.ERR_INVALID_ARG),
+    (dict(dtype=B.FP32, d=96, H=2), B.ERR_UNSUPPORTED),   # d_h = 48
+])
+def test_create_rejects_bad_configs(kw, code):
+    h = ctypes.c_void_p()
+    assert tab.lib().stca_create(ctypes.byref(_cfg(**kw)), ctypes.byref(h)) == code
+    assert h.value is None
+
+
+def test_null_arguments_rejected_on_host():
+    L = tab.lib()
+    assert L.stca_create(None, None) == B.ERR_INVALID_ARG
+    h = ctypes.c_void_p()
+    assert L.stca_create(None, ctypes.byref(h)) == B.ERR_INVALID_ARG
+    w = B.StcaWeights()
+    assert L.stca_forward(None, None, None, None, None, None, 1, 1, 1, ctypes.byref(w), None, None, None) \
+        == B.ERR_INVALID_ARG
+    assert L.stca_pointwise_forward(None, None, None, None, None, 1, 1, 1, None, None) == B.ERR_INVALID_ARG
+    assert L.stca_sync_status(None) == B.ERR_INVALID_ARG
+    L.stca_destroy(None)
+    # kernel-level entry points validate before launching
+    assert L.stca_k_attention(1, None, None, None, None, 1, 1, 256, 3, 1, 0, None, None, None, None, None) \
+        == B.ERR_INVALID_ARG
+    assert L.stca_k_pack_weight(None, 4, 4, None, 0, 0, None) == B.ERR_INVALID_ARG
+    assert L.stca_k_gemm_resident(1, 1, None, None, None, None, None, 0, 5, 256, None, 128, None, 128, None,
+                                  None) == B.ERR_INVALID_ARG
+    assert L.stca_k_gemm_rowwise(5, None, 0, 64, None, 256, None, None, 1e-5, None, 256, None, None) \
+        == B.ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(B, "_LIB", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        B.lib()

@@ -1,0 +1,244 @@
+"""Per-kernel parity of libstca's steps against the fp64 oracle's component functions,
+called through the kernel-level C entry points (include/stca_kernels.h)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import stca_ref as R
+from target_attention_b200 import binding as B
+from tests._util import bf16_to_f64, bits_of, zeros_err
+
+pytestmark = pytest.mark.gpu
+dev = "cuda"
+
+
+def _bf16(a64, seed=None):
+    return torch.from_numpy(np.asarray(a64, np.float32)).to(torch.bfloat16).to(dev)
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _pack(W, mode, rows, row_offset=0, dst=None):
+    """W: bf16 [K, N] device tensor -> packed [rows, K] via the library."""
+    K, N = W.shape
+    if dst is None:
+        dst = torch.zeros(rows, K, dtype=torch.bfloat16, device=dev)
+    B.check(B.stca_k_pack_weight(W, K, N, dst, mode, row_offset))
+    return dst
+
+
+# ---------------------------------------------------------------- a1: ragged offsets
+
+
+def test_offsets_bit_exact_and_checks():
+    lengths = _rng(0).integers(0, 3000, size=2500).astype(np.int32)
+    lengths[[0, 7, 2499]] = 0
+    L = torch.from_numpy(lengths).to(dev)
+    off = torch.full((2501,), -1, dtype=torch.int32, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_offsets(L, 2500, off, int(lengths.sum()), err))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(off.cpu().numpy(), R.exclusive_offsets(lengths))
+    assert err.item() == 0
+    # a total that does not match is reported, as is a negative length
+    B.check(B.stca_k_offsets(L, 2500, off, int(lengths.sum()) + 1, err))
+    torch.cuda.synchronize()
+    assert err.item() == B.ERR_BAD_LENGTHS
+    err.zero_()
+    lengths[5] = -3
+    B.check(B.stca_k_offsets(torch.from_numpy(lengths).to(dev), 2500, off, 0, err))
+    torch.cuda.synchronize()
+    assert err.item() == B.ERR_BAD_LENGTHS
+
+
+# ---------------------------------------------------------------- weight packing
+
+
+def test_pack_weight_layouts():
+    W = _bf16(_rng(1).standard_normal((256, 384)))
+    Wb = bits_of(W)
+    p0 = _pack(W, 0, 384 + 5, row_offset=5)
+    np.testing.assert_array_equal(bits_of(p0)[5:], Wb.T)
+    p1 = _pack(W, 1, 768)
+    p1 = _pack(W, 2, 768, dst=p1)
+    pb = bits_of(p1)
+    for n in range(384):
+        g = (n // 128) * 256 + n % 128
+        np.testing.assert_array_equal(pb[g], Wb[:, n])
+        np.testing.assert_array_equal(pb[g + 128], Wb[:, n])
+
+
+# ---------------------------------------------------------------- a2: fused gather (bit exact)
+
+
+@pytest.mark.parametrize("K, with_dt", [(256, False), (512, True), (512, False)])
+def test_fused_gather_is_bit_exact(K, with_dt):
+    """Identity weights make the tensor-core GEMM copy its A operand, so the output rows
+    are exactly the gathered rows: bf16(E[id] (+ T[bucket(dt)])), rounded from fp32."""
+    g = _rng(2)
+    n_items, M = 5000, 389                      # 4 tiles, ragged tail
+    E = _bf16(g.standard_normal((n_items, K)) * 0.02)
+    T = _bf16(g.standard_normal((16, K)) * 0.02) if with_dt else None
+    ids = g.integers(0, n_items, size=M).astype(np.int32)
+    dt = (np.floor(np.exp2(g.uniform(0, 16, size=M))) - 1).astype(np.int32) if with_dt else None
+    Wp = torch.eye(K, dtype=torch.bfloat16, device=dev)           # packed identity [K, K]
+    C = torch.full((M, K), float("nan"), dtype=torch.bfloat16, device=dev)
+    err = zeros_err()
+    ids_t = torch.from_numpy(ids).to(dev)
+    dt_t = torch.from_numpy(dt).to(dev) if with_dt else None
+    B.check(B.stca_k_gemm_resident(1, 0, None, ids_t, dt_t, E, T, n_items, M, K, Wp, K, C, K, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    Ef = E.float().cpu().numpy()[ids]
+    if with_dt:
+        Ef = Ef + T.float().cpu().numpy()[R.dt_bucket(dt)]    # fp32 sum, as the kernel
+    expect = torch.from_numpy(Ef.astype(np.float32)).to(torch.bfloat16)
+    np.testing.assert_array_equal(bits_of(C), bits_of(expect))
+
+
+def test_fused_gather_flags_bad_ids():
+    K, n_items, M = 256, 100, 130
+    E = _bf16(_rng(3).standard_normal((n_items, K)))
+    ids = np.arange(M, dtype=np.int32) % n_items
+    ids[17] = n_items           # out of range
+    ids[129] = -1
+    Wp = torch.eye(K, dtype=torch.bfloat16, device=dev)
+    C = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_gemm_resident(1, 0, None, torch.from_numpy(ids).to(dev), None, E, None, n_items, M, K, Wp, K, C,
+                                   K, err))
+    torch.cuda.synchronize()
+    assert err.item() == B.ERR_ID_OUT_OF_RANGE
+    c = C.float().cpu().numpy()
+    assert (c[17] == 0).all() and (c[129] == 0).all()
+    np.testing.assert_array_equal(c[18], E.float().cpu().numpy()[18])
+
+
+# ---------------------------------------------------------------- a3/a4: tensor-core GEMMs
+
+
+def _close_bf16(got, ref, tol=1e-2):
+    err = R.row_rel_err(got, ref)
+    assert err <= tol, err
+
+
+@pytest.mark.parametrize("K, N, M", [(256, 512, 300), (512, 1024, 257), (512, 256, 1)])
+def test_gemm_resident_plain(K, N, M):
+    g = _rng(4)
+    A = _bf16(g.standard_normal((M, K)))
+    W = _bf16(g.standard_normal((K, N)) / math.sqrt(K))
+    Wp = _pack(W, 0, N)
+    C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_gemm_resident(0, 0, A, None, None, None, None, 0, M, K, Wp, N, C, N, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    _close_bf16(bf16_to_f64(C), bf16_to_f64(A) @ bf16_to_f64(W))
+
+
+@pytest.mark.parametrize("K, hidden, M", [(256, 512, 200), (512, 1024, 390)])
+def test_gemm_gather_swiglu(K, hidden, M):
+    g = _rng(5)
+    n_items = 3000
+    E = _bf16(g.standard_normal((n_items, K)) * 0.5)
+    ids = g.integers(0, n_items, size=M).astype(np.int32)
+    W1 = _bf16(g.standard_normal((K, hidden)) / math.sqrt(K))
+    W3 = _bf16(g.standard_normal((K, hidden)) / math.sqrt(K))
+    Wp = _pack(W1, 1, 2 * hidden)
+    _pack(W3, 2, 2 * hidden, dst=Wp)
+    C = torch.empty((M, hidden), dtype=torch.bfloat16, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_gemm_resident(1, 1, None, torch.from_numpy(ids).to(dev), None, E, None, n_items, M, K, Wp,
+                                   hidden, C, hidden, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    X = bf16_to_f64(E)[ids]
+    ref = R.silu(X @ bf16_to_f64(W1)) * (X @ bf16_to_f64(W3))
+    _close_bf16(bf16_to_f64(C), ref)
+
+
+@pytest.mark.parametrize("K, N, M, ln", [(1024, 512, 333, True), (512, 256, 129, True), (1024, 512, 200, False)])
+def test_gemm_rowwise(K, N, M, ln):
+    g = _rng(6)
+    A = _bf16(g.standard_normal((M, K)))
+    W = _bf16(g.standard_normal((K, N)) / math.sqrt(K))
+    Wp = _pack(W, 0, N)
+    gamma = torch.from_numpy((1 + 0.1 * g.standard_normal(N)).astype(np.float32)).to(dev)
+    beta = torch.from_numpy((0.1 * g.standard_normal(N)).astype(np.float32)).to(dev)
+    C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_gemm_rowwise(2 if ln else 0, A, M, K, Wp, N, gamma if ln else None, beta if ln else None, 1e-5,
+                                  C, N, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    Y = bf16_to_f64(A) @ bf16_to_f64(W)
+    if ln:
+        Y = R.layer_norm(Y, gamma.cpu().numpy(), beta.cpu().numpy(), 1e-5)
+    _close_bf16(bf16_to_f64(C), Y)
+
+
+# ---------------------------------------------------------------- a6/a7: attention + merge
+
+
+def _attention_case(kv_bf16, d, H, lengths, targets, splits, score, seed):
+    g = _rng(seed)
+    n_tok, T = int(sum(lengths)), int(sum(targets))
+    KV = g.standard_normal((max(n_tok, 1), 2 * d))
+    Q = g.standard_normal((max(T, 1), d)).astype(np.float32)
+    if kv_bf16:
+        KVt = _bf16(KV)
+        KV64 = bf16_to_f64(KVt)
+    else:
+        KVt = torch.from_numpy(KV.astype(np.float32)).to(dev)
+        KV64 = KV.astype(np.float32).astype(np.float64)
+    hoff = R.exclusive_offsets(lengths)
+    toff = R.exclusive_offsets(targets)
+    Bu = len(lengths)
+    part_acc = torch.empty((splits, max(T, 1), d), dtype=torch.float32, device=dev)
+    part_ml = torch.empty((splits, max(T, 1), H, 2), dtype=torch.float32, device=dev)
+    out = torch.full((max(T, 1), d), float("nan"), dtype=torch.float32, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_attention(1 if kv_bf16 else 0, torch.from_numpy(Q).to(dev), KVt,
+                               torch.from_numpy(hoff.astype(np.int32)).to(dev),
+                               torch.from_numpy(toff.astype(np.int32)).to(dev), Bu, T, d, H, splits, score,
+                               part_acc, part_ml, out, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    dh = d // H
+    ref = np.zeros((T, d))
+    for u in range(Bu):
+        K = KV64[hoff[u]:hoff[u + 1], :d]
+        V = KV64[hoff[u]:hoff[u + 1], d:]
+        for t in range(toff[u], toff[u + 1]):
+            for h in range(H):
+                cols = slice(h * dh, (h + 1) * dh)
+                ref[t, cols] = R.head_attention(Q[t, cols].astype(np.float64), K[:, cols], V[:, cols],
+                                                "softmax" if score == 0 else "relu", 1 / math.sqrt(dh))
+    return out.cpu().numpy()[:T], ref
+
+
+@pytest.mark.parametrize("score", [0, 1])
+@pytest.mark.parametrize("splits", [1, 3])
+def test_attention_bf16(score, splits):
+    lengths = [0, 1, 31, 33, 700, 2049, 5]
+    targets = [2, 1, 16, 17, 33, 40, 0]
+    got, ref = _attention_case(True, 256, 4, lengths, targets, splits, score, seed=7 + score)
+    # per-head rows: compare each (target, head) block on its own scale
+    err = R.row_rel_err(got.reshape(-1, 64), ref.reshape(-1, 64))
+    assert err <= 2e-2, err
+    # the empty history gives exactly zero
+    assert (got[:2] == 0).all()
+
+
+@pytest.mark.parametrize("score", [0, 1])
+def test_attention_f32(score):
+    lengths = [0, 1, 9, 600]
+    targets = [1, 3, 4, 4]
+    got, ref = _attention_case(False, 64, 2, lengths, targets, 2, score, seed=9)
+    err = R.row_rel_err(got.reshape(-1, 32), ref.reshape(-1, 32))
+    assert err <= 1e-5, err
+    assert (got[:1] == 0).all()

@@ -1,0 +1,177 @@
+"""End-to-end parity of the three forward entry points against the fp64 oracle, on the
+same seeded inputs, through the C ABI.  Tolerances (row-normwise max relative error):
+2e-2 for bf16 storage with fp32 accumulation, 1e-4 for the fp32 configuration."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import stca_ref as R
+from target_attention_b200 import binding as B
+from target_attention_b200.device import HyformerModel, PointwiseModel, StcaModel
+from workloads import make_hyformer, make_pointwise, make_stca
+
+pytestmark = pytest.mark.gpu
+dev = "cuda"
+TOL_BF16, TOL_FP32 = 2e-2, 1e-4
+
+
+def _run_stca(wl, with_o=True, model=None):
+    m = model or StcaModel(wl)
+    x = m.inputs(wl)
+    T, d, M = x["t_tot"], wl["cfg"]["d"], wl["cfg"]["M"]
+    z = torch.full((max(T, 1), d), float("nan"), device=dev)
+    o = torch.full((M, max(T, 1), d), float("nan"), device=dev) if with_o else None
+    B.check(m.forward(x, z, o), "stca_forward")
+    assert B.stca_sync_status(m.handle) == B.OK
+    res = (z.cpu().numpy()[:T], None if o is None else o.cpu().numpy()[:, :T])
+    if model is None:
+        m.close()
+    return res
+
+
+def _check_stca(wl, tol, users=None):
+    z, o = _run_stca(wl)
+    zr, orr = R.stca_forward(wl, users=users)
+    if users is not None:
+        toff = R.exclusive_offsets(wl["targets_per_user"])
+        rows = np.concatenate([np.arange(toff[u], toff[u + 1]) for u in users])
+        z, o = z[rows], o[:, rows]
+    for i in range(wl["cfg"]["M"]):
+        e = R.row_rel_err(o[i], orr[i])
+        assert e <= tol, f"o^({i + 1}) err {e}"
+    e = R.row_rel_err(z, zr)
+    assert e <= tol, f"z err {e}"
+    return z
+
+
+def test_config1_fp32_full():
+    _check_stca(make_stca(1), TOL_FP32)
+
+
+def test_config2_bf16_small():
+    _check_stca(make_stca(2, users=6, n_items=20_000), TOL_BF16)
+
+
+def test_config3_bf16_small_time_feature():
+    _check_stca(make_stca(3, users=3, L=600, n_items=50_000), TOL_BF16)
+
+
+def test_config3_relu_scores():
+    _check_stca(make_stca(3, users=2, L=300, n_items=10_000, M=2, score="relu"), TOL_BF16)
+
+
+def test_ragged_edge_cases():
+    """Empty histories, a single-token history, users without targets, ragged tails."""
+    lengths = np.array([0, 1, 129, 0, 257, 40], np.int32)
+    wl = make_stca(2, lengths=lengths, n_items=3000)
+    wl["targets_per_user"] = np.array([3, 2, 0, 1, 5, 0], np.int32)
+    wl["x_t"] = wl["x_t"][:11]
+    _check_stca(wl, TOL_BF16)
+
+
+def test_fp32_ragged_edge_cases():
+    lengths = np.array([0, 3, 70], np.int32)
+    wl = make_stca(1, lengths=lengths)
+    wl["targets_per_user"] = np.array([2, 0, 3], np.int32)
+    wl["x_t"] = wl["x_t"][:5]
+    _check_stca(wl, TOL_FP32)
+
+
+def test_rlb_batched_equals_single_target_runs():
+    """The m targets of a user, run together, give bit-for-bit the same z as m runs with
+    one target each: the per-user K/V is shared, never mixed between targets."""
+    wl = make_stca(3, users=1, L=500, n_items=20_000, m=5)
+    z_all, _ = _run_stca(wl, with_o=False)
+    m = StcaModel(wl)
+    for k in range(5):
+        one = dict(wl, x_t=wl["x_t"][k:k + 1], targets_per_user=np.array([1], np.int32))
+        z1, _ = _run_stca(one, with_o=False, model=m)
+        np.testing.assert_array_equal(z1[0], z_all[k])
+    m.close()
+
+
+def test_bad_ids_reported_not_faulting():
+    wl = make_stca(2, users=2, L=50, n_items=1000)
+    wl["ids"] = wl["ids"].copy()
+    wl["ids"][7] = 1000
+    m = StcaModel(wl)
+    x = m.inputs(wl)
+    z = torch.empty((x["t_tot"], 256), device=dev)
+    B.check(m.forward(x, z))
+    assert B.stca_sync_status(m.handle) == B.ERR_ID_OUT_OF_RANGE
+    assert B.stca_sync_status(m.handle) == B.OK          # read-and-clear
+    m.close()
+
+
+def test_capacity_and_argument_errors():
+    wl = make_stca(2, users=2, L=50, n_items=1000)
+    m = StcaModel(wl)
+    x = m.inputs(wl)
+    z = torch.empty((x["t_tot"], 256), device=dev)
+    assert B.stca_forward(m.handle, x["ids"], x["lengths"], None, x["x_t"], x["targets_per_user"], 3, x["n_tok"],
+                          x["t_tot"], m.weights, z) == B.ERR_CAPACITY
+    assert B.stca_forward(m.handle, None, x["lengths"], None, x["x_t"], x["targets_per_user"], 2, x["n_tok"],
+                          x["t_tot"], m.weights, z) == B.ERR_INVALID_ARG
+    # lengths that do not add up to n_tok are detected on the device
+    B.check(B.stca_forward(m.handle, x["ids"], x["lengths"], None, x["x_t"], x["targets_per_user"], 2,
+                           x["n_tok"] - 1, x["t_tot"], m.weights, z))
+    assert B.stca_sync_status(m.handle) == B.ERR_BAD_LENGTHS
+    m.close()
+
+
+def test_host_buffer_entry_matches_device_entry():
+    wl = make_stca(3, users=2, L=300, n_items=10_000)
+    m = StcaModel(wl)
+    x = m.inputs(wl)
+    z_dev = torch.empty((x["t_tot"], 512), device=dev)
+    B.check(m.forward(x, z_dev))
+    xh = {k: (v.cpu().pin_memory() if torch.is_tensor(v) else v) for k, v in x.items()}
+    z_host = torch.empty((x["t_tot"], 512), pin_memory=True)
+    B.check(m.forward_host(xh, z_host))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(z_host.numpy(), z_dev.cpu().numpy())
+    m.close()
+
+
+# ---------------------------------------------------------------- pointwise ReLU TA
+
+
+def _run_pointwise(wl):
+    m = PointwiseModel(wl)
+    x = m.inputs(wl)
+    out = torch.full((x["B"], 128), float("nan"), device=dev)
+    B.check(m.forward(x, out))
+    assert B.stca_sync_status(m.handle) == B.OK
+    m.close()
+    return out.cpu().numpy()
+
+
+def test_pointwise_small():
+    wl = make_pointwise(users=40, L=3000, L_lo=1, n_items=50_000)
+    wl["lengths"] = wl["lengths"].copy()
+    got = _run_pointwise(wl)
+    ref = R.pointwise_relu_ta(wl)
+    assert R.row_rel_err(got, ref) <= 1e-4
+
+
+def test_pointwise_empty_rows():
+    wl = make_pointwise(users=4, L=10, L_lo=1, n_items=100, lengths=np.array([0, 5, 0, 1], np.int32))
+    got = _run_pointwise(wl)
+    assert (got[0] == 0).all() and (got[2] == 0).all()
+    assert R.row_rel_err(got, R.pointwise_relu_ta(wl)) <= 1e-4
+
+
+# ---------------------------------------------------------------- multi-sequence decode
+
+
+def test_hyformer_small():
+    wl = make_hyformer(users=3, L_feed=700, L_search=130, n_items=20_000)
+    m = HyformerModel(wl)
+    x = m.inputs(wl)
+    out = torch.full((x["B"], 32, 512), float("nan"), device=dev)
+    B.check(m.forward(x, out))
+    assert B.stca_sync_status(m.handle) == B.OK
+    m.close()
+    ref = R.hyformer_forward(wl)
+    e = R.row_rel_err(out.cpu().numpy(), ref)
+    assert e <= TOL_BF16, e
