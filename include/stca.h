@@ -58,8 +58,9 @@ enum stca_dtype { STCA_FP32 = 0, STCA_BF16 = 1 };
 enum stca_mode { STCA_MODE_STCA = 0, STCA_MODE_POINTWISE = 1, STCA_MODE_HYFORMER = 2 };
 enum stca_score { STCA_SOFTMAX = 0, STCA_RELU = 1 };
 
-/* Model shape and capacity.  mode: enum stca_mode.  M layers (or HyFormer blocks), model width d, H heads (d_h = d/H, which must be
- * 32 for STCA_FP32 or 64 for STCA_BF16 in this build), SwiGLU hidden width `hidden`.
+/* Model shape and capacity.  mode: enum stca_mode.  M layers (or HyFormer blocks), model
+ * width d, H heads (d_h = d/H, which must be 32, 64 or 128 for STCA_FP32 and 64 for
+ * STCA_BF16 in this build), SwiGLU hidden width `hidden`.
  * time_buckets: 0, or 16 for the time-difference feature of [review] §四.
  * max_users / max_tokens / max_targets bound B, n_tok and t_tot of every later call;
  * stca_create sizes all device workspace from them, and later calls allocate nothing. */
@@ -195,6 +196,31 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
                      const int32_t* ids_search, const int32_t* len_search, int n_search,
                      const void* q0, int B, int n_query, const hyf_weights* w, float* out,
                      void* stream);
+
+/* Per-stage device timing for measurement: when enabled, each stage's launches are
+ * bracketed by CUDA events on the call's stream.  Stages: */
+enum stca_stage {
+  STCA_STAGE_SETUP = 0,      /* offsets, weight packing, input conversion */
+  STCA_STAGE_GATHER_FFN = 1, /* fused gather + X [W1|W3] + SwiGLU (tensor cores) */
+  STCA_STAGE_FFN_OUT = 2,    /* A W2 (+ LayerNorm) (tensor cores) */
+  STCA_STAGE_KV = 3,         /* X~ [W_K|W_V] (tensor cores) */
+  STCA_STAGE_ATTENTION = 4,  /* split-L attention */
+  STCA_STAGE_MERGE = 5,      /* merge of the splits */
+  STCA_STAGE_QUERY = 6,      /* target side: SwiGLU/LN, W_Q, W_O, W_C, W_Z */
+  STCA_STAGE_POINTWISE = 7,  /* fused pointwise ReLU target attention */
+  STCA_STAGE_BOOST = 8,      /* token mix + per-token SwiGLU + residual */
+  STCA_N_STAGES = 9
+};
+
+/* enable = 1 starts recording (totals reset), 0 stops it. */
+int stca_profile_enable(stca_handle* h, int enable);
+
+/* Waits for the recorded work, then writes per stage the summed device milliseconds
+ * and the number of recorded stage intervals (arrays of STCA_N_STAGES entries). */
+int stca_profile_read(stca_handle* h, double* total_ms, int64_t* calls);
+
+/* Kernel launches this library has issued since it was loaded (all handles). */
+uint64_t stca_launch_count(void);
 
 /* Synchronises the stream of the handle's last call, then returns and clears the device
  * error word (STCA_OK if no error was recorded), or STCA_ERR_CUDA. */

@@ -77,6 +77,9 @@ _SIGS = [
     ("hyformer_forward", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, ctypes.POINTER(HyfWeights),
                                 _vp, _vp]),
     ("stca_sync_status", _i32, [_vp]),
+    ("stca_profile_enable", _i32, [_vp, _i32]),
+    ("stca_profile_read", _i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
+    ("stca_launch_count", ctypes.c_uint64, []),
     ("stca_strerror", ctypes.c_char_p, [_i32]),
     ("stca_k_offsets", _i32, [_vp, _i32, _vp, _i32, _vp, _vp]),
     ("stca_k_pack_weight", _i32, [_vp, _i32, _i32, _vp, _i32, _i32, _vp]),
@@ -145,6 +148,26 @@ def stca_destroy(h):
 
 def stca_sync_status(h) -> int:
     return lib().stca_sync_status(h)
+
+
+STAGES = ["setup", "gather_ffn", "ffn_out", "kv", "attention", "merge", "query", "pointwise", "boost"]
+
+
+def stca_profile_enable(h, enable=True) -> int:
+    return lib().stca_profile_enable(h, 1 if enable else 0)
+
+
+def stca_profile_read(h):
+    """{stage: (total_ms, calls)} for the intervals recorded since enabling."""
+    n = len(STAGES)
+    ms = (ctypes.c_double * n)()
+    calls = (ctypes.c_int64 * n)()
+    check(lib().stca_profile_read(h, ms, calls), "stca_profile_read")
+    return {STAGES[i]: (ms[i], calls[i]) for i in range(n)}
+
+
+def stca_launch_count() -> int:
+    return lib().stca_launch_count()
 
 
 # --------------------------------------------------------------------------- forwards

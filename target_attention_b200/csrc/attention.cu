@@ -437,10 +437,10 @@ int attention_bf16(const AttnArgs& a, cudaStream_t s) {
   dim3 grid(a.B * a.splits, a.H);
   if (a.score == 0) {
     cudaFuncSetAttribute(attn_bf16_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_SMEM);
-    attn_bf16_kernel<0><<<grid, 128, ATTN_SMEM, s>>>(a);
+    attn_bf16_kernel<0><<<grid, 128, ATTN_SMEM, s>>>(a); note_launch();
   } else {
     cudaFuncSetAttribute(attn_bf16_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_SMEM);
-    attn_bf16_kernel<1><<<grid, 128, ATTN_SMEM, s>>>(a);
+    attn_bf16_kernel<1><<<grid, 128, ATTN_SMEM, s>>>(a); note_launch();
   }
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
@@ -449,14 +449,23 @@ int attention_f32(const AttnArgs& a, cudaStream_t s) {
   if (a.B == 0 || a.T == 0) return 0;
   const int dh = a.d / a.H;
   dim3 grid(a.B * a.splits, a.H);
-#define STCA_F32(DPL)                                                    \
-  (a.score == 0 ? (attn_f32_kernel<DPL, 0><<<grid, 128, 0, s>>>(a), 0) \
-                : (attn_f32_kernel<DPL, 1><<<grid, 128, 0, s>>>(a), 0))
-  if (dh == 32) STCA_F32(1);
-  else if (dh == 64) STCA_F32(2);
-  else if (dh == 128) STCA_F32(4);
-  else return STCA_ERR_UNSUPPORTED;
-#undef STCA_F32
+switch (dh) {
+    case 32:
+      if (a.score == 0) attn_f32_kernel<1, 0><<<grid, 128, 0, s>>>(a);
+      else attn_f32_kernel<1, 1><<<grid, 128, 0, s>>>(a);
+      break;
+    case 64:
+      if (a.score == 0) attn_f32_kernel<2, 0><<<grid, 128, 0, s>>>(a);
+      else attn_f32_kernel<2, 1><<<grid, 128, 0, s>>>(a);
+      break;
+    case 128:
+      if (a.score == 0) attn_f32_kernel<4, 0><<<grid, 128, 0, s>>>(a);
+      else attn_f32_kernel<4, 1><<<grid, 128, 0, s>>>(a);
+      break;
+    default:
+      return STCA_ERR_UNSUPPORTED;
+  }
+  note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -466,6 +475,7 @@ int attention_merge(const AttnArgs& a, cudaStream_t s) {
   const int blocks = int((warps * 32 + 255) / 256);
   if (a.score == 0) attn_merge_kernel<0><<<blocks, 256, 0, s>>>(a);
   else attn_merge_kernel<1><<<blocks, 256, 0, s>>>(a);
+  note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 

@@ -6,6 +6,9 @@
 
 namespace stca {
 
+// Counts one kernel launch of this library (read with stca_launch_count()).
+void note_launch();
+
 // Rows of A read straight from an embedding table by item id ("lookup while
 // computing"): row r of A is table[ids[r]] (+ dt_table[bucket(dt[r])]).
 struct GatherSrc {

@@ -114,11 +114,11 @@ int pointwise_relu_ta(const int32_t* ids, const int32_t* offsets, const void* q,
   float* dst = splits == 1 ? out : partials;
   pointwise_kernel<<<B * splits, PW_THREADS, 0, s>>>(ids, offsets, reinterpret_cast<const bf16*>(q),
                                                       reinterpret_cast<const bf16*>(table), n_items, B, splits, dst,
-                                                      err);
+                                                      err); note_launch();
   if (cudaGetLastError() != cudaSuccess) return STCA_ERR_CUDA;
   if (splits > 1) {
     const int64_t n = int64_t(B) * PD;
-    pointwise_sum_kernel<<<int((n + 255) / 256), 256, 0, s>>>(partials, B, splits, out);
+    pointwise_sum_kernel<<<int((n + 255) / 256), 256, 0, s>>>(partials, B, splits, out); note_launch();
     if (cudaGetLastError() != cudaSuccess) return STCA_ERR_CUDA;
   }
   return 0;

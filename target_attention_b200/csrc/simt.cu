@@ -247,7 +247,7 @@ __global__ void arange_kernel(int32_t* out, int n, int step) {
 
 int fill_arange(int32_t* out, int n, int step, cudaStream_t s) {
   if (n <= 0) return 0;
-  arange_kernel<<<(n + 255) / 256, 256, 0, s>>>(out, n, step);
+  arange_kernel<<<(n + 255) / 256, 256, 0, s>>>(out, n, step); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -258,6 +258,7 @@ int simt_gemm(const SimtGemmArgs<TA, TB>& a, cudaStream_t s) {
   dim3 grid((a.N + SB_N - 1) / SB_N, (a.M + SB_M - 1) / SB_M, a.batch);
   if (a.B2) simt_gemm_kernel<TA, TB, true><<<grid, 256, 0, s>>>(a);
   else simt_gemm_kernel<TA, TB, false><<<grid, 256, 0, s>>>(a);
+  note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -269,12 +270,12 @@ int layer_norm_f32(const float* x, int64_t ldx, float* y, int64_t ldy, int rows,
                    const float* beta, float eps, cudaStream_t s) {
   if (rows == 0) return 0;
   if (d > 1024) return STCA_ERR_UNSUPPORTED;
-  layer_norm_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, ldx, y, ldy, rows, d, gamma, beta, eps);
+  layer_norm_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, ldx, y, ldy, rows, d, gamma, beta, eps); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
 int exclusive_offsets(const int32_t* lengths, int B, int32_t* offsets, int expected, int32_t* err, cudaStream_t s) {
-  offsets_kernel<<<1, 1024, 0, s>>>(lengths, B, offsets, expected, err);
+  offsets_kernel<<<1, 1024, 0, s>>>(lengths, B, offsets, expected, err); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -285,13 +286,14 @@ int copy_rows_to_f32(const void* src, int src_bf16, int rows, int d, float* dst,
   const int blocks = int((n + 255) / 256);
   if (src_bf16) copy_rows_kernel<bf16><<<blocks, 256, 0, s>>>(reinterpret_cast<const bf16*>(src), rows, d, dst, ldd, col0);
   else copy_rows_kernel<float><<<blocks, 256, 0, s>>>(reinterpret_cast<const float*>(src), rows, d, dst, ldd, col0);
+  note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
 int token_mix(const float* Q, int B, int T, int d, float* mixed, cudaStream_t s) {
   const int64_t n = int64_t(B) * T * d;
   if (n == 0) return 0;
-  token_mix_kernel<<<int((n + 255) / 256), 256, 0, s>>>(Q, B, T, d, mixed);
+  token_mix_kernel<<<int((n + 255) / 256), 256, 0, s>>>(Q, B, T, d, mixed); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 

@@ -1,6 +1,7 @@
 // C ABI of libstca: argument checks, the workspace, and the launch sequence of each
 // forward pass.  Every step of the path runs in this library's kernels; PyTorch (or any
 // other caller) only provides device memory and the stream.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <new>
@@ -36,7 +37,20 @@ struct stca_handle {
   int32_t *in_ids = nullptr, *in_len = nullptr, *in_dt = nullptr, *in_tpu = nullptr;
   void* in_xt = nullptr;
   float* out_z = nullptr;
+  // per-stage timing
+  bool prof = false;
+  struct Rec {
+    int stage;
+    cudaEvent_t a, b;
+  };
+  std::vector<Rec> recs;
+  std::vector<cudaEvent_t> spare;
 };
+
+namespace stca {
+static std::atomic<uint64_t> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace stca
 
 namespace {
 
@@ -45,6 +59,52 @@ namespace {
     const int _rc = (x);           \
     if (_rc != STCA_OK) return _rc; \
   } while (0)
+
+cudaEvent_t take_event(stca_handle* h) {
+  if (!h->spare.empty()) {
+    cudaEvent_t e = h->spare.back();
+    h->spare.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Brackets one stage's launches with events when the handle records timings.
+struct Prof {
+  stca_handle* h;
+  int stage;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  Prof(stca_handle* h_, int stage_, cudaStream_t s_) : h(h_), stage(stage_), s(s_) {
+    if (h->prof) {
+      a = take_event(h);
+      cudaEventRecord(a, s);
+    }
+  }
+  ~Prof() {
+    if (a) {
+      cudaEvent_t b = take_event(h);
+      cudaEventRecord(b, s);
+      h->recs.push_back({stage, a, b});
+    }
+  }
+};
+
+#define STAGE(h, st, s, expr)       \
+  do {                              \
+    Prof _prof((h), (st), (s));     \
+    CK(expr);                       \
+  } while (0)
+
+void recycle_events(stca_handle* h) {
+  for (auto& r : h->recs) {
+    h->spare.push_back(r.a);
+    h->spare.push_back(r.b);
+  }
+  h->recs.clear();
+}
 
 template <typename T>
 bool dalloc(stca_handle* h, T** p, size_t bytes) {
@@ -206,10 +266,13 @@ int history_bf16(stca_handle* h, size_t slot, const GatherSrc& g, int n_tok, con
   const bf16* wp3 = wp2 + size_t(d) * hd;
   GatherSrc none;
   memset(&none, 0, sizeof(none));
-  CK(tc_gemm_resident(A_GATHER, EPI_SWIGLU, nullptr, g, n_tok, d, wp1, hd, h->hidden, hd, h->err, s));
-  CK(tc_gemm_rowwise(gamma ? EPI_LN : EPI_PLAIN, h->hidden, n_tok, hd, wp2, d, gamma, beta, h->cfg.ln_eps, h->xt, d,
-                     h->err, s));
-  CK(tc_gemm_resident(A_TMA, EPI_PLAIN, h->xt, none, n_tok, d, wp3, 2 * d, h->kv, 2 * d, h->err, s));
+  STAGE(h, STCA_STAGE_GATHER_FFN, s,
+        tc_gemm_resident(A_GATHER, EPI_SWIGLU, nullptr, g, n_tok, d, wp1, hd, h->hidden, hd, h->err, s));
+  STAGE(h, STCA_STAGE_FFN_OUT, s,
+        tc_gemm_rowwise(gamma ? EPI_LN : EPI_PLAIN, h->hidden, n_tok, hd, wp2, d, gamma, beta, h->cfg.ln_eps, h->xt,
+                        d, h->err, s));
+  STAGE(h, STCA_STAGE_KV, s,
+        tc_gemm_resident(A_TMA, EPI_PLAIN, h->xt, none, n_tok, d, wp3, 2 * d, h->kv, 2 * d, h->err, s));
   return STCA_OK;
 }
 
@@ -223,11 +286,17 @@ int history_f32(stca_handle* h, const GatherSrc& g, int n_tok, const stca_ffn& f
   auto a = gemm_args<float>(n_tok, hd, d, nullptr, d, f.W1, hid, hd, h->err);
   a.B2 = reinterpret_cast<const float*>(f.W3);
   a.gather = g;
-  CK(simt_gemm(a, s));
-  CK(simt_gemm(gemm_args<float>(n_tok, d, hd, hid, hd, f.W2, xt, d, h->err), s));
-  CK(layer_norm_f32(xt, d, xt, d, n_tok, d, f.gamma, f.beta, h->cfg.ln_eps, s));
-  CK(simt_gemm(gemm_args<float>(n_tok, d, d, xt, d, WK, kv, 2 * d, h->err), s));
-  CK(simt_gemm(gemm_args<float>(n_tok, d, d, xt, d, WV, kv + d, 2 * d, h->err), s));
+  STAGE(h, STCA_STAGE_GATHER_FFN, s, simt_gemm(a, s));
+  {
+    Prof p(h, STCA_STAGE_FFN_OUT, s);
+    CK(simt_gemm(gemm_args<float>(n_tok, d, hd, hid, hd, f.W2, xt, d, h->err), s));
+    CK(layer_norm_f32(xt, d, xt, d, n_tok, d, f.gamma, f.beta, h->cfg.ln_eps, s));
+  }
+  {
+    Prof p(h, STCA_STAGE_KV, s);
+    CK(simt_gemm(gemm_args<float>(n_tok, d, d, xt, d, WK, kv, 2 * d, h->err), s));
+    CK(simt_gemm(gemm_args<float>(n_tok, d, d, xt, d, WV, kv + d, 2 * d, h->err), s));
+  }
   return STCA_OK;
 }
 
@@ -248,8 +317,8 @@ int run_attention(stca_handle* h, const float* Q, const int32_t* hoff, const int
   a.part_ml = h->part_ml;
   a.out = h->attn;
   a.err = h->err;
-  CK(h->cfg.dtype == STCA_BF16 ? attention_bf16(a, s) : attention_f32(a, s));
-  CK(attention_merge(a, s));
+  STAGE(h, STCA_STAGE_ATTENTION, s, h->cfg.dtype == STCA_BF16 ? attention_bf16(a, s) : attention_f32(a, s));
+  STAGE(h, STCA_STAGE_MERGE, s, attention_merge(a, s));
   return STCA_OK;
 }
 
@@ -261,14 +330,17 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
   const int d = c.d, M = c.M;
   const bool bf = c.dtype == STCA_BF16;
   const int64_t ldcat = int64_t(M + 1) * d;
-  CK(exclusive_offsets(lens, B, h->hoff, n_tok, h->err, s));
-  CK(exclusive_offsets(tpu, B, h->toff, t_tot, h->err, s));
-  CK(copy_rows_to_f32(x_t, bf, t_tot, d, h->cat, ldcat, M * d, s));
-  if (bf)
-    for (int i = 0; i < M; ++i) CK(pack_layer(h, i, w->hist[i], w->WK[i], w->WV[i], s));
+  {
+    Prof p(h, STCA_STAGE_SETUP, s);
+    CK(exclusive_offsets(lens, B, h->hoff, n_tok, h->err, s));
+    CK(exclusive_offsets(tpu, B, h->toff, t_tot, h->err, s));
+    CK(copy_rows_to_f32(x_t, bf, t_tot, d, h->cat, ldcat, M * d, s));
+    if (bf)
+      for (int i = 0; i < M; ++i) CK(pack_layer(h, i, w->hist[i], w->WK[i], w->WV[i], s));
+  }
   const float* xcol = h->cat + int64_t(M) * d;
   // q^(1) = LN(SwiGLU_t(x_t))
-  CK(query_ffn<TB>(h, xcol, ldcat, t_tot, w->tgt, h->qbuf, d, s));
+  STAGE(h, STCA_STAGE_QUERY, s, query_ffn<TB>(h, xcol, ldcat, t_tot, w->tgt, h->qbuf, d, s));
   GatherSrc g;
   g.ids = ids;
   g.dt = c.time_buckets ? dt : nullptr;
@@ -279,8 +351,10 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
   for (int i = 0; i < M; ++i) {
     if (bf) CK(history_bf16(h, i, g, n_tok, w->hist[i].gamma, w->hist[i].beta, s));
     else CK(history_f32(h, g, n_tok, w->hist[i], w->WK[i], w->WV[i], s));
-    CK(simt_gemm(gemm_args<TB>(t_tot, d, d, h->qbuf, d, w->WQ[i], h->qproj, d, h->err), s));
+    STAGE(h, STCA_STAGE_QUERY, s,
+          simt_gemm(gemm_args<TB>(t_tot, d, d, h->qbuf, d, w->WQ[i], h->qproj, d, h->err), s));
     CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, splits, c.score, s));
+    Prof p(h, STCA_STAGE_QUERY, s);
     CK(simt_gemm(gemm_args<TB>(t_tot, d, d, h->attn, d, w->WO[i], h->cat + int64_t(i) * d, ldcat, h->err), s));
     if (i + 1 < M) {
       // q^(i+2) = LN(SwiGLU([o^(1) .. o^(i+1) | x_t] W_C))
@@ -293,8 +367,11 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
     }
   }
   // z = SwiGLU_Z([o^(1) .. o^(M) | x_t] W_Z)
-  CK(simt_gemm(gemm_args<TB>(t_tot, d, int(ldcat), h->cat, ldcat, w->WZ, h->tmp_d, d, h->err), s));
-  CK(query_ffn<TB>(h, h->tmp_d, d, t_tot, w->zffn, z_out, d, s));
+  {
+    Prof p(h, STCA_STAGE_QUERY, s);
+    CK(simt_gemm(gemm_args<TB>(t_tot, d, int(ldcat), h->cat, ldcat, w->WZ, h->tmp_d, d, h->err), s));
+    CK(query_ffn<TB>(h, h->tmp_d, d, t_tot, w->zffn, z_out, d, s));
+  }
   if (o_out && t_tot > 0) {
     for (int i = 0; i < M; ++i)
       if (cudaMemcpy2DAsync(o_out + int64_t(i) * t_tot * d, size_t(d) * 4, h->cat + int64_t(i) * d, size_t(ldcat) * 4,
@@ -359,6 +436,9 @@ int stca_create(const stca_config* cfg, stca_handle** out) {
 void stca_destroy(stca_handle* h) {
   if (!h) return;
   cudaSetDevice(h->device);
+  if (!h->recs.empty()) cudaDeviceSynchronize();
+  recycle_events(h);
+  for (cudaEvent_t e : h->spare) cudaEventDestroy(e);
   free_all(h);
   delete h;
 }
@@ -417,9 +497,11 @@ int stca_pointwise_forward(stca_handle* h, const int32_t* ids, const int32_t* le
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   h->last_stream = s;
   if (B == 0) return STCA_OK;
-  CK(exclusive_offsets(lengths, B, h->hoff, n_tok, h->err, s));
+  STAGE(h, STCA_STAGE_SETUP, s, exclusive_offsets(lengths, B, h->hoff, n_tok, h->err, s));
   const int splits = choose_splits(n_tok, B, 2048);
-  return pointwise_relu_ta(ids, h->hoff, q, table, n_items, B, h->cfg.d, splits, h->part_acc, out, h->err, s);
+  STAGE(h, STCA_STAGE_POINTWISE, s,
+        pointwise_relu_ta(ids, h->hoff, q, table, n_items, B, h->cfg.d, splits, h->part_acc, out, h->err, s));
+  return STCA_OK;
 }
 
 int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len_feed, int n_feed,
@@ -449,15 +531,18 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
   h->last_stream = s;
   if (B == 0) return STCA_OK;
   const int rows = B * T, rows_s = B * n_query;
-  CK(exclusive_offsets(len_feed, B, h->hoff, n_feed, h->err, s));
-  CK(exclusive_offsets(len_search, B, h->hoff2, n_search, h->err, s));
-  CK(fill_arange(h->toff, B + 1, n_query, s));
-  CK(copy_rows_to_f32(q0, 1, rows, d, h->hq, d, 0, s));
-  for (int l = 0; l < c.M; ++l)
-    for (int sq = 0; sq < 2; ++sq) {
-      const hyf_seq_weights& f = w->blk[l].seq[sq];
-      CK(pack_layer(h, size_t(l) * 2 + sq, f.ffn, f.WK, f.WV, s));
-    }
+  {
+    Prof p(h, STCA_STAGE_SETUP, s);
+    CK(exclusive_offsets(len_feed, B, h->hoff, n_feed, h->err, s));
+    CK(exclusive_offsets(len_search, B, h->hoff2, n_search, h->err, s));
+    CK(fill_arange(h->toff, B + 1, n_query, s));
+    CK(copy_rows_to_f32(q0, 1, rows, d, h->hq, d, 0, s));
+    for (int l = 0; l < c.M; ++l)
+      for (int sq = 0; sq < 2; ++sq) {
+        const hyf_seq_weights& f = w->blk[l].seq[sq];
+        CK(pack_layer(h, size_t(l) * 2 + sq, f.ffn, f.WK, f.WV, s));
+      }
+  }
   const int32_t* ids[2] = {ids_feed, ids_search};
   const int32_t* offs[2] = {h->hoff, h->hoff2};
   const int ntok[2] = {n_feed, n_search};
@@ -476,15 +561,16 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
       qa.a_grp = n_query;
       qa.a_gstride = T;
       qa.a_goff = sq * n_query;
-      CK(simt_gemm(qa, s));
+      STAGE(h, STCA_STAGE_QUERY, s, simt_gemm(qa, s));
       CK(run_attention(h, h->qproj, offs[sq], h->toff, B, rows_s, choose_splits(ntok[sq], B, 1024), STCA_SOFTMAX, s));
       auto oa = gemm_args<bf16>(rows_s, d, d, h->attn, d, f.WO, h->hqhat, d, h->err);
       oa.c_grp = n_query;
       oa.c_gstride = T;
       oa.c_goff = sq * n_query;
-      CK(simt_gemm(oa, s));
+      STAGE(h, STCA_STAGE_QUERY, s, simt_gemm(oa, s));
     }
     // query boosting: token mix (eq 11-13), per-token SwiGLU (eq 14), residual (eq 15)
+    Prof p(h, STCA_STAGE_BOOST, s);
     CK(token_mix(h->hqhat, B, T, d, h->hmix, s));
     auto a1 = gemm_args<bf16>(B, hd, d, h->hmix, int64_t(T) * d, nullptr, h->tmp_h, int64_t(T) * hd, h->err);
     a1.batch = T;
@@ -509,6 +595,34 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
   }
   return STCA_OK;
 }
+
+int stca_profile_enable(stca_handle* h, int enable) {
+  if (!h) return STCA_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  if (!h->recs.empty() && cudaDeviceSynchronize() != cudaSuccess) return STCA_ERR_CUDA;
+  recycle_events(h);
+  h->prof = enable != 0;
+  return STCA_OK;
+}
+
+int stca_profile_read(stca_handle* h, double* total_ms, int64_t* calls) {
+  if (!h || !total_ms || !calls) return STCA_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  for (int i = 0; i < STCA_N_STAGES; ++i) {
+    total_ms[i] = 0.0;
+    calls[i] = 0;
+  }
+  for (auto& r : h->recs) {
+    if (cudaEventSynchronize(r.b) != cudaSuccess) return STCA_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) return STCA_ERR_CUDA;
+    total_ms[r.stage] += ms;
+    calls[r.stage] += 1;
+  }
+  return STCA_OK;
+}
+
+uint64_t stca_launch_count(void) { return stca::g_launches.load(); }
 
 int stca_sync_status(stca_handle* h) {
   if (!h) return STCA_ERR_INVALID_ARG;

@@ -10,9 +10,10 @@
 // shared memory as K-major rows of 128 bytes with the 128-byte swizzle; TMA writes that
 // layout for dense operands, and the fused gather producer writes it with cp.async.
 //
-// Warp roles (256 threads): warp 0 lane 0 issues TMA, warp 1 owns TMEM and lane 0
-// issues tcgen05.mma, warps 4..7 (TMEM lane quarters 0..3) gather A rows and run the
-// epilogue.  Waits are bounded (see common.cuh).
+// Warp roles (384 threads): warp 0 lane 0 issues TMA, warp 1 owns TMEM and lane 0
+// issues tcgen05.mma, warps 4..11 gather A rows and run the epilogue, two warps per TMEM
+// lane quarter (warp w reads lanes 32 (w % 4) .. + 32), each on half of the columns.
+// Waits are bounded (see common.cuh).
 #include <mutex>
 
 #include "common.cuh"
@@ -61,11 +62,12 @@ __device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
   }
 }
 
-// Gather producer: thread r (0..127) loads row r of the A tile, all K chunks, with
-// cp.async into the swizzled K-major layout, then (time feature) adds the bucket row
-// and releases chunk kc on a_full[kc] as soon as it has landed.
+// Gather producer, 256 threads: thread (r, half) loads 16-byte chunks [4 half, 4 half + 4)
+// of row r of the A tile for every K chunk, with cp.async into the swizzled K-major
+// layout, then (time feature) adds the bucket row, and releases chunk kc on a_full[kc]
+// as soon as its own copies have landed.
 __device__ __forceinline__ void gather_a_tile(const GatherSrc& g, uint8_t* sA, uint64_t* a_full, int m0,
-                                              int M, int K, int r, int32_t* err) {
+                                              int M, int K, int r, int half, int32_t* err) {
   const int KC = K / 64;
   const int grow = m0 + r;
   bool valid = grow < M;
@@ -84,27 +86,36 @@ __device__ __forceinline__ void gather_a_tile(const GatherSrc& g, uint8_t* sA, u
       bucket = dt_bucket(dt < 0 ? 0 : dt);
     }
   }
-  const bf16* src = reinterpret_cast<const bf16*>(g.table) + id * int64_t(K);
+  const bf16* src = reinterpret_cast<const bf16*>(g.table) + id * int64_t(K) + half * 32;
   const uint32_t nbytes = valid ? 16u : 0u;
   for (int kc = 0; kc < KC; ++kc) {
     uint8_t* rowp = sA + kc * A_CHUNK + r * 128;
 #pragma unroll
-    for (int c = 0; c < 8; ++c)
-      cp_async_16(rowp + ((c ^ (r & 7)) << 4), src + kc * 64 + c * 8, nbytes);
+    for (int c = 0; c < 4; ++c)
+      cp_async_16(rowp + (((half * 4 + c) ^ (r & 7)) << 4), src + kc * 64 + c * 8, nbytes);
     cp_async_commit();
   }
-  const bf16* trow = g.dt_table ? reinterpret_cast<const bf16*>(g.dt_table) + int64_t(bucket) * K : nullptr;
+  const bf16* trow = (g.dt_table != nullptr && grow < M)
+                         ? reinterpret_cast<const bf16*>(g.dt_table) + int64_t(bucket) * K + half * 32
+                         : nullptr;
+  uint4 t[4];
+  if (trow != nullptr)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) t[c] = __ldg(reinterpret_cast<const uint4*>(trow) + c);
   for (int kc = 0; kc < KC; ++kc) {
     cp_async_wait_dyn(KC - 1 - kc);
-    if (trow != nullptr && grow < M) {
+    if (trow != nullptr) {
+      uint4 tn[4];
+      if (kc + 1 < KC)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tn[c] = __ldg(reinterpret_cast<const uint4*>(trow + (kc + 1) * 64) + c);
       uint8_t* rowp = sA + kc * A_CHUNK + r * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4* p = reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4));
+      for (int c = 0; c < 4; ++c) {
+        uint4* p = reinterpret_cast<uint4*>(rowp + (((half * 4 + c) ^ (r & 7)) << 4));
         uint4 x = *p;
-        const uint4 t = __ldg(reinterpret_cast<const uint4*>(trow + kc * 64 + c * 8));
         const __nv_bfloat162* xa = reinterpret_cast<const __nv_bfloat162*>(&x);
-        const __nv_bfloat162* ta = reinterpret_cast<const __nv_bfloat162*>(&t);
+        const __nv_bfloat162* ta = reinterpret_cast<const __nv_bfloat162*>(&t[c]);
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -114,18 +125,32 @@ __device__ __forceinline__ void gather_a_tile(const GatherSrc& g, uint8_t* sA, u
         }
         *p = make_uint4(o[0], o[1], o[2], o[3]);
       }
+      if (kc + 1 < KC)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) t[c] = tn[c];
     }
     fence_proxy_async_smem();
     mbar_arrive(&a_full[kc]);
   }
 }
 
+// SiLU(x) = x sigmoid(x) = h + h tanh(h) with h = x/2: one MUFU op per element.
+__device__ __forceinline__ float silu_tanh(float x) {
+  const float h = 0.5f * x;
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(h));
+  return fmaf(h, t, h);
+}
+
+// Named barrier over the 256 epilogue threads (warps 4..11).
+__device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 // ------------------------------------------------------------------------------------
 // Kernel R: A resident in shared memory (K <= 512), N walked in 256-column tiles with a
 // double-buffered TMEM accumulator so the epilogue of tile n overlaps the MMAs of n+1.
 
 template <int AMODE, int EPI, int STAGES>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     tc_gemm_resident_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             GatherSrc g, int M, int K, int NT, bf16* __restrict__ C, int ldc, int32_t* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -147,14 +172,14 @@ __global__ void __launch_bounds__(256, 1)
   const int m0 = blockIdx.x * BM;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < KC; ++i) mbar_init(&a_full[i], AMODE == A_GATHER ? 128 : 1);
+    for (int i = 0; i < KC; ++i) mbar_init(&a_full[i], AMODE == A_GATHER ? 256 : 1);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&t_full[i], 1);
-      mbar_init(&t_empty[i], 128);
+      mbar_init(&t_empty[i], 256);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -233,9 +258,11 @@ __global__ void __launch_bounds__(256, 1)
       mbar_wait(mma_done, 0);
     }
   } else if (warp >= 4) {
+    // two epilogue warps per TMEM lane quarter, each taking half of the columns
     const int quarter = warp & 3;
+    const int half = (warp - 4) >> 2;
     const int r = quarter * 32 + lane;  // tile row == TMEM lane
-    if (AMODE == A_GATHER) gather_a_tile(g, sA, a_full, m0, M, K, r, err);
+    if (AMODE == A_GATHER) gather_a_tile(g, sA, a_full, m0, M, K, r, half, err);
     const int grow = m0 + r;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
     for (int nt = 0; nt < NT; ++nt) {
@@ -248,22 +275,24 @@ __global__ void __launch_bounds__(256, 1)
       const uint32_t tb = lane_base + buf * 256;
       if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < 2; ++j) {
+          const int col = half * 64 + j * 32;
           float gv[32], uv[32];
-          tmem_ld_32x32b_x32(tb + j * 32, gv);
-          tmem_ld_32x32b_x32(tb + 128 + j * 32, uv);
+          tmem_ld_32x32b_x32(tb + col, gv);
+          tmem_ld_32x32b_x32(tb + 128 + col, uv);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) gv[e] = silu_f(gv[e]) * uv[e];
-          if (grow < M) store_bf16x32(C + int64_t(grow) * ldc + nt * 128 + j * 32, gv);
+          for (int e = 0; e < 32; ++e) gv[e] = silu_tanh(gv[e]) * uv[e];
+          if (grow < M) store_bf16x32(C + int64_t(grow) * ldc + nt * 128 + col, gv);
         }
       } else {
 #pragma unroll 1
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
+          const int col = half * 128 + j * 32;
           float v[32];
-          tmem_ld_32x32b_x32(tb + j * 32, v);
+          tmem_ld_32x32b_x32(tb + col, v);
           tmem_ld_wait();
-          if (grow < M) store_bf16x32(C + int64_t(grow) * ldc + nt * 256 + j * 32, v);
+          if (grow < M) store_bf16x32(C + int64_t(grow) * ldc + nt * 256 + col, v);
         }
       }
       tc_fence_before();
@@ -283,7 +312,7 @@ __global__ void __launch_bounds__(256, 1)
 // columns) accumulated in TMEM, then LayerNorm (or a plain store) per row.
 
 template <int EPI, int NB, int STAGES>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     tc_gemm_rowwise_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            int M, int K, bf16* __restrict__ C, int ldc, const float* __restrict__ gamma,
                            const float* __restrict__ beta, float eps, int32_t* err) {
@@ -298,6 +327,9 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* mma_done = t_full + 1;        // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_gamma = reinterpret_cast<float*>(bars + 2 * STAGES + 8);  // [N]
+  float* s_beta = s_gamma + N;                                       // [N]
+  float* s_red = s_beta + N;                                         // [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * BM;
@@ -373,56 +405,76 @@ __global__ void __launch_bounds__(256, 1)
     }
   } else if (warp >= 4) {
     const int quarter = warp & 3;
+    const int half = (warp - 4) >> 2;
     const int r = quarter * 32 + lane;
     const int grow = m0 + r;
-    const uint32_t tb = tmem + (uint32_t(quarter * 32) << 16);
-    if (mbar_wait(t_full, 0) && !abort_set(abort_flag)) {
-      tc_fence_after();
-      bf16* crow = C + int64_t(grow) * ldc;
-      if (EPI == EPI_LN) {
-        float sum = 0.f;
+    const int et = threadIdx.x - 128;
+    constexpr int HN = N / 2;  // columns per epilogue warp
+    if (EPI == EPI_LN) {
+      for (int c = et; c < N; c += 256) {
+        s_gamma[c] = gamma[c];
+        s_beta[c] = beta[c];
+      }
+    }
+    const uint32_t tb = tmem + (uint32_t(quarter * 32) << 16) + half * HN;
+    const bool ok = mbar_wait(t_full, 0) && !abort_set(abort_flag);
+    if (!ok) fail(abort_flag, err);
+    tc_fence_after();
+    bf16* crow = C + int64_t(grow) * ldc + half * HN;
+    if (EPI == EPI_LN) {
+      float sum = 0.f;
+      if (ok) {
 #pragma unroll 1
-        for (int j = 0; j < N / 32; ++j) {
+        for (int j = 0; j < HN / 32; ++j) {
           float v[32];
           tmem_ld_32x32b_x32(tb + j * 32, v);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) sum += v[e];
         }
-        const float mean = sum * (1.0f / N);
-        float sq = 0.f;
+      }
+      s_red[half * 128 + r] = sum;
+      epilogue_sync();
+      const float mean = (s_red[r] + s_red[128 + r]) * (1.0f / N);
+      float sq = 0.f;
+      if (ok) {
 #pragma unroll 1
-        for (int j = 0; j < N / 32; ++j) {
+        for (int j = 0; j < HN / 32; ++j) {
           float v[32];
           tmem_ld_32x32b_x32(tb + j * 32, v);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const float t = v[e] - mean;
-            sq += t * t;
+            sq = fmaf(t, t, sq);
           }
         }
-        const float rstd = rsqrtf(sq * (1.0f / N) + eps);
+      }
+      epilogue_sync();  // everyone has read the sums before they are overwritten
+      s_red[half * 128 + r] = sq;
+      epilogue_sync();
+      const float rstd = rsqrtf((s_red[r] + s_red[128 + r]) * (1.0f / N) + eps);
+      if (ok) {
+        const float* gm = s_gamma + half * HN;
+        const float* bt = s_beta + half * HN;
 #pragma unroll 1
-        for (int j = 0; j < N / 32; ++j) {
+        for (int j = 0; j < HN / 32; ++j) {
           float v[32];
           tmem_ld_32x32b_x32(tb + j * 32, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = (v[e] - mean) * rstd * __ldg(gamma + j * 32 + e) + __ldg(beta + j * 32 + e);
-          if (grow < M) store_bf16x32(crow + j * 32, v);
-        }
-      } else {
-#pragma unroll 1
-        for (int j = 0; j < N / 32; ++j) {
-          float v[32];
-          tmem_ld_32x32b_x32(tb + j * 32, v);
-          tmem_ld_wait();
+          for (int e = 0; e < 32; ++e) v[e] = fmaf((v[e] - mean) * rstd, gm[j * 32 + e], bt[j * 32 + e]);
           if (grow < M) store_bf16x32(crow + j * 32, v);
         }
       }
-    } else {
-      fail(abort_flag, err);
+    } else if (ok) {
+#pragma unroll 1
+      for (int j = 0; j < HN / 32; ++j) {
+        float v[32];
+        tmem_ld_32x32b_x32(tb + j * 32, v);
+        tmem_ld_wait();
+        if (grow < M) store_bf16x32(crow + j * 32, v);
+      }
     }
   }
   tc_fence_before();
@@ -490,22 +542,13 @@ bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename Kern>
-int launch_tc(Kern kern, int grid, size_t smem, cudaStream_t s, const CUtensorMap& a, const CUtensorMap& b) {
-  (void)a;
-  (void)b;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-    return STCA_ERR_CUDA;
-  return 0;
-}
-
 size_t resident_smem(int K, int stages) {
   size_t bytes = 1024 + size_t(K / 64) * A_CHUNK + size_t(stages) * B_STAGE_256 + 256;
   return bytes < MIN_SMEM ? MIN_SMEM : bytes;
 }
 
 size_t rowwise_smem(int nb, int stages) {
-  size_t bytes = 1024 + size_t(stages) * (A_CHUNK + nb * B_STAGE_256) + 256;
+  size_t bytes = 1024 + size_t(stages) * (A_CHUNK + nb * B_STAGE_256) + 256 + 2 * nb * 256 * 4 + 2 * 128 * 4;
   return bytes < MIN_SMEM ? MIN_SMEM : bytes;
 }
 
@@ -517,7 +560,7 @@ int run_resident(const CUtensorMap& ta, const CUtensorMap& tb, const GatherSrc& 
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
   const int grid = (M + BM - 1) / BM;
-  kern<<<grid, 256, smem, s>>>(ta, tb, g, M, K, NT, reinterpret_cast<bf16*>(C), ldc, err);
+  kern<<<grid, 384, smem, s>>>(ta, tb, g, M, K, NT, reinterpret_cast<bf16*>(C), ldc, err); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -529,7 +572,7 @@ int run_rowwise(const CUtensorMap& ta, const CUtensorMap& tb, int M, int K, void
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
   const int grid = (M + BM - 1) / BM;
-  kern<<<grid, 256, smem, s>>>(ta, tb, M, K, reinterpret_cast<bf16*>(C), ldc, gamma, beta, eps, err);
+  kern<<<grid, 384, smem, s>>>(ta, tb, M, K, reinterpret_cast<bf16*>(C), ldc, gamma, beta, eps, err); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -539,7 +582,7 @@ int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_off
   if (K <= 0 || N <= 0) return STCA_ERR_INVALID_ARG;
   dim3 grid((N + 31) / 32, (K + 31) / 32), block(32, 8);
   pack_weight_kernel<<<grid, block, 0, s>>>(reinterpret_cast<const bf16*>(W), K, N, reinterpret_cast<bf16*>(dst),
-                                            mode, row_offset);
+                                            mode, row_offset); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 

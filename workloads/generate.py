@@ -139,12 +139,19 @@ def _ffn(g, d, hidden, dtype, affine=None, ln=True):
 
 
 def make_stca(config_id: int, *, users=None, L=None, n_items=None, m=None, lengths=None,
-              seed=None, ln_affine="random", **over) -> dict:
-    """Inputs and random-init weights for an STCA workload (configs 1-3 and variants)."""
+              seed=None, data_seed=None, ln_affine="random", **over) -> dict:
+    """Inputs and random-init weights for an STCA workload (configs 1-3 and variants).
+
+    ``data_seed``, when given, draws the per-request inputs (lengths, ids, dt, x_t) from
+    its own seed while the table and weights keep ``seed``: several replicas then serve
+    different users with the same model.
+    """
     cfg = _config(config_id, users=users, L=L, n_items=n_items, m=m, **over)
     assert cfg["kind"] == "stca"
     ss = np.random.SeedSequence(1000 + config_id if seed is None else seed)
     s_len, s_ids, s_dt, s_xt, s_tab, s_dtab, s_w = ss.spawn(7)
+    if data_seed is not None:
+        s_len, s_ids, s_dt, s_xt = np.random.SeedSequence(data_seed).spawn(4)
     dtype, d, hidden, M = cfg["dtype"], cfg["d"], cfg["hidden"], cfg["M"]
     B = cfg["users"]
     if lengths is None:
