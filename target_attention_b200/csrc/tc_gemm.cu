@@ -10,10 +10,14 @@
 // shared memory as K-major rows of 128 bytes with the 128-byte swizzle; TMA writes that
 // layout for dense operands, and the fused gather producer writes it with cp.async.
 //
-// Warp roles (384 threads): warp 0 lane 0 issues TMA, warp 1 owns TMEM and lane 0
-// issues tcgen05.mma, warps 4..11 gather A rows and run the epilogue, two warps per TMEM
-// lane quarter (warp w reads lanes 32 (w % 4) .. + 32), each on half of the columns.
+// A pair of CTAs (a cluster of 2) computes 256-row tiles with cta_group::2 MMAs: each CTA
+// holds its 128 rows of A and half of each weight tile, so each SM streams half the
+// weight bytes.  The kernels are persistent (one pair per two SMs).  Warp roles: warp 0
+// lane 0 issues TMA, warp 1 owns TMEM and (leader CTA) lane 0 issues tcgen05.mma, warps
+// 4..11 run the epilogue, two warps per TMEM lane quarter (warp w reads lanes
+// 32 (w % 4) .. + 32), each on half of the columns; warps 12..15 gather A rows.
 // Waits are bounded (see common.cuh).
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -25,8 +29,9 @@ namespace {
 
 constexpr int BM = 128;                        // tile rows = TMEM lanes
 constexpr int A_CHUNK = BM * 64 * 2;           // one 64-wide K chunk of A: 16 KB
-constexpr int B_BOX_ROWS = 256;                // TMA box height for weights
-constexpr int B_STAGE_256 = B_BOX_ROWS * 128;  // 256 weight rows x 64 K: 32 KB
+constexpr int B_HALF = BM * 128;               // one CTA's 128 weight rows x 64 K: 16 KB
+constexpr int OUT_STAGE = 32 * 64;             // one epilogue warp's 32 x 32 bf16 output tile
+constexpr int T_BYTES = 16 * 512 * 2;          // time-bucket table, K <= 512
 constexpr int MIN_SMEM = 120 * 1024;           // keeps one CTA per SM (TMEM is not shared)
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -48,89 +53,29 @@ __device__ __forceinline__ void drain_ring(uint64_t* full, int stages, int issue
   }
 }
 
-// Epilogue store of 32 consecutive fp32 values as bf16 (64 bytes, 16-byte aligned).
-__device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+// Epilogue store: lane r of a warp holds 32 consecutive fp32 values of output row r of
+// the warp's 32-row block.  They are staged as bf16 in the warp's 2 KB shared buffer
+// (64-byte rows with the 64-byte swizzle: 16-byte chunk c of row r sits at chunk
+// c ^ ((r >> 1) & 3), which keeps the lanes' writes on distinct banks) and written with
+// one TMA tile store of 32 x 32 at (x, y); rows or columns outside C are clipped by TMA.
+// The buffer is reused once the previous store has read it.
+__device__ __forceinline__ void epi_store(uint8_t* stage, const float (&v)[32], int lane, const CUtensorMap* tmC,
+                                          int x, int y) {
+  uint32_t packed[16];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    uint4 u;
-    u.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
-    u.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
-    u.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
-    u.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
-    d4[q] = u;
-  }
-}
-
-// Gather producer, 256 threads: thread (r, half) loads 16-byte chunks [4 half, 4 half + 4)
-// of row r of the A tile for every K chunk, with cp.async into the swizzled K-major
-// layout, then (time feature) adds the bucket row, and releases chunk kc on a_full[kc]
-// as soon as its own copies have landed.
-__device__ __forceinline__ void gather_a_tile(const GatherSrc& g, uint8_t* sA, uint64_t* a_full, int m0,
-                                              int M, int K, int r, int half, int32_t* err) {
-  const int KC = K / 64;
-  const int grow = m0 + r;
-  bool valid = grow < M;
-  int64_t id = 0;
-  int bucket = 0;
-  if (valid) {
-    id = g.ids[grow];
-    if (id < 0 || id >= g.n_items) {
-      set_error(err, STCA_ERR_ID_OUT_OF_RANGE);
-      valid = false;
-      id = 0;
-    }
-    if (g.dt) {
-      const int32_t dt = g.dt[grow];
-      if (dt < 0) set_error(err, STCA_ERR_INVALID_ARG);
-      bucket = dt_bucket(dt < 0 ? 0 : dt);
-    }
-  }
-  const bf16* src = reinterpret_cast<const bf16*>(g.table) + id * int64_t(K) + half * 32;
-  const uint32_t nbytes = valid ? 16u : 0u;
-  for (int kc = 0; kc < KC; ++kc) {
-    uint8_t* rowp = sA + kc * A_CHUNK + r * 128;
+  for (int q = 0; q < 16; ++q) packed[q] = pack_bf16x2(v[2 * q], v[2 * q + 1]);
+  if (lane == 0) bulk_wait_read<0>();
+  __syncwarp();
+  uint8_t* rowp = stage + lane * 64;
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
-      cp_async_16(rowp + (((half * 4 + c) ^ (r & 7)) << 4), src + kc * 64 + c * 8, nbytes);
-    cp_async_commit();
-  }
-  const bf16* trow = (g.dt_table != nullptr && grow < M)
-                         ? reinterpret_cast<const bf16*>(g.dt_table) + int64_t(bucket) * K + half * 32
-                         : nullptr;
-  uint4 t[4];
-  if (trow != nullptr)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) t[c] = __ldg(reinterpret_cast<const uint4*>(trow) + c);
-  for (int kc = 0; kc < KC; ++kc) {
-    cp_async_wait_dyn(KC - 1 - kc);
-    if (trow != nullptr) {
-      uint4 tn[4];
-      if (kc + 1 < KC)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tn[c] = __ldg(reinterpret_cast<const uint4*>(trow + (kc + 1) * 64) + c);
-      uint8_t* rowp = sA + kc * A_CHUNK + r * 128;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint4* p = reinterpret_cast<uint4*>(rowp + (((half * 4 + c) ^ (r & 7)) << 4));
-        uint4 x = *p;
-        const __nv_bfloat162* xa = reinterpret_cast<const __nv_bfloat162*>(&x);
-        const __nv_bfloat162* ta = reinterpret_cast<const __nv_bfloat162*>(&t[c]);
-        uint32_t o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 xf = __bfloat1622float2(xa[e]);
-          const float2 tf = __bfloat1622float2(ta[e]);
-          o[e] = pack_bf16x2(xf.x + tf.x, xf.y + tf.y);
-        }
-        *p = make_uint4(o[0], o[1], o[2], o[3]);
-      }
-      if (kc + 1 < KC)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) t[c] = tn[c];
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(&a_full[kc]);
+  for (int c = 0; c < 4; ++c)
+    *reinterpret_cast<uint4*>(rowp + ((c ^ ((lane >> 1) & 3)) << 4)) =
+        make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmC, x, y, stage);
+    bulk_commit();
   }
 }
 
@@ -145,52 +90,110 @@ __device__ __forceinline__ float silu_tanh(float x) {
 // Named barrier over the 256 epilogue threads (warps 4..11).
 __device__ __forceinline__ void epilogue_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
+// Same barrier, returning whether any of the 256 epilogue threads passed `flag` != 0, so
+// that they all take the same branch afterwards.
+__device__ __forceinline__ bool epilogue_any(bool flag) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 256, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(flag))
+      : "memory");
+  return r != 0;
+}
+
+// Named barrier over the 128 gather threads (warps 12..15).
+__device__ __forceinline__ void gather_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+// Item id and time bucket of global row `grow`; false (and a zero row) when the row is
+// past M or the id is out of range (recorded in the error word).
+__device__ __forceinline__ bool gather_row(const GatherSrc& g, int grow, int M, int64_t& id, int& bucket,
+                                           int32_t* err) {
+  id = 0;
+  bucket = 0;
+  if (grow >= M) return false;
+  id = g.ids[grow];
+  if (g.dt) {
+    const int32_t dt = g.dt[grow];
+    if (dt < 0) set_error(err, STCA_ERR_INVALID_ARG);
+    bucket = dt_bucket(dt < 0 ? 0 : dt);
+  }
+  if (id < 0 || id >= g.n_items) {
+    set_error(err, STCA_ERR_ID_OUT_OF_RANGE);
+    id = 0;
+    return false;
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------------------------
-// Kernel R: A resident in shared memory (K <= 512), N walked in 256-column tiles with a
-// double-buffered TMEM accumulator so the epilogue of tile n overlaps the MMAs of n+1.
+// Kernel R (persistent): each CTA pair walks 256-row tiles; each CTA keeps its 128 rows
+// of A resident in shared memory (K <= 512) and streams its half of every 256-column
+// weight tile.  N is walked in 256-column tiles with a double-buffered TMEM accumulator
+// (the epilogue of one tile overlaps the MMAs of the next, across row tiles too), and
+// chunk kc of the next row tile's A is loaded as soon as the last N tile has used it.
+//
+// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer (leader CTA), 4..11 epilogue,
+// 12..15 gather producer (gather mode): thread r copies row r of the CTA's A tile with
+// cp.async into the swizzled layout, adds the time-bucket row from shared memory, and
+// asks L2 for its row of the next tile one tile ahead.
 
 template <int AMODE, int EPI, int STAGES>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     tc_gemm_resident_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                            GatherSrc g, int M, int K, int NT, bf16* __restrict__ C, int ldc, int32_t* err) {
+                            const __grid_constant__ CUtensorMap tmC, GatherSrc g, int M, int K, int NT,
+                            int32_t* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const int KC = K / 64;
   uint8_t* sA = smem;
-  uint8_t* sB = smem + KC * A_CHUNK;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE_256);
-  uint64_t* a_full = bars;                 // [8]
-  uint64_t* b_full = bars + 8;             // [STAGES]
-  uint64_t* b_empty = b_full + STAGES;     // [STAGES]
-  uint64_t* t_full = b_empty + STAGES;     // [2]
-  uint64_t* t_empty = t_full + 2;          // [2]
-  uint64_t* mma_done = t_empty + 2;        // [1]
+  uint8_t* sB = sA + KC * A_CHUNK;
+  uint8_t* sOut = sB + STAGES * B_HALF;               // 8 warps x 2 KB
+  uint8_t* sT = sOut + 8 * OUT_STAGE;                 // 16 x K bf16 (gather mode)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sT + (AMODE == A_GATHER ? T_BYTES : 0));
+  uint64_t* a_full = bars;                 // [8]      leader
+  uint64_t* a_empty = bars + 8;            // [8]      both
+  uint64_t* b_full = bars + 16;            // [STAGES] leader
+  uint64_t* b_empty = b_full + STAGES;     // [STAGES] both
+  uint64_t* t_full = b_empty + STAGES;     // [2]      both
+  uint64_t* t_empty = t_full + 2;          // [2]      leader
+  uint64_t* mma_done = t_empty + 2;        // [1]      leader
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * BM;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int num_tiles = (M + 2 * BM - 1) / (2 * BM);
+  const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < KC; ++i) mbar_init(&a_full[i], AMODE == A_GATHER ? 256 : 1);
+    for (int i = 0; i < KC; ++i) {
+      mbar_init(&a_full[i], AMODE == A_GATHER ? 256 : 1);
+      mbar_init(&a_empty[i], 1);
+    }
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&t_full[i], 1);
-      mbar_init(&t_empty[i], 256);
+      mbar_init(&t_empty[i], 512);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // the peer's barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -198,142 +201,251 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       if (AMODE == A_TMA) prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
-      if (AMODE == A_TMA) {
-        for (int kc = 0; kc < KC; ++kc) {
-          mbar_arrive_expect_tx(&a_full[kc], A_CHUNK);
-          tma_load_2d(sA + kc * A_CHUNK, &tmA, kc * 64, m0, &a_full[kc]);
+      prefetch_tmap(&tmC);
+      const uint32_t a_full0 = cluster_addr(&a_full[0], 0), b_full0 = cluster_addr(&b_full[0], 0);
+      int it = 0, li = 0;
+      bool ok = true;
+      for (int tile = cl; tile < num_tiles && ok; tile += ncl, ++li) {
+        const int m0 = tile * 2 * BM + int(rank) * BM;
+        for (int nt = 0; nt < NT && ok; ++nt) {
+          for (int kc = 0; kc < KC; ++kc, ++it) {
+            if (AMODE == A_TMA && nt == 0) {
+              if (li > 0 && !mbar_wait(&a_empty[kc], (li - 1) & 1)) {
+                fail(abort_flag, err);
+                ok = false;
+                break;
+              }
+              if (leader) mbar_arrive_expect_tx(&a_full[kc], 2 * A_CHUNK);
+              tma_load_2d_pair(sA + kc * A_CHUNK, &tmA, kc * 64, m0, a_full0 + kc * 8);
+            }
+            const int s = it % STAGES, round = it / STAGES;
+            if ((round > 0 && !mbar_wait(&b_empty[s], (round - 1) & 1)) || abort_set(abort_flag)) {
+              fail(abort_flag, err);
+              ok = false;
+              break;
+            }
+            if (leader) mbar_arrive_expect_tx(&b_full[s], 2 * B_HALF);
+            tma_load_2d_pair(sB + s * B_HALF, &tmB, kc * 64, nt * 256 + int(rank) * BM, b_full0 + s * 8);
+          }
         }
       }
-      int it = 0;
-      const int total = NT * KC;
-      for (; it < total; ++it) {
-        const int s = it % STAGES;
-        const int round = it / STAGES;
-        if (round > 0 && !mbar_wait(&b_empty[s], (round - 1) & 1)) {
-          fail(abort_flag, err);
-          break;
-        }
-        if (abort_set(abort_flag)) break;
-        const int nt = it / KC, kc = it % KC;
-        mbar_arrive_expect_tx(&b_full[s], B_STAGE_256);
-        tma_load_2d(sB + s * B_STAGE_256, &tmB, kc * 64, nt * 256, &b_full[s]);
+      if (leader) {
+        // the leader's full barriers count both CTAs' bytes
+        drain_ring(b_full, STAGES, it);
+        if (AMODE == A_TMA && li > 0)
+          for (int kc = 0; kc < KC; ++kc) mbar_wait(&a_full[kc], (li - 1) & 1);
       }
-      drain_ring(b_full, STAGES, it);
-      if (AMODE == A_TMA)
-        for (int kc = 0; kc < KC; ++kc) mbar_wait(&a_full[kc], 0);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16(128, 256);
-      int it = 0;
+    if (leader && lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(256, 256);
+      const uint32_t own_b_empty0 = cluster_addr(&b_empty[0], 0), peer_b_empty0 = cluster_addr(&b_empty[0], 1);
+      const uint32_t own_a_empty0 = cluster_addr(&a_empty[0], 0), peer_a_empty0 = cluster_addr(&a_empty[0], 1);
+      const uint32_t own_t_full0 = cluster_addr(&t_full[0], 0), peer_t_full0 = cluster_addr(&t_full[0], 1);
+      int it = 0, gnt = 0, li = 0;
       bool ok = true;
-      for (int nt = 0; nt < NT && ok; ++nt) {
-        const int buf = nt & 1, use = nt >> 1;
-        if (use > 0 && !mbar_wait(&t_empty[buf], (use - 1) & 1)) {
-          fail(abort_flag, err);
-          break;
-        }
-        tc_fence_after();
-        const uint32_t dcol = tmem + buf * 256;
-        for (int kc = 0; kc < KC; ++kc, ++it) {
-          const int s = it % STAGES;
-          if ((nt == 0 && !mbar_wait(&a_full[kc], 0)) || !mbar_wait(&b_full[s], (it / STAGES) & 1) ||
-              abort_set(abort_flag)) {
+      for (int tile = cl; tile < num_tiles && ok; tile += ncl, ++li) {
+        for (int nt = 0; nt < NT && ok; ++nt, ++gnt) {
+          const int buf = gnt & 1, use = gnt >> 1;
+          if (use > 0 && !mbar_wait_cluster(&t_empty[buf], (use - 1) & 1)) {
             fail(abort_flag, err);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(sA + kc * A_CHUNK);
-          const uint32_t b_addr = smem_u32(sB + s * B_STAGE_256);
+          const uint32_t dcol = tmem + buf * 256;
+          for (int kc = 0; kc < KC; ++kc, ++it) {
+            const int s = it % STAGES;
+            if ((nt == 0 && !mbar_wait_cluster(&a_full[kc], li & 1)) || !mbar_wait(&b_full[s], (it / STAGES) & 1) ||
+                abort_set(abort_flag)) {
+              fail(abort_flag, err);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(sA + kc * A_CHUNK);
+            const uint32_t b_addr = smem_u32(sB + s * B_HALF);
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(dcol, umma_sdesc_sw128(a_addr + k * 32), umma_sdesc_sw128(b_addr + k * 32), idesc,
-                      (kc | k) != 0);
-          umma_commit(&b_empty[s]);
+            for (int k = 0; k < 4; ++k)
+              umma_bf16_pair(dcol, umma_sdesc_sw128(a_addr + k * 32), umma_sdesc_sw128(b_addr + k * 32), idesc,
+                             (kc | k) != 0);
+            umma_commit_pair(own_b_empty0 + s * 8);
+            umma_commit_pair(peer_b_empty0 + s * 8);
+            if (nt == NT - 1) {
+              umma_commit_pair(own_a_empty0 + kc * 8);
+              umma_commit_pair(peer_a_empty0 + kc * 8);
+            }
+          }
+          if (ok) {
+            umma_commit_pair(own_t_full0 + buf * 8);
+            umma_commit_pair(peer_t_full0 + buf * 8);
+          }
         }
-        if (ok) umma_commit(&t_full[buf]);
       }
-      umma_commit(mma_done);
+      umma_commit_pair(cluster_addr(mma_done, 0));
       mbar_wait(mma_done, 0);
+    }
+  } else if (warp >= 12) {
+    if (AMODE == A_GATHER) {
+      const int r = (warp - 12) * 32 + lane;
+      const bool with_dt = g.dt != nullptr && g.dt_table != nullptr;
+      if (with_dt) {
+        const uint4* src = reinterpret_cast<const uint4*>(g.dt_table);
+        for (int i = r; i < 16 * K / 8; i += 128) reinterpret_cast<uint4*>(sT)[i] = __ldg(src + i);
+      }
+      gather_sync();
+      const bf16* table = reinterpret_cast<const bf16*>(g.table);
+      const uint32_t a_full0 = cluster_addr(&a_full[0], 0);
+      int64_t id;
+      int bucket;
+      bool valid = cl < num_tiles && gather_row(g, cl * 2 * BM + int(rank) * BM + r, M, id, bucket, err);
+      if (valid) prefetch_l2_bulk(table + id * K, uint32_t(K) * 2);
+      int li = 0;
+      bool ok = true;
+      for (int tile = cl; tile < num_tiles && ok; tile += ncl, ++li) {
+        // ask L2 for this thread's row of the next tile while this one is in flight
+        int64_t nid = 0;
+        int nbucket = 0;
+        const int next = tile + ncl;
+        const bool nvalid = next < num_tiles && gather_row(g, next * 2 * BM + int(rank) * BM + r, M, nid, nbucket, err);
+        if (nvalid) prefetch_l2_bulk(table + nid * K, uint32_t(K) * 2);
+        const bf16* src = table + id * int64_t(K);
+        const uint32_t nbytes = valid ? 16u : 0u;
+        for (int kc = 0; kc < KC; ++kc) {
+          if (li > 0 && !mbar_wait(&a_empty[kc], (li - 1) & 1)) {
+            fail(abort_flag, err);
+            ok = false;
+            break;
+          }
+          uint8_t* rowp = sA + kc * A_CHUNK + r * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) cp_async_16(rowp + ((c ^ (r & 7)) << 4), src + kc * 64 + c * 8, nbytes);
+          cp_async_commit();
+        }
+        if (!ok) break;
+        const uint8_t* trow = sT + bucket * K * 2;
+        for (int kc = 0; kc < KC; ++kc) {
+          cp_async_wait_dyn(KC - 1 - kc);
+          if (with_dt && valid) {
+            uint8_t* rowp = sA + kc * A_CHUNK + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              uint4* p = reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4));
+              const uint4 x = *p;
+              const uint4 t = *reinterpret_cast<const uint4*>(trow + kc * 128 + c * 16);
+              const __nv_bfloat162* xa = reinterpret_cast<const __nv_bfloat162*>(&x);
+              const __nv_bfloat162* ta = reinterpret_cast<const __nv_bfloat162*>(&t);
+              uint32_t o[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float2 xf = __bfloat1622float2(xa[e]);
+                const float2 tf = __bfloat1622float2(ta[e]);
+                o[e] = pack_bf16x2(xf.x + tf.x, xf.y + tf.y);
+              }
+              *p = make_uint4(o[0], o[1], o[2], o[3]);
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive_remote(a_full0 + kc * 8);  // the leader counts both CTAs' rows
+        }
+        id = nid;
+        bucket = nbucket;
+        valid = nvalid;
+      }
+      cp_async_wait_all();
     }
   } else if (warp >= 4) {
     // two epilogue warps per TMEM lane quarter, each taking half of the columns
     const int quarter = warp & 3;
     const int half = (warp - 4) >> 2;
-    const int r = quarter * 32 + lane;  // tile row == TMEM lane
-    if (AMODE == A_GATHER) gather_a_tile(g, sA, a_full, m0, M, K, r, half, err);
-    const int grow = m0 + r;
+    uint8_t* stage = sOut + (warp - 4) * OUT_STAGE;
     const uint32_t lane_base = tmem + (uint32_t(quarter * 32) << 16);
-    for (int nt = 0; nt < NT; ++nt) {
-      const int buf = nt & 1, use = nt >> 1;
-      if (!mbar_wait(&t_full[buf], use & 1) || abort_set(abort_flag)) {
-        fail(abort_flag, err);
-        break;
-      }
-      tc_fence_after();
-      const uint32_t tb = lane_base + buf * 256;
-      if (EPI == EPI_SWIGLU) {
+    const uint32_t t_empty0 = cluster_addr(&t_empty[0], 0);
+    int gnt = 0;
+    bool ok = true;
+    for (int tile = cl; tile < num_tiles && ok; tile += ncl) {
+      const int y = tile * 2 * BM + int(rank) * BM + quarter * 32;
+      for (int nt = 0; nt < NT; ++nt, ++gnt) {
+        const int buf = gnt & 1, use = gnt >> 1;
+        if (!mbar_wait(&t_full[buf], use & 1) || abort_set(abort_flag)) {
+          fail(abort_flag, err);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tb = lane_base + buf * 256;
+        if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
-        for (int j = 0; j < 2; ++j) {
-          const int col = half * 64 + j * 32;
-          float gv[32], uv[32];
-          tmem_ld_32x32b_x32(tb + col, gv);
-          tmem_ld_32x32b_x32(tb + 128 + col, uv);
-          tmem_ld_wait();
+          for (int j = 0; j < 2; ++j) {
+            const int col = half * 64 + j * 32;
+            float gv[32], uv[32];
+            tmem_ld_32x32b_x32(tb + col, gv);
+            tmem_ld_32x32b_x32(tb + 128 + col, uv);
+            tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) gv[e] = silu_tanh(gv[e]) * uv[e];
-          if (grow < M) store_bf16x32(C + int64_t(grow) * ldc + nt * 128 + col, gv);
-        }
-      } else {
+            for (int e = 0; e < 32; ++e) gv[e] = silu_tanh(gv[e]) * uv[e];
+            epi_store(stage, gv, lane, &tmC, nt * 128 + col, y);
+          }
+        } else {
 #pragma unroll 1
-        for (int j = 0; j < 4; ++j) {
-          const int col = half * 128 + j * 32;
-          float v[32];
-          tmem_ld_32x32b_x32(tb + col, v);
-          tmem_ld_wait();
-          if (grow < M) store_bf16x32(C + int64_t(grow) * ldc + nt * 256 + col, v);
+          for (int j = 0; j < 4; ++j) {
+            const int col = half * 128 + j * 32;
+            float v[32];
+            tmem_ld_32x32b_x32(tb + col, v);
+            tmem_ld_wait();
+            epi_store(stage, v, lane, &tmC, nt * 256 + col, y);
+          }
         }
+        tc_fence_before();
+        mbar_arrive_remote_relaxed(t_empty0 + buf * 8);
       }
-      tc_fence_before();
-      mbar_arrive(&t_empty[buf]);
     }
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();  // neither CTA frees its memory while the pair still uses it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
 // ------------------------------------------------------------------------------------
-// Kernel S: A and B streamed through a STAGES-deep ring, the full output row (NB x 256
-// columns) accumulated in TMEM, then LayerNorm (or a plain store) per row.
+// Kernel S (persistent): each CTA pair walks 256-row tiles, streaming A (its own 128
+// rows each) and its half of every 256-row weight group through a STAGES-deep ring,
+// accumulates the full output row (NB x 256 columns) in TMEM, then applies LayerNorm
+// (or a plain store) per row.  The ring keeps loading the next tile during the epilogue.
 
 template <int EPI, int NB, int STAGES>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     tc_gemm_rowwise_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                           int M, int K, bf16* __restrict__ C, int ldc, const float* __restrict__ gamma,
+                           const __grid_constant__ CUtensorMap tmC, int M, int K, const float* __restrict__ gamma,
                            const float* __restrict__ beta, float eps, int32_t* err) {
   constexpr int N = NB * 256;
-  constexpr int STAGE_BYTES = A_CHUNK + NB * B_STAGE_256;
+  constexpr int STAGE_BYTES = A_CHUNK + NB * B_HALF;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint64_t* full = bars;                  // [STAGES]
-  uint64_t* empty = bars + STAGES;        // [STAGES]
-  uint64_t* t_full = empty + STAGES;      // [1]
-  uint64_t* mma_done = t_full + 1;        // [1]
+  uint8_t* sOut = smem + STAGES * STAGE_BYTES;            // 8 warps x 2 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + 8 * OUT_STAGE);
+  uint64_t* full = bars;                  // [STAGES] leader
+  uint64_t* empty = bars + STAGES;        // [STAGES] both
+  uint64_t* t_full = empty + STAGES;      // [1]      both
+  uint64_t* t_empty = t_full + 1;         // [1]      leader
+  uint64_t* mma_done = t_empty + 1;       // [1]      leader
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* s_gamma = reinterpret_cast<float*>(bars + 2 * STAGES + 8);  // [N]
   float* s_beta = s_gamma + N;                                       // [N]
-  float* s_red = s_beta + N;                                         // [2][128]
+  float* s_sum = s_beta + N;                                         // [2][128]
+  float* s_sq = s_sum + 256;                                         // [2][128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * BM;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
   const int KC = K / 64;
+  const int num_tiles = (M + 2 * BM - 1) / (2 * BM);
+  const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -341,16 +453,18 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(t_full, 1);
+    mbar_init(t_empty, 512);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, N);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, N);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
@@ -358,58 +472,78 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
+      prefetch_tmap(&tmC);
+      const uint32_t full0 = cluster_addr(&full[0], 0);
       int it = 0;
-      for (; it < KC; ++it) {
-        const int s = it % STAGES, round = it / STAGES;
-        if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1)) {
-          fail(abort_flag, err);
-          break;
-        }
-        if (abort_set(abort_flag)) break;
-        uint8_t* st = smem + s * STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-        tma_load_2d(st, &tmA, it * 64, m0, &full[s]);
+      bool ok = true;
+      for (int tile = cl; tile < num_tiles && ok; tile += ncl) {
+        const int m0 = tile * 2 * BM + int(rank) * BM;
+        for (int kc = 0; kc < KC; ++kc, ++it) {
+          const int s = it % STAGES, round = it / STAGES;
+          if ((round > 0 && !mbar_wait(&empty[s], (round - 1) & 1)) || abort_set(abort_flag)) {
+            fail(abort_flag, err);
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * STAGE_BYTES;
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * STAGE_BYTES);
+          tma_load_2d_pair(st, &tmA, kc * 64, m0, full0 + s * 8);
 #pragma unroll
-        for (int nb = 0; nb < NB; ++nb)
-          tma_load_2d(st + A_CHUNK + nb * B_STAGE_256, &tmB, it * 64, nb * 256, &full[s]);
+          for (int nb = 0; nb < NB; ++nb)
+            tma_load_2d_pair(st + A_CHUNK + nb * B_HALF, &tmB, kc * 64, nb * 256 + int(rank) * BM, full0 + s * 8);
+        }
       }
-      drain_ring(full, STAGES, it);
+      if (leader) drain_ring(full, STAGES, it);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16(128, 256);
+    if (leader && lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(256, 256);
+      const uint32_t own_empty0 = cluster_addr(&empty[0], 0), peer_empty0 = cluster_addr(&empty[0], 1);
+      const uint32_t own_t_full = cluster_addr(t_full, 0), peer_t_full = cluster_addr(t_full, 1);
+      int it = 0, li = 0;
       bool ok = true;
-      for (int it = 0; it < KC; ++it) {
-        const int s = it % STAGES;
-        if (!mbar_wait(&full[s], (it / STAGES) & 1) || abort_set(abort_flag)) {
+      for (int tile = cl; tile < num_tiles && ok; tile += ncl, ++li) {
+        if (li > 0 && !mbar_wait_cluster(t_empty, (li - 1) & 1)) {
           fail(abort_flag, err);
-          ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-#pragma unroll
-          for (int nb = 0; nb < NB; ++nb) {
-            const uint32_t b_addr = a_addr + A_CHUNK + nb * B_STAGE_256;
-            umma_bf16(tmem + nb * 256, umma_sdesc_sw128(a_addr + k * 32), umma_sdesc_sw128(b_addr + k * 32),
-                      idesc, (it | k) != 0);
+        for (int kc = 0; kc < KC; ++kc, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(&full[s], (it / STAGES) & 1) || abort_set(abort_flag)) {
+            fail(abort_flag, err);
+            ok = false;
+            break;
           }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+              const uint32_t b_addr = a_addr + A_CHUNK + nb * B_HALF;
+              umma_bf16_pair(tmem + nb * 256, umma_sdesc_sw128(a_addr + k * 32),
+                             umma_sdesc_sw128(b_addr + k * 32), idesc, (kc | k) != 0);
+            }
+          }
+          umma_commit_pair(own_empty0 + s * 8);
+          umma_commit_pair(peer_empty0 + s * 8);
         }
-        umma_commit(&empty[s]);
+        if (ok) {
+          umma_commit_pair(own_t_full);
+          umma_commit_pair(peer_t_full);
+        }
       }
-      if (ok) umma_commit(t_full);
-      umma_commit(mma_done);
+      umma_commit_pair(cluster_addr(mma_done, 0));
       mbar_wait(mma_done, 0);
     }
   } else if (warp >= 4) {
     const int quarter = warp & 3;
     const int half = (warp - 4) >> 2;
     const int r = quarter * 32 + lane;
-    const int grow = m0 + r;
     const int et = threadIdx.x - 128;
     constexpr int HN = N / 2;  // columns per epilogue warp
+    uint8_t* stage = sOut + (warp - 4) * OUT_STAGE;
     if (EPI == EPI_LN) {
       for (int c = et; c < N; c += 256) {
         s_gamma[c] = gamma[c];
@@ -417,71 +551,79 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     const uint32_t tb = tmem + (uint32_t(quarter * 32) << 16) + half * HN;
-    const bool ok = mbar_wait(t_full, 0) && !abort_set(abort_flag);
-    if (!ok) fail(abort_flag, err);
-    tc_fence_after();
-    bf16* crow = C + int64_t(grow) * ldc + half * HN;
-    if (EPI == EPI_LN) {
-      float sum = 0.f;
-      if (ok) {
+    const uint32_t t_empty_addr = cluster_addr(t_empty, 0);
+    const float* gm = s_gamma + half * HN;
+    const float* bt = s_beta + half * HN;
+    int li = 0;
+    for (int tile = cl; tile < num_tiles; tile += ncl, ++li) {
+      const int y = tile * 2 * BM + int(rank) * BM + quarter * 32;
+      const bool ok = !epilogue_any(!mbar_wait(t_full, li & 1) || abort_set(abort_flag));
+      if (!ok) fail(abort_flag, err);
+      tc_fence_after();
+      if (EPI == EPI_LN) {
+        float sum = 0.f;
+        if (ok) {
 #pragma unroll 1
-        for (int j = 0; j < HN / 32; ++j) {
-          float v[32];
-          tmem_ld_32x32b_x32(tb + j * 32, v);
-          tmem_ld_wait();
+          for (int j = 0; j < HN / 32; ++j) {
+            float v[32];
+            tmem_ld_32x32b_x32(tb + j * 32, v);
+            tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) sum += v[e];
-        }
-      }
-      s_red[half * 128 + r] = sum;
-      epilogue_sync();
-      const float mean = (s_red[r] + s_red[128 + r]) * (1.0f / N);
-      float sq = 0.f;
-      if (ok) {
-#pragma unroll 1
-        for (int j = 0; j < HN / 32; ++j) {
-          float v[32];
-          tmem_ld_32x32b_x32(tb + j * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float t = v[e] - mean;
-            sq = fmaf(t, t, sq);
+            for (int e = 0; e < 32; ++e) sum += v[e];
           }
         }
-      }
-      epilogue_sync();  // everyone has read the sums before they are overwritten
-      s_red[half * 128 + r] = sq;
-      epilogue_sync();
-      const float rstd = rsqrtf((s_red[r] + s_red[128 + r]) * (1.0f / N) + eps);
-      if (ok) {
-        const float* gm = s_gamma + half * HN;
-        const float* bt = s_beta + half * HN;
+        s_sum[half * 128 + r] = sum;
+        epilogue_sync();
+        const float mean = (s_sum[r] + s_sum[128 + r]) * (1.0f / N);
+        float sq = 0.f;
+        if (ok) {
+#pragma unroll 1
+          for (int j = 0; j < HN / 32; ++j) {
+            float v[32];
+            tmem_ld_32x32b_x32(tb + j * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float t = v[e] - mean;
+              sq = fmaf(t, t, sq);
+            }
+          }
+        }
+        s_sq[half * 128 + r] = sq;
+        epilogue_sync();
+        const float rstd = rsqrtf((s_sq[r] + s_sq[128 + r]) * (1.0f / N) + eps);
+        if (ok) {
+#pragma unroll 1
+          for (int j = 0; j < HN / 32; ++j) {
+            float v[32];
+            tmem_ld_32x32b_x32(tb + j * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = fmaf((v[e] - mean) * rstd, gm[j * 32 + e], bt[j * 32 + e]);
+            epi_store(stage, v, lane, &tmC, half * HN + j * 32, y);
+          }
+        }
+      } else if (ok) {
 #pragma unroll 1
         for (int j = 0; j < HN / 32; ++j) {
           float v[32];
           tmem_ld_32x32b_x32(tb + j * 32, v);
           tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = fmaf((v[e] - mean) * rstd, gm[j * 32 + e], bt[j * 32 + e]);
-          if (grow < M) store_bf16x32(crow + j * 32, v);
+          epi_store(stage, v, lane, &tmC, half * HN + j * 32, y);
         }
       }
-    } else if (ok) {
-#pragma unroll 1
-      for (int j = 0; j < HN / 32; ++j) {
-        float v[32];
-        tmem_ld_32x32b_x32(tb + j * 32, v);
-        tmem_ld_wait();
-        if (grow < M) store_bf16x32(crow + j * 32, v);
-      }
+      tc_fence_before();
+      mbar_arrive_remote_relaxed(t_empty_addr);
+      if (!ok) break;
     }
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, N);
+    tmem_dealloc_pair(tmem, N);
   }
 }
 
@@ -542,37 +684,58 @@ bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t resident_smem(int K, int stages) {
-  size_t bytes = 1024 + size_t(K / 64) * A_CHUNK + size_t(stages) * B_STAGE_256 + 256;
+// Output map for the epilogue's TMA stores: 32 x 32 boxes, 64-byte swizzle.
+bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Streaming multiprocessors of the current device (persistent grids cover each SM once).
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n >= 2 ? n : 2;
+}
+
+size_t resident_smem(int K, int stages, bool gather) {
+  size_t bytes = 1024 + size_t(K / 64) * A_CHUNK + size_t(stages) * B_HALF + 8 * OUT_STAGE + (gather ? T_BYTES : 0) + 512;
   return bytes < MIN_SMEM ? MIN_SMEM : bytes;
 }
 
 size_t rowwise_smem(int nb, int stages) {
-  size_t bytes = 1024 + size_t(stages) * (A_CHUNK + nb * B_STAGE_256) + 256 + 2 * nb * 256 * 4 + 2 * 128 * 4;
+  size_t bytes = 1024 + size_t(stages) * (A_CHUNK + nb * B_HALF) + 8 * OUT_STAGE + 256 + 2 * nb * 256 * 4 + 4 * 128 * 4;
   return bytes < MIN_SMEM ? MIN_SMEM : bytes;
 }
 
 template <int AMODE, int EPI, int STAGES>
-int run_resident(const CUtensorMap& ta, const CUtensorMap& tb, const GatherSrc& g, int M, int K, int NT, void* C,
-                 int ldc, int32_t* err, cudaStream_t s) {
+int run_resident(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GatherSrc& g, int M,
+                 int K, int NT, int32_t* err, cudaStream_t s) {
   auto kern = tc_gemm_resident_kernel<AMODE, EPI, STAGES>;
-  const size_t smem = resident_smem(K, STAGES);
+  const size_t smem = resident_smem(K, STAGES, AMODE == A_GATHER);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
-  const int grid = (M + BM - 1) / BM;
-  kern<<<grid, 384, smem, s>>>(ta, tb, g, M, K, NT, reinterpret_cast<bf16*>(C), ldc, err); note_launch();
+  const int grid = 2 * std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
+  kern<<<grid, 512, smem, s>>>(ta, tb, tc, g, M, K, NT, err); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
 template <int EPI, int NB, int STAGES>
-int run_rowwise(const CUtensorMap& ta, const CUtensorMap& tb, int M, int K, void* C, int ldc, const float* gamma,
-                const float* beta, float eps, int32_t* err, cudaStream_t s) {
+int run_rowwise(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, int M, int K,
+                const float* gamma, const float* beta, float eps, int32_t* err, cudaStream_t s) {
   auto kern = tc_gemm_rowwise_kernel<EPI, NB, STAGES>;
   const size_t smem = rowwise_smem(NB, STAGES);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
-  const int grid = (M + BM - 1) / BM;
-  kern<<<grid, 384, smem, s>>>(ta, tb, M, K, reinterpret_cast<bf16*>(C), ldc, gamma, beta, eps, err); note_launch();
+  const int grid = 2 * std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
+  kern<<<grid, 384, smem, s>>>(ta, tb, tc, M, K, gamma, beta, eps, err); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -593,17 +756,20 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
   const int N = epi == EPI_SWIGLU ? 2 * Nout : Nout;
   if (N % 256 != 0) return STCA_ERR_UNSUPPORTED;
   const int NT = N / 256;
-  CUtensorMap ta, tb;
+  if (reinterpret_cast<uintptr_t>(C) % 16 != 0) return STCA_ERR_INVALID_ARG;
+  CUtensorMap ta, tb, tc;
   memset(&ta, 0, sizeof(ta));
-  if (!make_tmap(&tb, Wp, N, K, K, B_BOX_ROWS)) return STCA_ERR_CUDA;
+  if (!make_tmap(&tb, Wp, N, K, K, BM)) return STCA_ERR_CUDA;
+  if (!make_tmap_out(&tc, C, M, Nout, ldc)) return STCA_ERR_CUDA;
   if (amode == A_TMA) {
     if (!make_tmap(&ta, A, M, K, K, BM)) return STCA_ERR_CUDA;
   } else {
     ta = tb;  // unused by the gather producer
   }
-#define STCA_RES(AM, EP)                                                                  \
-  (K == 512 ? run_resident<AM, EP, 3>(ta, tb, g, M, K, NT, C, ldc, err, s)               \
-            : run_resident<AM, EP, 5>(ta, tb, g, M, K, NT, C, ldc, err, s))
+  // stage counts fill the 227 KB of shared memory (see resident_smem)
+#define STCA_RES(AM, EP)                                                                                   \
+  (K == 512 ? run_resident<AM, EP, (AM == A_GATHER ? 4 : 5)>(ta, tb, tc, g, M, K, NT, err, s)               \
+            : run_resident<AM, EP, (AM == A_GATHER ? 8 : 9)>(ta, tb, tc, g, M, K, NT, err, s))
   if (amode == A_TMA && epi == EPI_PLAIN) return STCA_RES(A_TMA, EPI_PLAIN);
   if (amode == A_TMA && epi == EPI_SWIGLU) return STCA_RES(A_TMA, EPI_SWIGLU);
   if (amode == A_GATHER && epi == EPI_PLAIN) return STCA_RES(A_GATHER, EPI_PLAIN);
@@ -617,15 +783,17 @@ int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N,
   if (M == 0) return 0;
   if (M < 0 || K <= 0 || K % 64 != 0 || (N != 256 && N != 512) || ldc % 8 != 0) return STCA_ERR_UNSUPPORTED;
   if (epi == EPI_LN && (!gamma || !beta)) return STCA_ERR_INVALID_ARG;
-  CUtensorMap ta, tb;
+  if (reinterpret_cast<uintptr_t>(C) % 16 != 0) return STCA_ERR_INVALID_ARG;
+  CUtensorMap ta, tb, tc;
   if (!make_tmap(&ta, A, M, K, K, BM)) return STCA_ERR_CUDA;
-  if (!make_tmap(&tb, Wp, N, K, K, B_BOX_ROWS)) return STCA_ERR_CUDA;
+  if (!make_tmap(&tb, Wp, N, K, K, BM)) return STCA_ERR_CUDA;
+  if (!make_tmap_out(&tc, C, M, N, ldc)) return STCA_ERR_CUDA;
   if (N == 512) {
-    return epi == EPI_LN ? run_rowwise<EPI_LN, 2, 2>(ta, tb, M, K, C, ldc, gamma, beta, eps, err, s)
-                         : run_rowwise<EPI_PLAIN, 2, 2>(ta, tb, M, K, C, ldc, gamma, beta, eps, err, s);
+    return epi == EPI_LN ? run_rowwise<EPI_LN, 2, 4>(ta, tb, tc, M, K, gamma, beta, eps, err, s)
+                         : run_rowwise<EPI_PLAIN, 2, 4>(ta, tb, tc, M, K, gamma, beta, eps, err, s);
   }
-  return epi == EPI_LN ? run_rowwise<EPI_LN, 1, 4>(ta, tb, M, K, C, ldc, gamma, beta, eps, err, s)
-                       : run_rowwise<EPI_PLAIN, 1, 4>(ta, tb, M, K, C, ldc, gamma, beta, eps, err, s);
+  return epi == EPI_LN ? run_rowwise<EPI_LN, 1, 6>(ta, tb, tc, M, K, gamma, beta, eps, err, s)
+                       : run_rowwise<EPI_PLAIN, 1, 6>(ta, tb, tc, M, K, gamma, beta, eps, err, s);
 }
 
 }  // namespace stca

@@ -242,3 +242,72 @@ def test_attention_f32(score):
     err = R.row_rel_err(got.reshape(-1, 32), ref.reshape(-1, 32))
     assert err <= 1e-5, err
     assert (got[:1] == 0).all()
+
+
+# ---------------------------------------------------------------- persistent tile walks
+
+
+def _rows_sample(M):
+    return np.unique(np.concatenate([np.arange(0, M, 97), np.arange(max(0, M - 300), M)]))
+
+
+@pytest.mark.parametrize("with_dt", [False, True])
+def test_gather_swiglu_many_tiles_per_pair(with_dt):
+    """M spans several 256-row tiles per CTA pair, so every barrier phase wraps."""
+    g = _rng(11)
+    K, hidden, n_items, M = 512, 1024, 200_000, 41_000
+    E = _bf16(g.standard_normal((n_items, K)) * 0.5)
+    T = _bf16(g.standard_normal((16, K)) * 0.5) if with_dt else None
+    ids = g.integers(0, n_items, size=M).astype(np.int32)
+    dt = (np.floor(np.exp2(g.uniform(0, 16, size=M))) - 1).astype(np.int32) if with_dt else None
+    W1 = _bf16(g.standard_normal((K, hidden)) / math.sqrt(K))
+    W3 = _bf16(g.standard_normal((K, hidden)) / math.sqrt(K))
+    Wp = _pack(W1, 1, 2 * hidden)
+    _pack(W3, 2, 2 * hidden, dst=Wp)
+    C = torch.empty((M, hidden), dtype=torch.bfloat16, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_gemm_resident(1, 1, None, torch.from_numpy(ids).to(dev),
+                                   torch.from_numpy(dt).to(dev) if with_dt else None, E, T, n_items, M, K, Wp,
+                                   hidden, C, hidden, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    rows = _rows_sample(M)
+    X = bf16_to_f64(E)[ids[rows]]
+    if with_dt:
+        X = X + bf16_to_f64(T)[R.dt_bucket(dt[rows])]
+    ref = R.silu(X @ bf16_to_f64(W1)) * (X @ bf16_to_f64(W3))
+    _close_bf16(bf16_to_f64(C)[rows], ref)
+
+
+def test_resident_plain_many_tiles_per_pair():
+    g = _rng(12)
+    K, N, M = 512, 1024, 45_123
+    A = _bf16(g.standard_normal((M, K)))
+    W = _bf16(g.standard_normal((K, N)) / math.sqrt(K))
+    Wp = _pack(W, 0, N)
+    C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_gemm_resident(0, 0, A, None, None, None, None, 0, M, K, Wp, N, C, N, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    rows = _rows_sample(M)
+    _close_bf16(bf16_to_f64(C)[rows], bf16_to_f64(A)[rows] @ bf16_to_f64(W))
+
+
+@pytest.mark.parametrize("N", [256, 512])
+def test_rowwise_ln_many_tiles_per_pair(N):
+    g = _rng(13)
+    K, M = 1024, 40_007
+    A = _bf16(g.standard_normal((M, K)))
+    W = _bf16(g.standard_normal((K, N)) / math.sqrt(K))
+    Wp = _pack(W, 0, N)
+    gamma = torch.from_numpy((1 + 0.1 * g.standard_normal(N)).astype(np.float32)).to(dev)
+    beta = torch.from_numpy((0.1 * g.standard_normal(N)).astype(np.float32)).to(dev)
+    C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_gemm_rowwise(2, A, M, K, Wp, N, gamma, beta, 1e-5, C, N, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    rows = _rows_sample(M)
+    Y = R.layer_norm(bf16_to_f64(A)[rows] @ bf16_to_f64(W), gamma.cpu().numpy(), beta.cpu().numpy(), 1e-5)
+    _close_bf16(bf16_to_f64(C)[rows], Y)

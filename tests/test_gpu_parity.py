@@ -38,8 +38,10 @@ def _check_stca(wl, tol, users=None):
         z, o = z[rows], o[:, rows]
     for i in range(wl["cfg"]["M"]):
         e = R.row_rel_err(o[i], orr[i])
+        print(f"parity o^({i + 1}) row-relative error {e:.3e}")
         assert e <= tol, f"o^({i + 1}) err {e}"
     e = R.row_rel_err(z, zr)
+    print(f"parity z row-relative error {e:.3e}")
     assert e <= tol, f"z err {e}"
     return z
 
@@ -151,6 +153,7 @@ def test_pointwise_small():
     wl["lengths"] = wl["lengths"].copy()
     got = _run_pointwise(wl)
     ref = R.pointwise_relu_ta(wl)
+    print(f"parity pointwise row-relative error {R.row_rel_err(got, ref):.3e}")
     assert R.row_rel_err(got, ref) <= 1e-4
 
 
@@ -174,4 +177,5 @@ def test_hyformer_small():
     m.close()
     ref = R.hyformer_forward(wl)
     e = R.row_rel_err(out.cpu().numpy(), ref)
+    print(f"parity hyformer row-relative error {e:.3e}")
     assert e <= TOL_BF16, e
