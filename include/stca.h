@@ -160,6 +160,26 @@ int stca_pointwise_forward(stca_handle* h, const int32_t* ids, const int32_t* le
                            const void* table, int64_t n_items, int B, int n_tok, float* out,
                            void* stream);
 
+/* Largest batch the allocation-free variant below accepts. */
+#define STCA_NOALLOC_MAX_USERS 2048
+
+/* stca_pointwise_forward without a handle and without any device allocation.  The pages
+ * have no counterpart to this entry point; it exists for callers that cannot call
+ * cudaMalloc (a plugin inside a host runtime that owns all device memory, or a request
+ * path where an allocation, which may synchronise the device, is not allowed).
+ * Same arguments and result as stca_pointwise_forward (D = 128, bf16 q and table,
+ * float32 out), plus err_out: a caller-owned device int32 that receives the first error
+ * the GPU detects (an id out of range, lengths not adding up to n_tok) if it was 0, or
+ * NULL.  Scratch lives in a fixed array of about 4.2 MB in the library's device image,
+ * which every GPU that loads the library holds until the process exits; B above
+ * STCA_NOALLOC_MAX_USERS returns STCA_ERR_CAPACITY.  The first call on a device looks up
+ * that array's device address (make that first call before any stream capture).  All
+ * calls share the array: calls that overlap on the GPU (different streams, or different
+ * host threads on the same device) race and give undefined results; calls serialised
+ * on one stream are safe. */
+int stca_pointwise_forward_noalloc(const int32_t* ids, const int32_t* lengths, const void* q, const void* table,
+                                   int64_t n_items, int B, int n_tok, float* out, int32_t* err_out, void* stream);
+
 /* Multi-query multi-sequence decode ([hyformer] §3.4-3.7).  Two sequences per user
  * (s = 0 "feed", s = 1 "search"), each with n_query query tokens.  Per block l and
  * sequence s: H = SwiGLU_{l,s}(X_s) (eq 7), K,V = H W_K, H W_V (eq 8), decoded queries

@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(PKG, "libstca.so")
 
 MAX_LAYERS = 8
 MAX_QUERY_TOKENS = 64
+NOALLOC_MAX_USERS = 2048
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_ID_OUT_OF_RANGE, ERR_TIMEOUT, \
     ERR_BAD_LENGTHS = range(8)
@@ -74,6 +75,7 @@ _SIGS = [
     ("stca_forward_host", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.POINTER(StcaWeights), _vp,
                                  _vp]),
     ("stca_pointwise_forward", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp]),
+    ("stca_pointwise_forward_noalloc", _i32, [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp]),
     ("hyformer_forward", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, ctypes.POINTER(HyfWeights),
                                 _vp, _vp]),
     ("stca_sync_status", _i32, [_vp]),
@@ -188,6 +190,12 @@ def stca_forward_host(h, ids, lengths, dt, x_t, tpu, B, n_tok, t_tot, weights: S
 def stca_pointwise_forward(h, ids, lengths, q, table, n_items, B, n_tok, out, stream=None) -> int:
     return lib().stca_pointwise_forward(h, ptr(ids), ptr(lengths), ptr(q), ptr(table), n_items, B, n_tok, ptr(out),
                                         stream_ptr(stream))
+
+
+def stca_pointwise_forward_noalloc(ids, lengths, q, table, n_items, B, n_tok, out, err=None, stream=None) -> int:
+    """Pointwise ReLU TA without a handle or any device allocation (scratch in the library)."""
+    return lib().stca_pointwise_forward_noalloc(ptr(ids), ptr(lengths), ptr(q), ptr(table), n_items, B, n_tok,
+                                                ptr(out), ptr(err), stream_ptr(stream))
 
 
 def hyformer_forward(h, ids_feed, len_feed, n_feed, ids_search, len_search, n_search, q0, B, n_query,
