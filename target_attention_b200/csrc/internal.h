@@ -1,6 +1,7 @@
 // Host-side launchers shared between the library's translation units.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -76,6 +77,11 @@ struct SimtGemmArgs {
 
 template <typename TA, typename TB>
 int simt_gemm(const SimtGemmArgs<TA, TB>& a, cudaStream_t s);
+
+// Tensor-core (mma.sync) form of simt_gemm<float, bf16> with fp32-accurate products
+// (activations split into two bf16 terms); used by simt_gemm when the shapes allow.
+bool query_gemm_supported(const SimtGemmArgs<float, __nv_bfloat16>& a);
+int query_gemm(const SimtGemmArgs<float, __nv_bfloat16>& a, cudaStream_t s);
 
 // y = LayerNorm(x) row-wise over d columns, fp32; x and y may alias.
 int layer_norm_f32(const float* x, int64_t ldx, float* y, int64_t ldy, int rows, int d, const float* gamma,

@@ -1,9 +1,11 @@
-// fp32-accumulating SIMT kernels: the target-side (query) path of every configuration,
-// the whole history path of the fp32 configuration, LayerNorm, the ragged-offset scan
-// and the token mix.
+// fp32-accumulating SIMT kernels: the whole path of the fp32 configuration, LayerNorm,
+// the ragged-offset scan and the token mix.  The target-side GEMMs with bf16 weights go
+// to the tensor-core form in query_gemm.cu when their shapes allow.
 //
 // The query path works on T_tot x d matrices (one row per target), which are small next
 // to the history side; it keeps fp32 activations throughout.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -255,6 +257,9 @@ template <typename TA, typename TB>
 int simt_gemm(const SimtGemmArgs<TA, TB>& a, cudaStream_t s) {
   if (a.M == 0 || a.N == 0 || a.batch == 0) return 0;
   if (a.M < 0 || a.N < 0 || a.K <= 0) return STCA_ERR_INVALID_ARG;
+  if constexpr (std::is_same<TA, float>::value && std::is_same<TB, bf16>::value) {
+    if (query_gemm_supported(a)) return query_gemm(a, s);
+  }
   dim3 grid((a.N + SB_N - 1) / SB_N, (a.M + SB_M - 1) / SB_M, a.batch);
   if (a.B2) simt_gemm_kernel<TA, TB, true><<<grid, 256, 0, s>>>(a);
   else simt_gemm_kernel<TA, TB, false><<<grid, 256, 0, s>>>(a);
