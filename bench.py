@@ -50,6 +50,7 @@ def parse():
     ap.add_argument("--n-items", type=int, default=None, help="override the table rows (testing only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dedup", action="store_true", help="run the history GEMMs once per token")
     return ap.parse_args()
 
 
@@ -192,8 +193,44 @@ def clocks_rejected(clk):
 # ------------------------------------------------------------------------------ roofline
 
 
-def stage_work(stage, wl):
-    """Algorithmic work of one step of a stage: (bound, amount, unit)."""
+def distinct_rows(ids, dt):
+    """Distinct (item id, time bucket) keys among a pass's history tokens."""
+    import numpy as np
+    key = ids.astype(np.int64) * 16
+    if dt is not None:
+        v = dt.astype(np.int64) + 1
+        key += np.minimum(15, np.floor(np.log2(v)).astype(np.int64))
+    return int(len(np.unique(key)))
+
+
+_PASSES = {}
+
+
+def gemm_passes(wl, dedup):
+    """(rows computed by the history GEMMs, history tokens, users, targets) per pass."""
+    key = (id(wl), bool(dedup))
+    if key not in _PASSES:
+        _PASSES[key] = _gemm_passes(wl, dedup)
+    return _PASSES[key]
+
+
+def _gemm_passes(wl, dedup):
+    c = wl["cfg"]
+    if c["kind"] == "stca":
+        n = int(wl["lengths"].sum())
+        rows = distinct_rows(wl["ids"], wl["dt"]) if dedup else n
+        return [(rows, n, len(wl["lengths"]), int(wl["targets_per_user"].sum()))] * c["M"]
+    nq, Bu = c["n_query"], len(wl["lengths"][0])
+    out = []
+    for s in (0, 1):
+        n = int(wl["lengths"][s].sum())
+        out.append((distinct_rows(wl["ids"][s], None) if dedup else n, n, Bu, Bu * nq))
+    return out * c["blocks"]
+
+
+def stage_work(stage, wl, dedup=False):
+    """Algorithmic work of one step of a stage: (bound, amount, unit).  The history GEMMs
+    count the rows they compute (distinct keys when dedup is on)."""
     c = wl["cfg"]
     d = c["d"]
     if c["kind"] == "pointwise":
@@ -204,22 +241,18 @@ def stage_work(stage, wl):
             return "hbm", n_tok * (2 * d + 4) + B * d * 2 + B * d * 4, "byte"
         return None, None, None
     h, H = c["hidden"], c["H"]
-    if c["kind"] == "stca":
-        passes = [(int(wl["lengths"].sum()), len(wl["lengths"]), int(wl["targets_per_user"].sum()))] * c["M"]
-    else:
-        nq, Bu = c["n_query"], len(wl["lengths"][0])
-        passes = [(int(wl["lengths"][s].sum()), Bu, Bu * nq) for s in (0, 1)] * c["blocks"]
+    passes = gemm_passes(wl, dedup)
     if stage == "gather_ffn":
-        return "tensor", sum(2.0 * n * d * 2 * h for n, _, _ in passes), "flop"
+        return "tensor", sum(2.0 * r * d * 2 * h for r, _, _, _ in passes), "flop"
     if stage == "ffn_out":
-        return "tensor", sum(2.0 * n * h * d for n, _, _ in passes), "flop"
+        return "tensor", sum(2.0 * r * h * d for r, _, _, _ in passes), "flop"
     if stage == "kv":
-        return "tensor", sum(2.0 * n * d * 2 * d for n, _, _ in passes), "flop"
+        return "tensor", sum(2.0 * r * d * 2 * d for r, _, _, _ in passes), "flop"
     if stage == "attention":
         tot = 0.0
-        for n, Bu, T in passes:
+        for _, n, Bu, T in passes:
             splits = max(1, min(16, -(-(n // max(1, Bu)) // 1024)))
-            # K and V rows read once (bf16), queries read, split partials written
+            # one K and one V row (bf16) read per history token, queries read, split partials written
             tot += n * 2 * d * 2 + T * d * 4 + splits * T * (d + 2 * H) * 4
         return "hbm", tot, "byte"
     return None, None, None
@@ -261,8 +294,9 @@ def run_ours(args):
     kind = wl["cfg"]["kind"]
     n_tok = history_tokens(wl)
     stream = torch.cuda.current_stream()
+    dedup = kind != "pointwise" and wl["cfg"]["dtype"] == "bf16" and not args.no_dedup
     if kind == "stca":
-        model = StcaModel(wl)
+        model = StcaModel(wl, dedup=int(dedup))
         x = model.inputs(wl)
         out = torch.empty((x["t_tot"], wl["cfg"]["d"]), device="cuda")
     elif kind == "pointwise":
@@ -270,12 +304,15 @@ def run_ours(args):
         x = model.inputs(wl)
         out = torch.empty((x["B"], wl["cfg"]["d"]), device="cuda")
     else:
-        model = HyformerModel(wl)
+        model = HyformerModel(wl, dedup=dedup)
         x = model.inputs(wl)
         out = torch.empty((x["B"], 2 * x["n_query"], wl["cfg"]["d"]), device="cuda")
 
-    def step():
-        B.check(model.forward(x, out, stream=stream), "forward")
+    def step(handle=None):
+        if handle is None:
+            B.check(model.forward(x, out, stream=stream), "forward")
+        else:
+            B.check(model.forward(x, out, stream=stream, handle=handle), "forward")
 
     def barrier():
         if world > 1:
@@ -339,7 +376,7 @@ def run_ours(args):
             continue
         entry = {"ms_per_step": round(tot / args.steps, 4), "share": round(tot / ms, 4),
                  "launches_per_step": calls // args.steps, "launch_ms": round(tot / calls, 4)}
-        bound, work, unit = stage_work(name, wl)
+        bound, work, unit = stage_work(name, wl, dedup)
         if bound == "tensor":
             ach = work * args.steps / (tot / 1e3) / 1e12
             entry.update(bound="tensor", achieved_tflops=round(ach, 1),
@@ -348,8 +385,8 @@ def run_ours(args):
             ach = work * args.steps / (tot / 1e3) / 1e9
             entry.update(bound="hbm", achieved_gbs=round(ach, 1), frac=round(ach / peaks["hbm_gbs"], 4))
         stages[name] = entry
-    dom = max((s for s in stages if stage_work(s, wl)[0]), key=lambda s: stages[s]["ms_per_step"])
-    bound, work, unit = stage_work(dom, wl)
+    dom = max((s for s in stages if stage_work(s, wl, dedup)[0]), key=lambda s: stages[s]["ms_per_step"])
+    bound, work, unit = stage_work(dom, wl, dedup)
     tot, calls = prof[dom]
     per_launch = work * args.steps / calls
     if bound == "tensor":
@@ -357,9 +394,34 @@ def run_ours(args):
     else:
         achieved, peak, runit = per_launch / (tot / calls / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s"
     roofline = {"bound": bound, "kernel": dom, "achieved": round(achieved, 2), "peak": peak, "unit": runit,
-                "frac": round(achieved / peak, 4), "traffic": traffic_from_profiles(dom, args.workload),
+                "frac": round(achieved / peak, 4),
+                "traffic": traffic_from_profiles(dom + ("+dedup" if dedup else ""), args.workload),
                 "work_per_launch": per_launch, "work_unit": unit, "launch_ms": round(tot / calls, 4),
                 "peak_source": f"{peaks['source']} ({'sustained bf16' if bound == 'tensor' else 'HBM copy'})"}
+
+    # the same step with the history GEMMs run per token (dedup off), for reference
+    per_token = None
+    if dedup:
+        h0 = model.other_handle(dedup=0)
+        for _ in range(args.warmup):
+            step(h0)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step(h0)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ms0 = max_over_ranks(e0.elapsed_time(e1))
+        B.stca_destroy(h0)
+        passes = gemm_passes(wl, True)
+        per_token = {"value": round(total_tokens * args.steps / (ms0 / 1e3), 1), "unit": UNIT,
+                     "ms_per_step": round(ms0 / args.steps, 3),
+                     "distinct_rows_fraction": round(sum(p[0] for p in passes) / sum(p[1] for p in passes), 4),
+                     "note": "same step with the history GEMMs run once per token instead of once per distinct "
+                             "(id, time bucket) key; identical results"}
 
     # end to end through the host-buffer entry point: pinned inputs in, z out, per step
     e2e = None
@@ -401,6 +463,8 @@ def run_ours(args):
         "data": "synthetic (seeded Zipf ids, random-init weights)", "config": config_block(wl, world),
         "token_layers_per_s": round(value * layers, 1),
         "roofline": roofline, "stages": stages, "e2e": e2e, "cpu_baseline": cpu,
+        "history_gemm_rows": "distinct (id, time bucket) keys per call" if dedup else "every history token",
+        "per_token_path": per_token,
         "gpu_launches": int(launches), "gpu_launches_per_step": round(launches / args.steps, 1), "clocks": clk,
     }
     print(json.dumps(line), flush=True)

@@ -63,7 +63,10 @@ enum stca_score { STCA_SOFTMAX = 0, STCA_RELU = 1 };
  * STCA_BF16 in this build), SwiGLU hidden width `hidden`.
  * time_buckets: 0, or 16 for the time-difference feature of [review] §四.
  * max_users / max_tokens / max_targets bound B, n_tok and t_tot of every later call;
- * stca_create sizes all device workspace from them, and later calls allocate nothing. */
+ * stca_create sizes all device workspace from them, and later calls allocate nothing.
+ * dedup follows the HyFormer page §3.8.1 (GPU pooling: few ids of a long sequence are
+ * distinct): X~, K and V of a history token depend only on its item id and time bucket,
+ * so they are computed once per distinct key and every token reads its key's K/V row. */
 typedef struct {
   int mode;         /* enum stca_mode */
   int M, d, H, hidden;
@@ -71,6 +74,8 @@ typedef struct {
   int score;        /* enum stca_score */
   int time_buckets; /* 0 or 16 */
   int max_users, max_tokens, max_targets;
+  int dedup;        /* 1: run the per-token history GEMMs once per distinct (id, time bucket)
+                       key of the call (STCA_BF16 only); results are unchanged */
   float ln_eps;     /* LayerNorm epsilon (biased variance) */
 } stca_config;
 
@@ -229,7 +234,8 @@ enum stca_stage {
   STCA_STAGE_QUERY = 6,      /* target side: SwiGLU/LN, W_Q, W_O, W_C, W_Z */
   STCA_STAGE_POINTWISE = 7,  /* fused pointwise ReLU target attention */
   STCA_STAGE_BOOST = 8,      /* token mix + per-token SwiGLU + residual */
-  STCA_N_STAGES = 9
+  STCA_STAGE_DEDUP = 9,      /* distinct history keys (when the handle has dedup = 1) */
+  STCA_N_STAGES = 10
 };
 
 /* enable = 1 starts recording (totals reset), 0 stops it. */

@@ -8,6 +8,7 @@
 #ifndef STCA_KERNELS_H
 #define STCA_KERNELS_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -52,6 +53,15 @@ int stca_k_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, in
 int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B,
                      int T, int d, int H, int splits, int score, float* part_acc, float* part_ml, float* out,
                      int32_t* err, void* stream);
+
+/* Distinct history keys (HyFormer page §3.8.1, GPU pooling): key(n) = (ids[n], bucket(dt[n]))
+ * (bucket 0 when dt is NULL).  Writes uniq_idx[n] in [0, *count) with equal keys mapped to
+ * the same index and distinct keys to distinct indices, and uniq_token[u] = a token whose
+ * key is u.  The numbering order is unspecified.  ws: caller scratch of at least
+ * stca_k_dedup_workspace_bytes(n) bytes; count: device int32. */
+size_t stca_k_dedup_workspace_bytes(int n);
+int stca_k_dedup(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws_bytes, int32_t* uniq_idx,
+                 int32_t* uniq_token, int32_t* count, int32_t* err, void* stream);
 
 #ifdef __cplusplus
 }

@@ -31,7 +31,7 @@ _i64 = ctypes.c_int64
 class StcaConfig(ctypes.Structure):
     _fields_ = [("mode", _i32), ("M", _i32), ("d", _i32), ("H", _i32), ("hidden", _i32),
                 ("dtype", _i32), ("score", _i32), ("time_buckets", _i32), ("max_users", _i32),
-                ("max_tokens", _i32), ("max_targets", _i32), ("ln_eps", ctypes.c_float)]
+                ("max_tokens", _i32), ("max_targets", _i32), ("dedup", _i32), ("ln_eps", ctypes.c_float)]
 
 
 class StcaFfn(ctypes.Structure):
@@ -90,6 +90,8 @@ _SIGS = [
     ("stca_k_gemm_rowwise", _i32, [_i32, _vp, _i32, _i32, _vp, _i32, _vp, _vp, ctypes.c_float, _vp, _i32, _vp, _vp]),
     ("stca_k_attention", _i32, [_i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
                                 _vp]),
+    ("stca_k_dedup_workspace_bytes", ctypes.c_size_t, [_i32]),
+    ("stca_k_dedup", _i32, [_vp, _vp, _i32, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]),
 ]
 
 EXPORTED = [s[0] for s in _SIGS]
@@ -152,7 +154,7 @@ def stca_sync_status(h) -> int:
     return lib().stca_sync_status(h)
 
 
-STAGES = ["setup", "gather_ffn", "ffn_out", "kv", "attention", "merge", "query", "pointwise", "boost"]
+STAGES = ["setup", "gather_ffn", "ffn_out", "kv", "attention", "merge", "query", "pointwise", "boost", "dedup"]
 
 
 def stca_profile_enable(h, enable=True) -> int:
@@ -231,3 +233,12 @@ def stca_k_attention(kv_bf16, Q, KV, hoff, toff, B, T, d, H, splits, score, part
                      stream=None) -> int:
     return lib().stca_k_attention(kv_bf16, ptr(Q), ptr(KV), ptr(hoff), ptr(toff), B, T, d, H, splits, score,
                                   ptr(part_acc), ptr(part_ml), ptr(out), ptr(err), stream_ptr(stream))
+
+
+def stca_k_dedup_workspace_bytes(n) -> int:
+    return lib().stca_k_dedup_workspace_bytes(n)
+
+
+def stca_k_dedup(ids, dt, n, ws, uniq_idx, uniq_token, count, err, stream=None) -> int:
+    return lib().stca_k_dedup(ptr(ids), ptr(dt), n, ptr(ws), ws.numel() * ws.element_size(), ptr(uniq_idx),
+                              ptr(uniq_token), ptr(count), ptr(err), stream_ptr(stream))

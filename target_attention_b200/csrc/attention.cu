@@ -61,7 +61,7 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
 
 // Issues the cp.async copies of K and V rows [key0, key0+32) of head h into one stage.
 __device__ __forceinline__ void load_kv_tile(uint8_t* stage, const bf16* KV, int64_t ld, int64_t row0, int valid,
-                                             int hcol, int d, int lane) {
+                                             int hcol, int d, int lane, const int32_t* kv_rows) {
   uint8_t* sK = stage;
   uint8_t* sV = stage + TILE_BYTES;
 #pragma unroll
@@ -69,7 +69,8 @@ __device__ __forceinline__ void load_kv_tile(uint8_t* stage, const bf16* KV, int
     const int idx = i * 32 + lane;
     const int key = idx >> 3, ch = idx & 7;
     const bool ok = key < valid;
-    const bf16* src = KV + (ok ? (row0 + key) * ld : 0) + hcol + ch * 8;
+    const int64_t row = ok ? (kv_rows ? int64_t(kv_rows[row0 + key]) : row0 + key) : 0;
+    const bf16* src = KV + row * ld + hcol + ch * 8;
     const int off = key * 128 + ((ch ^ (key & 7)) << 4);
     cp_async_16(sK + off, src, ok ? 16u : 0u);
     cp_async_16(sV + off, src + d, ok ? 16u : 0u);
@@ -130,13 +131,14 @@ __global__ void __launch_bounds__(128, 2) attn_bf16_kernel(AttnArgs a) {
     // ---- stream this warp's tiles: warp w takes tiles w, w+4, ...
     int stage = 0;
     int tile = warp;
-    if (tile < n_tiles) load_kv_tile(wbuf, KV, ld, k0 + int64_t(tile) * KT, min(KT, nk - tile * KT), hcol, d, lane);
+    if (tile < n_tiles)
+      load_kv_tile(wbuf, KV, ld, k0 + int64_t(tile) * KT, min(KT, nk - tile * KT), hcol, d, lane, a.kv_rows);
     cp_async_commit();
     for (; tile < n_tiles; tile += 4) {
       const int next = tile + 4;
       if (next < n_tiles)
         load_kv_tile(wbuf + (stage ^ 1) * WARP_STAGE, KV, ld, k0 + int64_t(next) * KT, min(KT, nk - next * KT),
-                     hcol, d, lane);
+                     hcol, d, lane, a.kv_rows);
       cp_async_commit();
       cp_async_wait<1>();
       __syncwarp();
@@ -338,7 +340,7 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(AttnArgs a) {
     }
     float mx = -INFINITY, l = 0.f;
     for (int j = warp; j < nk; j += 4) {
-      const float* krow = KV + (k0 + j) * ld + h * dh;
+      const float* krow = KV + (a.kv_rows ? int64_t(a.kv_rows[k0 + j]) : k0 + j) * ld + h * dh;
       float sc = 0.f;
 #pragma unroll
       for (int i = 0; i < DPL; ++i) sc += q[i] * krow[lane + 32 * i];

@@ -15,6 +15,7 @@ void note_launch();
 struct GatherSrc {
   const int32_t* ids;
   const int32_t* dt;      // may be null
+  const int32_t* rows;    // row r reads token rows[r] (distinct-row form), or null: token r
   const void* table;      // [n_items, K] (bf16 or fp32, the kernel's type)
   const void* dt_table;   // [16, K] or null
   int64_t n_items;
@@ -35,13 +36,16 @@ int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_off
 //   amode A_TMA: A is a dense bf16 [M, K] matrix; A_GATHER: rows gathered via `g`.
 //   epi EPI_PLAIN:  C = A Wp^T, Wp packed [N, K], N a multiple of 256, Nout = N
 //   epi EPI_SWIGLU: Wp packed gate/up interleaved [2*Nout, K], C = SiLU(A W1) * (A W3)
+// M_dev, when not null, is a device int holding the number of rows actually present
+// (<= M); M then only sizes the tensor maps and buffers.
 int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int K, const void* Wp,
-                     int Nout, void* C, int ldc, int32_t* err, cudaStream_t s);
+                     int Nout, void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev = nullptr);
 
 // C[M, N] (bf16) = epi(A Wp^T), A dense bf16 [M, K] streamed (K a multiple of 64),
 // N in {256, 512}; epi EPI_LN applies LayerNorm (gamma, beta, eps) over the full row.
 int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
-                    const float* beta, float eps, void* C, int ldc, int32_t* err, cudaStream_t s);
+                    const float* beta, float eps, void* C, int ldc, int32_t* err, cudaStream_t s,
+                    const int32_t* M_dev = nullptr);
 
 // ---------------------------------------------------------------- SIMT fp32 GEMMs
 
@@ -94,6 +98,7 @@ struct AttnArgs {
   const void* KV;       // [N, 2d]: K in columns [0, d), V in [d, 2d); bf16 or fp32
   const int32_t* hoff;  // [B+1] history offsets
   const int32_t* toff;  // [B+1] target offsets
+  const int32_t* kv_rows;  // K/V row of history token n (distinct-row form), or null: row n
   int B, T, d, H, splits;
   int score;            // 0 softmax, 1 relu
   float* part_acc;      // [splits, T, d]
@@ -114,6 +119,16 @@ int exclusive_offsets(const int32_t* lengths, int B, int32_t* offsets, int expec
 // dst[r, col0 + c] = float(src[r, c]) for c < d (src bf16 or fp32 by `src_bf16`).
 int copy_rows_to_f32(const void* src, int src_bf16, int rows, int d, float* dst, int64_t ldd, int col0,
                      cudaStream_t s);
+
+// ---------------------------------------------------------------- distinct history rows
+
+// Table slots and workspace bytes for up to max_tokens rows.
+size_t dedup_table_slots(int max_tokens);
+size_t dedup_workspace_bytes(int max_tokens);
+// Distinct keys (id, time bucket) of n history tokens: uniq_idx[n] in [0, *count),
+// uniq_token[u] = one token with key u.  All on the stream.
+int dedup_rows(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws_bytes, int32_t* uniq_idx,
+               int32_t* uniq_token, int32_t* count, int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- pointwise ReLU TA
 

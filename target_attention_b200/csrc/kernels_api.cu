@@ -57,6 +57,7 @@ int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t*
   a.KV = KV;
   a.hoff = hoff;
   a.toff = toff;
+  a.kv_rows = nullptr;
   a.B = B;
   a.T = T;
   a.d = d;
@@ -71,6 +72,15 @@ int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t*
   const int rc = kv_bf16 ? attention_bf16(a, s) : attention_f32(a, s);
   if (rc != STCA_OK) return rc;
   return attention_merge(a, s);
+}
+
+size_t stca_k_dedup_workspace_bytes(int n) { return n < 0 ? 0 : dedup_workspace_bytes(n); }
+
+int stca_k_dedup(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws_bytes, int32_t* uniq_idx,
+                 int32_t* uniq_token, int32_t* count, int32_t* err, void* stream) {
+  if (n < 0 || !count || (n > 0 && (!ids || !ws || !uniq_idx || !uniq_token))) return STCA_ERR_INVALID_ARG;
+  return dedup_rows(ids, dt, n, ws, ws_bytes, uniq_idx, uniq_token, count, err,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

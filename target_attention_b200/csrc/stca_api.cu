@@ -33,6 +33,10 @@ struct stca_handle {
   float *cat = nullptr, *qbuf = nullptr, *qproj = nullptr, *attn = nullptr, *tmp_h = nullptr, *tmp_d = nullptr;
   float *part_acc = nullptr, *part_ml = nullptr;
   float *hq = nullptr, *hqhat = nullptr, *hmix = nullptr;
+  // distinct history rows
+  void* dedup_ws = nullptr;
+  size_t dedup_ws_bytes = 0;
+  int32_t *uniq_idx = nullptr, *uniq_token = nullptr, *uniq_count = nullptr;
   // staging for the host-buffer entry point
   int32_t *in_ids = nullptr, *in_len = nullptr, *in_dt = nullptr, *in_tpu = nullptr;
   void* in_xt = nullptr;
@@ -142,10 +146,12 @@ int validate_config(const stca_config& c) {
   if (c.dtype != STCA_FP32 && c.dtype != STCA_BF16) return STCA_ERR_INVALID_ARG;
   if (c.score != STCA_SOFTMAX && c.score != STCA_RELU) return STCA_ERR_INVALID_ARG;
   if (c.time_buckets != 0 && c.time_buckets != 16) return STCA_ERR_UNSUPPORTED;
+  if (c.dedup != 0 && c.dedup != 1) return STCA_ERR_INVALID_ARG;
   if (c.mode == STCA_MODE_POINTWISE) {
-    if (c.dtype != STCA_BF16 || c.d != 128) return STCA_ERR_UNSUPPORTED;
+    if (c.dtype != STCA_BF16 || c.d != 128 || c.dedup) return STCA_ERR_UNSUPPORTED;
     return STCA_OK;
   }
+  if (c.dedup && c.dtype != STCA_BF16) return STCA_ERR_UNSUPPORTED;
   if (c.hidden <= 0 || c.d % c.H != 0) return STCA_ERR_INVALID_ARG;
   const int dh = c.d / c.H;
   if (c.mode == STCA_MODE_HYFORMER) {
@@ -183,6 +189,11 @@ int allocate(stca_handle* h) {
        dalloc(h, &h->tmp_d, T * d * 4);
   ok = ok && dalloc(h, &h->part_acc, size_t(MAX_SPLITS) * T * d * 4) &&
        dalloc(h, &h->part_ml, size_t(MAX_SPLITS) * T * c.H * 2 * 4);
+  if (c.dedup) {
+    h->dedup_ws_bytes = dedup_workspace_bytes(c.max_tokens);
+    ok = ok && dalloc(h, &h->dedup_ws, h->dedup_ws_bytes) && dalloc(h, &h->uniq_idx, N * 4) &&
+         dalloc(h, &h->uniq_token, N * 4) && dalloc(h, &h->uniq_count, 16);
+  }
   if (c.mode == STCA_MODE_STCA) {
     ok = ok && dalloc(h, &h->cat, T * (c.M + 1) * d * 4) && dalloc(h, &h->qbuf, T * d * 4);
     ok = ok && dalloc(h, &h->in_ids, N * 4) && dalloc(h, &h->in_len, U * 4) && dalloc(h, &h->in_tpu, U * 4) &&
@@ -258,7 +269,7 @@ int pack_layer(stca_handle* h, size_t slot, const stca_ffn& f, const void* WK, c
 
 // K/V of every history token for one layer: bf16 tensor-core path.
 int history_bf16(stca_handle* h, size_t slot, const GatherSrc& g, int n_tok, const float* gamma, const float* beta,
-                 cudaStream_t s) {
+                 cudaStream_t s, const int32_t* M_dev) {
   const int d = h->cfg.d, hd = h->cfg.hidden;
   const bf16* base = reinterpret_cast<const bf16*>(h->wpack) + slot * h->wpack_layer;
   const bf16* wp1 = base;
@@ -267,12 +278,12 @@ int history_bf16(stca_handle* h, size_t slot, const GatherSrc& g, int n_tok, con
   GatherSrc none;
   memset(&none, 0, sizeof(none));
   STAGE(h, STCA_STAGE_GATHER_FFN, s,
-        tc_gemm_resident(A_GATHER, EPI_SWIGLU, nullptr, g, n_tok, d, wp1, hd, h->hidden, hd, h->err, s));
+        tc_gemm_resident(A_GATHER, EPI_SWIGLU, nullptr, g, n_tok, d, wp1, hd, h->hidden, hd, h->err, s, M_dev));
   STAGE(h, STCA_STAGE_FFN_OUT, s,
         tc_gemm_rowwise(gamma ? EPI_LN : EPI_PLAIN, h->hidden, n_tok, hd, wp2, d, gamma, beta, h->cfg.ln_eps, h->xt,
-                        d, h->err, s));
+                        d, h->err, s, M_dev));
   STAGE(h, STCA_STAGE_KV, s,
-        tc_gemm_resident(A_TMA, EPI_PLAIN, h->xt, none, n_tok, d, wp3, 2 * d, h->kv, 2 * d, h->err, s));
+        tc_gemm_resident(A_TMA, EPI_PLAIN, h->xt, none, n_tok, d, wp3, 2 * d, h->kv, 2 * d, h->err, s, M_dev));
   return STCA_OK;
 }
 
@@ -301,12 +312,13 @@ int history_f32(stca_handle* h, const GatherSrc& g, int n_tok, const stca_ffn& f
 }
 
 int run_attention(stca_handle* h, const float* Q, const int32_t* hoff, const int32_t* toff, int B, int T,
-                  int splits, int score, cudaStream_t s) {
+                  int splits, int score, cudaStream_t s, const int32_t* kv_rows) {
   AttnArgs a;
   a.Q = Q;
   a.KV = h->kv;
   a.hoff = hoff;
   a.toff = toff;
+  a.kv_rows = kv_rows;
   a.B = B;
   a.T = T;
   a.d = h->cfg.d;
@@ -342,18 +354,29 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
   // q^(1) = LN(SwiGLU_t(x_t))
   STAGE(h, STCA_STAGE_QUERY, s, query_ffn<TB>(h, xcol, ldcat, t_tot, w->tgt, h->qbuf, d, s));
   GatherSrc g;
+  memset(&g, 0, sizeof(g));
   g.ids = ids;
   g.dt = c.time_buckets ? dt : nullptr;
   g.table = w->table;
   g.dt_table = c.time_buckets ? w->dt_table : nullptr;
   g.n_items = w->n_items;
+  const int32_t* M_dev = nullptr;
+  const int32_t* kv_rows = nullptr;
+  if (c.dedup) {
+    STAGE(h, STCA_STAGE_DEDUP, s,
+          dedup_rows(ids, g.dt, n_tok, h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx, h->uniq_token, h->uniq_count,
+                     h->err, s));
+    g.rows = h->uniq_token;
+    M_dev = h->uniq_count;
+    kv_rows = h->uniq_idx;
+  }
   const int splits = choose_splits(n_tok, B, 1024);
   for (int i = 0; i < M; ++i) {
-    if (bf) CK(history_bf16(h, i, g, n_tok, w->hist[i].gamma, w->hist[i].beta, s));
+    if (bf) CK(history_bf16(h, i, g, n_tok, w->hist[i].gamma, w->hist[i].beta, s, M_dev));
     else CK(history_f32(h, g, n_tok, w->hist[i], w->WK[i], w->WV[i], s));
     STAGE(h, STCA_STAGE_QUERY, s,
           simt_gemm(gemm_args<TB>(t_tot, d, d, h->qbuf, d, w->WQ[i], h->qproj, d, h->err), s));
-    CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, splits, c.score, s));
+    CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, splits, c.score, s, kv_rows));
     Prof p(h, STCA_STAGE_QUERY, s);
     CK(simt_gemm(gemm_args<TB>(t_tot, d, d, h->attn, d, w->WO[i], h->cat + int64_t(i) * d, ldcat, h->err), s));
     if (i + 1 < M) {
@@ -555,14 +578,25 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
       g.table = w->table;
       g.n_items = w->n_items;
       // H = SwiGLU(X_s) (eq 7), K/V = H W_K, H W_V (eq 8)
-      CK(history_bf16(h, size_t(l) * 2 + sq, g, ntok[sq], nullptr, nullptr, s));
+      const int32_t* M_dev = nullptr;
+      const int32_t* kv_rows = nullptr;
+      if (c.dedup) {
+        STAGE(h, STCA_STAGE_DEDUP, s,
+              dedup_rows(ids[sq], nullptr, ntok[sq], h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx, h->uniq_token,
+                         h->uniq_count, h->err, s));
+        g.rows = h->uniq_token;
+        M_dev = h->uniq_count;
+        kv_rows = h->uniq_idx;
+      }
+      CK(history_bf16(h, size_t(l) * 2 + sq, g, ntok[sq], nullptr, nullptr, s, M_dev));
       // queries of sequence sq: rows b*T + sq*n_query + n
       auto qa = gemm_args<bf16>(rows_s, d, d, h->hq, d, f.WQ, h->qproj, d, h->err);
       qa.a_grp = n_query;
       qa.a_gstride = T;
       qa.a_goff = sq * n_query;
       STAGE(h, STCA_STAGE_QUERY, s, simt_gemm(qa, s));
-      CK(run_attention(h, h->qproj, offs[sq], h->toff, B, rows_s, choose_splits(ntok[sq], B, 1024), STCA_SOFTMAX, s));
+      CK(run_attention(h, h->qproj, offs[sq], h->toff, B, rows_s, choose_splits(ntok[sq], B, 1024), STCA_SOFTMAX, s,
+                       kv_rows));
       auto oa = gemm_args<bf16>(rows_s, d, d, h->attn, d, f.WO, h->hqhat, d, h->err);
       oa.c_grp = n_query;
       oa.c_gstride = T;

@@ -115,9 +115,10 @@ __device__ __forceinline__ bool gather_row(const GatherSrc& g, int grow, int M, 
   id = 0;
   bucket = 0;
   if (grow >= M) return false;
-  id = g.ids[grow];
+  const int tok = g.rows ? g.rows[grow] : grow;
+  id = g.ids[tok];
   if (g.dt) {
-    const int32_t dt = g.dt[grow];
+    const int32_t dt = g.dt[tok];
     if (dt < 0) set_error(err, STCA_ERR_INVALID_ARG);
     bucket = dt_bucket(dt < 0 ? 0 : dt);
   }
@@ -144,8 +145,8 @@ __device__ __forceinline__ bool gather_row(const GatherSrc& g, int grow, int M, 
 template <int AMODE, int EPI, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     tc_gemm_resident_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                            const __grid_constant__ CUtensorMap tmC, GatherSrc g, int M, int K, int NT,
-                            int32_t* err) {
+                            const __grid_constant__ CUtensorMap tmC, GatherSrc g, int M_max, int K, int NT,
+                            int32_t* err, const int32_t* M_dev) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const int KC = K / 64;
@@ -167,6 +168,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
+  const int M = M_dev ? min(M_max, *M_dev) : M_max;  // rows present in this call
   const int num_tiles = (M + 2 * BM - 1) / (2 * BM);
   const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
 
@@ -420,8 +422,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
 template <int EPI, int NB, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     tc_gemm_rowwise_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                           const __grid_constant__ CUtensorMap tmC, int M, int K, const float* __restrict__ gamma,
-                           const float* __restrict__ beta, float eps, int32_t* err) {
+                           const __grid_constant__ CUtensorMap tmC, int M_max, int K,
+                           const float* __restrict__ gamma, const float* __restrict__ beta, float eps, int32_t* err,
+                           const int32_t* M_dev) {
   constexpr int N = NB * 256;
   constexpr int STAGE_BYTES = A_CHUNK + NB * B_HALF;
   extern __shared__ uint8_t smem_raw[];
@@ -444,6 +447,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
   const int KC = K / 64;
+  const int M = M_dev ? min(M_max, *M_dev) : M_max;  // rows present in this call
   const int num_tiles = (M + 2 * BM - 1) / (2 * BM);
   const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
 
@@ -717,25 +721,26 @@ size_t rowwise_smem(int nb, int stages) {
 
 template <int AMODE, int EPI, int STAGES>
 int run_resident(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GatherSrc& g, int M,
-                 int K, int NT, int32_t* err, cudaStream_t s) {
+                 int K, int NT, int32_t* err, cudaStream_t s, const int32_t* M_dev) {
   auto kern = tc_gemm_resident_kernel<AMODE, EPI, STAGES>;
   const size_t smem = resident_smem(K, STAGES, AMODE == A_GATHER);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
   const int grid = 2 * std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
-  kern<<<grid, 512, smem, s>>>(ta, tb, tc, g, M, K, NT, err); note_launch();
+  kern<<<grid, 512, smem, s>>>(ta, tb, tc, g, M, K, NT, err, M_dev); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
 template <int EPI, int NB, int STAGES>
 int run_rowwise(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, int M, int K,
-                const float* gamma, const float* beta, float eps, int32_t* err, cudaStream_t s) {
+                const float* gamma, const float* beta, float eps, int32_t* err, cudaStream_t s,
+                const int32_t* M_dev) {
   auto kern = tc_gemm_rowwise_kernel<EPI, NB, STAGES>;
   const size_t smem = rowwise_smem(NB, STAGES);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
   const int grid = 2 * std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
-  kern<<<grid, 384, smem, s>>>(ta, tb, tc, M, K, gamma, beta, eps, err); note_launch();
+  kern<<<grid, 384, smem, s>>>(ta, tb, tc, M, K, gamma, beta, eps, err, M_dev); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -750,7 +755,7 @@ int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_off
 }
 
 int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int K, const void* Wp, int Nout,
-                     void* C, int ldc, int32_t* err, cudaStream_t s) {
+                     void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev) {
   if (M == 0) return 0;
   if (M < 0 || (K != 256 && K != 512) || Nout <= 0 || ldc % 8 != 0) return STCA_ERR_UNSUPPORTED;
   const int N = epi == EPI_SWIGLU ? 2 * Nout : Nout;
@@ -768,8 +773,8 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
   }
   // stage counts fill the 227 KB of shared memory (see resident_smem)
 #define STCA_RES(AM, EP)                                                                                   \
-  (K == 512 ? run_resident<AM, EP, (AM == A_GATHER ? 4 : 5)>(ta, tb, tc, g, M, K, NT, err, s)               \
-            : run_resident<AM, EP, (AM == A_GATHER ? 8 : 9)>(ta, tb, tc, g, M, K, NT, err, s))
+  (K == 512 ? run_resident<AM, EP, (AM == A_GATHER ? 4 : 5)>(ta, tb, tc, g, M, K, NT, err, s, M_dev)               \
+            : run_resident<AM, EP, (AM == A_GATHER ? 8 : 9)>(ta, tb, tc, g, M, K, NT, err, s, M_dev))
   if (amode == A_TMA && epi == EPI_PLAIN) return STCA_RES(A_TMA, EPI_PLAIN);
   if (amode == A_TMA && epi == EPI_SWIGLU) return STCA_RES(A_TMA, EPI_SWIGLU);
   if (amode == A_GATHER && epi == EPI_PLAIN) return STCA_RES(A_GATHER, EPI_PLAIN);
@@ -779,7 +784,8 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
 }
 
 int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
-                    const float* beta, float eps, void* C, int ldc, int32_t* err, cudaStream_t s) {
+                    const float* beta, float eps, void* C, int ldc, int32_t* err, cudaStream_t s,
+                    const int32_t* M_dev) {
   if (M == 0) return 0;
   if (M < 0 || K <= 0 || K % 64 != 0 || (N != 256 && N != 512) || ldc % 8 != 0) return STCA_ERR_UNSUPPORTED;
   if (epi == EPI_LN && (!gamma || !beta)) return STCA_ERR_INVALID_ARG;
@@ -789,11 +795,11 @@ int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N,
   if (!make_tmap(&tb, Wp, N, K, K, BM)) return STCA_ERR_CUDA;
   if (!make_tmap_out(&tc, C, M, N, ldc)) return STCA_ERR_CUDA;
   if (N == 512) {
-    return epi == EPI_LN ? run_rowwise<EPI_LN, 2, 4>(ta, tb, tc, M, K, gamma, beta, eps, err, s)
-                         : run_rowwise<EPI_PLAIN, 2, 4>(ta, tb, tc, M, K, gamma, beta, eps, err, s);
+    return epi == EPI_LN ? run_rowwise<EPI_LN, 2, 4>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev)
+                         : run_rowwise<EPI_PLAIN, 2, 4>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev);
   }
-  return epi == EPI_LN ? run_rowwise<EPI_LN, 1, 6>(ta, tb, tc, M, K, gamma, beta, eps, err, s)
-                       : run_rowwise<EPI_PLAIN, 1, 6>(ta, tb, tc, M, K, gamma, beta, eps, err, s);
+  return epi == EPI_LN ? run_rowwise<EPI_LN, 1, 6>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev)
+                       : run_rowwise<EPI_PLAIN, 1, 6>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev);
 }
 
 }  // namespace stca

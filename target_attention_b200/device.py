@@ -47,9 +47,10 @@ class _Holder:
 
 
 class StcaModel(_Holder):
-    """Weights of an STCA workload on the device plus a handle sized for it."""
+    """Weights of an STCA workload on the device plus a handle sized for it.  dedup
+    defaults to on for bf16 workloads (the history GEMMs run once per distinct key)."""
 
-    def __init__(self, wl, device="cuda", max_users=None, max_tokens=None, max_targets=None):
+    def __init__(self, wl, device="cuda", max_users=None, max_tokens=None, max_targets=None, dedup=None):
         super().__init__(device)
         c = wl["cfg"]
         self.cfg = c
@@ -58,7 +59,8 @@ class StcaModel(_Holder):
             dtype=B.BF16 if c["dtype"] == "bf16" else B.FP32,
             score=B.RELU if c["score"] == "relu" else B.SOFTMAX, time_buckets=c["time_buckets"],
             max_users=max_users or len(wl["lengths"]), max_tokens=max_tokens or int(wl["lengths"].sum()),
-            max_targets=max_targets or int(wl["targets_per_user"].sum()), ln_eps=c.get("ln_eps", 1e-5))
+            max_targets=max_targets or int(wl["targets_per_user"].sum()),
+            dedup=int(c["dtype"] == "bf16" if dedup is None else dedup), ln_eps=c.get("ln_eps", 1e-5))
         w = wl["weights"]
         ws = B.StcaWeights()
         ws.table = self.p(wl["table"])
@@ -77,6 +79,13 @@ class StcaModel(_Holder):
         self.weights = ws
         self.handle = B.stca_create(self.config)
 
+    def other_handle(self, **changes):
+        """A second handle over the same device weights with some config fields changed."""
+        cfg = B.StcaConfig.from_buffer_copy(self.config)
+        for k, v in changes.items():
+            setattr(cfg, k, v)
+        return B.stca_create(cfg)
+
     def inputs(self, wl):
         d = {k: to_device(wl[k], self.device) for k in ("ids", "lengths", "dt", "x_t", "targets_per_user")}
         d["B"] = len(wl["lengths"])
@@ -84,8 +93,8 @@ class StcaModel(_Holder):
         d["t_tot"] = int(wl["targets_per_user"].sum())
         return d
 
-    def forward(self, x, z_out, o_out=None, stream=None):
-        return B.stca_forward(self.handle, x["ids"], x["lengths"], x["dt"], x["x_t"], x["targets_per_user"],
+    def forward(self, x, z_out, o_out=None, stream=None, handle=None):
+        return B.stca_forward(handle or self.handle, x["ids"], x["lengths"], x["dt"], x["x_t"], x["targets_per_user"],
                               x["B"], x["n_tok"], x["t_tot"], self.weights, z_out, o_out, stream)
 
     def forward_host(self, x, z_out, stream=None):
@@ -107,7 +116,8 @@ class PointwiseModel(_Holder):
         self.cfg = c
         self.config = B.StcaConfig(mode=B.MODE_POINTWISE, M=1, d=c["d"], H=1, hidden=c["d"], dtype=B.BF16,
                                    score=B.RELU, time_buckets=0, max_users=max_users or len(wl["lengths"]),
-                                   max_tokens=max_tokens or int(wl["lengths"].sum()), max_targets=0, ln_eps=1e-5)
+                                   max_tokens=max_tokens or int(wl["lengths"].sum()), max_targets=0, dedup=0,
+                                   ln_eps=1e-5)
         self.table = self.up(wl["table"])
         self.handle = B.stca_create(self.config)
 
@@ -128,7 +138,7 @@ class PointwiseModel(_Holder):
 
 
 class HyformerModel(_Holder):
-    def __init__(self, wl, device="cuda", max_users=None, max_tokens=None):
+    def __init__(self, wl, device="cuda", max_users=None, max_tokens=None, dedup=True):
         super().__init__(device)
         c = wl["cfg"]
         self.cfg = c
@@ -138,7 +148,7 @@ class HyformerModel(_Holder):
             mode=B.MODE_HYFORMER, M=c["blocks"], d=c["d"], H=c["H"], hidden=c["hidden"], dtype=B.BF16,
             score=B.SOFTMAX, time_buckets=0, max_users=max_users or Bu,
             max_tokens=max_tokens or int(max(wl["lengths"][0].sum(), wl["lengths"][1].sum())),
-            max_targets=(max_users or Bu) * 2 * nq, ln_eps=1e-5)
+            max_targets=(max_users or Bu) * 2 * nq, dedup=int(dedup), ln_eps=1e-5)
         ws = B.HyfWeights()
         ws.table = self.p(wl["table"])
         ws.n_items = wl["table"].shape[0]
@@ -162,8 +172,14 @@ class HyformerModel(_Holder):
                     B=len(wl["lengths"][0]), n_feed=int(wl["lengths"][0].sum()),
                     n_search=int(wl["lengths"][1].sum()), n_query=self.cfg["n_query"])
 
-    def forward(self, x, out, stream=None):
-        return B.hyformer_forward(self.handle, x["ids_feed"], x["len_feed"], x["n_feed"], x["ids_search"],
+    def other_handle(self, **changes):
+        cfg = B.StcaConfig.from_buffer_copy(self.config)
+        for k, v in changes.items():
+            setattr(cfg, k, v)
+        return B.stca_create(cfg)
+
+    def forward(self, x, out, stream=None, handle=None):
+        return B.hyformer_forward(handle or self.handle, x["ids_feed"], x["len_feed"], x["n_feed"], x["ids_search"],
                                   x["len_search"], x["n_search"], x["q0"], x["B"], x["n_query"], self.weights, out,
                                   stream)
 

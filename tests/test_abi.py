@@ -33,7 +33,7 @@ def test_library_exports_every_declared_function():
 
 def test_struct_layouts_match_c():
     # sizes computed by the C compiler from include/stca.h
-    assert ctypes.sizeof(B.StcaConfig) == 48
+    assert ctypes.sizeof(B.StcaConfig) == 52
     assert ctypes.sizeof(B.StcaWeights) == 1072
     assert ctypes.sizeof(B.HyfWeights) == 21656
 
@@ -46,7 +46,7 @@ def test_strerror_covers_all_codes():
 
 def _cfg(**kw):
     base = dict(mode=B.MODE_STCA, M=2, d=256, H=4, hidden=512, dtype=B.BF16, score=B.SOFTMAX, time_buckets=0,
-                max_users=4, max_tokens=100, max_targets=8, ln_eps=1e-5)
+                max_users=4, max_tokens=100, max_targets=8, dedup=0, ln_eps=1e-5)
     base.update(kw)
     return B.StcaConfig(**base)
 
@@ -65,6 +65,8 @@ def _cfg(**kw):
     (dict(mode=B.MODE_HYFORMER, d=256), B.ERR_UNSUPPORTED),
     (dict(mode=5), B.ERR_INVALID_ARG),
     (dict(dtype=B.FP32, d=96, H=2), B.ERR_UNSUPPORTED),   # d_h = 48
+    (dict(dtype=B.FP32, d=64, H=2, dedup=1), B.ERR_UNSUPPORTED),
+    (dict(dedup=2), B.ERR_INVALID_ARG),
 ])
 def test_create_rejects_bad_configs(kw, code):
     h = ctypes.c_void_p()
