@@ -59,18 +59,28 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
                : "r"(addr));
 }
 
-// Issues the cp.async copies of K and V rows [key0, key0+32) of head h into one stage.
-__device__ __forceinline__ void load_kv_tile(uint8_t* stage, const bf16* KV, int64_t ld, int64_t row0, int valid,
-                                             int hcol, int d, int lane, const int32_t* kv_rows) {
-  uint8_t* sK = stage;
-  uint8_t* sV = stage + TILE_BYTES;
+// Row of each key this lane copies in a 32-key tile: lane copies chunk (lane & 7) of keys
+// 4 i + (lane >> 3), i = 0..7.  Resolved one tile ahead so that the copies of a tile never
+// wait for their row-index loads; -1 marks keys past the slice end.
+__device__ __forceinline__ void tile_rows(int (&rows)[8], const int32_t* kv_rows, int64_t row0, int valid, int lane) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int idx = i * 32 + lane;
-    const int key = idx >> 3, ch = idx & 7;
-    const bool ok = key < valid;
-    const int64_t row = ok ? (kv_rows ? int64_t(kv_rows[row0 + key]) : row0 + key) : 0;
-    const bf16* src = KV + row * ld + hcol + ch * 8;
+    const int key = i * 4 + (lane >> 3);
+    rows[i] = key < valid ? (kv_rows ? kv_rows[row0 + key] : int(row0 + key)) : -1;
+  }
+}
+
+// Issues the cp.async copies of the K and V slices of head h for the tile's 32 keys.
+__device__ __forceinline__ void load_kv_tile(uint8_t* stage, const bf16* KV, int64_t ld, const int (&rows)[8],
+                                             int hcol, int d, int lane) {
+  uint8_t* sK = stage;
+  uint8_t* sV = stage + TILE_BYTES;
+  const int ch = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int key = i * 4 + (lane >> 3);
+    const bool ok = rows[i] >= 0;
+    const bf16* src = KV + (ok ? int64_t(rows[i]) * ld : 0) + hcol + ch * 8;
     const int off = key * 128 + ((ch ^ (key & 7)) << 4);
     cp_async_16(sK + off, src, ok ? 16u : 0u);
     cp_async_16(sV + off, src + d, ok ? 16u : 0u);
@@ -131,14 +141,20 @@ __global__ void __launch_bounds__(128, 2) attn_bf16_kernel(AttnArgs a) {
     // ---- stream this warp's tiles: warp w takes tiles w, w+4, ...
     int stage = 0;
     int tile = warp;
-    if (tile < n_tiles)
-      load_kv_tile(wbuf, KV, ld, k0 + int64_t(tile) * KT, min(KT, nk - tile * KT), hcol, d, lane, a.kv_rows);
+    int rows[8];
+    if (tile < n_tiles) {
+      tile_rows(rows, a.kv_rows, k0 + int64_t(tile) * KT, min(KT, nk - tile * KT), lane);
+      load_kv_tile(wbuf, KV, ld, rows, hcol, d, lane);
+    }
     cp_async_commit();
+    if (tile + 4 < n_tiles) tile_rows(rows, a.kv_rows, k0 + int64_t(tile + 4) * KT, min(KT, nk - (tile + 4) * KT), lane);
     for (; tile < n_tiles; tile += 4) {
       const int next = tile + 4;
-      if (next < n_tiles)
-        load_kv_tile(wbuf + (stage ^ 1) * WARP_STAGE, KV, ld, k0 + int64_t(next) * KT, min(KT, nk - next * KT),
-                     hcol, d, lane, a.kv_rows);
+      if (next < n_tiles) {
+        load_kv_tile(wbuf + (stage ^ 1) * WARP_STAGE, KV, ld, rows, hcol, d, lane);
+        if (next + 4 < n_tiles)
+          tile_rows(rows, a.kv_rows, k0 + int64_t(next + 4) * KT, min(KT, nk - (next + 4) * KT), lane);
+      }
       cp_async_commit();
       cp_async_wait<1>();
       __syncwarp();

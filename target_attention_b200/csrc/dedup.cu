@@ -9,13 +9,14 @@
 //
 // Build, all on the stream, no host round trip:
 //   1. clear an open-addressing table of 2^k slots (keys = all ones = empty);
-//   2. insert every token's key (atomicCAS, linear probing), remember its slot and, for
-//      the token that created the slot, that token;
-//   3. number the occupied slots (warp-aggregated atomicAdd): uniq_token[u] = a token with
-//      that key, count = number of distinct keys;
-//   4. uniq_idx[n] = number of token n's slot.
-// The numbering order depends on scheduling; results do not, because each distinct row
-// is computed independently of where it sits.
+//   2. insert every token's key (atomicCAS, linear probing), remember its slot, and keep
+//      the smallest token index with that key (atomicMin);
+//   3. number the keys in order of their first token (a prefix scan over the tokens that
+//      are first occurrences): uniq_token[u] = first token of key u, count = number of keys;
+//   4. uniq_idx[n] = number of token n's key.
+// Numbering by first occurrence is deterministic and keeps a user's new items on
+// consecutive K/V rows, while repeated items point at rows of popular (cache-resident)
+// keys.
 #include "common.cuh"
 #include "internal.h"
 
@@ -50,12 +51,8 @@ __global__ void insert_kernel(const int32_t* __restrict__ ids, const int32_t* __
   unsigned slot = unsigned(mix64(key)) & mask;
   for (unsigned probe = 0; probe <= mask; ++probe) {
     const unsigned long long prev = atomicCAS(&keys[slot], EMPTY_KEY, key);
-    if (prev == EMPTY_KEY) {
-      first[slot] = i;
-      slot_of[i] = int32_t(slot);
-      return;
-    }
-    if (prev == key) {
+    if (prev == EMPTY_KEY || prev == key) {
+      atomicMin(&first[slot], i);
       slot_of[i] = int32_t(slot);
       return;
     }
@@ -65,28 +62,99 @@ __global__ void insert_kernel(const int32_t* __restrict__ ids, const int32_t* __
   slot_of[i] = 0;
 }
 
-__global__ void number_kernel(const unsigned long long* __restrict__ keys, const int32_t* __restrict__ first,
-                              unsigned cap, int32_t* __restrict__ slot_index, int32_t* __restrict__ uniq_token,
-                              int32_t* __restrict__ count) {
-  const unsigned s = blockIdx.x * blockDim.x + threadIdx.x;
-  const bool occ = s < cap && keys[s] != EMPTY_KEY;
-  const unsigned ballot = __ballot_sync(0xffffffffu, occ);
-  if (ballot == 0) return;
-  const int lane = threadIdx.x & 31;
-  int base = 0;
-  if (lane == 0) base = atomicAdd(count, __popc(ballot));
-  base = __shfl_sync(0xffffffffu, base, 0);
-  if (occ) {
-    const int idx = base + __popc(ballot & ((1u << lane) - 1u));
-    slot_index[s] = idx;
-    uniq_token[idx] = first[s];
-  }
+constexpr int SCAN_THREADS = 1024, SCAN_ITEMS = 4, SCAN_TILE = SCAN_THREADS * SCAN_ITEMS;
+
+__device__ __forceinline__ bool is_first(const int32_t* first, const int32_t* slot_of, int i) {
+  return first[slot_of[i]] == i;
 }
 
-__global__ void map_kernel(const int32_t* __restrict__ slot_of, const int32_t* __restrict__ slot_index, int n,
-                           int32_t* __restrict__ uniq_idx) {
+// Block-wide exclusive scan of one int per thread; returns the block total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int& excl) {
+  __shared__ int warp_tot[SCAN_THREADS / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += x;
+  }
+  if (lane == 31) warp_tot[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < SCAN_THREADS / 32 ? warp_tot[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += x;
+    }
+    warp_tot[lane] = w;
+  }
+  __syncthreads();
+  excl = (warp > 0 ? warp_tot[warp - 1] : 0) + incl - v;
+  const int total = warp_tot[SCAN_THREADS / 32 - 1];
+  __syncthreads();
+  return total;
+}
+
+// first-occurrence count per tile of SCAN_TILE tokens
+__global__ void __launch_bounds__(SCAN_THREADS) count_kernel(const int32_t* __restrict__ first,
+                                                             const int32_t* __restrict__ slot_of, int n,
+                                                             int32_t* __restrict__ tile_counts) {
+  const int base = blockIdx.x * SCAN_TILE + threadIdx.x * SCAN_ITEMS;
+  int c = 0;
+#pragma unroll
+  for (int k = 0; k < SCAN_ITEMS; ++k)
+    if (base + k < n && is_first(first, slot_of, base + k)) ++c;
+  int excl;
+  const int total = block_exclusive_scan(c, excl);
+  if (threadIdx.x == 0) tile_counts[blockIdx.x] = total;
+}
+
+// exclusive scan of the tile counts in place (one block); count = grand total
+__global__ void __launch_bounds__(SCAN_THREADS) scan_tiles_kernel(int32_t* __restrict__ tile_counts, int tiles,
+                                                                  int32_t* __restrict__ count) {
+  int carry = 0;
+  for (int b = 0; b < tiles; b += SCAN_THREADS) {
+    const int i = b + threadIdx.x;
+    const int v = i < tiles ? tile_counts[i] : 0;
+    int excl;
+    const int total = block_exclusive_scan(v, excl);
+    if (i < tiles) tile_counts[i] = carry + excl;
+    carry += total;
+  }
+  if (threadIdx.x == 0) *count = carry;
+}
+
+// number of each first occurrence; uniq_token[number] = its token
+__global__ void __launch_bounds__(SCAN_THREADS) number_kernel(const int32_t* __restrict__ first,
+                                                              const int32_t* __restrict__ slot_of, int n,
+                                                              const int32_t* __restrict__ tile_offsets,
+                                                              int32_t* __restrict__ pos,
+                                                              int32_t* __restrict__ uniq_token) {
+  const int base = blockIdx.x * SCAN_TILE + threadIdx.x * SCAN_ITEMS;
+  bool f[SCAN_ITEMS];
+  int c = 0;
+#pragma unroll
+  for (int k = 0; k < SCAN_ITEMS; ++k) {
+    f[k] = base + k < n && is_first(first, slot_of, base + k);
+    c += f[k];
+  }
+  int excl;
+  block_exclusive_scan(c, excl);
+  int p = tile_offsets[blockIdx.x] + excl;
+#pragma unroll
+  for (int k = 0; k < SCAN_ITEMS; ++k)
+    if (f[k]) {
+      pos[base + k] = p;
+      uniq_token[p] = base + k;
+      ++p;
+    }
+}
+
+__global__ void map_kernel(const int32_t* __restrict__ first, const int32_t* __restrict__ slot_of,
+                           const int32_t* __restrict__ pos, int n, int32_t* __restrict__ uniq_idx) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) uniq_idx[i] = slot_index[slot_of[i]];
+  if (i < n) uniq_idx[i] = pos[first[slot_of[i]]];
 }
 
 }  // namespace
@@ -97,31 +165,41 @@ size_t dedup_table_slots(int max_tokens) {
   return cap;
 }
 
-size_t dedup_workspace_bytes(int max_tokens) {
-  const size_t cap = dedup_table_slots(max_tokens);
-  return cap * 8 + cap * 4 * 2 + size_t(max_tokens) * 4 + 16;
+namespace {
+// keys [cap] u64 | first [cap] i32 | slot_of [n] i32 | pos [n] i32 | tile offsets
+size_t layout_bytes(size_t cap, int n) {
+  const size_t tiles = (size_t(n) + SCAN_TILE - 1) / SCAN_TILE + 1;
+  return cap * 8 + cap * 4 + size_t(n) * 8 + tiles * 4 + 64;
 }
+}  // namespace
+
+size_t dedup_workspace_bytes(int max_tokens) { return layout_bytes(dedup_table_slots(max_tokens), max_tokens); }
 
 int dedup_rows(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws_bytes, int32_t* uniq_idx,
                int32_t* uniq_token, int32_t* count, int32_t* err, cudaStream_t s) {
   if (n < 0) return STCA_ERR_INVALID_ARG;
-  size_t cap = 1024;
-  while (cap < size_t(2) * size_t(n)) cap <<= 1;
-  if (cap * 8 + cap * 8 + size_t(n) * 4 + 16 > ws_bytes) return STCA_ERR_CAPACITY;
+  const size_t cap = dedup_table_slots(n);
+  if (layout_bytes(cap, n) > ws_bytes) return STCA_ERR_CAPACITY;
   uint8_t* p = reinterpret_cast<uint8_t*>(ws);
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(p);
   int32_t* first = reinterpret_cast<int32_t*>(p + cap * 8);
-  int32_t* slot_index = first + cap;
-  int32_t* slot_of = slot_index + cap;
+  int32_t* slot_of = first + cap;
+  int32_t* pos = slot_of + n;
+  int32_t* tile_off = pos + n;
   if (cudaMemsetAsync(count, 0, sizeof(int32_t), s) != cudaSuccess) return STCA_ERR_CUDA;
   if (n == 0) return STCA_OK;
+  const int tiles = (n + SCAN_TILE - 1) / SCAN_TILE;
   if (cudaMemsetAsync(keys, 0xFF, cap * 8, s) != cudaSuccess) return STCA_ERR_CUDA;
+  if (cudaMemsetAsync(first, 0x7F, cap * 4, s) != cudaSuccess) return STCA_ERR_CUDA;  // INT_MAX-like
   insert_kernel<<<(n + 255) / 256, 256, 0, s>>>(ids, dt, n, keys, first, slot_of, unsigned(cap - 1), err);
   note_launch();
-  number_kernel<<<unsigned((cap + 255) / 256), 256, 0, s>>>(keys, first, unsigned(cap), slot_index, uniq_token,
-                                                             count);
+  count_kernel<<<tiles, SCAN_THREADS, 0, s>>>(first, slot_of, n, tile_off);
   note_launch();
-  map_kernel<<<(n + 255) / 256, 256, 0, s>>>(slot_of, slot_index, n, uniq_idx);
+  scan_tiles_kernel<<<1, SCAN_THREADS, 0, s>>>(tile_off, tiles, count);
+  note_launch();
+  number_kernel<<<tiles, SCAN_THREADS, 0, s>>>(first, slot_of, n, tile_off, pos, uniq_token);
+  note_launch();
+  map_kernel<<<(n + 255) / 256, 256, 0, s>>>(first, slot_of, pos, n, uniq_idx);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? STCA_OK : STCA_ERR_CUDA;
 }

@@ -190,9 +190,10 @@ int allocate(stca_handle* h) {
   ok = ok && dalloc(h, &h->part_acc, size_t(MAX_SPLITS) * T * d * 4) &&
        dalloc(h, &h->part_ml, size_t(MAX_SPLITS) * T * c.H * 2 * 4);
   if (c.dedup) {
+    // one map per history sequence (the decode variant keeps both of its sequences' maps)
     h->dedup_ws_bytes = dedup_workspace_bytes(c.max_tokens);
-    ok = ok && dalloc(h, &h->dedup_ws, h->dedup_ws_bytes) && dalloc(h, &h->uniq_idx, N * 4) &&
-         dalloc(h, &h->uniq_token, N * 4) && dalloc(h, &h->uniq_count, 16);
+    ok = ok && dalloc(h, &h->dedup_ws, h->dedup_ws_bytes) && dalloc(h, &h->uniq_idx, nseq * N * 4) &&
+         dalloc(h, &h->uniq_token, nseq * N * 4) && dalloc(h, &h->uniq_count, 16);
   }
   if (c.mode == STCA_MODE_STCA) {
     ok = ok && dalloc(h, &h->cat, T * (c.M + 1) * d * 4) && dalloc(h, &h->qbuf, T * d * 4);
@@ -581,12 +582,14 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
       const int32_t* M_dev = nullptr;
       const int32_t* kv_rows = nullptr;
       if (c.dedup) {
-        STAGE(h, STCA_STAGE_DEDUP, s,
-              dedup_rows(ids[sq], nullptr, ntok[sq], h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx, h->uniq_token,
-                         h->uniq_count, h->err, s));
-        g.rows = h->uniq_token;
-        M_dev = h->uniq_count;
-        kv_rows = h->uniq_idx;
+        const size_t off = size_t(sq) * c.max_tokens;
+        if (l == 0)
+          STAGE(h, STCA_STAGE_DEDUP, s,
+                dedup_rows(ids[sq], nullptr, ntok[sq], h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx + off,
+                           h->uniq_token + off, h->uniq_count + sq, h->err, s));
+        g.rows = h->uniq_token + off;
+        M_dev = h->uniq_count + sq;
+        kv_rows = h->uniq_idx + off;
       }
       CK(history_bf16(h, size_t(l) * 2 + sq, g, ntok[sq], nullptr, nullptr, s, M_dev));
       // queries of sequence sq: rows b*T + sq*n_query + n
