@@ -138,9 +138,9 @@ __device__ __forceinline__ bool gather_row(const GatherSrc& g, int grow, int M, 
 // chunk kc of the next row tile's A is loaded as soon as the last N tile has used it.
 //
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer (leader CTA), 4..11 epilogue,
-// 12..15 gather producer (gather mode): thread r copies row r of the CTA's A tile with
-// cp.async into the swizzled layout, adds the time-bucket row from shared memory, and
-// asks L2 for its row of the next tile one tile ahead.
+// 12..15 gather producer (gather mode): cp.async of the CTA's A rows into the swizzled
+// layout (8 lanes per 128-byte row segment), the time-bucket row added from shared
+// memory, and an L2 prefetch of the next tile's rows one tile ahead.
 
 template <int AMODE, int EPI, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
@@ -288,53 +288,74 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
       mbar_wait(mma_done, 0);
     }
   } else if (warp >= 12) {
+    // gather warps: warp gw copies rows 32 gw .. 32 gw + 31 of this CTA's A tile; in each
+    // copy instruction 8 consecutive lanes take the 8 16-byte chunks of one row, so a warp
+    // moves 4 whole 128-byte row segments per instruction (row r_i = 32 gw + 4 i + lane/8)
     if (AMODE == A_GATHER) {
-      const int r = (warp - 12) * 32 + lane;
+      const int gw = warp - 12;
+      const int sub = lane >> 3, c = lane & 7;
+      const int t128 = gw * 32 + lane;
       const bool with_dt = g.dt != nullptr && g.dt_table != nullptr;
       if (with_dt) {
         const uint4* src = reinterpret_cast<const uint4*>(g.dt_table);
-        for (int i = r; i < 16 * K / 8; i += 128) reinterpret_cast<uint4*>(sT)[i] = __ldg(src + i);
+        for (int i = t128; i < 16 * K / 8; i += 128) reinterpret_cast<uint4*>(sT)[i] = __ldg(src + i);
       }
       gather_sync();
       const bf16* table = reinterpret_cast<const bf16*>(g.table);
       const uint32_t a_full0 = cluster_addr(&a_full[0], 0);
-      int64_t id;
-      int bucket;
-      bool valid = cl < num_tiles && gather_row(g, cl * 2 * BM + int(rank) * BM + r, M, id, bucket, err);
-      if (valid) prefetch_l2_bulk(table + id * K, uint32_t(K) * 2);
+      int32_t id[8], nid[8];
+      int bk[8], nbk[8];
+      uint32_t vmask = 0, nvmask = 0;
+      auto rows_of = [&](int tile, int32_t (&ids)[8], int (&bks)[8], uint32_t& mask) {
+        mask = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          int64_t idl;
+          const bool v = gather_row(g, tile * 2 * BM + int(rank) * BM + gw * 32 + i * 4 + sub, M, idl, bks[i],
+                                    c == 0 ? err : nullptr);
+          ids[i] = int32_t(idl);
+          if (v) {
+            mask |= 1u << i;
+            if (c == 0) prefetch_l2_bulk(table + idl * K, uint32_t(K) * 2);
+          }
+        }
+      };
+      if (cl < num_tiles) rows_of(cl, id, bk, vmask);
       int li = 0;
       bool ok = true;
       for (int tile = cl; tile < num_tiles && ok; tile += ncl, ++li) {
-        // ask L2 for this thread's row of the next tile while this one is in flight
-        int64_t nid = 0;
-        int nbucket = 0;
+        // this lane's rows of the next tile (and an L2 prefetch of them) while this one is in flight
         const int next = tile + ncl;
-        const bool nvalid = next < num_tiles && gather_row(g, next * 2 * BM + int(rank) * BM + r, M, nid, nbucket, err);
-        if (nvalid) prefetch_l2_bulk(table + nid * K, uint32_t(K) * 2);
-        const bf16* src = table + id * int64_t(K);
-        const uint32_t nbytes = valid ? 16u : 0u;
+        if (next < num_tiles) rows_of(next, nid, nbk, nvmask);
+        else nvmask = 0;
         for (int kc = 0; kc < KC; ++kc) {
           if (li > 0 && !mbar_wait(&a_empty[kc], (li - 1) & 1)) {
             fail(abort_flag, err);
             ok = false;
             break;
           }
-          uint8_t* rowp = sA + kc * A_CHUNK + r * 128;
+          uint8_t* chunk = sA + kc * A_CHUNK;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) cp_async_16(rowp + ((c ^ (r & 7)) << 4), src + kc * 64 + c * 8, nbytes);
+          for (int i = 0; i < 8; ++i) {
+            const int r = gw * 32 + i * 4 + sub;
+            const bool v = (vmask >> i) & 1u;
+            cp_async_16(chunk + r * 128 + ((c ^ (r & 7)) << 4), table + int64_t(v ? id[i] : 0) * K + kc * 64 + c * 8,
+                        v ? 16u : 0u);
+          }
           cp_async_commit();
         }
         if (!ok) break;
-        const uint8_t* trow = sT + bucket * K * 2;
         for (int kc = 0; kc < KC; ++kc) {
           cp_async_wait_dyn(KC - 1 - kc);
-          if (with_dt && valid) {
-            uint8_t* rowp = sA + kc * A_CHUNK + r * 128;
+          if (with_dt) {
+            uint8_t* chunk = sA + kc * A_CHUNK;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              uint4* p = reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4));
+            for (int i = 0; i < 8; ++i) {
+              if (!((vmask >> i) & 1u)) continue;
+              const int r = gw * 32 + i * 4 + sub;
+              uint4* p = reinterpret_cast<uint4*>(chunk + r * 128 + ((c ^ (r & 7)) << 4));
               const uint4 x = *p;
-              const uint4 t = *reinterpret_cast<const uint4*>(trow + kc * 128 + c * 16);
+              const uint4 t = *reinterpret_cast<const uint4*>(sT + bk[i] * K * 2 + kc * 128 + c * 16);
               const __nv_bfloat162* xa = reinterpret_cast<const __nv_bfloat162*>(&x);
               const __nv_bfloat162* ta = reinterpret_cast<const __nv_bfloat162*>(&t);
               uint32_t o[4];
@@ -350,9 +371,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
           fence_proxy_async_smem();
           mbar_arrive_remote(a_full0 + kc * 8);  // the leader counts both CTAs' rows
         }
-        id = nid;
-        bucket = nbucket;
-        valid = nvalid;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          id[i] = nid[i];
+          bk[i] = nbk[i];
+        }
+        vmask = nvmask;
       }
       cp_async_wait_all();
     }
