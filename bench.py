@@ -251,9 +251,9 @@ def stage_work(stage, wl, dedup=False):
     if stage == "attention":
         tot = 0.0
         for _, n, Bu, T in passes:
-            splits = max(1, min(16, -(-(n // max(1, Bu)) // 1024)))
-            # one K and one V row (bf16) read per history token, queries read, split partials written
-            tot += n * 2 * d * 2 + T * d * 4 + splits * T * (d + 2 * H) * 4
+            # one K and one V row (bf16) read per history token, the fp32 queries read and
+            # outputs written (partial states of L-slices are overhead, not counted)
+            tot += n * 2 * d * 2 + 2 * T * d * 4
         return "hbm", tot, "byte"
     return None, None, None
 

@@ -34,10 +34,13 @@ int stca_k_pack_weight(const void* W, int K, int N, void* dst, int mode, int row
  *   "lookup while computing"; time feature of [review] §四).
  *   epi 0: C = A Wp^T (Wp packed mode 0, [Nout, K], Nout % 256 == 0)
  *   epi 1: C = SiLU(A W1) * (A W3) (Wp packed modes 1+2, [2 Nout, K], Nout % 128 == 0).
- * An id outside [0, n_items) reads as a zero row and records STCA_ERR_ID_OUT_OF_RANGE. */
+ * An id outside [0, n_items) reads as a zero row and records STCA_ERR_ID_OUT_OF_RANGE.
+ * x_out (amode 1 only, else STCA_ERR_INVALID_ARG; may be null): bf16 [M, K], 16-byte
+ * aligned, receives the gathered A rows exactly as the MMAs consumed them, so that later
+ * GEMMs over the same rows can take them as a dense amode-0 operand. */
 int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, const int32_t* dt, const void* table,
                          const void* dt_table, int64_t n_items, int M, int K, const void* Wp, int Nout, void* C,
-                         int ldc, int32_t* err, void* stream);
+                         int ldc, void* x_out, int32_t* err, void* stream);
 
 /* Tensor-core GEMM with A streamed (K % 64 == 0) and the full output row (N = 256 or
  * 512) in tensor memory: epi 0 plain, epi 2 LayerNorm(gamma, beta, eps) of each row
@@ -48,8 +51,9 @@ int stca_k_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, in
 /* Split-L cross attention plus merge ([review] 核心公式; [wechat] §1.1 local attention,
  * then merge; §1.2 ReLU scores).  Q [T, d] fp32 projected queries, KV [N, 2d] (K in
  * columns [0, d), V in [d, 2d)) bf16 when kv_bf16 else fp32, hoff/toff [B+1] offsets of
- * the users' keys and queries.  score 0 softmax, 1 relu.  part_acc [splits, T, d] and
- * part_ml [splits, T, H, 2] float32 scratch; out [T, d] float32. */
+ * the users' keys and queries.  score 0 softmax, 1 relu.  1 <= splits <= 32 slices of each
+ * user's keys (else STCA_ERR_INVALID_ARG).  part_acc [splits, T, d] and part_ml
+ * [splits, T, H, 2] float32 scratch; out [T, d] float32. */
 int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B,
                      int T, int d, int H, int splits, int score, float* part_acc, float* part_ml, float* out,
                      int32_t* err, void* stream);

@@ -7,7 +7,8 @@
 //   relu:    acc = sum_j relu(s_j) v_j
 // with s_j = q.k_j / sqrt(d_h) (scores kept in log2 units for the softmax form).
 // The merge kernel combines the slices (WeChat TA article §1.1: items of a sequence do
-// not interact, so local attention results can be merged):
+// not interact, so local attention results can be merged); with a single slice the bf16
+// kernel writes the normalised output itself and no merge runs:
 //   softmax: M = max_c mx_c, o = sum_c 2^(mx_c - M) acc_c / sum_c 2^(mx_c - M) l_c
 //   relu:    o = sum_c acc_c
 // An empty key set gives o = 0.
@@ -311,15 +312,18 @@ __global__ void __launch_bounds__(128, 2) attn_bf16_kernel(AttnArgs a) {
 #pragma unroll
           for (int w = 0; w < 4; ++w) wgt[w] = 1.f;
         }
-        float* pacc = a.part_acc + (int64_t(s) * a.T + t) * d + hcol + seg * 16;
+        // one slice: the state is final, so write the normalised output (no merge pass)
+        const bool direct = a.splits == 1;
+        const float scale = (SCORE == 0 && direct) ? (Lsum > 0.f ? 1.f / Lsum : 0.f) : 1.f;
+        float* pacc = (direct ? a.out + int64_t(t) * d : a.part_acc + (int64_t(s) * a.T + t) * d) + hcol + seg * 16;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           float v = 0.f;
 #pragma unroll
           for (int w = 0; w < 4; ++w) v += wgt[w] * comb[(w * 32 + row) * DH + seg * 16 + c];
-          pacc[c] = v;
+          pacc[c] = v * scale;
         }
-        if (SCORE == 0 && seg == 0) {
+        if (SCORE == 0 && seg == 0 && !direct) {
           float* pml = a.part_ml + ((int64_t(s) * a.T + t) * a.H + h) * 2;
           pml[0] = M;
           pml[1] = Lsum;
@@ -417,7 +421,9 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(AttnArgs a) {
 }
 
 // ------------------------------------------------------------------------------------
-// merge of the per-slice states; one warp per (target, head)
+// merge of the per-slice states; one warp per (target, head).  Lane s < splits turns
+// slice s's running max and sum into its weight once; the column loop then reads every
+// slice's accumulator with the weights broadcast by shuffles, four slices in flight.
 
 template <int SCORE>
 __global__ void attn_merge_kernel(AttnArgs a) {
@@ -426,24 +432,41 @@ __global__ void attn_merge_kernel(AttnArgs a) {
   if (wid >= int64_t(a.T) * a.H) return;
   const int t = int(wid / a.H), h = int(wid % a.H);
   const int dh = a.d / a.H;
-  float M = -INFINITY;
-  if (SCORE == 0)
-    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[((int64_t(s) * a.T + t) * a.H + h) * 2]);
-  float Lsum = 0.f;
+  const int S = a.splits;
+  float w = 0.f, inv = 1.f;
+  if (SCORE == 0) {
+    float m = -INFINITY, l = 0.f;
+    if (lane < S) {
+      const float2 ml = *reinterpret_cast<const float2*>(a.part_ml + ((int64_t(lane) * a.T + t) * a.H + h) * 2);
+      m = ml.x;
+      l = ml.y;
+    }
+    float M = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    w = (m == -INFINITY) ? 0.f : exp2f(m - M);
+    float Lsum = w * l;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+    inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+  } else {
+    w = 1.f;
+  }
+  const int64_t slice = int64_t(a.T) * a.d;
+  const float* acc = a.part_acc + int64_t(t) * a.d + h * dh;
   for (int c = lane; c < dh; c += 32) {
     float v = 0.f;
-    Lsum = 0.f;
-    for (int s = 0; s < a.splits; ++s) {
-      float w = 1.f;
-      if (SCORE == 0) {
-        const float* ml = a.part_ml + ((int64_t(s) * a.T + t) * a.H + h) * 2;
-        w = (ml[0] == -INFINITY) ? 0.f : exp2f(ml[0] - M);
-        Lsum += w * ml[1];
-      }
-      v += w * a.part_acc[(int64_t(s) * a.T + t) * a.d + h * dh + c];
+    int s = 0;
+    for (; s + 4 <= S; s += 4) {
+      const float x0 = acc[(s + 0) * slice + c], x1 = acc[(s + 1) * slice + c];
+      const float x2 = acc[(s + 2) * slice + c], x3 = acc[(s + 3) * slice + c];
+      v += __shfl_sync(0xffffffffu, w, s + 0) * x0;
+      v += __shfl_sync(0xffffffffu, w, s + 1) * x1;
+      v += __shfl_sync(0xffffffffu, w, s + 2) * x2;
+      v += __shfl_sync(0xffffffffu, w, s + 3) * x3;
     }
-    if (SCORE == 0) v = Lsum > 0.f ? v / Lsum : 0.f;
-    a.out[int64_t(t) * a.d + h * dh + c] = v;
+    for (; s < S; ++s) v += __shfl_sync(0xffffffffu, w, s) * acc[s * slice + c];
+    a.out[int64_t(t) * a.d + h * dh + c] = SCORE == 0 ? v * inv : v;
   }
 }
 
@@ -489,6 +512,7 @@ switch (dh) {
 
 int attention_merge(const AttnArgs& a, cudaStream_t s) {
   if (a.T == 0) return 0;
+  if (a.splits < 1 || a.splits > 32) return STCA_ERR_INVALID_ARG;  // one lane per slice
   const int64_t warps = int64_t(a.T) * a.H;
   const int blocks = int((warps * 32 + 255) / 256);
   if (a.score == 0) attn_merge_kernel<0><<<blocks, 256, 0, s>>>(a);

@@ -37,9 +37,11 @@ int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_off
 //   epi EPI_PLAIN:  C = A Wp^T, Wp packed [N, K], N a multiple of 256, Nout = N
 //   epi EPI_SWIGLU: Wp packed gate/up interleaved [2*Nout, K], C = SiLU(A W1) * (A W3)
 // M_dev, when not null, is a device int holding the number of rows actually present
-// (<= M); M then only sizes the tensor maps and buffers.
+// (<= M); M then only sizes the tensor maps and buffers.  x_out (A_GATHER only, may be
+// null): bf16 [M, K] receiving the gathered A rows (E[id] + T[bucket]) as the MMAs used them.
 int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int K, const void* Wp,
-                     int Nout, void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev = nullptr);
+                     int Nout, void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev = nullptr,
+                     void* x_out = nullptr);
 
 // C[M, N] (bf16) = epi(A Wp^T), A dense bf16 [M, K] streamed (K a multiple of 64),
 // N in {256, 512}; epi EPI_LN applies LayerNorm (gamma, beta, eps) over the full row.
@@ -108,7 +110,11 @@ struct AttnArgs {
 };
 int attention_bf16(const AttnArgs& a, cudaStream_t s);
 int attention_f32(const AttnArgs& a, cudaStream_t s);
+// combines the slices; not needed after attention_bf16 with splits == 1, which writes out
 int attention_merge(const AttnArgs& a, cudaStream_t s);
+inline bool attention_needs_merge(const AttnArgs& a, bool kv_bf16) { return !(kv_bf16 && a.splits == 1); }
+// streaming multiprocessors of the current device
+int sm_count();
 
 // ---------------------------------------------------------------- small kernels
 

@@ -21,8 +21,9 @@ int stca_k_pack_weight(const void* W, int K, int N, void* dst, int mode, int row
 
 int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, const int32_t* dt, const void* table,
                          const void* dt_table, int64_t n_items, int M, int K, const void* Wp, int Nout, void* C,
-                         int ldc, int32_t* err, void* stream) {
+                         int ldc, void* x_out, int32_t* err, void* stream) {
   if (M < 0 || !Wp || (M > 0 && !C)) return STCA_ERR_INVALID_ARG;
+  if (x_out && amode != A_GATHER) return STCA_ERR_INVALID_ARG;
   if (epi != EPI_PLAIN && epi != EPI_SWIGLU) return STCA_ERR_INVALID_ARG;
   GatherSrc g;
   memset(&g, 0, sizeof(g));
@@ -36,7 +37,8 @@ int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, 
   } else if (amode != A_TMA || (M > 0 && !A)) {
     return STCA_ERR_INVALID_ARG;
   }
-  return tc_gemm_resident(amode, epi, A, g, M, K, Wp, Nout, C, ldc, err, reinterpret_cast<cudaStream_t>(stream));
+  return tc_gemm_resident(amode, epi, A, g, M, K, Wp, Nout, C, ldc, err, reinterpret_cast<cudaStream_t>(stream),
+                          nullptr, x_out);
 }
 
 int stca_k_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
@@ -49,7 +51,7 @@ int stca_k_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, in
 int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B,
                      int T, int d, int H, int splits, int score, float* part_acc, float* part_ml, float* out,
                      int32_t* err, void* stream) {
-  if (B < 0 || T < 0 || d <= 0 || H <= 0 || d % H != 0 || splits < 1 || (score != 0 && score != 1))
+  if (B < 0 || T < 0 || d <= 0 || H <= 0 || d % H != 0 || splits < 1 || splits > 32 || (score != 0 && score != 1))
     return STCA_ERR_INVALID_ARG;
   if (B > 0 && T > 0 && (!Q || !KV || !hoff || !toff || !part_acc || !part_ml || !out)) return STCA_ERR_INVALID_ARG;
   AttnArgs a;
@@ -71,7 +73,7 @@ int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t*
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int rc = kv_bf16 ? attention_bf16(a, s) : attention_f32(a, s);
   if (rc != STCA_OK) return rc;
-  return attention_merge(a, s);
+  return attention_needs_merge(a, kv_bf16 != 0) ? attention_merge(a, s) : STCA_OK;
 }
 
 size_t stca_k_dedup_workspace_bytes(int n) { return n < 0 ? 0 : dedup_workspace_bytes(n); }

@@ -29,6 +29,7 @@ struct stca_handle {
   void* wpack = nullptr;
   size_t wpack_layer = 0;  // elements per layer (per sequence for the decode variant)
   void *hidden = nullptr, *xt = nullptr, *kv = nullptr;
+  void* xg = nullptr;  // gathered history rows, written by the first layer, read by the rest
   // query side
   float *cat = nullptr, *qbuf = nullptr, *qproj = nullptr, *attn = nullptr, *tmp_h = nullptr, *tmp_d = nullptr;
   float *part_acc = nullptr, *part_ml = nullptr;
@@ -137,6 +138,18 @@ int choose_splits(int64_t n_tok, int B, int per_split) {
   return int(s);
 }
 
+// L-slices per user for the attention.  Every slice adds a partial state to write and
+// merge, so slices are only added while the grid (users x heads x slices) is short of
+// four waves of two CTAs per SM, and never below min_keys keys per slice on average.
+int attention_splits(int64_t n_tok, int B, int H, int min_keys) {
+  if (B <= 0 || H <= 0) return 1;
+  const int64_t ctas = int64_t(B) * H;
+  const int64_t want = (int64_t(8) * sm_count() + ctas - 1) / ctas;
+  const int64_t cap = choose_splits(n_tok, B, min_keys);
+  const int64_t s = want < cap ? want : cap;
+  return int(s < 1 ? 1 : s);
+}
+
 int esize(const stca_config& c) { return c.dtype == STCA_BF16 ? 2 : 4; }
 
 int validate_config(const stca_config& c) {
@@ -185,6 +198,7 @@ int allocate(stca_handle* h) {
     ok = ok && dalloc(h, &h->wpack, size_t(c.M) * nseq * h->wpack_layer * 2);
   }
   ok = ok && dalloc(h, &h->hidden, N * hd * E) && dalloc(h, &h->xt, N * d * E) && dalloc(h, &h->kv, N * 2 * d * E);
+  if (c.dtype == STCA_BF16 && c.M > 1) ok = ok && dalloc(h, &h->xg, nseq * N * d * 2);
   ok = ok && dalloc(h, &h->qproj, T * d * 4) && dalloc(h, &h->attn, T * d * 4) && dalloc(h, &h->tmp_h, T * hd * 4) &&
        dalloc(h, &h->tmp_d, T * d * 4);
   ok = ok && dalloc(h, &h->part_acc, size_t(MAX_SPLITS) * T * d * 4) &&
@@ -269,8 +283,10 @@ int pack_layer(stca_handle* h, size_t slot, const stca_ffn& f, const void* WK, c
 }
 
 // K/V of every history token for one layer: bf16 tensor-core path.
+// x_load: rows gathered by an earlier layer (dense operand); else gather, writing the rows
+// to x_store when it is not null.
 int history_bf16(stca_handle* h, size_t slot, const GatherSrc& g, int n_tok, const float* gamma, const float* beta,
-                 cudaStream_t s, const int32_t* M_dev) {
+                 cudaStream_t s, const int32_t* M_dev, void* x_store, const void* x_load) {
   const int d = h->cfg.d, hd = h->cfg.hidden;
   const bf16* base = reinterpret_cast<const bf16*>(h->wpack) + slot * h->wpack_layer;
   const bf16* wp1 = base;
@@ -278,8 +294,13 @@ int history_bf16(stca_handle* h, size_t slot, const GatherSrc& g, int n_tok, con
   const bf16* wp3 = wp2 + size_t(d) * hd;
   GatherSrc none;
   memset(&none, 0, sizeof(none));
-  STAGE(h, STCA_STAGE_GATHER_FFN, s,
-        tc_gemm_resident(A_GATHER, EPI_SWIGLU, nullptr, g, n_tok, d, wp1, hd, h->hidden, hd, h->err, s, M_dev));
+  if (x_load)
+    STAGE(h, STCA_STAGE_GATHER_FFN, s,
+          tc_gemm_resident(A_TMA, EPI_SWIGLU, x_load, none, n_tok, d, wp1, hd, h->hidden, hd, h->err, s, M_dev));
+  else
+    STAGE(h, STCA_STAGE_GATHER_FFN, s,
+          tc_gemm_resident(A_GATHER, EPI_SWIGLU, nullptr, g, n_tok, d, wp1, hd, h->hidden, hd, h->err, s, M_dev,
+                           x_store));
   STAGE(h, STCA_STAGE_FFN_OUT, s,
         tc_gemm_rowwise(gamma ? EPI_LN : EPI_PLAIN, h->hidden, n_tok, hd, wp2, d, gamma, beta, h->cfg.ln_eps, h->xt,
                         d, h->err, s, M_dev));
@@ -330,8 +351,9 @@ int run_attention(stca_handle* h, const float* Q, const int32_t* hoff, const int
   a.part_ml = h->part_ml;
   a.out = h->attn;
   a.err = h->err;
-  STAGE(h, STCA_STAGE_ATTENTION, s, h->cfg.dtype == STCA_BF16 ? attention_bf16(a, s) : attention_f32(a, s));
-  STAGE(h, STCA_STAGE_MERGE, s, attention_merge(a, s));
+  const bool bf = h->cfg.dtype == STCA_BF16;
+  STAGE(h, STCA_STAGE_ATTENTION, s, bf ? attention_bf16(a, s) : attention_f32(a, s));
+  if (attention_needs_merge(a, bf)) STAGE(h, STCA_STAGE_MERGE, s, attention_merge(a, s));
   return STCA_OK;
 }
 
@@ -371,9 +393,11 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
     M_dev = h->uniq_count;
     kv_rows = h->uniq_idx;
   }
-  const int splits = choose_splits(n_tok, B, 1024);
+  const int splits = attention_splits(n_tok, B, c.H, 1024);
   for (int i = 0; i < M; ++i) {
-    if (bf) CK(history_bf16(h, i, g, n_tok, w->hist[i].gamma, w->hist[i].beta, s, M_dev));
+    if (bf)
+      CK(history_bf16(h, i, g, n_tok, w->hist[i].gamma, w->hist[i].beta, s, M_dev, i == 0 ? h->xg : nullptr,
+                      i > 0 ? h->xg : nullptr));
     else CK(history_f32(h, g, n_tok, w->hist[i], w->WK[i], w->WV[i], s));
     STAGE(h, STCA_STAGE_QUERY, s,
           simt_gemm(gemm_args<TB>(t_tot, d, d, h->qbuf, d, w->WQ[i], h->qproj, d, h->err), s));
@@ -591,15 +615,17 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
         M_dev = h->uniq_count + sq;
         kv_rows = h->uniq_idx + off;
       }
-      CK(history_bf16(h, size_t(l) * 2 + sq, g, ntok[sq], nullptr, nullptr, s, M_dev));
+      void* xs = h->xg ? static_cast<bf16*>(h->xg) + size_t(sq) * size_t(h->cfg.max_tokens) * d : nullptr;
+      CK(history_bf16(h, size_t(l) * 2 + sq, g, ntok[sq], nullptr, nullptr, s, M_dev, l == 0 ? xs : nullptr,
+                      l > 0 ? xs : nullptr));
       // queries of sequence sq: rows b*T + sq*n_query + n
       auto qa = gemm_args<bf16>(rows_s, d, d, h->hq, d, f.WQ, h->qproj, d, h->err);
       qa.a_grp = n_query;
       qa.a_gstride = T;
       qa.a_goff = sq * n_query;
       STAGE(h, STCA_STAGE_QUERY, s, simt_gemm(qa, s));
-      CK(run_attention(h, h->qproj, offs[sq], h->toff, B, rows_s, choose_splits(ntok[sq], B, 1024), STCA_SOFTMAX, s,
-                       kv_rows));
+      CK(run_attention(h, h->qproj, offs[sq], h->toff, B, rows_s, attention_splits(ntok[sq], B, h->cfg.H, 1024),
+                       STCA_SOFTMAX, s, kv_rows));
       auto oa = gemm_args<bf16>(rows_s, d, d, h->attn, d, f.WO, h->hqhat, d, h->err);
       oa.c_grp = n_query;
       oa.c_gstride = T;

@@ -140,13 +140,16 @@ __device__ __forceinline__ bool gather_row(const GatherSrc& g, int grow, int M, 
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer (leader CTA), 4..11 epilogue,
 // 12..15 gather producer (gather mode): cp.async of the CTA's A rows into the swizzled
 // layout (8 lanes per 128-byte row segment), the time-bucket row added from shared
-// memory, and an L2 prefetch of the next tile's rows one tile ahead.
+// memory, and an L2 prefetch of the next tile's rows one tile ahead.  With store_x the
+// gather warps also write the finished A rows to X (TMA tile stores straight from the
+// swizzled chunks), so that later layers over the same rows read X with TMA instead of
+// gathering again.
 
 template <int AMODE, int EPI, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     tc_gemm_resident_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                            const __grid_constant__ CUtensorMap tmC, GatherSrc g, int M_max, int K, int NT,
-                            int32_t* err, const int32_t* M_dev) {
+                            const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmX,
+                            GatherSrc g, int M_max, int K, int NT, int store_x, int32_t* err, const int32_t* M_dev) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const int KC = K / 64;
@@ -321,6 +324,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
         }
       };
       if (cl < num_tiles) rows_of(cl, id, bk, vmask);
+      if (store_x && lane == 0) prefetch_tmap(&tmX);
       int li = 0;
       bool ok = true;
       for (int tile = cl; tile < num_tiles && ok; tile += ncl, ++li) {
@@ -328,6 +332,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
         const int next = tile + ncl;
         if (next < num_tiles) rows_of(next, nid, nbk, nvmask);
         else nvmask = 0;
+        if (store_x && li > 0) {
+          // the previous tile's X stores have read their chunks before the chunks refill
+          if (lane == 0) bulk_wait_read<0>();
+          __syncwarp();
+        }
         for (int kc = 0; kc < KC; ++kc) {
           if (li > 0 && !mbar_wait(&a_empty[kc], (li - 1) & 1)) {
             fail(abort_flag, err);
@@ -370,6 +379,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
           }
           fence_proxy_async_smem();
           mbar_arrive_remote(a_full0 + kc * 8);  // the leader counts both CTAs' rows
+          if (store_x) {
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmX, kc * 64, tile * 2 * BM + int(rank) * BM + gw * 32, sA + kc * A_CHUNK + gw * 32 * 128);
+              bulk_commit();
+            }
+          }
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -379,6 +395,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
         vmask = nvmask;
       }
       cp_async_wait_all();
+      if (store_x && lane == 0) bulk_wait_all();
     }
   } else if (warp >= 4) {
     // two epilogue warps per TMEM lane quarter, each taking half of the columns
@@ -725,14 +742,6 @@ bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t c
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Streaming multiprocessors of the current device (persistent grids cover each SM once).
-int sm_count() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n >= 2 ? n : 2;
-}
-
 size_t resident_smem(int K, int stages, bool gather) {
   size_t bytes = 1024 + size_t(K / 64) * A_CHUNK + size_t(stages) * B_HALF + 8 * OUT_STAGE + (gather ? T_BYTES : 0) + 512;
   return bytes < MIN_SMEM ? MIN_SMEM : bytes;
@@ -744,14 +753,15 @@ size_t rowwise_smem(int nb, int stages) {
 }
 
 template <int AMODE, int EPI, int STAGES>
-int run_resident(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GatherSrc& g, int M,
-                 int K, int NT, int32_t* err, cudaStream_t s, const int32_t* M_dev) {
+int run_resident(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tx,
+                 int store_x, const GatherSrc& g, int M, int K, int NT, int32_t* err, cudaStream_t s,
+                 const int32_t* M_dev) {
   auto kern = tc_gemm_resident_kernel<AMODE, EPI, STAGES>;
   const size_t smem = resident_smem(K, STAGES, AMODE == A_GATHER);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
   const int grid = 2 * std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
-  kern<<<grid, 512, smem, s>>>(ta, tb, tc, g, M, K, NT, err, M_dev); note_launch();
+  kern<<<grid, 512, smem, s>>>(ta, tb, tc, tx, g, M, K, NT, store_x, err, M_dev); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -770,6 +780,14 @@ int run_rowwise(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
 
 }  // namespace
 
+// Streaming multiprocessors of the current device (persistent grids cover each SM once).
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n >= 2 ? n : 2;
+}
+
 int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_offset, cudaStream_t s) {
   if (K <= 0 || N <= 0) return STCA_ERR_INVALID_ARG;
   dim3 grid((N + 31) / 32, (K + 31) / 32), block(32, 8);
@@ -779,14 +797,15 @@ int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_off
 }
 
 int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int K, const void* Wp, int Nout,
-                     void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev) {
+                     void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev, void* x_out) {
   if (M == 0) return 0;
   if (M < 0 || (K != 256 && K != 512) || Nout <= 0 || ldc % 8 != 0) return STCA_ERR_UNSUPPORTED;
   const int N = epi == EPI_SWIGLU ? 2 * Nout : Nout;
   if (N % 256 != 0) return STCA_ERR_UNSUPPORTED;
   const int NT = N / 256;
   if (reinterpret_cast<uintptr_t>(C) % 16 != 0) return STCA_ERR_INVALID_ARG;
-  CUtensorMap ta, tb, tc;
+  if (x_out && (amode != A_GATHER || reinterpret_cast<uintptr_t>(x_out) % 16 != 0)) return STCA_ERR_INVALID_ARG;
+  CUtensorMap ta, tb, tc, tx;
   memset(&ta, 0, sizeof(ta));
   if (!make_tmap(&tb, Wp, N, K, K, BM)) return STCA_ERR_CUDA;
   if (!make_tmap_out(&tc, C, M, Nout, ldc)) return STCA_ERR_CUDA;
@@ -795,10 +814,17 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
   } else {
     ta = tb;  // unused by the gather producer
   }
+  // X [M, K] written by the gather warps: one 64-column x 32-row box per warp and chunk
+  if (x_out) {
+    if (!make_tmap(&tx, x_out, M, K, K, 32)) return STCA_ERR_CUDA;
+  } else {
+    tx = tb;  // unused
+  }
+  const int sx = x_out != nullptr;
   // stage counts fill the 227 KB of shared memory (see resident_smem)
 #define STCA_RES(AM, EP)                                                                                   \
-  (K == 512 ? run_resident<AM, EP, (AM == A_GATHER ? 4 : 5)>(ta, tb, tc, g, M, K, NT, err, s, M_dev)               \
-            : run_resident<AM, EP, (AM == A_GATHER ? 8 : 9)>(ta, tb, tc, g, M, K, NT, err, s, M_dev))
+  (K == 512 ? run_resident<AM, EP, (AM == A_GATHER ? 4 : 5)>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev)     \
+            : run_resident<AM, EP, (AM == A_GATHER ? 8 : 9)>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev))
   if (amode == A_TMA && epi == EPI_PLAIN) return STCA_RES(A_TMA, EPI_PLAIN);
   if (amode == A_TMA && epi == EPI_SWIGLU) return STCA_RES(A_TMA, EPI_SWIGLU);
   if (amode == A_GATHER && epi == EPI_PLAIN) return STCA_RES(A_GATHER, EPI_PLAIN);

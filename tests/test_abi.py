@@ -89,8 +89,12 @@ def test_null_arguments_rejected_on_host():
     assert L.stca_k_attention(1, None, None, None, None, 1, 1, 256, 3, 1, 0, None, None, None, None, None) \
         == B.ERR_INVALID_ARG
     assert L.stca_k_pack_weight(None, 4, 4, None, 0, 0, None) == B.ERR_INVALID_ARG
-    assert L.stca_k_gemm_resident(1, 1, None, None, None, None, None, 0, 5, 256, None, 128, None, 128, None,
+    assert L.stca_k_gemm_resident(1, 1, None, None, None, None, None, 0, 5, 256, None, 128, None, 128, None, None,
                                   None) == B.ERR_INVALID_ARG
+    # x_out only with the gather
+    assert L.stca_k_gemm_resident(0, 0, 16, None, None, None, None, 0, 5, 256, 16, 256, 16, 256, 16, None,
+                                  None) == B.ERR_INVALID_ARG
+    assert L.stca_k_attention(1, 16, 16, 16, 16, 1, 1, 256, 4, 33, 0, 16, 16, 16, None, None) == B.ERR_INVALID_ARG
     assert L.stca_k_gemm_rowwise(5, None, 0, 64, None, 256, None, None, 1e-5, None, 256, None, None) \
         == B.ERR_INVALID_ARG
 

@@ -87,10 +87,11 @@ def test_fused_gather_is_bit_exact(K, with_dt):
     dt = (np.floor(np.exp2(g.uniform(0, 16, size=M))) - 1).astype(np.int32) if with_dt else None
     Wp = torch.eye(K, dtype=torch.bfloat16, device=dev)           # packed identity [K, K]
     C = torch.full((M, K), float("nan"), dtype=torch.bfloat16, device=dev)
+    X = torch.full((M, K), float("nan"), dtype=torch.bfloat16, device=dev)
     err = zeros_err()
     ids_t = torch.from_numpy(ids).to(dev)
     dt_t = torch.from_numpy(dt).to(dev) if with_dt else None
-    B.check(B.stca_k_gemm_resident(1, 0, None, ids_t, dt_t, E, T, n_items, M, K, Wp, K, C, K, err))
+    B.check(B.stca_k_gemm_resident(1, 0, None, ids_t, dt_t, E, T, n_items, M, K, Wp, K, C, K, err, x_out=X))
     torch.cuda.synchronize()
     assert err.item() == 0
     Ef = E.float().cpu().numpy()[ids]
@@ -98,6 +99,12 @@ def test_fused_gather_is_bit_exact(K, with_dt):
         Ef = Ef + T.float().cpu().numpy()[R.dt_bucket(dt)]    # fp32 sum, as the kernel
     expect = torch.from_numpy(Ef.astype(np.float32)).to(torch.bfloat16)
     np.testing.assert_array_equal(bits_of(C), bits_of(expect))
+    # the written-through rows are the same bits, and a dense GEMM over them matches
+    np.testing.assert_array_equal(bits_of(X), bits_of(expect))
+    C2 = torch.full((M, K), float("nan"), dtype=torch.bfloat16, device=dev)
+    B.check(B.stca_k_gemm_resident(0, 0, X, None, None, None, None, 0, M, K, Wp, K, C2, K, err))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bits_of(C2), bits_of(expect))
 
 
 def test_fused_gather_flags_bad_ids():
@@ -222,7 +229,7 @@ def _attention_case(kv_bf16, d, H, lengths, targets, splits, score, seed):
 
 
 @pytest.mark.parametrize("score", [0, 1])
-@pytest.mark.parametrize("splits", [1, 3])
+@pytest.mark.parametrize("splits", [1, 3, 16])
 def test_attention_bf16(score, splits):
     lengths = [0, 1, 31, 33, 700, 2049, 5]
     targets = [2, 1, 16, 17, 33, 40, 0]
@@ -265,12 +272,18 @@ def test_gather_swiglu_many_tiles_per_pair(with_dt):
     Wp = _pack(W1, 1, 2 * hidden)
     _pack(W3, 2, 2 * hidden, dst=Wp)
     C = torch.empty((M, hidden), dtype=torch.bfloat16, device=dev)
+    Xw = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
     err = zeros_err()
     B.check(B.stca_k_gemm_resident(1, 1, None, torch.from_numpy(ids).to(dev),
                                    torch.from_numpy(dt).to(dev) if with_dt else None, E, T, n_items, M, K, Wp,
-                                   hidden, C, hidden, err))
+                                   hidden, C, hidden, err, x_out=Xw))
     torch.cuda.synchronize()
     assert err.item() == 0
+    # every written-through row, bit for bit (fp32 sum rounded once to bf16)
+    Ef = E.float().cpu().numpy()[ids]
+    if with_dt:
+        Ef = Ef + T.float().cpu().numpy()[R.dt_bucket(dt)]
+    np.testing.assert_array_equal(bits_of(Xw), bits_of(torch.from_numpy(Ef.astype(np.float32)).to(torch.bfloat16)))
     rows = _rows_sample(M)
     X = bf16_to_f64(E)[ids[rows]]
     if with_dt:
