@@ -42,6 +42,18 @@ int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, 
                          const void* dt_table, int64_t n_items, int M, int K, const void* Wp, int Nout, void* C,
                          int ldc, void* x_out, int32_t* err, void* stream);
 
+/* Target-side tensor-core GEMM ([review] §三 fusion formula; [notes] STCA query update):
+ * fp32 activations A (each split into two bf16 terms, so products keep fp32 accuracy),
+ * packed bf16 weights, fp32 result C [M, ldc]:
+ *   dual 0: C = A W (+ R),  Wp = stca_k_pack_weight mode 0 of W [K, N] ([N, K]);
+ *   dual 1: C = SiLU(A W1) * (A W3) (+ R), Wp = modes 1 + 2 of W1, W3 ([2N, K]).
+ * Logical column k of A is read at k (k < ksplit) or k + kshift (two concatenated blocks).
+ * Needs K % 64 == 0, ksplit % 64 == 0 when ksplit < K, N % 32 == 0 (N % 128 == 0 when dual),
+ * A, C, R 16-byte aligned with lda, ldc, ldr % 4 == 0, else STCA_ERR_UNSUPPORTED.  R may be
+ * null. */
+int stca_k_gemm_query(const float* A, int64_t lda, int M, int K, int ksplit, int kshift, const void* Wp, int N,
+                      int dual, const float* R, int64_t ldr, float* C, int64_t ldc, int32_t* err, void* stream);
+
 /* Tensor-core GEMM with A streamed (K % 64 == 0) and the full output row (N = 256 or
  * 512) in tensor memory: epi 0 plain, epi 2 LayerNorm(gamma, beta, eps) of each row
  * ([notes] STCA: X~ = LN(SwiGLU(X))).  C [M, ldc] bf16. */

@@ -87,6 +87,8 @@ _SIGS = [
     ("stca_k_pack_weight", _i32, [_vp, _i32, _i32, _vp, _i32, _i32, _vp]),
     ("stca_k_gemm_resident", _i32, [_i32, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _i32, _vp, _i32, _vp,
                                     _vp, _vp]),
+    ("stca_k_gemm_query", _i32, [_vp, _i64, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _vp, _i64, _vp, _i64, _vp,
+                                 _vp]),
     ("stca_k_gemm_rowwise", _i32, [_i32, _vp, _i32, _i32, _vp, _i32, _vp, _vp, ctypes.c_float, _vp, _i32, _vp, _vp]),
     ("stca_k_attention", _i32, [_i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
                                 _vp]),
@@ -222,6 +224,11 @@ def stca_k_gemm_resident(amode, epi, A, ids, dt, table, dt_table, n_items, M, K,
                          stream=None, x_out=None) -> int:
     return lib().stca_k_gemm_resident(amode, epi, ptr(A), ptr(ids), ptr(dt), ptr(table), ptr(dt_table), n_items, M,
                                       K, ptr(Wp), Nout, ptr(C), ldc, ptr(x_out), ptr(err), stream_ptr(stream))
+
+
+def stca_k_gemm_query(A, lda, M, K, ksplit, kshift, Wp, N, dual, R, ldr, C, ldc, err, stream=None) -> int:
+    return lib().stca_k_gemm_query(ptr(A), lda, M, K, ksplit, kshift, ptr(Wp), N, int(dual), ptr(R), ldr, ptr(C),
+                                   ldc, ptr(err), stream_ptr(stream))
 
 
 def stca_k_gemm_rowwise(epi, A, M, K, Wp, N, gamma, beta, eps, C, ldc, err, stream=None) -> int:

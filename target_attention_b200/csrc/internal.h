@@ -1,6 +1,7 @@
 // Host-side launchers shared between the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -32,6 +33,15 @@ enum Epi { EPI_PLAIN = 0, EPI_SWIGLU = 1, EPI_LN = 2 };
 // mode 2: SwiGLU up half:    dst row (n/128)*256 + 128 + n%128 <- column n of W3
 int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_offset, cudaStream_t s);
 
+// The same packing for many matrices with one launch per PACK_MAX_JOBS jobs.
+struct PackJob {
+  const void* W;  // [K, N] bf16
+  void* dst;
+  int K, N, mode, row_offset;
+};
+constexpr int PACK_MAX_JOBS = 48;
+int tc_pack_weights(const PackJob* jobs, int n, cudaStream_t s);
+
 // C[M, Nout] (bf16, row stride ldc) from A (resident in shared memory, K in {256, 512}):
 //   amode A_TMA: A is a dense bf16 [M, K] matrix; A_GATHER: rows gathered via `g`.
 //   epi EPI_PLAIN:  C = A Wp^T, Wp packed [N, K], N a multiple of 256, Nout = N
@@ -48,6 +58,10 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
 int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
                     const float* beta, float eps, void* C, int ldc, int32_t* err, cudaStream_t s,
                     const int32_t* M_dev = nullptr);
+
+// 2-D bf16 tensor map over a [rows, cols] row-major matrix (row stride ld elements),
+// box = 64 columns x box_rows rows, 128-byte swizzle, zero fill outside the matrix.
+bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows);
 
 // ---------------------------------------------------------------- SIMT fp32 GEMMs
 
@@ -88,6 +102,14 @@ int simt_gemm(const SimtGemmArgs<TA, TB>& a, cudaStream_t s);
 // (activations split into two bf16 terms); used by simt_gemm when the shapes allow.
 bool query_gemm_supported(const SimtGemmArgs<float, __nv_bfloat16>& a);
 int query_gemm(const SimtGemmArgs<float, __nv_bfloat16>& a, cudaStream_t s);
+
+// tcgen05 form of simt_gemm<float, bf16> (same fp32-accurate split products) without
+// gather, K % 64 == 0, ksplit % 64 == 0 (when < K), N % 32 == 0 (N % 128 == 0 with B2),
+// 16-byte aligned A, C, R with row strides % 4 == 0.  Wp holds B (and B2) packed K-major:
+// tc_pack_weight mode 0 [N, K], or modes 1 + 2 [2N, K] for the SwiGLU pair; with batch > 1
+// the batches' packed matrices follow one another (and a.B / a.Bz are not read).
+bool tc_query_supported(const SimtGemmArgs<float, __nv_bfloat16>& a);
+int tc_query_gemm(const SimtGemmArgs<float, __nv_bfloat16>& a, const void* Wp, cudaStream_t s);
 
 // y = LayerNorm(x) row-wise over d columns, fp32; x and y may alias.
 int layer_norm_f32(const float* x, int64_t ldx, float* y, int64_t ldy, int rows, int d, const float* gamma,

@@ -41,6 +41,31 @@ int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, 
                           nullptr, x_out);
 }
 
+int stca_k_gemm_query(const float* A, int64_t lda, int M, int K, int ksplit, int kshift, const void* Wp, int N,
+                      int dual, const float* R, int64_t ldr, float* C, int64_t ldc, int32_t* err, void* stream) {
+  if (M < 0 || K <= 0 || N <= 0 || !Wp || (M > 0 && (!A || !C)) || ksplit < 0 || kshift < 0 ||
+      (dual != 0 && dual != 1))
+    return STCA_ERR_INVALID_ARG;
+  SimtGemmArgs<float, bf16> a;
+  memset(&a, 0, sizeof(a));
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.A = A;
+  a.lda = lda;
+  a.ksplit = ksplit < K ? ksplit : K;
+  a.kshift = ksplit < K ? kshift : 0;
+  a.B = reinterpret_cast<const bf16*>(Wp);
+  a.B2 = dual ? reinterpret_cast<const bf16*>(Wp) : nullptr;
+  a.C = C;
+  a.ldc = ldc;
+  a.R = R;
+  a.ldr = ldr;
+  a.batch = 1;
+  a.err = err;
+  return tc_query_gemm(a, Wp, reinterpret_cast<cudaStream_t>(stream));
+}
+
 int stca_k_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
                         const float* beta, float eps, void* C, int ldc, int32_t* err, void* stream) {
   if (M < 0 || (M > 0 && (!A || !C)) || !Wp) return STCA_ERR_INVALID_ARG;

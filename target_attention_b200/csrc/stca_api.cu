@@ -30,6 +30,12 @@ struct stca_handle {
   size_t wpack_layer = 0;  // elements per layer (per sequence for the decode variant)
   void *hidden = nullptr, *xt = nullptr, *kv = nullptr;
   void* xg = nullptr;  // gathered history rows, written by the first layer, read by the rest
+  // target-side weights packed K-major for the tensor cores (bf16 STCA), element offsets
+  void* qpack = nullptr;
+  struct QLayout {
+    size_t tgt13, tgt2, wq[STCA_MAX_LAYERS], wo[STCA_MAX_LAYERS], wc[STCA_MAX_LAYERS], fuse13[STCA_MAX_LAYERS],
+        fuse2[STCA_MAX_LAYERS], wz, z13, z2, total;
+  } ql{};
   // query side
   float *cat = nullptr, *qbuf = nullptr, *qproj = nullptr, *attn = nullptr, *tmp_h = nullptr, *tmp_d = nullptr;
   float *part_acc = nullptr, *part_ml = nullptr;
@@ -181,6 +187,34 @@ int validate_config(const stca_config& c) {
   return STCA_OK;
 }
 
+// Element offsets of every target-side weight in the packed buffer.
+stca_handle::QLayout q_layout(const stca_config& c) {
+  stca_handle::QLayout q{};
+  const size_t d = size_t(c.d), hd = size_t(c.hidden);
+  size_t at = 0;
+  auto take = [&](size_t n) {
+    const size_t o = at;
+    at += (n + 63) / 64 * 64;  // keep every matrix 128-byte aligned
+    return o;
+  };
+  q.tgt13 = take(2 * hd * d);
+  q.tgt2 = take(d * hd);
+  for (int i = 0; i < c.M; ++i) {
+    q.wq[i] = take(d * d);
+    q.wo[i] = take(d * d);
+    if (i > 0) {
+      q.wc[i] = take(d * (i + 1) * d);
+      q.fuse13[i] = take(2 * hd * d);
+      q.fuse2[i] = take(d * hd);
+    }
+  }
+  q.wz = take(d * (c.M + 1) * d);
+  q.z13 = take(2 * hd * d);
+  q.z2 = take(d * hd);
+  q.total = at;
+  return q;
+}
+
 int allocate(stca_handle* h) {
   const stca_config& c = h->cfg;
   const size_t U = size_t(c.max_users) + 1, N = size_t(c.max_tokens), T = size_t(c.max_targets);
@@ -214,6 +248,10 @@ int allocate(stca_handle* h) {
     ok = ok && dalloc(h, &h->in_ids, N * 4) && dalloc(h, &h->in_len, U * 4) && dalloc(h, &h->in_tpu, U * 4) &&
          dalloc(h, &h->in_xt, T * d * E) && dalloc(h, &h->out_z, T * d * 4);
     if (c.time_buckets) ok = ok && dalloc(h, &h->in_dt, N * 4);
+    if (c.dtype == STCA_BF16) {
+      h->ql = q_layout(c);
+      ok = ok && dalloc(h, &h->qpack, h->ql.total * 2);
+    }
   } else {
     ok = ok && dalloc(h, &h->hoff2, U * 4) && dalloc(h, &h->hq, T * d * 4) && dalloc(h, &h->hqhat, T * d * 4) &&
          dalloc(h, &h->hmix, T * d * 4);
@@ -240,16 +278,29 @@ SimtGemmArgs<float, TB> gemm_args(int M, int N, int K, const float* A, int64_t l
   return a;
 }
 
+// Target-side GEMM: tcgen05 with the packed weights Wp when given and the shape allows,
+// else the generic kernels (fp32 weights, per-batch weights).
+int qgemm(const SimtGemmArgs<float, float>& a, const bf16*, cudaStream_t s) { return simt_gemm(a, s); }
+int qgemm(const SimtGemmArgs<float, bf16>& a, const bf16* Wp, cudaStream_t s) {
+  if (Wp && tc_query_supported(a)) return tc_query_gemm(a, Wp, s);
+  return simt_gemm(a, s);
+}
+
+const bf16* qp(const stca_handle* h, size_t off) {
+  return h->qpack ? reinterpret_cast<const bf16*>(h->qpack) + off : nullptr;
+}
+
 // out[rows, d] = SwiGLU(A) (then LayerNorm when ffn.gamma != null); A [rows, K=d] fp32.
+// p13 / p2: the FFN's packed W1|W3 and W2 (or null).
 template <typename TB>
 int query_ffn(stca_handle* h, const float* A, int64_t lda, int rows, const stca_ffn& f, float* out, int64_t ldo,
-              cudaStream_t s) {
+              cudaStream_t s, const bf16* p13 = nullptr, const bf16* p2 = nullptr) {
   const int d = h->cfg.d, hd = h->cfg.hidden;
   auto g = gemm_args<TB>(rows, hd, d, A, lda, f.W1, h->tmp_h, hd, h->err);
   g.B2 = reinterpret_cast<const TB*>(f.W3);
-  CK(simt_gemm(g, s));
+  CK(qgemm(g, p13, s));
   auto g2 = gemm_args<TB>(rows, d, hd, h->tmp_h, hd, f.W2, out, ldo, h->err);
-  CK(simt_gemm(g2, s));
+  CK(qgemm(g2, p2, s));
   if (f.gamma) CK(layer_norm_f32(out, ldo, out, ldo, rows, d, f.gamma, f.beta, h->cfg.ln_eps, s));
   return STCA_OK;
 }
@@ -267,19 +318,43 @@ int check_weights(const stca_config& c, const stca_weights* w) {
   return STCA_OK;
 }
 
-// Packs one layer's history weights into K-major operand order (bf16).
-int pack_layer(stca_handle* h, size_t slot, const stca_ffn& f, const void* WK, const void* WV, cudaStream_t s) {
+// Packing jobs (K-major operand order, bf16) for one SwiGLU FFN: W1|W3 interleaved into
+// p13 [2 hd, d], W2 into p2 [d, hd].
+void ffn_jobs(const stca_ffn& f, int d, int hd, bf16* p13, bf16* p2, std::vector<PackJob>& jobs) {
+  jobs.push_back({f.W1, p13, d, hd, 1, 0});
+  jobs.push_back({f.W3, p13, d, hd, 2, 0});
+  jobs.push_back({f.W2, p2, hd, d, 0, 0});
+}
+
+// One history layer: the FFN, then W_K and W_V stacked into [2 d, d] (K rows, then V rows).
+void layer_jobs(stca_handle* h, size_t slot, const stca_ffn& f, const void* WK, const void* WV,
+                std::vector<PackJob>& jobs) {
   const int d = h->cfg.d, hd = h->cfg.hidden;
   bf16* base = reinterpret_cast<bf16*>(h->wpack) + slot * h->wpack_layer;
-  bf16* wp1 = base;                          // [2 hd, d]  gate/up interleaved
-  bf16* wp2 = base + size_t(2) * hd * d;     // [d, hd]
-  bf16* wp3 = wp2 + size_t(d) * hd;          // [2 d, d]   K rows then V rows
-  CK(tc_pack_weight(f.W1, d, hd, wp1, 1, 0, s));
-  CK(tc_pack_weight(f.W3, d, hd, wp1, 2, 0, s));
-  CK(tc_pack_weight(f.W2, hd, d, wp2, 0, 0, s));
-  CK(tc_pack_weight(WK, d, d, wp3, 0, 0, s));
-  CK(tc_pack_weight(WV, d, d, wp3, 0, d, s));
-  return STCA_OK;
+  bf16* wp1 = base;
+  bf16* wp2 = base + size_t(2) * hd * d;
+  bf16* wp3 = wp2 + size_t(d) * hd;
+  ffn_jobs(f, d, hd, wp1, wp2, jobs);
+  jobs.push_back({WK, wp3, d, d, 0, 0});
+  jobs.push_back({WV, wp3, d, d, 0, d});
+}
+
+// The target-side weights of a bf16 STCA call.
+void query_jobs(stca_handle* h, const stca_weights* w, std::vector<PackJob>& jobs) {
+  const int d = h->cfg.d, hd = h->cfg.hidden, M = h->cfg.M;
+  bf16* q = reinterpret_cast<bf16*>(h->qpack);
+  const stca_handle::QLayout& L = h->ql;
+  ffn_jobs(w->tgt, d, hd, q + L.tgt13, q + L.tgt2, jobs);
+  for (int i = 0; i < M; ++i) {
+    jobs.push_back({w->WQ[i], q + L.wq[i], d, d, 0, 0});
+    jobs.push_back({w->WO[i], q + L.wo[i], d, d, 0, 0});
+    if (i > 0) {
+      jobs.push_back({w->WC[i], q + L.wc[i], (i + 1) * d, d, 0, 0});
+      ffn_jobs(w->fuse[i], d, hd, q + L.fuse13[i], q + L.fuse2[i], jobs);
+    }
+  }
+  jobs.push_back({w->WZ, q + L.wz, (M + 1) * d, d, 0, 0});
+  ffn_jobs(w->zffn, d, hd, q + L.z13, q + L.z2, jobs);
 }
 
 // K/V of every history token for one layer: bf16 tensor-core path.
@@ -370,12 +445,18 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
     CK(exclusive_offsets(lens, B, h->hoff, n_tok, h->err, s));
     CK(exclusive_offsets(tpu, B, h->toff, t_tot, h->err, s));
     CK(copy_rows_to_f32(x_t, bf, t_tot, d, h->cat, ldcat, M * d, s));
-    if (bf)
-      for (int i = 0; i < M; ++i) CK(pack_layer(h, i, w->hist[i], w->WK[i], w->WV[i], s));
+    if (bf) {
+      std::vector<PackJob> jobs;
+      for (int i = 0; i < M; ++i) layer_jobs(h, i, w->hist[i], w->WK[i], w->WV[i], jobs);
+      if (h->qpack) query_jobs(h, w, jobs);
+      CK(tc_pack_weights(jobs.data(), int(jobs.size()), s));
+    }
   }
+  const stca_handle::QLayout& L = h->ql;
   const float* xcol = h->cat + int64_t(M) * d;
   // q^(1) = LN(SwiGLU_t(x_t))
-  STAGE(h, STCA_STAGE_QUERY, s, query_ffn<TB>(h, xcol, ldcat, t_tot, w->tgt, h->qbuf, d, s));
+  STAGE(h, STCA_STAGE_QUERY, s,
+        query_ffn<TB>(h, xcol, ldcat, t_tot, w->tgt, h->qbuf, d, s, qp(h, L.tgt13), qp(h, L.tgt2)));
   GatherSrc g;
   memset(&g, 0, sizeof(g));
   g.ids = ids;
@@ -400,25 +481,27 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
                       i > 0 ? h->xg : nullptr));
     else CK(history_f32(h, g, n_tok, w->hist[i], w->WK[i], w->WV[i], s));
     STAGE(h, STCA_STAGE_QUERY, s,
-          simt_gemm(gemm_args<TB>(t_tot, d, d, h->qbuf, d, w->WQ[i], h->qproj, d, h->err), s));
+          qgemm(gemm_args<TB>(t_tot, d, d, h->qbuf, d, w->WQ[i], h->qproj, d, h->err), qp(h, L.wq[i]), s));
     CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, splits, c.score, s, kv_rows));
     Prof p(h, STCA_STAGE_QUERY, s);
-    CK(simt_gemm(gemm_args<TB>(t_tot, d, d, h->attn, d, w->WO[i], h->cat + int64_t(i) * d, ldcat, h->err), s));
+    CK(qgemm(gemm_args<TB>(t_tot, d, d, h->attn, d, w->WO[i], h->cat + int64_t(i) * d, ldcat, h->err),
+             qp(h, L.wo[i]), s));
     if (i + 1 < M) {
       // q^(i+2) = LN(SwiGLU([o^(1) .. o^(i+1) | x_t] W_C))
       const int K = (i + 2) * d;
       auto a = gemm_args<TB>(t_tot, d, K, h->cat, ldcat, w->WC[i + 1], h->tmp_d, d, h->err);
       a.ksplit = (i + 1) * d;
       a.kshift = (M - (i + 1)) * d;
-      CK(simt_gemm(a, s));
-      CK(query_ffn<TB>(h, h->tmp_d, d, t_tot, w->fuse[i + 1], h->qbuf, d, s));
+      CK(qgemm(a, qp(h, L.wc[i + 1]), s));
+      CK(query_ffn<TB>(h, h->tmp_d, d, t_tot, w->fuse[i + 1], h->qbuf, d, s, qp(h, L.fuse13[i + 1]),
+                       qp(h, L.fuse2[i + 1])));
     }
   }
   // z = SwiGLU_Z([o^(1) .. o^(M) | x_t] W_Z)
   {
     Prof p(h, STCA_STAGE_QUERY, s);
-    CK(simt_gemm(gemm_args<TB>(t_tot, d, int(ldcat), h->cat, ldcat, w->WZ, h->tmp_d, d, h->err), s));
-    CK(query_ffn<TB>(h, h->tmp_d, d, t_tot, w->zffn, z_out, d, s));
+    CK(qgemm(gemm_args<TB>(t_tot, d, int(ldcat), h->cat, ldcat, w->WZ, h->tmp_d, d, h->err), qp(h, L.wz), s));
+    CK(query_ffn<TB>(h, h->tmp_d, d, t_tot, w->zffn, z_out, d, s, qp(h, L.z13), qp(h, L.z2)));
   }
   if (o_out && t_tot > 0) {
     for (int i = 0; i < M; ++i)
@@ -585,11 +668,13 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
     CK(exclusive_offsets(len_search, B, h->hoff2, n_search, h->err, s));
     CK(fill_arange(h->toff, B + 1, n_query, s));
     CK(copy_rows_to_f32(q0, 1, rows, d, h->hq, d, 0, s));
+    std::vector<PackJob> jobs;
     for (int l = 0; l < c.M; ++l)
       for (int sq = 0; sq < 2; ++sq) {
         const hyf_seq_weights& f = w->blk[l].seq[sq];
-        CK(pack_layer(h, size_t(l) * 2 + sq, f.ffn, f.WK, f.WV, s));
+        layer_jobs(h, size_t(l) * 2 + sq, f.ffn, f.WK, f.WV, jobs);
       }
+    CK(tc_pack_weights(jobs.data(), int(jobs.size()), s));
   }
   const int32_t* ids[2] = {ids_feed, ids_search};
   const int32_t* offs[2] = {h->hoff, h->hoff2};

@@ -25,6 +25,37 @@
 
 namespace stca {
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a [rows, cols] row-major matrix (row stride ld elements),
+// box = 64 columns x box_rows rows, 128-byte swizzle, zero fill outside the matrix.
+bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 namespace {
 
 constexpr int BM = 128;                        // tile rows = TMEM lanes
@@ -695,39 +726,34 @@ __global__ void pack_weight_kernel(const bf16* __restrict__ W, int K, int N, bf1
   }
 }
 
+// many matrices in one launch: blockIdx.z picks the job, blocks past a job's extent return
+struct PackJobs {
+  PackJob j[PACK_MAX_JOBS];
+};
+
+__global__ void pack_many_kernel(PackJobs jobs) {
+  const PackJob& jb = jobs.j[blockIdx.z];
+  const int k0 = blockIdx.y * 32, n0 = blockIdx.x * 32;
+  if (k0 >= jb.K || n0 >= jb.N) return;
+  __shared__ bf16 tile[32][33];
+  const bf16* W = reinterpret_cast<const bf16*>(jb.W);
+  bf16* dst = reinterpret_cast<bf16*>(jb.dst);
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int k = k0 + i, n = n0 + threadIdx.x;
+    tile[i][threadIdx.x] = (k < jb.K && n < jb.N) ? W[int64_t(k) * jb.N + n] : __float2bfloat16(0.f);
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int n = n0 + i, k = k0 + threadIdx.x;
+    if (n < jb.N && k < jb.K) {
+      const int row = jb.mode == 0 ? jb.row_offset + n : (n / 128) * 256 + (jb.mode == 2 ? 128 : 0) + (n % 128);
+      dst[int64_t(row) * jb.K + k] = tile[threadIdx.x][i];
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------------
 // host side
-
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// 2-D bf16 tensor map over a [rows, cols] row-major matrix (row stride ld elements),
-// box = 64 columns x box_rows rows, 128-byte swizzle, zero fill outside the matrix.
-bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 // Output map for the epilogue's TMA stores: 32 x 32 boxes, 64-byte swizzle.
 bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld) {
@@ -793,6 +819,25 @@ int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_off
   dim3 grid((N + 31) / 32, (K + 31) / 32), block(32, 8);
   pack_weight_kernel<<<grid, block, 0, s>>>(reinterpret_cast<const bf16*>(W), K, N, reinterpret_cast<bf16*>(dst),
                                             mode, row_offset); note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
+}
+
+int tc_pack_weights(const PackJob* jobs, int n, cudaStream_t s) {
+  for (int b = 0; b < n; b += PACK_MAX_JOBS) {
+    PackJobs batch;
+    memset(&batch, 0, sizeof(batch));
+    const int cnt = std::min(PACK_MAX_JOBS, n - b);
+    int gx = 1, gy = 1;
+    for (int i = 0; i < cnt; ++i) {
+      const PackJob& jb = jobs[b + i];
+      if (jb.K <= 0 || jb.N <= 0 || !jb.W || !jb.dst || jb.mode < 0 || jb.mode > 2) return STCA_ERR_INVALID_ARG;
+      batch.j[i] = jb;
+      gx = std::max(gx, (jb.N + 31) / 32);
+      gy = std::max(gy, (jb.K + 31) / 32);
+    }
+    pack_many_kernel<<<dim3(gx, gy, cnt), dim3(32, 8), 0, s>>>(batch);
+    note_launch();
+  }
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 

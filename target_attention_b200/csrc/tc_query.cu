@@ -1,0 +1,327 @@
+// tcgen05 GEMMs for the target-side (query) path.
+//
+// C = A W (+ R) or C = SiLU(A W1) * (A W3), with fp32 activations A, bf16 weights and
+// fp32 results: the query projection and W_O of every layer, the fusion W_C, W_Z and the
+// target-side SwiGLU FFNs (STCA notes, section "STCA"; review §三 fusion formula).  The
+// query path keeps fp32 activations: each activation a enters the tensor cores as two bf16
+// terms hi = bf16(a) and lo = bf16(a - hi), both multiplied by the same bf16 weight and
+// accumulated in fp32, so every product is within ~2^-17 relative of the fp32 product.
+//
+// One CTA computes a 128-row x 256-column tile with cta_group::1 MMAs (M = 128, N = 256,
+// K = 16) into 256 TMEM columns.  K streams through a 3-stage ring of 64-wide chunks: the
+// weight chunk arrives by TMA (K-major packed weights, 128-byte swizzle); four producer
+// warps load the fp32 activation rows, split them and store the hi and lo tiles in the
+// same swizzled layout.  Those warps then run the epilogue (one TMEM lane quarter each).
+// Warp 0 lane 0 issues TMA, warp 1 owns TMEM and its lane 0 issues the MMAs.  Every wait
+// is bounded (see common.cuh); a timeout sets STCA_ERR_TIMEOUT and the CTA winds down.
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace stca {
+
+namespace {
+
+constexpr int QBM = 128, QBN = 256, QKC = 64, QSTAGES = 3;
+constexpr int QA_TILE = QBM * QKC * 2;          // one bf16 activation tile: 16 KB
+constexpr int QB_TILE = QBN * QKC * 2;          // one weight chunk: 32 KB
+constexpr int QSTAGE = 2 * QA_TILE + QB_TILE;   // hi | lo | weights: 64 KB
+constexpr size_t QSMEM = 1024 + size_t(QSTAGES) * QSTAGE + 256;
+
+struct TcqArgs {
+  const float* A;
+  int64_t lda;
+  int ksplit, kshift;
+  int a_grp, a_gstride, a_goff;
+  float* C;
+  int64_t ldc;
+  int c_grp, c_gstride, c_goff;
+  const float* R;
+  int64_t ldr;
+  int M, N, K;  // N output columns
+  int64_t bsA, bsC, bsR;  // element offsets per batch (grid z)
+  int wrows;              // packed weight rows per batch
+  int32_t* err;
+};
+
+__device__ __forceinline__ uint8_t* q_align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ int64_t q_remap(int r, int grp, int gstride, int goff) {
+  return grp ? int64_t(r / grp) * gstride + goff + r % grp : int64_t(r);
+}
+
+__device__ __forceinline__ float silu_precise(float x) { return x / (1.0f + expf(-x)); }
+
+// hi and lo bf16 pairs of two fp32 values
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+template <bool DUAL>
+__global__ void __launch_bounds__(256, 1) tc_query_kernel(const __grid_constant__ CUtensorMap tmB, TcqArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = q_align1024(smem_raw);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + QSTAGES * QSTAGE);
+  uint64_t* a_full = bars;                 // [QSTAGES] 128 producer arrivals
+  uint64_t* b_full = bars + QSTAGES;       // [QSTAGES] TMA bytes
+  uint64_t* empty = bars + 2 * QSTAGES;    // [QSTAGES] MMA commit
+  uint64_t* d_full = bars + 3 * QSTAGES;   // accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(d_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * QBM;
+  const int z = blockIdx.z;
+  const int wrow0 = z * a.wrows + blockIdx.x * QBN;  // first packed weight row of this tile
+  const int KC = a.K / QKC;
+  const float* A = a.A + z * a.bsA;
+  float* C = a.C + z * a.bsC;
+  const float* R = a.R ? a.R + z * a.bsR : nullptr;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < QSTAGES; ++s) {
+      mbar_init(&a_full[s], 128);
+      mbar_init(&b_full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(d_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, QBN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tmB);
+      int issued = 0;
+      for (int kc = 0; kc < KC; ++kc, ++issued) {
+        const int s = kc % QSTAGES, round = kc / QSTAGES;
+        if ((round > 0 && !mbar_wait(&empty[s], (round - 1) & 1)) || *abort_flag) {
+          *abort_flag = 1;
+          set_error(a.err, STCA_ERR_TIMEOUT);
+          break;
+        }
+        mbar_arrive_expect_tx(&b_full[s], QB_TILE);
+        tma_load_2d(smem + s * QSTAGE + 2 * QA_TILE, &tmB, kc * QKC, wrow0, &b_full[s]);
+      }
+      // no copy may still be writing shared memory when the CTA exits
+      for (int s = 0; s < QSTAGES && s < issued; ++s) {
+        const int last = s + QSTAGES * ((issued - 1 - s) / QSTAGES);
+        mbar_wait(&b_full[s], (last / QSTAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = umma_idesc_bf16(QBM, QBN);
+      bool ok = true;
+      for (int kc = 0; kc < KC; ++kc) {
+        const int s = kc % QSTAGES;
+        const uint32_t par = (kc / QSTAGES) & 1;
+        if (!mbar_wait(&a_full[s], par) || !mbar_wait(&b_full[s], par) || *abort_flag) {
+          *abort_flag = 1;
+          set_error(a.err, STCA_ERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_hi = smem_u32(smem + s * QSTAGE);
+        const uint32_t a_lo = a_hi + QA_TILE;
+        const uint32_t b = a_hi + 2 * QA_TILE;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t bd = umma_sdesc_sw128(b + k * 32);
+          umma_bf16(tmem, umma_sdesc_sw128(a_hi + k * 32), bd, idesc, (kc | k) != 0);
+          umma_bf16(tmem, umma_sdesc_sw128(a_lo + k * 32), bd, idesc, 1);
+        }
+        umma_commit(&empty[s]);
+      }
+      if (ok) umma_commit(d_full);
+    }
+  } else if (warp >= 4) {
+    // ---- producers: lane -> (row sub = lane / 8, 8-column group c = lane % 8); warp pw
+    // takes rows 32 pw + 4 i + sub, i = 0..7, so each load instruction covers 4 whole
+    // 256-byte row segments of the chunk
+    const int pw = warp - 4;
+    const int sub = lane >> 3, c = lane & 7;
+    const float* rowp[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = m0 + pw * 32 + 4 * i + sub;
+      rowp[i] = r < a.M ? A + q_remap(r, a.a_grp, a.a_gstride, a.a_goff) * a.lda : nullptr;
+    }
+    float4 buf[16];
+    auto load = [&](int kc) {
+      const int k = kc * QKC;
+      const int col = k + (k >= a.ksplit ? a.kshift : 0) + c * 8;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (rowp[i]) {
+          buf[2 * i] = __ldg(reinterpret_cast<const float4*>(rowp[i] + col));
+          buf[2 * i + 1] = __ldg(reinterpret_cast<const float4*>(rowp[i] + col + 4));
+        } else {
+          buf[2 * i] = buf[2 * i + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    };
+    load(0);
+    bool ok = true;
+    for (int kc = 0; kc < KC; ++kc) {
+      const int s = kc % QSTAGES, round = kc / QSTAGES;
+      if ((round > 0 && !mbar_wait(&empty[s], (round - 1) & 1)) || *abort_flag) {
+        *abort_flag = 1;
+        set_error(a.err, STCA_ERR_TIMEOUT);
+        ok = false;
+        break;
+      }
+      uint8_t* hi_t = smem + s * QSTAGE;
+      uint8_t* lo_t = hi_t + QA_TILE;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int rr = pw * 32 + 4 * i + sub;
+        const int off = rr * 128 + ((c ^ (rr & 7)) << 4);
+        uint4 h, l;
+        split2(buf[2 * i].x, buf[2 * i].y, h.x, l.x);
+        split2(buf[2 * i].z, buf[2 * i].w, h.y, l.y);
+        split2(buf[2 * i + 1].x, buf[2 * i + 1].y, h.z, l.z);
+        split2(buf[2 * i + 1].z, buf[2 * i + 1].w, h.w, l.w);
+        *reinterpret_cast<uint4*>(hi_t + off) = h;
+        *reinterpret_cast<uint4*>(lo_t + off) = l;
+      }
+      if (kc + 1 < KC) load(kc + 1);  // next chunk's rows in flight while this one is consumed
+      fence_proxy_async_smem();
+      mbar_arrive(&a_full[s]);
+    }
+
+    // ---- epilogue: warp pw reads TMEM lanes 32 pw .. 32 pw + 31 (one output row per lane)
+    if (ok && !mbar_wait(d_full, 0)) {
+      *abort_flag = 1;
+      set_error(a.err, STCA_ERR_TIMEOUT);
+      ok = false;
+    }
+    __syncwarp();
+    if (ok) {
+      tc_fence_after();
+      const int row = m0 + pw * 32 + lane;
+      const uint32_t tbase = tmem + (uint32_t(pw * 32) << 16);
+      float* crow = row < a.M ? C + q_remap(row, a.c_grp, a.c_gstride, a.c_goff) * a.ldc : nullptr;
+      const float* rrow = (row < a.M && R) ? R + int64_t(row) * a.ldr : nullptr;
+      constexpr int NCH = DUAL ? 4 : 8;  // 32-column output chunks per tile
+#pragma unroll 1
+      for (int j = 0; j < NCH; ++j) {
+        float v[32];
+        tmem_ld_32x32b_x32(tbase + j * 32, v);
+        if (DUAL) {
+          float u[32];
+          tmem_ld_32x32b_x32(tbase + 128 + j * 32, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = silu_precise(v[e]) * u[e];
+        } else {
+          tmem_ld_wait();
+        }
+        const int col = (DUAL ? blockIdx.x * 128 : blockIdx.x * QBN) + j * 32;
+        if (crow && col < a.N) {
+          if (rrow) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const float4 r4 = *reinterpret_cast<const float4*>(rrow + col + e);
+              v[e] += r4.x;
+              v[e + 1] += r4.y;
+              v[e + 2] += r4.z;
+              v[e + 3] += r4.w;
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(crow + col + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, QBN);
+  }
+}
+
+}  // namespace
+
+bool tc_query_supported(const SimtGemmArgs<float, bf16>& a) {
+  auto al16 = [](const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; };
+  if (a.gather.ids || a.batch < 1) return false;
+  if (a.K <= 0 || a.K % QKC != 0 || a.N <= 0 || a.N % (a.B2 ? 128 : 32) != 0) return false;
+  if (a.ksplit < a.K && (a.ksplit % QKC != 0 || a.kshift % 4 != 0)) return false;
+  if (!al16(a.A) || a.lda % 4 != 0 || !al16(a.C) || a.ldc % 4 != 0) return false;
+  if (a.R && (!al16(a.R) || a.ldr % 4 != 0)) return false;
+  if (a.batch > 1) {
+    // per-batch weights sit back to back in the packed buffer, whole 256-row tiles each
+    const int wrows = a.B2 ? 2 * a.N : a.N;
+    if (wrows % QBN != 0 || a.bsA % 4 != 0 || a.bsC % 4 != 0 || a.bsR % 4 != 0) return false;
+  }
+  return true;
+}
+
+int tc_query_gemm(const SimtGemmArgs<float, bf16>& a, const void* Wp, cudaStream_t s) {
+  if (a.M == 0) return 0;
+  if (!tc_query_supported(a) || !Wp || a.M < 0) return STCA_ERR_UNSUPPORTED;
+  const bool dual = a.B2 != nullptr;
+  // packed rows: N (plain), or 256 per 128 output columns (gate and up halves)
+  const int wrows = dual ? 2 * a.N : a.N;
+  CUtensorMap tb;
+  if (!make_tmap(&tb, Wp, uint64_t(wrows) * a.batch, uint64_t(a.K), uint64_t(a.K), QBN)) return STCA_ERR_CUDA;
+  TcqArgs q;
+  q.A = a.A;
+  q.lda = a.lda;
+  q.ksplit = a.ksplit;
+  q.kshift = a.kshift;
+  q.a_grp = a.a_grp;
+  q.a_gstride = a.a_gstride;
+  q.a_goff = a.a_goff;
+  q.C = a.C;
+  q.ldc = a.ldc;
+  q.c_grp = a.c_grp;
+  q.c_gstride = a.c_gstride;
+  q.c_goff = a.c_goff;
+  q.R = a.R;
+  q.ldr = a.ldr;
+  q.M = a.M;
+  q.N = a.N;
+  q.K = a.K;
+  q.bsA = a.bsA;
+  q.bsC = a.bsC;
+  q.bsR = a.bsR;
+  q.wrows = wrows;
+  q.err = a.err;
+  const dim3 grid((wrows + QBN - 1) / QBN, (a.M + QBM - 1) / QBM, a.batch);
+  if (dual) {
+    if (cudaFuncSetAttribute(tc_query_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(QSMEM)) !=
+        cudaSuccess)
+      return STCA_ERR_CUDA;
+    tc_query_kernel<true><<<grid, 256, QSMEM, s>>>(tb, q);
+  } else {
+    if (cudaFuncSetAttribute(tc_query_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(QSMEM)) !=
+        cudaSuccess)
+      return STCA_ERR_CUDA;
+    tc_query_kernel<false><<<grid, 256, QSMEM, s>>>(tb, q);
+  }
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
+}
+
+}  // namespace stca

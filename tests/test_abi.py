@@ -95,6 +95,13 @@ def test_null_arguments_rejected_on_host():
     assert L.stca_k_gemm_resident(0, 0, 16, None, None, None, None, 0, 5, 256, 16, 256, 16, 256, 16, None,
                                   None) == B.ERR_INVALID_ARG
     assert L.stca_k_attention(1, 16, 16, 16, 16, 1, 1, 256, 4, 33, 0, 16, 16, 16, None, None) == B.ERR_INVALID_ARG
+    # target-side GEMM: missing operands, then shapes the tensor-core kernel does not take
+    assert L.stca_k_gemm_query(None, 64, 1, 64, 64, 0, None, 32, 0, None, 0, None, 32, None, None) \
+        == B.ERR_INVALID_ARG
+    assert L.stca_k_gemm_query(16, 100, 1, 100, 100, 0, 16, 32, 0, None, 0, 16, 32, None, None) \
+        == B.ERR_UNSUPPORTED                          # K % 64
+    assert L.stca_k_gemm_query(16, 64, 1, 64, 64, 0, 16, 64, 1, None, 0, 16, 64, None, None) \
+        == B.ERR_UNSUPPORTED                          # dual needs N % 128
     assert L.stca_k_gemm_rowwise(5, None, 0, 64, None, 256, None, None, 1e-5, None, 256, None, None) \
         == B.ERR_INVALID_ARG
 

@@ -188,6 +188,54 @@ def test_gemm_rowwise(K, N, M, ln):
     _close_bf16(bf16_to_f64(C), Y)
 
 
+# ---------------------------------------------------------------- a5/a8/a9: target-side GEMMs
+
+
+def _f32(a):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+
+
+@pytest.mark.parametrize("M, K, N, dual, split, resid", [
+    (8192 + 77, 512, 512, False, False, False),   # many row tiles and a ragged tail
+    (300, 1536, 512, False, True, True),          # two concatenated A blocks, residual
+    (129, 512, 1024, True, False, False),         # SwiGLU pair
+    (1, 1024, 96, False, False, False),           # one row; N not a multiple of the tile
+])
+def test_query_gemm_keeps_fp32_accuracy(M, K, N, dual, split, resid):
+    """The tensor-core target-side GEMM splits fp32 activations into two bf16 terms, so the
+    result matches the fp64 product of the fp32 inputs far more closely than one bf16
+    rounding of A would (2^-9)."""
+    g = _rng(21 + M)
+    lda = K + (512 if split else 0)
+    A = g.standard_normal((M, lda)).astype(np.float32)
+    ksplit, kshift = ((K // 3) // 64 * 64, 512) if split else (K, 0)
+    Al = np.concatenate([A[:, :ksplit], A[:, ksplit + kshift:K + kshift]], axis=1) if split else A[:, :K]
+    Al = Al.astype(np.float64)
+    W1 = _bf16(g.standard_normal((K, N)) / math.sqrt(K))
+    if dual:
+        W3 = _bf16(g.standard_normal((K, N)) / math.sqrt(K))
+        Wp = _pack(W1, 1, 2 * N)
+        _pack(W3, 2, 2 * N, dst=Wp)
+        ref = R.silu(Al @ bf16_to_f64(W1)) * (Al @ bf16_to_f64(W3))
+    else:
+        Wp = _pack(W1, 0, N)
+        ref = Al @ bf16_to_f64(W1)
+    Rt = None
+    if resid:
+        Rm = g.standard_normal((M, N)).astype(np.float32)
+        Rt = _f32(Rm)
+        ref = ref + Rm
+    C = torch.full((M, N), float("nan"), dtype=torch.float32, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_gemm_query(_f32(A), lda, M, K, ksplit, kshift, Wp, N, dual, Rt, N, C, N, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    got = C.cpu().numpy().astype(np.float64)
+    rel = np.abs(got - ref).max(axis=1) / np.maximum(np.abs(ref).max(axis=1), 1e-30)
+    print(f"query GEMM M={M} K={K} N={N} dual={dual}: max row rel err {rel.max():.2e}")
+    assert rel.max() < 3e-5
+
+
 # ---------------------------------------------------------------- a6/a7: attention + merge
 
 
