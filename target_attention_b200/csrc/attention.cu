@@ -20,6 +20,7 @@ namespace stca {
 namespace {
 
 constexpr float LOG2E = 1.4426950408889634f;
+constexpr float RESCALE_SLACK = 8.f;  // log2 units a running max may lag the true max
 
 __device__ __forceinline__ void slice_bounds(const AttnArgs& a, int u, int s, int64_t& k0, int& nk, int& t0, int& m) {
   const int h0 = a.hoff[u], h1 = a.hoff[u + 1];
@@ -38,8 +39,9 @@ constexpr int DH = 64;
 constexpr int KT = 32;                    // keys per warp tile
 constexpr int TILE_BYTES = KT * DH * 2;   // 4 KB for K (same for V)
 constexpr int WARP_STAGE = 2 * TILE_BYTES;
-constexpr int WARP_BYTES = 2 * WARP_STAGE;   // double-buffered K+V: 16 KB
-constexpr int ATTN_SMEM = 4 * WARP_BYTES;    // 64 KB per CTA
+constexpr int KV_STAGES = 3;                          // tiles in flight per warp
+constexpr int WARP_BYTES = KV_STAGES * WARP_STAGE;    // 24 KB
+constexpr int ATTN_SMEM = 4 * WARP_BYTES;             // 96 KB per CTA, two CTAs per SM
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -139,25 +141,31 @@ __global__ void __launch_bounds__(128, 2) attn_bf16_kernel(AttnArgs a) {
       lrow[gi][0] = lrow[gi][1] = 0.f;
     }
 
-    // ---- stream this warp's tiles: warp w takes tiles w, w+4, ...
+    // ---- stream this warp's tiles: warp w takes tiles w, w+4, ...; KV_STAGES - 1 tiles
+    // are in flight while one is computed, and the row indices run one tile further ahead
     int stage = 0;
     int tile = warp;
     int rows[8];
-    if (tile < n_tiles) {
-      tile_rows(rows, a.kv_rows, k0 + int64_t(tile) * KT, min(KT, nk - tile * KT), lane);
-      load_kv_tile(wbuf, KV, ld, rows, hcol, d, lane);
+    auto fetch_rows = [&](int tl) {
+      if (tl < n_tiles) tile_rows(rows, a.kv_rows, k0 + int64_t(tl) * KT, min(KT, nk - tl * KT), lane);
+    };
+    fetch_rows(tile);
+#pragma unroll
+    for (int p = 0; p < KV_STAGES - 1; ++p) {
+      const int tl = tile + 4 * p;
+      if (tl < n_tiles) load_kv_tile(wbuf + p * WARP_STAGE, KV, ld, rows, hcol, d, lane);
+      cp_async_commit();
+      fetch_rows(tl + 4);
     }
-    cp_async_commit();
-    if (tile + 4 < n_tiles) tile_rows(rows, a.kv_rows, k0 + int64_t(tile + 4) * KT, min(KT, nk - (tile + 4) * KT), lane);
     for (; tile < n_tiles; tile += 4) {
-      const int next = tile + 4;
-      if (next < n_tiles) {
-        load_kv_tile(wbuf + (stage ^ 1) * WARP_STAGE, KV, ld, rows, hcol, d, lane);
-        if (next + 4 < n_tiles)
-          tile_rows(rows, a.kv_rows, k0 + int64_t(next + 4) * KT, min(KT, nk - (next + 4) * KT), lane);
+      const int ahead = tile + 4 * (KV_STAGES - 1);
+      if (ahead < n_tiles) {
+        const int st = stage + KV_STAGES - 1;
+        load_kv_tile(wbuf + (st >= KV_STAGES ? st - KV_STAGES : st) * WARP_STAGE, KV, ld, rows, hcol, d, lane);
+        fetch_rows(ahead + 4);
       }
       cp_async_commit();
-      cp_async_wait<1>();
+      cp_async_wait<KV_STAGES - 1>();
       __syncwarp();
       const uint32_t sK = smem_u32(wbuf + stage * WARP_STAGE);
       const uint32_t sV = sK + TILE_BYTES;
@@ -187,16 +195,20 @@ __global__ void __launch_bounds__(128, 2) attn_bf16_kernel(AttnArgs a) {
           }
         }
       }
-      // mask keys past the slice end, then scores -> weights
+      // mask keys past the slice end (last tile only), then scores -> weights
+      if (valid < KT) {
+#pragma unroll
+        for (int gi = 0; gi < 2; ++gi)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int kidx = j * 8 + 2 * tq + (e & 1);
+              if (kidx >= valid) sacc[gi][j][e] = (SCORE == 0) ? -INFINITY : 0.f;
+            }
+      }
 #pragma unroll
       for (int gi = 0; gi < 2; ++gi) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int kidx = j * 8 + 2 * tq + (e & 1);
-            if (kidx >= valid) sacc[gi][j][e] = (SCORE == 0) ? -INFINITY : 0.f;
-          }
         if (SCORE == 0) {
 #pragma unroll
           for (int hr = 0; hr < 2; ++hr) {
@@ -205,10 +217,23 @@ __global__ void __launch_bounds__(128, 2) attn_bf16_kernel(AttnArgs a) {
             for (int j = 0; j < 4; ++j) mx = fmaxf(mx, fmaxf(sacc[gi][j][2 * hr], sacc[gi][j][2 * hr + 1]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float mnew = fmaxf(mrow[gi][hr], mx);
-            const float muse = (mnew == -INFINITY) ? 0.f : mnew;
-            const float corr = exp2f(mrow[gi][hr] - muse);
-            mrow[gi][hr] = mnew;
+            // The reference point of a row moves only when a score exceeds it by more than
+            // RESCALE_SLACK (log2 units): weights 2^(s - m) then stay <= 2^RESCALE_SLACK, exact
+            // in fp32, and the accumulators are rescaled rarely (the warp skips it when no row
+            // of it moves).  Numerator and denominator share m, so the quotient is unchanged.
+            const bool move = mx > mrow[gi][hr] + RESCALE_SLACK;
+            if (__any_sync(0xffffffffu, move)) {
+              const float mnew = move ? mx : mrow[gi][hr];
+              const float corr = (mnew == mrow[gi][hr]) ? 1.f : exp2f(mrow[gi][hr] - mnew);
+              mrow[gi][hr] = mnew;
+              lrow[gi][hr] *= corr;
+#pragma unroll
+              for (int nt = 0; nt < 8; ++nt) {
+                o[gi][nt][2 * hr] *= corr;
+                o[gi][nt][2 * hr + 1] *= corr;
+              }
+            }
+            const float muse = (mrow[gi][hr] == -INFINITY) ? 0.f : mrow[gi][hr];
             float sum = 0.f;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -218,12 +243,7 @@ __global__ void __launch_bounds__(128, 2) attn_bf16_kernel(AttnArgs a) {
               sacc[gi][j][2 * hr + 1] = p1;
               sum += p0 + p1;
             }
-            lrow[gi][hr] = lrow[gi][hr] * corr + sum;
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-              o[gi][nt][2 * hr] *= corr;
-              o[gi][nt][2 * hr + 1] *= corr;
-            }
+            lrow[gi][hr] += sum;
           }
         } else {
 #pragma unroll
@@ -258,7 +278,7 @@ __global__ void __launch_bounds__(128, 2) attn_bf16_kernel(AttnArgs a) {
         }
       }
       __syncwarp();
-      stage ^= 1;
+      stage = stage + 1 == KV_STAGES ? 0 : stage + 1;
     }
     cp_async_wait_all();
 
