@@ -34,14 +34,24 @@ __device__ __forceinline__ void slice_bounds(const AttnArgs& a, int u, int s, in
 
 // ------------------------------------------------------------------------------------
 // bf16 K/V, d_h = 64, tensor-core (mma.sync m16n8k16) scores and P V.
+//
+// A CTA of 8 warps serves one (user, L-slice, head).  The warps form 4 teams of 2; team t
+// streams the 32-key tiles t, t+4, ... of the slice through its own ring of KV_STAGES
+// shared-memory stages, both warps of the team copying half of each tile.  Within a team
+// the two warps split the work of a tile: by queries when the user has more than 16
+// targets in the current chunk (warp w takes 16 of the up to 32), else by keys (warp w
+// takes keys 16 w .. 16 w + 15 of every tile, all queries).  Each warp keeps its own
+// online-softmax state; the states are combined in shared memory at the end.
 
 constexpr int DH = 64;
-constexpr int KT = 32;                    // keys per warp tile
-constexpr int TILE_BYTES = KT * DH * 2;   // 4 KB for K (same for V)
-constexpr int WARP_STAGE = 2 * TILE_BYTES;
-constexpr int KV_STAGES = 3;                          // tiles in flight per warp
-constexpr int WARP_BYTES = KV_STAGES * WARP_STAGE;    // 24 KB
-constexpr int ATTN_SMEM = 4 * WARP_BYTES;             // 96 KB per CTA, two CTAs per SM
+constexpr int KT = 32;                        // keys per tile
+constexpr int TILE_BYTES = KT * DH * 2;       // 4 KB for K (same for V)
+constexpr int TEAM_STAGE = 2 * TILE_BYTES;    // K tile | V tile
+constexpr int KV_STAGES = 3;                  // tiles in flight per team
+constexpr int TEAMS = 4;
+constexpr int ATT_THREADS = 2 * 32 * TEAMS;   // 256
+constexpr int TEAM_BYTES = KV_STAGES * TEAM_STAGE;   // 24 KB
+constexpr int ATTN_SMEM = TEAMS * TEAM_BYTES;        // 96 KB per CTA, two CTAs per SM
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -62,26 +72,32 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
                : "r"(addr));
 }
 
-// Row of each key this lane copies in a 32-key tile: lane copies chunk (lane & 7) of keys
-// 4 i + (lane >> 3), i = 0..7.  Resolved one tile ahead so that the copies of a tile never
-// wait for their row-index loads; -1 marks keys past the slice end.
-__device__ __forceinline__ void tile_rows(int (&rows)[8], const int32_t* kv_rows, int64_t row0, int valid, int lane) {
+// Named barrier of one team's 64 threads (ids 1..TEAMS; 0 is __syncthreads).
+__device__ __forceinline__ void team_sync(int team) {
+  asm volatile("bar.sync %0, 64;" ::"r"(team + 1) : "memory");
+}
+
+// Rows of the keys that thread tt (0..63) of a team copies in a 32-key tile: chunk tt % 8
+// of keys tt / 8 + 8 i, i = 0..3.  Resolved one tile ahead so that the copies of a tile
+// never wait for their row-index loads; -1 marks keys past the slice end.
+__device__ __forceinline__ void tile_rows(int (&rows)[4], const int32_t* kv_rows, int64_t row0, int valid, int tt) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int key = i * 4 + (lane >> 3);
+  for (int i = 0; i < 4; ++i) {
+    const int key = (tt >> 3) + 8 * i;
     rows[i] = key < valid ? (kv_rows ? kv_rows[row0 + key] : int(row0 + key)) : -1;
   }
 }
 
-// Issues the cp.async copies of the K and V slices of head h for the tile's 32 keys.
-__device__ __forceinline__ void load_kv_tile(uint8_t* stage, const bf16* KV, int64_t ld, const int (&rows)[8],
-                                             int hcol, int d, int lane) {
+// Issues this thread's cp.async copies of the K and V slices of head h for a tile
+// (128-byte key rows, 16-byte chunk c of key k at chunk c ^ (k % 8)).
+__device__ __forceinline__ void load_kv_tile(uint8_t* stage, const bf16* KV, int64_t ld, const int (&rows)[4],
+                                             int hcol, int d, int tt) {
   uint8_t* sK = stage;
   uint8_t* sV = stage + TILE_BYTES;
-  const int ch = lane & 7;
+  const int ch = tt & 7;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int key = i * 4 + (lane >> 3);
+  for (int i = 0; i < 4; ++i) {
+    const int key = (tt >> 3) + 8 * i;
     const bool ok = rows[i] >= 0;
     const bf16* src = KV + (ok ? int64_t(rows[i]) * ld : 0) + hcol + ch * 8;
     const int off = key * 128 + ((ch ^ (key & 7)) << 4);
@@ -90,8 +106,105 @@ __device__ __forceinline__ void load_kv_tile(uint8_t* stage, const bf16* KV, int
   }
 }
 
+// One warp's work on one tile: its 16 queries (A fragments qa, pre-scaled) against the NJ
+// groups of 8 keys starting at group j0, then O += P V.  State per row half hr (rows g and
+// g + 8 of the warp's 16): running reference point mrow and sum lrow (softmax), O in o.
+template <int SCORE, int NJ>
+__device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, int j0, const uint32_t (&qa)[4][4],
+                                          float (&o)[8][4], float (&mrow)[2], float (&lrow)[2], int valid,
+                                          int lane) {
+  const int tq = lane & 3;
+  // S = Q K^T
+  float sacc[NJ][4];
+#pragma unroll
+  for (int jj = 0; jj < NJ; ++jj)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sacc[jj][e] = 0.f;
+#pragma unroll
+  for (int jj = 0; jj < NJ; ++jj) {
+    const int key = (j0 + jj) * 8 + (lane & 7);
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      const int ch = 4 * p + (lane >> 3);
+      uint32_t kb[4];
+      ldsm_x4(sK + key * 128 + ((ch ^ (key & 7)) << 4), kb);
+      mma_bf16_16816(sacc[jj], qa[2 * p], kb[0], kb[1]);
+      mma_bf16_16816(sacc[jj], qa[2 * p + 1], kb[2], kb[3]);
+    }
+  }
+  // keys past the slice end (last tile only)
+  if (valid < KT) {
+#pragma unroll
+    for (int jj = 0; jj < NJ; ++jj)
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        if ((j0 + jj) * 8 + 2 * tq + (e & 1) >= valid) sacc[jj][e] = (SCORE == 0) ? -INFINITY : 0.f;
+  }
+  // scores -> weights
+  if (SCORE == 0) {
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      float mx = -INFINITY;
+#pragma unroll
+      for (int jj = 0; jj < NJ; ++jj) mx = fmaxf(mx, fmaxf(sacc[jj][2 * hr], sacc[jj][2 * hr + 1]));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+      // The reference point of a row moves only when a score exceeds it by more than
+      // RESCALE_SLACK (log2 units): weights 2^(s - m) then stay <= 2^RESCALE_SLACK, exact in
+      // fp32, and the state is rescaled rarely (skipped when no row of the warp moves).
+      // Numerator and denominator share m, so the quotient is unchanged.
+      const bool move = mx > mrow[hr] + RESCALE_SLACK;
+      if (__any_sync(0xffffffffu, move)) {
+        const float mnew = move ? mx : mrow[hr];
+        const float corr = (mnew == mrow[hr]) ? 1.f : exp2f(mrow[hr] - mnew);
+        mrow[hr] = mnew;
+        lrow[hr] *= corr;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+          o[nt][2 * hr] *= corr;
+          o[nt][2 * hr + 1] *= corr;
+        }
+      }
+      const float muse = (mrow[hr] == -INFINITY) ? 0.f : mrow[hr];
+      float sum = 0.f;
+#pragma unroll
+      for (int jj = 0; jj < NJ; ++jj) {
+        const float p0 = exp2f(sacc[jj][2 * hr] - muse);
+        const float p1 = exp2f(sacc[jj][2 * hr + 1] - muse);
+        sacc[jj][2 * hr] = p0;
+        sacc[jj][2 * hr + 1] = p1;
+        sum += p0 + p1;
+      }
+      lrow[hr] += sum;
+    }
+  } else {
+#pragma unroll
+    for (int jj = 0; jj < NJ; ++jj)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[jj][e] = fmaxf(sacc[jj][e], 0.f);
+  }
+  // O += P V   (P as A fragments straight from the score accumulators)
+#pragma unroll
+  for (int kb = 0; kb < NJ / 2; ++kb) {
+    uint32_t pa[4];
+    pa[0] = pack_bf16x2(sacc[2 * kb][0], sacc[2 * kb][1]);
+    pa[1] = pack_bf16x2(sacc[2 * kb][2], sacc[2 * kb][3]);
+    pa[2] = pack_bf16x2(sacc[2 * kb + 1][0], sacc[2 * kb + 1][1]);
+    pa[3] = pack_bf16x2(sacc[2 * kb + 1][2], sacc[2 * kb + 1][3]);
+    const int key = (j0 / 2 + kb) * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int np = 0; np < 4; ++np) {
+      const int ch = 2 * np + (lane >> 4);
+      uint32_t vb[4];
+      ldsm_x4_t(sV + key * 128 + ((ch ^ (key & 7)) << 4), vb);
+      mma_bf16_16816(o[2 * np], pa, vb[0], vb[1]);
+      mma_bf16_16816(o[2 * np + 1], pa, vb[2], vb[3]);
+    }
+  }
+}
+
 template <int SCORE>
-__global__ void __launch_bounds__(128, 2) attn_bf16_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int u = blockIdx.x / a.splits, s = blockIdx.x % a.splits, h = blockIdx.y;
   int64_t k0;
@@ -100,249 +213,154 @@ __global__ void __launch_bounds__(128, 2) attn_bf16_kernel(AttnArgs a) {
   if (m <= 0) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tq = lane & 3;
+  const int team = warp >> 1, mem = warp & 1, tt = mem * 32 + lane;
   const int d = a.d;
   const int64_t ld = 2 * int64_t(d);
   const int hcol = h * DH;
   const bf16* KV = reinterpret_cast<const bf16*>(a.KV);
-  uint8_t* wbuf = smem + warp * WARP_BYTES;
+  uint8_t* tbuf = smem + team * TEAM_BYTES;
   const float qscale = (SCORE == 0 ? LOG2E : 1.0f) * rsqrtf(float(DH));
   const int n_tiles = (nk + KT - 1) / KT;
 
   for (int qp = 0; qp < m; qp += 32) {
     const int mq = min(32, m - qp);
-    const int groups = mq > 16 ? 2 : 1;
+    const bool ksplit = mq <= 16;           // the warps of a team split keys, else queries
+    const int qr0 = ksplit ? 0 : 16 * mem;  // this warp's first query row in the chunk
     // ---- query fragments (A operand), scaled, bf16
-    uint32_t qa[2][4][4];
+    uint32_t qa[4][4];
 #pragma unroll
-    for (int gi = 0; gi < 2; ++gi)
+    for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int row = gi * 16 + g + ((e & 1) ? 8 : 0);
-          const int col = kk * 16 + 2 * tq + ((e & 2) ? 8 : 0);
-          float x0 = 0.f, x1 = 0.f;
-          if (row < mq) {
-            const float* qrow = a.Q + int64_t(t0 + qp + row) * d + hcol + col;
-            x0 = qrow[0] * qscale;
-            x1 = qrow[1] * qscale;
-          }
-          qa[gi][kk][e] = pack_bf16x2(x0, x1);
+      for (int e = 0; e < 4; ++e) {
+        const int row = qr0 + g + ((e & 1) ? 8 : 0);
+        const int col = kk * 16 + 2 * tq + ((e & 2) ? 8 : 0);
+        float x0 = 0.f, x1 = 0.f;
+        if (row < mq) {
+          const float* qrow = a.Q + int64_t(t0 + qp + row) * d + hcol + col;
+          x0 = qrow[0] * qscale;
+          x1 = qrow[1] * qscale;
         }
-    float o[2][8][4];
-    float mrow[2][2], lrow[2][2];
+        qa[kk][e] = pack_bf16x2(x0, x1);
+      }
+    float o[8][4];
 #pragma unroll
-    for (int gi = 0; gi < 2; ++gi) {
+    for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[gi][nt][e] = 0.f;
-      mrow[gi][0] = mrow[gi][1] = -INFINITY;
-      lrow[gi][0] = lrow[gi][1] = 0.f;
-    }
+      for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+    float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
 
-    // ---- stream this warp's tiles: warp w takes tiles w, w+4, ...; KV_STAGES - 1 tiles
-    // are in flight while one is computed, and the row indices run one tile further ahead
+    // ---- stream the team's tiles: KV_STAGES - 1 in flight while one is computed; the
+    // row indices run one tile further ahead
     int stage = 0;
-    int tile = warp;
-    int rows[8];
+    int tile = team;
+    int rows[4];
     auto fetch_rows = [&](int tl) {
-      if (tl < n_tiles) tile_rows(rows, a.kv_rows, k0 + int64_t(tl) * KT, min(KT, nk - tl * KT), lane);
+      if (tl < n_tiles) tile_rows(rows, a.kv_rows, k0 + int64_t(tl) * KT, min(KT, nk - tl * KT), tt);
     };
     fetch_rows(tile);
 #pragma unroll
     for (int p = 0; p < KV_STAGES - 1; ++p) {
-      const int tl = tile + 4 * p;
-      if (tl < n_tiles) load_kv_tile(wbuf + p * WARP_STAGE, KV, ld, rows, hcol, d, lane);
+      const int tl = tile + TEAMS * p;
+      if (tl < n_tiles) load_kv_tile(tbuf + p * TEAM_STAGE, KV, ld, rows, hcol, d, tt);
       cp_async_commit();
-      fetch_rows(tl + 4);
+      fetch_rows(tl + TEAMS);
     }
-    for (; tile < n_tiles; tile += 4) {
-      const int ahead = tile + 4 * (KV_STAGES - 1);
+    for (; tile < n_tiles; tile += TEAMS) {
+      cp_async_wait<KV_STAGES - 2>();
+      // this thread's copies of the tile have landed; after the barrier the team's have,
+      // and both warps are done with the stage that is refilled next
+      team_sync(team);
+      const int ahead = tile + TEAMS * (KV_STAGES - 1);
       if (ahead < n_tiles) {
         const int st = stage + KV_STAGES - 1;
-        load_kv_tile(wbuf + (st >= KV_STAGES ? st - KV_STAGES : st) * WARP_STAGE, KV, ld, rows, hcol, d, lane);
-        fetch_rows(ahead + 4);
+        load_kv_tile(tbuf + (st >= KV_STAGES ? st - KV_STAGES : st) * TEAM_STAGE, KV, ld, rows, hcol, d, tt);
+        fetch_rows(ahead + TEAMS);
       }
       cp_async_commit();
-      cp_async_wait<KV_STAGES - 1>();
-      __syncwarp();
-      const uint32_t sK = smem_u32(wbuf + stage * WARP_STAGE);
+      const uint32_t sK = smem_u32(tbuf + stage * TEAM_STAGE);
       const uint32_t sV = sK + TILE_BYTES;
       const int valid = min(KT, nk - tile * KT);
-
-      // S = Q K^T for 32 keys (4 n-tiles of 8)
-      float sacc[2][4][4];
-#pragma unroll
-      for (int gi = 0; gi < 2; ++gi)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) sacc[gi][j][e] = 0.f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-          const int key = j * 8 + (lane & 7);
-          const int ch = 4 * p + (lane >> 3);
-          uint32_t kb[4];
-          ldsm_x4(sK + key * 128 + ((ch ^ (key & 7)) << 4), kb);
-          mma_bf16_16816(sacc[0][j], qa[0][2 * p], kb[0], kb[1]);
-          mma_bf16_16816(sacc[0][j], qa[0][2 * p + 1], kb[2], kb[3]);
-          if (groups > 1) {
-            mma_bf16_16816(sacc[1][j], qa[1][2 * p], kb[0], kb[1]);
-            mma_bf16_16816(sacc[1][j], qa[1][2 * p + 1], kb[2], kb[3]);
-          }
-        }
-      }
-      // mask keys past the slice end (last tile only), then scores -> weights
-      if (valid < KT) {
-#pragma unroll
-        for (int gi = 0; gi < 2; ++gi)
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int kidx = j * 8 + 2 * tq + (e & 1);
-              if (kidx >= valid) sacc[gi][j][e] = (SCORE == 0) ? -INFINITY : 0.f;
-            }
-      }
-#pragma unroll
-      for (int gi = 0; gi < 2; ++gi) {
-        if (SCORE == 0) {
-#pragma unroll
-          for (int hr = 0; hr < 2; ++hr) {
-            float mx = -INFINITY;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) mx = fmaxf(mx, fmaxf(sacc[gi][j][2 * hr], sacc[gi][j][2 * hr + 1]));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            // The reference point of a row moves only when a score exceeds it by more than
-            // RESCALE_SLACK (log2 units): weights 2^(s - m) then stay <= 2^RESCALE_SLACK, exact
-            // in fp32, and the accumulators are rescaled rarely (the warp skips it when no row
-            // of it moves).  Numerator and denominator share m, so the quotient is unchanged.
-            const bool move = mx > mrow[gi][hr] + RESCALE_SLACK;
-            if (__any_sync(0xffffffffu, move)) {
-              const float mnew = move ? mx : mrow[gi][hr];
-              const float corr = (mnew == mrow[gi][hr]) ? 1.f : exp2f(mrow[gi][hr] - mnew);
-              mrow[gi][hr] = mnew;
-              lrow[gi][hr] *= corr;
-#pragma unroll
-              for (int nt = 0; nt < 8; ++nt) {
-                o[gi][nt][2 * hr] *= corr;
-                o[gi][nt][2 * hr + 1] *= corr;
-              }
-            }
-            const float muse = (mrow[gi][hr] == -INFINITY) ? 0.f : mrow[gi][hr];
-            float sum = 0.f;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float p0 = exp2f(sacc[gi][j][2 * hr] - muse);
-              const float p1 = exp2f(sacc[gi][j][2 * hr + 1] - muse);
-              sacc[gi][j][2 * hr] = p0;
-              sacc[gi][j][2 * hr + 1] = p1;
-              sum += p0 + p1;
-            }
-            lrow[gi][hr] += sum;
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) sacc[gi][j][e] = fmaxf(sacc[gi][j][e], 0.f);
-        }
-      }
-      // O += P V   (P as A fragments straight from the score accumulators)
-#pragma unroll
-      for (int kb = 0; kb < 2; ++kb) {
-        uint32_t pa[2][4];
-#pragma unroll
-        for (int gi = 0; gi < 2; ++gi) {
-          pa[gi][0] = pack_bf16x2(sacc[gi][2 * kb][0], sacc[gi][2 * kb][1]);
-          pa[gi][1] = pack_bf16x2(sacc[gi][2 * kb][2], sacc[gi][2 * kb][3]);
-          pa[gi][2] = pack_bf16x2(sacc[gi][2 * kb + 1][0], sacc[gi][2 * kb + 1][1]);
-          pa[gi][3] = pack_bf16x2(sacc[gi][2 * kb + 1][2], sacc[gi][2 * kb + 1][3]);
-        }
-#pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          const int key = kb * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-          const int ch = 2 * np + (lane >> 4);
-          uint32_t vb[4];
-          ldsm_x4_t(sV + key * 128 + ((ch ^ (key & 7)) << 4), vb);
-          mma_bf16_16816(o[0][2 * np], pa[0], vb[0], vb[1]);
-          mma_bf16_16816(o[0][2 * np + 1], pa[0], vb[2], vb[3]);
-          if (groups > 1) {
-            mma_bf16_16816(o[1][2 * np], pa[1], vb[0], vb[1]);
-            mma_bf16_16816(o[1][2 * np + 1], pa[1], vb[2], vb[3]);
-          }
-        }
-      }
-      __syncwarp();
+      if (ksplit) tile_step<SCORE, 2>(sK, sV, 2 * mem, qa, o, mrow, lrow, valid, lane);
+      else tile_step<SCORE, 4>(sK, sV, 0, qa, o, mrow, lrow, valid, lane);
       stage = stage + 1 == KV_STAGES ? 0 : stage + 1;
     }
     cp_async_wait_all();
 
-    // ---- combine the four warps' states through shared memory
+    // ---- combine the warps' states through shared memory
     if (SCORE == 0) {
 #pragma unroll
-      for (int gi = 0; gi < 2; ++gi)
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          lrow[gi][hr] += __shfl_xor_sync(0xffffffffu, lrow[gi][hr], 1);
-          lrow[gi][hr] += __shfl_xor_sync(0xffffffffu, lrow[gi][hr], 2);
-        }
+      for (int hr = 0; hr < 2; ++hr) {
+        lrow[hr] += __shfl_xor_sync(0xffffffffu, lrow[hr], 1);
+        lrow[hr] += __shfl_xor_sync(0xffffffffu, lrow[hr], 2);
+      }
     }
     __syncthreads();
-    float* comb = reinterpret_cast<float*>(smem);        // [4 warps][32 rows][64]
-    float* cm = comb + 4 * 32 * DH;                        // [4][32]
-    float* cl = cm + 4 * 32;                               // [4][32]
+    float* comb = reinterpret_cast<float*>(smem);  // [8 warps][16 rows][64]
+    float* cm = comb + 8 * 16 * DH;                // [8][16]
+    float* cl = cm + 8 * 16;                       // [8][16]
 #pragma unroll
-    for (int gi = 0; gi < 2; ++gi)
+    for (int hr = 0; hr < 2; ++hr) {
+      const int r = g + 8 * hr;
+      float* dst = comb + (warp * 16 + r) * DH;
 #pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        const int row = gi * 16 + g + hr * 8;
-        float* dst = comb + (warp * 32 + row) * DH;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          dst[nt * 8 + 2 * tq] = o[gi][nt][2 * hr];
-          dst[nt * 8 + 2 * tq + 1] = o[gi][nt][2 * hr + 1];
-        }
-        if (tq == 0) {
-          cm[warp * 32 + row] = mrow[gi][hr];
-          cl[warp * 32 + row] = lrow[gi][hr];
-        }
+      for (int nt = 0; nt < 8; ++nt) {
+        dst[nt * 8 + 2 * tq] = o[nt][2 * hr];
+        dst[nt * 8 + 2 * tq + 1] = o[nt][2 * hr + 1];
       }
+      if (tq == 0) {
+        cm[warp * 16 + r] = mrow[hr];
+        cl[warp * 16 + r] = lrow[hr];
+      }
+    }
     __syncthreads();
     {
-      const int row = threadIdx.x >> 2, seg = threadIdx.x & 3;
+      // 32 rows x 8 segments of 8 dims; a row's states sit in all 8 warps (key split) or in
+      // the 4 warps w with w % 2 == row / 16 (query split)
+      const int row = threadIdx.x >> 3, seg = threadIdx.x & 7;
       if (row < mq) {
         const int t = t0 + qp + row;
-        float wgt[4];
+        const int nsrc = ksplit ? 8 : 4;
+        const int lr = ksplit ? row : (row & 15);
+        float wgt[8];
         float M = -INFINITY, Lsum = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int w = ksplit ? i : (row >> 4) + 2 * i;
+          wgt[i] = 0.f;
+          if (i < nsrc) {
+            if (SCORE == 0) M = fmaxf(M, cm[w * 16 + lr]);
+            else wgt[i] = 1.f;
+          }
+        }
         if (SCORE == 0) {
 #pragma unroll
-          for (int w = 0; w < 4; ++w) M = fmaxf(M, cm[w * 32 + row]);
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const float mw = cm[w * 32 + row];
-            wgt[w] = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-            Lsum += wgt[w] * cl[w * 32 + row];
+          for (int i = 0; i < 8; ++i) {
+            const int w = ksplit ? i : (row >> 4) + 2 * i;
+            if (i < nsrc) {
+              const float mw = cm[w * 16 + lr];
+              wgt[i] = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+              Lsum += wgt[i] * cl[w * 16 + lr];
+            }
           }
-        } else {
-#pragma unroll
-          for (int w = 0; w < 4; ++w) wgt[w] = 1.f;
         }
         // one slice: the state is final, so write the normalised output (no merge pass)
         const bool direct = a.splits == 1;
         const float scale = (SCORE == 0 && direct) ? (Lsum > 0.f ? 1.f / Lsum : 0.f) : 1.f;
-        float* pacc = (direct ? a.out + int64_t(t) * d : a.part_acc + (int64_t(s) * a.T + t) * d) + hcol + seg * 16;
+        float v[8];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          float v = 0.f;
+        for (int c = 0; c < 8; ++c) v[c] = 0.f;
 #pragma unroll
-          for (int w = 0; w < 4; ++w) v += wgt[w] * comb[(w * 32 + row) * DH + seg * 16 + c];
-          pacc[c] = v * scale;
+        for (int i = 0; i < 8; ++i) {
+          if (i < nsrc) {
+            const int w = ksplit ? i : (row >> 4) + 2 * i;
+            const float* srcp = comb + (w * 16 + lr) * DH + seg * 8;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) v[c] += wgt[i] * srcp[c];
+          }
         }
+        float* pacc = (direct ? a.out + int64_t(t) * d : a.part_acc + (int64_t(s) * a.T + t) * d) + hcol + seg * 8;
+        reinterpret_cast<float4*>(pacc)[0] = make_float4(v[0] * scale, v[1] * scale, v[2] * scale, v[3] * scale);
+        reinterpret_cast<float4*>(pacc)[1] = make_float4(v[4] * scale, v[5] * scale, v[6] * scale, v[7] * scale);
         if (SCORE == 0 && seg == 0 && !direct) {
           float* pml = a.part_ml + ((int64_t(s) * a.T + t) * a.H + h) * 2;
           pml[0] = M;
@@ -498,10 +516,10 @@ int attention_bf16(const AttnArgs& a, cudaStream_t s) {
   dim3 grid(a.B * a.splits, a.H);
   if (a.score == 0) {
     cudaFuncSetAttribute(attn_bf16_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_SMEM);
-    attn_bf16_kernel<0><<<grid, 128, ATTN_SMEM, s>>>(a); note_launch();
+    attn_bf16_kernel<0><<<grid, ATT_THREADS, ATTN_SMEM, s>>>(a); note_launch();
   } else {
     cudaFuncSetAttribute(attn_bf16_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_SMEM);
-    attn_bf16_kernel<1><<<grid, 128, ATTN_SMEM, s>>>(a); note_launch();
+    attn_bf16_kernel<1><<<grid, ATT_THREADS, ATTN_SMEM, s>>>(a); note_launch();
   }
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
