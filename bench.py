@@ -104,6 +104,9 @@ def config_block(wl, world):
     common = {"users_per_gpu": users, "global_batch_users": users * world, "n_items": c["n_items"], "d": c["d"],
               "history_tokens_per_step": n_tok * world,
               "parallelism": f"replicas x{world} (users sharded, no collective on the data path)"}
+    if c["dtype"] == "bf16" and c["kind"] != "pointwise":
+        common["weights"] = "random-init, converted to the tensor-core operand layout once before timing " \
+                            "(stca_pin_weights, as at model load)"
     if c["kind"] == "stca":
         L = int(wl["lengths"].max())
         lengths = f"L={L}" if int(wl["lengths"].min()) == L else f"ragged L (mean {n_tok / users:.0f})"
@@ -193,22 +196,39 @@ def clocks_rejected(clk):
 # ------------------------------------------------------------------------------ roofline
 
 
-def distinct_rows(ids, dt):
-    """Distinct (item id, time bucket) keys among a pass's history tokens."""
+def _row_keys(ids, dt):
     import numpy as np
     key = ids.astype(np.int64) * 16
     if dt is not None:
         v = dt.astype(np.int64) + 1
         key += np.minimum(15, np.floor(np.log2(v)).astype(np.int64))
-    return int(len(np.unique(key)))
+    return key
+
+
+def distinct_rows(ids, dt):
+    """Distinct (item id, time bucket) keys among a pass's history tokens."""
+    import numpy as np
+    return int(len(np.unique(_row_keys(ids, dt))))
+
+
+def user_distinct_rows(ids, dt, lengths):
+    """Sum over users of each user's distinct keys (the keys compacted attention reads);
+    a user of 16384 or more tokens keeps every token."""
+    import numpy as np
+    lengths = np.asarray(lengths, np.int64)
+    user = np.repeat(np.arange(len(lengths), dtype=np.int64), lengths)
+    long_user = np.repeat(lengths >= 16384, lengths)
+    key = np.where(long_user, np.arange(len(user), dtype=np.int64), _row_keys(ids, dt))
+    return int(len(np.unique(user * (1 << 40) + key)))
 
 
 _PASSES = {}
 
 
 def gemm_passes(wl, dedup):
-    """(rows computed by the history GEMMs, history tokens, users, targets) per pass."""
-    key = (id(wl), bool(dedup))
+    """(rows computed by the history GEMMs, history tokens, users, targets, keys attention
+    reads) per pass."""
+    key = (id(wl), int(dedup))
     if key not in _PASSES:
         _PASSES[key] = _gemm_passes(wl, dedup)
     return _PASSES[key]
@@ -219,12 +239,14 @@ def _gemm_passes(wl, dedup):
     if c["kind"] == "stca":
         n = int(wl["lengths"].sum())
         rows = distinct_rows(wl["ids"], wl["dt"]) if dedup else n
-        return [(rows, n, len(wl["lengths"]), int(wl["targets_per_user"].sum()))] * c["M"]
+        keys = user_distinct_rows(wl["ids"], wl["dt"], wl["lengths"]) if dedup == 2 else n
+        return [(rows, n, len(wl["lengths"]), int(wl["targets_per_user"].sum()), keys)] * c["M"]
     nq, Bu = c["n_query"], len(wl["lengths"][0])
     out = []
     for s in (0, 1):
         n = int(wl["lengths"][s].sum())
-        out.append((distinct_rows(wl["ids"][s], None) if dedup else n, n, Bu, Bu * nq))
+        keys = user_distinct_rows(wl["ids"][s], None, wl["lengths"][s]) if dedup == 2 else n
+        out.append((distinct_rows(wl["ids"][s], None) if dedup else n, n, Bu, Bu * nq, keys))
     return out * c["blocks"]
 
 
@@ -243,17 +265,18 @@ def stage_work(stage, wl, dedup=False):
     h, H = c["hidden"], c["H"]
     passes = gemm_passes(wl, dedup)
     if stage == "gather_ffn":
-        return "tensor", sum(2.0 * r * d * 2 * h for r, _, _, _ in passes), "flop"
+        return "tensor", sum(2.0 * p[0] * d * 2 * h for p in passes), "flop"
     if stage == "ffn_out":
-        return "tensor", sum(2.0 * r * h * d for r, _, _, _ in passes), "flop"
+        return "tensor", sum(2.0 * p[0] * h * d for p in passes), "flop"
     if stage == "kv":
-        return "tensor", sum(2.0 * r * d * 2 * d for r, _, _, _ in passes), "flop"
+        return "tensor", sum(2.0 * p[0] * d * 2 * d for p in passes), "flop"
     if stage == "attention":
         tot = 0.0
-        for _, n, Bu, T in passes:
-            # one K and one V row (bf16) read per history token, the fp32 queries read and
-            # outputs written (partial states of L-slices are overhead, not counted)
-            tot += n * 2 * d * 2 + 2 * T * d * 4
+        for _, _, _, T, keys in passes:
+            # one K and one V row (bf16) read per key attended (each token, or each distinct
+            # key of a user when compacted), the fp32 queries read and outputs written
+            # (partial states of L-slices are overhead, not counted)
+            tot += keys * 2 * d * 2 + 2 * T * d * 4
         return "hbm", tot, "byte"
     return None, None, None
 
@@ -294,9 +317,9 @@ def run_ours(args):
     kind = wl["cfg"]["kind"]
     n_tok = history_tokens(wl)
     stream = torch.cuda.current_stream()
-    dedup = kind != "pointwise" and wl["cfg"]["dtype"] == "bf16" and not args.no_dedup
+    dedup = 2 if (kind != "pointwise" and wl["cfg"]["dtype"] == "bf16" and not args.no_dedup) else 0
     if kind == "stca":
-        model = StcaModel(wl, dedup=int(dedup))
+        model = StcaModel(wl, dedup=dedup)
         x = model.inputs(wl)
         out = torch.empty((x["t_tot"], wl["cfg"]["d"]), device="cuda")
     elif kind == "pointwise":
@@ -307,6 +330,9 @@ def run_ours(args):
         model = HyformerModel(wl, dedup=dedup)
         x = model.inputs(wl)
         out = torch.empty((x["B"], 2 * x["n_query"], wl["cfg"]["d"]), device="cuda")
+
+    if kind != "pointwise" and wl["cfg"]["dtype"] == "bf16":
+        model.pin()  # weights converted to the tensor-core layout once, as at model load
 
     def step(handle=None):
         if handle is None:
@@ -416,12 +442,14 @@ def run_ours(args):
         barrier()
         ms0 = max_over_ranks(e0.elapsed_time(e1))
         B.stca_destroy(h0)
-        passes = gemm_passes(wl, True)
+        passes = gemm_passes(wl, dedup)
         per_token = {"value": round(total_tokens * args.steps / (ms0 / 1e3), 1), "unit": UNIT,
                      "ms_per_step": round(ms0 / args.steps, 3),
                      "distinct_rows_fraction": round(sum(p[0] for p in passes) / sum(p[1] for p in passes), 4),
-                     "note": "same step with the history GEMMs run once per token instead of once per distinct "
-                             "(id, time bucket) key; identical results"}
+                     "attended_keys_fraction": round(sum(p[4] for p in passes) / sum(p[1] for p in passes), 4),
+                     "note": "same step with the history GEMMs and the attention run once per token instead of "
+                             "once per distinct (id, time bucket) key of the call (GEMMs) and of each user "
+                             "(attention, weighted by token counts); the same function up to summation order"}
 
     # end to end through the host-buffer entry point: pinned inputs in, z out, per step
     e2e = None
@@ -464,6 +492,7 @@ def run_ours(args):
         "token_layers_per_s": round(value * layers, 1),
         "roofline": roofline, "stages": stages, "e2e": e2e, "cpu_baseline": cpu,
         "history_gemm_rows": "distinct (id, time bucket) keys per call" if dedup else "every history token",
+        "attention_keys": "distinct keys per user, weighted by token count" if dedup == 2 else "every history token",
         "per_token_path": per_token,
         "gpu_launches": int(launches), "gpu_launches_per_step": round(launches / args.steps, 1), "clocks": clk,
     }

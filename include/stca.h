@@ -66,7 +66,10 @@ enum stca_score { STCA_SOFTMAX = 0, STCA_RELU = 1 };
  * stca_create sizes all device workspace from them, and later calls allocate nothing.
  * dedup follows the HyFormer page §3.8.1 (GPU pooling: few ids of a long sequence are
  * distinct): X~, K and V of a history token depend only on its item id and time bucket,
- * so they are computed once per distinct key and every token reads its key's K/V row. */
+ * so they are computed once per distinct key and every token reads its key's K/V row.
+ * Tokens of one user with the same key also have equal scores, so a softmax (or ReLU)
+ * over them equals one over the user's distinct keys with each weight multiplied by the
+ * key's token count (dedup = 2). */
 typedef struct {
   int mode;         /* enum stca_mode */
   int M, d, H, hidden;
@@ -74,8 +77,10 @@ typedef struct {
   int score;        /* enum stca_score */
   int time_buckets; /* 0 or 16 */
   int max_users, max_tokens, max_targets;
-  int dedup;        /* 1: run the per-token history GEMMs once per distinct (id, time bucket)
-                       key of the call (STCA_BF16 only); results are unchanged */
+  int dedup;        /* STCA_BF16 only.  1: run the per-token history GEMMs once per distinct
+                       (id, time bucket) key of the call; results are bit-identical to 0.
+                       2: also attend once per distinct key of each user, weighting the key
+                       by the number of its tokens; the same result up to summation order */
   float ln_eps;     /* LayerNorm epsilon (biased variance) */
 } stca_config;
 
@@ -254,6 +259,22 @@ int stca_sync_status(stca_handle* h);
 
 /* Static description of a status code. */
 const char* stca_strerror(int code);
+
+/* Weight conversion done once (no counterpart on the pages: a load-time layout step, as a
+ * serving system prepares constant weights when it loads a model).  Every bf16 forward
+ * call converts the weights it is given into the tensor cores' K-major operand layout in
+ * handle workspace.  stca_pin_weights does that now, on `stream`, for `weights` (a
+ * `const stca_weights*` for STCA handles, a `const hyf_weights*` for HyFormer handles; for
+ * the latter also the per-token FFNs of every query token slot whose three matrices are
+ * set, up to max_targets / max_users tokens) and records the struct's address and
+ * contents: later calls given the same struct skip the conversion.  Between pin and
+ * unpin (or destroy) the weight arrays must not change.  Pinning other weights replaces
+ * the pin.  Errors: STCA_ERR_INVALID_ARG (null or incomplete weights, pointwise handle),
+ * STCA_ERR_UNSUPPORTED (fp32 handle), STCA_ERR_CUDA. */
+int stca_pin_weights(stca_handle* h, const void* weights, void* stream);
+
+/* Forgets the pin; later calls convert the weights they are given again. */
+void stca_unpin_weights(stca_handle* h);
 
 /* Frees the handle's device memory.  NULL is a no-op. */
 void stca_destroy(stca_handle* h);

@@ -79,6 +79,16 @@ size_t stca_k_dedup_workspace_bytes(int n);
 int stca_k_dedup(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws_bytes, int32_t* uniq_idx,
                  int32_t* uniq_token, int32_t* count, int32_t* err, void* stream);
 
+/* Per-user compaction of K/V rows (keys of one user with the same row have equal scores, so
+ * attention may weigh one entry by the number of its tokens).  User u owns tokens
+ * hoff[u] .. hoff[u+1]-1 ([B+1] device offsets) with K/V rows rows[n]; on return
+ * out_rows[hoff[u] + i] (i < out_len[u]) are the user's distinct rows in order of first
+ * token and out_mult[hoff[u] + i] their token counts.  A user with 16384 or more tokens
+ * keeps one entry per token (count 1).  out_rows / out_mult: [hoff[B]] int32, out_len: [B]
+ * int32, device memory, not aliasing the inputs. */
+int stca_k_compact_user_rows(const int32_t* hoff, int B, const int32_t* rows, int32_t* out_rows, int32_t* out_mult,
+                             int32_t* out_len, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -70,6 +70,8 @@ _LIB = None
 _SIGS = [
     ("stca_create", _i32, [ctypes.POINTER(StcaConfig), ctypes.POINTER(_vp)]),
     ("stca_destroy", None, [_vp]),
+    ("stca_pin_weights", _i32, [_vp, _vp, _vp]),
+    ("stca_unpin_weights", None, [_vp]),
     ("stca_forward", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.POINTER(StcaWeights), _vp, _vp,
                             _vp]),
     ("stca_forward_host", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.POINTER(StcaWeights), _vp,
@@ -94,6 +96,7 @@ _SIGS = [
                                 _vp]),
     ("stca_k_dedup_workspace_bytes", ctypes.c_size_t, [_i32]),
     ("stca_k_dedup", _i32, [_vp, _vp, _i32, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]),
+    ("stca_k_compact_user_rows", _i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp]),
 ]
 
 EXPORTED = [s[0] for s in _SIGS]
@@ -150,6 +153,15 @@ def stca_create(cfg: StcaConfig):
 
 def stca_destroy(h):
     lib().stca_destroy(h)
+
+
+def stca_pin_weights(h, weights, stream=None) -> int:
+    """weights: the StcaWeights / HyfWeights object later passed to the forward calls."""
+    return lib().stca_pin_weights(h, ctypes.byref(weights), stream_ptr(stream))
+
+
+def stca_unpin_weights(h):
+    lib().stca_unpin_weights(h)
 
 
 def stca_sync_status(h) -> int:
@@ -249,3 +261,8 @@ def stca_k_dedup_workspace_bytes(n) -> int:
 def stca_k_dedup(ids, dt, n, ws, uniq_idx, uniq_token, count, err, stream=None) -> int:
     return lib().stca_k_dedup(ptr(ids), ptr(dt), n, ptr(ws), ws.numel() * ws.element_size(), ptr(uniq_idx),
                               ptr(uniq_token), ptr(count), ptr(err), stream_ptr(stream))
+
+
+def stca_k_compact_user_rows(hoff, B, rows, out_rows, out_mult, out_len, stream=None) -> int:
+    return lib().stca_k_compact_user_rows(ptr(hoff), B, ptr(rows), ptr(out_rows), ptr(out_mult), ptr(out_len),
+                                          stream_ptr(stream))

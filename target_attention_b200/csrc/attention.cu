@@ -24,7 +24,7 @@ constexpr float RESCALE_SLACK = 8.f;  // log2 units a running max may lag the tr
 
 __device__ __forceinline__ void slice_bounds(const AttnArgs& a, int u, int s, int64_t& k0, int& nk, int& t0, int& m) {
   const int h0 = a.hoff[u], h1 = a.hoff[u + 1];
-  const int64_t L = h1 - h0;
+  const int64_t L = a.kv_len ? a.kv_len[u] : h1 - h0;
   k0 = h0 + (L * s) / a.splits;
   const int64_t k1 = h0 + (L * (s + 1)) / a.splits;
   nk = int(k1 - k0);
@@ -51,7 +51,12 @@ constexpr int KV_STAGES = 3;                  // tiles in flight per team
 constexpr int TEAMS = 4;
 constexpr int ATT_THREADS = 2 * 32 * TEAMS;   // 256
 constexpr int TEAM_BYTES = KV_STAGES * TEAM_STAGE;   // 24 KB
-constexpr int ATTN_SMEM = TEAMS * TEAM_BYTES;        // 96 KB per CTA, two CTAs per SM
+constexpr int RING_BYTES = TEAMS * TEAM_BYTES;       // 96 KB
+// K/V row indices and key multiplicities of a team's tiles, copied two tiles ahead of the
+// K/V copies that need them: slots for the tile computed, the tiles in flight and the next
+constexpr int IDX_STAGES = KV_STAGES + 2;
+constexpr int IDX_BYTES = TEAMS * IDX_STAGES * 2 * KT * 4;
+constexpr int ATTN_SMEM = RING_BYTES + IDX_BYTES;    // two CTAs per SM
 
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -77,29 +82,32 @@ __device__ __forceinline__ void team_sync(int team) {
   asm volatile("bar.sync %0, 64;" ::"r"(team + 1) : "memory");
 }
 
-// Rows of the keys that thread tt (0..63) of a team copies in a 32-key tile: chunk tt % 8
-// of keys tt / 8 + 8 i, i = 0..3.  Resolved one tile ahead so that the copies of a tile
-// never wait for their row-index loads; -1 marks keys past the slice end.
-__device__ __forceinline__ void tile_rows(int (&rows)[4], const int32_t* kv_rows, int64_t row0, int valid, int tt) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int key = (tt >> 3) + 8 * i;
-    rows[i] = key < valid ? (kv_rows ? kv_rows[row0 + key] : int(row0 + key)) : -1;
-  }
+// Row-index side of a tile (compacted or distinct-row keys): thread tt of the team copies
+// entry tt % 32 of the tile's K/V rows (tt < 32) or multiplicities (tt >= 32) into the
+// tile's index slot; entries past the slice end read as 0 and are never used.
+__device__ __forceinline__ void copy_tile_index(int* slot, const int32_t* kv_rows, const int32_t* kv_mult,
+                                                int64_t row0, int valid, int tt) {
+  const int key = tt & 31;
+  const int32_t* src = tt < 32 ? kv_rows : kv_mult;
+  if (!src) return;
+  cp_async_4(slot + (tt >> 5) * KT + key, src + row0 + (key < valid ? key : 0), key < valid ? 4u : 0u);
 }
 
-// Issues this thread's cp.async copies of the K and V slices of head h for a tile
-// (128-byte key rows, 16-byte chunk c of key k at chunk c ^ (k % 8)).
-__device__ __forceinline__ void load_kv_tile(uint8_t* stage, const bf16* KV, int64_t ld, const int (&rows)[4],
-                                             int hcol, int d, int tt) {
+// Issues this thread's cp.async copies of the K and V slices of head h for a tile: chunk
+// tt % 8 of keys tt / 8 + 8 i, i = 0..3 (128-byte key rows, 16-byte chunk c of key k at
+// chunk c ^ (k % 8)).  Rows come from the tile's index slot, or are row0 + key; keys past
+// the slice end are zero-filled.
+__device__ __forceinline__ void load_kv_tile(uint8_t* stage, const int* slot, int64_t row0, int valid,
+                                             const bf16* KV, int64_t ld, int hcol, int d, int tt) {
   uint8_t* sK = stage;
   uint8_t* sV = stage + TILE_BYTES;
   const int ch = tt & 7;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int key = (tt >> 3) + 8 * i;
-    const bool ok = rows[i] >= 0;
-    const bf16* src = KV + (ok ? int64_t(rows[i]) * ld : 0) + hcol + ch * 8;
+    const bool ok = key < valid;
+    const int64_t row = ok ? (slot ? int64_t(slot[key]) : row0 + key) : 0;
+    const bf16* src = KV + row * ld + hcol + ch * 8;
     const int off = key * 128 + ((ch ^ (key & 7)) << 4);
     cp_async_16(sK + off, src, ok ? 16u : 0u);
     cp_async_16(sV + off, src + d, ok ? 16u : 0u);
@@ -110,9 +118,9 @@ __device__ __forceinline__ void load_kv_tile(uint8_t* stage, const bf16* KV, int
 // groups of 8 keys starting at group j0, then O += P V.  State per row half hr (rows g and
 // g + 8 of the warp's 16): running reference point mrow and sum lrow (softmax), O in o.
 template <int SCORE, int NJ>
-__device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, int j0, const uint32_t (&qa)[4][4],
-                                          float (&o)[8][4], float (&mrow)[2], float (&lrow)[2], int valid,
-                                          int lane) {
+__device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, const int* smul, int j0,
+                                          const uint32_t (&qa)[4][4], float (&o)[8][4], float (&mrow)[2],
+                                          float (&lrow)[2], int valid, int lane) {
   const int tq = lane & 3;
   // S = Q K^T
   float sacc[NJ][4];
@@ -169,8 +177,13 @@ __device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, int j0, cons
       float sum = 0.f;
 #pragma unroll
       for (int jj = 0; jj < NJ; ++jj) {
-        const float p0 = exp2f(sacc[jj][2 * hr] - muse);
-        const float p1 = exp2f(sacc[jj][2 * hr + 1] - muse);
+        float p0 = exp2f(sacc[jj][2 * hr] - muse);
+        float p1 = exp2f(sacc[jj][2 * hr + 1] - muse);
+        if (smul) {  // a compacted key weighs as many tokens as it stands for
+          const int2 c = *reinterpret_cast<const int2*>(smul + (j0 + jj) * 8 + 2 * tq);
+          p0 *= float(c.x);
+          p1 *= float(c.y);
+        }
         sacc[jj][2 * hr] = p0;
         sacc[jj][2 * hr + 1] = p1;
         sum += p0 + p1;
@@ -179,9 +192,17 @@ __device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, int j0, cons
     }
   } else {
 #pragma unroll
-    for (int jj = 0; jj < NJ; ++jj)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[jj][e] = fmaxf(sacc[jj][e], 0.f);
+    for (int jj = 0; jj < NJ; ++jj) {
+      float2 c = make_float2(1.f, 1.f);
+      if (smul) {
+        const int2 ci = *reinterpret_cast<const int2*>(smul + (j0 + jj) * 8 + 2 * tq);
+        c = make_float2(float(ci.x), float(ci.y));
+      }
+      sacc[jj][0] = fmaxf(sacc[jj][0], 0.f) * c.x;
+      sacc[jj][1] = fmaxf(sacc[jj][1], 0.f) * c.y;
+      sacc[jj][2] = fmaxf(sacc[jj][2], 0.f) * c.x;
+      sacc[jj][3] = fmaxf(sacc[jj][3], 0.f) * c.y;
+    }
   }
   // O += P V   (P as A fragments straight from the score accumulators)
 #pragma unroll
@@ -219,6 +240,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
   const int hcol = h * DH;
   const bf16* KV = reinterpret_cast<const bf16*>(a.KV);
   uint8_t* tbuf = smem + team * TEAM_BYTES;
+  int* tidx = a.kv_rows ? reinterpret_cast<int*>(smem + RING_BYTES) + team * IDX_STAGES * 2 * KT : nullptr;
   const float qscale = (SCORE == 0 ? LOG2E : 1.0f) * rsqrtf(float(DH));
   const int n_tiles = (nk + KT - 1) / KT;
 
@@ -249,39 +271,55 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
       for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
     float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
 
-    // ---- stream the team's tiles: KV_STAGES - 1 in flight while one is computed; the
-    // row indices run one tile further ahead
-    int stage = 0;
-    int tile = team;
-    int rows[4];
-    auto fetch_rows = [&](int tl) {
-      if (tl < n_tiles) tile_rows(rows, a.kv_rows, k0 + int64_t(tl) * KT, min(KT, nk - tl * KT), tt);
+    // ---- stream the team's tiles (local tile j is tile team + TEAMS j): the K/V of
+    // KV_STAGES - 1 tiles are in flight while one is computed, and the row indices (with
+    // multiplicities) of a tile are copied two tiles before its K/V
+    const int n_local = n_tiles > team ? (n_tiles - team + TEAMS - 1) / TEAMS : 0;
+    auto tile_of = [&](int j) { return team + TEAMS * j; };
+    auto idx_slot = [&](int j) { return tidx ? tidx + (j % IDX_STAGES) * 2 * KT : nullptr; };
+    auto copy_idx = [&](int j) {
+      if (tidx && j < n_local) {
+        const int tl = tile_of(j);
+        copy_tile_index(idx_slot(j), a.kv_rows, a.kv_mult, k0 + int64_t(tl) * KT, min(KT, nk - tl * KT), tt);
+      }
     };
-    fetch_rows(tile);
+    auto load_kv = [&](int j, int st) {
+      if (j < n_local) {
+        const int tl = tile_of(j);
+        load_kv_tile(tbuf + st * TEAM_STAGE, idx_slot(j), k0 + int64_t(tl) * KT, min(KT, nk - tl * KT), KV, ld,
+                     hcol, d, tt);
+      }
+    };
+    if (tidx) {
+      copy_idx(0);
+      copy_idx(1);
+      cp_async_commit();
+      cp_async_wait_all();
+      team_sync(team);
+    }
 #pragma unroll
     for (int p = 0; p < KV_STAGES - 1; ++p) {
-      const int tl = tile + TEAMS * p;
-      if (tl < n_tiles) load_kv_tile(tbuf + p * TEAM_STAGE, KV, ld, rows, hcol, d, tt);
+      load_kv(p, p);
+      copy_idx(p + KV_STAGES - 1);
       cp_async_commit();
-      fetch_rows(tl + TEAMS);
     }
-    for (; tile < n_tiles; tile += TEAMS) {
+    int stage = 0;
+    for (int j = 0; j < n_local; ++j) {
       cp_async_wait<KV_STAGES - 2>();
-      // this thread's copies of the tile have landed; after the barrier the team's have,
-      // and both warps are done with the stage that is refilled next
+      // this thread's copies of tile j (and the indices of tile j + KV_STAGES - 1) have
+      // landed; after the barrier the team's have, and both warps are done with tile j - 1
       team_sync(team);
-      const int ahead = tile + TEAMS * (KV_STAGES - 1);
-      if (ahead < n_tiles) {
-        const int st = stage + KV_STAGES - 1;
-        load_kv_tile(tbuf + (st >= KV_STAGES ? st - KV_STAGES : st) * TEAM_STAGE, KV, ld, rows, hcol, d, tt);
-        fetch_rows(ahead + TEAMS);
-      }
+      int st = stage + KV_STAGES - 1;
+      st = st >= KV_STAGES ? st - KV_STAGES : st;
+      load_kv(j + KV_STAGES - 1, st);
+      copy_idx(j + KV_STAGES + 1);
       cp_async_commit();
       const uint32_t sK = smem_u32(tbuf + stage * TEAM_STAGE);
       const uint32_t sV = sK + TILE_BYTES;
-      const int valid = min(KT, nk - tile * KT);
-      if (ksplit) tile_step<SCORE, 2>(sK, sV, 2 * mem, qa, o, mrow, lrow, valid, lane);
-      else tile_step<SCORE, 4>(sK, sV, 0, qa, o, mrow, lrow, valid, lane);
+      const int valid = min(KT, nk - tile_of(j) * KT);
+      const int* smul = a.kv_mult ? idx_slot(j) + KT : nullptr;
+      if (ksplit) tile_step<SCORE, 2>(sK, sV, smul, 2 * mem, qa, o, mrow, lrow, valid, lane);
+      else tile_step<SCORE, 4>(sK, sV, smul, 0, qa, o, mrow, lrow, valid, lane);
       stage = stage + 1 == KV_STAGES ? 0 : stage + 1;
     }
     cp_async_wait_all();

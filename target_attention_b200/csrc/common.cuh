@@ -129,6 +129,11 @@ __device__ __forceinline__ void cp_async_16(void* smem_dst, const void* gsrc, ui
                "r"(src_bytes)
                : "memory");
 }
+// 4-byte copy (through L1), zero-filled when src_bytes == 0.
+__device__ __forceinline__ void cp_async_4(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc), "r"(src_bytes)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {

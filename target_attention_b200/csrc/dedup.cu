@@ -157,7 +157,100 @@ __global__ void map_kernel(const int32_t* __restrict__ first, const int32_t* __r
   if (i < n) uniq_idx[i] = pos[first[slot_of[i]]];
 }
 
+// ---- per-user compaction: one CTA per user, open-addressing table in shared memory.
+// The user's tokens map to K/V rows; every distinct row of the user is kept once, in order
+// of its first token, with its number of tokens.  The list overwrites nothing: it is
+// written into the user's own token range [hoff[u], hoff[u] + len[u]).
+constexpr int CU_SLOTS = 16384;  // table slots (a user with more tokens keeps them all)
+constexpr size_t CU_SMEM = size_t(3) * CU_SLOTS * 4;
+
+__device__ __forceinline__ uint32_t mix32(uint32_t x) {
+  // the 32-bit finalizer of MurmurHash3 (Appleby)
+  x ^= x >> 16;
+  x *= 0x85ebca6bu;
+  x ^= x >> 13;
+  x *= 0xc2b2ae35u;
+  x ^= x >> 16;
+  return x;
+}
+
+__global__ void __launch_bounds__(SCAN_THREADS) compact_user_kernel(const int32_t* __restrict__ hoff,
+                                                                    const int32_t* __restrict__ rows,
+                                                                    int32_t* __restrict__ out_rows,
+                                                                    int32_t* __restrict__ out_mult,
+                                                                    int32_t* __restrict__ out_len) {
+  extern __shared__ int32_t cu_smem[];
+  const int u = blockIdx.x;
+  const int h0 = hoff[u], L = hoff[u + 1] - h0;
+  if (L >= CU_SLOTS) {  // too long for the table: every token is its own entry
+    for (int i = threadIdx.x; i < L; i += blockDim.x) {
+      out_rows[h0 + i] = rows[h0 + i];
+      out_mult[h0 + i] = 1;
+    }
+    if (threadIdx.x == 0) out_len[u] = L;
+    return;
+  }
+  int cap = 64;
+  while (cap < 2 * L && cap < CU_SLOTS) cap <<= 1;
+  const uint32_t mask = uint32_t(cap - 1);
+  int32_t* keys = cu_smem;
+  int32_t* first = keys + CU_SLOTS;
+  int32_t* cnt = first + CU_SLOTS;
+  for (int i = threadIdx.x; i < cap; i += blockDim.x) {
+    keys[i] = -1;
+    first[i] = 0x7fffffff;
+    cnt[i] = 0;
+  }
+  __syncthreads();
+  // insert (L < cap, so a free slot always exists)
+  for (int i = threadIdx.x; i < L; i += blockDim.x) {
+    const int32_t r = rows[h0 + i];
+    uint32_t slot = mix32(uint32_t(r)) & mask;
+    while (true) {
+      const int32_t prev = atomicCAS(&keys[slot], -1, r);
+      if (prev == -1 || prev == r) break;
+      slot = (slot + 1) & mask;
+    }
+    atomicMin(&first[slot], i);
+    atomicAdd(&cnt[slot], 1);
+  }
+  __syncthreads();
+  // first occurrences in token order, numbered by a block scan per chunk of tokens
+  int base = 0;
+  for (int c0 = 0; c0 < L; c0 += SCAN_THREADS) {
+    const int i = c0 + threadIdx.x;
+    int f = 0;
+    int32_t r = 0, m = 0;
+    if (i < L) {
+      r = rows[h0 + i];
+      uint32_t slot = mix32(uint32_t(r)) & mask;
+      while (keys[slot] != r) slot = (slot + 1) & mask;
+      f = first[slot] == i;
+      m = cnt[slot];
+    }
+    int excl;
+    const int total = block_exclusive_scan(f, excl);
+    if (f) {
+      out_rows[h0 + base + excl] = r;
+      out_mult[h0 + base + excl] = m;
+    }
+    base += total;
+  }
+  if (threadIdx.x == 0) out_len[u] = base;
+}
+
 }  // namespace
+
+int compact_user_rows(const int32_t* hoff, int B, const int32_t* rows, int32_t* out_rows, int32_t* out_mult,
+                      int32_t* out_len, cudaStream_t s) {
+  if (B <= 0) return STCA_OK;
+  if (cudaFuncSetAttribute(compact_user_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CU_SMEM)) !=
+      cudaSuccess)
+    return STCA_ERR_CUDA;
+  compact_user_kernel<<<B, SCAN_THREADS, CU_SMEM, s>>>(hoff, rows, out_rows, out_mult, out_len);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? STCA_OK : STCA_ERR_CUDA;
+}
 
 size_t dedup_table_slots(int max_tokens) {
   size_t cap = 1024;

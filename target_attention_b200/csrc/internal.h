@@ -123,6 +123,10 @@ struct AttnArgs {
   const int32_t* hoff;  // [B+1] history offsets
   const int32_t* toff;  // [B+1] target offsets
   const int32_t* kv_rows;  // K/V row of history token n (distinct-row form), or null: row n
+  // per-user compacted keys (with kv_rows): user u has kv_len[u] entries from hoff[u], entry
+  // n standing for kv_mult[n] tokens with the same K/V row; null: one entry per token
+  const int32_t* kv_len;
+  const int32_t* kv_mult;
   int B, T, d, H, splits;
   int score;            // 0 softmax, 1 relu
   float* part_acc;      // [splits, T, d]
@@ -157,6 +161,12 @@ size_t dedup_workspace_bytes(int max_tokens);
 // uniq_token[u] = one token with key u.  All on the stream.
 int dedup_rows(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws_bytes, int32_t* uniq_idx,
                int32_t* uniq_token, int32_t* count, int32_t* err, cudaStream_t s);
+// Per user u (tokens hoff[u] .. hoff[u+1]-1 with K/V rows rows[n]): the distinct rows of
+// the user in order of first token, out_rows[hoff[u] + i], with their token counts
+// out_mult[hoff[u] + i], i < out_len[u].  A user of 16384 or more tokens keeps one entry
+// per token (multiplicity 1).
+int compact_user_rows(const int32_t* hoff, int B, const int32_t* rows, int32_t* out_rows, int32_t* out_mult,
+                      int32_t* out_len, cudaStream_t s);
 
 // ---------------------------------------------------------------- pointwise ReLU TA
 

@@ -85,6 +85,8 @@ int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t*
   a.hoff = hoff;
   a.toff = toff;
   a.kv_rows = nullptr;
+  a.kv_len = nullptr;
+  a.kv_mult = nullptr;
   a.B = B;
   a.T = T;
   a.d = d;
@@ -108,6 +110,12 @@ int stca_k_dedup(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t 
   if (n < 0 || !count || (n > 0 && (!ids || !ws || !uniq_idx || !uniq_token))) return STCA_ERR_INVALID_ARG;
   return dedup_rows(ids, dt, n, ws, ws_bytes, uniq_idx, uniq_token, count, err,
                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int stca_k_compact_user_rows(const int32_t* hoff, int B, const int32_t* rows, int32_t* out_rows, int32_t* out_mult,
+                             int32_t* out_len, void* stream) {
+  if (B < 0 || (B > 0 && (!hoff || !rows || !out_rows || !out_mult || !out_len))) return STCA_ERR_INVALID_ARG;
+  return compact_user_rows(hoff, B, rows, out_rows, out_mult, out_len, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -33,8 +33,14 @@ struct stca_handle {
   // target-side weights packed K-major for the tensor cores (bf16 STCA), element offsets
   void* qpack = nullptr;
   struct QLayout {
+    // STCA
     size_t tgt13, tgt2, wq[STCA_MAX_LAYERS], wo[STCA_MAX_LAYERS], wc[STCA_MAX_LAYERS], fuse13[STCA_MAX_LAYERS],
-        fuse2[STCA_MAX_LAYERS], wz, z13, z2, total;
+        fuse2[STCA_MAX_LAYERS], wz, z13, z2;
+    // decode blocks: W_Q / W_O per block and sequence, the per-token FFNs of a block back to
+    // back (tok_cap tokens at most)
+    size_t hwq[2 * STCA_MAX_LAYERS], hwo[2 * STCA_MAX_LAYERS], htok13[STCA_MAX_LAYERS], htok2[STCA_MAX_LAYERS];
+    int tok_cap;
+    size_t total;
   } ql{};
   // query side
   float *cat = nullptr, *qbuf = nullptr, *qproj = nullptr, *attn = nullptr, *tmp_h = nullptr, *tmp_d = nullptr;
@@ -44,6 +50,13 @@ struct stca_handle {
   void* dedup_ws = nullptr;
   size_t dedup_ws_bytes = 0;
   int32_t *uniq_idx = nullptr, *uniq_token = nullptr, *uniq_count = nullptr;
+  // per-user compacted K/V rows with multiplicities (dedup = 2), per history sequence
+  int32_t *c_rows = nullptr, *c_mult = nullptr, *c_len = nullptr;
+  // weights converted once by stca_pin_weights (address, a copy of the struct, and the
+  // number of decode query tokens whose FFNs were converted)
+  const void* pinned = nullptr;
+  std::vector<uint8_t> pinned_copy;
+  int pinned_tokens = 0;
   // staging for the host-buffer entry point
   int32_t *in_ids = nullptr, *in_len = nullptr, *in_dt = nullptr, *in_tpu = nullptr;
   void* in_xt = nullptr;
@@ -165,7 +178,7 @@ int validate_config(const stca_config& c) {
   if (c.dtype != STCA_FP32 && c.dtype != STCA_BF16) return STCA_ERR_INVALID_ARG;
   if (c.score != STCA_SOFTMAX && c.score != STCA_RELU) return STCA_ERR_INVALID_ARG;
   if (c.time_buckets != 0 && c.time_buckets != 16) return STCA_ERR_UNSUPPORTED;
-  if (c.dedup != 0 && c.dedup != 1) return STCA_ERR_INVALID_ARG;
+  if (c.dedup < 0 || c.dedup > 2) return STCA_ERR_INVALID_ARG;
   if (c.mode == STCA_MODE_POINTWISE) {
     if (c.dtype != STCA_BF16 || c.d != 128 || c.dedup) return STCA_ERR_UNSUPPORTED;
     return STCA_OK;
@@ -215,6 +228,30 @@ stca_handle::QLayout q_layout(const stca_config& c) {
   return q;
 }
 
+stca_handle::QLayout hq_layout(const stca_config& c) {
+  stca_handle::QLayout q{};
+  const size_t d = size_t(c.d), hd = size_t(c.hidden);
+  // query tokens per user that the workspace was sized for (max_targets = users x tokens)
+  int cap = c.max_users > 0 ? c.max_targets / c.max_users : 0;
+  q.tok_cap = cap < STCA_MAX_QUERY_TOKENS ? cap : STCA_MAX_QUERY_TOKENS;
+  size_t at = 0;
+  auto take = [&](size_t n) {
+    const size_t o = at;
+    at += (n + 63) / 64 * 64;
+    return o;
+  };
+  for (int l = 0; l < c.M; ++l) {
+    for (int sq = 0; sq < 2; ++sq) {
+      q.hwq[2 * l + sq] = take(d * d);
+      q.hwo[2 * l + sq] = take(d * d);
+    }
+    q.htok13[l] = take(size_t(q.tok_cap) * 2 * hd * d);
+    q.htok2[l] = take(size_t(q.tok_cap) * d * hd);
+  }
+  q.total = at;
+  return q;
+}
+
 int allocate(stca_handle* h) {
   const stca_config& c = h->cfg;
   const size_t U = size_t(c.max_users) + 1, N = size_t(c.max_tokens), T = size_t(c.max_targets);
@@ -242,6 +279,9 @@ int allocate(stca_handle* h) {
     h->dedup_ws_bytes = dedup_workspace_bytes(c.max_tokens);
     ok = ok && dalloc(h, &h->dedup_ws, h->dedup_ws_bytes) && dalloc(h, &h->uniq_idx, nseq * N * 4) &&
          dalloc(h, &h->uniq_token, nseq * N * 4) && dalloc(h, &h->uniq_count, 16);
+    if (c.dedup == 2)
+      ok = ok && dalloc(h, &h->c_rows, nseq * N * 4) && dalloc(h, &h->c_mult, nseq * N * 4) &&
+           dalloc(h, &h->c_len, nseq * U * 4);
   }
   if (c.mode == STCA_MODE_STCA) {
     ok = ok && dalloc(h, &h->cat, T * (c.M + 1) * d * 4) && dalloc(h, &h->qbuf, T * d * 4);
@@ -255,6 +295,8 @@ int allocate(stca_handle* h) {
   } else {
     ok = ok && dalloc(h, &h->hoff2, U * 4) && dalloc(h, &h->hq, T * d * 4) && dalloc(h, &h->hqhat, T * d * 4) &&
          dalloc(h, &h->hmix, T * d * 4);
+    h->ql = hq_layout(c);
+    ok = ok && dalloc(h, &h->qpack, h->ql.total * 2);
   }
   return ok ? STCA_OK : STCA_ERR_CUDA;
 }
@@ -326,6 +368,12 @@ void ffn_jobs(const stca_ffn& f, int d, int hd, bf16* p13, bf16* p2, std::vector
   jobs.push_back({f.W2, p2, hd, d, 0, 0});
 }
 
+// True when `w` is the weight struct stca_pin_weights converted (same address and contents).
+bool is_pinned(const stca_handle* h, const void* w, size_t bytes) {
+  return h->pinned && h->pinned == w && h->pinned_copy.size() == bytes &&
+         memcmp(h->pinned_copy.data(), w, bytes) == 0;
+}
+
 // One history layer: the FFN, then W_K and W_V stacked into [2 d, d] (K rows, then V rows).
 void layer_jobs(stca_handle* h, size_t slot, const stca_ffn& f, const void* WK, const void* WV,
                 std::vector<PackJob>& jobs) {
@@ -355,6 +403,31 @@ void query_jobs(stca_handle* h, const stca_weights* w, std::vector<PackJob>& job
   }
   jobs.push_back({w->WZ, q + L.wz, (M + 1) * d, d, 0, 0});
   ffn_jobs(w->zffn, d, hd, q + L.z13, q + L.z2, jobs);
+}
+
+// Every tensor-core operand of a bf16 STCA call.
+void stca_jobs(stca_handle* h, const stca_weights* w, std::vector<PackJob>& jobs) {
+  for (int i = 0; i < h->cfg.M; ++i) layer_jobs(h, i, w->hist[i], w->WK[i], w->WV[i], jobs);
+  if (h->qpack) query_jobs(h, w, jobs);
+}
+
+// The decode blocks' operands: per block and sequence the history FFN, W_K|W_V, W_Q and
+// W_O; then the per-token FFNs of query tokens 0 .. tokens-1 of every block.
+void hyf_jobs(stca_handle* h, const hyf_weights* w, int tokens, std::vector<PackJob>& jobs) {
+  const int d = h->cfg.d, hd = h->cfg.hidden;
+  const stca_handle::QLayout& L = h->ql;
+  bf16* q = reinterpret_cast<bf16*>(h->qpack);
+  for (int l = 0; l < h->cfg.M; ++l)
+    for (int sq = 0; sq < 2; ++sq) {
+      const hyf_seq_weights& f = w->blk[l].seq[sq];
+      layer_jobs(h, size_t(l) * 2 + sq, f.ffn, f.WK, f.WV, jobs);
+      jobs.push_back({f.WQ, q + L.hwq[2 * l + sq], d, d, 0, 0});
+      jobs.push_back({f.WO, q + L.hwo[2 * l + sq], d, d, 0, 0});
+    }
+  for (int l = 0; l < h->cfg.M; ++l)
+    for (int t = 0; t < tokens; ++t)
+      ffn_jobs(w->blk[l].tok[t], d, hd, q + L.htok13[l] + size_t(t) * 2 * hd * d, q + L.htok2[l] + size_t(t) * d * hd,
+               jobs);
 }
 
 // K/V of every history token for one layer: bf16 tensor-core path.
@@ -409,13 +482,16 @@ int history_f32(stca_handle* h, const GatherSrc& g, int n_tok, const stca_ffn& f
 }
 
 int run_attention(stca_handle* h, const float* Q, const int32_t* hoff, const int32_t* toff, int B, int T,
-                  int splits, int score, cudaStream_t s, const int32_t* kv_rows) {
+                  int splits, int score, cudaStream_t s, const int32_t* kv_rows, const int32_t* kv_len = nullptr,
+                  const int32_t* kv_mult = nullptr) {
   AttnArgs a;
   a.Q = Q;
   a.KV = h->kv;
   a.hoff = hoff;
   a.toff = toff;
   a.kv_rows = kv_rows;
+  a.kv_len = kv_len;
+  a.kv_mult = kv_mult;
   a.B = B;
   a.T = T;
   a.d = h->cfg.d;
@@ -445,10 +521,9 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
     CK(exclusive_offsets(lens, B, h->hoff, n_tok, h->err, s));
     CK(exclusive_offsets(tpu, B, h->toff, t_tot, h->err, s));
     CK(copy_rows_to_f32(x_t, bf, t_tot, d, h->cat, ldcat, M * d, s));
-    if (bf) {
+    if (bf && !is_pinned(h, w, sizeof(*w))) {
       std::vector<PackJob> jobs;
-      for (int i = 0; i < M; ++i) layer_jobs(h, i, w->hist[i], w->WK[i], w->WV[i], jobs);
-      if (h->qpack) query_jobs(h, w, jobs);
+      stca_jobs(h, w, jobs);
       CK(tc_pack_weights(jobs.data(), int(jobs.size()), s));
     }
   }
@@ -473,7 +548,14 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
     g.rows = h->uniq_token;
     M_dev = h->uniq_count;
     kv_rows = h->uniq_idx;
+    if (c.dedup == 2) {
+      // attention over each user's distinct rows, each weighted by its token count
+      STAGE(h, STCA_STAGE_DEDUP, s, compact_user_rows(h->hoff, B, h->uniq_idx, h->c_rows, h->c_mult, h->c_len, s));
+      kv_rows = h->c_rows;
+    }
   }
+  const int32_t* kv_len = c.dedup == 2 ? h->c_len : nullptr;
+  const int32_t* kv_mult = c.dedup == 2 ? h->c_mult : nullptr;
   const int splits = attention_splits(n_tok, B, c.H, 1024);
   for (int i = 0; i < M; ++i) {
     if (bf)
@@ -482,7 +564,7 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
     else CK(history_f32(h, g, n_tok, w->hist[i], w->WK[i], w->WV[i], s));
     STAGE(h, STCA_STAGE_QUERY, s,
           qgemm(gemm_args<TB>(t_tot, d, d, h->qbuf, d, w->WQ[i], h->qproj, d, h->err), qp(h, L.wq[i]), s));
-    CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, splits, c.score, s, kv_rows));
+    CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, splits, c.score, s, kv_rows, kv_len, kv_mult));
     Prof p(h, STCA_STAGE_QUERY, s);
     CK(qgemm(gemm_args<TB>(t_tot, d, d, h->attn, d, w->WO[i], h->cat + int64_t(i) * d, ldcat, h->err),
              qp(h, L.wo[i]), s));
@@ -562,6 +644,53 @@ int stca_create(const stca_config* cfg, stca_handle** out) {
   }
   *out = h;
   return STCA_OK;
+}
+
+int stca_pin_weights(stca_handle* h, const void* weights, void* stream) {
+  if (!h || !weights || h->cfg.mode == STCA_MODE_POINTWISE) return STCA_ERR_INVALID_ARG;
+  if (h->cfg.dtype != STCA_BF16) return STCA_ERR_UNSUPPORTED;
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  h->pinned = nullptr;
+  h->pinned_copy.clear();
+  std::vector<PackJob> jobs;
+  size_t bytes = 0;
+  int tokens = 0;
+  if (h->cfg.mode == STCA_MODE_STCA) {
+    const stca_weights* w = static_cast<const stca_weights*>(weights);
+    CK(check_weights(h->cfg, w));
+    stca_jobs(h, w, jobs);
+    bytes = sizeof(*w);
+  } else {
+    const hyf_weights* w = static_cast<const hyf_weights*>(weights);
+    if (w->blocks != h->cfg.M) return STCA_ERR_INVALID_ARG;
+    for (int l = 0; l < h->cfg.M; ++l)
+      for (int sq = 0; sq < 2; ++sq) {
+        const hyf_seq_weights& f = w->blk[l].seq[sq];
+        if (!ffn_ok(f.ffn, false) || !f.WQ || !f.WK || !f.WV || !f.WO) return STCA_ERR_INVALID_ARG;
+      }
+    // the leading query-token slots whose FFNs are set in every block
+    while (tokens < h->ql.tok_cap) {
+      bool all = true;
+      for (int l = 0; l < h->cfg.M; ++l) all = all && ffn_ok(w->blk[l].tok[tokens], false);
+      if (!all) break;
+      ++tokens;
+    }
+    hyf_jobs(h, w, tokens, jobs);
+    bytes = sizeof(*w);
+  }
+  CK(tc_pack_weights(jobs.data(), int(jobs.size()), s));
+  h->pinned = weights;
+  h->pinned_copy.assign(static_cast<const uint8_t*>(weights), static_cast<const uint8_t*>(weights) + bytes);
+  h->pinned_tokens = tokens;
+  return STCA_OK;
+}
+
+void stca_unpin_weights(stca_handle* h) {
+  if (!h) return;
+  h->pinned = nullptr;
+  h->pinned_copy.clear();
+  h->pinned_tokens = 0;
 }
 
 void stca_destroy(stca_handle* h) {
@@ -662,19 +791,22 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
   h->last_stream = s;
   if (B == 0) return STCA_OK;
   const int rows = B * T, rows_s = B * n_query;
+  const stca_handle::QLayout& L = h->ql;
+  const bool pinned = is_pinned(h, w, sizeof(*w));
+  const bool tok_tc = pinned && T <= h->pinned_tokens;  // per-token FFNs converted at pin time
   {
     Prof p(h, STCA_STAGE_SETUP, s);
     CK(exclusive_offsets(len_feed, B, h->hoff, n_feed, h->err, s));
     CK(exclusive_offsets(len_search, B, h->hoff2, n_search, h->err, s));
     CK(fill_arange(h->toff, B + 1, n_query, s));
     CK(copy_rows_to_f32(q0, 1, rows, d, h->hq, d, 0, s));
-    std::vector<PackJob> jobs;
-    for (int l = 0; l < c.M; ++l)
-      for (int sq = 0; sq < 2; ++sq) {
-        const hyf_seq_weights& f = w->blk[l].seq[sq];
-        layer_jobs(h, size_t(l) * 2 + sq, f.ffn, f.WK, f.WV, jobs);
-      }
-    CK(tc_pack_weights(jobs.data(), int(jobs.size()), s));
+    if (!pinned) {
+      // per call only the per-sequence operands; the per-token FFNs then run on the generic
+      // kernels, which read the weights as given
+      std::vector<PackJob> jobs;
+      hyf_jobs(h, w, 0, jobs);
+      CK(tc_pack_weights(jobs.data(), int(jobs.size()), s));
+    }
   }
   const int32_t* ids[2] = {ids_feed, ids_search};
   const int32_t* offs[2] = {h->hoff, h->hoff2};
@@ -690,15 +822,27 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
       // H = SwiGLU(X_s) (eq 7), K/V = H W_K, H W_V (eq 8)
       const int32_t* M_dev = nullptr;
       const int32_t* kv_rows = nullptr;
+      const int32_t *kv_len = nullptr, *kv_mult = nullptr;
       if (c.dedup) {
         const size_t off = size_t(sq) * c.max_tokens;
-        if (l == 0)
+        const size_t uoff = size_t(sq) * (size_t(c.max_users) + 1);
+        if (l == 0) {
           STAGE(h, STCA_STAGE_DEDUP, s,
                 dedup_rows(ids[sq], nullptr, ntok[sq], h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx + off,
                            h->uniq_token + off, h->uniq_count + sq, h->err, s));
+          if (c.dedup == 2)
+            STAGE(h, STCA_STAGE_DEDUP, s,
+                  compact_user_rows(offs[sq], B, h->uniq_idx + off, h->c_rows + off, h->c_mult + off,
+                                    h->c_len + uoff, s));
+        }
         g.rows = h->uniq_token + off;
         M_dev = h->uniq_count + sq;
         kv_rows = h->uniq_idx + off;
+        if (c.dedup == 2) {
+          kv_rows = h->c_rows + off;
+          kv_len = h->c_len + uoff;
+          kv_mult = h->c_mult + off;
+        }
       }
       void* xs = h->xg ? static_cast<bf16*>(h->xg) + size_t(sq) * size_t(h->cfg.max_tokens) * d : nullptr;
       CK(history_bf16(h, size_t(l) * 2 + sq, g, ntok[sq], nullptr, nullptr, s, M_dev, l == 0 ? xs : nullptr,
@@ -708,14 +852,14 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
       qa.a_grp = n_query;
       qa.a_gstride = T;
       qa.a_goff = sq * n_query;
-      STAGE(h, STCA_STAGE_QUERY, s, simt_gemm(qa, s));
+      STAGE(h, STCA_STAGE_QUERY, s, qgemm(qa, qp(h, L.hwq[2 * l + sq]), s));
       CK(run_attention(h, h->qproj, offs[sq], h->toff, B, rows_s, attention_splits(ntok[sq], B, h->cfg.H, 1024),
-                       STCA_SOFTMAX, s, kv_rows));
+                       STCA_SOFTMAX, s, kv_rows, kv_len, kv_mult));
       auto oa = gemm_args<bf16>(rows_s, d, d, h->attn, d, f.WO, h->hqhat, d, h->err);
       oa.c_grp = n_query;
       oa.c_gstride = T;
       oa.c_goff = sq * n_query;
-      STAGE(h, STCA_STAGE_QUERY, s, simt_gemm(oa, s));
+      STAGE(h, STCA_STAGE_QUERY, s, qgemm(oa, qp(h, L.hwo[2 * l + sq]), s));
     }
     // query boosting: token mix (eq 11-13), per-token SwiGLU (eq 14), residual (eq 15)
     Prof p(h, STCA_STAGE_BOOST, s);
@@ -729,7 +873,7 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
       a1.B2z[t] = reinterpret_cast<const bf16*>(w->blk[l].tok[t].W3);
     }
     a1.B2 = a1.B2z[0];
-    CK(simt_gemm(a1, s));
+    CK(qgemm(a1, tok_tc ? qp(h, L.htok13[l]) : nullptr, s));
     float* dst = (l + 1 == c.M) ? out : h->hq;
     auto a2 = gemm_args<bf16>(B, d, hd, h->tmp_h, int64_t(T) * hd, nullptr, dst, int64_t(T) * d, h->err);
     a2.batch = T;
@@ -739,7 +883,7 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
     a2.ldr = int64_t(T) * d;
     a2.bsR = d;
     for (int t = 0; t < T; ++t) a2.Bz[t] = reinterpret_cast<const bf16*>(w->blk[l].tok[t].W2);
-    CK(simt_gemm(a2, s));
+    CK(qgemm(a2, tok_tc ? qp(h, L.htok2[l]) : nullptr, s));
   }
   return STCA_OK;
 }

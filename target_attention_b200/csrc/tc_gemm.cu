@@ -637,22 +637,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       if (!ok) fail(abort_flag, err);
       tc_fence_after();
       if (EPI == EPI_LN) {
-        float sum = 0.f;
+        // one pass for both moments, shifted by the row's first value c (a sample of the
+        // row, so |mean - c| is of the order of the spread and the shifted sums do not cancel)
+        float s1 = 0.f, s2 = 0.f, c0 = 0.f;
         if (ok) {
-#pragma unroll 1
-          for (int j = 0; j < HN / 32; ++j) {
+          {
             float v[32];
-            tmem_ld_32x32b_x32(tb + j * 32, v);
+            tmem_ld_32x32b_x32(tb - half * HN, v);
             tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) sum += v[e];
+            c0 = v[0];
           }
-        }
-        s_sum[half * 128 + r] = sum;
-        epilogue_sync();
-        const float mean = (s_sum[r] + s_sum[128 + r]) * (1.0f / N);
-        float sq = 0.f;
-        if (ok) {
 #pragma unroll 1
           for (int j = 0; j < HN / 32; ++j) {
             float v[32];
@@ -660,14 +654,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const float t = v[e] - mean;
-              sq = fmaf(t, t, sq);
+              const float dv = v[e] - c0;
+              s1 += dv;
+              s2 = fmaf(dv, dv, s2);
             }
           }
         }
-        s_sq[half * 128 + r] = sq;
+        s_sum[half * 128 + r] = s1;
+        s_sq[half * 128 + r] = s2;
         epilogue_sync();
-        const float rstd = rsqrtf((s_sq[r] + s_sq[128 + r]) * (1.0f / N) + eps);
+        const float m1 = (s_sum[r] + s_sum[128 + r]) * (1.0f / N);
+        const float mean = c0 + m1;
+        const float var = fmaxf((s_sq[r] + s_sq[128 + r]) * (1.0f / N) - m1 * m1, 0.f);
+        const float rstd = rsqrtf(var + eps);
         if (ok) {
 #pragma unroll 1
           for (int j = 0; j < HN / 32; ++j) {

@@ -48,7 +48,8 @@ class _Holder:
 
 class StcaModel(_Holder):
     """Weights of an STCA workload on the device plus a handle sized for it.  dedup
-    defaults to on for bf16 workloads (the history GEMMs run once per distinct key)."""
+    (stca_config.dedup) defaults to 2 for bf16 workloads: the history GEMMs run once per
+    distinct key of the call, attention once per distinct key of each user."""
 
     def __init__(self, wl, device="cuda", max_users=None, max_tokens=None, max_targets=None, dedup=None):
         super().__init__(device)
@@ -60,7 +61,7 @@ class StcaModel(_Holder):
             score=B.RELU if c["score"] == "relu" else B.SOFTMAX, time_buckets=c["time_buckets"],
             max_users=max_users or len(wl["lengths"]), max_tokens=max_tokens or int(wl["lengths"].sum()),
             max_targets=max_targets or int(wl["targets_per_user"].sum()),
-            dedup=int(c["dtype"] == "bf16" if dedup is None else dedup), ln_eps=c.get("ln_eps", 1e-5))
+            dedup=int((2 if c["dtype"] == "bf16" else 0) if dedup is None else dedup), ln_eps=c.get("ln_eps", 1e-5))
         w = wl["weights"]
         ws = B.StcaWeights()
         ws.table = self.p(wl["table"])
@@ -85,6 +86,10 @@ class StcaModel(_Holder):
         for k, v in changes.items():
             setattr(cfg, k, v)
         return B.stca_create(cfg)
+
+    def pin(self, stream=None):
+        """Convert the weights to the tensor-core layout once (stca_pin_weights)."""
+        B.check(B.stca_pin_weights(self.handle, self.weights, stream), "stca_pin_weights")
 
     def inputs(self, wl):
         d = {k: to_device(wl[k], self.device) for k in ("ids", "lengths", "dt", "x_t", "targets_per_user")}
@@ -138,7 +143,7 @@ class PointwiseModel(_Holder):
 
 
 class HyformerModel(_Holder):
-    def __init__(self, wl, device="cuda", max_users=None, max_tokens=None, dedup=True):
+    def __init__(self, wl, device="cuda", max_users=None, max_tokens=None, dedup=2):
         super().__init__(device)
         c = wl["cfg"]
         self.cfg = c
@@ -164,6 +169,10 @@ class HyformerModel(_Holder):
                 ws.blk[l].tok[t] = self.ffn(f, ln=False)
         self.weights = ws
         self.handle = B.stca_create(self.config)
+
+    def pin(self, stream=None):
+        """Convert the weights (per-token FFNs included) to the tensor-core layout once."""
+        B.check(B.stca_pin_weights(self.handle, self.weights, stream), "stca_pin_weights")
 
     def inputs(self, wl):
         return dict(ids_feed=to_device(wl["ids"][0], self.device), len_feed=to_device(wl["lengths"][0], self.device),

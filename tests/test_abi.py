@@ -66,7 +66,9 @@ def _cfg(**kw):
     (dict(mode=5), B.ERR_INVALID_ARG),
     (dict(dtype=B.FP32, d=96, H=2), B.ERR_UNSUPPORTED),   # d_h = 48
     (dict(dtype=B.FP32, d=64, H=2, dedup=1), B.ERR_UNSUPPORTED),
-    (dict(dedup=2), B.ERR_INVALID_ARG),
+    (dict(dtype=B.FP32, d=64, H=2, dedup=2), B.ERR_UNSUPPORTED),
+    (dict(dedup=3), B.ERR_INVALID_ARG),
+    (dict(dedup=-1), B.ERR_INVALID_ARG),
 ])
 def test_create_rejects_bad_configs(kw, code):
     h = ctypes.c_void_p()
@@ -84,6 +86,8 @@ def test_null_arguments_rejected_on_host():
         == B.ERR_INVALID_ARG
     assert L.stca_pointwise_forward(None, None, None, None, None, 1, 1, 1, None, None) == B.ERR_INVALID_ARG
     assert L.stca_sync_status(None) == B.ERR_INVALID_ARG
+    assert L.stca_pin_weights(None, None, None) == B.ERR_INVALID_ARG
+    L.stca_unpin_weights(None)
     L.stca_destroy(None)
     # kernel-level entry points validate before launching
     assert L.stca_k_attention(1, None, None, None, None, 1, 1, 256, 3, 1, 0, None, None, None, None, None) \
