@@ -9,9 +9,10 @@
 //
 // One CTA computes a 128-row x 256-column tile with cta_group::1 MMAs (M = 128, N = 256,
 // K = 16) into 256 TMEM columns.  K streams through a 3-stage ring of 64-wide chunks: the
-// weight chunk arrives by TMA (K-major packed weights, 128-byte swizzle); four producer
-// warps load the fp32 activation rows, split them and store the hi and lo tiles in the
-// same swizzled layout.  Those warps then run the epilogue (one TMEM lane quarter each).
+// weight chunk arrives by TMA (K-major packed weights, 128-byte swizzle); eight producer
+// warps load the fp32 activation rows (three chunks in flight), split them and store the
+// hi and lo tiles in the same swizzled layout.  Those warps then run the epilogue (two per
+// TMEM lane quarter).
 // Warp 0 lane 0 issues TMA, warp 1 owns TMEM and its lane 0 issues the MMAs.  Every wait
 // is bounded (see common.cuh); a timeout sets STCA_ERR_TIMEOUT and the CTA winds down.
 #include <algorithm>
@@ -65,11 +66,11 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
 }
 
 template <bool DUAL>
-__global__ void __launch_bounds__(256, 1) tc_query_kernel(const __grid_constant__ CUtensorMap tmB, TcqArgs a) {
+__global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant__ CUtensorMap tmB, TcqArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = q_align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + QSTAGES * QSTAGE);
-  uint64_t* a_full = bars;                 // [QSTAGES] 128 producer arrivals
+  uint64_t* a_full = bars;                 // [QSTAGES] 256 producer arrivals
   uint64_t* b_full = bars + QSTAGES;       // [QSTAGES] TMA bytes
   uint64_t* empty = bars + 2 * QSTAGES;    // [QSTAGES] MMA commit
   uint64_t* d_full = bars + 3 * QSTAGES;   // accumulator complete
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(256, 1) tc_query_kernel(const __grid_constant_
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < QSTAGES; ++s) {
-      mbar_init(&a_full[s], 128);
+      mbar_init(&a_full[s], 256);
       mbar_init(&b_full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -153,60 +154,71 @@ __global__ void __launch_bounds__(256, 1) tc_query_kernel(const __grid_constant_
     }
   } else if (warp >= 4) {
     // ---- producers: lane -> (row sub = lane / 8, 8-column group c = lane % 8); warp pw
-    // takes rows 32 pw + 4 i + sub, i = 0..7, so each load instruction covers 4 whole
-    // 256-byte row segments of the chunk
+    // takes rows 16 pw + 4 i + sub, i = 0..3, so each load instruction covers 4 whole
+    // 256-byte row segments of the chunk.  Three chunks are in flight per thread (register
+    // buffers b0..b2 in turn): the loads of chunk kc + 3 go out once chunk kc is stored.
     const int pw = warp - 4;
     const int sub = lane >> 3, c = lane & 7;
-    const float* rowp[8];
+    const float* rowp[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = m0 + pw * 32 + 4 * i + sub;
+    for (int i = 0; i < 4; ++i) {
+      const int r = m0 + pw * 16 + 4 * i + sub;
       rowp[i] = r < a.M ? A + q_remap(r, a.a_grp, a.a_gstride, a.a_goff) * a.lda : nullptr;
     }
-    float4 buf[16];
-    auto load = [&](int kc) {
+    auto load = [&](int kc, float4 (&b)[8]) {
+      if (kc >= KC) return;
       const int k = kc * QKC;
       const int col = k + (k >= a.ksplit ? a.kshift : 0) + c * 8;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 4; ++i) {
         if (rowp[i]) {
-          buf[2 * i] = __ldg(reinterpret_cast<const float4*>(rowp[i] + col));
-          buf[2 * i + 1] = __ldg(reinterpret_cast<const float4*>(rowp[i] + col + 4));
+          b[2 * i] = __ldg(reinterpret_cast<const float4*>(rowp[i] + col));
+          b[2 * i + 1] = __ldg(reinterpret_cast<const float4*>(rowp[i] + col + 4));
         } else {
-          buf[2 * i] = buf[2 * i + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+          b[2 * i] = b[2 * i + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
     };
-    load(0);
     bool ok = true;
-    for (int kc = 0; kc < KC; ++kc) {
+    auto step = [&](int kc, float4 (&b)[8]) {
+      if (kc >= KC || !ok) return;
       const int s = kc % QSTAGES, round = kc / QSTAGES;
       if ((round > 0 && !mbar_wait(&empty[s], (round - 1) & 1)) || *abort_flag) {
         *abort_flag = 1;
         set_error(a.err, STCA_ERR_TIMEOUT);
         ok = false;
-        break;
+        return;
       }
       uint8_t* hi_t = smem + s * QSTAGE;
       uint8_t* lo_t = hi_t + QA_TILE;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int rr = pw * 32 + 4 * i + sub;
+      for (int i = 0; i < 4; ++i) {
+        const int rr = pw * 16 + 4 * i + sub;
         const int off = rr * 128 + ((c ^ (rr & 7)) << 4);
         uint4 h, l;
-        split2(buf[2 * i].x, buf[2 * i].y, h.x, l.x);
-        split2(buf[2 * i].z, buf[2 * i].w, h.y, l.y);
-        split2(buf[2 * i + 1].x, buf[2 * i + 1].y, h.z, l.z);
-        split2(buf[2 * i + 1].z, buf[2 * i + 1].w, h.w, l.w);
+        split2(b[2 * i].x, b[2 * i].y, h.x, l.x);
+        split2(b[2 * i].z, b[2 * i].w, h.y, l.y);
+        split2(b[2 * i + 1].x, b[2 * i + 1].y, h.z, l.z);
+        split2(b[2 * i + 1].z, b[2 * i + 1].w, h.w, l.w);
         *reinterpret_cast<uint4*>(hi_t + off) = h;
         *reinterpret_cast<uint4*>(lo_t + off) = l;
       }
-      if (kc + 1 < KC) load(kc + 1);  // next chunk's rows in flight while this one is consumed
+      load(kc + 3, b);
       fence_proxy_async_smem();
       mbar_arrive(&a_full[s]);
+    };
+    float4 b0[8], b1[8], b2[8];
+    load(0, b0);
+    load(1, b1);
+    load(2, b2);
+    for (int kc = 0; kc < KC && ok; kc += 3) {
+      step(kc, b0);
+      step(kc + 1, b1);
+      step(kc + 2, b2);
     }
 
-    // ---- epilogue: warp pw reads TMEM lanes 32 pw .. 32 pw + 31 (one output row per lane)
+    // ---- epilogue: two warps per TMEM lane quarter (warp % 4), each on half the columns;
+    // lane l holds output row 32 quarter + l
     if (ok && !mbar_wait(d_full, 0)) {
       *abort_flag = 1;
       set_error(a.err, STCA_ERR_TIMEOUT);
@@ -215,25 +227,27 @@ __global__ void __launch_bounds__(256, 1) tc_query_kernel(const __grid_constant_
     __syncwarp();
     if (ok) {
       tc_fence_after();
-      const int row = m0 + pw * 32 + lane;
-      const uint32_t tbase = tmem + (uint32_t(pw * 32) << 16);
+      const int quarter = warp & 3, half = (warp - 4) >> 2;
+      const int row = m0 + quarter * 32 + lane;
+      const uint32_t tbase = tmem + (uint32_t(quarter * 32) << 16);
       float* crow = row < a.M ? C + q_remap(row, a.c_grp, a.c_gstride, a.c_goff) * a.ldc : nullptr;
       const float* rrow = (row < a.M && R) ? R + int64_t(row) * a.ldr : nullptr;
-      constexpr int NCH = DUAL ? 4 : 8;  // 32-column output chunks per tile
+      constexpr int NCH = DUAL ? 2 : 4;  // 32-column output chunks per warp
 #pragma unroll 1
       for (int j = 0; j < NCH; ++j) {
+        const int tc = half * NCH * 32 + j * 32;  // accumulator column (gate half when DUAL)
         float v[32];
-        tmem_ld_32x32b_x32(tbase + j * 32, v);
+        tmem_ld_32x32b_x32(tbase + tc, v);
         if (DUAL) {
           float u[32];
-          tmem_ld_32x32b_x32(tbase + 128 + j * 32, u);
+          tmem_ld_32x32b_x32(tbase + 128 + tc, u);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = silu_precise(v[e]) * u[e];
         } else {
           tmem_ld_wait();
         }
-        const int col = (DUAL ? blockIdx.x * 128 : blockIdx.x * QBN) + j * 32;
+        const int col = (DUAL ? blockIdx.x * 128 : blockIdx.x * QBN) + tc;
         if (crow && col < a.N) {
           if (rrow) {
 #pragma unroll
@@ -313,12 +327,12 @@ int tc_query_gemm(const SimtGemmArgs<float, bf16>& a, const void* Wp, cudaStream
     if (cudaFuncSetAttribute(tc_query_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(QSMEM)) !=
         cudaSuccess)
       return STCA_ERR_CUDA;
-    tc_query_kernel<true><<<grid, 256, QSMEM, s>>>(tb, q);
+    tc_query_kernel<true><<<grid, 384, QSMEM, s>>>(tb, q);
   } else {
     if (cudaFuncSetAttribute(tc_query_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(QSMEM)) !=
         cudaSuccess)
       return STCA_ERR_CUDA;
-    tc_query_kernel<false><<<grid, 256, QSMEM, s>>>(tb, q);
+    tc_query_kernel<false><<<grid, 384, QSMEM, s>>>(tb, q);
   }
   note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
