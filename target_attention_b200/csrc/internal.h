@@ -55,9 +55,10 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
 
 // C[M, N] (bf16) = epi(A Wp^T), A dense bf16 [M, K] streamed (K a multiple of 64),
 // N in {256, 512}; epi EPI_LN applies LayerNorm (gamma, beta, eps) over the full row.
+// lda: row stride of A in elements (0: K).
 int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
                     const float* beta, float eps, void* C, int ldc, int32_t* err, cudaStream_t s,
-                    const int32_t* M_dev = nullptr);
+                    const int32_t* M_dev = nullptr, int lda = 0);
 
 // 2-D bf16 tensor map over a [rows, cols] row-major matrix (row stride ld elements),
 // box = 64 columns x box_rows rows, 128-byte swizzle, zero fill outside the matrix.

@@ -26,10 +26,12 @@ struct stca_handle {
   int32_t* err = nullptr;
   int32_t *hoff = nullptr, *toff = nullptr, *hoff2 = nullptr;
   // history side
+  // history weights in tensor-core operand order, per slot (sequence sq, layer l) at
+  // sq * M + l: all slots' W1|W3 [2h, d] back to back (so one GEMM covers the M layers of
+  // a sequence), then all W2 [d, h], then all W_K|W_V [2d, d]
   void* wpack = nullptr;
-  size_t wpack_layer = 0;  // elements per layer (per sequence for the decode variant)
+  int wslots = 0;
   void *hidden = nullptr, *xt = nullptr, *kv = nullptr;
-  void* xg = nullptr;  // gathered history rows, written by the first layer, read by the rest
   // target-side weights packed K-major for the tensor cores (bf16 STCA), element offsets
   void* qpack = nullptr;
   struct QLayout {
@@ -265,11 +267,12 @@ int allocate(stca_handle* h) {
   const size_t E = esize(c);
   const int nseq = c.mode == STCA_MODE_HYFORMER ? 2 : 1;
   if (c.dtype == STCA_BF16) {
-    h->wpack_layer = 2 * hd * d + d * hd + 2 * d * d;
-    ok = ok && dalloc(h, &h->wpack, size_t(c.M) * nseq * h->wpack_layer * 2);
+    h->wslots = c.M * nseq;
+    ok = ok && dalloc(h, &h->wpack, size_t(h->wslots) * (2 * hd * d + d * hd + 2 * d * d) * 2);
   }
-  ok = ok && dalloc(h, &h->hidden, N * hd * E) && dalloc(h, &h->xt, N * d * E) && dalloc(h, &h->kv, N * 2 * d * E);
-  if (c.dtype == STCA_BF16 && c.M > 1) ok = ok && dalloc(h, &h->xg, nseq * N * d * 2);
+  // bf16: the hidden activations of all M layers of every sequence ([N, M h] per sequence)
+  const size_t hid_elems = c.dtype == STCA_BF16 ? nseq * N * size_t(c.M) * hd : N * hd;
+  ok = ok && dalloc(h, &h->hidden, hid_elems * E) && dalloc(h, &h->xt, N * d * E) && dalloc(h, &h->kv, N * 2 * d * E);
   ok = ok && dalloc(h, &h->qproj, T * d * 4) && dalloc(h, &h->attn, T * d * 4) && dalloc(h, &h->tmp_h, T * hd * 4) &&
        dalloc(h, &h->tmp_d, T * d * 4);
   ok = ok && dalloc(h, &h->part_acc, size_t(MAX_SPLITS) * T * d * 4) &&
@@ -374,17 +377,27 @@ bool is_pinned(const stca_handle* h, const void* w, size_t bytes) {
          memcmp(h->pinned_copy.data(), w, bytes) == 0;
 }
 
+// Packed history operands of slot sq * M + l.
+bf16* wp13(const stca_handle* h, int slot) {
+  const size_t d = size_t(h->cfg.d), hd = size_t(h->cfg.hidden);
+  return reinterpret_cast<bf16*>(h->wpack) + size_t(slot) * 2 * hd * d;
+}
+bf16* wp2(const stca_handle* h, int slot) {
+  const size_t d = size_t(h->cfg.d), hd = size_t(h->cfg.hidden);
+  return wp13(h, h->wslots) + size_t(slot) * d * hd;
+}
+bf16* wp3(const stca_handle* h, int slot) {
+  const size_t d = size_t(h->cfg.d), hd = size_t(h->cfg.hidden);
+  return reinterpret_cast<bf16*>(h->wpack) + size_t(h->wslots) * (2 * hd * d + d * hd) + size_t(slot) * 2 * d * d;
+}
+
 // One history layer: the FFN, then W_K and W_V stacked into [2 d, d] (K rows, then V rows).
-void layer_jobs(stca_handle* h, size_t slot, const stca_ffn& f, const void* WK, const void* WV,
+void layer_jobs(stca_handle* h, int slot, const stca_ffn& f, const void* WK, const void* WV,
                 std::vector<PackJob>& jobs) {
   const int d = h->cfg.d, hd = h->cfg.hidden;
-  bf16* base = reinterpret_cast<bf16*>(h->wpack) + slot * h->wpack_layer;
-  bf16* wp1 = base;
-  bf16* wp2 = base + size_t(2) * hd * d;
-  bf16* wp3 = wp2 + size_t(d) * hd;
-  ffn_jobs(f, d, hd, wp1, wp2, jobs);
-  jobs.push_back({WK, wp3, d, d, 0, 0});
-  jobs.push_back({WV, wp3, d, d, 0, d});
+  ffn_jobs(f, d, hd, wp13(h, slot), wp2(h, slot), jobs);
+  jobs.push_back({WK, wp3(h, slot), d, d, 0, 0});
+  jobs.push_back({WV, wp3(h, slot), d, d, 0, d});
 }
 
 // The target-side weights of a bf16 STCA call.
@@ -420,7 +433,7 @@ void hyf_jobs(stca_handle* h, const hyf_weights* w, int tokens, std::vector<Pack
   for (int l = 0; l < h->cfg.M; ++l)
     for (int sq = 0; sq < 2; ++sq) {
       const hyf_seq_weights& f = w->blk[l].seq[sq];
-      layer_jobs(h, size_t(l) * 2 + sq, f.ffn, f.WK, f.WV, jobs);
+      layer_jobs(h, sq * h->cfg.M + l, f.ffn, f.WK, f.WV, jobs);
       jobs.push_back({f.WQ, q + L.hwq[2 * l + sq], d, d, 0, 0});
       jobs.push_back({f.WO, q + L.hwo[2 * l + sq], d, d, 0, 0});
     }
@@ -430,30 +443,35 @@ void hyf_jobs(stca_handle* h, const hyf_weights* w, int tokens, std::vector<Pack
                jobs);
 }
 
-// K/V of every history token for one layer: bf16 tensor-core path.
-// x_load: rows gathered by an earlier layer (dense operand); else gather, writing the rows
-// to x_store when it is not null.
-int history_bf16(stca_handle* h, size_t slot, const GatherSrc& g, int n_tok, const float* gamma, const float* beta,
-                 cudaStream_t s, const int32_t* M_dev, void* x_store, const void* x_load) {
-  const int d = h->cfg.d, hd = h->cfg.hidden;
-  const bf16* base = reinterpret_cast<const bf16*>(h->wpack) + slot * h->wpack_layer;
-  const bf16* wp1 = base;
-  const bf16* wp2 = base + size_t(2) * hd * d;
-  const bf16* wp3 = wp2 + size_t(d) * hd;
+// SwiGLU hidden activations of all M layers of history sequence sq in one launch: the X
+// rows are gathered once (E[id] + T[bucket]) and multiplied by the M layers' W1|W3 packed
+// back to back (N = M 2h); layer l's hidden lands in columns [l h, (l+1) h) of the
+// sequence's [n_tok, M h] buffer.  Every layer reads the ORIGINAL X, so this is exact.
+int history_hidden_bf16(stca_handle* h, int sq, const GatherSrc& g, int n_tok, cudaStream_t s,
+                        const int32_t* M_dev) {
+  const int d = h->cfg.d, hd = h->cfg.hidden, M = h->cfg.M;
+  bf16* hid = reinterpret_cast<bf16*>(h->hidden) + size_t(sq) * size_t(h->cfg.max_tokens) * M * hd;
+  STAGE(h, STCA_STAGE_GATHER_FFN, s,
+        tc_gemm_resident(A_GATHER, EPI_SWIGLU, nullptr, g, n_tok, d, wp13(h, sq * M), M * hd, hid, M * hd, h->err, s,
+                         M_dev));
+  return STCA_OK;
+}
+
+// X~ = LN(A W2) and [K | V] = X~ [W_K | W_V] of layer l of sequence sq (bf16 tensor cores).
+int history_kv_bf16(stca_handle* h, int sq, int l, int n_tok, const float* gamma, const float* beta, cudaStream_t s,
+                    const int32_t* M_dev) {
+  const int d = h->cfg.d, hd = h->cfg.hidden, M = h->cfg.M;
+  const int slot = sq * M + l;
+  const bf16* hid = reinterpret_cast<const bf16*>(h->hidden) + size_t(sq) * size_t(h->cfg.max_tokens) * M * hd +
+                    size_t(l) * hd;
   GatherSrc none;
   memset(&none, 0, sizeof(none));
-  if (x_load)
-    STAGE(h, STCA_STAGE_GATHER_FFN, s,
-          tc_gemm_resident(A_TMA, EPI_SWIGLU, x_load, none, n_tok, d, wp1, hd, h->hidden, hd, h->err, s, M_dev));
-  else
-    STAGE(h, STCA_STAGE_GATHER_FFN, s,
-          tc_gemm_resident(A_GATHER, EPI_SWIGLU, nullptr, g, n_tok, d, wp1, hd, h->hidden, hd, h->err, s, M_dev,
-                           x_store));
   STAGE(h, STCA_STAGE_FFN_OUT, s,
-        tc_gemm_rowwise(gamma ? EPI_LN : EPI_PLAIN, h->hidden, n_tok, hd, wp2, d, gamma, beta, h->cfg.ln_eps, h->xt,
-                        d, h->err, s, M_dev));
+        tc_gemm_rowwise(gamma ? EPI_LN : EPI_PLAIN, hid, n_tok, hd, wp2(h, slot), d, gamma, beta, h->cfg.ln_eps, h->xt,
+                        d, h->err, s, M_dev, M * hd));
   STAGE(h, STCA_STAGE_KV, s,
-        tc_gemm_resident(A_TMA, EPI_PLAIN, h->xt, none, n_tok, d, wp3, 2 * d, h->kv, 2 * d, h->err, s, M_dev));
+        tc_gemm_resident(A_TMA, EPI_PLAIN, h->xt, none, n_tok, d, wp3(h, slot), 2 * d, h->kv, 2 * d, h->err, s,
+                         M_dev));
   return STCA_OK;
 }
 
@@ -558,9 +576,10 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
   const int32_t* kv_mult = c.dedup == 2 ? h->c_mult : nullptr;
   const int splits = attention_splits(n_tok, B, c.H, 1024);
   for (int i = 0; i < M; ++i) {
-    if (bf)
-      CK(history_bf16(h, i, g, n_tok, w->hist[i].gamma, w->hist[i].beta, s, M_dev, i == 0 ? h->xg : nullptr,
-                      i > 0 ? h->xg : nullptr));
+    if (bf) {
+      if (i == 0) CK(history_hidden_bf16(h, 0, g, n_tok, s, M_dev));
+      CK(history_kv_bf16(h, 0, i, n_tok, w->hist[i].gamma, w->hist[i].beta, s, M_dev));
+    }
     else CK(history_f32(h, g, n_tok, w->hist[i], w->WK[i], w->WV[i], s));
     STAGE(h, STCA_STAGE_QUERY, s,
           qgemm(gemm_args<TB>(t_tot, d, d, h->qbuf, d, w->WQ[i], h->qproj, d, h->err), qp(h, L.wq[i]), s));
@@ -844,9 +863,8 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
           kv_mult = h->c_mult + off;
         }
       }
-      void* xs = h->xg ? static_cast<bf16*>(h->xg) + size_t(sq) * size_t(h->cfg.max_tokens) * d : nullptr;
-      CK(history_bf16(h, size_t(l) * 2 + sq, g, ntok[sq], nullptr, nullptr, s, M_dev, l == 0 ? xs : nullptr,
-                      l > 0 ? xs : nullptr));
+      if (l == 0) CK(history_hidden_bf16(h, sq, g, ntok[sq], s, M_dev));
+      CK(history_kv_bf16(h, sq, l, ntok[sq], nullptr, nullptr, s, M_dev));
       // queries of sequence sq: rows b*T + sq*n_query + n
       auto qa = gemm_args<bf16>(rows_s, d, d, h->hq, d, f.WQ, h->qproj, d, h->err);
       qa.a_grp = n_query;

@@ -879,13 +879,16 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
 
 int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
                     const float* beta, float eps, void* C, int ldc, int32_t* err, cudaStream_t s,
-                    const int32_t* M_dev) {
+                    const int32_t* M_dev, int lda) {
   if (M == 0) return 0;
-  if (M < 0 || K <= 0 || K % 64 != 0 || (N != 256 && N != 512) || ldc % 8 != 0) return STCA_ERR_UNSUPPORTED;
+  if (lda == 0) lda = K;
+  if (M < 0 || K <= 0 || K % 64 != 0 || (N != 256 && N != 512) || ldc % 8 != 0 || lda < K || lda % 8 != 0 ||
+      reinterpret_cast<uintptr_t>(A) % 16 != 0)
+    return STCA_ERR_UNSUPPORTED;
   if (epi == EPI_LN && (!gamma || !beta)) return STCA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(C) % 16 != 0) return STCA_ERR_INVALID_ARG;
   CUtensorMap ta, tb, tc;
-  if (!make_tmap(&ta, A, M, K, K, BM)) return STCA_ERR_CUDA;
+  if (!make_tmap(&ta, A, M, K, lda, BM)) return STCA_ERR_CUDA;
   if (!make_tmap(&tb, Wp, N, K, K, BM)) return STCA_ERR_CUDA;
   if (!make_tmap_out(&tc, C, M, N, ldc)) return STCA_ERR_CUDA;
   if (N == 512) {
