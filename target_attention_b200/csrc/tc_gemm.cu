@@ -274,11 +274,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     }
   } else if (warp == 1) {
     if (leader && lane == 0) {
+      // The issue loop is the kernel's critical thread: everything per MMA is precomputed
+      // (descriptor bases advance by constant steps; the ring slot and phase are counters).
       const uint32_t idesc = umma_idesc_bf16(256, 256);
       const uint32_t own_b_empty0 = cluster_addr(&b_empty[0], 0), peer_b_empty0 = cluster_addr(&b_empty[0], 1);
       const uint32_t own_a_empty0 = cluster_addr(&a_empty[0], 0), peer_a_empty0 = cluster_addr(&a_empty[0], 1);
       const uint32_t own_t_full0 = cluster_addr(&t_full[0], 0), peer_t_full0 = cluster_addr(&t_full[0], 1);
-      int it = 0, gnt = 0, li = 0;
+      // descriptor start addresses are in 16-byte units: +2 per 16-element K step
+      const uint64_t adesc0 = umma_sdesc_sw128(smem_u32(sA)), bdesc0 = umma_sdesc_sw128(smem_u32(sB));
+      int s = 0, gnt = 0, li = 0;
+      uint32_t bphase = 0;
       bool ok = true;
       for (int tile = cl; tile < num_tiles && ok; tile += ncl, ++li) {
         for (int nt = 0; nt < NT && ok; ++nt, ++gnt) {
@@ -290,26 +295,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
           }
           tc_fence_after();
           const uint32_t dcol = tmem + buf * 256;
-          for (int kc = 0; kc < KC; ++kc, ++it) {
-            const int s = it % STAGES;
-            if ((nt == 0 && !mbar_wait_cluster(&a_full[kc], li & 1)) || !mbar_wait(&b_full[s], (it / STAGES) & 1) ||
-                abort_set(abort_flag)) {
+          for (int kc = 0; kc < KC; ++kc) {
+            if ((nt == 0 && !mbar_wait_cluster(&a_full[kc], li & 1)) || !mbar_wait(&b_full[s], bphase)) {
               fail(abort_flag, err);
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t a_addr = smem_u32(sA + kc * A_CHUNK);
-            const uint32_t b_addr = smem_u32(sB + s * B_HALF);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              umma_bf16_pair(dcol, umma_sdesc_sw128(a_addr + k * 32), umma_sdesc_sw128(b_addr + k * 32), idesc,
-                             (kc | k) != 0);
+            const uint64_t ad = adesc0 + uint64_t(kc * (A_CHUNK >> 4));
+            const uint64_t bd = bdesc0 + uint64_t(s * (B_HALF >> 4));
+            umma_bf16_pair(dcol, ad, bd, idesc, kc != 0);
+            umma_bf16_pair(dcol, ad + 2, bd + 2, idesc, 1);
+            umma_bf16_pair(dcol, ad + 4, bd + 4, idesc, 1);
+            umma_bf16_pair(dcol, ad + 6, bd + 6, idesc, 1);
             umma_commit_pair(own_b_empty0 + s * 8);
             umma_commit_pair(peer_b_empty0 + s * 8);
             if (nt == NT - 1) {
               umma_commit_pair(own_a_empty0 + kc * 8);
               umma_commit_pair(peer_a_empty0 + kc * 8);
+            }
+            if (++s == STAGES) {
+              s = 0;
+              bphase ^= 1;
             }
           }
           if (ok) {
@@ -576,7 +583,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       const uint32_t idesc = umma_idesc_bf16(256, 256);
       const uint32_t own_empty0 = cluster_addr(&empty[0], 0), peer_empty0 = cluster_addr(&empty[0], 1);
       const uint32_t own_t_full = cluster_addr(t_full, 0), peer_t_full = cluster_addr(t_full, 1);
-      int it = 0, li = 0;
+      // lean issue loop: descriptor bases advance by constant steps (16-byte units)
+      const uint64_t desc0 = umma_sdesc_sw128(smem_u32(smem));
+      int s = 0, li = 0;
+      uint32_t phase = 0;
       bool ok = true;
       for (int tile = cl; tile < num_tiles && ok; tile += ncl, ++li) {
         if (li > 0 && !mbar_wait_cluster(t_empty, (li - 1) & 1)) {
@@ -584,26 +594,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           break;
         }
         tc_fence_after();
-        for (int kc = 0; kc < KC; ++kc, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(&full[s], (it / STAGES) & 1) || abort_set(abort_flag)) {
+        for (int kc = 0; kc < KC; ++kc) {
+          if (!mbar_wait(&full[s], phase)) {
             fail(abort_flag, err);
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * STAGE_BYTES);
+          const uint64_t ad = desc0 + uint64_t(s * (STAGE_BYTES >> 4));
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-              const uint32_t b_addr = a_addr + A_CHUNK + nb * B_HALF;
-              umma_bf16_pair(tmem + nb * 256, umma_sdesc_sw128(a_addr + k * 32),
-                             umma_sdesc_sw128(b_addr + k * 32), idesc, (kc | k) != 0);
-            }
+            for (int nb = 0; nb < NB; ++nb)
+              umma_bf16_pair(tmem + nb * 256, ad + 2 * k, ad + ((A_CHUNK + nb * B_HALF) >> 4) + 2 * k, idesc,
+                             (kc | k) != 0);
           }
           umma_commit_pair(own_empty0 + s * 8);
           umma_commit_pair(peer_empty0 + s * 8);
+          if (++s == STAGES) {
+            s = 0;
+            phase ^= 1;
+          }
         }
         if (ok) {
           umma_commit_pair(own_t_full);

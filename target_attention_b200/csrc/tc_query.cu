@@ -128,27 +128,32 @@ __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant_
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = umma_idesc_bf16(QBM, QBN);
+      // lean issue loop: descriptor bases advance by constant steps (16-byte units)
+      const uint64_t desc0 = umma_sdesc_sw128(smem_u32(smem));
       bool ok = true;
+      int s = 0;
+      uint32_t par = 0;
       for (int kc = 0; kc < KC; ++kc) {
-        const int s = kc % QSTAGES;
-        const uint32_t par = (kc / QSTAGES) & 1;
-        if (!mbar_wait(&a_full[s], par) || !mbar_wait(&b_full[s], par) || *abort_flag) {
+        if (!mbar_wait(&a_full[s], par) || !mbar_wait(&b_full[s], par)) {
           *abort_flag = 1;
           set_error(a.err, STCA_ERR_TIMEOUT);
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a_hi = smem_u32(smem + s * QSTAGE);
-        const uint32_t a_lo = a_hi + QA_TILE;
-        const uint32_t b = a_hi + 2 * QA_TILE;
+        const uint64_t hi = desc0 + uint64_t(s * (QSTAGE >> 4));
+        const uint64_t lo = hi + (QA_TILE >> 4);
+        const uint64_t b = hi + ((2 * QA_TILE) >> 4);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint64_t bd = umma_sdesc_sw128(b + k * 32);
-          umma_bf16(tmem, umma_sdesc_sw128(a_hi + k * 32), bd, idesc, (kc | k) != 0);
-          umma_bf16(tmem, umma_sdesc_sw128(a_lo + k * 32), bd, idesc, 1);
+          umma_bf16(tmem, hi + 2 * k, b + 2 * k, idesc, (kc | k) != 0);
+          umma_bf16(tmem, lo + 2 * k, b + 2 * k, idesc, 1);
         }
         umma_commit(&empty[s]);
+        if (++s == QSTAGES) {
+          s = 0;
+          par ^= 1;
+        }
       }
       if (ok) umma_commit(d_full);
     }
