@@ -332,6 +332,15 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t cluster_bar) {
                : "memory");
 }
 
+// One arrive on the mbarrier at the same shared offset in each CTA of cta_mask (the pair:
+// 0b11) when the pair MMAs issued so far are done: one instruction instead of two commits.
+__device__ __forceinline__ void umma_commit_pair_both(const void* bar, uint16_t cta_mask) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+                   smem_u32(bar)),
+               "h"(cta_mask)
+               : "memory");
+}
+
 // ------------------------------------------------------------------ misc math
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }

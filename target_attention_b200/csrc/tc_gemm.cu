@@ -15,7 +15,8 @@
 // weight bytes.  The kernels are persistent (one pair per two SMs).  Warp roles: warp 0
 // lane 0 issues TMA, warp 1 owns TMEM and (leader CTA) lane 0 issues tcgen05.mma, warps
 // 4..11 run the epilogue, two warps per TMEM lane quarter (warp w reads lanes
-// 32 (w % 4) .. + 32), each on half of the columns; warps 12..15 gather A rows.
+// 32 (w % 4) .. + 32), each on half of the columns; warps 12, 14, 15 and 2 gather A rows
+// (none on the MMA warp's scheduler, warp % 4 == 1, whose issue slots stay free).
 // Waits are bounded (see common.cuh).
 #include <algorithm>
 #include <mutex>
@@ -136,7 +137,7 @@ __device__ __forceinline__ bool epilogue_any(bool flag) {
   return r != 0;
 }
 
-// Named barrier over the 128 gather threads (warps 12..15).
+// Named barrier over the 128 gather threads (warps 12, 14, 15, 2).
 __device__ __forceinline__ void gather_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 // Item id and time bucket of global row `grow`; false (and a zero row) when the row is
@@ -169,7 +170,7 @@ __device__ __forceinline__ bool gather_row(const GatherSrc& g, int grow, int M, 
 // chunk kc of the next row tile's A is loaded as soon as the last N tile has used it.
 //
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer (leader CTA), 4..11 epilogue,
-// 12..15 gather producer (gather mode): cp.async of the CTA's A rows into the swizzled
+// 12, 14, 15, 2 gather producer (gather mode): cp.async of the CTA's A rows into the swizzled
 // layout (8 lanes per 128-byte row segment), the time-bucket row added from shared
 // memory, and an L2 prefetch of the next tile's rows one tile ahead.  With store_x the
 // gather warps also write the finished A rows to X (TMA tile stores straight from the
@@ -277,9 +278,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
       // The issue loop is the kernel's critical thread: everything per MMA is precomputed
       // (descriptor bases advance by constant steps; the ring slot and phase are counters).
       const uint32_t idesc = umma_idesc_bf16(256, 256);
-      const uint32_t own_b_empty0 = cluster_addr(&b_empty[0], 0), peer_b_empty0 = cluster_addr(&b_empty[0], 1);
-      const uint32_t own_a_empty0 = cluster_addr(&a_empty[0], 0), peer_a_empty0 = cluster_addr(&a_empty[0], 1);
-      const uint32_t own_t_full0 = cluster_addr(&t_full[0], 0), peer_t_full0 = cluster_addr(&t_full[0], 1);
       // descriptor start addresses are in 16-byte units: +2 per 16-element K step
       const uint64_t adesc0 = umma_sdesc_sw128(smem_u32(sA)), bdesc0 = umma_sdesc_sw128(smem_u32(sB));
       int s = 0, gnt = 0, li = 0;
@@ -308,32 +306,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
             umma_bf16_pair(dcol, ad + 2, bd + 2, idesc, 1);
             umma_bf16_pair(dcol, ad + 4, bd + 4, idesc, 1);
             umma_bf16_pair(dcol, ad + 6, bd + 6, idesc, 1);
-            umma_commit_pair(own_b_empty0 + s * 8);
-            umma_commit_pair(peer_b_empty0 + s * 8);
-            if (nt == NT - 1) {
-              umma_commit_pair(own_a_empty0 + kc * 8);
-              umma_commit_pair(peer_a_empty0 + kc * 8);
-            }
+            umma_commit_pair_both(&b_empty[s], 0x3);
+            if (nt == NT - 1) umma_commit_pair_both(&a_empty[kc], 0x3);
             if (++s == STAGES) {
               s = 0;
               bphase ^= 1;
             }
           }
           if (ok) {
-            umma_commit_pair(own_t_full0 + buf * 8);
-            umma_commit_pair(peer_t_full0 + buf * 8);
+            umma_commit_pair_both(&t_full[buf], 0x3);
           }
         }
       }
       umma_commit_pair(cluster_addr(mma_done, 0));
       mbar_wait(mma_done, 0);
     }
-  } else if (warp >= 12) {
+  } else if (warp == 2 || warp == 12 || warp >= 14) {
     // gather warps: warp gw copies rows 32 gw .. 32 gw + 31 of this CTA's A tile; in each
     // copy instruction 8 consecutive lanes take the 8 16-byte chunks of one row, so a warp
     // moves 4 whole 128-byte row segments per instruction (row r_i = 32 gw + 4 i + lane/8)
     if (AMODE == A_GATHER) {
-      const int gw = warp - 12;
+      const int gw = warp == 2 ? 3 : (warp == 12 ? 0 : warp - 13);
       const int sub = lane >> 3, c = lane & 7;
       const int t128 = gw * 32 + lane;
       const bool with_dt = g.dt != nullptr && g.dt_table != nullptr;
@@ -435,7 +428,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
       cp_async_wait_all();
       if (store_x && lane == 0) bulk_wait_all();
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 12) {
     // two epilogue warps per TMEM lane quarter, each taking half of the columns
     const int quarter = warp & 3;
     const int half = (warp - 4) >> 2;
@@ -581,8 +574,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   } else if (warp == 1) {
     if (leader && lane == 0) {
       const uint32_t idesc = umma_idesc_bf16(256, 256);
-      const uint32_t own_empty0 = cluster_addr(&empty[0], 0), peer_empty0 = cluster_addr(&empty[0], 1);
-      const uint32_t own_t_full = cluster_addr(t_full, 0), peer_t_full = cluster_addr(t_full, 1);
       // lean issue loop: descriptor bases advance by constant steps (16-byte units)
       const uint64_t desc0 = umma_sdesc_sw128(smem_u32(smem));
       int s = 0, li = 0;
@@ -609,16 +600,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
               umma_bf16_pair(tmem + nb * 256, ad + 2 * k, ad + ((A_CHUNK + nb * B_HALF) >> 4) + 2 * k, idesc,
                              (kc | k) != 0);
           }
-          umma_commit_pair(own_empty0 + s * 8);
-          umma_commit_pair(peer_empty0 + s * 8);
+          umma_commit_pair_both(&empty[s], 0x3);
           if (++s == STAGES) {
             s = 0;
             phase ^= 1;
           }
         }
         if (ok) {
-          umma_commit_pair(own_t_full);
-          umma_commit_pair(peer_t_full);
+          umma_commit_pair_both(t_full, 0x3);
         }
       }
       umma_commit_pair(cluster_addr(mma_done, 0));
