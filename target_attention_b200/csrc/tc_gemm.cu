@@ -63,8 +63,8 @@ constexpr int BM = 128;                        // tile rows = TMEM lanes
 constexpr int A_CHUNK = BM * 64 * 2;           // one 64-wide K chunk of A: 16 KB
 constexpr int B_HALF = BM * 128;               // one CTA's 128 weight rows x 64 K: 16 KB
 constexpr int OUT_STAGE = 32 * 64;             // one epilogue warp's 32 x 32 bf16 output tile
-constexpr int T_BYTES = 16 * 512 * 2;          // time-bucket table, K <= 512
 constexpr int MIN_SMEM = 120 * 1024;           // keeps one CTA per SM (TMEM is not shared)
+constexpr int GATHER_LAG = 2;                  // gathered chunks in flight before one is published
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -137,8 +137,6 @@ __device__ __forceinline__ bool epilogue_any(bool flag) {
   return r != 0;
 }
 
-// Named barrier over the 128 gather threads (warps 12, 14, 15, 2).
-__device__ __forceinline__ void gather_sync() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
 // Item id and time bucket of global row `grow`; false (and a zero row) when the row is
 // past M or the id is out of range (recorded in the error word).
@@ -171,8 +169,8 @@ __device__ __forceinline__ bool gather_row(const GatherSrc& g, int grow, int M, 
 //
 // Warps: 0 TMA producer, 1 TMEM owner + MMA issuer (leader CTA), 4..11 epilogue,
 // 12, 14, 15, 2 gather producer (gather mode): cp.async of the CTA's A rows into the swizzled
-// layout (8 lanes per 128-byte row segment), the time-bucket row added from shared
-// memory, and an L2 prefetch of the next tile's rows one tile ahead.  With store_x the
+// layout (8 lanes per 128-byte row segment), the time-bucket row added (from L1), and
+// an L2 prefetch of the next tile's rows one tile ahead.  With store_x the
 // gather warps also write the finished A rows to X (TMA tile stores straight from the
 // swizzled chunks), so that later layers over the same rows read X with TMA instead of
 // gathering again.
@@ -188,8 +186,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
   uint8_t* sA = smem;
   uint8_t* sB = sA + KC * A_CHUNK;
   uint8_t* sOut = sB + STAGES * B_HALF;               // 8 warps x 2 KB
-  uint8_t* sT = sOut + 8 * OUT_STAGE;                 // 16 x K bf16 (gather mode)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sT + (AMODE == A_GATHER ? T_BYTES : 0));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + 8 * OUT_STAGE);
   uint64_t* a_full = bars;                 // [8]      leader
   uint64_t* a_empty = bars + 8;            // [8]      both
   uint64_t* b_full = bars + 16;            // [STAGES] leader
@@ -328,13 +325,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     if (AMODE == A_GATHER) {
       const int gw = warp == 2 ? 3 : (warp == 12 ? 0 : warp - 13);
       const int sub = lane >> 3, c = lane & 7;
-      const int t128 = gw * 32 + lane;
       const bool with_dt = g.dt != nullptr && g.dt_table != nullptr;
-      if (with_dt) {
-        const uint4* src = reinterpret_cast<const uint4*>(g.dt_table);
-        for (int i = t128; i < 16 * K / 8; i += 128) reinterpret_cast<uint4*>(sT)[i] = __ldg(src + i);
-      }
-      gather_sync();
+      const bf16* dtt = reinterpret_cast<const bf16*>(g.dt_table);
       const bf16* table = reinterpret_cast<const bf16*>(g.table);
       const uint32_t a_full0 = cluster_addr(&a_full[0], 0);
       int32_t id[8], nid[8];
@@ -368,25 +360,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
           if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
         }
-        for (int kc = 0; kc < KC; ++kc) {
-          if (li > 0 && !mbar_wait(&a_empty[kc], (li - 1) & 1)) {
-            fail(abort_flag, err);
-            ok = false;
-            break;
-          }
-          uint8_t* chunk = sA + kc * A_CHUNK;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r = gw * 32 + i * 4 + sub;
-            const bool v = (vmask >> i) & 1u;
-            cp_async_16(chunk + r * 128 + ((c ^ (r & 7)) << 4), table + int64_t(v ? id[i] : 0) * K + kc * 64 + c * 8,
-                        v ? 16u : 0u);
-          }
-          cp_async_commit();
-        }
-        if (!ok) break;
-        for (int kc = 0; kc < KC; ++kc) {
-          cp_async_wait_dyn(KC - 1 - kc);
+        // chunk kc - GATHER_LAG is completed and published right after chunk kc is issued,
+        // so chunk 0 of a tile is ready while the MMAs still work through the previous
+        // tile's last chunks (each chunk is only refilled once those MMAs released it)
+        auto publish = [&](int kc) {
           if (with_dt) {
             uint8_t* chunk = sA + kc * A_CHUNK;
 #pragma unroll
@@ -395,7 +372,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
               const int r = gw * 32 + i * 4 + sub;
               uint4* p = reinterpret_cast<uint4*>(chunk + r * 128 + ((c ^ (r & 7)) << 4));
               const uint4 x = *p;
-              const uint4 t = *reinterpret_cast<const uint4*>(sT + bk[i] * K * 2 + kc * 128 + c * 16);
+              // the 16-row time table (16 K bf16) stays in L1
+              const uint4 t = __ldg(reinterpret_cast<const uint4*>(dtt + int64_t(bk[i]) * K + kc * 64 + c * 8));
               const __nv_bfloat162* xa = reinterpret_cast<const __nv_bfloat162*>(&x);
               const __nv_bfloat162* ta = reinterpret_cast<const __nv_bfloat162*>(&t);
               uint32_t o[4];
@@ -417,6 +395,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
               bulk_commit();
             }
           }
+        };
+        for (int kc = 0; kc < KC; ++kc) {
+          if (li > 0 && !mbar_wait(&a_empty[kc], (li - 1) & 1)) {
+            fail(abort_flag, err);
+            ok = false;
+            break;
+          }
+          uint8_t* chunk = sA + kc * A_CHUNK;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = gw * 32 + i * 4 + sub;
+            const bool v = (vmask >> i) & 1u;
+            cp_async_16(chunk + r * 128 + ((c ^ (r & 7)) << 4), table + int64_t(v ? id[i] : 0) * K + kc * 64 + c * 8,
+                        v ? 16u : 0u);
+          }
+          cp_async_commit();
+          if (kc >= GATHER_LAG) {
+            cp_async_wait<GATHER_LAG>();
+            publish(kc - GATHER_LAG);
+          }
+        }
+        if (!ok) break;
+        for (int kc = KC - GATHER_LAG; kc < KC; ++kc) {
+          cp_async_wait_dyn(KC - 1 - kc);
+          publish(kc);
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -768,7 +771,7 @@ bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t c
 }
 
 size_t resident_smem(int K, int stages, bool gather) {
-  size_t bytes = 1024 + size_t(K / 64) * A_CHUNK + size_t(stages) * B_HALF + 8 * OUT_STAGE + (gather ? T_BYTES : 0) + 512;
+  size_t bytes = 1024 + size_t(K / 64) * A_CHUNK + size_t(stages) * B_HALF + 8 * OUT_STAGE + 512;
   return bytes < MIN_SMEM ? MIN_SMEM : bytes;
 }
 
@@ -867,8 +870,8 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
   const int sx = x_out != nullptr;
   // stage counts fill the 227 KB of shared memory (see resident_smem)
 #define STCA_RES(AM, EP)                                                                                   \
-  (K == 512 ? run_resident<AM, EP, (AM == A_GATHER ? 4 : 5)>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev)     \
-            : run_resident<AM, EP, (AM == A_GATHER ? 8 : 9)>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev))
+  (K == 512 ? run_resident<AM, EP, 5>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev)     \
+            : run_resident<AM, EP, 9>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev))
   if (amode == A_TMA && epi == EPI_PLAIN) return STCA_RES(A_TMA, EPI_PLAIN);
   if (amode == A_TMA && epi == EPI_SWIGLU) return STCA_RES(A_TMA, EPI_SWIGLU);
   if (amode == A_GATHER && epi == EPI_PLAIN) return STCA_RES(A_GATHER, EPI_PLAIN);
