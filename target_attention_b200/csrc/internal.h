@@ -23,7 +23,21 @@ struct GatherSrc {
 };
 
 enum AMode { A_TMA = 0, A_GATHER = 1 };
-enum Epi { EPI_PLAIN = 0, EPI_SWIGLU = 1, EPI_LN = 2 };
+enum Epi { EPI_PLAIN = 0, EPI_SWIGLU = 1, EPI_LN = 2, EPI_LNSTAT = 3, EPI_LNFOLD = 4 };
+
+// LayerNorm folded into the GEMM that follows it.  With s = (mean_r, rstd_r) of row r of y
+// and y' = y * gamma (per column), LN(y) W = rstd_r (y' W - mean_r c) + b with
+// c = gamma^T W and b = beta^T W, so the LN GEMM only has to write y' and the row moments
+// (EPI_LNSTAT) and the next GEMM applies the row scale and shift in its epilogue
+// (EPI_LNFOLD).  stats: [rows][2] fp32; cvec, bvec: [N] fp32 for the N output columns.
+struct EpiFold {
+  const float* stats;
+  const float* cvec;
+  const float* bvec;
+};
+// c and b of the fold for W = [WK | WV] ([d, d] bf16 each, row-major): out [2][2d] fp32.
+int fold_consts(const float* gamma, const float* beta, const void* WK, const void* WV, int d, float* out,
+                cudaStream_t s);
 
 // ---------------------------------------------------------------- tcgen05 GEMMs (bf16)
 
@@ -51,14 +65,15 @@ int tc_pack_weights(const PackJob* jobs, int n, cudaStream_t s);
 // null): bf16 [M, K] receiving the gathered A rows (E[id] + T[bucket]) as the MMAs used them.
 int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int K, const void* Wp,
                      int Nout, void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev = nullptr,
-                     void* x_out = nullptr);
+                     void* x_out = nullptr, const EpiFold* fold = nullptr);
 
 // C[M, N] (bf16) = epi(A Wp^T), A dense bf16 [M, K] streamed (K a multiple of 64),
 // N in {256, 512}; epi EPI_LN applies LayerNorm (gamma, beta, eps) over the full row.
-// lda: row stride of A in elements (0: K).
+// lda: row stride of A in elements (0: K).  epi EPI_LNSTAT writes C = (A Wp^T) * gamma and
+// the row moments (mean, rstd) to stats [M][2].
 int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
                     const float* beta, float eps, void* C, int ldc, int32_t* err, cudaStream_t s,
-                    const int32_t* M_dev = nullptr, int lda = 0);
+                    const int32_t* M_dev = nullptr, int lda = 0, float* stats = nullptr);
 
 // 2-D bf16 tensor map over a [rows, cols] row-major matrix (row stride ld elements),
 // box = 64 columns x box_rows rows, 128-byte swizzle, zero fill outside the matrix.

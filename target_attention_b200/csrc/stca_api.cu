@@ -31,6 +31,9 @@ struct stca_handle {
   // a sequence), then all W2 [d, h], then all W_K|W_V [2d, d]
   void* wpack = nullptr;
   int wslots = 0;
+  // LayerNorm folded into the K/V GEMM: per slot c = gamma^T [WK|WV] and b = beta^T [WK|WV]
+  // ([2][2d] fp32), and the row moments of the current layer ([N][2] fp32)
+  float *fold = nullptr, *rowstats = nullptr;
   void *hidden = nullptr, *xt = nullptr, *kv = nullptr;
   // target-side weights packed K-major for the tensor cores (bf16 STCA), element offsets
   void* qpack = nullptr;
@@ -269,6 +272,7 @@ int allocate(stca_handle* h) {
   if (c.dtype == STCA_BF16) {
     h->wslots = c.M * nseq;
     ok = ok && dalloc(h, &h->wpack, size_t(h->wslots) * (2 * hd * d + d * hd + 2 * d * d) * 2);
+    ok = ok && dalloc(h, &h->fold, size_t(h->wslots) * 4 * d * 4) && dalloc(h, &h->rowstats, N * 2 * 4);
   }
   // bf16: the hidden activations of all M layers of every sequence ([N, M h] per sequence)
   const size_t hid_elems = c.dtype == STCA_BF16 ? nseq * N * size_t(c.M) * hd : N * hd;
@@ -424,6 +428,14 @@ void stca_jobs(stca_handle* h, const stca_weights* w, std::vector<PackJob>& jobs
   if (h->qpack) query_jobs(h, w, jobs);
 }
 
+// The fold constants of every history layer's LayerNorm (see EpiFold).
+int stca_folds(stca_handle* h, const stca_weights* w, cudaStream_t s) {
+  const int d = h->cfg.d;
+  for (int i = 0; i < h->cfg.M; ++i)
+    CK(fold_consts(w->hist[i].gamma, w->hist[i].beta, w->WK[i], w->WV[i], d, h->fold + size_t(i) * 4 * d, s));
+  return STCA_OK;
+}
+
 // The decode blocks' operands: per block and sequence the history FFN, W_K|W_V, W_Q and
 // W_O; then the per-token FFNs of query tokens 0 .. tokens-1 of every block.
 void hyf_jobs(stca_handle* h, const hyf_weights* w, int tokens, std::vector<PackJob>& jobs) {
@@ -466,12 +478,24 @@ int history_kv_bf16(stca_handle* h, int sq, int l, int n_tok, const float* gamma
                     size_t(l) * hd;
   GatherSrc none;
   memset(&none, 0, sizeof(none));
+  if (!gamma) {  // no LayerNorm (decode blocks): X~ = A W2
+    STAGE(h, STCA_STAGE_FFN_OUT, s,
+          tc_gemm_rowwise(EPI_PLAIN, hid, n_tok, hd, wp2(h, slot), d, nullptr, nullptr, h->cfg.ln_eps, h->xt, d,
+                          h->err, s, M_dev, M * hd));
+    STAGE(h, STCA_STAGE_KV, s,
+          tc_gemm_resident(A_TMA, EPI_PLAIN, h->xt, none, n_tok, d, wp3(h, slot), 2 * d, h->kv, 2 * d, h->err, s,
+                           M_dev));
+    return STCA_OK;
+  }
+  // X~ = LN(A W2) folded into the K/V GEMM: the LN GEMM writes (A W2) * gamma and the row
+  // moments, the K/V GEMM applies rstd (acc - mean c) + b per row and column
   STAGE(h, STCA_STAGE_FFN_OUT, s,
-        tc_gemm_rowwise(gamma ? EPI_LN : EPI_PLAIN, hid, n_tok, hd, wp2(h, slot), d, gamma, beta, h->cfg.ln_eps, h->xt,
-                        d, h->err, s, M_dev, M * hd));
+        tc_gemm_rowwise(EPI_LNSTAT, hid, n_tok, hd, wp2(h, slot), d, gamma, beta, h->cfg.ln_eps, h->xt, d, h->err,
+                        s, M_dev, M * hd, h->rowstats));
+  const EpiFold fold{h->rowstats, h->fold + size_t(slot) * 4 * d, h->fold + size_t(slot) * 4 * d + 2 * d};
   STAGE(h, STCA_STAGE_KV, s,
-        tc_gemm_resident(A_TMA, EPI_PLAIN, h->xt, none, n_tok, d, wp3(h, slot), 2 * d, h->kv, 2 * d, h->err, s,
-                         M_dev));
+        tc_gemm_resident(A_TMA, EPI_LNFOLD, h->xt, none, n_tok, d, wp3(h, slot), 2 * d, h->kv, 2 * d, h->err, s,
+                         M_dev, nullptr, &fold));
   return STCA_OK;
 }
 
@@ -543,6 +567,7 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
       std::vector<PackJob> jobs;
       stca_jobs(h, w, jobs);
       CK(tc_pack_weights(jobs.data(), int(jobs.size()), s));
+      CK(stca_folds(h, w, s));
     }
   }
   const stca_handle::QLayout& L = h->ql;
@@ -679,6 +704,7 @@ int stca_pin_weights(stca_handle* h, const void* weights, void* stream) {
     const stca_weights* w = static_cast<const stca_weights*>(weights);
     CK(check_weights(h->cfg, w));
     stca_jobs(h, w, jobs);
+    CK(stca_folds(h, w, s));
     bytes = sizeof(*w);
   } else {
     const hyf_weights* w = static_cast<const hyf_weights*>(weights);

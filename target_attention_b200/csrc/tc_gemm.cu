@@ -179,7 +179,8 @@ template <int AMODE, int EPI, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     tc_gemm_resident_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmX,
-                            GatherSrc g, int M_max, int K, int NT, int store_x, int32_t* err, const int32_t* M_dev) {
+                            GatherSrc g, int M_max, int K, int NT, int store_x, int32_t* err, const int32_t* M_dev,
+                            EpiFold fold) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const int KC = K / 64;
@@ -464,12 +465,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
             epi_store(stage, gv, lane, &tmC, nt * 128 + col, y);
           }
         } else {
+          float mean = 0.f, rstd = 1.f;
+          if (EPI == EPI_LNFOLD) {  // row moments of the LayerNorm folded into this GEMM
+            const int row = y + lane;
+            if (row < M) {
+              const float2 st = __ldg(reinterpret_cast<const float2*>(fold.stats) + row);
+              mean = st.x;
+              rstd = st.y;
+            }
+          }
 #pragma unroll 1
           for (int j = 0; j < 4; ++j) {
             const int col = half * 128 + j * 32;
             float v[32];
             tmem_ld_32x32b_x32(tb + col, v);
             tmem_ld_wait();
+            if (EPI == EPI_LNFOLD) {
+              const float4* cv = reinterpret_cast<const float4*>(fold.cvec + nt * 256 + col);
+              const float4* bv = reinterpret_cast<const float4*>(fold.bvec + nt * 256 + col);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 c4 = __ldg(cv + q), b4 = __ldg(bv + q);
+                v[4 * q] = fmaf(rstd, fmaf(-mean, c4.x, v[4 * q]), b4.x);
+                v[4 * q + 1] = fmaf(rstd, fmaf(-mean, c4.y, v[4 * q + 1]), b4.y);
+                v[4 * q + 2] = fmaf(rstd, fmaf(-mean, c4.z, v[4 * q + 2]), b4.z);
+                v[4 * q + 3] = fmaf(rstd, fmaf(-mean, c4.w, v[4 * q + 3]), b4.w);
+              }
+            }
             epi_store(stage, v, lane, &tmC, nt * 256 + col, y);
           }
         }
@@ -499,7 +521,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     tc_gemm_rowwise_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmC, int M_max, int K,
                            const float* __restrict__ gamma, const float* __restrict__ beta, float eps, int32_t* err,
-                           const int32_t* M_dev) {
+                           const int32_t* M_dev, float* __restrict__ stats) {
   constexpr int N = NB * 256;
   constexpr int STAGE_BYTES = A_CHUNK + NB * B_HALF;
   extern __shared__ uint8_t smem_raw[];
@@ -623,7 +645,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     const int et = threadIdx.x - 128;
     constexpr int HN = N / 2;  // columns per epilogue warp
     uint8_t* stage = sOut + (warp - 4) * OUT_STAGE;
-    if (EPI == EPI_LN) {
+    if (EPI == EPI_LN || EPI == EPI_LNSTAT) {
       for (int c = et; c < N; c += 256) {
         s_gamma[c] = gamma[c];
         s_beta[c] = beta[c];
@@ -680,6 +702,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
             for (int e = 0; e < 32; ++e) v[e] = fmaf((v[e] - mean) * rstd, gm[j * 32 + e], bt[j * 32 + e]);
             epi_store(stage, v, lane, &tmC, half * HN + j * 32, y);
           }
+        }
+      } else if (EPI == EPI_LNSTAT) {
+        // one pass: the row moments (shifted by the row's first value c, as above) and
+        // y * gamma stored; the next GEMM applies (mean, rstd) and beta (EpiFold)
+        float s1 = 0.f, s2 = 0.f, c0 = 0.f;
+        if (ok) {
+          {
+            float v[32];
+            tmem_ld_32x32b_x32(tb - half * HN, v);
+            tmem_ld_wait();
+            c0 = v[0];
+          }
+#pragma unroll 1
+          for (int j = 0; j < HN / 32; ++j) {
+            float v[32];
+            tmem_ld_32x32b_x32(tb + j * 32, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float dv = v[e] - c0;
+              s1 += dv;
+              s2 = fmaf(dv, dv, s2);
+              v[e] *= gm[j * 32 + e];
+            }
+            epi_store(stage, v, lane, &tmC, half * HN + j * 32, y);
+          }
+        }
+        s_sum[half * 128 + r] = s1;
+        s_sq[half * 128 + r] = s2;
+        epilogue_sync();
+        if (ok && half == 0 && y + lane < M) {
+          const float m1 = (s_sum[r] + s_sum[128 + r]) * (1.0f / N);
+          const float var = fmaxf((s_sq[r] + s_sq[128 + r]) * (1.0f / N) - m1 * m1, 0.f);
+          reinterpret_cast<float2*>(stats)[y + lane] = make_float2(c0 + m1, rsqrtf(var + eps));
         }
       } else if (ok) {
 #pragma unroll 1
@@ -754,6 +810,25 @@ __global__ void pack_many_kernel(PackJobs jobs) {
   }
 }
 
+// c = gamma^T [WK | WV], b = beta^T [WK | WV]: thread per output column, rows of the
+// [d, d] weights read in order (coalesced across threads)
+__global__ void fold_consts_kernel(const float* __restrict__ gamma, const float* __restrict__ beta,
+                                   const bf16* __restrict__ WK, const bf16* __restrict__ WV, int d,
+                                   float* __restrict__ out) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= 2 * d) return;
+  const bf16* W = c < d ? WK : WV;
+  const int col = c < d ? c : c - d;
+  float sc = 0.f, sb = 0.f;
+  for (int k = 0; k < d; ++k) {
+    const float w = __bfloat162float(W[int64_t(k) * d + col]);
+    sc = fmaf(gamma[k], w, sc);
+    sb = fmaf(beta[k], w, sb);
+  }
+  out[c] = sc;
+  out[2 * d + c] = sb;
+}
+
 // ------------------------------------------------------------------------------------
 // host side
 
@@ -783,26 +858,26 @@ size_t rowwise_smem(int nb, int stages) {
 template <int AMODE, int EPI, int STAGES>
 int run_resident(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tx,
                  int store_x, const GatherSrc& g, int M, int K, int NT, int32_t* err, cudaStream_t s,
-                 const int32_t* M_dev) {
+                 const int32_t* M_dev, const EpiFold& fold) {
   auto kern = tc_gemm_resident_kernel<AMODE, EPI, STAGES>;
   const size_t smem = resident_smem(K, STAGES, AMODE == A_GATHER);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
   const int grid = 2 * std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
-  kern<<<grid, 512, smem, s>>>(ta, tb, tc, tx, g, M, K, NT, store_x, err, M_dev); note_launch();
+  kern<<<grid, 512, smem, s>>>(ta, tb, tc, tx, g, M, K, NT, store_x, err, M_dev, fold); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
 template <int EPI, int NB, int STAGES>
 int run_rowwise(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, int M, int K,
                 const float* gamma, const float* beta, float eps, int32_t* err, cudaStream_t s,
-                const int32_t* M_dev) {
+                const int32_t* M_dev, float* stats) {
   auto kern = tc_gemm_rowwise_kernel<EPI, NB, STAGES>;
   const size_t smem = rowwise_smem(NB, STAGES);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
   const int grid = 2 * std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
-  kern<<<grid, 384, smem, s>>>(ta, tb, tc, M, K, gamma, beta, eps, err, M_dev); note_launch();
+  kern<<<grid, 384, smem, s>>>(ta, tb, tc, M, K, gamma, beta, eps, err, M_dev, stats); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -821,6 +896,15 @@ int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_off
   dim3 grid((N + 31) / 32, (K + 31) / 32), block(32, 8);
   pack_weight_kernel<<<grid, block, 0, s>>>(reinterpret_cast<const bf16*>(W), K, N, reinterpret_cast<bf16*>(dst),
                                             mode, row_offset); note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
+}
+
+int fold_consts(const float* gamma, const float* beta, const void* WK, const void* WV, int d, float* out,
+                cudaStream_t s) {
+  if (!gamma || !beta || !WK || !WV || !out || d <= 0) return STCA_ERR_INVALID_ARG;
+  fold_consts_kernel<<<(2 * d + 255) / 256, 256, 0, s>>>(gamma, beta, reinterpret_cast<const bf16*>(WK),
+                                                         reinterpret_cast<const bf16*>(WV), d, out);
+  note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -844,7 +928,8 @@ int tc_pack_weights(const PackJob* jobs, int n, cudaStream_t s) {
 }
 
 int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int K, const void* Wp, int Nout,
-                     void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev, void* x_out) {
+                     void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev, void* x_out,
+                     const EpiFold* fold) {
   if (M == 0) return 0;
   if (M < 0 || (K != 256 && K != 512) || Nout <= 0 || ldc % 8 != 0) return STCA_ERR_UNSUPPORTED;
   const int N = epi == EPI_SWIGLU ? 2 * Nout : Nout;
@@ -852,6 +937,11 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
   const int NT = N / 256;
   if (reinterpret_cast<uintptr_t>(C) % 16 != 0) return STCA_ERR_INVALID_ARG;
   if (x_out && (amode != A_GATHER || reinterpret_cast<uintptr_t>(x_out) % 16 != 0)) return STCA_ERR_INVALID_ARG;
+  if (epi == EPI_LNFOLD && (!fold || !fold->stats || !fold->cvec || !fold->bvec || amode != A_TMA))
+    return STCA_ERR_INVALID_ARG;
+  EpiFold fz;
+  memset(&fz, 0, sizeof(fz));
+  const EpiFold& fo = fold ? *fold : fz;
   CUtensorMap ta, tb, tc, tx;
   memset(&ta, 0, sizeof(ta));
   if (!make_tmap(&tb, Wp, N, K, K, BM)) return STCA_ERR_CUDA;
@@ -870,9 +960,10 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
   const int sx = x_out != nullptr;
   // stage counts fill the 227 KB of shared memory (see resident_smem)
 #define STCA_RES(AM, EP)                                                                                   \
-  (K == 512 ? run_resident<AM, EP, 5>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev)     \
-            : run_resident<AM, EP, 9>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev))
+  (K == 512 ? run_resident<AM, EP, 5>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev, fo)     \
+            : run_resident<AM, EP, 9>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev, fo))
   if (amode == A_TMA && epi == EPI_PLAIN) return STCA_RES(A_TMA, EPI_PLAIN);
+  if (amode == A_TMA && epi == EPI_LNFOLD) return STCA_RES(A_TMA, EPI_LNFOLD);
   if (amode == A_TMA && epi == EPI_SWIGLU) return STCA_RES(A_TMA, EPI_SWIGLU);
   if (amode == A_GATHER && epi == EPI_PLAIN) return STCA_RES(A_GATHER, EPI_PLAIN);
   if (amode == A_GATHER && epi == EPI_SWIGLU) return STCA_RES(A_GATHER, EPI_SWIGLU);
@@ -882,24 +973,29 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
 
 int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N, const float* gamma,
                     const float* beta, float eps, void* C, int ldc, int32_t* err, cudaStream_t s,
-                    const int32_t* M_dev, int lda) {
+                    const int32_t* M_dev, int lda, float* stats) {
   if (M == 0) return 0;
   if (lda == 0) lda = K;
   if (M < 0 || K <= 0 || K % 64 != 0 || (N != 256 && N != 512) || ldc % 8 != 0 || lda < K || lda % 8 != 0 ||
       reinterpret_cast<uintptr_t>(A) % 16 != 0)
     return STCA_ERR_UNSUPPORTED;
-  if (epi == EPI_LN && (!gamma || !beta)) return STCA_ERR_INVALID_ARG;
+  if ((epi == EPI_LN || epi == EPI_LNSTAT) && (!gamma || !beta)) return STCA_ERR_INVALID_ARG;
+  if (epi == EPI_LNSTAT && (!stats || reinterpret_cast<uintptr_t>(stats) % 8 != 0)) return STCA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(C) % 16 != 0) return STCA_ERR_INVALID_ARG;
   CUtensorMap ta, tb, tc;
   if (!make_tmap(&ta, A, M, K, lda, BM)) return STCA_ERR_CUDA;
   if (!make_tmap(&tb, Wp, N, K, K, BM)) return STCA_ERR_CUDA;
   if (!make_tmap_out(&tc, C, M, N, ldc)) return STCA_ERR_CUDA;
   if (N == 512) {
-    return epi == EPI_LN ? run_rowwise<EPI_LN, 2, 4>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev)
-                         : run_rowwise<EPI_PLAIN, 2, 4>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev);
+    if (epi == EPI_LN) return run_rowwise<EPI_LN, 2, 4>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev, stats);
+    if (epi == EPI_LNSTAT)
+      return run_rowwise<EPI_LNSTAT, 2, 4>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev, stats);
+    return run_rowwise<EPI_PLAIN, 2, 4>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev, stats);
   }
-  return epi == EPI_LN ? run_rowwise<EPI_LN, 1, 6>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev)
-                       : run_rowwise<EPI_PLAIN, 1, 6>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev);
+  if (epi == EPI_LN) return run_rowwise<EPI_LN, 1, 6>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev, stats);
+  if (epi == EPI_LNSTAT)
+    return run_rowwise<EPI_LNSTAT, 1, 6>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev, stats);
+  return run_rowwise<EPI_PLAIN, 1, 6>(ta, tb, tc, M, K, gamma, beta, eps, err, s, M_dev, stats);
 }
 
 }  // namespace stca
