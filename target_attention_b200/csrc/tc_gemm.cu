@@ -810,23 +810,39 @@ __global__ void pack_many_kernel(PackJobs jobs) {
   }
 }
 
-// c = gamma^T [WK | WV], b = beta^T [WK | WV]: thread per output column, rows of the
-// [d, d] weights read in order (coalesced across threads)
-__global__ void fold_consts_kernel(const float* __restrict__ gamma, const float* __restrict__ beta,
-                                   const bf16* __restrict__ WK, const bf16* __restrict__ WV, int d,
-                                   float* __restrict__ out) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= 2 * d) return;
-  const bf16* W = c < d ? WK : WV;
-  const int col = c < d ? c : c - d;
+// c = gamma^T [WK | WV], b = beta^T [WK | WV]: a block of 8 warps per 32 output columns;
+// lane l takes column c0 + l, warp w the rows w, w + 8, ... (reads coalesced across lanes),
+// and the 8 partial sums meet in shared memory
+__global__ void __launch_bounds__(256) fold_consts_kernel(const float* __restrict__ gamma,
+                                                          const float* __restrict__ beta,
+                                                          const bf16* __restrict__ WK, const bf16* __restrict__ WV,
+                                                          int d, float* __restrict__ out) {
+  __shared__ float part[2][8][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int c = blockIdx.x * 32 + lane;
   float sc = 0.f, sb = 0.f;
-  for (int k = 0; k < d; ++k) {
-    const float w = __bfloat162float(W[int64_t(k) * d + col]);
-    sc = fmaf(gamma[k], w, sc);
-    sb = fmaf(beta[k], w, sb);
+  if (c < 2 * d) {
+    const bf16* W = c < d ? WK : WV;
+    const int col = c < d ? c : c - d;
+    for (int k = w; k < d; k += 8) {
+      const float x = __bfloat162float(W[int64_t(k) * d + col]);
+      sc = fmaf(gamma[k], x, sc);
+      sb = fmaf(beta[k], x, sb);
+    }
   }
-  out[c] = sc;
-  out[2 * d + c] = sb;
+  part[0][w][lane] = sc;
+  part[1][w][lane] = sb;
+  __syncthreads();
+  if (w == 0 && c < 2 * d) {
+    float a = 0.f, b = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      a += part[0][i][lane];
+      b += part[1][i][lane];
+    }
+    out[c] = a;
+    out[2 * d + c] = b;
+  }
 }
 
 // ------------------------------------------------------------------------------------
@@ -902,8 +918,8 @@ int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_off
 int fold_consts(const float* gamma, const float* beta, const void* WK, const void* WV, int d, float* out,
                 cudaStream_t s) {
   if (!gamma || !beta || !WK || !WV || !out || d <= 0) return STCA_ERR_INVALID_ARG;
-  fold_consts_kernel<<<(2 * d + 255) / 256, 256, 0, s>>>(gamma, beta, reinterpret_cast<const bf16*>(WK),
-                                                         reinterpret_cast<const bf16*>(WV), d, out);
+  fold_consts_kernel<<<(2 * d + 31) / 32, 256, 0, s>>>(gamma, beta, reinterpret_cast<const bf16*>(WK),
+                                                       reinterpret_cast<const bf16*>(WV), d, out);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
