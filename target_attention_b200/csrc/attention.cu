@@ -55,6 +55,7 @@ constexpr int RING_BYTES = TEAMS * TEAM_BYTES;       // 96 KB
 // K/V row indices and key multiplicities of a team's tiles, copied two tiles ahead of the
 // K/V copies that need them: slots for the tile computed, the tiles in flight and the next
 constexpr int IDX_STAGES = KV_STAGES + 2;
+static_assert(KV_STAGES == 2 || KV_STAGES == 3, "the index copy schedule below is laid out for 2 or 3 stages");
 constexpr int IDX_BYTES = TEAMS * IDX_STAGES * 2 * KT * 4;
 constexpr int ATTN_SMEM = RING_BYTES + IDX_BYTES;    // two CTAs per SM
 
@@ -300,7 +301,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
 #pragma unroll
     for (int p = 0; p < KV_STAGES - 1; ++p) {
       load_kv(p, p);
-      copy_idx(p + KV_STAGES - 1);
+      copy_idx(p + 2);  // indices of tiles 0 and 1 came first
       cp_async_commit();
     }
     int stage = 0;
