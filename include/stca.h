@@ -150,9 +150,12 @@ int stca_forward(stca_handle* h, const int32_t* hist_ids, const int32_t* hist_le
                  void* stream);
 
 /* stca_forward with the per-request inputs and the output in HOST memory (pinned memory
- * makes the copies asynchronous): the library copies the inputs into its workspace,
- * runs the forward on `stream` and copies z back.  Weights and the table stay device
- * pointers.  Returns after enqueueing; synchronise `stream` before reading z_out_host. */
+ * makes the copies asynchronous): the library copies the inputs into one of two staging
+ * slots of its workspace on an internal copy stream (so one call's input copies overlap the
+ * previous call's forward), runs the forward on `stream` once they have landed, and copies
+ * z back on `stream`.  Weights and the table stay device pointers.  Returns after
+ * enqueueing; once `stream` has been synchronised the inputs have been read and
+ * z_out_host holds the result (keep the host inputs unchanged until then). */
 int stca_forward_host(stca_handle* h, const int32_t* hist_ids_host, const int32_t* hist_lengths_host,
                       const int32_t* hist_dt_host, const void* target_emb_host,
                       const int32_t* targets_per_user_host, int B, int n_tok, int t_tot,

@@ -62,10 +62,15 @@ struct stca_handle {
   const void* pinned = nullptr;
   std::vector<uint8_t> pinned_copy;
   int pinned_tokens = 0;
-  // staging for the host-buffer entry point
-  int32_t *in_ids = nullptr, *in_len = nullptr, *in_dt = nullptr, *in_tpu = nullptr;
-  void* in_xt = nullptr;
+  // staging for the host-buffer entry point: two input slots, so the copies of one call's
+  // inputs (on copy_stream) overlap the previous call's forward
+  int32_t *in_ids[2] = {}, *in_len[2] = {}, *in_dt[2] = {}, *in_tpu[2] = {};
+  void* in_xt[2] = {};
   float* out_z = nullptr;
+  cudaStream_t copy_stream = nullptr;
+  cudaEvent_t in_ready[2] = {}, in_free[2] = {};  // slot copied / slot read by its forward
+  bool in_used[2] = {false, false};
+  int in_slot = 0;
   // per-stage timing
   bool prof = false;
   struct Rec {
@@ -292,9 +297,12 @@ int allocate(stca_handle* h) {
   }
   if (c.mode == STCA_MODE_STCA) {
     ok = ok && dalloc(h, &h->cat, T * (c.M + 1) * d * 4) && dalloc(h, &h->qbuf, T * d * 4);
-    ok = ok && dalloc(h, &h->in_ids, N * 4) && dalloc(h, &h->in_len, U * 4) && dalloc(h, &h->in_tpu, U * 4) &&
-         dalloc(h, &h->in_xt, T * d * E) && dalloc(h, &h->out_z, T * d * 4);
-    if (c.time_buckets) ok = ok && dalloc(h, &h->in_dt, N * 4);
+    for (int b = 0; b < 2; ++b) {
+      ok = ok && dalloc(h, &h->in_ids[b], N * 4) && dalloc(h, &h->in_len[b], U * 4) &&
+           dalloc(h, &h->in_tpu[b], U * 4) && dalloc(h, &h->in_xt[b], T * d * E);
+      if (c.time_buckets) ok = ok && dalloc(h, &h->in_dt[b], N * 4);
+    }
+    ok = ok && dalloc(h, &h->out_z, T * d * 4);
     if (c.dtype == STCA_BF16) {
       h->ql = q_layout(c);
       ok = ok && dalloc(h, &h->qpack, h->ql.total * 2);
@@ -744,6 +752,14 @@ void stca_destroy(stca_handle* h) {
   if (!h->recs.empty()) cudaDeviceSynchronize();
   recycle_events(h);
   for (cudaEvent_t e : h->spare) cudaEventDestroy(e);
+  if (h->copy_stream) {
+    cudaStreamSynchronize(h->copy_stream);
+    cudaStreamDestroy(h->copy_stream);
+    for (int b = 0; b < 2; ++b) {
+      cudaEventDestroy(h->in_ready[b]);
+      cudaEventDestroy(h->in_free[b]);
+    }
+  }
   free_all(h);
   delete h;
 }
@@ -773,18 +789,36 @@ int stca_forward_host(stca_handle* h, const int32_t* ids, const int32_t* lens, c
   if (B == 0) return STCA_OK;
   const size_t E = esize(h->cfg);
   const size_t d = size_t(h->cfg.d);
-  bool ok = cudaMemcpyAsync(h->in_len, lens, size_t(B) * 4, cudaMemcpyHostToDevice, s) == cudaSuccess &&
-            cudaMemcpyAsync(h->in_tpu, tpu, size_t(B) * 4, cudaMemcpyHostToDevice, s) == cudaSuccess;
-  if (n_tok > 0) ok = ok && cudaMemcpyAsync(h->in_ids, ids, size_t(n_tok) * 4, cudaMemcpyHostToDevice, s) == cudaSuccess;
+  if (!h->copy_stream) {
+    bool made = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking) == cudaSuccess;
+    for (int b = 0; b < 2; ++b)
+      made = made && cudaEventCreateWithFlags(&h->in_ready[b], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&h->in_free[b], cudaEventDisableTiming) == cudaSuccess;
+    if (!made) return STCA_ERR_CUDA;
+  }
+  // this call's inputs go to slot b on the copy stream, once the forward that read slot b
+  // two calls ago is done; the forward on s waits for them
+  const int b = h->in_slot;
+  cudaStream_t c = h->copy_stream;
+  bool ok = !h->in_used[b] || cudaStreamWaitEvent(c, h->in_free[b], 0) == cudaSuccess;
+  ok = ok && cudaMemcpyAsync(h->in_len[b], lens, size_t(B) * 4, cudaMemcpyHostToDevice, c) == cudaSuccess &&
+       cudaMemcpyAsync(h->in_tpu[b], tpu, size_t(B) * 4, cudaMemcpyHostToDevice, c) == cudaSuccess;
+  if (n_tok > 0) ok = ok && cudaMemcpyAsync(h->in_ids[b], ids, size_t(n_tok) * 4, cudaMemcpyHostToDevice, c) == cudaSuccess;
   if (n_tok > 0 && h->cfg.time_buckets)
-    ok = ok && cudaMemcpyAsync(h->in_dt, dt, size_t(n_tok) * 4, cudaMemcpyHostToDevice, s) == cudaSuccess;
-  if (t_tot > 0) ok = ok && cudaMemcpyAsync(h->in_xt, x_t, size_t(t_tot) * d * E, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    ok = ok && cudaMemcpyAsync(h->in_dt[b], dt, size_t(n_tok) * 4, cudaMemcpyHostToDevice, c) == cudaSuccess;
+  if (t_tot > 0)
+    ok = ok && cudaMemcpyAsync(h->in_xt[b], x_t, size_t(t_tot) * d * E, cudaMemcpyHostToDevice, c) == cudaSuccess;
+  ok = ok && cudaEventRecord(h->in_ready[b], c) == cudaSuccess && cudaStreamWaitEvent(s, h->in_ready[b], 0) == cudaSuccess;
   if (!ok) return STCA_ERR_CUDA;
+  h->in_slot ^= 1;
   const int rc = h->cfg.dtype == STCA_BF16
-                     ? run_stca<bf16>(h, h->in_ids, h->in_len, h->in_dt, h->in_xt, h->in_tpu, B, n_tok, t_tot, w,
-                                      h->out_z, nullptr, s)
-                     : run_stca<float>(h, h->in_ids, h->in_len, h->in_dt, h->in_xt, h->in_tpu, B, n_tok, t_tot, w,
-                                       h->out_z, nullptr, s);
+                     ? run_stca<bf16>(h, h->in_ids[b], h->in_len[b], h->in_dt[b], h->in_xt[b], h->in_tpu[b], B, n_tok,
+                                      t_tot, w, h->out_z, nullptr, s)
+                     : run_stca<float>(h, h->in_ids[b], h->in_len[b], h->in_dt[b], h->in_xt[b], h->in_tpu[b], B,
+                                       n_tok, t_tot, w, h->out_z, nullptr, s);
+  // slot b is free for the call after next once this forward has read it (recorded even
+  // when the forward returned early, so that call never waits on a stale event)
+  h->in_used[b] = cudaEventRecord(h->in_free[b], s) == cudaSuccess;
   CK(rc);
   if (t_tot > 0 && cudaMemcpyAsync(z_host, h->out_z, size_t(t_tot) * d * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return STCA_ERR_CUDA;

@@ -135,6 +135,30 @@ def test_host_buffer_entry_matches_device_entry():
     m.close()
 
 
+def test_host_buffer_entry_back_to_back_calls():
+    """Host-buffer calls with different inputs, enqueued back to back with no synchronisation
+    between them (the inputs alternate between two staging slots while the previous forward
+    runs): each result equals the device entry's for the same inputs."""
+    wl = make_stca(3, users=3, L=400, n_items=10_000)
+    m = StcaModel(wl)
+    inputs = [m.inputs(make_stca(3, users=3, L=400, n_items=10_000, data_seed=100 + i)) for i in range(5)]
+    want = []
+    for x in inputs:
+        z = torch.empty((x["t_tot"], 512), device=dev)
+        B.check(m.forward(x, z))
+        want.append(z.cpu().numpy())
+    hosts = [{k: (v.cpu().pin_memory() if torch.is_tensor(v) else v) for k, v in x.items()} for x in inputs]
+    outs = [torch.full((x["t_tot"], 512), float("nan"), pin_memory=True) for x in inputs]
+    torch.cuda.synchronize()
+    for xh, zh in zip(hosts, outs):
+        B.check(m.forward_host(xh, zh))
+    torch.cuda.synchronize()
+    assert B.stca_sync_status(m.handle) == B.OK
+    for zh, w in zip(outs, want):
+        np.testing.assert_array_equal(zh.numpy(), w)
+    m.close()
+
+
 # ---------------------------------------------------------------- pointwise ReLU TA
 
 
