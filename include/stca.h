@@ -161,6 +161,36 @@ int stca_forward_host(stca_handle* h, const int32_t* hist_ids_host, const int32_
                       const int32_t* targets_per_user_host, int B, int n_tok, int t_tot,
                       const stca_weights* w, float* z_out_host, void* stream);
 
+/* Sequence-parallel (L-split) forward, in phases, for histories split across R ranks (one
+ * GPU each).  Attention over a history is a merge of attention over its slices: each slice
+ * keeps its running max m, sum l and weighted sum acc of V, and the slices combine exactly
+ * ([wechat] §1.1, local attention then merge).  Every rank calls, on its own handle:
+ *
+ *   stca_lsplit_begin   with ITS slice of every user's history (hist_lengths = the slice
+ *                       lengths, zeros allowed; ids/dt of the slices back to back) and ALL
+ *                       of the users' targets (the same on every rank);
+ *   for layer i = 0 .. M-1:
+ *     stca_lsplit_partial(i, acc, ml)   this rank's attention state of layer i:
+ *                       acc [t_tot, d] fp32, unnormalised sum of weights x V per head
+ *                       ml  [t_tot, H, 2] fp32, (max in log2 units, sum of weights) per
+ *                       target and head (softmax; not written for the ReLU score)
+ *     the caller gathers acc and ml of all ranks in rank order: all_acc [R, t_tot, d],
+ *                       all_ml [R, t_tot, H, 2] (e.g. an NCCL all-gather on `stream`)
+ *     stca_lsplit_merge(i, R, all_acc, all_ml, z_out)   merges the R states into o^(i),
+ *                       then q^(i+1), and after the last layer z [t_tot, d] into z_out
+ *
+ * Everything but the attention is computed on every rank (the target side is small).
+ * The phases must come in this order; another order returns STCA_ERR_INVALID_ARG, and a
+ * stca_forward on the handle closes an open sequence-parallel forward.  The device
+ * pointers given to stca_lsplit_begin (ids, dt, lengths, target rows, weights) must stay
+ * valid until the last merge.  1 <= R <= 32. */
+int stca_lsplit_begin(stca_handle* h, const int32_t* hist_ids, const int32_t* hist_lengths,
+                      const int32_t* hist_dt, const void* target_emb, const int32_t* targets_per_user,
+                      int B, int n_tok, int t_tot, const stca_weights* w, void* stream);
+int stca_lsplit_partial(stca_handle* h, int layer, float* acc, float* ml, void* stream);
+int stca_lsplit_merge(stca_handle* h, int layer, int ranks, const float* all_acc, const float* all_ml,
+                      float* z_out, void* stream);
+
 /* Pointwise ReLU target attention with fused lookup ([wechat] §1.1 low-memory TA
  * operator, §1.2 ReLU scores): for each sample b,
  *   out[b] = sum_{j < L_b} relu(q_b . e_j / sqrt(D)) e_j,   e_j = table[ids_b[j]]

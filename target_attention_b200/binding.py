@@ -76,6 +76,9 @@ _SIGS = [
                             _vp]),
     ("stca_forward_host", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.POINTER(StcaWeights), _vp,
                                  _vp]),
+    ("stca_lsplit_begin", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.POINTER(StcaWeights), _vp]),
+    ("stca_lsplit_partial", _i32, [_vp, _i32, _vp, _vp, _vp]),
+    ("stca_lsplit_merge", _i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     ("stca_pointwise_forward", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp]),
     ("stca_pointwise_forward_noalloc", _i32, [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp]),
     ("hyformer_forward", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, ctypes.POINTER(HyfWeights),
@@ -201,6 +204,19 @@ def stca_forward_host(h, ids, lengths, dt, x_t, tpu, B, n_tok, t_tot, weights: S
                       stream=None) -> int:
     return lib().stca_forward_host(h, ptr(ids), ptr(lengths), ptr(dt), ptr(x_t), ptr(tpu), B, n_tok, t_tot,
                                    ctypes.byref(weights), ptr(z_out), stream_ptr(stream))
+
+
+def stca_lsplit_begin(h, ids, lengths, dt, x_t, tpu, B, n_tok, t_tot, weights: StcaWeights, stream=None) -> int:
+    return lib().stca_lsplit_begin(h, ptr(ids), ptr(lengths), ptr(dt), ptr(x_t), ptr(tpu), B, n_tok, t_tot,
+                                   ctypes.byref(weights), stream_ptr(stream))
+
+
+def stca_lsplit_partial(h, layer, acc, ml, stream=None) -> int:
+    return lib().stca_lsplit_partial(h, layer, ptr(acc), ptr(ml), stream_ptr(stream))
+
+
+def stca_lsplit_merge(h, layer, ranks, all_acc, all_ml, z_out, stream=None) -> int:
+    return lib().stca_lsplit_merge(h, layer, ranks, ptr(all_acc), ptr(all_ml), ptr(z_out), stream_ptr(stream))
 
 
 def stca_pointwise_forward(h, ids, lengths, q, table, n_items, B, n_tok, out, stream=None) -> int:

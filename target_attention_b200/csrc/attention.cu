@@ -383,7 +383,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
           }
         }
         // one slice: the state is final, so write the normalised output (no merge pass)
-        const bool direct = a.splits == 1;
+        const bool direct = a.splits == 1 && !a.partial_out;
         const float scale = (SCORE == 0 && direct) ? (Lsum > 0.f ? 1.f / Lsum : 0.f) : 1.f;
         float v[8];
 #pragma unroll
@@ -510,7 +510,7 @@ __global__ void attn_merge_kernel(AttnArgs a) {
   const int t = int(wid / a.H), h = int(wid % a.H);
   const int dh = a.d / a.H;
   const int S = a.splits;
-  float w = 0.f, inv = 1.f;
+  float w = 0.f, inv = 1.f, M = -INFINITY, Lsum = 0.f;
   if (SCORE == 0) {
     float m = -INFINITY, l = 0.f;
     if (lane < S) {
@@ -518,11 +518,11 @@ __global__ void attn_merge_kernel(AttnArgs a) {
       m = ml.x;
       l = ml.y;
     }
-    float M = m;
+    M = m;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     w = (m == -INFINITY) ? 0.f : exp2f(m - M);
-    float Lsum = w * l;
+    Lsum = w * l;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
     inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
@@ -543,7 +543,12 @@ __global__ void attn_merge_kernel(AttnArgs a) {
       v += __shfl_sync(0xffffffffu, w, s + 3) * x3;
     }
     for (; s < S; ++s) v += __shfl_sync(0xffffffffu, w, s) * acc[s * slice + c];
-    a.out[int64_t(t) * a.d + h * dh + c] = SCORE == 0 ? v * inv : v;
+    // one combined state (unnormalised, with its max and sum), or the output
+    a.out[int64_t(t) * a.d + h * dh + c] = (SCORE == 0 && !a.ml_out) ? v * inv : v;
+  }
+  if (SCORE == 0 && a.ml_out && lane == 0) {
+    float2* ml = reinterpret_cast<float2*>(a.ml_out + (int64_t(t) * a.H + h) * 2);
+    *ml = make_float2(M, Lsum);
   }
 }
 

@@ -149,12 +149,19 @@ struct AttnArgs {
   float* part_ml;       // [splits, T, H, 2]
   float* out;           // [T, d]
   int32_t* err;
+  // attention: write the slice states (part_acc, part_ml) even when splits == 1
+  int partial_out = 0;
+  // merge: when set, combine the slices into ONE state instead of the output: out gets
+  // the unnormalised acc and ml_out [T, H, 2] the (max, sum) of the softmax
+  float* ml_out = nullptr;
 };
 int attention_bf16(const AttnArgs& a, cudaStream_t s);
 int attention_f32(const AttnArgs& a, cudaStream_t s);
 // combines the slices; not needed after attention_bf16 with splits == 1, which writes out
 int attention_merge(const AttnArgs& a, cudaStream_t s);
-inline bool attention_needs_merge(const AttnArgs& a, bool kv_bf16) { return !(kv_bf16 && a.splits == 1); }
+inline bool attention_needs_merge(const AttnArgs& a, bool kv_bf16) {
+  return !(kv_bf16 && a.splits == 1 && !a.partial_out);
+}
 // streaming multiprocessors of the current device
 int sm_count();
 

@@ -71,6 +71,15 @@ struct stca_handle {
   cudaEvent_t in_ready[2] = {}, in_free[2] = {};  // slot copied / slot read by its forward
   bool in_used[2] = {false, false};
   int in_slot = 0;
+  // one STCA forward between its phases (set by its first phase)
+  struct Fwd {
+    int B = 0, n_tok = 0, t_tot = 0, splits = 1;
+    const stca_weights* w = nullptr;
+    GatherSrc g{};
+    const int32_t *M_dev = nullptr, *kv_rows = nullptr, *kv_len = nullptr, *kv_mult = nullptr;
+    int next_layer = -1;  // sequence-parallel forward: next layer to run, -1 when none is open
+    bool partial_done = false;
+  } fwd;
   // per-stage timing
   bool prof = false;
   struct Rec {
@@ -558,10 +567,11 @@ int run_attention(stca_handle* h, const float* Q, const int32_t* hoff, const int
   return STCA_OK;
 }
 
+// First phase of an STCA forward: offsets, targets into the concatenation buffer, weights
+// converted (unless pinned), q^(1) = LN(SwiGLU_t(x_t)), distinct keys; fills h->fwd.
 template <typename TB>
-int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int32_t* dt, const void* x_t,
-             const int32_t* tpu, int B, int n_tok, int t_tot, const stca_weights* w, float* z_out, float* o_out,
-             cudaStream_t s) {
+int fwd_begin(stca_handle* h, const int32_t* ids, const int32_t* lens, const int32_t* dt, const void* x_t,
+              const int32_t* tpu, int B, int n_tok, int t_tot, const stca_weights* w, cudaStream_t s) {
   const stca_config& c = h->cfg;
   const int d = c.d, M = c.M;
   const bool bf = c.dtype == STCA_BF16;
@@ -583,45 +593,69 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
   // q^(1) = LN(SwiGLU_t(x_t))
   STAGE(h, STCA_STAGE_QUERY, s,
         query_ffn<TB>(h, xcol, ldcat, t_tot, w->tgt, h->qbuf, d, s, qp(h, L.tgt13), qp(h, L.tgt2)));
-  GatherSrc g;
-  memset(&g, 0, sizeof(g));
-  g.ids = ids;
-  g.dt = c.time_buckets ? dt : nullptr;
-  g.table = w->table;
-  g.dt_table = c.time_buckets ? w->dt_table : nullptr;
-  g.n_items = w->n_items;
-  const int32_t* M_dev = nullptr;
-  const int32_t* kv_rows = nullptr;
+  stca_handle::Fwd& f = h->fwd;
+  f = stca_handle::Fwd{};
+  f.B = B;
+  f.n_tok = n_tok;
+  f.t_tot = t_tot;
+  f.w = w;
+  f.g.ids = ids;
+  f.g.dt = c.time_buckets ? dt : nullptr;
+  f.g.table = w->table;
+  f.g.dt_table = c.time_buckets ? w->dt_table : nullptr;
+  f.g.n_items = w->n_items;
   if (c.dedup) {
     STAGE(h, STCA_STAGE_DEDUP, s,
-          dedup_rows(ids, g.dt, n_tok, h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx, h->uniq_token, h->uniq_count,
+          dedup_rows(ids, f.g.dt, n_tok, h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx, h->uniq_token, h->uniq_count,
                      h->err, s));
-    g.rows = h->uniq_token;
-    M_dev = h->uniq_count;
-    kv_rows = h->uniq_idx;
+    f.g.rows = h->uniq_token;
+    f.M_dev = h->uniq_count;
+    f.kv_rows = h->uniq_idx;
     if (c.dedup == 2) {
       // attention over each user's distinct rows, each weighted by its token count
       STAGE(h, STCA_STAGE_DEDUP, s, compact_user_rows(h->hoff, B, h->uniq_idx, h->c_rows, h->c_mult, h->c_len, s));
-      kv_rows = h->c_rows;
+      f.kv_rows = h->c_rows;
+      f.kv_len = h->c_len;
+      f.kv_mult = h->c_mult;
     }
   }
-  const int32_t* kv_len = c.dedup == 2 ? h->c_len : nullptr;
-  const int32_t* kv_mult = c.dedup == 2 ? h->c_mult : nullptr;
-  const int splits = attention_splits(n_tok, B, c.H, 1024);
-  for (int i = 0; i < M; ++i) {
-    if (bf) {
-      if (i == 0) CK(history_hidden_bf16(h, 0, g, n_tok, s, M_dev));
-      CK(history_kv_bf16(h, 0, i, n_tok, w->hist[i].gamma, w->hist[i].beta, s, M_dev));
-    }
-    else CK(history_f32(h, g, n_tok, w->hist[i], w->WK[i], w->WV[i], s));
-    STAGE(h, STCA_STAGE_QUERY, s,
-          qgemm(gemm_args<TB>(t_tot, d, d, h->qbuf, d, w->WQ[i], h->qproj, d, h->err), qp(h, L.wq[i]), s));
-    CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, splits, c.score, s, kv_rows, kv_len, kv_mult));
+  f.splits = attention_splits(n_tok, B, c.H, 1024);
+  return STCA_OK;
+}
+
+// Layer i up to the attention: the history side (K/V of every key) and Q^(i) = q^(i) W_Q.
+template <typename TB>
+int fwd_layer_inputs(stca_handle* h, int i, cudaStream_t s) {
+  const stca_config& c = h->cfg;
+  const stca_handle::Fwd& f = h->fwd;
+  const stca_weights* w = f.w;
+  if (c.dtype == STCA_BF16) {
+    if (i == 0) CK(history_hidden_bf16(h, 0, f.g, f.n_tok, s, f.M_dev));
+    CK(history_kv_bf16(h, 0, i, f.n_tok, w->hist[i].gamma, w->hist[i].beta, s, f.M_dev));
+  } else {
+    CK(history_f32(h, f.g, f.n_tok, w->hist[i], w->WK[i], w->WV[i], s));
+  }
+  STAGE(h, STCA_STAGE_QUERY, s,
+        qgemm(gemm_args<TB>(f.t_tot, c.d, c.d, h->qbuf, c.d, w->WQ[i], h->qproj, c.d, h->err), qp(h, h->ql.wq[i]), s));
+  return STCA_OK;
+}
+
+// Layer i after the attention (heads in h->attn): o^(i) = [o_1 .. o_H] W_O into the
+// concatenation buffer, then q^(i+2) = LN(SwiGLU([o^(1) .. o^(i+1) | x_t] W_C)), or after
+// the last layer z = SwiGLU_Z([o^(1) .. o^(M) | x_t] W_Z).
+template <typename TB>
+int fwd_layer_outputs(stca_handle* h, int i, float* z_out, cudaStream_t s) {
+  const stca_config& c = h->cfg;
+  const stca_handle::Fwd& f = h->fwd;
+  const stca_weights* w = f.w;
+  const stca_handle::QLayout& L = h->ql;
+  const int d = c.d, M = c.M, t_tot = f.t_tot;
+  const int64_t ldcat = int64_t(M + 1) * d;
+  {
     Prof p(h, STCA_STAGE_QUERY, s);
     CK(qgemm(gemm_args<TB>(t_tot, d, d, h->attn, d, w->WO[i], h->cat + int64_t(i) * d, ldcat, h->err),
              qp(h, L.wo[i]), s));
     if (i + 1 < M) {
-      // q^(i+2) = LN(SwiGLU([o^(1) .. o^(i+1) | x_t] W_C))
       const int K = (i + 2) * d;
       auto a = gemm_args<TB>(t_tot, d, K, h->cat, ldcat, w->WC[i + 1], h->tmp_d, d, h->err);
       a.ksplit = (i + 1) * d;
@@ -631,11 +665,28 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
                        qp(h, L.fuse2[i + 1])));
     }
   }
-  // z = SwiGLU_Z([o^(1) .. o^(M) | x_t] W_Z)
-  {
+  if (i + 1 == M) {
     Prof p(h, STCA_STAGE_QUERY, s);
     CK(qgemm(gemm_args<TB>(t_tot, d, int(ldcat), h->cat, ldcat, w->WZ, h->tmp_d, d, h->err), qp(h, L.wz), s));
     CK(query_ffn<TB>(h, h->tmp_d, d, t_tot, w->zffn, z_out, d, s, qp(h, L.z13), qp(h, L.z2)));
+  }
+  return STCA_OK;
+}
+
+template <typename TB>
+int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int32_t* dt, const void* x_t,
+             const int32_t* tpu, int B, int n_tok, int t_tot, const stca_weights* w, float* z_out, float* o_out,
+             cudaStream_t s) {
+  const stca_config& c = h->cfg;
+  const int d = c.d, M = c.M;
+  const int64_t ldcat = int64_t(M + 1) * d;
+  h->fwd.next_layer = -1;  // a whole forward closes any open sequence-parallel one
+  CK(fwd_begin<TB>(h, ids, lens, dt, x_t, tpu, B, n_tok, t_tot, w, s));
+  const stca_handle::Fwd& f = h->fwd;
+  for (int i = 0; i < M; ++i) {
+    CK(fwd_layer_inputs<TB>(h, i, s));
+    CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, f.splits, c.score, s, f.kv_rows, f.kv_len, f.kv_mult));
+    CK(fwd_layer_outputs<TB>(h, i, z_out, s));
   }
   if (o_out && t_tot > 0) {
     for (int i = 0; i < M; ++i)
@@ -647,13 +698,15 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
 }
 
 int check_forward_args(stca_handle* h, const int32_t* ids, const int32_t* lens, const int32_t* dt, const void* x_t,
-                       const int32_t* tpu, int B, int n_tok, int t_tot, const stca_weights* w, const float* z) {
+                       const int32_t* tpu, int B, int n_tok, int t_tot, const stca_weights* w, const float* z,
+                       bool need_z = true) {
   if (!h) return STCA_ERR_INVALID_ARG;
   const stca_config& c = h->cfg;
   if (c.mode != STCA_MODE_STCA) return STCA_ERR_INVALID_ARG;
   if (B < 0 || n_tok < 0 || t_tot < 0) return STCA_ERR_INVALID_ARG;
   if (B > c.max_users || n_tok > c.max_tokens || t_tot > c.max_targets) return STCA_ERR_CAPACITY;
-  if ((B > 0 && (!lens || !tpu)) || (n_tok > 0 && !ids) || (t_tot > 0 && (!x_t || !z))) return STCA_ERR_INVALID_ARG;
+  if ((B > 0 && (!lens || !tpu)) || (n_tok > 0 && !ids) || (t_tot > 0 && (!x_t || (need_z && !z))))
+    return STCA_ERR_INVALID_ARG;
   if (c.time_buckets && n_tok > 0 && !dt) return STCA_ERR_INVALID_ARG;
   return check_weights(c, w);
 }
@@ -822,6 +875,101 @@ int stca_forward_host(stca_handle* h, const int32_t* ids, const int32_t* lens, c
   CK(rc);
   if (t_tot > 0 && cudaMemcpyAsync(z_host, h->out_z, size_t(t_tot) * d * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return STCA_ERR_CUDA;
+  return STCA_OK;
+}
+
+// ---- sequence-parallel (L-split) forward in phases: every rank holds a slice of each
+// user's history and all of the user's targets; per layer the slices' attention states are
+// exchanged by the caller and merged here ([wechat] §1.1: local attentions merge exactly).
+
+int stca_lsplit_begin(stca_handle* h, const int32_t* hist_ids, const int32_t* hist_lengths, const int32_t* hist_dt,
+                      const void* target_emb, const int32_t* targets_per_user, int B, int n_tok, int t_tot,
+                      const stca_weights* w, void* stream) {
+  CK(check_forward_args(h, hist_ids, hist_lengths, hist_dt, target_emb, targets_per_user, B, n_tok, t_tot, w,
+                        nullptr, false));
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  h->fwd.next_layer = -1;
+  CK(h->cfg.dtype == STCA_BF16
+         ? fwd_begin<bf16>(h, hist_ids, hist_lengths, hist_dt, target_emb, targets_per_user, B, n_tok, t_tot, w, s)
+         : fwd_begin<float>(h, hist_ids, hist_lengths, hist_dt, target_emb, targets_per_user, B, n_tok, t_tot, w, s));
+  h->fwd.next_layer = 0;
+  h->fwd.partial_done = false;
+  return STCA_OK;
+}
+
+int stca_lsplit_partial(stca_handle* h, int layer, float* acc, float* ml, void* stream) {
+  if (!h || h->cfg.mode != STCA_MODE_STCA) return STCA_ERR_INVALID_ARG;
+  stca_handle::Fwd& f = h->fwd;
+  if (f.next_layer < 0 || layer != f.next_layer || f.partial_done) return STCA_ERR_INVALID_ARG;
+  if (f.t_tot > 0 && (!acc || (h->cfg.score == 0 && !ml))) return STCA_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  const bool bf = h->cfg.dtype == STCA_BF16;
+  CK(bf ? fwd_layer_inputs<bf16>(h, layer, s) : fwd_layer_inputs<float>(h, layer, s));
+  AttnArgs a;
+  a.Q = h->qproj;
+  a.KV = h->kv;
+  a.hoff = h->hoff;
+  a.toff = h->toff;
+  a.kv_rows = f.kv_rows;
+  a.kv_len = f.kv_len;
+  a.kv_mult = f.kv_mult;
+  a.B = f.B;
+  a.T = f.t_tot;
+  a.d = h->cfg.d;
+  a.H = h->cfg.H;
+  a.splits = f.splits;
+  a.score = h->cfg.score;
+  a.err = h->err;
+  if (bf && f.splits == 1) {  // the one slice's state straight into the caller's buffers
+    a.part_acc = acc;
+    a.part_ml = ml;
+    a.out = nullptr;
+    a.partial_out = 1;
+    STAGE(h, STCA_STAGE_ATTENTION, s, attention_bf16(a, s));
+  } else {  // this rank's slices, combined into one state
+    a.part_acc = h->part_acc;
+    a.part_ml = h->part_ml;
+    a.out = h->attn;
+    STAGE(h, STCA_STAGE_ATTENTION, s, bf ? attention_bf16(a, s) : attention_f32(a, s));
+    a.out = acc;
+    a.ml_out = h->cfg.score == 0 ? ml : nullptr;
+    STAGE(h, STCA_STAGE_MERGE, s, attention_merge(a, s));
+  }
+  f.partial_done = true;
+  return STCA_OK;
+}
+
+int stca_lsplit_merge(stca_handle* h, int layer, int ranks, const float* all_acc, const float* all_ml, float* z_out,
+                      void* stream) {
+  if (!h || h->cfg.mode != STCA_MODE_STCA) return STCA_ERR_INVALID_ARG;
+  stca_handle::Fwd& f = h->fwd;
+  if (f.next_layer < 0 || layer != f.next_layer || !f.partial_done) return STCA_ERR_INVALID_ARG;
+  if (ranks < 1 || ranks > 32) return STCA_ERR_INVALID_ARG;
+  const bool last = layer + 1 == h->cfg.M;
+  if (f.t_tot > 0 && (!all_acc || (h->cfg.score == 0 && !all_ml) || (last && !z_out))) return STCA_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  h->last_stream = s;
+  AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.T = f.t_tot;
+  a.d = h->cfg.d;
+  a.H = h->cfg.H;
+  a.splits = ranks;
+  a.score = h->cfg.score;
+  a.part_acc = const_cast<float*>(all_acc);
+  a.part_ml = const_cast<float*>(all_ml);
+  a.out = h->attn;
+  a.err = h->err;
+  STAGE(h, STCA_STAGE_MERGE, s, attention_merge(a, s));
+  const bool bf = h->cfg.dtype == STCA_BF16;
+  CK(bf ? fwd_layer_outputs<bf16>(h, layer, z_out, s) : fwd_layer_outputs<float>(h, layer, z_out, s));
+  f.partial_done = false;
+  f.next_layer = last ? -1 : layer + 1;
   return STCA_OK;
 }
 

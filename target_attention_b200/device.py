@@ -102,6 +102,32 @@ class StcaModel(_Holder):
         return B.stca_forward(handle or self.handle, x["ids"], x["lengths"], x["dt"], x["x_t"], x["targets_per_user"],
                               x["B"], x["n_tok"], x["t_tot"], self.weights, z_out, o_out, stream)
 
+    def slice_inputs(self, wl, ranks, rank):
+        """Inputs of rank ``rank`` of a sequence-parallel forward: its slice of every user's
+        history (``lsplit.slice_histories``) and all of the targets."""
+        from .lsplit import slice_histories
+
+        lens, ids, dt = slice_histories(wl["lengths"], wl["ids"], wl["dt"], ranks, rank)
+        d = {"ids": to_device(ids, self.device), "lengths": to_device(lens, self.device),
+             "dt": to_device(dt, self.device), "x_t": to_device(wl["x_t"], self.device),
+             "targets_per_user": to_device(wl["targets_per_user"], self.device)}
+        d["B"] = len(lens)
+        d["n_tok"] = int(lens.sum())
+        d["t_tot"] = int(wl["targets_per_user"].sum())
+        return d
+
+    def lsplit_engine(self, x, z_out, stream=None):
+        """The library's sequence-parallel phases for this rank's inputs ``x`` (see
+        ``lsplit.run_phases``)."""
+        return _LsplitEngine(self, x, z_out, stream)
+
+    def forward_lsplit(self, x, z_out, gather, stream=None):
+        """Sequence-parallel forward of this rank's slice ``x``; ``gather`` exchanges the
+        per-layer attention states (``lsplit.all_gather_fn``)."""
+        from .lsplit import run_phases
+
+        return run_phases(self.lsplit_engine(x, z_out, stream), self.cfg["M"], gather)
+
     def forward_host(self, x, z_out, stream=None):
         return B.stca_forward_host(self.handle, x["ids"], x["lengths"], x["dt"], x["x_t"], x["targets_per_user"],
                                    x["B"], x["n_tok"], x["t_tot"], self.weights, z_out, stream)
@@ -112,6 +138,36 @@ class StcaModel(_Holder):
             self.handle = None
 
     __del__ = close
+
+
+class _LsplitEngine:
+    """One rank's side of a sequence-parallel forward: stca_lsplit_begin, then per layer
+    stca_lsplit_partial into (acc [t_tot, d], ml [t_tot, H, 2]) and stca_lsplit_merge of
+    all ranks' states; z lands in z_out after the last layer."""
+
+    def __init__(self, model, x, z_out, stream):
+        self.m, self.x, self.z, self.stream = model, x, z_out, stream
+        c = model.cfg
+        T = x["t_tot"]
+        self.acc = torch.empty((T, c["d"]), device=model.device)
+        self.ml = torch.empty((T, c["H"], 2), device=model.device)
+
+    def begin(self):
+        x = self.x
+        B.check(B.stca_lsplit_begin(self.m.handle, x["ids"], x["lengths"], x["dt"], x["x_t"], x["targets_per_user"],
+                                    x["B"], x["n_tok"], x["t_tot"], self.m.weights, self.stream), "stca_lsplit_begin")
+
+    def partial(self, i):
+        B.check(B.stca_lsplit_partial(self.m.handle, i, self.acc, self.ml, self.stream), "stca_lsplit_partial")
+        return self.acc, self.ml
+
+    def merge(self, i, all_acc, all_ml):
+        last = i + 1 == self.m.cfg["M"]
+        B.check(B.stca_lsplit_merge(self.m.handle, i, all_acc.shape[0], all_acc, all_ml, self.z if last else None,
+                                    self.stream), "stca_lsplit_merge")
+
+    def result(self):
+        return self.z
 
 
 class PointwiseModel(_Holder):

@@ -87,6 +87,10 @@ def test_null_arguments_rejected_on_host():
     assert L.stca_pointwise_forward(None, None, None, None, None, 1, 1, 1, None, None) == B.ERR_INVALID_ARG
     assert L.stca_sync_status(None) == B.ERR_INVALID_ARG
     assert L.stca_pin_weights(None, None, None) == B.ERR_INVALID_ARG
+    assert L.stca_lsplit_begin(None, None, None, None, None, None, 1, 1, 1, ctypes.byref(w), None) \
+        == B.ERR_INVALID_ARG
+    assert L.stca_lsplit_partial(None, 0, None, None, None) == B.ERR_INVALID_ARG
+    assert L.stca_lsplit_merge(None, 0, 2, None, None, None, None) == B.ERR_INVALID_ARG
     L.stca_unpin_weights(None)
     L.stca_destroy(None)
     # kernel-level entry points validate before launching
