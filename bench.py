@@ -61,6 +61,22 @@ def dist_info():
     return rank, world, local
 
 
+def rank_data_seed(workload, rank):
+    """Seed of rank ``rank``'s requests: every rank serves its own users (same shapes)."""
+    return 1000 + workload + 7919 * rank
+
+
+def reduce_over_ranks(v, world, op="max", device="cuda"):
+    """max (timings) or sum (work) of a per-rank number over all ranks (every rank gets it)."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -97,12 +113,12 @@ def history_tokens(wl):
     return int(wl["lengths"].sum())
 
 
-def config_block(wl, world):
+def config_block(wl, world, total_tokens=None):
     c = wl["cfg"]
     users = len(wl["lengths"][0]) if c["kind"] == "hyformer" else len(wl["lengths"])
     n_tok = history_tokens(wl)
     common = {"users_per_gpu": users, "global_batch_users": users * world, "n_items": c["n_items"], "d": c["d"],
-              "history_tokens_per_step": n_tok * world,
+              "history_tokens_per_step": int(total_tokens if total_tokens is not None else n_tok * world),
               "parallelism": f"replicas x{world} (users sharded, no collective on the data path)"}
     if c["dtype"] == "bf16" and c["kind"] != "pointwise":
         common["weights"] = "random-init, converted to the tensor-core operand layout once before timing " \
@@ -313,7 +329,7 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
-    wl = make_workload(args, data_seed=1000 + args.workload + 7919 * rank)
+    wl = make_workload(args, data_seed=rank_data_seed(args.workload, rank))
     kind = wl["cfg"]["kind"]
     n_tok = history_tokens(wl)
     stream = torch.cuda.current_stream()
@@ -345,11 +361,7 @@ def run_ours(args):
             dist.barrier()
 
     def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_over_ranks(v, world, "max")
 
     for _ in range(args.warmup):
         step()
@@ -390,7 +402,7 @@ def run_ours(args):
         raise RuntimeError(f"device status {st} ({B.strerror(st)}) in the timed region")
     ms_max = max_over_ranks(ms)
     ms_step = ms_max / args.steps
-    total_tokens = n_tok * world
+    total_tokens = reduce_over_ranks(n_tok, world, "sum")  # ranks draw their own lengths
     value = total_tokens * args.steps / (ms_max / 1e3)
 
     # per-stage live timings (CUDA events around each stage's launches on this stream)
@@ -488,7 +500,7 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if wl["cfg"]["dtype"] == "bf16" else "f32",
-        "data": "synthetic (seeded Zipf ids, random-init weights)", "config": config_block(wl, world),
+        "data": "synthetic (seeded Zipf ids, random-init weights)", "config": config_block(wl, world, total_tokens),
         "token_layers_per_s": round(value * layers, 1),
         "roofline": roofline, "stages": stages, "e2e": e2e, "cpu_baseline": cpu,
         "history_gemm_rows": "distinct (id, time bucket) keys per call" if dedup else "every history token",
@@ -550,7 +562,7 @@ def run_reference(args):
     rank, world, _ = dist_info()
     if rank != 0:
         return
-    wl = make_workload(args, data_seed=1000 + args.workload)
+    wl = make_workload(args, data_seed=rank_data_seed(args.workload, 0))
     n_users = len(wl["lengths"][0]) if wl["cfg"]["kind"] == "hyformer" else len(wl["lengths"])
     per = sample_users(wl)
     batches = [list(range(i * per % n_users, min(n_users, i * per % n_users + per)))

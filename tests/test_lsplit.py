@@ -117,3 +117,36 @@ def test_gloo_two_ranks_merge_equals_unsplit_attention(score):
     want = np.array([[[R.head_attention(q[i][t, h], K[i][:, h], V[i][:, h], score, 1 / math.sqrt(dh))
                        for h in range(H)] for t in range(T)] for i in range(layers)])
     np.testing.assert_allclose(got[0], want, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- bench's rank logic
+
+
+def _bench_rank_main(rank, world, port, results):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        from workloads import make_stca
+        wl = make_stca(2, users=3, data_seed=bench.rank_data_seed(2, rank))
+        n_tok = int(wl["lengths"].sum())
+        results[rank] = dict(
+            n_tok=n_tok, ids_head=wl["ids"][:16].tolist(),
+            total=bench.reduce_over_ranks(n_tok, world, "sum", device="cpu"),
+            slowest=bench.reduce_over_ranks(10.0 + rank, world, "max", device="cpu"))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gloo_two_ranks_bench_shards_users_and_reduces():
+    """bench.py at N > 1: each rank draws its own users (different ids and lengths), the
+    step time is the max over ranks and the work the sum over ranks."""
+    world = 2
+    with mp.Manager() as man:
+        results = man.dict()
+        mp.spawn(_bench_rank_main, args=(world, _free_port(), results), nprocs=world, join=True)
+        r = [dict(results[i]) for i in range(world)]
+    assert r[0]["ids_head"] != r[1]["ids_head"]
+    assert r[0]["total"] == r[1]["total"] == r[0]["n_tok"] + r[1]["n_tok"]
+    assert r[0]["slowest"] == r[1]["slowest"] == 11.0
