@@ -50,9 +50,14 @@ __global__ void insert_kernel(const int32_t* __restrict__ ids, const int32_t* __
   const unsigned long long key = row_key(ids, dt, i);
   unsigned slot = unsigned(mix64(key)) & mask;
   for (unsigned probe = 0; probe <= mask; ++probe) {
-    const unsigned long long prev = atomicCAS(&keys[slot], EMPTY_KEY, key);
+    // Popular keys (Zipf ids) are met by thousands of tokens: a plain read finds a key
+    // that is already in place without an atomic on its hot slot, and the first-token
+    // minimum is only lowered when this token can lower it.  A stale read costs one
+    // atomic more, never a wrong result (keys are only ever set once, minima only fall).
+    unsigned long long prev = __ldcg(&keys[slot]);
+    if (prev == EMPTY_KEY) prev = atomicCAS(&keys[slot], EMPTY_KEY, key);
     if (prev == EMPTY_KEY || prev == key) {
-      atomicMin(&first[slot], i);
+      if (__ldcg(&first[slot]) > i) atomicMin(&first[slot], i);
       slot_of[i] = int32_t(slot);
       return;
     }
