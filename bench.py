@@ -436,6 +436,8 @@ def run_ours(args):
                 "traffic": traffic_from_profiles(dom + ("+dedup" if dedup else ""), args.workload),
                 "work_per_launch": per_launch, "work_unit": unit, "launch_ms": round(tot / calls, 4),
                 "peak_source": f"{peaks['source']} ({'sustained bf16' if bound == 'tensor' else 'HBM copy'})"}
+    if bound == "tensor":  # the same against the burst figure (a GEMM timed alone at full clocks)
+        roofline["frac_of_burst_peak"] = round(achieved / peaks["bf16_tflops"], 4)
 
     # the same step with the history GEMMs run per token (dedup off), for reference
     per_token = None
