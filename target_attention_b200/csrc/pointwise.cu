@@ -53,22 +53,35 @@ __global__ void __launch_bounds__(PW_THREADS) pointwise_kernel(const int32_t* __
 
   const uint4* tab4 = reinterpret_cast<const uint4*>(table);
   // Rows j0 + 16*k + hw for k = 0, 1, ...; the loop bound is warp-uniform so both
-  // half-warps run the same iterations (the shuffles below use the full mask).
+  // half-warps run the same iterations (the shuffles below use the full mask).  The ids of
+  // the next UNROLL rows are loaded while this iteration's rows are in flight, so a row
+  // load waits on one memory latency, not on an id load and then a row load.
   constexpr int STEP = PW_THREADS / 16;
   const int warp_first = 2 * (tid >> 5);
+  const int64_t first = j0 + warp_first + (hw & 1);
+  int idn[UNROLL];
+#pragma unroll
+  for (int u = 0; u < UNROLL; ++u) {
+    const int64_t jj = first + int64_t(u) * STEP;
+    idn[u] = jj < j1 ? __ldg(ids + jj) : 0;
+  }
   for (int64_t base = j0 + warp_first; base < j1; base += STEP * UNROLL) {
     uint4 row[UNROLL];
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
       const int64_t jj = base + int64_t(u) * STEP + (hw & 1);
       bool ok = jj < j1;
-      int64_t id = ok ? __ldg(ids + jj) : 0;
+      int64_t id = idn[u];
       if (ok && (id < 0 || id >= n_items)) {
         set_error(err, STCA_ERR_ID_OUT_OF_RANGE);
         ok = false;
-        id = 0;
       }
       row[u] = ok ? __ldg(tab4 + id * (PD / 8) + li) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int64_t jj = base + int64_t(STEP * UNROLL) + int64_t(u) * STEP + (hw & 1);
+      idn[u] = jj < j1 ? __ldg(ids + jj) : 0;
     }
 #pragma unroll
     for (int u = 0; u < UNROLL; ++u) {
