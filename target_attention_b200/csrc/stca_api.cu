@@ -891,9 +891,15 @@ int stca_lsplit_begin(stca_handle* h, const int32_t* hist_ids, const int32_t* hi
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   h->last_stream = s;
   h->fwd.next_layer = -1;
-  CK(h->cfg.dtype == STCA_BF16
-         ? fwd_begin<bf16>(h, hist_ids, hist_lengths, hist_dt, target_emb, targets_per_user, B, n_tok, t_tot, w, s)
-         : fwd_begin<float>(h, hist_ids, hist_lengths, hist_dt, target_emb, targets_per_user, B, n_tok, t_tot, w, s));
+  if (B > 0 && t_tot > 0) {
+    CK(h->cfg.dtype == STCA_BF16
+           ? fwd_begin<bf16>(h, hist_ids, hist_lengths, hist_dt, target_emb, targets_per_user, B, n_tok, t_tot, w, s)
+           : fwd_begin<float>(h, hist_ids, hist_lengths, hist_dt, target_emb, targets_per_user, B, n_tok, t_tot, w,
+                              s));
+  } else {  // no targets: the phases run without work, so every rank still makes every call
+    h->fwd = stca_handle::Fwd{};
+    h->fwd.w = w;
+  }
   h->fwd.next_layer = 0;
   h->fwd.partial_done = false;
   return STCA_OK;
@@ -907,6 +913,10 @@ int stca_lsplit_partial(stca_handle* h, int layer, float* acc, float* ml, void* 
   if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   h->last_stream = s;
+  if (f.t_tot == 0) {
+    f.partial_done = true;
+    return STCA_OK;
+  }
   const bool bf = h->cfg.dtype == STCA_BF16;
   CK(bf ? fwd_layer_inputs<bf16>(h, layer, s) : fwd_layer_inputs<float>(h, layer, s));
   AttnArgs a;
@@ -954,6 +964,11 @@ int stca_lsplit_merge(stca_handle* h, int layer, int ranks, const float* all_acc
   if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   h->last_stream = s;
+  if (f.t_tot == 0) {
+    f.partial_done = false;
+    f.next_layer = last ? -1 : layer + 1;
+    return STCA_OK;
+  }
   AttnArgs a;
   memset(&a, 0, sizeof(a));
   a.T = f.t_tot;

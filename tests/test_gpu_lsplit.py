@@ -102,3 +102,21 @@ def test_lsplit_phase_order_is_checked():
     torch.cuda.synchronize()
     assert R.row_rel_err(z.cpu().numpy(), want.cpu().numpy()) <= 1e-5
     m.close()
+
+
+def test_lsplit_without_targets_runs_every_phase():
+    """Ranks whose request has no targets still make every call (the collectives must match
+    across ranks); the phases do no work."""
+    wl = make_stca(2, users=2, L=300, m=0)
+    m = StcaModel(wl, max_targets=1)
+    x = m.slice_inputs(wl, 2, 1)
+    z = torch.empty((1, wl["cfg"]["d"]), device=dev)
+    e = m.lsplit_engine(x, z)
+    e.begin()
+    for i in range(wl["cfg"]["M"]):
+        acc, ml = e.partial(i)
+        assert acc.shape[0] == 0
+        e.merge(i, torch.stack([acc, acc]), torch.stack([ml, ml]))
+    torch.cuda.synchronize()
+    assert B.stca_sync_status(m.handle) == B.OK
+    m.close()
