@@ -575,11 +575,13 @@ def run_reference(args):
     toks = sum(oracle_sample(wl, b) for b in batches[args.warmup:])
     dt = time.perf_counter() - t0
     value = toks / dt
+    cfg = config_block(wl, 1)
+    cfg.pop("weights", None)  # the oracle reads the weights as stored
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic (seeded Zipf ids, random-init weights)", "config": config_block(wl, 1),
+        "data": "synthetic (seeded Zipf ids, random-init weights)", "config": cfg,
         "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
                          "sample": f"{per} user(s) of the workload per step, fp64 oracle on the host"},
         "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
