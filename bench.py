@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dedup", action="store_true", help="run the history GEMMs once per token")
+    ap.add_argument("--uniform-ids", action="store_true",
+                    help="control run: history ids uniform over the table instead of Zipf")
     return ap.parse_args()
 
 
@@ -100,8 +102,9 @@ def make_workload(args, data_seed):
     """The seeded workload dict for --workload (sizes overridable for small runs)."""
     from workloads import make_hyformer, make_pointwise, make_stca
     c, users, L, n_items = workload_config(args)
+    over = {"id_dist": "uniform"} if getattr(args, "uniform_ids", False) else {}
     if c["kind"] == "stca":
-        return make_stca(args.workload, users=users, L=L, n_items=n_items, data_seed=data_seed)
+        return make_stca(args.workload, users=users, L=L, n_items=n_items, data_seed=data_seed, **over)
     if c["kind"] == "pointwise":
         return make_pointwise(args.workload, users=users, L=L, n_items=n_items, seed=data_seed)
     return make_hyformer(args.workload, users=users, L_feed=L, n_items=n_items, seed=data_seed)
