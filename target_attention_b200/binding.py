@@ -85,6 +85,7 @@ _SIGS = [
                                 _vp, _vp]),
     ("stca_sync_status", _i32, [_vp]),
     ("stca_profile_enable", _i32, [_vp, _i32]),
+    ("stca_profile_stages", _i32, [_vp, ctypes.c_uint32]),
     ("stca_profile_read", _i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
     ("stca_launch_count", ctypes.c_uint64, []),
     ("stca_strerror", ctypes.c_char_p, [_i32]),
@@ -176,6 +177,14 @@ STAGES = ["setup", "gather_ffn", "ffn_out", "kv", "attention", "merge", "query",
 
 def stca_profile_enable(h, enable=True) -> int:
     return lib().stca_profile_enable(h, 1 if enable else 0)
+
+
+def stca_profile_stages(h, names) -> int:
+    """Record only the named stages (an empty list stops recording)."""
+    mask = 0
+    for n in names:
+        mask |= 1 << STAGES.index(n)
+    return lib().stca_profile_stages(h, mask)
 
 
 def stca_profile_read(h):

@@ -80,8 +80,8 @@ struct stca_handle {
     int next_layer = -1;  // sequence-parallel forward: next layer to run, -1 when none is open
     bool partial_done = false;
   } fwd;
-  // per-stage timing
-  bool prof = false;
+  // per-stage timing: bit s set = stage s's launches are bracketed by events
+  uint32_t prof = 0;
   struct Rec {
     int stage;
     cudaEvent_t a, b;
@@ -121,7 +121,7 @@ struct Prof {
   cudaStream_t s;
   cudaEvent_t a = nullptr;
   Prof(stca_handle* h_, int stage_, cudaStream_t s_) : h(h_), stage(stage_), s(s_) {
-    if (h->prof) {
+    if ((h->prof >> stage) & 1u) {
       a = take_event(h);
       cudaEventRecord(a, s);
     }
@@ -1129,13 +1129,17 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
   return STCA_OK;
 }
 
-int stca_profile_enable(stca_handle* h, int enable) {
+int stca_profile_stages(stca_handle* h, uint32_t stage_mask) {
   if (!h) return STCA_ERR_INVALID_ARG;
   if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
   if (!h->recs.empty() && cudaDeviceSynchronize() != cudaSuccess) return STCA_ERR_CUDA;
   recycle_events(h);
-  h->prof = enable != 0;
+  h->prof = stage_mask & ((1u << STCA_N_STAGES) - 1u);
   return STCA_OK;
+}
+
+int stca_profile_enable(stca_handle* h, int enable) {
+  return stca_profile_stages(h, enable ? (1u << STCA_N_STAGES) - 1u : 0u);
 }
 
 int stca_profile_read(stca_handle* h, double* total_ms, int64_t* calls) {
