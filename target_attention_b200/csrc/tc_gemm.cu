@@ -167,7 +167,8 @@ __device__ __forceinline__ bool gather_row(const GatherSrc& g, int grow, int M, 
 // (the epilogue of one tile overlaps the MMAs of the next, across row tiles too), and
 // chunk kc of the next row tile's A is loaded as soon as the last N tile has used it.
 //
-// Warps: 0 TMA producer, 1 TMEM owner + MMA issuer (leader CTA), 4..11 epilogue,
+// Warps: 0 weight-tile TMA producer, 3 A-tile TMA producer (TMA mode), 1 TMEM owner + MMA
+// issuer (leader CTA), 4..11 epilogue,
 // 12, 14, 15, 2 gather producer (gather mode): cp.async of the CTA's A rows into the swizzled
 // layout (8 lanes per 128-byte row segment), the time-bucket row added (from L1), and
 // an L2 prefetch of the next tile's rows one tile ahead.  With store_x the
@@ -234,25 +235,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      if (AMODE == A_TMA) prefetch_tmap(&tmA);
       prefetch_tmap(&tmB);
       prefetch_tmap(&tmC);
-      const uint32_t a_full0 = cluster_addr(&a_full[0], 0), b_full0 = cluster_addr(&b_full[0], 0);
-      int it = 0, li = 0;
+      const uint32_t b_full0 = cluster_addr(&b_full[0], 0);
+      int it = 0;
       bool ok = true;
-      for (int tile = cl; tile < num_tiles && ok; tile += ncl, ++li) {
-        const int m0 = tile * 2 * BM + int(rank) * BM;
+      for (int tile = cl; tile < num_tiles && ok; tile += ncl) {
         for (int nt = 0; nt < NT && ok; ++nt) {
           for (int kc = 0; kc < KC; ++kc, ++it) {
-            if (AMODE == A_TMA && nt == 0) {
-              if (li > 0 && !mbar_wait(&a_empty[kc], (li - 1) & 1)) {
-                fail(abort_flag, err);
-                ok = false;
-                break;
-              }
-              if (leader) mbar_arrive_expect_tx(&a_full[kc], 2 * A_CHUNK);
-              tma_load_2d_pair(sA + kc * A_CHUNK, &tmA, kc * 64, m0, a_full0 + kc * 8);
-            }
             const int s = it % STAGES, round = it / STAGES;
             if ((round > 0 && !mbar_wait(&b_empty[s], (round - 1) & 1)) || abort_set(abort_flag)) {
               fail(abort_flag, err);
@@ -264,12 +254,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
           }
         }
       }
-      if (leader) {
-        // the leader's full barriers count both CTAs' bytes
-        drain_ring(b_full, STAGES, it);
-        if (AMODE == A_TMA && li > 0)
-          for (int kc = 0; kc < KC; ++kc) mbar_wait(&a_full[kc], (li - 1) & 1);
+      // the leader's full barriers count both CTAs' bytes
+      if (leader) drain_ring(b_full, STAGES, it);
+    }
+  } else if (warp == 3) {
+    // A producer (TMA mode): chunk kc of the next row tile is requested as soon as the last
+    // column tile of the current one has consumed chunk kc, apart from the weight ring, so
+    // the new rows arrive while the last column tile is still being multiplied
+    if (AMODE == A_TMA && lane == 0) {
+      prefetch_tmap(&tmA);
+      const uint32_t a_full0 = cluster_addr(&a_full[0], 0);
+      int li = 0;
+      bool ok = true;
+      for (int tile = cl; tile < num_tiles && ok; tile += ncl, ++li) {
+        const int m0 = tile * 2 * BM + int(rank) * BM;
+        for (int kc = 0; kc < KC; ++kc) {
+          if ((li > 0 && !mbar_wait(&a_empty[kc], (li - 1) & 1)) || abort_set(abort_flag)) {
+            fail(abort_flag, err);
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&a_full[kc], 2 * A_CHUNK);
+          tma_load_2d_pair(sA + kc * A_CHUNK, &tmA, kc * 64, m0, a_full0 + kc * 8);
+        }
       }
+      // no copy may still be writing shared memory when the pair exits
+      if (leader && li > 0)
+        for (int kc = 0; kc < KC; ++kc) mbar_wait(&a_full[kc], (li - 1) & 1);
     }
   } else if (warp == 1) {
     if (leader && lane == 0) {
