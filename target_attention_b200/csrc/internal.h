@@ -78,6 +78,8 @@ int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N,
 // 2-D bf16 tensor map over a [rows, cols] row-major matrix (row stride ld elements),
 // box = 64 columns x box_rows rows, 128-byte swizzle, zero fill outside the matrix.
 bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows);
+// fp32 [rows, cols] (row stride ld elements), box 32 x 32, 128-byte swizzle: tile stores.
+bool make_tmap_f32_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld);
 
 // ---------------------------------------------------------------- SIMT fp32 GEMMs
 

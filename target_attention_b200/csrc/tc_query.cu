@@ -43,6 +43,7 @@ struct TcqArgs {
   int M, N, K;  // N output columns
   int64_t bsA, bsC, bsR;  // element offsets per batch (grid z)
   int wrows;              // packed weight rows per batch
+  int c_tma;              // C written by TMA tile stores (one batch, rows not remapped)
   int32_t* err;
 };
 
@@ -54,7 +55,10 @@ __device__ __forceinline__ int64_t q_remap(int r, int grp, int gstride, int goff
   return grp ? int64_t(r / grp) * gstride + goff + r % grp : int64_t(r);
 }
 
-__device__ __forceinline__ float silu_precise(float x) { return x / (1.0f + expf(-x)); }
+// SiLU(x) = x / (1 + e^-x) with the fast exponential and division intrinsics: a few
+// ulp of fp32 (the target side keeps fp32 accuracy; the bf16 history side uses tanh.approx).
+// For x below about -88, e^-x is +inf and the quotient is 0, the limit of SiLU.
+__device__ __forceinline__ float silu_fast(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 
 // hi and lo bf16 pairs of two fp32 values
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
@@ -66,7 +70,8 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
 }
 
 template <bool DUAL>
-__global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant__ CUtensorMap tmB, TcqArgs a) {
+__global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant__ CUtensorMap tmB,
+                                                          const __grid_constant__ CUtensorMap tmC, TcqArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = q_align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + QSTAGES * QSTAGE);
@@ -232,11 +237,16 @@ __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant_
     __syncwarp();
     if (ok) {
       tc_fence_after();
+      fence_proxy_async_smem();  // the ring's last async reads come before the staging writes
       const int quarter = warp & 3, half = (warp - 4) >> 2;
       const int row = m0 + quarter * 32 + lane;
       const uint32_t tbase = tmem + (uint32_t(quarter * 32) << 16);
       float* crow = row < a.M ? C + q_remap(row, a.c_grp, a.c_gstride, a.c_goff) * a.ldc : nullptr;
       const float* rrow = (row < a.M && R) ? R + int64_t(row) * a.ldr : nullptr;
+      // With tile stores, each warp stages its 32 x 32 blocks in two 4 KB buffers of the
+      // (now idle) operand ring, rows 128-byte swizzled, and TMA writes whole rows; rows or
+      // columns outside C are clipped.  Otherwise each lane stores its own row.
+      uint8_t* stage = smem + (warp - 4) * 8192;
       constexpr int NCH = DUAL ? 2 : 4;  // 32-column output chunks per warp
 #pragma unroll 1
       for (int j = 0; j < NCH; ++j) {
@@ -248,27 +258,43 @@ __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant_
           tmem_ld_32x32b_x32(tbase + 128 + tc, u);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = silu_precise(v[e]) * u[e];
+          for (int e = 0; e < 32; ++e) v[e] = silu_fast(v[e]) * u[e];
         } else {
           tmem_ld_wait();
         }
         const int col = (DUAL ? blockIdx.x * 128 : blockIdx.x * QBN) + tc;
-        if (crow && col < a.N) {
-          if (rrow) {
+        if (col >= a.N) continue;  // warp-uniform
+        if (rrow) {
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float4 r4 = *reinterpret_cast<const float4*>(rrow + col + e);
-              v[e] += r4.x;
-              v[e + 1] += r4.y;
-              v[e + 2] += r4.z;
-              v[e + 3] += r4.w;
-            }
+          for (int e = 0; e < 32; e += 4) {
+            const float4 r4 = *reinterpret_cast<const float4*>(rrow + col + e);
+            v[e] += r4.x;
+            v[e + 1] += r4.y;
+            v[e + 2] += r4.z;
+            v[e + 3] += r4.w;
           }
+        }
+        if (a.c_tma) {
+          uint8_t* buf = stage + (j & 1) * 4096;
+          if (lane == 0 && j >= 2) bulk_wait_read<1>();  // the store that read this buffer
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<float4*>(buf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, col, m0 + quarter * 32, buf);
+            bulk_commit();
+          }
+        } else if (crow) {
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4*>(crow + col + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
         }
       }
+      if (a.c_tma && lane == 0) bulk_wait_all();
     }
   }
   tc_fence_before();
@@ -327,17 +353,25 @@ int tc_query_gemm(const SimtGemmArgs<float, bf16>& a, const void* Wp, cudaStream
   q.bsR = a.bsR;
   q.wrows = wrows;
   q.err = a.err;
+  // tile stores need one contiguous [M, N] block: one batch, rows not remapped
+  q.c_tma = a.batch == 1 && a.c_grp == 0;
+  CUtensorMap tc;
+  if (q.c_tma) {
+    if (!make_tmap_f32_out(&tc, a.C, uint64_t(a.M), uint64_t(a.N), uint64_t(a.ldc))) return STCA_ERR_CUDA;
+  } else {
+    tc = tb;  // unused
+  }
   const dim3 grid((wrows + QBN - 1) / QBN, (a.M + QBM - 1) / QBM, a.batch);
   if (dual) {
     if (cudaFuncSetAttribute(tc_query_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(QSMEM)) !=
         cudaSuccess)
       return STCA_ERR_CUDA;
-    tc_query_kernel<true><<<grid, 384, QSMEM, s>>>(tb, q);
+    tc_query_kernel<true><<<grid, 384, QSMEM, s>>>(tb, tc, q);
   } else {
     if (cudaFuncSetAttribute(tc_query_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(QSMEM)) !=
         cudaSuccess)
       return STCA_ERR_CUDA;
-    tc_query_kernel<false><<<grid, 384, QSMEM, s>>>(tb, q);
+    tc_query_kernel<false><<<grid, 384, QSMEM, s>>>(tb, tc, q);
   }
   note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
