@@ -105,6 +105,12 @@ __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant_
     tmem_alloc(tmem_slot, QBN);
     tmem_relinquish();
   }
+  if (threadIdx.x == 0) prefetch_tmap(&tmB);
+  // Launched as a programmatic dependent of the previous kernel on the stream: the setup
+  // above overlaps that kernel's tail; nothing it writes (or anything before it) is touched
+  // before this wait.  The next target-side GEMM may start its own setup now.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -112,7 +118,6 @@ __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant_
 
   if (warp == 0) {
     if (lane == 0) {
-      prefetch_tmap(&tmB);
       int issued = 0;
       for (int kc = 0; kc < KC; ++kc, ++issued) {
         const int s = kc % QSTAGES, round = kc / QSTAGES;
@@ -362,17 +367,23 @@ int tc_query_gemm(const SimtGemmArgs<float, bf16>& a, const void* Wp, cudaStream
     tc = tb;  // unused
   }
   const dim3 grid((wrows + QBN - 1) / QBN, (a.M + QBM - 1) / QBM, a.batch);
-  if (dual) {
-    if (cudaFuncSetAttribute(tc_query_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(QSMEM)) !=
-        cudaSuccess)
-      return STCA_ERR_CUDA;
-    tc_query_kernel<true><<<grid, 384, QSMEM, s>>>(tb, tc, q);
-  } else {
-    if (cudaFuncSetAttribute(tc_query_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(QSMEM)) !=
-        cudaSuccess)
-      return STCA_ERR_CUDA;
-    tc_query_kernel<false><<<grid, 384, QSMEM, s>>>(tb, tc, q);
-  }
+  auto kern = dual ? tc_query_kernel<true> : tc_query_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(QSMEM)) != cudaSuccess)
+    return STCA_ERR_CUDA;
+  // programmatic dependent launch: the CTAs may start (barriers, TMEM, descriptor prefetch)
+  // while the previous kernel on the stream drains; the kernel waits for it before any data
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(384);
+  cfg.dynamicSmemBytes = QSMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tb, tc, q) != cudaSuccess) return STCA_ERR_CUDA;
   note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
