@@ -227,6 +227,8 @@ __device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, const int* s
 
 template <int SCORE>
 __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
+  griddep_wait();
+  griddep_launch();
   extern __shared__ __align__(128) uint8_t smem[];
   const int u = blockIdx.x / a.splits, s = blockIdx.x % a.splits, h = blockIdx.y;
   int64_t k0;
@@ -504,6 +506,8 @@ __global__ void __launch_bounds__(128) attn_f32_kernel(AttnArgs a) {
 
 template <int SCORE>
 __global__ void attn_merge_kernel(AttnArgs a) {
+  griddep_wait();
+  griddep_launch();
   const int64_t wid = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= int64_t(a.T) * a.H) return;
@@ -560,10 +564,10 @@ int attention_bf16(const AttnArgs& a, cudaStream_t s) {
   dim3 grid(a.B * a.splits, a.H);
   if (a.score == 0) {
     cudaFuncSetAttribute(attn_bf16_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_SMEM);
-    attn_bf16_kernel<0><<<grid, ATT_THREADS, ATTN_SMEM, s>>>(a); note_launch();
+    launch_dep(attn_bf16_kernel<0>, grid, dim3(ATT_THREADS), ATTN_SMEM, s, a); note_launch();
   } else {
     cudaFuncSetAttribute(attn_bf16_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, ATTN_SMEM);
-    attn_bf16_kernel<1><<<grid, ATT_THREADS, ATTN_SMEM, s>>>(a); note_launch();
+    launch_dep(attn_bf16_kernel<1>, grid, dim3(ATT_THREADS), ATTN_SMEM, s, a); note_launch();
   }
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
@@ -597,8 +601,8 @@ int attention_merge(const AttnArgs& a, cudaStream_t s) {
   if (a.splits < 1 || a.splits > 32) return STCA_ERR_INVALID_ARG;  // one lane per slice
   const int64_t warps = int64_t(a.T) * a.H;
   const int blocks = int((warps * 32 + 255) / 256);
-  if (a.score == 0) attn_merge_kernel<0><<<blocks, 256, 0, s>>>(a);
-  else attn_merge_kernel<1><<<blocks, 256, 0, s>>>(a);
+  if (a.score == 0) launch_dep(attn_merge_kernel<0>, dim3(blocks), dim3(256), 0, s, a);
+  else launch_dep(attn_merge_kernel<1>, dim3(blocks), dim3(256), 0, s, a);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }

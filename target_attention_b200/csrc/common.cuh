@@ -82,6 +82,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// ------------------------------------------------------------------ dependent launches
+// Kernels launched with launch_dep() may begin while the previous kernel on the stream is
+// still running; they wait here for it (and its memory) before touching any data, then let
+// the next dependent kernel begin its own launch.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ async proxy / TMA
 
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -45,6 +45,8 @@ __device__ __forceinline__ unsigned long long row_key(const int32_t* ids, const 
 __global__ void insert_kernel(const int32_t* __restrict__ ids, const int32_t* __restrict__ dt, int n,
                               unsigned long long* __restrict__ keys, int32_t* __restrict__ first,
                               int32_t* __restrict__ slot_of, unsigned mask, int32_t* err) {
+  griddep_wait();
+  griddep_launch();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const unsigned long long key = row_key(ids, dt, i);
@@ -105,6 +107,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int& excl) {
 __global__ void __launch_bounds__(SCAN_THREADS) count_kernel(const int32_t* __restrict__ first,
                                                              const int32_t* __restrict__ slot_of, int n,
                                                              int32_t* __restrict__ tile_counts) {
+  griddep_wait();
+  griddep_launch();
   const int base = blockIdx.x * SCAN_TILE + threadIdx.x * SCAN_ITEMS;
   int c = 0;
 #pragma unroll
@@ -118,6 +122,8 @@ __global__ void __launch_bounds__(SCAN_THREADS) count_kernel(const int32_t* __re
 // exclusive scan of the tile counts in place (one block); count = grand total
 __global__ void __launch_bounds__(SCAN_THREADS) scan_tiles_kernel(int32_t* __restrict__ tile_counts, int tiles,
                                                                   int32_t* __restrict__ count) {
+  griddep_wait();
+  griddep_launch();
   int carry = 0;
   for (int b = 0; b < tiles; b += SCAN_THREADS) {
     const int i = b + threadIdx.x;
@@ -136,6 +142,8 @@ __global__ void __launch_bounds__(SCAN_THREADS) number_kernel(const int32_t* __r
                                                               const int32_t* __restrict__ tile_offsets,
                                                               int32_t* __restrict__ pos,
                                                               int32_t* __restrict__ uniq_token) {
+  griddep_wait();
+  griddep_launch();
   const int base = blockIdx.x * SCAN_TILE + threadIdx.x * SCAN_ITEMS;
   bool f[SCAN_ITEMS];
   int c = 0;
@@ -158,6 +166,8 @@ __global__ void __launch_bounds__(SCAN_THREADS) number_kernel(const int32_t* __r
 
 __global__ void map_kernel(const int32_t* __restrict__ first, const int32_t* __restrict__ slot_of,
                            const int32_t* __restrict__ pos, int n, int32_t* __restrict__ uniq_idx) {
+  griddep_wait();
+  griddep_launch();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) uniq_idx[i] = pos[first[slot_of[i]]];
 }
@@ -184,6 +194,8 @@ __global__ void __launch_bounds__(SCAN_THREADS) compact_user_kernel(const int32_
                                                                     int32_t* __restrict__ out_rows,
                                                                     int32_t* __restrict__ out_mult,
                                                                     int32_t* __restrict__ out_len) {
+  griddep_wait();
+  griddep_launch();
   extern __shared__ int32_t cu_smem[];
   const int u = blockIdx.x;
   const int h0 = hoff[u], L = hoff[u + 1] - h0;
@@ -252,7 +264,7 @@ int compact_user_rows(const int32_t* hoff, int B, const int32_t* rows, int32_t* 
   if (cudaFuncSetAttribute(compact_user_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CU_SMEM)) !=
       cudaSuccess)
     return STCA_ERR_CUDA;
-  compact_user_kernel<<<B, SCAN_THREADS, CU_SMEM, s>>>(hoff, rows, out_rows, out_mult, out_len);
+  launch_dep(compact_user_kernel, dim3(B), dim3(SCAN_THREADS), CU_SMEM, s, hoff, rows, out_rows, out_mult, out_len);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? STCA_OK : STCA_ERR_CUDA;
 }
@@ -289,15 +301,16 @@ int dedup_rows(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws
   const int tiles = (n + SCAN_TILE - 1) / SCAN_TILE;
   if (cudaMemsetAsync(keys, 0xFF, cap * 8, s) != cudaSuccess) return STCA_ERR_CUDA;
   if (cudaMemsetAsync(first, 0x7F, cap * 4, s) != cudaSuccess) return STCA_ERR_CUDA;  // INT_MAX-like
-  insert_kernel<<<(n + 255) / 256, 256, 0, s>>>(ids, dt, n, keys, first, slot_of, unsigned(cap - 1), err);
+  launch_dep(insert_kernel, dim3((n + 255) / 256), dim3(256), 0, s, ids, dt, n, keys, first, slot_of,
+             unsigned(cap - 1), err);
   note_launch();
-  count_kernel<<<tiles, SCAN_THREADS, 0, s>>>(first, slot_of, n, tile_off);
+  launch_dep(count_kernel, dim3(tiles), dim3(SCAN_THREADS), 0, s, first, slot_of, n, tile_off);
   note_launch();
-  scan_tiles_kernel<<<1, SCAN_THREADS, 0, s>>>(tile_off, tiles, count);
+  launch_dep(scan_tiles_kernel, dim3(1), dim3(SCAN_THREADS), 0, s, tile_off, tiles, count);
   note_launch();
-  number_kernel<<<tiles, SCAN_THREADS, 0, s>>>(first, slot_of, n, tile_off, pos, uniq_token);
+  launch_dep(number_kernel, dim3(tiles), dim3(SCAN_THREADS), 0, s, first, slot_of, n, tile_off, pos, uniq_token);
   note_launch();
-  map_kernel<<<(n + 255) / 256, 256, 0, s>>>(first, slot_of, pos, n, uniq_idx);
+  launch_dep(map_kernel, dim3((n + 255) / 256), dim3(256), 0, s, first, slot_of, pos, n, uniq_idx);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? STCA_OK : STCA_ERR_CUDA;
 }

@@ -1,6 +1,9 @@
 // Host-side launchers shared between the library's translation units.
 #pragma once
 
+#include <cstring>
+#include <utility>
+
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -163,6 +166,25 @@ int attention_f32(const AttnArgs& a, cudaStream_t s);
 int attention_merge(const AttnArgs& a, cudaStream_t s);
 inline bool attention_needs_merge(const AttnArgs& a, bool kv_bf16) {
   return !(kv_bf16 && a.splits == 1 && !a.partial_out);
+}
+// Launches kern as a programmatic dependent of the previous kernel on stream s (its CTAs
+// may start while that kernel drains).  Every kernel launched this way calls griddep_wait()
+// before it reads or writes any data.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dep(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 // streaming multiprocessors of the current device
 int sm_count();

@@ -136,6 +136,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtGemmArgs<TA, TB> a) 
 __global__ void layer_norm_kernel(const float* __restrict__ x, int64_t ldx, float* __restrict__ y, int64_t ldy,
                                   int rows, int d, const float* __restrict__ gamma, const float* __restrict__ beta,
                                   float eps) {
+  griddep_wait();
+  griddep_launch();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -174,6 +176,8 @@ __global__ void layer_norm_kernel(const float* __restrict__ x, int64_t ldx, floa
 // Exclusive scan of B lengths in one block; validates signs and the total.
 __global__ void offsets_kernel(const int32_t* __restrict__ lengths, int B, int32_t* __restrict__ offsets,
                                int expected, int32_t* err) {
+  griddep_wait();
+  griddep_launch();
   __shared__ long long warp_sums[32];
   __shared__ long long carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -222,6 +226,8 @@ __global__ void offsets_kernel(const int32_t* __restrict__ lengths, int B, int32
 template <typename T>
 __global__ void copy_rows_kernel(const T* __restrict__ src, int rows, int d, float* __restrict__ dst, int64_t ldd,
                                  int col0) {
+  griddep_wait();
+  griddep_launch();
   const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= int64_t(rows) * d) return;
   const int64_t r = i / d;
@@ -230,6 +236,8 @@ __global__ void copy_rows_kernel(const T* __restrict__ src, int rows, int d, flo
 }
 
 __global__ void token_mix_kernel(const float* __restrict__ Q, int B, int T, int d, float* __restrict__ out) {
+  griddep_wait();
+  griddep_launch();
   const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (i >= int64_t(B) * T * d) return;
   const int sub = d / T;
@@ -241,6 +249,8 @@ __global__ void token_mix_kernel(const float* __restrict__ Q, int B, int T, int 
 }
 
 __global__ void arange_kernel(int32_t* out, int n, int step) {
+  griddep_wait();
+  griddep_launch();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = i * step;
 }
@@ -249,7 +259,7 @@ __global__ void arange_kernel(int32_t* out, int n, int step) {
 
 int fill_arange(int32_t* out, int n, int step, cudaStream_t s) {
   if (n <= 0) return 0;
-  arange_kernel<<<(n + 255) / 256, 256, 0, s>>>(out, n, step); note_launch();
+  launch_dep(arange_kernel, dim3((n + 255) / 256), dim3(256), 0, s, out, n, step); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -275,12 +285,13 @@ int layer_norm_f32(const float* x, int64_t ldx, float* y, int64_t ldy, int rows,
                    const float* beta, float eps, cudaStream_t s) {
   if (rows == 0) return 0;
   if (d > 1024) return STCA_ERR_UNSUPPORTED;
-  layer_norm_kernel<<<(rows + 7) / 8, 256, 0, s>>>(x, ldx, y, ldy, rows, d, gamma, beta, eps); note_launch();
+  launch_dep(layer_norm_kernel, dim3((rows + 7) / 8), dim3(256), 0, s, x, ldx, y, ldy, rows, d, gamma, beta, eps);
+  note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
 int exclusive_offsets(const int32_t* lengths, int B, int32_t* offsets, int expected, int32_t* err, cudaStream_t s) {
-  offsets_kernel<<<1, 1024, 0, s>>>(lengths, B, offsets, expected, err); note_launch();
+  launch_dep(offsets_kernel, dim3(1), dim3(1024), 0, s, lengths, B, offsets, expected, err); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -289,8 +300,12 @@ int copy_rows_to_f32(const void* src, int src_bf16, int rows, int d, float* dst,
   const int64_t n = int64_t(rows) * d;
   if (n == 0) return 0;
   const int blocks = int((n + 255) / 256);
-  if (src_bf16) copy_rows_kernel<bf16><<<blocks, 256, 0, s>>>(reinterpret_cast<const bf16*>(src), rows, d, dst, ldd, col0);
-  else copy_rows_kernel<float><<<blocks, 256, 0, s>>>(reinterpret_cast<const float*>(src), rows, d, dst, ldd, col0);
+  if (src_bf16)
+    launch_dep(copy_rows_kernel<bf16>, dim3(blocks), dim3(256), 0, s, reinterpret_cast<const bf16*>(src), rows, d, dst,
+               ldd, col0);
+  else
+    launch_dep(copy_rows_kernel<float>, dim3(blocks), dim3(256), 0, s, reinterpret_cast<const float*>(src), rows, d, dst,
+               ldd, col0);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
@@ -298,7 +313,7 @@ int copy_rows_to_f32(const void* src, int src_bf16, int rows, int d, float* dst,
 int token_mix(const float* Q, int B, int T, int d, float* mixed, cudaStream_t s) {
   const int64_t n = int64_t(B) * T * d;
   if (n == 0) return 0;
-  token_mix_kernel<<<int((n + 255) / 256), 256, 0, s>>>(Q, B, T, d, mixed); note_launch();
+  launch_dep(token_mix_kernel, dim3(int((n + 255) / 256)), dim3(256), 0, s, Q, B, T, d, mixed); note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 

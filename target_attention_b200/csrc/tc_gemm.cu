@@ -195,6 +195,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
                             const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmX,
                             GatherSrc g, int M_max, int K, int NT, int store_x, int32_t* err, const int32_t* M_dev,
                             EpiFold fold) {
+  griddep_wait();
+  griddep_launch();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   const int KC = K / 64;
@@ -546,6 +548,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
                            const __grid_constant__ CUtensorMap tmC, int M_max, int K,
                            const float* __restrict__ gamma, const float* __restrict__ beta, float eps, int32_t* err,
                            const int32_t* M_dev, float* __restrict__ stats) {
+  griddep_wait();
+  griddep_launch();
   constexpr int N = NB * 256;
   constexpr int STAGE_BYTES = A_CHUNK + NB * B_HALF;
   extern __shared__ uint8_t smem_raw[];
@@ -904,7 +908,8 @@ int run_resident(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
   const int grid = 2 * std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
-  kern<<<grid, 512, smem, s>>>(ta, tb, tc, tx, g, M, K, NT, store_x, err, M_dev, fold); note_launch();
+  launch_dep(kern, dim3(grid), dim3(512), smem, s, ta, tb, tc, tx, g, M, K, NT, store_x, err, M_dev, fold);
+  note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
@@ -917,7 +922,8 @@ int run_rowwise(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap&
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
   const int grid = 2 * std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
-  kern<<<grid, 384, smem, s>>>(ta, tb, tc, M, K, gamma, beta, eps, err, M_dev, stats); note_launch();
+  launch_dep(kern, dim3(grid), dim3(384), smem, s, ta, tb, tc, M, K, gamma, beta, eps, err, M_dev, stats);
+  note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
