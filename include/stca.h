@@ -296,6 +296,12 @@ uint64_t stca_launch_count(void);
  * error word (STCA_OK if no error was recorded), or STCA_ERR_CUDA. */
 int stca_sync_status(stca_handle* h);
 
+/* Host watchdog: waits at most timeout_ms for the work enqueued so far on `stream` (a
+ * cudaStream_t; NULL = legacy default stream), polling an event.  STCA_OK when it has
+ * finished, STCA_ERR_TIMEOUT when the deadline passed first (the work keeps running and
+ * may be waited for again), STCA_ERR_CUDA on a CUDA error.  Never blocks past the deadline. */
+int stca_stream_wait(void* stream, int timeout_ms);
+
 /* Static description of a status code. */
 const char* stca_strerror(int code);
 

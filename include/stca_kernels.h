@@ -89,6 +89,12 @@ int stca_k_dedup(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t 
 int stca_k_compact_user_rows(const int32_t* hoff, int B, const int32_t* rows, int32_t* out_rows, int32_t* out_mult,
                              int32_t* out_len, void* stream);
 
+/* Self-test of the bounded waits every pipelined kernel uses: one CTA waits on a barrier
+ * that nothing completes, gives up after the library's wait limit (about 2 s), records
+ * STCA_ERR_TIMEOUT in *err (device int32) and exits normally, leaving the context usable.
+ * Asynchronous on `stream`. */
+int stca_k_wait_selftest(int32_t* err, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

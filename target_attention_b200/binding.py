@@ -84,6 +84,8 @@ _SIGS = [
     ("hyformer_forward", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, ctypes.POINTER(HyfWeights),
                                 _vp, _vp]),
     ("stca_sync_status", _i32, [_vp]),
+    ("stca_stream_wait", _i32, [_vp, _i32]),
+    ("stca_k_wait_selftest", _i32, [_vp, _vp]),
     ("stca_profile_enable", _i32, [_vp, _i32]),
     ("stca_profile_stages", _i32, [_vp, ctypes.c_uint32]),
     ("stca_profile_read", _i32, [_vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
@@ -177,6 +179,15 @@ STAGES = ["setup", "gather_ffn", "ffn_out", "kv", "attention", "merge", "query",
 
 def stca_profile_enable(h, enable=True) -> int:
     return lib().stca_profile_enable(h, 1 if enable else 0)
+
+
+def stca_stream_wait(stream=None, timeout_ms=0) -> int:
+    """Waits at most timeout_ms for the work enqueued on the stream (OK or ERR_TIMEOUT)."""
+    return lib().stca_stream_wait(stream_ptr(stream), timeout_ms)
+
+
+def stca_k_wait_selftest(err, stream=None) -> int:
+    return lib().stca_k_wait_selftest(ptr(err), stream_ptr(stream))
 
 
 def stca_profile_stages(h, names) -> int:

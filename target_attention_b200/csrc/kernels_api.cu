@@ -7,7 +7,32 @@
 
 using namespace stca;
 
+namespace {
+
+// One CTA waits on an mbarrier whose phase never completes: the bounded wait gives up and
+// the kernel records the timeout and returns (the pattern of every pipelined kernel).
+__global__ void wait_selftest_kernel(int32_t* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0)) set_error(err, STCA_ERR_TIMEOUT);
+  __syncthreads();
+}
+
+}  // namespace
+
 extern "C" {
+
+int stca_k_wait_selftest(int32_t* err, void* stream) {
+  if (!err) return STCA_ERR_INVALID_ARG;
+  wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(err);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
+}
+
 
 int stca_k_offsets(const int32_t* lengths, int B, int32_t* offsets, int expected, int32_t* err, void* stream) {
   if (B < 0 || !offsets || (B > 0 && !lengths)) return STCA_ERR_INVALID_ARG;

@@ -2,9 +2,11 @@
 // forward pass.  Every step of the path runs in this library's kernels; PyTorch (or any
 // other caller) only provides device memory and the stream.
 #include <atomic>
+#include <chrono>
 #include <cstdio>
 #include <cstring>
 #include <new>
+#include <thread>
 #include <vector>
 
 #include "common.cuh"
@@ -1160,6 +1162,33 @@ int stca_profile_read(stca_handle* h, double* total_ms, int64_t* calls) {
 }
 
 uint64_t stca_launch_count(void) { return stca::g_launches.load(); }
+
+int stca_stream_wait(void* stream, int timeout_ms) {
+  if (timeout_ms < 0) return STCA_ERR_INVALID_ARG;
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return STCA_ERR_CUDA;
+  int rc = STCA_OK;
+  if (cudaEventRecord(e, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    rc = STCA_ERR_CUDA;
+  } else {
+    const auto deadline = std::chrono::steady_clock::now() + std::chrono::milliseconds(timeout_ms);
+    while (true) {
+      const cudaError_t q = cudaEventQuery(e);
+      if (q == cudaSuccess) break;
+      if (q != cudaErrorNotReady) {
+        rc = STCA_ERR_CUDA;
+        break;
+      }
+      if (std::chrono::steady_clock::now() >= deadline) {
+        rc = STCA_ERR_TIMEOUT;
+        break;
+      }
+      std::this_thread::sleep_for(std::chrono::microseconds(200));
+    }
+  }
+  cudaEventDestroy(e);  // released once the recorded work completes
+  return rc;
+}
 
 int stca_sync_status(stca_handle* h) {
   if (!h) return STCA_ERR_INVALID_ARG;

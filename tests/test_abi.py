@@ -91,6 +91,8 @@ def test_null_arguments_rejected_on_host():
         == B.ERR_INVALID_ARG
     assert L.stca_lsplit_partial(None, 0, None, None, None) == B.ERR_INVALID_ARG
     assert L.stca_lsplit_merge(None, 0, 2, None, None, None, None) == B.ERR_INVALID_ARG
+    assert L.stca_k_wait_selftest(None, None) == B.ERR_INVALID_ARG
+    assert L.stca_stream_wait(None, -1) == B.ERR_INVALID_ARG
     L.stca_unpin_weights(None)
     L.stca_destroy(None)
     # kernel-level entry points validate before launching
