@@ -508,6 +508,7 @@ def run_ours(args):
         e0.record(stream)
         for _ in range(args.steps):
             B.check(model.forward_host(xh, zh, stream=stream))
+        B.check(model.host_fence(stream))  # the last step's z has landed in host memory
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()

@@ -151,15 +151,23 @@ int stca_forward(stca_handle* h, const int32_t* hist_ids, const int32_t* hist_le
 
 /* stca_forward with the per-request inputs and the output in HOST memory (pinned memory
  * makes the copies asynchronous): the library copies the inputs into one of two staging
- * slots of its workspace on an internal copy stream (so one call's input copies overlap the
- * previous call's forward), runs the forward on `stream` once they have landed, and copies
- * z back on `stream`.  Weights and the table stay device pointers.  Returns after
- * enqueueing; once `stream` has been synchronised the inputs have been read and
- * z_out_host holds the result (keep the host inputs unchanged until then). */
+ * slots of its workspace on an internal copy stream, runs the forward on `stream` once
+ * they have landed into one of two output slots, and copies z back to z_out_host on a
+ * second internal stream.  So one call's input copies and the previous call's read-back
+ * both overlap the forward in between.  Weights and the table stay device pointers.
+ * Returns after enqueueing.  Once `stream` has been synchronised the inputs have been
+ * read (keep the host inputs unchanged until then); z_out_host holds the result once
+ * stca_host_fence(h, stream) has been called after this call and `stream` synchronised,
+ * or once stca_sync_status(h) has returned (or the device has been synchronised). */
 int stca_forward_host(stca_handle* h, const int32_t* hist_ids_host, const int32_t* hist_lengths_host,
                       const int32_t* hist_dt_host, const void* target_emb_host,
                       const int32_t* targets_per_user_host, int B, int n_tok, int t_tot,
                       const stca_weights* w, float* z_out_host, void* stream);
+
+/* Makes `stream` wait until the z read-backs of every stca_forward_host call enqueued on
+ * the handle so far have landed in host memory (nothing to wait for before the first
+ * call).  Enqueues a wait and returns; STCA_ERR_CUDA if that fails. */
+int stca_host_fence(stca_handle* h, void* stream);
 
 /* Sequence-parallel (L-split) forward, in phases, for histories split across R ranks (one
  * GPU each).  Attention over a history is a merge of attention over its slices: each slice
@@ -292,8 +300,9 @@ int stca_profile_read(stca_handle* h, double* total_ms, int64_t* calls);
 /* Kernel launches this library has issued since it was loaded (all handles). */
 uint64_t stca_launch_count(void);
 
-/* Synchronises the stream of the handle's last call, then returns and clears the device
- * error word (STCA_OK if no error was recorded), or STCA_ERR_CUDA. */
+/* Synchronises the stream of the handle's last call and the host entry's read-back
+ * stream, then returns and clears the device error word (STCA_OK if no error was
+ * recorded), or STCA_ERR_CUDA. */
 int stca_sync_status(stca_handle* h);
 
 /* Host watchdog: waits at most timeout_ms for the work enqueued so far on `stream` (a

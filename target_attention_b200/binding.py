@@ -76,6 +76,7 @@ _SIGS = [
                             _vp]),
     ("stca_forward_host", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.POINTER(StcaWeights), _vp,
                                  _vp]),
+    ("stca_host_fence", _i32, [_vp, _vp]),
     ("stca_lsplit_begin", _i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, ctypes.POINTER(StcaWeights), _vp]),
     ("stca_lsplit_partial", _i32, [_vp, _i32, _vp, _vp, _vp]),
     ("stca_lsplit_merge", _i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
@@ -224,6 +225,10 @@ def stca_forward_host(h, ids, lengths, dt, x_t, tpu, B, n_tok, t_tot, weights: S
                       stream=None) -> int:
     return lib().stca_forward_host(h, ptr(ids), ptr(lengths), ptr(dt), ptr(x_t), ptr(tpu), B, n_tok, t_tot,
                                    ctypes.byref(weights), ptr(z_out), stream_ptr(stream))
+
+
+def stca_host_fence(h, stream=None) -> int:
+    return lib().stca_host_fence(h, stream_ptr(stream))
 
 
 def stca_lsplit_begin(h, ids, lengths, dt, x_t, tpu, B, n_tok, t_tot, weights: StcaWeights, stream=None) -> int:

@@ -64,15 +64,17 @@ struct stca_handle {
   const void* pinned = nullptr;
   std::vector<uint8_t> pinned_copy;
   int pinned_tokens = 0;
-  // staging for the host-buffer entry point: two input slots, so the copies of one call's
-  // inputs (on copy_stream) overlap the previous call's forward
+  // staging for the host-buffer entry point: two input slots and two output slots, so the
+  // copies of one call's inputs (on copy_stream) and the read-back of its z (on back_stream)
+  // overlap the neighbouring calls' forwards
   int32_t *in_ids[2] = {}, *in_len[2] = {}, *in_dt[2] = {}, *in_tpu[2] = {};
   void* in_xt[2] = {};
-  float* out_z = nullptr;
-  cudaStream_t copy_stream = nullptr;
+  float* out_z[2] = {};
+  cudaStream_t copy_stream = nullptr, back_stream = nullptr;
   cudaEvent_t in_ready[2] = {}, in_free[2] = {};  // slot copied / slot read by its forward
-  bool in_used[2] = {false, false};
-  int in_slot = 0;
+  cudaEvent_t z_ready[2] = {}, z_free[2] = {};    // slot written by its forward / slot read back
+  bool in_used[2] = {false, false}, z_used[2] = {false, false};
+  int in_slot = 0, z_last = -1;  // z_last: slot of the latest read-back, -1 before the first
   // one STCA forward between its phases (set by its first phase)
   struct Fwd {
     int B = 0, n_tok = 0, t_tot = 0, splits = 1;
@@ -313,7 +315,7 @@ int allocate(stca_handle* h) {
            dalloc(h, &h->in_tpu[b], U * 4) && dalloc(h, &h->in_xt[b], T * d * E);
       if (c.time_buckets) ok = ok && dalloc(h, &h->in_dt[b], N * 4);
     }
-    ok = ok && dalloc(h, &h->out_z, T * d * 4);
+    ok = ok && dalloc(h, &h->out_z[0], T * d * 4) && dalloc(h, &h->out_z[1], T * d * 4);
     if (c.dtype == STCA_BF16) {
       h->ql = q_layout(c);
       ok = ok && dalloc(h, &h->qpack, h->ql.total * 2);
@@ -809,10 +811,14 @@ void stca_destroy(stca_handle* h) {
   for (cudaEvent_t e : h->spare) cudaEventDestroy(e);
   if (h->copy_stream) {
     cudaStreamSynchronize(h->copy_stream);
+    cudaStreamSynchronize(h->back_stream);
     cudaStreamDestroy(h->copy_stream);
+    cudaStreamDestroy(h->back_stream);
     for (int b = 0; b < 2; ++b) {
       cudaEventDestroy(h->in_ready[b]);
       cudaEventDestroy(h->in_free[b]);
+      cudaEventDestroy(h->z_ready[b]);
+      cudaEventDestroy(h->z_free[b]);
     }
   }
   free_all(h);
@@ -845,10 +851,13 @@ int stca_forward_host(stca_handle* h, const int32_t* ids, const int32_t* lens, c
   const size_t E = esize(h->cfg);
   const size_t d = size_t(h->cfg.d);
   if (!h->copy_stream) {
-    bool made = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking) == cudaSuccess;
+    bool made = cudaStreamCreateWithFlags(&h->copy_stream, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaStreamCreateWithFlags(&h->back_stream, cudaStreamNonBlocking) == cudaSuccess;
     for (int b = 0; b < 2; ++b)
       made = made && cudaEventCreateWithFlags(&h->in_ready[b], cudaEventDisableTiming) == cudaSuccess &&
-             cudaEventCreateWithFlags(&h->in_free[b], cudaEventDisableTiming) == cudaSuccess;
+             cudaEventCreateWithFlags(&h->in_free[b], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&h->z_ready[b], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&h->z_free[b], cudaEventDisableTiming) == cudaSuccess;
     if (!made) return STCA_ERR_CUDA;
   }
   // this call's inputs go to slot b on the copy stream, once the forward that read slot b
@@ -864,20 +873,38 @@ int stca_forward_host(stca_handle* h, const int32_t* ids, const int32_t* lens, c
   if (t_tot > 0)
     ok = ok && cudaMemcpyAsync(h->in_xt[b], x_t, size_t(t_tot) * d * E, cudaMemcpyHostToDevice, c) == cudaSuccess;
   ok = ok && cudaEventRecord(h->in_ready[b], c) == cudaSuccess && cudaStreamWaitEvent(s, h->in_ready[b], 0) == cudaSuccess;
+  // the forward writes output slot b once the read-back of the call before last has left it
+  ok = ok && (!h->z_used[b] || cudaStreamWaitEvent(s, h->z_free[b], 0) == cudaSuccess);
   if (!ok) return STCA_ERR_CUDA;
   h->in_slot ^= 1;
   const int rc = h->cfg.dtype == STCA_BF16
                      ? run_stca<bf16>(h, h->in_ids[b], h->in_len[b], h->in_dt[b], h->in_xt[b], h->in_tpu[b], B, n_tok,
-                                      t_tot, w, h->out_z, nullptr, s)
+                                      t_tot, w, h->out_z[b], nullptr, s)
                      : run_stca<float>(h, h->in_ids[b], h->in_len[b], h->in_dt[b], h->in_xt[b], h->in_tpu[b], B,
-                                       n_tok, t_tot, w, h->out_z, nullptr, s);
+                                       n_tok, t_tot, w, h->out_z[b], nullptr, s);
   // slot b is free for the call after next once this forward has read it (recorded even
   // when the forward returned early, so that call never waits on a stale event)
   h->in_used[b] = cudaEventRecord(h->in_free[b], s) == cudaSuccess;
   CK(rc);
-  if (t_tot > 0 && cudaMemcpyAsync(z_host, h->out_z, size_t(t_tot) * d * 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-    return STCA_ERR_CUDA;
+  // z goes back on back_stream, so the next call's forward does not queue behind the copy
+  cudaStream_t r = h->back_stream;
+  ok = cudaEventRecord(h->z_ready[b], s) == cudaSuccess && cudaStreamWaitEvent(r, h->z_ready[b], 0) == cudaSuccess;
+  if (t_tot > 0)
+    ok = ok && cudaMemcpyAsync(z_host, h->out_z[b], size_t(t_tot) * d * 4, cudaMemcpyDeviceToHost, r) == cudaSuccess;
+  h->z_used[b] = ok && cudaEventRecord(h->z_free[b], r) == cudaSuccess;
+  if (!h->z_used[b]) return STCA_ERR_CUDA;
+  h->z_last = b;
   return STCA_OK;
+}
+
+int stca_host_fence(stca_handle* h, void* stream) {
+  if (!h) return STCA_ERR_INVALID_ARG;
+  if (h->z_last < 0) return STCA_OK;
+  if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
+  // back_stream runs its copies in call order, so the latest one landing means all have
+  return cudaStreamWaitEvent(reinterpret_cast<cudaStream_t>(stream), h->z_free[h->z_last], 0) == cudaSuccess
+             ? STCA_OK
+             : STCA_ERR_CUDA;
 }
 
 // ---- sequence-parallel (L-split) forward in phases: every rank holds a slice of each
@@ -1194,6 +1221,7 @@ int stca_sync_status(stca_handle* h) {
   if (!h) return STCA_ERR_INVALID_ARG;
   if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
   if (cudaStreamSynchronize(h->last_stream) != cudaSuccess) return STCA_ERR_CUDA;
+  if (h->back_stream && cudaStreamSynchronize(h->back_stream) != cudaSuccess) return STCA_ERR_CUDA;
   int32_t e = 0;
   if (cudaMemcpy(&e, h->err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return STCA_ERR_CUDA;
   if (e != 0 && cudaMemset(h->err, 0, 4) != cudaSuccess) return STCA_ERR_CUDA;

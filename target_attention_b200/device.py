@@ -132,6 +132,10 @@ class StcaModel(_Holder):
         return B.stca_forward_host(self.handle, x["ids"], x["lengths"], x["dt"], x["x_t"], x["targets_per_user"],
                                    x["B"], x["n_tok"], x["t_tot"], self.weights, z_out, stream)
 
+    def host_fence(self, stream=None):
+        """`stream` waits for the z read-backs of the forward_host calls so far."""
+        return B.stca_host_fence(self.handle, stream)
+
     def close(self):
         if getattr(self, "handle", None) is not None:
             B.stca_destroy(self.handle)

@@ -159,6 +159,33 @@ def test_host_buffer_entry_back_to_back_calls():
     m.close()
 
 
+def test_host_buffer_entry_fence_on_caller_stream():
+    """Back-to-back host-buffer calls on a side stream, completed by stca_host_fence on that
+    stream and a synchronisation of that stream alone (no device-wide synchronise): every
+    z read-back has landed, each equal to the device entry's result."""
+    wl = make_stca(3, users=2, L=350, n_items=10_000)
+    m = StcaModel(wl)
+    side = torch.cuda.Stream()
+    assert m.host_fence(side) == B.OK  # nothing enqueued yet
+    inputs = [m.inputs(make_stca(3, users=2, L=350, n_items=10_000, data_seed=200 + i)) for i in range(4)]
+    want = []
+    for x in inputs:
+        z = torch.empty((x["t_tot"], 512), device=dev)
+        B.check(m.forward(x, z))
+        want.append(z.cpu().numpy())
+    hosts = [{k: (v.cpu().pin_memory() if torch.is_tensor(v) else v) for k, v in x.items()} for x in inputs]
+    outs = [torch.full((x["t_tot"], 512), float("nan"), pin_memory=True) for x in inputs]
+    torch.cuda.synchronize()
+    for xh, zh in zip(hosts, outs):
+        B.check(m.forward_host(xh, zh, stream=side))
+    B.check(m.host_fence(side))
+    side.synchronize()
+    for zh, w in zip(outs, want):
+        np.testing.assert_array_equal(zh.numpy(), w)
+    assert B.stca_sync_status(m.handle) == B.OK
+    m.close()
+
+
 # ---------------------------------------------------------------- pointwise ReLU TA
 
 
