@@ -7,8 +7,11 @@
 // terms hi = bf16(a) and lo = bf16(a - hi), both multiplied by the same bf16 weight and
 // accumulated in fp32, so every product is within ~2^-17 relative of the fp32 product.
 //
-// One CTA computes a 128-row x 256-column tile with cta_group::1 MMAs (M = 128, N = 256,
-// K = 16) into 256 TMEM columns.  K streams through a 3-stage ring of 64-wide chunks: the
+// One CTA computes a 128-row x BN-column tile with cta_group::1 MMAs (M = 128, N = BN,
+// K = 16) into BN TMEM columns; BN = 256, or 128 / 64 for plain GEMMs whose 256-column
+// grid would leave SMs idle (a few hundred target rows: every launch is then a chain of
+// MMA latencies, and narrower tiles both spread it over more SMs and shorten each MMA).
+// K streams through a 3-stage ring of 64-wide chunks: the
 // weight chunk arrives by TMA (K-major packed weights, 128-byte swizzle); eight producer
 // warps load the fp32 activation rows (three chunks in flight), split them and store the
 // hi and lo tiles in the same swizzled layout.  Those warps then run the epilogue (two per
@@ -24,11 +27,15 @@ namespace stca {
 
 namespace {
 
-constexpr int QBM = 128, QBN = 256, QKC = 64, QSTAGES = 3;
+constexpr int QBM = 128, QKC = 64, QSTAGES = 3;
 constexpr int QA_TILE = QBM * QKC * 2;          // one bf16 activation tile: 16 KB
-constexpr int QB_TILE = QBN * QKC * 2;          // one weight chunk: 32 KB
-constexpr int QSTAGE = 2 * QA_TILE + QB_TILE;   // hi | lo | weights: 64 KB
-constexpr size_t QSMEM = 1024 + size_t(QSTAGES) * QSTAGE + 256;
+template <int BN>
+struct QShape {
+  static constexpr int B_TILE = BN * QKC * 2;            // one weight chunk: 8, 16 or 32 KB
+  static constexpr int STAGE = 2 * QA_TILE + B_TILE;     // hi | lo | weights
+  static constexpr size_t SMEM = 1024 + size_t(QSTAGES) * STAGE + 256;
+  static_assert(QSTAGES * STAGE >= 8 * 8192, "the epilogue stages its blocks in the ring");
+};
 
 struct TcqArgs {
   const float* A;
@@ -69,9 +76,11 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-template <bool DUAL>
+template <bool DUAL, int BN>
 __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant__ CUtensorMap tmB,
                                                           const __grid_constant__ CUtensorMap tmC, TcqArgs a) {
+  static_assert(!DUAL || BN == 256, "the SwiGLU pair is packed as 128 gate + 128 up rows");
+  constexpr int QB_TILE = QShape<BN>::B_TILE, QSTAGE = QShape<BN>::STAGE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = q_align1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + QSTAGES * QSTAGE);
@@ -85,7 +94,7 @@ __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * QBM;
   const int z = blockIdx.z;
-  const int wrow0 = z * a.wrows + blockIdx.x * QBN;  // first packed weight row of this tile
+  const int wrow0 = z * a.wrows + blockIdx.x * BN;  // first packed weight row of this tile
   const int KC = a.K / QKC;
   const float* A = a.A + z * a.bsA;
   float* C = a.C + z * a.bsC;
@@ -102,7 +111,7 @@ __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant_
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, QBN);
+    tmem_alloc(tmem_slot, BN);
     tmem_relinquish();
   }
   if (threadIdx.x == 0) prefetch_tmap(&tmB);
@@ -137,7 +146,7 @@ __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant_
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t idesc = umma_idesc_bf16(QBM, QBN);
+      constexpr uint32_t idesc = umma_idesc_bf16(QBM, BN);
       // lean issue loop: descriptor bases advance by constant steps (16-byte units)
       const uint64_t desc0 = umma_sdesc_sw128(smem_u32(smem));
       bool ok = true;
@@ -252,7 +261,7 @@ __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant_
       // (now idle) operand ring, rows 128-byte swizzled, and TMA writes whole rows; rows or
       // columns outside C are clipped.  Otherwise each lane stores its own row.
       uint8_t* stage = smem + (warp - 4) * 8192;
-      constexpr int NCH = DUAL ? 2 : 4;  // 32-column output chunks per warp
+      constexpr int NCH = DUAL ? 2 : BN / 64;  // 32-column output chunks per warp
 #pragma unroll 1
       for (int j = 0; j < NCH; ++j) {
         const int tc = half * NCH * 32 + j * 32;  // accumulator column (gate half when DUAL)
@@ -267,7 +276,7 @@ __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant_
         } else {
           tmem_ld_wait();
         }
-        const int col = (DUAL ? blockIdx.x * 128 : blockIdx.x * QBN) + tc;
+        const int col = (DUAL ? blockIdx.x * 128 : blockIdx.x * BN) + tc;
         if (col >= a.N) continue;  // warp-uniform
         if (rrow) {
 #pragma unroll
@@ -306,7 +315,7 @@ __global__ void __launch_bounds__(384, 1) tc_query_kernel(const __grid_constant_
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, QBN);
+    tmem_dealloc(tmem, BN);
   }
 }
 
@@ -322,7 +331,7 @@ bool tc_query_supported(const SimtGemmArgs<float, bf16>& a) {
   if (a.batch > 1) {
     // per-batch weights sit back to back in the packed buffer, whole 256-row tiles each
     const int wrows = a.B2 ? 2 * a.N : a.N;
-    if (wrows % QBN != 0 || a.bsA % 4 != 0 || a.bsC % 4 != 0 || a.bsR % 4 != 0) return false;
+    if (wrows % 256 != 0 || a.bsA % 4 != 0 || a.bsC % 4 != 0 || a.bsR % 4 != 0) return false;
   }
   return true;
 }
@@ -333,8 +342,12 @@ int tc_query_gemm(const SimtGemmArgs<float, bf16>& a, const void* Wp, cudaStream
   const bool dual = a.B2 != nullptr;
   // packed rows: N (plain), or 256 per 128 output columns (gate and up halves)
   const int wrows = dual ? 2 * a.N : a.N;
+  // column tile: 256, unless that grid would fill under ~4/5 of the SMs (plain GEMMs only)
+  auto ctas = [&](int bn) { return int64_t((wrows + bn - 1) / bn) * ((a.M + QBM - 1) / QBM) * a.batch; };
+  const int64_t fill = int64_t(sm_count()) * 4 / 5;
+  const int bn = dual || ctas(256) >= fill ? 256 : (ctas(128) >= fill ? 128 : 64);
   CUtensorMap tb;
-  if (!make_tmap(&tb, Wp, uint64_t(wrows) * a.batch, uint64_t(a.K), uint64_t(a.K), QBN)) return STCA_ERR_CUDA;
+  if (!make_tmap(&tb, Wp, uint64_t(wrows) * a.batch, uint64_t(a.K), uint64_t(a.K), bn)) return STCA_ERR_CUDA;
   TcqArgs q;
   q.A = a.A;
   q.lda = a.lda;
@@ -366,9 +379,12 @@ int tc_query_gemm(const SimtGemmArgs<float, bf16>& a, const void* Wp, cudaStream
   } else {
     tc = tb;  // unused
   }
-  const dim3 grid((wrows + QBN - 1) / QBN, (a.M + QBM - 1) / QBM, a.batch);
-  auto kern = dual ? tc_query_kernel<true> : tc_query_kernel<false>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(QSMEM)) != cudaSuccess)
+  const dim3 grid((wrows + bn - 1) / bn, (a.M + QBM - 1) / QBM, a.batch);
+  auto kern = dual ? tc_query_kernel<true, 256>
+                   : (bn == 256 ? tc_query_kernel<false, 256>
+                                : (bn == 128 ? tc_query_kernel<false, 128> : tc_query_kernel<false, 64>));
+  const size_t smem = bn == 256 ? QShape<256>::SMEM : (bn == 128 ? QShape<128>::SMEM : QShape<64>::SMEM);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
   // programmatic dependent launch: the CTAs may start (barriers, TMEM, descriptor prefetch)
   // while the previous kernel on the stream drains; the kernel waits for it before any data
@@ -376,7 +392,7 @@ int tc_query_gemm(const SimtGemmArgs<float, bf16>& a, const void* Wp, cudaStream
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = grid;
   cfg.blockDim = dim3(384);
-  cfg.dynamicSmemBytes = QSMEM;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -197,6 +197,8 @@ def _f32(a):
 
 @pytest.mark.parametrize("M, K, N, dual, split, resid", [
     (8192 + 77, 512, 512, False, False, False),   # many row tiles and a ragged tail
+    (4096, 512, 512, False, False, True),         # 128-column tiles (a 256-wide grid fills too few SMs)
+    (512, 256, 256, False, False, False),         # 64-column tiles
     (300, 1536, 512, False, True, True),          # two concatenated A blocks, residual
     (129, 512, 1024, True, False, False),         # SwiGLU pair
     (1, 1024, 96, False, False, False),           # one row; N not a multiple of the tile
