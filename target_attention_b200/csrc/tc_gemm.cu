@@ -77,7 +77,10 @@ constexpr int A_CHUNK = BM * 64 * 2;           // one 64-wide K chunk of A: 16 K
 constexpr int B_HALF = BM * 128;               // one CTA's 128 weight rows x 64 K: 16 KB
 constexpr int OUT_STAGE = 32 * 64;             // one epilogue warp's 32 x 32 bf16 output tile
 constexpr int MIN_SMEM = 120 * 1024;           // keeps one CTA per SM (TMEM is not shared)
-constexpr int GATHER_LAG = 2;                  // gathered chunks in flight before one is published
+constexpr int GATHER_LAG = 2;
+// N tiles before the end of a row tile at which the gather prefetches the next row
+// tile's table rows into L2
+constexpr int PREFETCH_LEAD = 3;                  // gathered chunks in flight before one is published
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -213,6 +216,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
   uint64_t* mma_done = t_empty + 2;        // [1]      leader
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // N tiles whose accumulators this CTA's epilogue has received (times the gather's L2
+  // prefetch of the next row tile)
+  volatile int* progress = abort_flag + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
@@ -222,6 +228,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
   const int cl = blockIdx.x >> 1, ncl = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
+    *progress = 0;
     for (int i = 0; i < KC; ++i) {
       mbar_init(&a_full[i], AMODE == A_GATHER ? 256 : 1);
       mbar_init(&a_empty[i], 1);
@@ -367,18 +374,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
           const bool v = gather_row(g, tile * 2 * BM + int(rank) * BM + gw * 32 + i * 4 + sub, M, idl, bks[i],
                                     c == 0 ? err : nullptr);
           ids[i] = int32_t(idl);
-          if (v) {
-            mask |= 1u << i;
-            if (c == 0) prefetch_l2_bulk(table + idl * K, uint32_t(K) * 2);
-          }
+          if (v) mask |= 1u << i;
         }
       };
-      if (cl < num_tiles) rows_of(cl, id, bk, vmask);
+      auto prefetch_rows = [&](const int32_t (&ids)[8], uint32_t mask) {
+        if (c != 0) return;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if ((mask >> i) & 1u) prefetch_l2_bulk(table + int64_t(ids[i]) * K, uint32_t(K) * 2);
+      };
+      if (cl < num_tiles) {
+        rows_of(cl, id, bk, vmask);
+        prefetch_rows(id, vmask);
+      }
       if (store_x && lane == 0) prefetch_tmap(&tmX);
       int li = 0;
       bool ok = true;
       for (int tile = cl; tile < num_tiles && ok; tile += ncl, ++li) {
-        // this lane's rows of the next tile (and an L2 prefetch of them) while this one is in flight
+        // this lane's rows of the next tile while this one is in flight (prefetched into L2
+        // below, a few N tiles before the gather needs them: prefetched a whole row tile
+        // ahead, the rows were evicted by the hidden stream again and read from DRAM twice)
         const int next = tile + ncl;
         if (next < num_tiles) rows_of(next, nid, nbk, nvmask);
         else nvmask = 0;
@@ -448,6 +463,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
           cp_async_wait_dyn(KC - 1 - kc);
           publish(kc);
         }
+        if (nvmask) {
+          // wait (bounded; the prefetch is only a hint) until all but the last few N tiles
+          // of this row tile have left the tensor cores, then prefetch the next tile's rows
+          const int target = li * NT + (NT > PREFETCH_LEAD ? NT - PREFETCH_LEAD : 0);
+          for (int it = 0; it < 16384 && *progress < target && !abort_set(abort_flag); ++it) __nanosleep(256);
+          prefetch_rows(nid, nvmask);
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           id[i] = nid[i];
@@ -476,6 +498,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
           ok = false;
           break;
         }
+        if (AMODE == A_GATHER && warp == 4 && lane == 0) *progress = gnt + 1;
         tc_fence_after();
         const uint32_t tb = lane_base + buf * 256;
         if (EPI == EPI_SWIGLU) {
