@@ -77,10 +77,10 @@ constexpr int A_CHUNK = BM * 64 * 2;           // one 64-wide K chunk of A: 16 K
 constexpr int B_HALF = BM * 128;               // one CTA's 128 weight rows x 64 K: 16 KB
 constexpr int OUT_STAGE = 32 * 64;             // one epilogue warp's 32 x 32 bf16 output tile
 constexpr int MIN_SMEM = 120 * 1024;           // keeps one CTA per SM (TMEM is not shared)
-constexpr int GATHER_LAG = 2;
+constexpr int GATHER_LAG = 2;                  // gathered chunks in flight before one is published
 // N tiles before the end of a row tile at which the gather prefetches the next row
 // tile's table rows into L2
-constexpr int PREFETCH_LEAD = 3;                  // gathered chunks in flight before one is published
+constexpr int PREFETCH_LEAD = 3;
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
