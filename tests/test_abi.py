@@ -93,6 +93,7 @@ def test_null_arguments_rejected_on_host():
     assert L.stca_lsplit_merge(None, 0, 2, None, None, None, None) == B.ERR_INVALID_ARG
     assert L.stca_k_wait_selftest(None, None) == B.ERR_INVALID_ARG
     assert L.stca_stream_wait(None, -1) == B.ERR_INVALID_ARG
+    assert L.stca_host_fence(None, None) == B.ERR_INVALID_ARG
     L.stca_unpin_weights(None)
     L.stca_destroy(None)
     # kernel-level entry points validate before launching
