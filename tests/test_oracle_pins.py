@@ -216,6 +216,50 @@ def test_single_token_history_closed_form():
                 np.testing.assert_allclose(o[i, t], expect, rtol=1e-11, atol=1e-12)
 
 
+def _torch_mha(d, H, WQ, WK, WV, WO):
+    """torch's own multi-head attention module in fp64, bias-free, holding the weights
+    given in the pages' [in, out] convention (torch stores [out, in])."""
+    mha = torch.nn.MultiheadAttention(d, H, bias=False, batch_first=True, dtype=torch.float64)
+    with torch.no_grad():
+        mha.in_proj_weight.copy_(torch.cat([torch.from_numpy(_f64(W)).T for W in (WQ, WK, WV)]))
+        mha.out_proj.weight.copy_(torch.from_numpy(_f64(WO)).T)
+    return mha
+
+
+@pytest.mark.parametrize("score_layers", [1, 2])
+def test_stca_score_path_vs_torch_multihead_attention(score_layers):
+    """Each layer's o^(i) is standard multi-head attention of the one query q^(i) over the
+    user's X~^(i) ([review] 核心公式: alpha = softmax(q W_Q (X~ W_K)^T / sqrt(d_h)),
+    o = alpha X~ W_V, heads joined by W_O).  torch.nn.MultiheadAttention does the
+    projections, the head split and the 1/sqrt(d_h) scale itself, so a wrong scale, a
+    swapped W_Q/W_K or a wrong head slice in the oracle fails here.  LayerNorm and SiLU
+    come from torch's functional ops."""
+    d, H, L = 64, 4, 7
+    wl = make_stca(2, users=1, lengths=np.array([L], np.int32), n_items=100, d=d, H=H, hidden=128, m=2,
+                   M=score_layers)
+    cfg, w = wl["cfg"], wl["weights"]
+    _, o = R.stca_forward(wl)
+    t = lambda a: torch.from_numpy(_f64(a))
+
+    def ln_swiglu(x, f, ln=True):
+        y = (F.silu(x @ t(f["W1"])) * (x @ t(f["W3"]))) @ t(f["W2"])
+        return F.layer_norm(y, (d,), t(f["gamma"]), t(f["beta"]), 1e-5) if ln else y
+
+    X = t(wl["table"])[torch.from_numpy(wl["ids"].astype(np.int64))]
+    for k in range(2):
+        x_t = t(wl["x_t"][k])
+        q = ln_swiglu(x_t, w["tgt"])
+        outs = []
+        for i in range(score_layers):
+            Xt = ln_swiglu(X, w["hist"][i])
+            mha = _torch_mha(d, H, w["WQ"][i], w["WK"][i], w["WV"][i], w["WO"][i])
+            oi, _ = mha(q[None, None], Xt[None], Xt[None], need_weights=False)
+            outs.append(oi[0, 0].detach())
+            np.testing.assert_allclose(o[i, k], outs[-1].numpy(), rtol=1e-11, atol=1e-12)
+            if i + 1 < score_layers:
+                q = ln_swiglu(torch.cat(outs + [x_t]) @ t(w["WC"][i + 1]), w["fuse"][i + 1])
+
+
 def test_rlb_batched_equals_independent_targets():
     wl = _small_stca(2, users=2, m=5)
     z, o = R.stca_forward(wl)
@@ -351,6 +395,28 @@ def test_hyformer_zero_ffn_leaves_decoded_queries():
         for b in range(2):
             np.testing.assert_allclose(out[b, 16 * s:16 * s + 16], np.tile(expect, (16, 1)),
                                        rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("k", [5, 30])
+def test_hyformer_per_token_ffn_index(k):
+    """[hyformer] eq (14): mixed token k goes through its own SwiGLU (the k-th of T).  With
+    every per-token W2 zero except token k's, the boost is zero on every row but k, so
+    those rows equal the decoded queries Q^ exactly (eq 15), and row k differs from Q^ by
+    the SwiGLU of mixed token k (eq 11-13) through token k's weights."""
+    wl = make_hyformer(users=1, L_feed=9, L_search=4, n_items=60, d=64, hidden=128, H=4, blocks=1)
+    wl["table"] = R.to_f64(wl["table"]) * 50.0   # rows of norm ~8, so the boost is not tiny
+    tok = wl["weights"]["blocks"][0]["tok"]
+    keep = {key: R.to_f64(v) for key, v in tok[k].items()}
+    for f in tok:
+        f["W2"] = np.zeros_like(R.to_f64(f["W2"]))
+    qhat = R.hyformer_forward(wl)[0]          # all boosts zero: the decoded queries
+    tok[k]["W2"] = keep["W2"]
+    out = R.hyformer_forward(wl)[0]
+    others = np.arange(32) != k
+    np.testing.assert_array_equal(out[others], qhat[others])
+    boost = R.swiglu(R.token_mix(qhat)[k], keep)
+    assert np.abs(boost).max() > 1e-2 * np.abs(qhat[k]).max()
+    np.testing.assert_allclose(out[k] - qhat[k], boost, rtol=1e-10, atol=1e-14)
 
 
 def test_hyformer_residual_adds_boost():
