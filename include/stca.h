@@ -27,6 +27,9 @@
  *     [0, n_items), lengths that do not add up, a bounded wait that ran out) are
  *     recorded in the handle's device error word; the kernels never trap and keep
  *     going, and outputs are then undefined.  stca_sync_status() reads and clears it.
+ *     Lengths that add up to more than n_tok (targets_per_user to more than t_tot) are
+ *     cut at the declared total: the ragged offsets are clamped to it, so no kernel
+ *     reads or writes past the buffers that n_tok and t_tot describe.
  *   - A handle is not thread-safe; use one handle per host thread or serialise calls.
  */
 #ifndef STCA_H
@@ -223,8 +226,9 @@ int stca_pointwise_forward(stca_handle* h, const int32_t* ids, const int32_t* le
  * the GPU detects (an id out of range, lengths not adding up to n_tok) if it was 0, or
  * NULL.  Scratch lives in a fixed array of about 4.2 MB in the library's device image,
  * which every GPU that loads the library holds until the process exits; B above
- * STCA_NOALLOC_MAX_USERS returns STCA_ERR_CAPACITY.  The first call on a device looks up
- * that array's device address (make that first call before any stream capture).  All
+ * STCA_NOALLOC_MAX_USERS returns STCA_ERR_CAPACITY.  The first call on a device, and the
+ * first one after a cudaDeviceReset there, looks up that array's device address (make
+ * that call before any stream capture).  All
  * calls share the array: calls that overlap on the GPU (different streams, or different
  * host threads on the same device) race and give undefined results; calls serialised
  * on one stream are safe. */

@@ -17,8 +17,10 @@ extern "C" {
 
 /* Ragged layout ([notes] problem statement: one history of length L_u per user; RLB:
  * targets grouped per user).  offsets[0] = 0, offsets[i+1] = offsets[i] + lengths[i]
- * ([B+1] int32); records STCA_ERR_BAD_LENGTHS in err for a negative length or a total
- * different from `expected`. */
+ * ([B+1] int32), every entry clamped to min(prefix sum, expected) with negative lengths
+ * counted as 0, so offsets[B] <= expected always holds and no later kernel that trusts
+ * the offsets leaves buffers sized by `expected`; records STCA_ERR_BAD_LENGTHS in err
+ * for a negative length or a total different from `expected`. */
 int stca_k_offsets(const int32_t* lengths, int B, int32_t* offsets, int expected, int32_t* err, void* stream);
 
 /* Packs a bf16 weight W [K, N] (row-major, y = x W) into the K-major operand layout of

@@ -191,8 +191,9 @@ int sm_count();
 
 // ---------------------------------------------------------------- small kernels
 
-// offsets[0] = 0, offsets[i+1] = offsets[i] + lengths[i]; checks lengths >= 0 and the
-// total against `expected` (records STCA_ERR_BAD_LENGTHS otherwise).
+// offsets[0] = 0, offsets[i+1] = offsets[i] + lengths[i], each clamped to `expected`
+// (negative lengths count as 0); checks lengths >= 0 and the total against `expected`
+// (records STCA_ERR_BAD_LENGTHS otherwise).
 int exclusive_offsets(const int32_t* lengths, int B, int32_t* offsets, int expected, int32_t* err,
                       cudaStream_t s);
 // dst[r, col0 + c] = float(src[r, c]) for c < d (src bf16 or fp32 by `src_bf16`).

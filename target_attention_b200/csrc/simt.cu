@@ -173,13 +173,17 @@ __global__ void layer_norm_kernel(const float* __restrict__ x, int64_t ldx, floa
   }
 }
 
-// Exclusive scan of B lengths in one block; validates signs and the total.
+// Exclusive scan of B lengths in one block; validates signs and the total. Every offset,
+// offsets[B] included, is clamped to `expected` (the caller's declared total, which sized its
+// buffers), so that lengths which sum above it are reported but can never send a later kernel
+// past the end of an id, row or output buffer. Negative lengths count as 0.
 __global__ void offsets_kernel(const int32_t* __restrict__ lengths, int B, int32_t* __restrict__ offsets,
                                int expected, int32_t* err) {
   griddep_wait();
   griddep_launch();
   __shared__ long long warp_sums[32];
   __shared__ long long carry;
+  const long long cap = expected > 0 ? expected : 0;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) carry = 0;
   __syncthreads();
@@ -212,13 +216,13 @@ __global__ void offsets_kernel(const int32_t* __restrict__ lengths, int B, int32
     }
     __syncthreads();
     const long long excl = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + incl - v;
-    if (i < B) offsets[i] = int32_t(excl > 0x7fffffffLL ? 0x7fffffffLL : excl);
+    if (i < B) offsets[i] = int32_t(excl < cap ? excl : cap);
     __syncthreads();
     if (tid == 0) carry += warp_sums[(blockDim.x >> 5) - 1];
     __syncthreads();
   }
   if (tid == 0) {
-    offsets[B] = int32_t(carry > 0x7fffffffLL ? 0x7fffffffLL : carry);
+    offsets[B] = int32_t(carry < cap ? carry : cap);
     if (carry != expected) set_error(err, STCA_ERR_BAD_LENGTHS);
   }
 }

@@ -55,6 +55,37 @@ def test_offsets_bit_exact_and_checks():
     assert err.item() == B.ERR_BAD_LENGTHS
 
 
+def _clamped_offsets(lengths, expected):
+    """Exclusive prefix sums with negative lengths counted as 0, each cut at `expected`."""
+    return np.minimum(R.exclusive_offsets(np.maximum(lengths, 0)), max(expected, 0))
+
+
+@pytest.mark.parametrize("case", ["far_above", "below", "negative", "zero_total"])
+def test_offsets_are_clamped_to_the_declared_total(case):
+    """Lengths that disagree with the declared total are reported and the offsets are cut
+    at that total, so that no later kernel leaves buffers sized by it."""
+    lengths = _rng(3).integers(0, 3000, size=2500).astype(np.int32)
+    total = int(lengths.sum())
+    if case == "far_above":
+        lengths[1234] = 1_000_000_000  # the sum is ~1e9 above the declared total
+        expected = total
+    elif case == "below":
+        expected = total + 777
+    elif case == "negative":
+        lengths[[3, 1800]] = [-5, -2_000_000_000]
+        expected = total // 2
+    else:
+        expected = 0
+    off = torch.full((2501,), -1, dtype=torch.int32, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_offsets(torch.from_numpy(lengths).to(dev), 2500, off, expected, err))
+    torch.cuda.synchronize()
+    got = off.cpu().numpy().astype(np.int64)
+    np.testing.assert_array_equal(got, _clamped_offsets(lengths, expected))
+    assert got[-1] <= expected and (np.diff(got) >= 0).all()
+    assert err.item() == B.ERR_BAD_LENGTHS
+
+
 # ---------------------------------------------------------------- weight packing
 
 

@@ -186,6 +186,53 @@ def test_host_buffer_entry_fence_on_caller_stream():
     m.close()
 
 
+def test_lengths_above_the_totals_are_cut_at_them():
+    """History lengths that add up to more than n_tok and target counts that add up to
+    more than t_tot are reported (ERR_BAD_LENGTHS) and cut at the declared totals: the
+    extra ids and target rows (valid, inside padded buffers here) are never used and no
+    z row past t_tot is written, so the result equals the run with consistent counts.
+    The handle has room for the extra tokens and targets, so the check stays inside every
+    buffer whatever the kernels do."""
+    wl = make_stca(2, users=5, n_items=20_000)
+    extra_tok, extra_tgt = 48, 3
+    m = StcaModel(wl, max_tokens=int(wl["lengths"].sum()) + extra_tok,
+                  max_targets=int(wl["targets_per_user"].sum()) + extra_tgt)
+    z_ok, _ = _run_stca(wl, with_o=False, model=m)
+    over = dict(wl, lengths=wl["lengths"].copy(), targets_per_user=wl["targets_per_user"].copy(),
+                ids=np.concatenate([wl["ids"], np.arange(extra_tok, dtype=np.int32) + 5]),
+                dt=None if wl["dt"] is None else np.concatenate([wl["dt"], np.zeros(extra_tok, np.int32)]),
+                x_t=np.concatenate([wl["x_t"], wl["x_t"][:extra_tgt]]))
+    over["lengths"][-1] += extra_tok
+    over["targets_per_user"][-1] += extra_tgt
+    x = m.inputs(over)
+    x["n_tok"], x["t_tot"] = int(wl["lengths"].sum()), int(wl["targets_per_user"].sum())
+    T, d = x["t_tot"], wl["cfg"]["d"]
+    z = torch.full((T + extra_tgt, d), float("nan"), device=dev)
+    B.check(m.forward(x, z), "stca_forward")
+    assert B.stca_sync_status(m.handle) == B.ERR_BAD_LENGTHS
+    m.close()
+    zc = z.cpu().numpy()
+    assert np.isnan(zc[T:]).all()
+    assert R.row_rel_err(zc[:T], z_ok) <= 1e-6
+
+
+def test_pointwise_lengths_above_n_tok_are_cut():
+    wl = make_pointwise(users=33, L=2500, L_lo=500, n_items=50_000, seed=81)
+    ref = _run_pointwise(wl)
+    n_tok, extra = int(wl["lengths"].sum()), 64
+    over = dict(wl, lengths=wl["lengths"].copy(),
+                ids=np.concatenate([wl["ids"], np.arange(extra, dtype=np.int32) + 7]))
+    over["lengths"][-1] += extra
+    m = PointwiseModel(over, max_tokens=n_tok + extra)
+    x = m.inputs(over)
+    x["n_tok"] = n_tok
+    out = torch.full((x["B"], 128), float("nan"), device=dev)
+    B.check(m.forward(x, out))
+    assert B.stca_sync_status(m.handle) == B.ERR_BAD_LENGTHS
+    m.close()
+    assert R.row_rel_err(out.cpu().numpy(), ref) <= 1e-6
+
+
 # ---------------------------------------------------------------- pointwise ReLU TA
 
 
