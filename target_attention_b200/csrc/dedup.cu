@@ -189,6 +189,16 @@ __device__ __forceinline__ uint32_t mix32(uint32_t x) {
   return x;
 }
 
+// Every token as its own entry with multiplicity 1 (the same attention result, no saving).
+__device__ void compact_per_token(const int32_t* __restrict__ rows, int h0, int L, int32_t* __restrict__ out_rows,
+                                  int32_t* __restrict__ out_mult, int32_t* __restrict__ out_len, int u) {
+  for (int i = threadIdx.x; i < L; i += blockDim.x) {
+    out_rows[h0 + i] = rows[h0 + i];
+    out_mult[h0 + i] = 1;
+  }
+  if (threadIdx.x == 0) out_len[u] = L;
+}
+
 __global__ void __launch_bounds__(SCAN_THREADS) compact_user_kernel(const int32_t* __restrict__ hoff,
                                                                     const int32_t* __restrict__ rows,
                                                                     int32_t* __restrict__ out_rows,
@@ -197,14 +207,11 @@ __global__ void __launch_bounds__(SCAN_THREADS) compact_user_kernel(const int32_
   griddep_wait();
   griddep_launch();
   extern __shared__ int32_t cu_smem[];
+  __shared__ int table_failed;
   const int u = blockIdx.x;
   const int h0 = hoff[u], L = hoff[u + 1] - h0;
   if (L >= CU_SLOTS) {  // too long for the table: every token is its own entry
-    for (int i = threadIdx.x; i < L; i += blockDim.x) {
-      out_rows[h0 + i] = rows[h0 + i];
-      out_mult[h0 + i] = 1;
-    }
-    if (threadIdx.x == 0) out_len[u] = L;
+    compact_per_token(rows, h0, L, out_rows, out_mult, out_len, u);
     return;
   }
   int cap = 64;
@@ -213,25 +220,36 @@ __global__ void __launch_bounds__(SCAN_THREADS) compact_user_kernel(const int32_
   int32_t* keys = cu_smem;
   int32_t* first = keys + CU_SLOTS;
   int32_t* cnt = first + CU_SLOTS;
+  if (threadIdx.x == 0) table_failed = 0;
   for (int i = threadIdx.x; i < cap; i += blockDim.x) {
     keys[i] = -1;
     first[i] = 0x7fffffff;
     cnt[i] = 0;
   }
   __syncthreads();
-  // insert (L < cap, so a free slot always exists)
+  // insert: L < cap, so a free slot always exists within cap probes; the probe count is
+  // bounded all the same, and a table that ran out sends the user to the per-token form
   for (int i = threadIdx.x; i < L; i += blockDim.x) {
     const int32_t r = rows[h0 + i];
     uint32_t slot = mix32(uint32_t(r)) & mask;
-    while (true) {
+    int probe = 0;
+    for (; probe < cap; ++probe) {
       const int32_t prev = atomicCAS(&keys[slot], -1, r);
       if (prev == -1 || prev == r) break;
       slot = (slot + 1) & mask;
+    }
+    if (probe == cap) {
+      table_failed = 1;
+      continue;
     }
     atomicMin(&first[slot], i);
     atomicAdd(&cnt[slot], 1);
   }
   __syncthreads();
+  if (table_failed) {
+    compact_per_token(rows, h0, L, out_rows, out_mult, out_len, u);
+    return;
+  }
   // first occurrences in token order, numbered by a block scan per chunk of tokens
   int base = 0;
   for (int c0 = 0; c0 < L; c0 += SCAN_THREADS) {
@@ -241,9 +259,17 @@ __global__ void __launch_bounds__(SCAN_THREADS) compact_user_kernel(const int32_
     if (i < L) {
       r = rows[h0 + i];
       uint32_t slot = mix32(uint32_t(r)) & mask;
-      while (keys[slot] != r) slot = (slot + 1) & mask;
-      f = first[slot] == i;
-      m = cnt[slot];
+      int probe = 0;
+      while (keys[slot] != r && probe < cap) {  // every key was inserted: found within cap probes
+        slot = (slot + 1) & mask;
+        ++probe;
+      }
+      if (probe < cap) {
+        f = first[slot] == i;
+        m = cnt[slot];
+      } else {
+        table_failed = 1;
+      }
     }
     int excl;
     const int total = block_exclusive_scan(f, excl);
@@ -252,6 +278,11 @@ __global__ void __launch_bounds__(SCAN_THREADS) compact_user_kernel(const int32_
       out_mult[h0 + base + excl] = m;
     }
     base += total;
+  }
+  __syncthreads();
+  if (table_failed) {  // a lookup that could not happen did: rewrite the user per token
+    compact_per_token(rows, h0, L, out_rows, out_mult, out_len, u);
+    return;
   }
   if (threadIdx.x == 0) out_len[u] = base;
 }
