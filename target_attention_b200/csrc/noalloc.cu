@@ -31,23 +31,63 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[sizeof(NoallocS
 
 constexpr int MAX_DEVICES = 64;
 std::mutex g_mutex;
-void* g_addr[MAX_DEVICES] = {};
+
+// The address is looked up once per device and context: it is kept with the id of the
+// context it was found in, and looked up again when the device's current context has
+// another id (after a cudaDeviceReset, the primary context is a new one and the array has
+// a new address).  Context ids come from the driver (cuCtxGetCurrent, cuCtxGetId), reached
+// through the runtime's entry-point query so the library needs no link against libcuda.
+struct ScratchAddr {
+  unsigned long long ctx_id;
+  void* addr;
+};
+ScratchAddr g_addr[MAX_DEVICES] = {};
+
+typedef int (*CtxGetCurrentFn)(void**);
+typedef int (*CtxGetIdFn)(void*, unsigned long long*);
+
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    looked_up = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    cudaGetLastError();
+  }
+  void* ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != 0 || !ctx) return false;
+  return get_id(ctx, id) == 0;
+}
 
 // Device address of the scratch array on the current device.  In host code the array's
-// name is only a host-side stand-in, so the address is looked up once per device.
+// name is only a host-side stand-in, so its device address is asked of the runtime, once
+// per device and context (see above; where the driver gives no context id, every call
+// asks).
 NoallocScratch* scratch_on_current_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return nullptr;
+  unsigned long long ctx_id = 0;
+  const bool have_id = current_context_id(&ctx_id);
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_addr[dev] == nullptr) {
+  if (!have_id || g_addr[dev].addr == nullptr || g_addr[dev].ctx_id != ctx_id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
       cudaGetLastError();
       return nullptr;
     }
-    g_addr[dev] = p;
+    g_addr[dev].addr = p;
+    g_addr[dev].ctx_id = have_id ? ctx_id : 0;
   }
-  return reinterpret_cast<NoallocScratch*>(g_addr[dev]);
+  return reinterpret_cast<NoallocScratch*>(g_addr[dev].addr);
 }
 
 __global__ void copy_error_word(const int32_t* src, int32_t* dst) {

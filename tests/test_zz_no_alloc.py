@@ -26,15 +26,21 @@ def _via_handle(wl):
     return out.cpu().numpy()
 
 
-def _via_noalloc(wl, table):
+def _via_noalloc(wl, table, n_tok=None, expect_err=0):
     ids, lengths, q = (to_device(wl[k], dev) for k in ("ids", "lengths", "q"))
     out = torch.full((len(wl["lengths"]), 128), float("nan"), device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
+    n_tok = int(wl["lengths"].sum()) if n_tok is None else n_tok
     B.check(B.stca_pointwise_forward_noalloc(ids, lengths, q, table, table.shape[0], len(wl["lengths"]),
-                                             int(wl["lengths"].sum()), out, err), "stca_pointwise_forward_noalloc")
+                                             n_tok, out, err), "stca_pointwise_forward_noalloc")
     torch.cuda.synchronize()
-    assert err.item() == 0
+    assert err.item() == expect_err
     return out.cpu().numpy()
+
+
+def _close(got, ref):
+    scale = np.maximum(np.abs(ref).max(axis=1, keepdims=True), 1e-6)
+    return (np.abs(got - ref) / scale).max() <= 1e-4
 
 
 def test_noalloc_matches_handle_entry_on_two_calls_in_a_row():
@@ -47,8 +53,35 @@ def test_noalloc_matches_handle_entry_on_two_calls_in_a_row():
         wl = dict(wl, table=wl1["table"])
         ref = _via_handle(wl)
         got = _via_noalloc(wl, table)
-        scale = np.maximum(np.abs(ref).max(axis=1, keepdims=True), 1e-6)
-        assert (np.abs(got - ref) / scale).max() <= 1e-4
+        assert _close(got, ref)
+
+
+def test_noalloc_reports_a_bad_id_and_the_next_call_starts_clean():
+    # the shared error word must not carry one call's error into the next call
+    wl = make_pointwise(users=40, L=3000, L_lo=100, n_items=50_000, seed=79)
+    table = to_device(wl["table"], dev)
+    bad = dict(wl, ids=wl["ids"].copy())
+    bad["ids"][17] = 50_000  # one past the last row
+    _via_noalloc(bad, table, expect_err=B.ERR_ID_OUT_OF_RANGE)
+    ref = _via_handle(wl)
+    got = _via_noalloc(wl, table)
+    assert _close(got, ref)
+
+
+def test_noalloc_cuts_lengths_at_n_tok():
+    # lengths that add up to more than n_tok are reported, and the histories are cut at
+    # n_tok: the ids past n_tok (valid rows here, inside the buffer) are never read, so
+    # the result equals that of the last sample's history ending at n_tok
+    wl = make_pointwise(users=33, L=2500, L_lo=500, n_items=50_000, seed=80)
+    table = to_device(wl["table"], dev)
+    n_tok = int(wl["lengths"].sum())
+    extra = 64
+    over = dict(wl, lengths=wl["lengths"].copy(),
+                ids=np.concatenate([wl["ids"], np.arange(extra, dtype=np.int32) + 123]))
+    over["lengths"][-1] += extra
+    ref = _via_handle(wl)
+    got = _via_noalloc(over, table, n_tok=n_tok, expect_err=B.ERR_BAD_LENGTHS)
+    assert _close(got, ref)
 
 
 def test_noalloc_rejects_batches_above_its_limit():
