@@ -39,6 +39,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "history tokens/s through STCA layer at L=10K"
 UNIT = "history tokens/s"
+NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, nominal (context beside the measured copy rate)
 
 
 def parse():
@@ -161,52 +162,133 @@ def config_block(wl, world, total_tokens=None):
 
 
 class ClockSampler:
-    """nvidia-smi samples of one GPU every 50 ms while the timed region runs."""
+    """SM clock, power and clock-event reasons of one GPU, sampled while the timed region
+    runs.  NVML is read from a host thread every 5 ms (a read of the GPU's state; nothing
+    is set), so even a timed region of a fraction of a second carries dozens of samples;
+    where NVML is missing, nvidia-smi samples every 20 ms.  ``start`` returns once the first
+    sample has landed; ``begin``/``end`` mark the timed window on the host clock (it covers
+    the GPU's work: the window closes after a synchronize), and only samples inside it are
+    summarised."""
 
-    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
-              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
-              "clocks_event_reasons.sw_power_cap"]
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    SMI_FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+                  "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+                  "clocks_event_reasons.sw_power_cap"]
 
-    def __init__(self, gpu_id):
-        self.gpu_id = gpu_id
-        self.proc = None
-        self.path = None
+    def __init__(self, gpu_uuid, period_s=0.005):
+        self.uuid, self.period = gpu_uuid, period_s
+        self.samples = []      # (t, sm_mhz, sm_max_mhz, power_w, set of reasons)
+        self.window = None
+        self.source = None
+        self._stop = None
+        self._thread = None
+        self._proc = None
+        self._path = None
+
+    # -- NVML
+    def _start_nvml(self):
+        import threading
+        import pynvml as nv
+        nv.nvmlInit()
+        h = nv.nvmlDeviceGetHandleByUUID(self.uuid)
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        sm_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    self.samples.append((time.monotonic(), sm, sm_max, pw, {n for n, b in bits.items() if r & b}))
+                except nv.NVMLError:
+                    pass
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+        self.source = f"NVML every {self.period * 1e3:.0f} ms"
+
+    # -- nvidia-smi fallback
+    def _start_smi(self):
+        fd, self._path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        self._t0 = time.monotonic()
+        self._proc = subprocess.Popen(
+            ["nvidia-smi", "-i", self.uuid, "--query-gpu=" + ",".join(self.SMI_FIELDS),
+             "--format=csv,noheader,nounits", "-lms", "20"],
+            stdout=open(self._path, "w"), stderr=subprocess.DEVNULL)
+        self.source = "nvidia-smi every 20 ms"
+
+    def _smi_rows(self):
+        rows = []
+        with open(self._path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == len(self.SMI_FIELDS):
+                    rows.append(parts)
+        return rows
 
     def start(self):
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            self._start_nvml()
+        except Exception:
+            self.source = None
+            try:
+                self._start_smi()
+            except (OSError, FileNotFoundError):
+                return
+        deadline = time.monotonic() + 5.0
+        while time.monotonic() < deadline:
+            if (self._thread is not None and self.samples) or (self._proc is not None and self._smi_rows()):
+                break
+            time.sleep(0.01)
+
+    def begin(self):
+        self.window = [time.monotonic(), None]
+
+    def end(self):
+        if self.window:
+            self.window[1] = time.monotonic()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "nvidia-smi unavailable"}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) == len(self.FIELDS):
-                    rows.append(parts)
-        os.unlink(self.path)
+        if self.source is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "no NVML and no nvidia-smi"}
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+            rows = list(self.samples)
+        else:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+            raw = self._smi_rows()
+            os.unlink(self._path)
+            # nvidia-smi lines carry no time stamp: spread them over the sampling span
+            t1 = time.monotonic()
+            rows = []
+            for i, r in enumerate(raw):
+                num = lambda v: float(v) if v.replace(".", "", 1).isdigit() else None
+                rows.append((self._t0 + (t1 - self._t0) * (i + 0.5) / max(len(raw), 1), num(r[0]), num(r[1]),
+                             num(r[2]), {n for n, v in zip(self.REASONS, r[3:]) if v == "Active"}))
+        if self.window and self.window[1] is not None:
+            rows = [r for r in rows if self.window[0] <= r[0] <= self.window[1]]
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "no samples"}
-        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        pw = [float(r[2]) for r in rows if r[2].replace(".", "", 1).isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = [n for i, n in enumerate(names) if any(r[3 + i] == "Active" for r in rows)]
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "power_w_max": max(pw) if pw else None, "samples": len(rows), "reasons": reasons}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        sm = [r[1] for r in rows if r[1]]
+        mx = [r[2] for r in rows if r[2]]
+        pw = [r[3] for r in rows if r[3]]
+        counts = {n: sum(n in r[4] for r in rows) for n in self.REASONS}
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_mhz_min": min(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "power_w_max": max(pw) if pw else None,
+                "samples": len(rows), "reasons": [n for n in self.REASONS if counts[n]],
+                "reason_samples": {n: c for n, c in counts.items() if c}, "source": self.source}
 
 
 def clocks_rejected(clk):
@@ -401,17 +483,18 @@ def run_ours(args):
     def timed_region():
         B.check(B.stca_profile_stages(model.handle, [dom]))
         sampler = ClockSampler(uuid)
+        sampler.start()  # returns once the first sample is in
         n0 = B.stca_launch_count()
         barrier()
         torch.cuda.synchronize()
-        sampler.start()
-        time.sleep(0.3)
+        sampler.begin()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
+        sampler.end()
         barrier()
         clk = sampler.stop()
         launches = B.stca_launch_count() - n0
@@ -450,7 +533,8 @@ def run_ours(args):
                          frac=round(ach / peaks["bf16_tflops_sustained"], 4))
         elif bound == "hbm":
             ach = work * args.steps / (tot / 1e3) / 1e9
-            entry.update(bound="hbm", achieved_gbs=round(ach, 1), frac=round(ach / peaks["hbm_gbs"], 4))
+            entry.update(bound="hbm", achieved_gbs=round(ach, 1), frac=round(ach / peaks["hbm_gbs"], 4),
+                         frac_of_nominal=round(ach / NOMINAL_HBM_GBS, 4))
         stages[name] = entry
     bound, work, unit = stage_work(dom, wl, dedup)
     tot, calls = prof_dom[dom]
@@ -467,6 +551,13 @@ def run_ours(args):
                 "timing": "CUDA events around this kernel's launches inside the timed region"}
     if bound == "tensor":  # the same against the burst figure (a GEMM timed alone at full clocks)
         roofline["frac_of_burst_peak"] = round(achieved / peaks["bf16_tflops"], 4)
+    else:
+        roofline["frac_of_nominal"] = round(achieved / NOMINAL_HBM_GBS, 4)
+        roofline["nominal_peak"] = NOMINAL_HBM_GBS
+    if clk.get("sm_mhz") and clk.get("sm_max_mhz"):
+        # the step time scaled to what it would be in SM cycles at the maximum clock: compares
+        # runs on boxes whose power cap held the clock at different levels
+        clk["ms_per_step_x_clock_over_max"] = round(ms_step * clk["sm_mhz"] / clk["sm_max_mhz"], 4)
 
     # the same step with the history GEMMs run per token (dedup off), for reference
     per_token = None
