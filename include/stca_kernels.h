@@ -63,8 +63,10 @@ int stca_k_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, in
                         const float* beta, float eps, void* C, int ldc, int32_t* err, void* stream);
 
 /* Split-L cross attention plus merge ([review] 核心公式; [wechat] §1.1 local attention,
- * then merge; §1.2 ReLU scores).  Q [T, d] fp32 projected queries, KV [N, 2d] (K in
- * columns [0, d), V in [d, 2d)) bf16 when kv_bf16 else fp32, hoff/toff [B+1] offsets of
+ * then merge; §1.2 ReLU scores).  Q [T, d] fp32 projected queries.  KV bf16 when kv_bf16:
+ * [N, H, 2 d_h], row n holding [K_h | V_h] of head h in columns [2 h d_h, 2 (h+1) d_h) (the
+ * layout the library's K/V GEMM writes); else fp32 [N, 2d] (K in columns [0, d), V in
+ * [d, 2d)).  hoff/toff [B+1] offsets of
  * the users' keys and queries.  score 0 softmax, 1 relu.  1 <= splits <= 32 slices of each
  * user's keys (else STCA_ERR_INVALID_ARG).  part_acc [splits, T, d] and part_ml
  * [splits, T, H, 2] float32 scratch; out [T, d] float32. */

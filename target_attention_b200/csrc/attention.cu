@@ -20,6 +20,7 @@ namespace stca {
 namespace {
 
 constexpr float LOG2E = 1.4426950408889634f;
+constexpr float LN2 = 0.6931471805599453f;
 constexpr float RESCALE_SLACK = 8.f;  // log2 units a running max may lag the true max
 
 __device__ __forceinline__ void slice_bounds(const AttnArgs& a, int u, int s, int64_t& k0, int& nk, int& t0, int& m) {
@@ -59,25 +60,6 @@ static_assert(KV_STAGES == 2 || KV_STAGES == 3, "the index copy schedule below i
 constexpr int IDX_BYTES = TEAMS * IDX_STAGES * 2 * KT * 4;
 constexpr int ATTN_SMEM = RING_BYTES + IDX_BYTES;    // two CTAs per SM
 
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
 // Named barrier of one team's 64 threads (ids 1..TEAMS; 0 is __syncthreads).
 __device__ __forceinline__ void team_sync(int team) {
   asm volatile("bar.sync %0, 64;" ::"r"(team + 1) : "memory");
@@ -96,10 +78,11 @@ __device__ __forceinline__ void copy_tile_index(int* slot, const int32_t* kv_row
 
 // Issues this thread's cp.async copies of the K and V slices of head h for a tile: chunk
 // tt % 8 of keys tt / 8 + 8 i, i = 0..3 (128-byte key rows, 16-byte chunk c of key k at
-// chunk c ^ (k % 8)).  Rows come from the tile's index slot, or are row0 + key; keys past
-// the slice end are zero-filled.
+// chunk c ^ (k % 8)).  K/V rows are head-interleaved ([K_h | V_h] at column kvcol = 2 h d_h),
+// so a key's K and V slices of head h are one contiguous 256-byte segment.  Rows come from
+// the tile's index slot, or are row0 + key; keys past the slice end are zero-filled.
 __device__ __forceinline__ void load_kv_tile(uint8_t* stage, const int* slot, int64_t row0, int valid,
-                                             const bf16* KV, int64_t ld, int hcol, int d, int tt) {
+                                             const bf16* KV, int64_t ld, int kvcol, int tt) {
   uint8_t* sK = stage;
   uint8_t* sV = stage + TILE_BYTES;
   const int ch = tt & 7;
@@ -108,10 +91,10 @@ __device__ __forceinline__ void load_kv_tile(uint8_t* stage, const int* slot, in
     const int key = (tt >> 3) + 8 * i;
     const bool ok = key < valid;
     const int64_t row = ok ? (slot ? int64_t(slot[key]) : row0 + key) : 0;
-    const bf16* src = KV + row * ld + hcol + ch * 8;
+    const bf16* src = KV + row * ld + kvcol + ch * 8;
     const int off = key * 128 + ((ch ^ (key & 7)) << 4);
     cp_async_16(sK + off, src, ok ? 16u : 0u);
-    cp_async_16(sV + off, src + d, ok ? 16u : 0u);
+    cp_async_16(sV + off, src + DH, ok ? 16u : 0u);
   }
 }
 
@@ -119,7 +102,7 @@ __device__ __forceinline__ void load_kv_tile(uint8_t* stage, const int* slot, in
 // groups of 8 keys starting at group j0, then O += P V.  State per row half hr (rows g and
 // g + 8 of the warp's 16): running reference point mrow and sum lrow (softmax), O in o.
 template <int SCORE, int NJ>
-__device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, const int* smul, int j0,
+__device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, const float* smul, int j0,
                                           const uint32_t (&qa)[4][4], float (&o)[8][4], float (&mrow)[2],
                                           float (&lrow)[2], int valid, int lane) {
   const int tq = lane & 3;
@@ -165,7 +148,7 @@ __device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, const int* s
       const bool move = mx > mrow[hr] + RESCALE_SLACK;
       if (__any_sync(0xffffffffu, move)) {
         const float mnew = move ? mx : mrow[hr];
-        const float corr = (mnew == mrow[hr]) ? 1.f : exp2f(mrow[hr] - mnew);
+        const float corr = (mnew == mrow[hr]) ? 1.f : exp2_approx(mrow[hr] - mnew);
         mrow[hr] = mnew;
         lrow[hr] *= corr;
 #pragma unroll
@@ -178,12 +161,12 @@ __device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, const int* s
       float sum = 0.f;
 #pragma unroll
       for (int jj = 0; jj < NJ; ++jj) {
-        float p0 = exp2f(sacc[jj][2 * hr] - muse);
-        float p1 = exp2f(sacc[jj][2 * hr + 1] - muse);
+        float p0 = exp2_approx(sacc[jj][2 * hr] - muse);
+        float p1 = exp2_approx(sacc[jj][2 * hr + 1] - muse);
         if (smul) {  // a compacted key weighs as many tokens as it stands for
-          const int2 c = *reinterpret_cast<const int2*>(smul + (j0 + jj) * 8 + 2 * tq);
-          p0 *= float(c.x);
-          p1 *= float(c.y);
+          const float2 c = *reinterpret_cast<const float2*>(smul + (j0 + jj) * 8 + 2 * tq);
+          p0 *= c.x;
+          p1 *= c.y;
         }
         sacc[jj][2 * hr] = p0;
         sacc[jj][2 * hr + 1] = p1;
@@ -195,10 +178,7 @@ __device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, const int* s
 #pragma unroll
     for (int jj = 0; jj < NJ; ++jj) {
       float2 c = make_float2(1.f, 1.f);
-      if (smul) {
-        const int2 ci = *reinterpret_cast<const int2*>(smul + (j0 + jj) * 8 + 2 * tq);
-        c = make_float2(float(ci.x), float(ci.y));
-      }
+      if (smul) c = *reinterpret_cast<const float2*>(smul + (j0 + jj) * 8 + 2 * tq);
       sacc[jj][0] = fmaxf(sacc[jj][0], 0.f) * c.x;
       sacc[jj][1] = fmaxf(sacc[jj][1], 0.f) * c.y;
       sacc[jj][2] = fmaxf(sacc[jj][2], 0.f) * c.x;
@@ -286,11 +266,20 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
         copy_tile_index(idx_slot(j), a.kv_rows, a.kv_mult, k0 + int64_t(tl) * KT, min(KT, nk - tl * KT), tt);
       }
     };
+    // the key multiplicities of a tile arrive as int32 counts; thread tt >= 32 of the team,
+    // which copied entry tt - 32, turns it into a float in place once its own copy has
+    // landed, and a team barrier orders that before the consumers read the float weights
+    auto to_float_mult = [&](int j) {
+      if (tidx && a.kv_mult && tt >= 32 && j < n_local) {
+        int* e = idx_slot(j) + KT + (tt - 32);
+        *reinterpret_cast<float*>(e) = float(*e);
+      }
+    };
     auto load_kv = [&](int j, int st) {
       if (j < n_local) {
         const int tl = tile_of(j);
         load_kv_tile(tbuf + st * TEAM_STAGE, idx_slot(j), k0 + int64_t(tl) * KT, min(KT, nk - tl * KT), KV, ld,
-                     hcol, d, tt);
+                     2 * hcol, tt);
       }
     };
     if (tidx) {
@@ -298,6 +287,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
       copy_idx(1);
       cp_async_commit();
       cp_async_wait_all();
+      to_float_mult(0);
+      to_float_mult(1);
       team_sync(team);
     }
 #pragma unroll
@@ -317,10 +308,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
       load_kv(j + KV_STAGES - 1, st);
       copy_idx(j + KV_STAGES + 1);
       cp_async_commit();
+      // tile j + 2's counts: their copy was in the group the wait above completed; the
+      // barriers of the next two iterations order this before their use
+      to_float_mult(j + 2);
       const uint32_t sK = smem_u32(tbuf + stage * TEAM_STAGE);
       const uint32_t sV = sK + TILE_BYTES;
       const int valid = min(KT, nk - tile_of(j) * KT);
-      const int* smul = a.kv_mult ? idx_slot(j) + KT : nullptr;
+      const float* smul = a.kv_mult ? reinterpret_cast<const float*>(idx_slot(j) + KT) : nullptr;
       if (ksplit) tile_step<SCORE, 2>(sK, sV, smul, 2 * mem, qa, o, mrow, lrow, valid, lane);
       else tile_step<SCORE, 4>(sK, sV, smul, 0, qa, o, mrow, lrow, valid, lane);
       stage = stage + 1 == KV_STAGES ? 0 : stage + 1;
@@ -407,6 +401,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
           pml[0] = M;
           pml[1] = Lsum;
         }
+        if (SCORE == 0 && seg == 0 && direct && a.lse_out)  // sum_j e^s_j = 2^M Lsum
+          a.lse_out[int64_t(t) * a.H + h] = Lsum > 0.f ? (M + log2f(Lsum)) * LN2 : -INFINITY;
       }
     }
     __syncthreads();
@@ -554,6 +550,8 @@ __global__ void attn_merge_kernel(AttnArgs a) {
     float2* ml = reinterpret_cast<float2*>(a.ml_out + (int64_t(t) * a.H + h) * 2);
     *ml = make_float2(M, Lsum);
   }
+  if (SCORE == 0 && a.lse_out && !a.ml_out && lane == 0)
+    a.lse_out[int64_t(t) * a.H + h] = Lsum > 0.f ? (M + log2f(Lsum)) * LN2 : -INFINITY;
 }
 
 }  // namespace

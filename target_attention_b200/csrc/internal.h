@@ -38,8 +38,10 @@ struct EpiFold {
   const float* cvec;
   const float* bvec;
 };
-// c and b of the fold for W = [WK | WV] ([d, d] bf16 each, row-major): out [2][2d] fp32.
-int fold_consts(const float* gamma, const float* beta, const void* WK, const void* WV, int d, float* out,
+// c and b of the fold for W = [WK | WV] ([d, d] bf16 each, row-major): out [2][2d] fp32,
+// in the K/V GEMM's output column order: head-interleaved [K_h | V_h] per head of width dh
+// (the order pack mode 3 gives), or K then V when dh == 0.
+int fold_consts(const float* gamma, const float* beta, const void* WK, const void* WV, int d, int dh, float* out,
                 cudaStream_t s);
 
 // ---------------------------------------------------------------- tcgen05 GEMMs (bf16)
@@ -48,6 +50,7 @@ int fold_consts(const float* gamma, const float* beta, const void* WK, const voi
 // mode 0: dst row (row_offset + n)        <- column n
 // mode 1: SwiGLU gate half:  dst row (n/128)*256 + n%128       <- column n of W1
 // mode 2: SwiGLU up half:    dst row (n/128)*256 + 128 + n%128 <- column n of W3
+// mode 3: head-interleaved:  dst row (n/group)*2*group + row_offset + n%group <- column n
 int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_offset, cudaStream_t s);
 
 // The same packing for many matrices with one launch per PACK_MAX_JOBS jobs.
@@ -55,6 +58,10 @@ struct PackJob {
   const void* W;  // [K, N] bf16
   void* dst;
   int K, N, mode, row_offset;
+  // mode 3 (head-interleaved K|V): column n goes to row (n / group) * 2 group + row_offset
+  // + n % group, so that W_K (row_offset 0) and W_V (row_offset group) of head n / group
+  // make one 2 group-row block and the GEMM output row holds [K_h | V_h] per head
+  int group;
 };
 constexpr int PACK_MAX_JOBS = 48;
 int tc_pack_weights(const PackJob* jobs, int n, cudaStream_t s);
@@ -140,7 +147,10 @@ int layer_norm_f32(const float* x, int64_t ldx, float* y, int64_t ldy, int rows,
 
 struct AttnArgs {
   const float* Q;       // [T, d] fp32 (projected queries)
-  const void* KV;       // [N, 2d]: K in columns [0, d), V in [d, 2d); bf16 or fp32
+  // bf16: [N, H, 2 d_h], row n holds [K_h | V_h] of head h in columns [2 h d_h, 2 (h+1) d_h)
+  // (one contiguous 256-byte segment per key and head); fp32: [N, 2d], K in columns
+  // [0, d), V in [d, 2d)
+  const void* KV;
   const int32_t* hoff;  // [B+1] history offsets
   const int32_t* toff;  // [B+1] target offsets
   const int32_t* kv_rows;  // K/V row of history token n (distinct-row form), or null: row n
@@ -159,8 +169,16 @@ struct AttnArgs {
   // merge: when set, combine the slices into ONE state instead of the output: out gets
   // the unnormalised acc and ml_out [T, H, 2] the (max, sum) of the softmax
   float* ml_out = nullptr;
+  // softmax, when set: lse_out [T, H] = log sum_j exp(s_j) over all of the user's keys
+  // (natural log; -inf for an empty history), written with the normalised output (bf16
+  // kernel with one slice, or the merge) for the backward pass
+  float* lse_out = nullptr;
 };
 int attention_bf16(const AttnArgs& a, cudaStream_t s);
+// Backward of the bf16 attention (per-token K/V rows, d_h = 64); see stca_attention_backward.
+int attention_bwd_bf16(const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B, int T, int d,
+                       int H, int splits, int score, const float* O, const float* lse, const float* dO, float* dQ,
+                       float* dKV, float* part_dq, cudaStream_t s);
 int attention_f32(const AttnArgs& a, cudaStream_t s);
 // combines the slices; not needed after attention_bf16 with splits == 1, which writes out
 int attention_merge(const AttnArgs& a, cudaStream_t s);

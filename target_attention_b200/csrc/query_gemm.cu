@@ -25,24 +25,6 @@ __device__ __forceinline__ int64_t qremap(int r, int grp, int gstride, int goff)
   return grp ? int64_t(r / grp) * gstride + goff + r % grp : int64_t(r);
 }
 
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm4t(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-
 // A tile [128 rows][32 k] bf16: 64-byte rows, 16-byte chunk c of row r at c ^ ((r >> 1) & 3)
 __device__ __forceinline__ int a_off(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
 // B tile [32 k rows][128 n] bf16: 256-byte rows, 16-byte chunk c of row k at c ^ (k & 7)
@@ -154,13 +136,13 @@ __global__ void __launch_bounds__(256, 1) query_gemm_kernel(SimtGemmArgs<float, 
         const int krow = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
         const int ch = (wn * 32 + np * 16) / 8 + (lane >> 4);
         uint32_t r[4];
-        ldsm4t(sB + b_off(krow, ch), r);
+        ldsm_x4_t(sB + b_off(krow, ch), r);
         bfr[2 * np][0] = r[0];
         bfr[2 * np][1] = r[1];
         bfr[2 * np + 1][0] = r[2];
         bfr[2 * np + 1][1] = r[3];
         if (DUAL) {
-          ldsm4t(sB + B_TILE + b_off(krow, ch), r);
+          ldsm_x4_t(sB + B_TILE + b_off(krow, ch), r);
           bfr2[2 * np][0] = r[0];
           bfr2[2 * np][1] = r[1];
           bfr2[2 * np + 1][0] = r[2];
@@ -172,15 +154,15 @@ __global__ void __launch_bounds__(256, 1) query_gemm_kernel(SimtGemmArgs<float, 
         const int row = wm * 64 + mi * 16 + (lane & 15);
         const int ch = kk * 2 + (lane >> 4);
         uint32_t ah[4], al[4];
-        ldsm4(sAh + a_off(row, ch), ah);
-        ldsm4(sAl + a_off(row, ch), al);
+        ldsm_x4(sAh + a_off(row, ch), ah);
+        ldsm_x4(sAl + a_off(row, ch), al);
 #pragma unroll
         for (int nj = 0; nj < 4; ++nj) {
-          mma16816(acc[mi][nj], ah, bfr[nj][0], bfr[nj][1]);
-          mma16816(acc[mi][nj], al, bfr[nj][0], bfr[nj][1]);
+          mma_bf16_16816(acc[mi][nj], ah, bfr[nj][0], bfr[nj][1]);
+          mma_bf16_16816(acc[mi][nj], al, bfr[nj][0], bfr[nj][1]);
           if (DUAL) {
-            mma16816(acc2[mi][nj], ah, bfr2[nj][0], bfr2[nj][1]);
-            mma16816(acc2[mi][nj], al, bfr2[nj][0], bfr2[nj][1]);
+            mma_bf16_16816(acc2[mi][nj], ah, bfr2[nj][0], bfr2[nj][1]);
+            mma_bf16_16816(acc2[mi][nj], al, bfr2[nj][0], bfr2[nj][1]);
           }
         }
       }

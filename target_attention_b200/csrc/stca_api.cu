@@ -416,13 +416,16 @@ bf16* wp3(const stca_handle* h, int slot) {
   return reinterpret_cast<bf16*>(h->wpack) + size_t(h->wslots) * (2 * hd * d + d * hd) + size_t(slot) * 2 * d * d;
 }
 
-// One history layer: the FFN, then W_K and W_V stacked into [2 d, d] (K rows, then V rows).
+// One history layer: the FFN, then W_K and W_V interleaved by head into [2 d, d] (rows
+// [2 h d_h, 2 h d_h + d_h) are head h of W_K, the next d_h rows head h of W_V), so that the
+// K/V GEMM writes each history row as [K_1 | V_1 | K_2 | V_2 | ...] and attention reads one
+// contiguous 2 d_h-element segment per (key, head).
 void layer_jobs(stca_handle* h, int slot, const stca_ffn& f, const void* WK, const void* WV,
                 std::vector<PackJob>& jobs) {
-  const int d = h->cfg.d, hd = h->cfg.hidden;
+  const int d = h->cfg.d, hd = h->cfg.hidden, dh = d / h->cfg.H;
   ffn_jobs(f, d, hd, wp13(h, slot), wp2(h, slot), jobs);
-  jobs.push_back({WK, wp3(h, slot), d, d, 0, 0});
-  jobs.push_back({WV, wp3(h, slot), d, d, 0, d});
+  jobs.push_back({WK, wp3(h, slot), d, d, 3, 0, dh});
+  jobs.push_back({WV, wp3(h, slot), d, d, 3, dh, dh});
 }
 
 // The target-side weights of a bf16 STCA call.
@@ -453,7 +456,8 @@ void stca_jobs(stca_handle* h, const stca_weights* w, std::vector<PackJob>& jobs
 int stca_folds(stca_handle* h, const stca_weights* w, cudaStream_t s) {
   const int d = h->cfg.d;
   for (int i = 0; i < h->cfg.M; ++i)
-    CK(fold_consts(w->hist[i].gamma, w->hist[i].beta, w->WK[i], w->WV[i], d, h->fold + size_t(i) * 4 * d, s));
+    CK(fold_consts(w->hist[i].gamma, w->hist[i].beta, w->WK[i], w->WV[i], d, d / h->cfg.H,
+                   h->fold + size_t(i) * 4 * d, s));
   return STCA_OK;
 }
 

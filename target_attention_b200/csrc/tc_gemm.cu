@@ -855,7 +855,9 @@ __global__ void pack_many_kernel(PackJobs jobs) {
   for (int i = threadIdx.y; i < 32; i += blockDim.y) {
     const int n = n0 + i, k = k0 + threadIdx.x;
     if (n < jb.N && k < jb.K) {
-      const int row = jb.mode == 0 ? jb.row_offset + n : (n / 128) * 256 + (jb.mode == 2 ? 128 : 0) + (n % 128);
+      const int row = jb.mode == 0   ? jb.row_offset + n
+                      : jb.mode == 3 ? (n / jb.group) * 2 * jb.group + jb.row_offset + n % jb.group
+                                     : (n / 128) * 256 + (jb.mode == 2 ? 128 : 0) + (n % 128);
       dst[int64_t(row) * jb.K + k] = tile[threadIdx.x][i];
     }
   }
@@ -863,18 +865,28 @@ __global__ void pack_many_kernel(PackJobs jobs) {
 
 // c = gamma^T [WK | WV], b = beta^T [WK | WV]: a block of 8 warps per 32 output columns;
 // lane l takes column c0 + l, warp w the rows w, w + 8, ... (reads coalesced across lanes),
-// and the 8 partial sums meet in shared memory
+// and the 8 partial sums meet in shared memory.  Output column c is the K/V GEMM's: with
+// dh > 0, head c / (2 dh), K for the first dh columns of the head's block and V after.
 __global__ void __launch_bounds__(256) fold_consts_kernel(const float* __restrict__ gamma,
                                                           const float* __restrict__ beta,
                                                           const bf16* __restrict__ WK, const bf16* __restrict__ WV,
-                                                          int d, float* __restrict__ out) {
+                                                          int d, int dh, float* __restrict__ out) {
   __shared__ float part[2][8][32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int c = blockIdx.x * 32 + lane;
   float sc = 0.f, sb = 0.f;
   if (c < 2 * d) {
-    const bf16* W = c < d ? WK : WV;
-    const int col = c < d ? c : c - d;
+    bool is_k;
+    int col;
+    if (dh > 0) {
+      const int j = c % (2 * dh);
+      is_k = j < dh;
+      col = (c / (2 * dh)) * dh + (is_k ? j : j - dh);
+    } else {
+      is_k = c < d;
+      col = is_k ? c : c - d;
+    }
+    const bf16* W = is_k ? WK : WV;
     for (int k = w; k < d; k += 8) {
       const float x = __bfloat162float(W[int64_t(k) * d + col]);
       sc = fmaf(gamma[k], x, sc);
@@ -968,11 +980,12 @@ int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_off
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
 
-int fold_consts(const float* gamma, const float* beta, const void* WK, const void* WV, int d, float* out,
+int fold_consts(const float* gamma, const float* beta, const void* WK, const void* WV, int d, int dh, float* out,
                 cudaStream_t s) {
-  if (!gamma || !beta || !WK || !WV || !out || d <= 0) return STCA_ERR_INVALID_ARG;
+  if (!gamma || !beta || !WK || !WV || !out || d <= 0 || dh < 0 || (dh > 0 && d % dh != 0))
+    return STCA_ERR_INVALID_ARG;
   fold_consts_kernel<<<(2 * d + 31) / 32, 256, 0, s>>>(gamma, beta, reinterpret_cast<const bf16*>(WK),
-                                                       reinterpret_cast<const bf16*>(WV), d, out);
+                                                       reinterpret_cast<const bf16*>(WV), d, dh, out);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
@@ -985,7 +998,8 @@ int tc_pack_weights(const PackJob* jobs, int n, cudaStream_t s) {
     int gx = 1, gy = 1;
     for (int i = 0; i < cnt; ++i) {
       const PackJob& jb = jobs[b + i];
-      if (jb.K <= 0 || jb.N <= 0 || !jb.W || !jb.dst || jb.mode < 0 || jb.mode > 2) return STCA_ERR_INVALID_ARG;
+      if (jb.K <= 0 || jb.N <= 0 || !jb.W || !jb.dst || jb.mode < 0 || jb.mode > 3) return STCA_ERR_INVALID_ARG;
+      if (jb.mode == 3 && (jb.group <= 0 || jb.N % jb.group != 0)) return STCA_ERR_INVALID_ARG;
       batch.j[i] = jb;
       gx = std::max(gx, (jb.N + 31) / 32);
       gy = std::max(gy, (jb.K + 31) / 32);

@@ -299,12 +299,15 @@ def _attention_case(kv_bf16, d, H, lengths, targets, splits, score, seed):
     dh = d // H
     ref = np.zeros((T, d))
     for u in range(Bu):
-        K = KV64[hoff[u]:hoff[u + 1], :d]
-        V = KV64[hoff[u]:hoff[u + 1], d:]
+        rows = KV64[hoff[u]:hoff[u + 1]]
         for t in range(toff[u], toff[u + 1]):
             for h in range(H):
                 cols = slice(h * dh, (h + 1) * dh)
-                ref[t, cols] = R.head_attention(Q[t, cols].astype(np.float64), K[:, cols], V[:, cols],
+                if kv_bf16:  # [N, H, 2 d_h]: head h's K then V in one segment
+                    K_h, V_h = rows[:, 2 * h * dh:(2 * h + 1) * dh], rows[:, (2 * h + 1) * dh:(2 * h + 2) * dh]
+                else:        # [N, 2d]: K in [0, d), V in [d, 2d)
+                    K_h, V_h = rows[:, cols], rows[:, d:][:, cols]
+                ref[t, cols] = R.head_attention(Q[t, cols].astype(np.float64), K_h, V_h,
                                                 "softmax" if score == 0 else "relu", 1 / math.sqrt(dh))
     return out.cpu().numpy()[:T], ref
 
