@@ -337,6 +337,45 @@ void stca_unpin_weights(stca_handle* h);
 /* Frees the handle's device memory.  NULL is a no-op. */
 void stca_destroy(stca_handle* h);
 
+/* ---------------------------------------------------------------------------------
+ * Training: the attention step's forward with its softmax statistics, and its backward.
+ * The pages train on ~2K-item histories and serve 10K ([notes] "短序列训练，长序列推理";
+ * [review] architecture branch (C) "Extrapolation Aware Training").  Handle-free: the
+ * caller passes every buffer (device pointers, caller-owned) and any scratch.  One K/V
+ * row per history token (no distinct-key compaction), bf16 K/V, d_h = d / H = 64 (else
+ * STCA_ERR_UNSUPPORTED); 1 <= splits <= 32 slices of each user's keys (else
+ * STCA_ERR_INVALID_ARG).  Layouts:
+ *   Q, out, dout, dQ   [T, d] float32, row t = target t (targets grouped by user, toff)
+ *   KV                 [N, H, 2 d_h] bf16: row n = history token n (users by hoff), head
+ *                      h's K in columns [2 h d_h, 2 h d_h + d_h) and V in the next d_h
+ *   dKV                [N, H, 2 d_h] float32 in the same layout ([dK_h | dV_h])
+ *   lse                [T, H] float32: log sum_j exp(q_h . k_j / sqrt(d_h)) over the
+ *                      user's keys (natural log; -inf for an empty history)
+ *   hoff, toff         [B + 1] int32 offsets of the users' keys and targets, trusted as
+ *                      given: rows hoff[0] .. hoff[B] - 1 of KV / dKV and toff[0] ..
+ *                      toff[B] - 1 of the [T, d] arrays must exist
+ * Scores: 0 softmax, 1 relu (the unnormalised ReLU form keeps no lse; lse may be NULL).
+ * ---------------------------------------------------------------------------------- */
+
+/* out[t, head h] = attention of query h of target t over its user's keys ([review] 核心公式;
+ * [wechat] §1.2 for relu), plus lse (softmax).  part_acc [splits, T, d] and part_ml
+ * [splits, T, H, 2] float32 scratch (unused, may be NULL, when splits == 1). */
+int stca_attention_train_forward(const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B,
+                                 int T, int d, int H, int splits, int score, float* part_acc, float* part_ml,
+                                 float* out, float* lse, int32_t* err, void* stream);
+
+/* Gradients of sum_t dout[t] . out[t] with respect to Q and K/V, given the forward's out
+ * and lse:
+ *   softmax: p = exp(s - lse), D_t = dout_t . out_t, ds = p (dout_t . v_j - D_t)
+ *   relu:    p = relu(s),                            ds = (dout_t . v_j) [s > 0]
+ *   dV_j = sum_t p_tj dout_t, dK_j = sum_t ds_tj q_t / sqrt(d_h), dQ_t = sum_j ds_tj k_j / sqrt(d_h)
+ * with s = q . k / sqrt(d_h) per head; a key's gradient sums over all of its user's
+ * targets, and a key with no target of its user gets 0.  part_dq [splits, T, d] float32
+ * scratch for splits > 1 (may be NULL when splits == 1).  Deterministic: no atomics. */
+int stca_attention_backward(const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B, int T,
+                            int d, int H, int splits, int score, const float* out, const float* lse,
+                            const float* dout, float* dQ, float* dKV, float* part_dq, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -82,6 +82,10 @@ _SIGS = [
     ("stca_lsplit_merge", _i32, [_vp, _i32, _i32, _vp, _vp, _vp, _vp]),
     ("stca_pointwise_forward", _i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp]),
     ("stca_pointwise_forward_noalloc", _i32, [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _vp, _vp]),
+    ("stca_attention_train_forward", _i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
+                                            _vp, _vp, _vp]),
+    ("stca_attention_backward", _i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
+                                       _vp, _vp, _vp]),
     ("hyformer_forward", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, ctypes.POINTER(HyfWeights),
                                 _vp, _vp]),
     ("stca_sync_status", _i32, [_vp]),
@@ -253,6 +257,21 @@ def stca_pointwise_forward_noalloc(ids, lengths, q, table, n_items, B, n_tok, ou
     """Pointwise ReLU TA without a handle or any device allocation (scratch in the library)."""
     return lib().stca_pointwise_forward_noalloc(ptr(ids), ptr(lengths), ptr(q), ptr(table), n_items, B, n_tok,
                                                 ptr(out), ptr(err), stream_ptr(stream))
+
+
+def stca_attention_train_forward(Q, KV, hoff, toff, B, T, d, H, splits, score, part_acc, part_ml, out, lse,
+                                 err=None, stream=None) -> int:
+    """Training forward of the attention step: out and (softmax) lse [T, H]."""
+    return lib().stca_attention_train_forward(ptr(Q), ptr(KV), ptr(hoff), ptr(toff), B, T, d, H, splits, score,
+                                              ptr(part_acc), ptr(part_ml), ptr(out), ptr(lse), ptr(err),
+                                              stream_ptr(stream))
+
+
+def stca_attention_backward(Q, KV, hoff, toff, B, T, d, H, splits, score, out, lse, dout, dQ, dKV, part_dq=None,
+                            stream=None) -> int:
+    """Backward of the attention step: dQ [T, d] and dKV [N, H, 2 d_h] (fp32)."""
+    return lib().stca_attention_backward(ptr(Q), ptr(KV), ptr(hoff), ptr(toff), B, T, d, H, splits, score, ptr(out),
+                                         ptr(lse), ptr(dout), ptr(dQ), ptr(dKV), ptr(part_dq), stream_ptr(stream))
 
 
 def hyformer_forward(h, ids_feed, len_feed, n_feed, ids_search, len_search, n_search, q0, B, n_query,

@@ -117,6 +117,23 @@ def test_null_arguments_rejected_on_host():
         == B.ERR_INVALID_ARG
 
 
+def test_training_entries_reject_bad_arguments_on_host():
+    L = tab.lib()
+    f, b = L.stca_attention_train_forward, L.stca_attention_backward
+    # splits outside 1..32, a bad score, a negative count, missing buffers
+    assert f(16, 16, 16, 16, 1, 1, 256, 4, 0, 0, None, None, 16, 16, None, None) == B.ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 1, 1, 256, 4, 33, 0, 16, 16, 16, 16, None, None) == B.ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 1, 1, 256, 4, 1, 2, None, None, 16, 16, None, None) == B.ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, -1, 1, 256, 4, 1, 0, None, None, 16, 16, None, None) == B.ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 1, 1, 256, 4, 1, 0, None, None, 16, None, None, None) == B.ERR_INVALID_ARG  # lse
+    assert f(16, 16, 16, 16, 1, 1, 256, 4, 2, 0, None, None, 16, 16, None, None) == B.ERR_INVALID_ARG  # scratch
+    assert f(16, 16, 16, 16, 1, 1, 256, 8, 1, 0, None, None, 16, 16, None, None) == B.ERR_UNSUPPORTED  # d_h 32
+    assert b(16, 16, 16, 16, 1, 1, 256, 4, 1, 0, 16, 16, 16, 16, None, None, None) == B.ERR_INVALID_ARG  # dKV
+    assert b(16, 16, 16, 16, 1, 1, 256, 4, 2, 0, 16, 16, 16, 16, 16, None, None) == B.ERR_INVALID_ARG  # part_dq
+    assert b(16, 16, 16, 16, 1, 1, 256, 4, 1, 0, None, None, 16, 16, 16, None, None) == B.ERR_INVALID_ARG  # out
+    assert b(16, 16, 16, 16, 1, 1, 512, 4, 1, 0, 16, 16, 16, 16, 16, None, None) == B.ERR_UNSUPPORTED  # d_h 128
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(B, "_LIB", None)
