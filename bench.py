@@ -112,7 +112,7 @@ def make_workload(args, data_seed):
     if c["kind"] == "stca":
         return make_stca(args.workload, users=users, L=L, n_items=n_items, data_seed=data_seed, **over)
     if c["kind"] == "pointwise":
-        return make_pointwise(args.workload, users=users, L=L, n_items=n_items, seed=data_seed)
+        return make_pointwise(args.workload, users=users, L=L, n_items=n_items, seed=data_seed, **over)
     return make_hyformer(args.workload, users=users, L_feed=L, n_items=n_items, seed=data_seed)
 
 
@@ -145,9 +145,10 @@ def config_block(wl, world, total_tokens=None):
             "targets_per_user": c["m"],
             "l2": "inputs larger than L2 (table, and K/V plus hidden activations of several GB per layer)"})
     elif c["kind"] == "pointwise":
+        ids = f"Zipf({c['zipf_s']})" if c["id_dist"] == "zipf" else "uniform"
         common.update({
             "workload": f"pointwise ReLU target attention with fused lookup, {users} samples x L~U[{c['L_lo']},"
-                        f"{c['L']}], D={c['d']}, Zipf({c['zipf_s']}) ids over {c['n_items']}x{c['d']} bf16 table",
+                        f"{c['L']}], D={c['d']}, {ids} ids over {c['n_items']}x{c['d']} bf16 table",
             "l2": "inputs larger than L2 (0.5 GB table, 22 MB ids; Zipf ids are partly L2-resident)"})
     else:
         common.update({

@@ -189,9 +189,9 @@ def make_stca(config_id: int, *, users=None, L=None, n_items=None, m=None, lengt
 
 
 def make_pointwise(config_id: int = 4, *, users=None, L=None, L_lo=None, n_items=None,
-                   lengths=None, seed=None) -> dict:
+                   lengths=None, seed=None, **over) -> dict:
     """Inputs for pointwise ReLU target attention with fused lookup (config 4)."""
-    cfg = _config(config_id, users=users, L=L, L_lo=L_lo, n_items=n_items)
+    cfg = _config(config_id, users=users, L=L, L_lo=L_lo, n_items=n_items, **over)
     assert cfg["kind"] == "pointwise"
     ss = np.random.SeedSequence(1000 + config_id if seed is None else seed)
     s_len, s_ids, s_q, s_tab = ss.spawn(4)
