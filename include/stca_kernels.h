@@ -44,6 +44,20 @@ int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, 
                          const void* dt_table, int64_t n_items, int M, int K, const void* Wp, int Nout, void* C,
                          int ldc, void* x_out, int32_t* err, void* stream);
 
+/* Fused history FFN of `layers` layers for d = 256 ([notes] STCA: X~_l = LN_l(SwiGLU_l(X))
+ * from the original X; [wechat] §1.1 lookup while computing).  Rows r < M of X are
+ * gathered as in stca_k_gemm_resident amode 1 (K = 256); the SwiGLU hidden activations of
+ * every layer stay on chip.  W13p: all layers' W1|W3 packed (modes 1 + 2) back to back,
+ * [layers 2 hidden, 256]; W2p: all layers' W2 packed (mode 0) back to back, [layers 256,
+ * hidden]; hidden % 128 == 0.  gammas: host array of `layers` device pointers (LayerNorm
+ * gamma [256] fp32 per layer).  Writes, per layer l and row r, y'[l layer_stride + r] =
+ * (A_l W2_l) * gamma_l (bf16 [256]) and stats[l layer_stride + r] = (mean, rstd) of A_l W2_l
+ * (float2), so that LN_l = rstd (y' - mean gamma) + beta.  layer_stride >= M, a multiple of
+ * 256; Y 16-byte aligned. */
+int stca_k_ffn_fused(const int32_t* ids, const int32_t* dt, const void* table, const void* dt_table, int64_t n_items,
+                     int M, int layers, int hidden, const void* W13p, const void* W2p, const float* const* gammas,
+                     float eps, void* Y, int layer_stride, float* stats, int32_t* err, void* stream);
+
 /* Target-side tensor-core GEMM ([review] §三 fusion formula; [notes] STCA query update):
  * fp32 activations A (each split into two bf16 terms, so products keep fp32 accuracy),
  * packed bf16 weights, fp32 result C [M, ldc]:

@@ -100,6 +100,8 @@ _SIGS = [
     ("stca_k_pack_weight", _i32, [_vp, _i32, _i32, _vp, _i32, _i32, _vp]),
     ("stca_k_gemm_resident", _i32, [_i32, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _i32, _vp, _i32, _vp,
                                     _vp, _vp]),
+    ("stca_k_ffn_fused", _i32, [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, ctypes.c_float, _vp,
+                          _i32, _vp, _vp, _vp]),
     ("stca_k_gemm_query", _i32, [_vp, _i64, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _vp, _i64, _vp, _i64, _vp,
                                  _vp]),
     ("stca_k_gemm_rowwise", _i32, [_i32, _vp, _i32, _i32, _vp, _i32, _vp, _vp, ctypes.c_float, _vp, _i32, _vp, _vp]),
@@ -257,6 +259,14 @@ def stca_pointwise_forward_noalloc(ids, lengths, q, table, n_items, B, n_tok, ou
     """Pointwise ReLU TA without a handle or any device allocation (scratch in the library)."""
     return lib().stca_pointwise_forward_noalloc(ptr(ids), ptr(lengths), ptr(q), ptr(table), n_items, B, n_tok,
                                                 ptr(out), ptr(err), stream_ptr(stream))
+
+
+def stca_k_ffn_fused(ids, dt, table, dt_table, n_items, M, layers, hidden, W13p, W2p, gammas, eps, Y, layer_stride,
+                     stats, err=None, stream=None) -> int:
+    """Fused history FFN (d = 256); gammas: list of per-layer device tensors."""
+    arr = (ctypes.c_void_p * len(gammas))(*[g.data_ptr() for g in gammas])
+    return lib().stca_k_ffn_fused(ptr(ids), ptr(dt), ptr(table), ptr(dt_table), n_items, M, layers, hidden, ptr(W13p),
+                                  ptr(W2p), arr, eps, ptr(Y), layer_stride, ptr(stats), ptr(err), stream_ptr(stream))
 
 
 def stca_attention_train_forward(Q, KV, hoff, toff, B, T, d, H, splits, score, part_acc, part_ml, out, lse,

@@ -90,6 +90,17 @@ int tc_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, int N,
 bool make_tmap(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows);
 // fp32 [rows, cols] (row stride ld elements), box 32 x 32, 128-byte swizzle: tile stores.
 bool make_tmap_f32_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld);
+// bf16 [rows, cols] (row stride ld elements), box 32 x 32, 64-byte swizzle: the epilogue's
+// staged tile stores.
+bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint64_t ld);
+// Fused history FFN of every layer for d = 256 (tc_ffn.cu): rows gathered via g (M rows, or
+// *M_dev when given), W13p = all layers' packed W1|W3 [layers 2 hidden, 256], W2p = all
+// layers' packed W2 [layers 256, hidden]; writes y'_l = (A_l W2_l) * gamma_l as bf16 rows
+// l * layer_stride + r of Y [layers layer_stride, 256] and the row moments (mean, rstd) to
+// stats [layers layer_stride] float2.  layer_stride >= M, a multiple of 256.
+int tc_ffn_fused(const GatherSrc& g, int M, const int32_t* M_dev, int layers, int hidden, const void* W13p,
+                 const void* W2p, const float* const* gammas, float eps, void* Y, int layer_stride, float* stats,
+                 int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- SIMT fp32 GEMMs
 

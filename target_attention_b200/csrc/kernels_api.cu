@@ -66,6 +66,21 @@ int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, 
                           nullptr, x_out);
 }
 
+int stca_k_ffn_fused(const int32_t* ids, const int32_t* dt, const void* table, const void* dt_table, int64_t n_items,
+                     int M, int layers, int hidden, const void* W13p, const void* W2p, const float* const* gammas,
+                     float eps, void* Y, int layer_stride, float* stats, int32_t* err, void* stream) {
+  if (M < 0 || (M > 0 && (!ids || !table || n_items <= 0 || !gammas))) return STCA_ERR_INVALID_ARG;
+  GatherSrc g;
+  memset(&g, 0, sizeof(g));
+  g.ids = ids;
+  g.dt = dt_table ? dt : nullptr;
+  g.table = table;
+  g.dt_table = dt ? dt_table : nullptr;
+  g.n_items = n_items;
+  return tc_ffn_fused(g, M, nullptr, layers, hidden, W13p, W2p, gammas, eps, Y, layer_stride, stats, err,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
 int stca_k_gemm_query(const float* A, int64_t lda, int M, int K, int ksplit, int kshift, const void* Wp, int N,
                       int dual, const float* R, int64_t ldr, float* C, int64_t ldc, int32_t* err, void* stream) {
   if (M < 0 || K <= 0 || N <= 0 || !Wp || (M > 0 && (!A || !C)) || ksplit < 0 || kshift < 0 ||

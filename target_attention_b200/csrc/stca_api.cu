@@ -275,6 +275,14 @@ stca_handle::QLayout hq_layout(const stca_config& c) {
   return q;
 }
 
+// bf16 STCA with d = 256: the history FFN of every layer runs in one fused kernel that
+// keeps the SwiGLU hidden activations on chip (tc_ffn_fused); its per-layer outputs sit
+// layer_stride rows apart.
+bool fused_ffn(const stca_config& c) {
+  return c.mode == STCA_MODE_STCA && c.dtype == STCA_BF16 && c.d == 256 && c.hidden % 128 == 0;
+}
+size_t ffn_layer_stride(const stca_config& c) { return (size_t(c.max_tokens) + 255) / 256 * 256; }
+
 int allocate(stca_handle* h) {
   const stca_config& c = h->cfg;
   const size_t U = size_t(c.max_users) + 1, N = size_t(c.max_tokens), T = size_t(c.max_targets);
@@ -290,11 +298,17 @@ int allocate(stca_handle* h) {
   if (c.dtype == STCA_BF16) {
     h->wslots = c.M * nseq;
     ok = ok && dalloc(h, &h->wpack, size_t(h->wslots) * (2 * hd * d + d * hd + 2 * d * d) * 2);
-    ok = ok && dalloc(h, &h->fold, size_t(h->wslots) * 4 * d * 4) && dalloc(h, &h->rowstats, N * 2 * 4);
   }
-  // bf16: the hidden activations of all M layers of every sequence ([N, M h] per sequence)
-  const size_t hid_elems = c.dtype == STCA_BF16 ? nseq * N * size_t(c.M) * hd : N * hd;
-  ok = ok && dalloc(h, &h->hidden, hid_elems * E) && dalloc(h, &h->xt, N * d * E) && dalloc(h, &h->kv, N * 2 * d * E);
+  const bool fused = fused_ffn(c);
+  // rows of the LN GEMM outputs and their moments: every layer's with the fused FFN
+  const size_t xt_rows = fused ? size_t(c.M) * ffn_layer_stride(c) : N;
+  if (c.dtype == STCA_BF16)
+    ok = ok && dalloc(h, &h->fold, size_t(h->wslots) * 4 * d * 4) && dalloc(h, &h->rowstats, xt_rows * 2 * 4);
+  // bf16: the hidden activations of all M layers of every sequence ([N, M h] per sequence),
+  // not needed when the fused FFN keeps them on chip
+  const size_t hid_elems = fused ? 0 : c.dtype == STCA_BF16 ? nseq * N * size_t(c.M) * hd : N * hd;
+  ok = ok && dalloc(h, &h->hidden, hid_elems * E) && dalloc(h, &h->xt, xt_rows * d * E) &&
+       dalloc(h, &h->kv, N * 2 * d * E);
   ok = ok && dalloc(h, &h->qproj, T * d * 4) && dalloc(h, &h->attn, T * d * 4) && dalloc(h, &h->tmp_h, T * hd * 4) &&
        dalloc(h, &h->tmp_d, T * d * 4);
   ok = ok && dalloc(h, &h->part_acc, size_t(MAX_SPLITS) * T * d * 4) &&
@@ -524,6 +538,34 @@ int history_kv_bf16(stca_handle* h, int sq, int l, int n_tok, const float* gamma
   return STCA_OK;
 }
 
+// d = 256: y'_l = (A_l W2_l) * gamma_l and the row moments of every layer in one fused
+// launch (the hidden activations A_l stay on chip).
+int history_ffn_fused(stca_handle* h, const GatherSrc& g, int n_tok, const stca_weights* w, cudaStream_t s,
+                      const int32_t* M_dev) {
+  const stca_config& c = h->cfg;
+  const float* gammas[STCA_MAX_LAYERS] = {};
+  for (int l = 0; l < c.M; ++l) gammas[l] = w->hist[l].gamma;
+  STAGE(h, STCA_STAGE_GATHER_FFN, s,
+        tc_ffn_fused(g, n_tok, M_dev, c.M, c.hidden, wp13(h, 0), wp2(h, 0), gammas, c.ln_eps, h->xt,
+                     int(ffn_layer_stride(c)), h->rowstats, h->err, s));
+  return STCA_OK;
+}
+
+// [K | V] of layer l from the fused FFN's outputs, with the LayerNorm folded in.
+int history_kv_fused(stca_handle* h, int l, int n_tok, cudaStream_t s, const int32_t* M_dev) {
+  const int d = h->cfg.d;
+  const size_t stride = ffn_layer_stride(h->cfg);
+  GatherSrc none;
+  memset(&none, 0, sizeof(none));
+  const bf16* y = reinterpret_cast<const bf16*>(h->xt) + size_t(l) * stride * d;
+  const EpiFold fold{h->rowstats + size_t(l) * stride * 2, h->fold + size_t(l) * 4 * d,
+                     h->fold + size_t(l) * 4 * d + 2 * d};
+  STAGE(h, STCA_STAGE_KV, s,
+        tc_gemm_resident(A_TMA, EPI_LNFOLD, y, none, n_tok, d, wp3(h, l), 2 * d, h->kv, 2 * d, h->err, s, M_dev,
+                         nullptr, &fold));
+  return STCA_OK;
+}
+
 // K/V of every history token for one layer: fp32 SIMT path.
 int history_f32(stca_handle* h, const GatherSrc& g, int n_tok, const stca_ffn& f, const void* WK, const void* WV,
                 cudaStream_t s) {
@@ -637,7 +679,10 @@ int fwd_layer_inputs(stca_handle* h, int i, cudaStream_t s) {
   const stca_config& c = h->cfg;
   const stca_handle::Fwd& f = h->fwd;
   const stca_weights* w = f.w;
-  if (c.dtype == STCA_BF16) {
+  if (c.dtype == STCA_BF16 && fused_ffn(c)) {
+    if (i == 0) CK(history_ffn_fused(h, f.g, f.n_tok, w, s, f.M_dev));
+    CK(history_kv_fused(h, i, f.n_tok, s, f.M_dev));
+  } else if (c.dtype == STCA_BF16) {
     if (i == 0) CK(history_hidden_bf16(h, 0, f.g, f.n_tok, s, f.M_dev));
     CK(history_kv_bf16(h, 0, i, f.n_tok, w->hist[i].gamma, w->hist[i].beta, s, f.M_dev));
   } else {

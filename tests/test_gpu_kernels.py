@@ -219,6 +219,53 @@ def test_gemm_rowwise(K, N, M, ln):
     _close_bf16(bf16_to_f64(C), Y)
 
 
+@pytest.mark.parametrize("M, layers, hidden, with_dt", [(700, 2, 512, False), (3000 + 77, 3, 256, True),
+                                                         (130, 1, 512, False)])
+def test_ffn_fused_layernorm_rows(M, layers, hidden, with_dt):
+    """The fused history FFN (d = 256): per layer, rstd (y' - mean gamma) + beta against the
+    oracle's LN(SwiGLU(X)) of the gathered rows; several row tiles per CTA pair, a ragged
+    tail, one to three layers, with and without the time-bucket row."""
+    g = _rng(12)
+    d, n_items = 256, 5000
+    E = _bf16(g.standard_normal((n_items, d)) * 0.5)
+    ids = g.integers(0, n_items, size=M).astype(np.int32)
+    dt = np.floor(2.0 ** g.uniform(0, 16, M)).astype(np.int32) - 1 if with_dt else None
+    T = _bf16(g.standard_normal((16, d)) * 0.5) if with_dt else None
+    W1s, W3s, W2s, gam, bet = [], [], [], [], []
+    W13p = torch.zeros((layers * 2 * hidden, d), dtype=torch.bfloat16, device=dev)
+    W2p = torch.zeros((layers * d, hidden), dtype=torch.bfloat16, device=dev)
+    for l in range(layers):
+        W1s.append(_bf16(g.standard_normal((d, hidden)) / math.sqrt(d)))
+        W3s.append(_bf16(g.standard_normal((d, hidden)) / math.sqrt(d)))
+        W2s.append(_bf16(g.standard_normal((hidden, d)) / math.sqrt(hidden)))
+        _pack(W1s[-1], 1, 2 * hidden, dst=W13p[l * 2 * hidden:(l + 1) * 2 * hidden])
+        _pack(W3s[-1], 2, 2 * hidden, dst=W13p[l * 2 * hidden:(l + 1) * 2 * hidden])
+        _pack(W2s[-1], 0, d, dst=W2p[l * d:(l + 1) * d])
+        gam.append(torch.from_numpy((1 + 0.1 * g.standard_normal(d)).astype(np.float32)).to(dev))
+        bet.append(0.1 * g.standard_normal(d))
+    stride = (M + 255) // 256 * 256
+    Y = torch.full((layers * stride, d), float("nan"), dtype=torch.bfloat16, device=dev)
+    stats = torch.full((layers * stride, 2), float("nan"), dtype=torch.float32, device=dev)
+    err = zeros_err()
+    B.check(B.stca_k_ffn_fused(torch.from_numpy(ids).to(dev), None if dt is None else torch.from_numpy(dt).to(dev),
+                               E, T, n_items, M, layers, hidden, W13p, W2p, gam, 1e-5, Y, stride, stats, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    X = R.gather_history(E.cpu().view(torch.int16).numpy().view(np.uint16), ids, dt,
+                         None if T is None else T.cpu().view(torch.int16).numpy().view(np.uint16))
+    Yh, st = bf16_to_f64(Y), stats.cpu().numpy().astype(np.float64)
+    for l in range(layers):
+        ffn = dict(W1=bf16_to_f64(W1s[l]), W3=bf16_to_f64(W3s[l]), W2=bf16_to_f64(W2s[l]),
+                   gamma=gam[l].cpu().numpy(), beta=bet[l])
+        ref = R.ffn_ln(X, ffn, 1e-5)
+        rows = slice(l * stride, l * stride + M)
+        mean, rstd = st[rows, :1], st[rows, 1:]
+        got = rstd * (Yh[rows] - mean * ffn["gamma"]) + bet[l]
+        e = R.row_rel_err(got, ref)
+        print(f"fused FFN layer {l}: row-relative error {e:.2e}")
+        assert e <= 2e-2, (l, e)
+
+
 # ---------------------------------------------------------------- a5/a8/a9: target-side GEMMs
 
 
