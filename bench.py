@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--no-dedup", action="store_true", help="run the history GEMMs once per token")
     ap.add_argument("--uniform-ids", action="store_true",
                     help="control run: history ids uniform over the table instead of Zipf")
+    ap.add_argument("--kv-fold", action="store_true",
+                    help="fold W_K / W_V into the queries (d = 256 STCA workloads only)")
     return ap.parse_args()
 
 
@@ -357,7 +359,7 @@ def _gemm_passes(wl, dedup):
     return out * c["blocks"]
 
 
-def stage_work(stage, wl, dedup=False, fused_ffn=False):
+def stage_work(stage, wl, dedup=False, fused_ffn=False, kv_fold=False):
     """Algorithmic work of one step of a stage: (bound, amount, unit).  The history GEMMs
     count the rows they compute (distinct keys when dedup is on).  With the fused FFN
     (d = 256: one kernel runs gather, SwiGLU and W2 of every layer) the gather stage also
@@ -380,6 +382,10 @@ def stage_work(stage, wl, dedup=False, fused_ffn=False):
         return "tensor", sum(2.0 * p[0] * h * d for p in passes), "flop"
     if stage == "kv":
         return "tensor", sum(2.0 * p[0] * d * 2 * d for p in passes), "flop"
+    if stage == "attention" and kv_fold:
+        # one d-wide bf16 history row and its two LayerNorm moments per attended key, the
+        # folded queries read and the weighted rows written (fp32, d per target and head)
+        return "hbm", sum(keys * (2 * d + 8) + 2 * T * c["H"] * d * 4 for _, _, _, T, keys in passes), "byte"
     if stage == "attention":
         tot = 0.0
         for _, _, _, T, keys in passes:
@@ -429,7 +435,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     dedup = 2 if (kind != "pointwise" and wl["cfg"]["dtype"] == "bf16" and not args.no_dedup) else 0
     if kind == "stca":
-        model = StcaModel(wl, dedup=dedup)
+        model = StcaModel(wl, dedup=dedup, kv_fold=int(args.kv_fold))
         x = model.inputs(wl)
         out = torch.empty((x["t_tot"], wl["cfg"]["d"]), device="cuda")
     elif kind == "pointwise":
@@ -482,7 +488,7 @@ def run_ours(args):
     probe = profiled_steps(2)
     # the fused history FFN (d = 256) shows no separate W2 stage
     fused = kind == "stca" and wl["cfg"]["dtype"] == "bf16" and not probe.get("ffn_out", (0, 0))[1]
-    work = lambda stage: stage_work(stage, wl, dedup, fused)
+    work = lambda stage: stage_work(stage, wl, dedup, fused, bool(args.kv_fold))
     dom = max((s for s in probe if probe[s][1] and work(s)[0]), key=lambda s: probe[s][0])
 
     # The timed region: events bracket only the dominant stage (each recorded stage adds two
@@ -626,11 +632,14 @@ def run_ours(args):
     if rank != 0:
         return
     layers = wl["cfg"].get("M", wl["cfg"].get("blocks", 1))
+    cfg_line = config_block(wl, world, total_tokens)
+    if args.kv_fold:
+        cfg_line["kv_fold"] = "W_K / W_V folded into the queries (no K/V rows)"
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16" if wl["cfg"]["dtype"] == "bf16" else "f32",
-        "data": "synthetic (seeded Zipf ids, random-init weights)", "config": config_block(wl, world, total_tokens),
+        "data": "synthetic (seeded Zipf ids, random-init weights)", "config": cfg_line,
         "token_layers_per_s": round(value * layers, 1),
         "roofline": roofline, "stages": stages,
         "stages_timing": "a second pass of the same steps with every stage bracketed by CUDA events",

@@ -85,6 +85,12 @@ typedef struct {
                        2: also attend once per distinct key of each user, weighting the key
                        by the number of its tokens; the same result up to summation order */
   float ln_eps;     /* LayerNorm epsilon (biased variance) */
+  int kv_fold;      /* 1: fold W_K and W_V into the queries ([review] 核心公式 by associativity:
+                       s = (q W_Q,h W_K,h^T) . x~, o_h = (sum a x~) W_V,h), so that no K/V row is
+                       ever computed; attention reads the d-wide history rows and their
+                       LayerNorm moments.  STCA_BF16 STCA handles with d = 256, d / H = 64
+                       only (else STCA_ERR_UNSUPPORTED), not with the sequence-parallel
+                       phases.  0: project K/V per history row (default) */
 } stca_config;
 
 /* One SwiGLU FFN, SwiGLU(x) = (SiLU(x W1) * (x W3)) W2 (the "dimension-preserving"

@@ -31,7 +31,8 @@ _i64 = ctypes.c_int64
 class StcaConfig(ctypes.Structure):
     _fields_ = [("mode", _i32), ("M", _i32), ("d", _i32), ("H", _i32), ("hidden", _i32),
                 ("dtype", _i32), ("score", _i32), ("time_buckets", _i32), ("max_users", _i32),
-                ("max_tokens", _i32), ("max_targets", _i32), ("dedup", _i32), ("ln_eps", ctypes.c_float)]
+                ("max_tokens", _i32), ("max_targets", _i32), ("dedup", _i32), ("ln_eps", ctypes.c_float),
+                ("kv_fold", _i32)]
 
 
 class StcaFfn(ctypes.Structure):

@@ -103,8 +103,9 @@ __device__ __forceinline__ void load_kv_tile(uint8_t* stage, const int* slot, in
 // g + 8 of the warp's 16): running reference point mrow and sum lrow (softmax), O in o.
 template <int SCORE, int NJ>
 __device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, const float* smul, int j0,
-                                          const uint32_t (&qa)[4][4], float (&o)[8][4], float (&mrow)[2],
-                                          float (&lrow)[2], int valid, int lane) {
+                                          const uint32_t (&qa)[4][4], const uint32_t (&qlo)[4][4],
+                                          float (&o)[8][4], float (&mrow)[2], float (&lrow)[2], int valid,
+                                          int lane) {
   const int tq = lane & 3;
   // S = Q K^T
   float sacc[NJ][4];
@@ -122,6 +123,10 @@ __device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, const float*
       ldsm_x4(sK + key * 128 + ((ch ^ (key & 7)) << 4), kb);
       mma_bf16_16816(sacc[jj], qa[2 * p], kb[0], kb[1]);
       mma_bf16_16816(sacc[jj], qa[2 * p + 1], kb[2], kb[3]);
+      if (SCORE == 1) {  // the low bf16 terms of the queries (see the query fragments)
+        mma_bf16_16816(sacc[jj], qlo[2 * p], kb[0], kb[1]);
+        mma_bf16_16816(sacc[jj], qlo[2 * p + 1], kb[2], kb[3]);
+      }
     }
   }
   // keys past the slice end (last tile only)
@@ -206,7 +211,7 @@ __device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, const float*
 }
 
 template <int SCORE>
-__global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
+__global__ void __launch_bounds__(ATT_THREADS, SCORE == 1 ? 1 : 2) attn_bf16_kernel(AttnArgs a) {
   griddep_wait();
   griddep_launch();
   extern __shared__ __align__(128) uint8_t smem[];
@@ -231,8 +236,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
     const int mq = min(32, m - qp);
     const bool ksplit = mq <= 16;           // the warps of a team split keys, else queries
     const int qr0 = ksplit ? 0 : 16 * mem;  // this warp's first query row in the chunk
-    // ---- query fragments (A operand), scaled, bf16
-    uint32_t qa[4][4];
+    // ---- query fragments (A operand), scaled, bf16.  The ReLU form's output is not
+    // normalised, so its score errors do not cancel: there each query value x is carried as
+    // bf16(x) + bf16(x - bf16(x)) (qlo, two MMAs per K step), which keeps the scores at fp32
+    // accuracy; one bf16 rounding of the queries dominated its error at d = 256.
+    uint32_t qa[4][4], qlo[4][4];
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
@@ -246,6 +254,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
           x1 = qrow[1] * qscale;
         }
         qa[kk][e] = pack_bf16x2(x0, x1);
+        if (SCORE == 1) {
+          const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qa[kk][e]));
+          qlo[kk][e] = pack_bf16x2(x0 - hf.x, x1 - hf.y);
+        } else {
+          qlo[kk][e] = 0u;
+        }
       }
     float o[8][4];
 #pragma unroll
@@ -315,8 +329,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) attn_bf16_kernel(AttnArgs a) {
       const uint32_t sV = sK + TILE_BYTES;
       const int valid = min(KT, nk - tile_of(j) * KT);
       const float* smul = a.kv_mult ? reinterpret_cast<const float*>(idx_slot(j) + KT) : nullptr;
-      if (ksplit) tile_step<SCORE, 2>(sK, sV, smul, 2 * mem, qa, o, mrow, lrow, valid, lane);
-      else tile_step<SCORE, 4>(sK, sV, smul, 0, qa, o, mrow, lrow, valid, lane);
+      if (ksplit) tile_step<SCORE, 2>(sK, sV, smul, 2 * mem, qa, qlo, o, mrow, lrow, valid, lane);
+      else tile_step<SCORE, 4>(sK, sV, smul, 0, qa, qlo, o, mrow, lrow, valid, lane);
       stage = stage + 1 == KV_STAGES ? 0 : stage + 1;
     }
     cp_async_wait_all();

@@ -51,6 +51,10 @@ int fold_consts(const float* gamma, const float* beta, const void* WK, const voi
 // mode 1: SwiGLU gate half:  dst row (n/128)*256 + n%128       <- column n of W1
 // mode 2: SwiGLU up half:    dst row (n/128)*256 + 128 + n%128 <- column n of W3
 // mode 3: head-interleaved:  dst row (n/group)*2*group + row_offset + n%group <- column n
+// modes 4, 5: block-diagonal folds of a [d, d] projection per head of width group (the
+//   W_K / W_V fold into the queries): mode 4 writes W[k][n] to dst[(n/group) K + k][n] of
+//   dst [H K, N]; mode 5 to dst[n][(n/group) K + k] of dst [N, H K]; the rest of dst stays
+//   as it was (zero it once)
 int tc_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_offset, cudaStream_t s);
 
 // The same packing for many matrices with one launch per PACK_MAX_JOBS jobs.
@@ -186,6 +190,30 @@ struct AttnArgs {
   float* lse_out = nullptr;
 };
 int attention_bf16(const AttnArgs& a, cudaStream_t s);
+// Attention with W_K / W_V folded into the queries (d = 256, d_h = 64): scores of the
+// folded queries Qf [T H, d] (row t H + h = Q_{t,h} W_K,h^T) against the history rows
+// y' = y * gamma with their LayerNorm moments, and r = sum_j a_j x~_j per (target, head)
+// into out [T H, d] (one slice), or unnormalised states [splits, T H, d] + (max, sum)
+// [splits, T H, 2] for attention_merge with T' = T H, H' = 1.
+struct FoldArgs {
+  const float* Qf;
+  const void* Y;           // [U, d] bf16 history rows y'
+  const float* stats;      // [U, 2] (mean, rstd)
+  const float* gamma;      // [d]
+  const float* beta;       // [d]
+  const int32_t* hoff;
+  const int32_t* toff;
+  const int32_t* kv_rows;  // as in AttnArgs
+  const int32_t* kv_len;
+  const int32_t* kv_mult;
+  int B, T, d, H, splits, score;
+  float* part_acc;
+  float* part_ml;
+  float* out;
+  int partial_out = 0;
+  int32_t* err;
+};
+int attention_fold_bf16(const FoldArgs& a, cudaStream_t s);
 // Backward of the bf16 attention (per-token K/V rows, d_h = 64); see stca_attention_backward.
 int attention_bwd_bf16(const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B, int T, int d,
                        int H, int splits, int score, const float* O, const float* lse, const float* dO, float* dQ,

@@ -43,6 +43,9 @@ struct stca_handle {
     // STCA
     size_t tgt13, tgt2, wq[STCA_MAX_LAYERS], wo[STCA_MAX_LAYERS], wc[STCA_MAX_LAYERS], fuse13[STCA_MAX_LAYERS],
         fuse2[STCA_MAX_LAYERS], wz, z13, z2;
+    // W_K / W_V folded into the queries (kv_fold): block-diagonal [H d, d] (q~ = Q Kfold^T
+    // per head) and [d, H d] (o = r Vfold^T), zero outside the diagonal blocks
+    size_t kfold[STCA_MAX_LAYERS], vfold[STCA_MAX_LAYERS], fold_begin, fold_end;
     // decode blocks: W_Q / W_O per block and sequence, the per-token FFNs of a block back to
     // back (tok_cap tokens at most)
     size_t hwq[2 * STCA_MAX_LAYERS], hwo[2 * STCA_MAX_LAYERS], htok13[STCA_MAX_LAYERS], htok2[STCA_MAX_LAYERS];
@@ -52,6 +55,7 @@ struct stca_handle {
   // query side
   float *cat = nullptr, *qbuf = nullptr, *qproj = nullptr, *attn = nullptr, *tmp_h = nullptr, *tmp_d = nullptr;
   float *part_acc = nullptr, *part_ml = nullptr;
+  float* qfold = nullptr;  // kv_fold: folded queries [T H, d], then the weighted rows r
   float *hq = nullptr, *hqhat = nullptr, *hmix = nullptr;
   // distinct history rows
   void* dedup_ws = nullptr;
@@ -77,7 +81,7 @@ struct stca_handle {
   int in_slot = 0, z_last = -1;  // z_last: slot of the latest read-back, -1 before the first
   // one STCA forward between its phases (set by its first phase)
   struct Fwd {
-    int B = 0, n_tok = 0, t_tot = 0, splits = 1;
+    int B = 0, n_tok = 0, t_tot = 0, splits = 1, fold_splits = 1;
     const stca_weights* w = nullptr;
     GatherSrc g{};
     const int32_t *M_dev = nullptr, *kv_rows = nullptr, *kv_len = nullptr, *kv_mult = nullptr;
@@ -202,6 +206,10 @@ int validate_config(const stca_config& c) {
   if (c.score != STCA_SOFTMAX && c.score != STCA_RELU) return STCA_ERR_INVALID_ARG;
   if (c.time_buckets != 0 && c.time_buckets != 16) return STCA_ERR_UNSUPPORTED;
   if (c.dedup < 0 || c.dedup > 2) return STCA_ERR_INVALID_ARG;
+  if (c.kv_fold != 0 && c.kv_fold != 1) return STCA_ERR_INVALID_ARG;
+  if (c.kv_fold && (c.mode != STCA_MODE_STCA || c.dtype != STCA_BF16 || c.d != 256 || c.H <= 0 || c.d % c.H != 0 ||
+                    c.d / c.H != 64))
+    return STCA_ERR_UNSUPPORTED;
   if (c.mode == STCA_MODE_POINTWISE) {
     if (c.dtype != STCA_BF16 || c.d != 128 || c.dedup) return STCA_ERR_UNSUPPORTED;
     return STCA_OK;
@@ -247,6 +255,15 @@ stca_handle::QLayout q_layout(const stca_config& c) {
   q.wz = take(d * (c.M + 1) * d);
   q.z13 = take(2 * hd * d);
   q.z2 = take(d * hd);
+  q.fold_begin = at;
+  if (c.kv_fold) {
+    const size_t H = size_t(c.H);
+    for (int i = 0; i < c.M; ++i) {
+      q.kfold[i] = take(H * d * d);
+      q.vfold[i] = take(d * H * d);
+    }
+  }
+  q.fold_end = at;
   q.total = at;
   return q;
 }
@@ -311,8 +328,11 @@ int allocate(stca_handle* h) {
        dalloc(h, &h->kv, N * 2 * d * E);
   ok = ok && dalloc(h, &h->qproj, T * d * 4) && dalloc(h, &h->attn, T * d * 4) && dalloc(h, &h->tmp_h, T * hd * 4) &&
        dalloc(h, &h->tmp_d, T * d * 4);
-  ok = ok && dalloc(h, &h->part_acc, size_t(MAX_SPLITS) * T * d * 4) &&
+  // the folded attention keeps a d-wide state per (target, head)
+  const size_t acc_rows = c.kv_fold ? T * size_t(c.H) : T;
+  ok = ok && dalloc(h, &h->part_acc, size_t(MAX_SPLITS) * acc_rows * d * 4) &&
        dalloc(h, &h->part_ml, size_t(MAX_SPLITS) * T * c.H * 2 * 4);
+  if (c.kv_fold) ok = ok && dalloc(h, &h->qfold, T * size_t(c.H) * d * 4);
   if (c.dedup) {
     // one map per history sequence (the decode variant keeps both of its sequences' maps)
     h->dedup_ws_bytes = dedup_workspace_bytes(c.max_tokens);
@@ -333,6 +353,10 @@ int allocate(stca_handle* h) {
     if (c.dtype == STCA_BF16) {
       h->ql = q_layout(c);
       ok = ok && dalloc(h, &h->qpack, h->ql.total * 2);
+      // the fold matrices are block-diagonal: zero once, packing writes the blocks only
+      if (ok && h->ql.fold_end > h->ql.fold_begin)
+        ok = cudaMemset(reinterpret_cast<bf16*>(h->qpack) + h->ql.fold_begin, 0,
+                        (h->ql.fold_end - h->ql.fold_begin) * 2) == cudaSuccess;
     }
   } else {
     ok = ok && dalloc(h, &h->hoff2, U * 4) && dalloc(h, &h->hq, T * d * 4) && dalloc(h, &h->hqhat, T * d * 4) &&
@@ -458,6 +482,13 @@ void query_jobs(stca_handle* h, const stca_weights* w, std::vector<PackJob>& job
   }
   jobs.push_back({w->WZ, q + L.wz, (M + 1) * d, d, 0, 0});
   ffn_jobs(w->zffn, d, hd, q + L.z13, q + L.z2, jobs);
+  if (h->cfg.kv_fold) {
+    const int dh = d / h->cfg.H;
+    for (int i = 0; i < M; ++i) {
+      jobs.push_back({w->WK[i], q + L.kfold[i], d, d, 4, 0, dh});
+      jobs.push_back({w->WV[i], q + L.vfold[i], d, d, 5, 0, dh});
+    }
+  }
 }
 
 // Every tensor-core operand of a bf16 STCA call.
@@ -670,6 +701,8 @@ int fwd_begin(stca_handle* h, const int32_t* ids, const int32_t* lens, const int
     }
   }
   f.splits = attention_splits(n_tok, B, c.H, 1024);
+  // the folded attention has one CTA per (user, slice) for all heads: slices of >= 256 keys
+  f.fold_splits = attention_splits(n_tok, B, 1, 256);
   return STCA_OK;
 }
 
@@ -681,7 +714,7 @@ int fwd_layer_inputs(stca_handle* h, int i, cudaStream_t s) {
   const stca_weights* w = f.w;
   if (c.dtype == STCA_BF16 && fused_ffn(c)) {
     if (i == 0) CK(history_ffn_fused(h, f.g, f.n_tok, w, s, f.M_dev));
-    CK(history_kv_fused(h, i, f.n_tok, s, f.M_dev));
+    if (!c.kv_fold) CK(history_kv_fused(h, i, f.n_tok, s, f.M_dev));  // the fold needs no K/V rows
   } else if (c.dtype == STCA_BF16) {
     if (i == 0) CK(history_hidden_bf16(h, 0, f.g, f.n_tok, s, f.M_dev));
     CK(history_kv_bf16(h, 0, i, f.n_tok, w->hist[i].gamma, w->hist[i].beta, s, f.M_dev));
@@ -690,6 +723,62 @@ int fwd_layer_inputs(stca_handle* h, int i, cudaStream_t s) {
   }
   STAGE(h, STCA_STAGE_QUERY, s,
         qgemm(gemm_args<TB>(f.t_tot, c.d, c.d, h->qbuf, c.d, w->WQ[i], h->qproj, c.d, h->err), qp(h, h->ql.wq[i]), s));
+  if (c.kv_fold) {  // q~_{t,h} = Q_{t,h} W_K,h^T: [T, d] x block-diagonal -> [T, H d]
+    const int Hd = c.H * c.d;
+    STAGE(h, STCA_STAGE_QUERY, s,
+          tc_query_gemm(gemm_args<bf16>(f.t_tot, Hd, c.d, h->qproj, c.d, nullptr, h->qfold, Hd, h->err),
+                        qp(h, h->ql.kfold[i]), s));
+  }
+  return STCA_OK;
+}
+
+// Layer i's attention with W_K / W_V folded into the queries: r = sum_j a_j x~_j per (target,
+// head) from the history rows y' and their LayerNorm moments, then o_h = r_h W_V,h for all
+// heads at once into the heads buffer.
+int run_attention_fold(stca_handle* h, int i, cudaStream_t s) {
+  const stca_config& c = h->cfg;
+  const stca_handle::Fwd& f = h->fwd;
+  const size_t stride = ffn_layer_stride(c);
+  FoldArgs a;
+  a.Qf = h->qfold;
+  a.Y = reinterpret_cast<const bf16*>(h->xt) + size_t(i) * stride * c.d;
+  a.stats = h->rowstats + size_t(i) * stride * 2;
+  a.gamma = f.w->hist[i].gamma;
+  a.beta = f.w->hist[i].beta;
+  a.hoff = h->hoff;
+  a.toff = h->toff;
+  a.kv_rows = f.kv_rows;
+  a.kv_len = f.kv_len;
+  a.kv_mult = f.kv_mult;
+  a.B = f.B;
+  a.T = f.t_tot;
+  a.d = c.d;
+  a.H = c.H;
+  a.splits = f.fold_splits;
+  a.score = c.score;
+  a.part_acc = h->part_acc;
+  a.part_ml = h->part_ml;
+  a.out = h->qfold;  // a CTA reads only its user's query rows before writing them
+  a.err = h->err;
+  STAGE(h, STCA_STAGE_ATTENTION, s, attention_fold_bf16(a, s));
+  if (a.splits > 1) {  // the slices' d-wide states: the merge with one "head" of width d
+    AttnArgs m;
+    memset(&m, 0, sizeof(m));
+    m.T = f.t_tot * c.H;
+    m.d = c.d;
+    m.H = 1;
+    m.splits = a.splits;
+    m.score = c.score;
+    m.part_acc = h->part_acc;
+    m.part_ml = h->part_ml;
+    m.out = h->qfold;
+    m.err = h->err;
+    STAGE(h, STCA_STAGE_MERGE, s, attention_merge(m, s));
+  }
+  const int Hd = c.H * c.d;
+  STAGE(h, STCA_STAGE_QUERY, s,
+        tc_query_gemm(gemm_args<bf16>(f.t_tot, c.d, Hd, h->qfold, Hd, nullptr, h->attn, c.d, h->err),
+                      qp(h, h->ql.vfold[i]), s));
   return STCA_OK;
 }
 
@@ -738,7 +827,9 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
   const stca_handle::Fwd& f = h->fwd;
   for (int i = 0; i < M; ++i) {
     CK(fwd_layer_inputs<TB>(h, i, s));
-    CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, f.splits, c.score, s, f.kv_rows, f.kv_len, f.kv_mult));
+    if (c.kv_fold) CK(run_attention_fold(h, i, s));
+    else CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, f.splits, c.score, s, f.kv_rows, f.kv_len,
+                          f.kv_mult));
     CK(fwd_layer_outputs<TB>(h, i, z_out, s));
   }
   if (o_out && t_tot > 0) {
@@ -965,6 +1056,7 @@ int stca_lsplit_begin(stca_handle* h, const int32_t* hist_ids, const int32_t* hi
                       const stca_weights* w, void* stream) {
   CK(check_forward_args(h, hist_ids, hist_lengths, hist_dt, target_emb, targets_per_user, B, n_tok, t_tot, w,
                         nullptr, false));
+  if (h->cfg.kv_fold) return STCA_ERR_UNSUPPORTED;  // the folded attention keeps no slice state API
   if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   h->last_stream = s;

@@ -766,10 +766,19 @@ __global__ void pack_many_kernel(PackJobs jobs) {
   for (int i = threadIdx.y; i < 32; i += blockDim.y) {
     const int n = n0 + i, k = k0 + threadIdx.x;
     if (n < jb.N && k < jb.K) {
-      const int row = jb.mode == 0   ? jb.row_offset + n
-                      : jb.mode == 3 ? (n / jb.group) * 2 * jb.group + jb.row_offset + n % jb.group
-                                     : (n / 128) * 256 + (jb.mode == 2 ? 128 : 0) + (n % 128);
-      dst[int64_t(row) * jb.K + k] = tile[threadIdx.x][i];
+      if (jb.mode >= 4) {
+        // block-diagonal folds of a [K, N] = [d, d] projection (g = group = d_h, H = N / g):
+        // mode 4: dst [H K, N], dst[(n / g) K + k][n] = W[k][n]   (q~ = Q dst^T per head)
+        // mode 5: dst [N, H K], dst[n][(n / g) K + k] = W[k][n]   (o = r dst^T per head)
+        const int64_t hk = int64_t(n / jb.group) * jb.K + k;
+        const int64_t at = jb.mode == 4 ? hk * jb.N + n : int64_t(n) * (int64_t(jb.N / jb.group) * jb.K) + hk;
+        dst[at] = tile[threadIdx.x][i];
+      } else {
+        const int row = jb.mode == 0   ? jb.row_offset + n
+                        : jb.mode == 3 ? (n / jb.group) * 2 * jb.group + jb.row_offset + n % jb.group
+                                       : (n / 128) * 256 + (jb.mode == 2 ? 128 : 0) + (n % 128);
+        dst[int64_t(row) * jb.K + k] = tile[threadIdx.x][i];
+      }
     }
   }
 }
@@ -896,8 +905,8 @@ int tc_pack_weights(const PackJob* jobs, int n, cudaStream_t s) {
     int gx = 1, gy = 1;
     for (int i = 0; i < cnt; ++i) {
       const PackJob& jb = jobs[b + i];
-      if (jb.K <= 0 || jb.N <= 0 || !jb.W || !jb.dst || jb.mode < 0 || jb.mode > 3) return STCA_ERR_INVALID_ARG;
-      if (jb.mode == 3 && (jb.group <= 0 || jb.N % jb.group != 0)) return STCA_ERR_INVALID_ARG;
+      if (jb.K <= 0 || jb.N <= 0 || !jb.W || !jb.dst || jb.mode < 0 || jb.mode > 5) return STCA_ERR_INVALID_ARG;
+      if (jb.mode >= 3 && (jb.group <= 0 || jb.N % jb.group != 0)) return STCA_ERR_INVALID_ARG;
       batch.j[i] = jb;
       gx = std::max(gx, (jb.N + 31) / 32);
       gy = std::max(gy, (jb.K + 31) / 32);

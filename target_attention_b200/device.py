@@ -51,7 +51,7 @@ class StcaModel(_Holder):
     (stca_config.dedup) defaults to 2 for bf16 workloads: the history GEMMs run once per
     distinct key of the call, attention once per distinct key of each user."""
 
-    def __init__(self, wl, device="cuda", max_users=None, max_tokens=None, max_targets=None, dedup=None):
+    def __init__(self, wl, device="cuda", max_users=None, max_tokens=None, max_targets=None, dedup=None, kv_fold=0):
         super().__init__(device)
         c = wl["cfg"]
         self.cfg = c
@@ -61,7 +61,8 @@ class StcaModel(_Holder):
             score=B.RELU if c["score"] == "relu" else B.SOFTMAX, time_buckets=c["time_buckets"],
             max_users=max_users or len(wl["lengths"]), max_tokens=max_tokens or int(wl["lengths"].sum()),
             max_targets=max_targets or int(wl["targets_per_user"].sum()),
-            dedup=int((2 if c["dtype"] == "bf16" else 0) if dedup is None else dedup), ln_eps=c.get("ln_eps", 1e-5))
+            dedup=int((2 if c["dtype"] == "bf16" else 0) if dedup is None else dedup), ln_eps=c.get("ln_eps", 1e-5),
+            kv_fold=int(kv_fold))
         w = wl["weights"]
         ws = B.StcaWeights()
         ws.table = self.p(wl["table"])

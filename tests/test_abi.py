@@ -33,7 +33,7 @@ def test_library_exports_every_declared_function():
 
 def test_struct_layouts_match_c():
     # sizes computed by the C compiler from include/stca.h
-    assert ctypes.sizeof(B.StcaConfig) == 52
+    assert ctypes.sizeof(B.StcaConfig) == 56
     assert ctypes.sizeof(B.StcaWeights) == 1072
     assert ctypes.sizeof(B.HyfWeights) == 21656
 
@@ -68,6 +68,9 @@ def _cfg(**kw):
     (dict(dtype=B.FP32, d=64, H=2, dedup=1), B.ERR_UNSUPPORTED),
     (dict(dtype=B.FP32, d=64, H=2, dedup=2), B.ERR_UNSUPPORTED),
     (dict(dedup=3), B.ERR_INVALID_ARG),
+    (dict(kv_fold=2), B.ERR_INVALID_ARG),
+    (dict(kv_fold=1, d=512, H=8, hidden=1024), B.ERR_UNSUPPORTED),   # the fold needs d = 256
+    (dict(kv_fold=1, dtype=B.FP32, d=64, H=2, hidden=128), B.ERR_UNSUPPORTED),
     (dict(dedup=-1), B.ERR_INVALID_ARG),
 ])
 def test_create_rejects_bad_configs(kw, code):

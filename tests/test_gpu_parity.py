@@ -62,6 +62,12 @@ def test_config3_relu_scores():
     _check_stca(make_stca(3, users=2, L=300, n_items=10_000, M=2, score="relu"), TOL_BF16)
 
 
+def test_config2_relu_scores():
+    """ReLU scores on the d = 256 shape (Beta-ragged ~1.4K histories, M = 2): unnormalised,
+    so the queries' rounding is not cancelled by a softmax denominator."""
+    _check_stca(make_stca(2, users=6, n_items=20_000, score="relu"), TOL_BF16)
+
+
 def test_ragged_edge_cases():
     """Empty histories, a single-token history, users without targets, ragged tails."""
     lengths = np.array([0, 1, 129, 0, 257, 40], np.int32)
