@@ -17,6 +17,8 @@
 // Numbering by first occurrence is deterministic and keeps a user's new items on
 // consecutive K/V rows, while repeated items point at rows of popular (cache-resident)
 // keys.
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -199,16 +201,12 @@ __device__ void compact_per_token(const int32_t* __restrict__ rows, int h0, int 
   if (threadIdx.x == 0) out_len[u] = L;
 }
 
-__global__ void __launch_bounds__(SCAN_THREADS) compact_user_kernel(const int32_t* __restrict__ hoff,
-                                                                    const int32_t* __restrict__ rows,
-                                                                    int32_t* __restrict__ out_rows,
-                                                                    int32_t* __restrict__ out_mult,
-                                                                    int32_t* __restrict__ out_len) {
-  griddep_wait();
-  griddep_launch();
-  extern __shared__ int32_t cu_smem[];
+// User u's compaction by the whole block, with cu_smem (CU_SMEM bytes) for its table.
+__device__ void compact_user(int u, const int32_t* __restrict__ hoff, const int32_t* __restrict__ rows,
+                             int32_t* __restrict__ out_rows, int32_t* __restrict__ out_mult,
+                             int32_t* __restrict__ out_len, int32_t* cu_smem) {
   __shared__ int table_failed;
-  const int u = blockIdx.x;
+  __syncthreads();  // a block that runs several users: the previous one is done with the table
   const int h0 = hoff[u], L = hoff[u + 1] - h0;
   if (L >= CU_SLOTS) {  // too long for the table: every token is its own entry
     compact_per_token(rows, h0, L, out_rows, out_mult, out_len, u);
@@ -287,6 +285,162 @@ __global__ void __launch_bounds__(SCAN_THREADS) compact_user_kernel(const int32_
   if (threadIdx.x == 0) out_len[u] = base;
 }
 
+__global__ void __launch_bounds__(SCAN_THREADS) compact_user_kernel(const int32_t* __restrict__ hoff,
+                                                                    const int32_t* __restrict__ rows,
+                                                                    int32_t* __restrict__ out_rows,
+                                                                    int32_t* __restrict__ out_mult,
+                                                                    int32_t* __restrict__ out_len) {
+  griddep_wait();
+  griddep_launch();
+  extern __shared__ int32_t cu_smem[];
+  compact_user(blockIdx.x, hoff, rows, out_rows, out_mult, out_len, cu_smem);
+}
+
+// ---- everything above in one cooperative launch (one block per SM): clear the table,
+// insert, count first occurrences per tile, number them, map every token, and (when hoff
+// is given) compact every user, with a grid-wide barrier between the phases.  At short
+// histories the separate launches (and their gaps) cost more than the work; a block
+// numbers a tile from the sum of the earlier tiles' counts, so no scan pass is needed.
+
+struct DedupFused {
+  const int32_t* ids;
+  const int32_t* dt;
+  int n;
+  unsigned long long* keys;
+  int32_t* first;
+  int32_t* slot_of;
+  int32_t* pos;
+  int32_t* tile_counts;
+  unsigned mask;
+  unsigned* barrier;  // zero at launch
+  int32_t* uniq_idx;
+  int32_t* uniq_token;
+  int32_t* count;
+  const int32_t* hoff;  // compaction when not null
+  int B;
+  int32_t* c_rows;
+  int32_t* c_mult;
+  int32_t* c_len;
+  int32_t* err;
+};
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Grid-wide barrier number k (1, 2, ...): every block arrives once; bounded wait (records
+// STCA_ERR_TIMEOUT and returns false when the other blocks do not arrive in time).
+__device__ bool grid_barrier(unsigned* ctr, unsigned k, int32_t* err) {
+  __shared__ int ok_s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1u);
+    const unsigned target = k * gridDim.x;
+    int ok = 1;
+    if (ld_acquire_gpu(ctr) < target) {
+      const uint64_t t0 = global_timer_ns();
+      while (ld_acquire_gpu(ctr) < target) {
+        if (global_timer_ns() - t0 > STCA_WAIT_NS) {
+          set_error(err, STCA_ERR_TIMEOUT);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
+__global__ void __launch_bounds__(SCAN_THREADS, 1) dedup_fused_kernel(DedupFused a) {
+  extern __shared__ int32_t cu_smem[];
+  const int tid = threadIdx.x, G = gridDim.x;
+  const int64_t gthreads = int64_t(G) * SCAN_THREADS, gtid = int64_t(blockIdx.x) * SCAN_THREADS + tid;
+  const int n = a.n;
+  const int64_t cap = int64_t(a.mask) + 1;
+  // 0. empty table
+  for (int64_t i = gtid; i < cap; i += gthreads) {
+    a.keys[i] = EMPTY_KEY;
+    a.first[i] = 0x7fffffff;
+  }
+  if (!grid_barrier(a.barrier, 1, a.err)) return;
+  // 1. insert every token's key
+  for (int64_t i = gtid; i < n; i += gthreads) {
+    const int ii = int(i);
+    const unsigned long long key = row_key(a.ids, a.dt, ii);
+    unsigned slot = unsigned(mix64(key)) & a.mask;
+    bool placed = false;
+    for (unsigned probe = 0; probe <= a.mask; ++probe) {
+      unsigned long long prev = __ldcg(&a.keys[slot]);
+      if (prev == EMPTY_KEY) prev = atomicCAS(&a.keys[slot], EMPTY_KEY, key);
+      if (prev == EMPTY_KEY || prev == key) {
+        if (__ldcg(&a.first[slot]) > ii) atomicMin(&a.first[slot], ii);
+        a.slot_of[ii] = int32_t(slot);
+        placed = true;
+        break;
+      }
+      slot = (slot + 1) & a.mask;
+    }
+    if (!placed) {
+      set_error(a.err, STCA_ERR_CAPACITY);
+      a.slot_of[ii] = 0;
+    }
+  }
+  if (!grid_barrier(a.barrier, 2, a.err)) return;
+  // 2. first occurrences per tile of SCAN_TILE tokens
+  const int tiles = (n + SCAN_TILE - 1) / SCAN_TILE;
+  for (int t = blockIdx.x; t < tiles; t += G) {
+    const int base = t * SCAN_TILE + tid * SCAN_ITEMS;
+    int c = 0;
+#pragma unroll
+    for (int k = 0; k < SCAN_ITEMS; ++k)
+      if (base + k < n && is_first(a.first, a.slot_of, base + k)) ++c;
+    int excl;
+    const int total = block_exclusive_scan(c, excl);
+    if (tid == 0) a.tile_counts[t] = total;
+  }
+  if (!grid_barrier(a.barrier, 3, a.err)) return;
+  // 3. number the first occurrences: tile t starts at the sum of the earlier tiles' counts
+  for (int t = blockIdx.x; t < tiles; t += G) {
+    int before = 0;
+    for (int i = tid; i < t; i += SCAN_THREADS) before += a.tile_counts[i];
+    int excl0;
+    const int start = block_exclusive_scan(before, excl0);  // the block total
+    const int base = t * SCAN_TILE + tid * SCAN_ITEMS;
+    bool f[SCAN_ITEMS];
+    int c = 0;
+#pragma unroll
+    for (int k = 0; k < SCAN_ITEMS; ++k) {
+      f[k] = base + k < n && is_first(a.first, a.slot_of, base + k);
+      c += f[k];
+    }
+    int excl;
+    const int total = block_exclusive_scan(c, excl);
+    int p = start + excl;
+#pragma unroll
+    for (int k = 0; k < SCAN_ITEMS; ++k)
+      if (f[k]) {
+        a.pos[base + k] = p;
+        a.uniq_token[p] = base + k;
+        ++p;
+      }
+    if (t == tiles - 1 && tid == 0) *a.count = start + total;
+  }
+  if (tiles == 0 && blockIdx.x == 0 && tid == 0) *a.count = 0;
+  if (!grid_barrier(a.barrier, 4, a.err)) return;
+  // 4. token -> number of its key
+  for (int64_t i = gtid; i < n; i += gthreads) a.uniq_idx[i] = a.pos[a.first[a.slot_of[i]]];
+  if (!a.hoff) return;
+  if (!grid_barrier(a.barrier, 5, a.err)) return;
+  // 5. per-user compaction of the K/V rows
+  for (int u = blockIdx.x; u < a.B; u += G) compact_user(u, a.hoff, a.uniq_idx, a.c_rows, a.c_mult, a.c_len, cu_smem);
+}
+
 }  // namespace
 
 int compact_user_rows(const int32_t* hoff, int B, const int32_t* rows, int32_t* out_rows, int32_t* out_mult,
@@ -307,10 +461,11 @@ size_t dedup_table_slots(int max_tokens) {
 }
 
 namespace {
-// keys [cap] u64 | first [cap] i32 | slot_of [n] i32 | pos [n] i32 | tile offsets
+// keys [cap] u64 | first [cap] i32 | slot_of [n] i32 | pos [n] i32 | tile offsets |
+// the fused kernel's barrier counter (16-byte aligned)
 size_t layout_bytes(size_t cap, int n) {
   const size_t tiles = (size_t(n) + SCAN_TILE - 1) / SCAN_TILE + 1;
-  return cap * 8 + cap * 4 + size_t(n) * 8 + tiles * 4 + 64;
+  return cap * 8 + cap * 4 + size_t(n) * 8 + tiles * 4 + 64 + 64;
 }
 }  // namespace
 
@@ -344,6 +499,64 @@ int dedup_rows(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws
   launch_dep(map_kernel, dim3((n + 255) / 256), dim3(256), 0, s, first, slot_of, pos, n, uniq_idx);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? STCA_OK : STCA_ERR_CUDA;
+}
+
+int dedup_fused(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws_bytes, int32_t* uniq_idx,
+                int32_t* uniq_token, int32_t* count, const int32_t* hoff, int B, int32_t* c_rows, int32_t* c_mult,
+                int32_t* c_len, int32_t* err, cudaStream_t s) {
+  if (n < 0 || B < 0) return STCA_ERR_INVALID_ARG;
+  const size_t cap = dedup_table_slots(n);
+  if (layout_bytes(cap, n) > ws_bytes) return STCA_ERR_CAPACITY;
+  uint8_t* p = reinterpret_cast<uint8_t*>(ws);
+  DedupFused a;
+  a.ids = ids;
+  a.dt = dt;
+  a.n = n;
+  a.keys = reinterpret_cast<unsigned long long*>(p);
+  a.first = reinterpret_cast<int32_t*>(p + cap * 8);
+  a.slot_of = a.first + cap;
+  a.pos = a.slot_of + n;
+  a.tile_counts = a.pos + n;
+  const size_t tiles = (size_t(n) + SCAN_TILE - 1) / SCAN_TILE + 1;
+  const uintptr_t bar = (reinterpret_cast<uintptr_t>(a.tile_counts + tiles) + 15) & ~uintptr_t(15);
+  a.barrier = reinterpret_cast<unsigned*>(bar);
+  a.mask = unsigned(cap - 1);
+  a.uniq_idx = uniq_idx;
+  a.uniq_token = uniq_token;
+  a.count = count;
+  a.hoff = (hoff && B > 0) ? hoff : nullptr;
+  a.B = B;
+  a.c_rows = c_rows;
+  a.c_mult = c_mult;
+  a.c_len = c_len;
+  a.err = err;
+  if (a.hoff && (!c_rows || !c_mult || !c_len)) return STCA_ERR_INVALID_ARG;
+  static int blocks_per_sm = -1;
+  if (blocks_per_sm < 0) {
+    if (cudaFuncSetAttribute(dedup_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(CU_SMEM)) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, dedup_fused_kernel, SCAN_THREADS, CU_SMEM) !=
+            cudaSuccess || blocks_per_sm < 1)
+      return STCA_ERR_CUDA;
+  }
+  if (cudaMemsetAsync(a.barrier, 0, sizeof(unsigned), s) != cudaSuccess) return STCA_ERR_CUDA;
+  int grid = sm_count() * blocks_per_sm;
+  const int64_t want = std::max<int64_t>(std::max<int64_t>((int64_t(n) + SCAN_THREADS - 1) / SCAN_THREADS, B), 1);
+  if (grid > want) grid = int(want);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(SCAN_THREADS);
+  cfg.dynamicSmemBytes = CU_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every block resident at once: the barriers need it
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, dedup_fused_kernel, a) != cudaSuccess) return STCA_ERR_CUDA;
+  note_launch();
+  return STCA_OK;
 }
 
 }  // namespace stca

@@ -270,6 +270,10 @@ int dedup_rows(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws
 // the user in order of first token, out_rows[hoff[u] + i], with their token counts
 // out_mult[hoff[u] + i], i < out_len[u].  A user of 16384 or more tokens keeps one entry
 // per token (multiplicity 1).
+// dedup_rows and (when hoff != null) compact_user_rows in one cooperative launch.
+int dedup_fused(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws_bytes, int32_t* uniq_idx,
+                int32_t* uniq_token, int32_t* count, const int32_t* hoff, int B, int32_t* c_rows, int32_t* c_mult,
+                int32_t* c_len, int32_t* err, cudaStream_t s);
 int compact_user_rows(const int32_t* hoff, int B, const int32_t* rows, int32_t* out_rows, int32_t* out_mult,
                       int32_t* out_len, cudaStream_t s);
 

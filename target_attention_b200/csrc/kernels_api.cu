@@ -148,8 +148,8 @@ size_t stca_k_dedup_workspace_bytes(int n) { return n < 0 ? 0 : dedup_workspace_
 int stca_k_dedup(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t ws_bytes, int32_t* uniq_idx,
                  int32_t* uniq_token, int32_t* count, int32_t* err, void* stream) {
   if (n < 0 || !count || (n > 0 && (!ids || !ws || !uniq_idx || !uniq_token))) return STCA_ERR_INVALID_ARG;
-  return dedup_rows(ids, dt, n, ws, ws_bytes, uniq_idx, uniq_token, count, err,
-                    reinterpret_cast<cudaStream_t>(stream));
+  return dedup_fused(ids, dt, n, ws, ws_bytes, uniq_idx, uniq_token, count, nullptr, 0, nullptr, nullptr, nullptr,
+                     err, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int stca_k_compact_user_rows(const int32_t* hoff, int B, const int32_t* rows, int32_t* out_rows, int32_t* out_mult,

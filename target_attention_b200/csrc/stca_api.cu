@@ -17,6 +17,11 @@ using namespace stca;
 namespace {
 
 constexpr int MAX_SPLITS = 16;
+// Distinct keys of calls up to this many tokens are found in one cooperative launch
+// (dedup_fused): at short histories the separate launches cost more than the work (config
+// 2, 87K tokens: 47 -> 41 us per call), while at 2.56M tokens the fused kernel's one block
+// per SM gives the atomic inserts half the occupancy of the separate kernels (102 -> 121 us).
+constexpr int FUSED_DEDUP_MAX_TOKENS = 1 << 18;
 
 }  // namespace
 
@@ -184,13 +189,17 @@ int choose_splits(int64_t n_tok, int B, int per_split) {
   return int(s);
 }
 
-// L-slices per user for the attention.  Every slice adds a partial state to write and
-// merge, so slices are only added while the grid (users x heads x slices) is short of
-// four waves of two CTAs per SM, and never below min_keys keys per slice on average.
-int attention_splits(int64_t n_tok, int B, int H, int min_keys) {
+// L-slices per user for the attention: about enough (user, head, slice) CTAs to fill one
+// wave of the GPU (ctas_per_sm resident CTAs per SM), never so many that a slice averages
+// fewer than min_keys keys.  Every extra slice costs a merge launch and a round trip of the
+// slice states, which on short, latency-bound steps outweighs the idle SMs of a partly
+// filled wave (config 2, 64 users x 4 heads: one slice 0.042 ms of attention and no merge,
+// against 0.050 + 0.017 ms with two).
+int attention_splits(int64_t n_tok, int B, int H, int min_keys, int ctas_per_sm = 2) {
   if (B <= 0 || H <= 0) return 1;
   const int64_t ctas = int64_t(B) * H;
-  const int64_t want = (int64_t(8) * sm_count() + ctas - 1) / ctas;
+  const int64_t slots = int64_t(ctas_per_sm) * sm_count();
+  const int64_t want = (slots + ctas / 2) / ctas;  // the nearest whole number of slices
   const int64_t cap = choose_splits(n_tok, B, min_keys);
   const int64_t s = want < cap ? want : cap;
   return int(s < 1 ? 1 : s);
@@ -686,15 +695,25 @@ int fwd_begin(stca_handle* h, const int32_t* ids, const int32_t* lens, const int
   f.g.dt_table = c.time_buckets ? w->dt_table : nullptr;
   f.g.n_items = w->n_items;
   if (c.dedup) {
-    STAGE(h, STCA_STAGE_DEDUP, s,
-          dedup_rows(ids, f.g.dt, n_tok, h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx, h->uniq_token, h->uniq_count,
-                     h->err, s));
+    // distinct keys of the call and (dedup = 2) each user's compacted rows, one launch
+    const bool compact = c.dedup == 2;
+    if (n_tok <= FUSED_DEDUP_MAX_TOKENS) {
+      STAGE(h, STCA_STAGE_DEDUP, s,
+            dedup_fused(ids, f.g.dt, n_tok, h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx, h->uniq_token,
+                        h->uniq_count, compact ? h->hoff : nullptr, B, h->c_rows, h->c_mult, h->c_len, h->err, s));
+    } else {
+      STAGE(h, STCA_STAGE_DEDUP, s,
+            dedup_rows(ids, f.g.dt, n_tok, h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx, h->uniq_token,
+                       h->uniq_count, h->err, s));
+      if (compact)
+        STAGE(h, STCA_STAGE_DEDUP, s,
+              compact_user_rows(h->hoff, B, h->uniq_idx, h->c_rows, h->c_mult, h->c_len, s));
+    }
     f.g.rows = h->uniq_token;
     f.M_dev = h->uniq_count;
     f.kv_rows = h->uniq_idx;
-    if (c.dedup == 2) {
+    if (compact) {
       // attention over each user's distinct rows, each weighted by its token count
-      STAGE(h, STCA_STAGE_DEDUP, s, compact_user_rows(h->hoff, B, h->uniq_idx, h->c_rows, h->c_mult, h->c_len, s));
       f.kv_rows = h->c_rows;
       f.kv_len = h->c_len;
       f.kv_mult = h->c_mult;
@@ -702,7 +721,7 @@ int fwd_begin(stca_handle* h, const int32_t* ids, const int32_t* lens, const int
   }
   f.splits = attention_splits(n_tok, B, c.H, 1024);
   // the folded attention has one CTA per (user, slice) for all heads: slices of >= 256 keys
-  f.fold_splits = attention_splits(n_tok, B, 1, 256);
+  f.fold_splits = attention_splits(n_tok, B, 1, 256, 3);
   return STCA_OK;
 }
 
@@ -1239,13 +1258,20 @@ int hyformer_forward(stca_handle* h, const int32_t* ids_feed, const int32_t* len
         const size_t off = size_t(sq) * c.max_tokens;
         const size_t uoff = size_t(sq) * (size_t(c.max_users) + 1);
         if (l == 0) {
-          STAGE(h, STCA_STAGE_DEDUP, s,
-                dedup_rows(ids[sq], nullptr, ntok[sq], h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx + off,
-                           h->uniq_token + off, h->uniq_count + sq, h->err, s));
-          if (c.dedup == 2)
+          if (ntok[sq] <= FUSED_DEDUP_MAX_TOKENS) {
             STAGE(h, STCA_STAGE_DEDUP, s,
-                  compact_user_rows(offs[sq], B, h->uniq_idx + off, h->c_rows + off, h->c_mult + off,
-                                    h->c_len + uoff, s));
+                  dedup_fused(ids[sq], nullptr, ntok[sq], h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx + off,
+                              h->uniq_token + off, h->uniq_count + sq, c.dedup == 2 ? offs[sq] : nullptr, B,
+                              h->c_rows + off, h->c_mult + off, h->c_len + uoff, h->err, s));
+          } else {
+            STAGE(h, STCA_STAGE_DEDUP, s,
+                  dedup_rows(ids[sq], nullptr, ntok[sq], h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx + off,
+                             h->uniq_token + off, h->uniq_count + sq, h->err, s));
+            if (c.dedup == 2)
+              STAGE(h, STCA_STAGE_DEDUP, s,
+                    compact_user_rows(offs[sq], B, h->uniq_idx + off, h->c_rows + off, h->c_mult + off,
+                                      h->c_len + uoff, s));
+          }
         }
         g.rows = h->uniq_token + off;
         M_dev = h->uniq_count + sq;
