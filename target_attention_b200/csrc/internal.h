@@ -77,9 +77,11 @@ int tc_pack_weights(const PackJob* jobs, int n, cudaStream_t s);
 // M_dev, when not null, is a device int holding the number of rows actually present
 // (<= M); M then only sizes the tensor maps and buffers.  x_out (A_GATHER only, may be
 // null): bf16 [M, K] receiving the gathered A rows (E[id] + T[bucket]) as the MMAs used them.
+// max_pairs > 0 caps the persistent grid at that many CTA pairs (leaving SMs to kernels that
+// run beside it on another stream).
 int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int K, const void* Wp,
                      int Nout, void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev = nullptr,
-                     void* x_out = nullptr, const EpiFold* fold = nullptr);
+                     void* x_out = nullptr, const EpiFold* fold = nullptr, int max_pairs = 0);
 
 // C[M, N] (bf16) = epi(A Wp^T), A dense bf16 [M, K] streamed (K a multiple of 64),
 // N in {256, 512}; epi EPI_LN applies LayerNorm (gamma, beta, eps) over the full row.

@@ -80,6 +80,10 @@ struct stca_handle {
   void* in_xt[2] = {};
   float* out_z[2] = {};
   cudaStream_t copy_stream = nullptr, back_stream = nullptr;
+  // the fused-FFN path's K/V GEMMs of layers >= 1 run on side_stream beside layer 0's
+  // attention and target side; kv_done[l] marks layer l's K/V rows ready
+  cudaStream_t side_stream = nullptr;
+  cudaEvent_t ffn_done = nullptr, kv_done[STCA_MAX_LAYERS] = {};
   cudaEvent_t in_ready[2] = {}, in_free[2] = {};  // slot copied / slot read by its forward
   cudaEvent_t z_ready[2] = {}, z_free[2] = {};    // slot written by its forward / slot read back
   bool in_used[2] = {false, false}, z_used[2] = {false, false};
@@ -87,6 +91,7 @@ struct stca_handle {
   // one STCA forward between its phases (set by its first phase)
   struct Fwd {
     int B = 0, n_tok = 0, t_tot = 0, splits = 1, fold_splits = 1;
+    bool kv_ahead = false;  // the K/V GEMMs of layers >= 1 were issued on the side stream
     const stca_weights* w = nullptr;
     GatherSrc g{};
     const int32_t *M_dev = nullptr, *kv_rows = nullptr, *kv_len = nullptr, *kv_mult = nullptr;
@@ -333,8 +338,10 @@ int allocate(stca_handle* h) {
   // bf16: the hidden activations of all M layers of every sequence ([N, M h] per sequence),
   // not needed when the fused FFN keeps them on chip
   const size_t hid_elems = fused ? 0 : c.dtype == STCA_BF16 ? nseq * N * size_t(c.M) * hd : N * hd;
+  // K/V rows: one buffer per layer on the fused-FFN path (its layers' K/V GEMMs run ahead)
+  const size_t kv_layers = (fused && !c.kv_fold) ? size_t(c.M) : 1;
   ok = ok && dalloc(h, &h->hidden, hid_elems * E) && dalloc(h, &h->xt, xt_rows * d * E) &&
-       dalloc(h, &h->kv, N * 2 * d * E);
+       dalloc(h, &h->kv, kv_layers * N * 2 * d * E);
   ok = ok && dalloc(h, &h->qproj, T * d * 4) && dalloc(h, &h->attn, T * d * 4) && dalloc(h, &h->tmp_h, T * hd * 4) &&
        dalloc(h, &h->tmp_d, T * d * 4);
   // the folded attention keeps a d-wide state per (target, head)
@@ -578,6 +585,22 @@ int history_kv_bf16(stca_handle* h, int sq, int l, int n_tok, const float* gamma
   return STCA_OK;
 }
 
+// K/V rows of layer l: their own buffer on the fused-FFN path, else the one shared buffer.
+void* kv_ptr(const stca_handle* h, int l) {
+  const stca_config& c = h->cfg;
+  if (!fused_ffn(c) || c.kv_fold) return h->kv;
+  return reinterpret_cast<bf16*>(h->kv) + size_t(l) * size_t(c.max_tokens) * 2 * c.d;
+}
+
+bool make_side_stream(stca_handle* h) {
+  if (h->side_stream) return true;
+  bool ok = cudaStreamCreateWithFlags(&h->side_stream, cudaStreamNonBlocking) == cudaSuccess &&
+            cudaEventCreateWithFlags(&h->ffn_done, cudaEventDisableTiming) == cudaSuccess;
+  for (int l = 0; l < STCA_MAX_LAYERS && ok; ++l)
+    ok = cudaEventCreateWithFlags(&h->kv_done[l], cudaEventDisableTiming) == cudaSuccess;
+  return ok;
+}
+
 // d = 256: y'_l = (A_l W2_l) * gamma_l and the row moments of every layer in one fused
 // launch (the hidden activations A_l stay on chip).
 int history_ffn_fused(stca_handle* h, const GatherSrc& g, int n_tok, const stca_weights* w, cudaStream_t s,
@@ -592,7 +615,7 @@ int history_ffn_fused(stca_handle* h, const GatherSrc& g, int n_tok, const stca_
 }
 
 // [K | V] of layer l from the fused FFN's outputs, with the LayerNorm folded in.
-int history_kv_fused(stca_handle* h, int l, int n_tok, cudaStream_t s, const int32_t* M_dev) {
+int history_kv_fused(stca_handle* h, int l, int n_tok, cudaStream_t s, const int32_t* M_dev, int max_pairs = 0) {
   const int d = h->cfg.d;
   const size_t stride = ffn_layer_stride(h->cfg);
   GatherSrc none;
@@ -601,10 +624,14 @@ int history_kv_fused(stca_handle* h, int l, int n_tok, cudaStream_t s, const int
   const EpiFold fold{h->rowstats + size_t(l) * stride * 2, h->fold + size_t(l) * 4 * d,
                      h->fold + size_t(l) * 4 * d + 2 * d};
   STAGE(h, STCA_STAGE_KV, s,
-        tc_gemm_resident(A_TMA, EPI_LNFOLD, y, none, n_tok, d, wp3(h, l), 2 * d, h->kv, 2 * d, h->err, s, M_dev,
-                         nullptr, &fold));
+        tc_gemm_resident(A_TMA, EPI_LNFOLD, y, none, n_tok, d, wp3(h, l), 2 * d, kv_ptr(h, l), 2 * d, h->err, s,
+                         M_dev, nullptr, &fold, max_pairs));
   return STCA_OK;
 }
+
+// SM pairs the K/V GEMMs that run ahead on the side stream may use: the rest stay free for
+// the latency-bound attention and target-side kernels of the current layer.
+constexpr int KV_AHEAD_PAIRS = 64;
 
 // K/V of every history token for one layer: fp32 SIMT path.
 int history_f32(stca_handle* h, const GatherSrc& g, int n_tok, const stca_ffn& f, const void* WK, const void* WV,
@@ -632,10 +659,10 @@ int history_f32(stca_handle* h, const GatherSrc& g, int n_tok, const stca_ffn& f
 
 int run_attention(stca_handle* h, const float* Q, const int32_t* hoff, const int32_t* toff, int B, int T,
                   int splits, int score, cudaStream_t s, const int32_t* kv_rows, const int32_t* kv_len = nullptr,
-                  const int32_t* kv_mult = nullptr) {
+                  const int32_t* kv_mult = nullptr, const void* kv = nullptr) {
   AttnArgs a;
   a.Q = Q;
-  a.KV = h->kv;
+  a.KV = kv ? kv : h->kv;
   a.hoff = hoff;
   a.toff = toff;
   a.kv_rows = kv_rows;
@@ -733,7 +760,22 @@ int fwd_layer_inputs(stca_handle* h, int i, cudaStream_t s) {
   const stca_weights* w = f.w;
   if (c.dtype == STCA_BF16 && fused_ffn(c)) {
     if (i == 0) CK(history_ffn_fused(h, f.g, f.n_tok, w, s, f.M_dev));
-    if (!c.kv_fold) CK(history_kv_fused(h, i, f.n_tok, s, f.M_dev));  // the fold needs no K/V rows
+    if (!c.kv_fold && f.kv_ahead) {
+      // every layer's K/V depends only on the fused FFN: layers >= 1 go to the side stream
+      // now and run beside this layer's attention and target side
+      if (i == 0) {
+        if (cudaEventRecord(h->ffn_done, s) != cudaSuccess ||
+            cudaStreamWaitEvent(h->side_stream, h->ffn_done, 0) != cudaSuccess)
+          return STCA_ERR_CUDA;
+        for (int l = 1; l < c.M; ++l) {
+          CK(history_kv_fused(h, l, f.n_tok, h->side_stream, f.M_dev, KV_AHEAD_PAIRS));
+          if (cudaEventRecord(h->kv_done[l], h->side_stream) != cudaSuccess) return STCA_ERR_CUDA;
+        }
+        CK(history_kv_fused(h, 0, f.n_tok, s, f.M_dev));
+      }
+    } else if (!c.kv_fold) {
+      CK(history_kv_fused(h, i, f.n_tok, s, f.M_dev));  // the fold needs no K/V rows
+    }
   } else if (c.dtype == STCA_BF16) {
     if (i == 0) CK(history_hidden_bf16(h, 0, f.g, f.n_tok, s, f.M_dev));
     CK(history_kv_bf16(h, 0, i, f.n_tok, w->hist[i].gamma, w->hist[i].beta, s, f.M_dev));
@@ -742,6 +784,7 @@ int fwd_layer_inputs(stca_handle* h, int i, cudaStream_t s) {
   }
   STAGE(h, STCA_STAGE_QUERY, s,
         qgemm(gemm_args<TB>(f.t_tot, c.d, c.d, h->qbuf, c.d, w->WQ[i], h->qproj, c.d, h->err), qp(h, h->ql.wq[i]), s));
+  if (f.kv_ahead && i > 0 && cudaStreamWaitEvent(s, h->kv_done[i], 0) != cudaSuccess) return STCA_ERR_CUDA;
   if (c.kv_fold) {  // q~_{t,h} = Q_{t,h} W_K,h^T: [T, d] x block-diagonal -> [T, H d]
     const int Hd = c.H * c.d;
     STAGE(h, STCA_STAGE_QUERY, s,
@@ -843,12 +886,16 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
   const int64_t ldcat = int64_t(M + 1) * d;
   h->fwd.next_layer = -1;  // a whole forward closes any open sequence-parallel one
   CK(fwd_begin<TB>(h, ids, lens, dt, x_t, tpu, B, n_tok, t_tot, w, s));
+  if (c.dtype == STCA_BF16 && fused_ffn(c) && !c.kv_fold && M > 1) {
+    if (!make_side_stream(h)) return STCA_ERR_CUDA;
+    h->fwd.kv_ahead = true;
+  }
   const stca_handle::Fwd& f = h->fwd;
   for (int i = 0; i < M; ++i) {
     CK(fwd_layer_inputs<TB>(h, i, s));
     if (c.kv_fold) CK(run_attention_fold(h, i, s));
     else CK(run_attention(h, h->qproj, h->hoff, h->toff, B, t_tot, f.splits, c.score, s, f.kv_rows, f.kv_len,
-                          f.kv_mult));
+                          f.kv_mult, kv_ptr(h, i)));
     CK(fwd_layer_outputs<TB>(h, i, z_out, s));
   }
   if (o_out && t_tot > 0) {
@@ -980,6 +1027,12 @@ void stca_destroy(stca_handle* h) {
       cudaEventDestroy(h->z_free[b]);
     }
   }
+  if (h->side_stream) {
+    cudaStreamSynchronize(h->side_stream);
+    cudaStreamDestroy(h->side_stream);
+    cudaEventDestroy(h->ffn_done);
+    for (int l = 0; l < STCA_MAX_LAYERS; ++l) cudaEventDestroy(h->kv_done[l]);
+  }
   free_all(h);
   delete h;
 }
@@ -1110,7 +1163,7 @@ int stca_lsplit_partial(stca_handle* h, int layer, float* acc, float* ml, void* 
   CK(bf ? fwd_layer_inputs<bf16>(h, layer, s) : fwd_layer_inputs<float>(h, layer, s));
   AttnArgs a;
   a.Q = h->qproj;
-  a.KV = h->kv;
+  a.KV = kv_ptr(h, layer);
   a.hoff = h->hoff;
   a.toff = h->toff;
   a.kv_rows = f.kv_rows;

@@ -844,12 +844,14 @@ size_t rowwise_smem(int nb, int stages) {
 template <int AMODE, int EPI, int STAGES>
 int run_resident(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tx,
                  int store_x, const GatherSrc& g, int M, int K, int NT, int32_t* err, cudaStream_t s,
-                 const int32_t* M_dev, const EpiFold& fold) {
+                 const int32_t* M_dev, const EpiFold& fold, int max_pairs) {
   auto kern = tc_gemm_resident_kernel<AMODE, EPI, STAGES>;
   const size_t smem = resident_smem(K, STAGES, AMODE == A_GATHER);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
-  const int grid = 2 * std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
+  int pairs = std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
+  if (max_pairs > 0) pairs = std::min(pairs, max_pairs);
+  const int grid = 2 * pairs;
   launch_dep(kern, dim3(grid), dim3(512), smem, s, ta, tb, tc, tx, g, M, K, NT, store_x, err, M_dev, fold);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
@@ -919,7 +921,7 @@ int tc_pack_weights(const PackJob* jobs, int n, cudaStream_t s) {
 
 int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int K, const void* Wp, int Nout,
                      void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev, void* x_out,
-                     const EpiFold* fold) {
+                     const EpiFold* fold, int max_pairs) {
   if (M == 0) return 0;
   if (M < 0 || (K != 256 && K != 512) || Nout <= 0 || ldc % 8 != 0) return STCA_ERR_UNSUPPORTED;
   const int N = epi == EPI_SWIGLU ? 2 * Nout : Nout;
@@ -950,8 +952,8 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
   const int sx = x_out != nullptr;
   // stage counts fill the 227 KB of shared memory (see resident_smem)
 #define STCA_RES(AM, EP)                                                                                   \
-  (K == 512 ? run_resident<AM, EP, 5>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev, fo)     \
-            : run_resident<AM, EP, 9>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev, fo))
+  (K == 512 ? run_resident<AM, EP, 5>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev, fo, max_pairs)     \
+            : run_resident<AM, EP, 9>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev, fo, max_pairs))
   if (amode == A_TMA && epi == EPI_PLAIN) return STCA_RES(A_TMA, EPI_PLAIN);
   if (amode == A_TMA && epi == EPI_LNFOLD) return STCA_RES(A_TMA, EPI_LNFOLD);
   if (amode == A_TMA && epi == EPI_SWIGLU) return STCA_RES(A_TMA, EPI_SWIGLU);
