@@ -106,7 +106,7 @@ bool make_tmap_out(CUtensorMap* map, const void* base, uint64_t rows, uint64_t c
 // stats [layers layer_stride] float2.  layer_stride >= M, a multiple of 256.
 int tc_ffn_fused(const GatherSrc& g, int M, const int32_t* M_dev, int layers, int hidden, const void* W13p,
                  const void* W2p, const float* const* gammas, float eps, void* Y, int layer_stride, float* stats,
-                 int32_t* err, cudaStream_t s);
+                 int32_t* err, cudaStream_t s, int max_pairs = 0);
 
 // ---------------------------------------------------------------- SIMT fp32 GEMMs
 

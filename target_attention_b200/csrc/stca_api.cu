@@ -604,13 +604,13 @@ bool make_side_stream(stca_handle* h) {
 // d = 256: y'_l = (A_l W2_l) * gamma_l and the row moments of every layer in one fused
 // launch (the hidden activations A_l stay on chip).
 int history_ffn_fused(stca_handle* h, const GatherSrc& g, int n_tok, const stca_weights* w, cudaStream_t s,
-                      const int32_t* M_dev) {
+                      const int32_t* M_dev, int max_pairs = 0) {
   const stca_config& c = h->cfg;
   const float* gammas[STCA_MAX_LAYERS] = {};
   for (int l = 0; l < c.M; ++l) gammas[l] = w->hist[l].gamma;
   STAGE(h, STCA_STAGE_GATHER_FFN, s,
         tc_ffn_fused(g, n_tok, M_dev, c.M, c.hidden, wp13(h, 0), wp2(h, 0), gammas, c.ln_eps, h->xt,
-                     int(ffn_layer_stride(c)), h->rowstats, h->err, s));
+                     int(ffn_layer_stride(c)), h->rowstats, h->err, s, max_pairs));
   return STCA_OK;
 }
 
@@ -629,8 +629,8 @@ int history_kv_fused(stca_handle* h, int l, int n_tok, cudaStream_t s, const int
   return STCA_OK;
 }
 
-// SM pairs the K/V GEMMs that run ahead on the side stream may use: the rest stay free for
-// the latency-bound attention and target-side kernels of the current layer.
+// SM pairs the history-side GEMMs on the side stream may use: the rest stay free for the
+// latency-bound target-side and attention kernels running beside them.
 constexpr int KV_AHEAD_PAIRS = 64;
 
 // K/V of every history token for one layer: fp32 SIMT path.
@@ -688,7 +688,8 @@ int run_attention(stca_handle* h, const float* Q, const int32_t* hoff, const int
 // converted (unless pinned), q^(1) = LN(SwiGLU_t(x_t)), distinct keys; fills h->fwd.
 template <typename TB>
 int fwd_begin(stca_handle* h, const int32_t* ids, const int32_t* lens, const int32_t* dt, const void* x_t,
-              const int32_t* tpu, int B, int n_tok, int t_tot, const stca_weights* w, cudaStream_t s) {
+              const int32_t* tpu, int B, int n_tok, int t_tot, const stca_weights* w, cudaStream_t s,
+              bool ahead = false) {
   const stca_config& c = h->cfg;
   const int d = c.d, M = c.M;
   const bool bf = c.dtype == STCA_BF16;
@@ -705,6 +706,14 @@ int fwd_begin(stca_handle* h, const int32_t* ids, const int32_t* lens, const int
       CK(stca_folds(h, w, s));
     }
   }
+  // `ahead`: the history side (distinct keys, FFN, every layer's K/V) runs on the side
+  // stream from here, beside the target side on the caller's stream
+  cudaStream_t hs = s;
+  if (ahead) {
+    if (cudaEventRecord(h->ffn_done, s) != cudaSuccess || cudaStreamWaitEvent(h->side_stream, h->ffn_done, 0) != cudaSuccess)
+      return STCA_ERR_CUDA;
+    hs = h->side_stream;
+  }
   const stca_handle::QLayout& L = h->ql;
   const float* xcol = h->cat + int64_t(M) * d;
   // q^(1) = LN(SwiGLU_t(x_t))
@@ -712,6 +721,7 @@ int fwd_begin(stca_handle* h, const int32_t* ids, const int32_t* lens, const int
         query_ffn<TB>(h, xcol, ldcat, t_tot, w->tgt, h->qbuf, d, s, qp(h, L.tgt13), qp(h, L.tgt2)));
   stca_handle::Fwd& f = h->fwd;
   f = stca_handle::Fwd{};
+  f.kv_ahead = ahead;
   f.B = B;
   f.n_tok = n_tok;
   f.t_tot = t_tot;
@@ -725,16 +735,16 @@ int fwd_begin(stca_handle* h, const int32_t* ids, const int32_t* lens, const int
     // distinct keys of the call and (dedup = 2) each user's compacted rows, one launch
     const bool compact = c.dedup == 2;
     if (n_tok <= FUSED_DEDUP_MAX_TOKENS) {
-      STAGE(h, STCA_STAGE_DEDUP, s,
+      STAGE(h, STCA_STAGE_DEDUP, hs,
             dedup_fused(ids, f.g.dt, n_tok, h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx, h->uniq_token,
-                        h->uniq_count, compact ? h->hoff : nullptr, B, h->c_rows, h->c_mult, h->c_len, h->err, s));
+                        h->uniq_count, compact ? h->hoff : nullptr, B, h->c_rows, h->c_mult, h->c_len, h->err, hs));
     } else {
-      STAGE(h, STCA_STAGE_DEDUP, s,
+      STAGE(h, STCA_STAGE_DEDUP, hs,
             dedup_rows(ids, f.g.dt, n_tok, h->dedup_ws, h->dedup_ws_bytes, h->uniq_idx, h->uniq_token,
-                       h->uniq_count, h->err, s));
+                       h->uniq_count, h->err, hs));
       if (compact)
-        STAGE(h, STCA_STAGE_DEDUP, s,
-              compact_user_rows(h->hoff, B, h->uniq_idx, h->c_rows, h->c_mult, h->c_len, s));
+        STAGE(h, STCA_STAGE_DEDUP, hs,
+              compact_user_rows(h->hoff, B, h->uniq_idx, h->c_rows, h->c_mult, h->c_len, hs));
     }
     f.g.rows = h->uniq_token;
     f.M_dev = h->uniq_count;
@@ -759,22 +769,20 @@ int fwd_layer_inputs(stca_handle* h, int i, cudaStream_t s) {
   const stca_handle::Fwd& f = h->fwd;
   const stca_weights* w = f.w;
   if (c.dtype == STCA_BF16 && fused_ffn(c)) {
-    if (i == 0) CK(history_ffn_fused(h, f.g, f.n_tok, w, s, f.M_dev));
-    if (!c.kv_fold && f.kv_ahead) {
-      // every layer's K/V depends only on the fused FFN: layers >= 1 go to the side stream
-      // now and run beside this layer's attention and target side
+    if (f.kv_ahead) {
+      // the history side on the side stream: the fused FFN, then every layer's K/V (each
+      // depends only on the FFN), each marked by its event; grids capped so that SMs stay
+      // free for the target side running beside them
       if (i == 0) {
-        if (cudaEventRecord(h->ffn_done, s) != cudaSuccess ||
-            cudaStreamWaitEvent(h->side_stream, h->ffn_done, 0) != cudaSuccess)
-          return STCA_ERR_CUDA;
-        for (int l = 1; l < c.M; ++l) {
+        CK(history_ffn_fused(h, f.g, f.n_tok, w, h->side_stream, f.M_dev, KV_AHEAD_PAIRS));
+        for (int l = 0; l < c.M; ++l) {
           CK(history_kv_fused(h, l, f.n_tok, h->side_stream, f.M_dev, KV_AHEAD_PAIRS));
           if (cudaEventRecord(h->kv_done[l], h->side_stream) != cudaSuccess) return STCA_ERR_CUDA;
         }
-        CK(history_kv_fused(h, 0, f.n_tok, s, f.M_dev));
       }
-    } else if (!c.kv_fold) {
-      CK(history_kv_fused(h, i, f.n_tok, s, f.M_dev));  // the fold needs no K/V rows
+    } else {
+      if (i == 0) CK(history_ffn_fused(h, f.g, f.n_tok, w, s, f.M_dev));
+      if (!c.kv_fold) CK(history_kv_fused(h, i, f.n_tok, s, f.M_dev));  // the fold needs no K/V rows
     }
   } else if (c.dtype == STCA_BF16) {
     if (i == 0) CK(history_hidden_bf16(h, 0, f.g, f.n_tok, s, f.M_dev));
@@ -784,7 +792,7 @@ int fwd_layer_inputs(stca_handle* h, int i, cudaStream_t s) {
   }
   STAGE(h, STCA_STAGE_QUERY, s,
         qgemm(gemm_args<TB>(f.t_tot, c.d, c.d, h->qbuf, c.d, w->WQ[i], h->qproj, c.d, h->err), qp(h, h->ql.wq[i]), s));
-  if (f.kv_ahead && i > 0 && cudaStreamWaitEvent(s, h->kv_done[i], 0) != cudaSuccess) return STCA_ERR_CUDA;
+  if (f.kv_ahead && cudaStreamWaitEvent(s, h->kv_done[i], 0) != cudaSuccess) return STCA_ERR_CUDA;
   if (c.kv_fold) {  // q~_{t,h} = Q_{t,h} W_K,h^T: [T, d] x block-diagonal -> [T, H d]
     const int Hd = c.H * c.d;
     STAGE(h, STCA_STAGE_QUERY, s,
@@ -885,11 +893,9 @@ int run_stca(stca_handle* h, const int32_t* ids, const int32_t* lens, const int3
   const int d = c.d, M = c.M;
   const int64_t ldcat = int64_t(M + 1) * d;
   h->fwd.next_layer = -1;  // a whole forward closes any open sequence-parallel one
-  CK(fwd_begin<TB>(h, ids, lens, dt, x_t, tpu, B, n_tok, t_tot, w, s));
-  if (c.dtype == STCA_BF16 && fused_ffn(c) && !c.kv_fold && M > 1) {
-    if (!make_side_stream(h)) return STCA_ERR_CUDA;
-    h->fwd.kv_ahead = true;
-  }
+  const bool ahead = c.dtype == STCA_BF16 && fused_ffn(c) && !c.kv_fold;
+  if (ahead && !make_side_stream(h)) return STCA_ERR_CUDA;
+  CK(fwd_begin<TB>(h, ids, lens, dt, x_t, tpu, B, n_tok, t_tot, w, s, ahead));
   const stca_handle::Fwd& f = h->fwd;
   for (int i = 0; i < M; ++i) {
     CK(fwd_layer_inputs<TB>(h, i, s));

@@ -445,7 +445,7 @@ size_t ffn_smem() {
 
 int tc_ffn_fused(const GatherSrc& g, int M, const int32_t* M_dev, int layers, int hidden, const void* W13p,
                  const void* W2p, const float* const* gammas, float eps, void* Y, int layer_stride, float* stats,
-                 int32_t* err, cudaStream_t s) {
+                 int32_t* err, cudaStream_t s, int max_pairs) {
   if (M == 0) return 0;
   if (M < 0 || layers < 1 || layers > STCA_MAX_LAYERS || hidden < F_HCH || hidden % F_HCH != 0 ||
       layer_stride < M || layer_stride % (2 * BM) != 0 || !W13p || !W2p || !Y || !stats || !gammas ||
@@ -466,7 +466,9 @@ int tc_ffn_fused(const GatherSrc& g, int M, const int32_t* M_dev, int layers, in
   const size_t smem = ffn_smem();
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return STCA_ERR_CUDA;
-  const int grid = 2 * std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
+  int pairs = std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
+  if (max_pairs > 0) pairs = std::min(pairs, max_pairs);
+  const int grid = 2 * pairs;
   launch_dep(kern, dim3(grid), dim3(512), smem, s, t13, t2, ty, g, M, layers, hidden, layer_stride, gam, eps, stats,
              err, M_dev);
   note_launch();
