@@ -215,7 +215,8 @@ int stca_lsplit_merge(stca_handle* h, int layer, int ranks, const float* all_acc
  * never written.  Handle: dtype STCA_BF16, d = D = 128 (the only width in this build),
  * max_users >= B, max_tokens >= n_tok.
  *   ids [n_tok] int32, lengths [B] int32, q [B, D] bf16, table [n_items, D] bf16,
- *   out [B, D] float32. */
+ *   out [B, D] float32.  q and table start on 16-byte boundaries (rows are moved by
+ *   16-byte copies), else STCA_ERR_INVALID_ARG with nothing launched. */
 int stca_pointwise_forward(stca_handle* h, const int32_t* ids, const int32_t* lengths, const void* q,
                            const void* table, int64_t n_items, int B, int n_tok, float* out,
                            void* stream);

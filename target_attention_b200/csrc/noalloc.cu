@@ -107,6 +107,7 @@ extern "C" int stca_pointwise_forward_noalloc(const int32_t* ids, const int32_t*
   if (B > NOALLOC_MAX_USERS) return STCA_ERR_CAPACITY;
   if (B > 0 && (!lengths || !q || !table || !out)) return STCA_ERR_INVALID_ARG;
   if (n_tok > 0 && !ids) return STCA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(table)) & 15) return STCA_ERR_INVALID_ARG;
   if (B == 0) return STCA_OK;
   NoallocScratch* sc = scratch_on_current_device();
   if (!sc) return STCA_ERR_CUDA;

@@ -1243,6 +1243,7 @@ int stca_pointwise_forward(stca_handle* h, const int32_t* ids, const int32_t* le
   if (B > h->cfg.max_users || n_tok > h->cfg.max_tokens) return STCA_ERR_CAPACITY;
   if (B > 0 && (!lengths || !q || !table || !out)) return STCA_ERR_INVALID_ARG;
   if (n_tok > 0 && !ids) return STCA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(table)) & 15) return STCA_ERR_INVALID_ARG;
   if (cudaSetDevice(h->device) != cudaSuccess) return STCA_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   h->last_stream = s;

@@ -88,6 +88,9 @@ def test_null_arguments_rejected_on_host():
     assert L.stca_forward(None, None, None, None, None, None, 1, 1, 1, ctypes.byref(w), None, None, None) \
         == B.ERR_INVALID_ARG
     assert L.stca_pointwise_forward(None, None, None, None, None, 1, 1, 1, None, None) == B.ERR_INVALID_ARG
+    # rows move by 16-byte-aligned copies: q or table off a 16-byte boundary is refused first
+    assert L.stca_pointwise_forward_noalloc(None, 16, 24, 16, 100, 1, 0, 16, None, None) == B.ERR_INVALID_ARG
+    assert L.stca_pointwise_forward_noalloc(None, 16, 16, 40, 100, 1, 0, 16, None, None) == B.ERR_INVALID_ARG
     assert L.stca_sync_status(None) == B.ERR_INVALID_ARG
     assert L.stca_pin_weights(None, None, None) == B.ERR_INVALID_ARG
     assert L.stca_lsplit_begin(None, None, None, None, None, None, 1, 1, 1, ctypes.byref(w), None) \

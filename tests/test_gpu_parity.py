@@ -268,6 +268,31 @@ def test_pointwise_empty_rows():
     assert R.row_rel_err(got, R.pointwise_relu_ta(wl)) <= 1e-4
 
 
+def test_pointwise_ragged_extremes():
+    """Ragged extremes in one batch: one sample 20K rows long (cut into several slices),
+    runs of empty samples, samples shorter than a ring stage and samples ending exactly on
+    a stage boundary."""
+    lengths = np.array([0, 1, 0, 0, 127, 128, 129, 20_000, 3, 0, 0, 0, 5000, 0, 256, 1], np.int32)
+    wl = make_pointwise(users=len(lengths), L=10, L_lo=1, n_items=30_000, lengths=lengths, seed=17)
+    got = _run_pointwise(wl)
+    for b in np.flatnonzero(lengths == 0):
+        assert (got[b] == 0).all()
+    e = R.row_rel_err(got, R.pointwise_relu_ta(wl))
+    print(f"parity pointwise (ragged extremes) row-relative error {e:.3e}")
+    assert e <= 1e-4
+
+
+def test_pointwise_all_histories_empty():
+    wl = make_pointwise(users=3, L=10, L_lo=1, n_items=100, lengths=np.zeros(3, np.int32))
+    m = PointwiseModel(wl, max_tokens=1)
+    x = m.inputs(wl)
+    out = torch.full((3, 128), float("nan"), device=dev)
+    B.check(m.forward(x, out))
+    assert B.stca_sync_status(m.handle) == B.OK
+    m.close()
+    assert (out.cpu().numpy() == 0).all()
+
+
 # ---------------------------------------------------------------- multi-sequence decode
 
 
