@@ -88,6 +88,19 @@ int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t*
                      int T, int d, int H, int splits, int score, float* part_acc, float* part_ml, float* out,
                      int32_t* err, void* stream);
 
+/* The same attention over gathered, weighted keys (the form the library runs with
+ * per-user compaction, [hyformer] §3.8.1 pooling of repeated keys): user u's keys are the
+ * entries n = hoff[u] .. hoff[u] + len_u - 1 of kv_rows, len_u = kv_len[u] (NULL:
+ * hoff[u+1] - hoff[u]); entry n is K/V row kv_rows[n] of KV and weighs kv_mult[n] tokens
+ * (NULL: 1), which equals repeating that key kv_mult[n] times.  kv_rows [hoff[B]] int32
+ * (required, each in [0, rows of KV): the caller's promise, not checked), kv_len [B],
+ * kv_mult [hoff[B]] int32 (>= 1), device memory.  bf16 K/V only (kv_bf16 = 0 returns
+ * STCA_ERR_UNSUPPORTED when kv_len or kv_mult is given); other arguments as above. */
+int stca_k_attention_rows(int kv_bf16, const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff,
+                          const int32_t* kv_rows, const int32_t* kv_len, const int32_t* kv_mult, int B, int T, int d,
+                          int H, int splits, int score, float* part_acc, float* part_ml, float* out, int32_t* err,
+                          void* stream);
+
 /* Distinct history keys (HyFormer page §3.8.1, GPU pooling): key(n) = (ids[n], bucket(dt[n]))
  * (bucket 0 when dt is NULL).  Writes uniq_idx[n] in [0, *count) with equal keys mapped to
  * the same index and distinct keys to distinct indices, and uniq_token[u] = a token whose

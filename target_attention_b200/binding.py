@@ -108,6 +108,8 @@ _SIGS = [
     ("stca_k_gemm_rowwise", _i32, [_i32, _vp, _i32, _i32, _vp, _i32, _vp, _vp, ctypes.c_float, _vp, _i32, _vp, _vp]),
     ("stca_k_attention", _i32, [_i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
                                 _vp]),
+    ("stca_k_attention_rows", _i32, [_i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+                                     _vp, _vp, _vp, _vp, _vp]),
     ("stca_k_dedup_workspace_bytes", ctypes.c_size_t, [_i32]),
     ("stca_k_dedup", _i32, [_vp, _vp, _i32, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]),
     ("stca_k_compact_user_rows", _i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp]),
@@ -323,6 +325,13 @@ def stca_k_attention(kv_bf16, Q, KV, hoff, toff, B, T, d, H, splits, score, part
                      stream=None) -> int:
     return lib().stca_k_attention(kv_bf16, ptr(Q), ptr(KV), ptr(hoff), ptr(toff), B, T, d, H, splits, score,
                                   ptr(part_acc), ptr(part_ml), ptr(out), ptr(err), stream_ptr(stream))
+
+
+def stca_k_attention_rows(kv_bf16, Q, KV, hoff, toff, kv_rows, kv_len, kv_mult, B, T, d, H, splits, score, part_acc,
+                          part_ml, out, err, stream=None) -> int:
+    return lib().stca_k_attention_rows(kv_bf16, ptr(Q), ptr(KV), ptr(hoff), ptr(toff), ptr(kv_rows), ptr(kv_len),
+                                       ptr(kv_mult), B, T, d, H, splits, score, ptr(part_acc), ptr(part_ml), ptr(out),
+                                       ptr(err), stream_ptr(stream))
 
 
 def stca_k_dedup_workspace_bytes(n) -> int:

@@ -139,29 +139,38 @@ __device__ __forceinline__ void tile_step(uint32_t sK, uint32_t sV, const float*
   }
   // scores -> weights
   if (SCORE == 0) {
+    // The reference point m of a row moves only when a score exceeds it by more than
+    // RESCALE_SLACK (log2 units): weights 2^(s - m) then stay <= 2^RESCALE_SLACK, exact in
+    // fp32, and the state is rescaled rarely.  Each thread checks its own scores against m;
+    // only when one of the warp's scores is above m + RESCALE_SLACK are the row maxima
+    // gathered across the four threads of each row (shuffles) and the rows that moved
+    // rescaled.  Numerator and denominator share m, so the quotient is unchanged.
+    float mx[2];
 #pragma unroll
     for (int hr = 0; hr < 2; ++hr) {
-      float mx = -INFINITY;
+      mx[hr] = -INFINITY;
 #pragma unroll
-      for (int jj = 0; jj < NJ; ++jj) mx = fmaxf(mx, fmaxf(sacc[jj][2 * hr], sacc[jj][2 * hr + 1]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      // The reference point of a row moves only when a score exceeds it by more than
-      // RESCALE_SLACK (log2 units): weights 2^(s - m) then stay <= 2^RESCALE_SLACK, exact in
-      // fp32, and the state is rescaled rarely (skipped when no row of the warp moves).
-      // Numerator and denominator share m, so the quotient is unchanged.
-      const bool move = mx > mrow[hr] + RESCALE_SLACK;
-      if (__any_sync(0xffffffffu, move)) {
-        const float mnew = move ? mx : mrow[hr];
-        const float corr = (mnew == mrow[hr]) ? 1.f : exp2_approx(mrow[hr] - mnew);
-        mrow[hr] = mnew;
-        lrow[hr] *= corr;
+      for (int jj = 0; jj < NJ; ++jj) mx[hr] = fmaxf(mx[hr], fmaxf(sacc[jj][2 * hr], sacc[jj][2 * hr + 1]));
+    }
+    if (__any_sync(0xffffffffu, mx[0] > mrow[0] + RESCALE_SLACK || mx[1] > mrow[1] + RESCALE_SLACK)) {
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          o[nt][2 * hr] *= corr;
-          o[nt][2 * hr + 1] *= corr;
+      for (int hr = 0; hr < 2; ++hr) {
+        float rm = fmaxf(mx[hr], __shfl_xor_sync(0xffffffffu, mx[hr], 1));
+        rm = fmaxf(rm, __shfl_xor_sync(0xffffffffu, rm, 2));
+        if (rm > mrow[hr] + RESCALE_SLACK) {
+          const float corr = exp2_approx(mrow[hr] - rm);  // 0 while m was -inf
+          mrow[hr] = rm;
+          lrow[hr] *= corr;
+#pragma unroll
+          for (int nt = 0; nt < 8; ++nt) {
+            o[nt][2 * hr] *= corr;
+            o[nt][2 * hr + 1] *= corr;
+          }
         }
       }
+    }
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
       const float muse = (mrow[hr] == -INFINITY) ? 0.f : mrow[hr];
       float sum = 0.f;
 #pragma unroll

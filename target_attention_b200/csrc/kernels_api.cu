@@ -113,20 +113,23 @@ int stca_k_gemm_rowwise(int epi, const void* A, int M, int K, const void* Wp, in
   return tc_gemm_rowwise(epi, A, M, K, Wp, N, gamma, beta, eps, C, ldc, err, reinterpret_cast<cudaStream_t>(stream));
 }
 
-int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B,
-                     int T, int d, int H, int splits, int score, float* part_acc, float* part_ml, float* out,
-                     int32_t* err, void* stream) {
+int stca_k_attention_rows(int kv_bf16, const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff,
+                          const int32_t* kv_rows, const int32_t* kv_len, const int32_t* kv_mult, int B, int T, int d,
+                          int H, int splits, int score, float* part_acc, float* part_ml, float* out, int32_t* err,
+                          void* stream) {
   if (B < 0 || T < 0 || d <= 0 || H <= 0 || d % H != 0 || splits < 1 || splits > 32 || (score != 0 && score != 1))
     return STCA_ERR_INVALID_ARG;
   if (B > 0 && T > 0 && (!Q || !KV || !hoff || !toff || !part_acc || !part_ml || !out)) return STCA_ERR_INVALID_ARG;
+  if (!kv_rows && (kv_len || kv_mult)) return STCA_ERR_INVALID_ARG;
+  if (!kv_bf16 && (kv_len || kv_mult)) return STCA_ERR_UNSUPPORTED;
   AttnArgs a;
   a.Q = Q;
   a.KV = KV;
   a.hoff = hoff;
   a.toff = toff;
-  a.kv_rows = nullptr;
-  a.kv_len = nullptr;
-  a.kv_mult = nullptr;
+  a.kv_rows = kv_rows;
+  a.kv_len = kv_len;
+  a.kv_mult = kv_mult;
   a.B = B;
   a.T = T;
   a.d = d;
@@ -141,6 +144,13 @@ int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t*
   const int rc = kv_bf16 ? attention_bf16(a, s) : attention_f32(a, s);
   if (rc != STCA_OK) return rc;
   return attention_needs_merge(a, kv_bf16 != 0) ? attention_merge(a, s) : STCA_OK;
+}
+
+int stca_k_attention(int kv_bf16, const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B,
+                     int T, int d, int H, int splits, int score, float* part_acc, float* part_ml, float* out,
+                     int32_t* err, void* stream) {
+  return stca_k_attention_rows(kv_bf16, Q, KV, hoff, toff, nullptr, nullptr, nullptr, B, T, d, H, splits, score,
+                               part_acc, part_ml, out, err, stream);
 }
 
 size_t stca_k_dedup_workspace_bytes(int n) { return n < 0 ? 0 : dedup_workspace_bytes(n); }

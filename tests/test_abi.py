@@ -105,6 +105,10 @@ def test_null_arguments_rejected_on_host():
     # kernel-level entry points validate before launching
     assert L.stca_k_attention(1, None, None, None, None, 1, 1, 256, 3, 1, 0, None, None, None, None, None) \
         == B.ERR_INVALID_ARG
+    assert L.stca_k_attention_rows(1, 16, 16, 16, 16, None, 16, None, 1, 1, 64, 1, 1, 0, 16, 16, 16, None, None) \
+        == B.ERR_INVALID_ARG                          # key lengths or weights without key rows
+    assert L.stca_k_attention_rows(0, 16, 16, 16, 16, 16, None, 16, 1, 1, 64, 1, 1, 0, 16, 16, 16, None, None) \
+        == B.ERR_UNSUPPORTED                          # key weights with fp32 K/V
     assert L.stca_k_pack_weight(None, 4, 4, None, 0, 0, None) == B.ERR_INVALID_ARG
     assert L.stca_k_gemm_resident(1, 1, None, None, None, None, None, 0, 5, 256, None, 128, None, 128, None, None,
                                   None) == B.ERR_INVALID_ARG

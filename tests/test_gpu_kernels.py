@@ -373,6 +373,53 @@ def test_attention_bf16(score, splits):
 
 
 @pytest.mark.parametrize("score", [0, 1])
+@pytest.mark.parametrize("splits", [1, 3])
+def test_attention_bf16_gathered_weighted_keys(score, splits):
+    """Keys gathered by row index with multiplicities (the compacted form): a key that
+    stands for c tokens must act like c copies of itself.  Each user's slot range is longer
+    than its key count (kv_len < allotted), rows repeat across users, and the reference
+    expands every key into its copies."""
+    g = _rng(13 + score)
+    d, H, dh, U = 256, 4, 64, 3000
+    lengths = np.array([0, 1, 33, 700, 2049, 5], np.int32)     # keys per user
+    slack = np.array([3, 0, 7, 1, 0, 2], np.int32)             # unused slots after them
+    targets = np.array([2, 1, 17, 33, 40, 3], np.int32)
+    hoff = R.exclusive_offsets(lengths + slack)
+    toff = R.exclusive_offsets(targets)
+    n_slots, T = int(hoff[-1]), int(toff[-1])
+    rows = g.integers(0, U, size=n_slots).astype(np.int32)
+    mult = g.integers(1, 6, size=n_slots).astype(np.int32)
+    KVt = _bf16(g.standard_normal((U, 2 * d)))
+    KV64 = bf16_to_f64(KVt)
+    Q = g.standard_normal((T, d)).astype(np.float32)
+    part_acc = torch.empty((splits, T, d), dtype=torch.float32, device=dev)
+    part_ml = torch.empty((splits, T, H, 2), dtype=torch.float32, device=dev)
+    out = torch.full((T, d), float("nan"), dtype=torch.float32, device=dev)
+    err = zeros_err()
+    i32 = lambda x: torch.from_numpy(np.ascontiguousarray(x, np.int32)).to(dev)
+    B.check(B.stca_k_attention_rows(1, torch.from_numpy(Q).to(dev), KVt, i32(hoff), i32(toff), i32(rows),
+                                    i32(lengths), i32(mult), len(lengths), T, d, H, splits, score, part_acc, part_ml,
+                                    out, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    got = out.cpu().numpy()
+    ref = np.zeros((T, d))
+    for u in range(len(lengths)):
+        ent = slice(hoff[u], hoff[u] + lengths[u])
+        expanded = KV64[np.repeat(rows[ent], mult[ent])]
+        for t in range(toff[u], toff[u + 1]):
+            for h in range(H):
+                K_h, V_h = expanded[:, 2 * h * dh:(2 * h + 1) * dh], expanded[:, (2 * h + 1) * dh:(2 * h + 2) * dh]
+                cols = slice(h * dh, (h + 1) * dh)
+                ref[t, cols] = R.head_attention(Q[t, cols].astype(np.float64), K_h, V_h,
+                                                "softmax" if score == 0 else "relu", 1 / math.sqrt(dh))
+    e = R.row_rel_err(got.reshape(-1, dh), ref.reshape(-1, dh))
+    print(f"gathered weighted keys: row-relative error {e:.2e}")
+    assert e <= 2e-2, e
+    assert (got[:2] == 0).all()
+
+
+@pytest.mark.parametrize("score", [0, 1])
 def test_attention_f32(score):
     lengths = [0, 1, 9, 600]
     targets = [1, 3, 4, 4]
