@@ -61,6 +61,10 @@ def parse():
                     help="control run: history ids uniform over the table instead of Zipf")
     ap.add_argument("--kv-fold", action="store_true",
                     help="fold W_K / W_V into the queries (d = 256 STCA workloads only)")
+    ap.add_argument("--probe", choices=["attention"], default=None,
+                    help="instead of the step: time one kernel alone on the workload's shapes and print "
+                         "one JSON line per input form (attention: contiguous keys, and the compacted "
+                         "per-user key lists of the workload's ids, through the kernel-level entries)")
     return ap.parse_args()
 
 
@@ -728,9 +732,108 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def compacted_keys(ids, dt, lengths):
+    """Each user's distinct (item id, time bucket) keys, numbered over the whole call, in
+    order of first token with their token counts: the key lists the library's per-user
+    compaction gives the attention.  Returns (rows, counts, per-user count, distinct keys)."""
+    import numpy as np
+    keys = _row_keys(ids, dt)
+    uniq, inv = np.unique(keys, return_inverse=True)
+    rows, mult, lens = [], [], []
+    off = 0
+    for L in np.asarray(lengths, np.int64):
+        seg = inv[off:off + L]
+        off += L
+        vals, first, cnt = np.unique(seg, return_index=True, return_counts=True)
+        order = np.argsort(first)
+        rows.append(vals[order]), mult.append(cnt[order]), lens.append(len(vals))
+    cat = lambda xs: np.concatenate(xs).astype(np.int32) if xs else np.zeros(0, np.int32)
+    return cat(rows), cat(mult), np.asarray(lens, np.int32), len(uniq)
+
+
+def run_probe_attention(args):
+    """The split-L attention kernel alone on config 3's shapes (d = 512, H = 8, m = 32):
+    one layer's keys, K/V and queries random (the kernel's time does not depend on their
+    values beyond the rare rescales), timed with CUDA events around each launch after
+    warm-up; the median of 3 x steps launches.  "contiguous": every user's keys are its own
+    consecutive K/V rows; "compacted": the per-user distinct keys of the workload's ids,
+    gathered by row from the call's distinct-key K/V matrix and weighted by their counts."""
+    import statistics
+    import numpy as np
+    import torch
+    from target_attention_b200 import binding as B
+    from workloads import STCA_CONFIGS, make_stca_history
+    c = STCA_CONFIGS[3]
+    over = {"id_dist": "uniform"} if args.uniform_ids else {}
+    hist = make_stca_history(3, users=args.users, L=args.length, n_items=args.n_items, data_seed=rank_data_seed(3, 0),
+                             **over)
+    d, H, m = c["d"], c["H"], c["m"]
+    lengths = hist["lengths"]
+    Bu = len(lengths)
+    rows, mult, lens, U = compacted_keys(hist["ids"], hist["dt"], lengths)
+    hoff = np.zeros(Bu + 1, np.int64)
+    hoff[1:] = np.cumsum(lengths)
+    # the compacted lists sit at each user's token offset, as the library lays them out
+    slot_rows = np.zeros(int(hoff[-1]), np.int32)
+    slot_mult = np.ones(int(hoff[-1]), np.int32)
+    o = 0
+    for u in range(Bu):
+        slot_rows[hoff[u]:hoff[u] + lens[u]] = rows[o:o + lens[u]]
+        slot_mult[hoff[u]:hoff[u] + lens[u]] = mult[o:o + lens[u]]
+        o += lens[u]
+    n_att = int(lens.sum())
+    T = Bu * m
+    dev = "cuda"
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    i32 = lambda x: torch.from_numpy(np.ascontiguousarray(x, np.int32)).to(dev)
+    KVu = (torch.randn((U, 2 * d), device=dev, generator=g) * 0.5).to(torch.bfloat16)
+    KVc = (torch.randn((n_att, 2 * d), device=dev, generator=g) * 0.5).to(torch.bfloat16)
+    Q = torch.randn((T, d), device=dev, generator=g)
+    hoff_t, toff_t = i32(hoff), i32(np.arange(0, T + 1, m))
+    hoff_c = i32(np.concatenate([[0], np.cumsum(lens)]))
+    rows_t, mult_t, lens_t = i32(slot_rows), i32(slot_mult), i32(lens)
+    pa = torch.empty((1, T, d), device=dev)
+    pm = torch.empty((1, T, H, 2), device=dev)
+    out = torch.empty((T, d), device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    modes = {
+        "contiguous": lambda: B.stca_k_attention(1, Q, KVc, hoff_c, toff_t, Bu, T, d, H, 1, 0, pa, pm, out, err),
+        "compacted": lambda: B.stca_k_attention_rows(1, Q, KVu, hoff_t, toff_t, rows_t, lens_t, mult_t, Bu, T, d, H,
+                                                     1, 0, pa, pm, out, err),
+    }
+    peaks = load_peaks()
+    times = {k: [] for k in modes}
+    for _ in range(3):
+        for k, f in modes.items():
+            for _ in range(max(args.warmup, 1)):
+                B.check(f())
+            torch.cuda.synchronize()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for e0, e1 in ev:
+                e0.record()
+                B.check(f())
+                e1.record()
+            torch.cuda.synchronize()
+            times[k] += [e0.elapsed_time(e1) for e0, e1 in ev]
+    assert int(err.item()) == 0
+    work = n_att * H * 4 * (d // H) + 2 * T * d * 4  # attended K/V segments + queries and outputs
+    for k in modes:
+        ms = statistics.median(times[k])
+        gbs = work / ms / 1e6
+        print(json.dumps({"probe": "attention", "mode": k, "users": Bu, "attended_keys": n_att,
+                          "distinct_keys": int(U), "ids": "uniform" if args.uniform_ids else "zipf",
+                          "median_ms": round(ms, 4), "launches": len(times[k]), "work_bytes": work,
+                          "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm_gbs"],
+                          "frac": round(gbs / peaks["hbm_gbs"], 4)}), flush=True)
+
+
 if __name__ == "__main__":
     a = parse()
-    if a.impl == "reference":
+    if a.probe == "attention":
+        run_probe_attention(a)
+    elif a.impl == "reference":
         run_reference(a)
     else:
         run_ours(a)

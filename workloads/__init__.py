@@ -10,4 +10,5 @@ from .generate import (  # noqa: F401
     make_hyformer,
     make_pointwise,
     make_stca,
+    make_stca_history,
 )

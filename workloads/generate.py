@@ -138,6 +138,39 @@ def _ffn(g, d, hidden, dtype, affine=None, ln=True):
     return f
 
 
+def _stca_streams(config_id, seed, data_seed):
+    ss = np.random.SeedSequence(1000 + config_id if seed is None else seed)
+    streams = list(ss.spawn(7))  # lengths, ids, dt, x_t, table, dt table, weights
+    if data_seed is not None:
+        streams[:4] = np.random.SeedSequence(data_seed).spawn(4)
+    return streams
+
+
+def _stca_history(cfg, lengths, s_len, s_ids, s_dt):
+    if lengths is None:
+        lengths = _lengths(_rng(s_len), cfg, cfg["users"])
+    lengths = np.asarray(lengths, dtype=np.int32)
+    n_tok = int(lengths.sum())
+    ids = _ids(_rng(s_ids), n_tok, cfg)
+    dt = None
+    if cfg["time_buckets"]:
+        # seconds since the interaction: floor(2^U[0,16)) - 1
+        e = _rng(s_dt).uniform(0.0, 16.0, size=n_tok)
+        dt = (np.floor(np.exp2(e)) - 1).astype(np.int32)
+    return lengths, ids, dt
+
+
+def make_stca_history(config_id: int, *, users=None, L=None, n_items=None, seed=None, data_seed=None,
+                      **over) -> dict:
+    """The history side of ``make_stca`` alone (lengths, ids, dt: the same draws), without
+    the table, targets and weights, for probes that only need the key lists."""
+    cfg = _config(config_id, users=users, L=L, n_items=n_items, **over)
+    assert cfg["kind"] == "stca"
+    s_len, s_ids, s_dt = _stca_streams(config_id, seed, data_seed)[:3]
+    lengths, ids, dt = _stca_history(cfg, None, s_len, s_ids, s_dt)
+    return dict(cfg=cfg, lengths=lengths, ids=ids, dt=dt)
+
+
 def make_stca(config_id: int, *, users=None, L=None, n_items=None, m=None, lengths=None,
               seed=None, data_seed=None, ln_affine="random", **over) -> dict:
     """Inputs and random-init weights for an STCA workload (configs 1-3 and variants).
@@ -148,23 +181,10 @@ def make_stca(config_id: int, *, users=None, L=None, n_items=None, m=None, lengt
     """
     cfg = _config(config_id, users=users, L=L, n_items=n_items, m=m, **over)
     assert cfg["kind"] == "stca"
-    ss = np.random.SeedSequence(1000 + config_id if seed is None else seed)
-    s_len, s_ids, s_dt, s_xt, s_tab, s_dtab, s_w = ss.spawn(7)
-    if data_seed is not None:
-        s_len, s_ids, s_dt, s_xt = np.random.SeedSequence(data_seed).spawn(4)
+    s_len, s_ids, s_dt, s_xt, s_tab, s_dtab, s_w = _stca_streams(config_id, seed, data_seed)
     dtype, d, hidden, M = cfg["dtype"], cfg["d"], cfg["hidden"], cfg["M"]
-    B = cfg["users"]
-    if lengths is None:
-        lengths = _lengths(_rng(s_len), cfg, B)
-    lengths = np.asarray(lengths, dtype=np.int32)
+    lengths, ids, dt = _stca_history(cfg, lengths, s_len, s_ids, s_dt)
     B = len(lengths)
-    n_tok = int(lengths.sum())
-    ids = _ids(_rng(s_ids), n_tok, cfg)
-    dt = None
-    if cfg["time_buckets"]:
-        # seconds since the interaction: floor(2^U[0,16)) - 1
-        e = _rng(s_dt).uniform(0.0, 16.0, size=n_tok)
-        dt = (np.floor(np.exp2(e)) - 1).astype(np.int32)
     tpu = np.full(B, cfg["m"], dtype=np.int32)
     t_tot = int(tpu.sum())
     x_t = _store(_rng(s_xt).standard_normal((t_tot, d), dtype=np.float32), dtype)
