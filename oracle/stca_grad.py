@@ -251,14 +251,30 @@ def stca_backward(wl, dZ):
         # history side, backward: K = Xt W_K, V = Xt W_V, Xt = LN(SwiGLU(X))
         dX = np.zeros_like(X)
         for i in range(M):
-            G["WK"][i] += Xt[i].T @ dK[i]
-            G["WV"][i] += Xt[i].T @ dV[i]
-            dXt = dK[i] @ f64(w["WK"][i]).T + dV[i] @ f64(w["WV"][i]).T
-            dx, g = ffn_ln_bwd(X, w["hist"][i], eps, dXt)
+            dx, g = history_layer_bwd(X, w["hist"][i], w["WK"][i], w["WV"][i], eps, dK[i], dV[i])
+            G["WK"][i] += g.pop("WK")
+            G["WV"][i] += g.pop("WV")
             _add_ffn(G["hist"][i], g)
             dX += dx
-        ids = np.asarray(wl["ids"][sl], dtype=np.int64)
-        np.add.at(dtable, ids, dX)
-        if has_dt:
-            np.add.at(ddt_table, dt_bucket(dt), dX)
+        table_rows_bwd(dtable, ddt_table, wl["ids"][sl], dt, dX)
     return G, dtable, ddt_table, dxt_all
+
+
+def history_layer_bwd(X, ffn, WK, WV, eps, dK, dV):
+    """One layer's history side, X -> Xt = LN(SwiGLU(X)) -> K = Xt W_K, V = Xt W_V
+    ([notes] section "STCA"; [review] 核心公式), backward from dK, dV [n, d]: returns dX and
+    {W1, W3, W2, gamma, beta, WK, WV}."""
+    Xt = layer_norm(swiglu(X, ffn), ffn["gamma"], ffn["beta"], eps)
+    dK, dV = np.asarray(dK, np.float64), np.asarray(dV, np.float64)
+    dXt = dK @ to_f64(WK).T + dV @ to_f64(WV).T
+    dX, g = ffn_ln_bwd(X, ffn, eps, dXt)
+    g.update(WK=Xt.T @ dK, WV=Xt.T @ dV)
+    return dX, g
+
+
+def table_rows_bwd(dtable, ddt_table, ids, dt, dX):
+    """The lookup x_n = E[ids_n] (+ T[bucket(dt_n)]) backward: every token's gradient row is
+    added to the table rows it read (in place)."""
+    np.add.at(dtable, np.asarray(ids, dtype=np.int64), dX)
+    if ddt_table is not None and dt is not None:
+        np.add.at(ddt_table, dt_bucket(dt), dX)

@@ -215,3 +215,38 @@ def test_whole_model_gradients_vs_central_differences(case):
         fd = (lp - lm) / (2 * eps)
         an = float((gr * v).sum())
         assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_history_layer_bwd_vs_autograd():
+    """X -> LN(SwiGLU(X)) -> [K | V]: every gradient of the composed layer against
+    torch.autograd in fp64, random LayerNorm affine."""
+    g = _rng(7)
+    n, d, h = 6, 8, 12
+    X = g.standard_normal((n, d))
+    f = {"W1": g.standard_normal((d, h)), "W3": g.standard_normal((d, h)), "W2": g.standard_normal((h, d)),
+         "gamma": g.standard_normal(d), "beta": g.standard_normal(d)}
+    WK, WV = g.standard_normal((d, d)), g.standard_normal((d, d))
+    dK, dV = g.standard_normal((n, d)), g.standard_normal((n, d))
+    tX, tf, tK, tV = t64(X), {k: t64(v) for k, v in f.items()}, t64(WK), t64(WV)
+    y = (F.silu(tX @ tf["W1"]) * (tX @ tf["W3"])) @ tf["W2"]
+    xt = F.layer_norm(y, (d,), tf["gamma"], tf["beta"], eps=1e-5)
+    loss = ((xt @ tK) * torch.from_numpy(dK)).sum() + ((xt @ tV) * torch.from_numpy(dV)).sum()
+    loss.backward()
+    dX, gw = G.history_layer_bwd(X, f, WK, WV, 1e-5, dK, dV)
+    np.testing.assert_allclose(dX, tX.grad.numpy(), rtol=1e-10, atol=1e-10)
+    for k in f:
+        np.testing.assert_allclose(gw[k], tf[k].grad.numpy(), rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(gw["WK"], tK.grad.numpy(), rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(gw["WV"], tV.grad.numpy(), rtol=1e-10, atol=1e-10)
+
+
+def test_table_rows_bwd_adds_each_token_to_its_rows():
+    dtab, ddt = np.zeros((5, 3)), np.zeros((16, 3))
+    ids = np.array([4, 0, 4, 2], np.int32)
+    dt = np.array([0, 1, 3, 100000], np.int32)       # buckets 0, 1, 2, 15
+    dX = np.arange(12, dtype=np.float64).reshape(4, 3)
+    G.table_rows_bwd(dtab, ddt, ids, dt, dX)
+    np.testing.assert_array_equal(dtab[4], dX[0] + dX[2])
+    np.testing.assert_array_equal(dtab[0], dX[1])
+    np.testing.assert_array_equal(dtab[[1, 3]], 0)
+    np.testing.assert_array_equal(ddt[[0, 1, 2, 15]], dX)
