@@ -26,7 +26,12 @@ int stca_k_offsets(const int32_t* lengths, int B, int32_t* offsets, int expected
 /* Packs a bf16 weight W [K, N] (row-major, y = x W) into the K-major operand layout of
  * the tensor-core GEMMs: mode 0 writes column n to row row_offset + n of dst [rows, K];
  * modes 1 / 2 write W1 / W3 of a SwiGLU into the gate / up halves of 256-row groups
- * (row (n/128)*256 + n%128, plus 128 for mode 2). */
+ * (row (n/128)*256 + n%128, plus 128 for mode 2).  Modes 3 and 4 place W's columns into a
+ * [K, 2N] matrix WITHOUT transposing, which is the operand layout of the backward GEMMs
+ * (dx = dy W^T takes W itself as its K-major operand): mode 3 puts column n at column
+ * 128 (n / 64) + row_offset + n % 64 (row_offset 0 for W_K, 64 for W_V: the head-
+ * interleaved [K_h | V_h] columns of the K/V rows, d_h = 64, N % 64 == 0), mode 4 at
+ * column row_offset + n (row_offset 0 or N: [W1 | W3] side by side). */
 int stca_k_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_offset, void* stream);
 
 /* Tensor-core GEMM with A resident in shared memory (K = 256 or 512), bf16 in, fp32
@@ -100,6 +105,46 @@ int stca_k_attention_rows(int kv_bf16, const float* Q, const void* KV, const int
                           const int32_t* kv_rows, const int32_t* kv_len, const int32_t* kv_mult, int B, int T, int d,
                           int H, int splits, int score, float* part_acc, float* part_ml, float* out, int32_t* err,
                           void* stream);
+
+/* ---- training: the backward of one layer's history side ([notes] STCA: Xt = LN(SwiGLU(X)),
+ * K, V = Xt W_K, Xt W_V; the pages train at about 2K-long histories).  The plain GEMMs of
+ * the backward (dXt = dKV [W_K | W_V]^T, dA = dy W2^T, dX = dP [W1 | W3]^T) run on
+ * stca_k_gemm_resident / stca_k_gemm_rowwise with the weights placed by pack modes 3 / 4
+ * or taken as they are; the entries below are the rest. */
+
+/* Weight gradient C [K, N] = A^T G (accumulate: C += A^T G) over M tokens: A [M, lda] and
+ * G [M, ldg] bf16 row-major (features K and N of each token), C [K, ldc] fp32.  K and N
+ * multiples of 128, lda and ldg multiples of 8, ldc of 4, pointers 16-byte aligned (else
+ * STCA_ERR_UNSUPPORTED / STCA_ERR_INVALID_ARG).  ws: device scratch of at least
+ * stca_k_gemm_wgrad_workspace_bytes(M, K, N) bytes (else STCA_ERR_CAPACITY): the token
+ * slices' partial tiles, added in a fixed order, so the result is the same every run. */
+size_t stca_k_gemm_wgrad_workspace_bytes(int M, int K, int N);
+int stca_k_gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, int M, int K, int N, float* C,
+                      int64_t ldc, int accumulate, void* ws, size_t ws_bytes, void* stream);
+
+/* LayerNorm backward over rows of d = 256 or 512 (biased variance, eps): y [M, d] bf16 the
+ * LayerNorm's input, dxt [M, d] bf16 the gradient of its output, gamma (beta may be NULL)
+ * [d] fp32.  Writes dy [M, d] bf16 and, when xt is not NULL, the output xt = LN(y) [M, d]
+ * bf16 (for the K/V weight gradients); dgamma, dbeta [d] fp32 are set (accumulate: added
+ * to).  ws: at least stca_k_layer_norm_bwd_workspace_bytes(M, d) bytes. */
+size_t stca_k_layer_norm_bwd_workspace_bytes(int M, int d);
+int stca_k_layer_norm_bwd(const void* y, const void* dxt, int M, int d, const float* gamma, const float* beta,
+                          float eps, void* dy, void* xt, float* dgamma, float* dbeta, int accumulate, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/* SwiGLU backward: A = SiLU(P1) * P3 with P = [P1 | P3] [M, 2h] bf16 (x W1 and x W3 side by
+ * side) and dA [M, h] bf16.  Writes dP = [dP1 | dP3] [M, 2h] bf16 with dP1 = dA P3 SiLU'(P1),
+ * dP3 = dA SiLU(P1), and A [M, h] bf16 into a_out when not NULL.  h % 8 == 0, pointers
+ * 16-byte aligned. */
+int stca_k_swiglu_bwd(const void* P, const void* dA, int M, int h, void* dP, void* a_out, void* stream);
+
+/* The lookup's backward: dtable[ids[n]] += dX[n] for n < M (dX [M, d] bf16, dtable
+ * [n_items, d] fp32) and, with dt and ddt_table, ddt_table[b(dt[n])] += dX[n] ([16, d] fp32,
+ * b as in stca_k_gemm_resident).  fp32 atomic adds: the order of the additions into a row
+ * varies between runs.  An id outside [0, n_items) is skipped and records
+ * STCA_ERR_ID_OUT_OF_RANGE in err. */
+int stca_k_table_rows_bwd(const void* dX, int M, int d, const int32_t* ids, const int32_t* dt, int64_t n_items,
+                          float* dtable, float* ddt_table, int32_t* err, void* stream);
 
 /* Distinct history keys (HyFormer page §3.8.1, GPU pooling): key(n) = (ids[n], bucket(dt[n]))
  * (bucket 0 when dt is NULL).  Writes uniq_idx[n] in [0, *count) with equal keys mapped to

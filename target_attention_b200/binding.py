@@ -110,6 +110,13 @@ _SIGS = [
                                 _vp]),
     ("stca_k_attention_rows", _i32, [_i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                      _vp, _vp, _vp, _vp, _vp]),
+    ("stca_k_gemm_wgrad_workspace_bytes", ctypes.c_size_t, [_i32, _i32, _i32]),
+    ("stca_k_gemm_wgrad", _i32, [_vp, _i64, _vp, _i64, _i32, _i32, _i32, _vp, _i64, _i32, _vp, ctypes.c_size_t, _vp]),
+    ("stca_k_layer_norm_bwd_workspace_bytes", ctypes.c_size_t, [_i32, _i32]),
+    ("stca_k_layer_norm_bwd", _i32, [_vp, _vp, _i32, _i32, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _i32, _vp,
+                                     ctypes.c_size_t, _vp]),
+    ("stca_k_swiglu_bwd", _i32, [_vp, _vp, _i32, _i32, _vp, _vp, _vp]),
+    ("stca_k_table_rows_bwd", _i32, [_vp, _i32, _i32, _vp, _vp, _i64, _vp, _vp, _vp, _vp]),
     ("stca_k_dedup_workspace_bytes", ctypes.c_size_t, [_i32]),
     ("stca_k_dedup", _i32, [_vp, _vp, _i32, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]),
     ("stca_k_compact_user_rows", _i32, [_vp, _i32, _vp, _vp, _vp, _vp, _vp]),
@@ -331,6 +338,34 @@ def stca_k_attention_rows(kv_bf16, Q, KV, hoff, toff, kv_rows, kv_len, kv_mult, 
                           part_ml, out, err, stream=None) -> int:
     return lib().stca_k_attention_rows(kv_bf16, ptr(Q), ptr(KV), ptr(hoff), ptr(toff), ptr(kv_rows), ptr(kv_len),
                                        ptr(kv_mult), B, T, d, H, splits, score, ptr(part_acc), ptr(part_ml), ptr(out),
+                                       ptr(err), stream_ptr(stream))
+
+
+def stca_k_gemm_wgrad_workspace_bytes(M, K, N) -> int:
+    return lib().stca_k_gemm_wgrad_workspace_bytes(M, K, N)
+
+
+def stca_k_gemm_wgrad(A, lda, G, ldg, M, K, N, C, ldc, accumulate, ws, ws_bytes, stream=None) -> int:
+    return lib().stca_k_gemm_wgrad(ptr(A), lda, ptr(G), ldg, M, K, N, ptr(C), ldc, accumulate, ptr(ws), ws_bytes,
+                                   stream_ptr(stream))
+
+
+def stca_k_layer_norm_bwd_workspace_bytes(M, d) -> int:
+    return lib().stca_k_layer_norm_bwd_workspace_bytes(M, d)
+
+
+def stca_k_layer_norm_bwd(y, dxt, M, d, gamma, beta, eps, dy, xt, dgamma, dbeta, accumulate, ws, ws_bytes,
+                          stream=None) -> int:
+    return lib().stca_k_layer_norm_bwd(ptr(y), ptr(dxt), M, d, ptr(gamma), ptr(beta), eps, ptr(dy), ptr(xt),
+                                       ptr(dgamma), ptr(dbeta), accumulate, ptr(ws), ws_bytes, stream_ptr(stream))
+
+
+def stca_k_swiglu_bwd(P, dA, M, h, dP, a_out, stream=None) -> int:
+    return lib().stca_k_swiglu_bwd(ptr(P), ptr(dA), M, h, ptr(dP), ptr(a_out), stream_ptr(stream))
+
+
+def stca_k_table_rows_bwd(dX, M, d, ids, dt, n_items, dtable, ddt_table, err, stream=None) -> int:
+    return lib().stca_k_table_rows_bwd(ptr(dX), M, d, ptr(ids), ptr(dt), n_items, ptr(dtable), ptr(ddt_table),
                                        ptr(err), stream_ptr(stream))
 
 

@@ -279,6 +279,21 @@ int dedup_fused(const int32_t* ids, const int32_t* dt, int n, void* ws, size_t w
 int compact_user_rows(const int32_t* hoff, int B, const int32_t* rows, int32_t* out_rows, int32_t* out_mult,
                       int32_t* out_len, cudaStream_t s);
 
+// ---------------------------------------------------------------- training: history side
+// C [K, N] (+)= A^T G over M tokens (A [M, K], G [M, N] bf16, C fp32); K, N % 128 == 0;
+// ws: gemm_wgrad_workspace_bytes(M, K, N) bytes (per-slice partial tiles).
+size_t gemm_wgrad_workspace_bytes(int M, int K, int N);
+int gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, int M, int K, int N, float* C, int64_t ldc,
+               int accumulate, void* ws, size_t ws_bytes, cudaStream_t s);
+size_t layer_norm_bwd_workspace_bytes(int M, int d);
+int layer_norm_bwd(const void* y, const void* dxt, int M, int d, const float* gamma, const float* beta, float eps,
+                   void* dy, void* xt, float* dgamma, float* dbeta, int accumulate, void* ws, size_t ws_bytes,
+                   cudaStream_t s);
+int swiglu_bwd(const void* P, const void* dA, int M, int h, void* dP, void* a_out, cudaStream_t s);
+int table_rows_bwd(const void* dX, int M, int d, const int32_t* ids, const int32_t* dt, int64_t n_items,
+                   float* dtable, float* ddt_table, int32_t* err, cudaStream_t s);
+int place_cols(const void* W, int K, int N, void* dst, int mode, int off, cudaStream_t s);
+
 // ---------------------------------------------------------------- pointwise ReLU TA
 
 int pointwise_relu_ta(const int32_t* ids, const int32_t* offsets, const void* q, const void* table,

@@ -40,8 +40,35 @@ int stca_k_offsets(const int32_t* lengths, int B, int32_t* offsets, int expected
 }
 
 int stca_k_pack_weight(const void* W, int K, int N, void* dst, int mode, int row_offset, void* stream) {
-  if (!W || !dst || mode < 0 || mode > 2) return STCA_ERR_INVALID_ARG;
+  if (!W || !dst || mode < 0 || mode > 4) return STCA_ERR_INVALID_ARG;
+  if (mode >= 3) return place_cols(W, K, N, dst, mode, row_offset, reinterpret_cast<cudaStream_t>(stream));
   return tc_pack_weight(W, K, N, dst, mode, row_offset, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t stca_k_gemm_wgrad_workspace_bytes(int M, int K, int N) { return gemm_wgrad_workspace_bytes(M, K, N); }
+
+int stca_k_gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, int M, int K, int N, float* C,
+                      int64_t ldc, int accumulate, void* ws, size_t ws_bytes, void* stream) {
+  if (M < 0 || (M > 0 && (!A || !G || !ws)) || !C) return STCA_ERR_INVALID_ARG;
+  return gemm_wgrad(A, lda, G, ldg, M, K, N, C, ldc, accumulate, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t stca_k_layer_norm_bwd_workspace_bytes(int M, int d) { return M < 0 ? 0 : layer_norm_bwd_workspace_bytes(M, d); }
+
+int stca_k_layer_norm_bwd(const void* y, const void* dxt, int M, int d, const float* gamma, const float* beta,
+                          float eps, void* dy, void* xt, float* dgamma, float* dbeta, int accumulate, void* ws,
+                          size_t ws_bytes, void* stream) {
+  return layer_norm_bwd(y, dxt, M, d, gamma, beta, eps, dy, xt, dgamma, dbeta, accumulate, ws, ws_bytes,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int stca_k_swiglu_bwd(const void* P, const void* dA, int M, int h, void* dP, void* a_out, void* stream) {
+  return swiglu_bwd(P, dA, M, h, dP, a_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int stca_k_table_rows_bwd(const void* dX, int M, int d, const int32_t* ids, const int32_t* dt, int64_t n_items,
+                          float* dtable, float* ddt_table, int32_t* err, void* stream) {
+  return table_rows_bwd(dX, M, d, ids, dt, n_items, dtable, ddt_table, err, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, const int32_t* dt, const void* table,

@@ -1,0 +1,463 @@
+// Backward (training) steps of the history side of one STCA layer, X -> Xt = LN(SwiGLU(X))
+// -> [K | V] = Xt [W_K | W_V] (STCA notes, section "STCA"; review §三 核心公式), given the
+// gradients of K and V from the attention backward:
+//   dXt = dKV [W_K | W_V]^T            (a plain GEMM, the library's tensor-core kernels)
+//   dW_KV = Xt^T dKV                   gemm_wgrad: a reduction over the tokens
+//   dy, dgamma, dbeta = LN backward    layer_norm_bwd (Xt recomputed on the way)
+//   dA = dy W2^T,  dW2 = A^T dy        plain GEMM + gemm_wgrad
+//   dP = SwiGLU backward of A = SiLU(P1) * P3     swiglu_bwd
+//   dX = dP [W1 | W3]^T, [dW1 | dW3] = X^T dP     plain GEMM + gemm_wgrad
+//   dE[ids], dT[bucket] += dX          table_rows_bwd (the lookup's backward)
+// The pages train at about 2K-long histories (STCA notes, "短序列训练，长序列推理").
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace stca {
+
+namespace {
+
+// ------------------------------------------------------------------ weight gradients
+// C [K, N] = A^T G over the M tokens: A [M, K] and G [M, N] bf16 row-major (tokens by
+// features), C fp32.  A CTA computes a 128 x 128 tile of C over one slice of the tokens,
+// accumulating in registers with mma.sync m16n8k16 (both operands come out of the
+// token-major tiles through ldmatrix.trans); slices write their partial tiles to a
+// workspace that a second kernel adds up in a fixed order, so the result does not depend
+// on scheduling.  Tokens stream through a 4-stage cp.async ring of 32-token stages
+// (8 KB of A and 8 KB of G, 256-byte rows with the 16-byte chunks XOR-swizzled by row).
+constexpr int WG_T = 128;       // C tile (K and N)
+constexpr int WG_TK = 32;       // tokens per stage
+constexpr int WG_STAGES = 4;
+constexpr int WG_TILE_BYTES = WG_TK * WG_T * 2;  // 8 KB
+constexpr int WG_SMEM = WG_STAGES * 2 * WG_TILE_BYTES;  // 64 KB
+
+__device__ __forceinline__ uint32_t wg_off(int tok, int chunk) {  // byte offset in a tile
+  return uint32_t(tok * 256 + ((chunk ^ (tok & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(256, 2) gemm_wgrad_kernel(const bf16* __restrict__ A, int64_t lda,
+                                                            const bf16* __restrict__ G, int64_t ldg, int M, int K,
+                                                            int N, int splits, float* __restrict__ part) {
+  griddep_wait();
+  extern __shared__ __align__(128) uint8_t wg_smem[];
+  const int n0 = blockIdx.x * WG_T, k0 = blockIdx.y * WG_T, sl = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int wm = warp >> 2, wn = warp & 3;  // warp tile: rows 64 wm .. +64 of C, columns 32 wn .. +32
+  const int m_lo = int(int64_t(M) * sl / splits), m_hi = int(int64_t(M) * (sl + 1) / splits);
+  const int n_st = (m_hi - m_lo + WG_TK - 1) / WG_TK;
+  const uint32_t base = smem_u32(wg_smem);
+
+  // stage s: A tile at base + s * 2 * TILE, G tile right after; thread t copies chunks
+  // t and t + 256 of each (token = chunk / 16, 16-byte chunk = chunk % 16)
+  auto load = [&](int st, int slot) {
+    if (st >= n_st) return;
+    const int t0 = m_lo + st * WG_TK;
+    uint8_t* sa = wg_smem + slot * 2 * WG_TILE_BYTES;
+    uint8_t* sg = sa + WG_TILE_BYTES;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int c = tid + 256 * i, tok = c >> 4, ch = c & 15;
+      const int m = t0 + tok;
+      const bool ok = m < m_hi;
+      const int64_t row = ok ? m : m_lo;
+      cp_async_16(sa + wg_off(tok, ch), A + row * lda + k0 + ch * 8, ok ? 16u : 0u);
+      cp_async_16(sg + wg_off(tok, ch), G + row * ldg + n0 + ch * 8, ok ? 16u : 0u);
+    }
+  };
+
+  float acc[4][4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[a][b][e] = 0.f;
+
+#pragma unroll
+  for (int s = 0; s < WG_STAGES - 1; ++s) {
+    load(s, s);
+    cp_async_commit();
+  }
+  for (int st = 0; st < n_st; ++st) {
+    cp_async_wait<WG_STAGES - 2>();
+    __syncthreads();  // stage st landed for every thread; stage st - 1 is free again
+    load(st + WG_STAGES - 1, (st + WG_STAGES - 1) % WG_STAGES);
+    cp_async_commit();
+    const uint32_t sa = base + (st % WG_STAGES) * 2 * WG_TILE_BYTES, sg = sa + WG_TILE_BYTES;
+#pragma unroll
+    for (int kk = 0; kk < WG_TK / 16; ++kk) {
+      // A^T fragments (rows = features of A, k = tokens): matrix q of lane l is rows
+      // tok = 16 kk + (l & 7) + 8 ((l >> 4) & 1), features f0 + 8 ((l >> 3) & 1)
+      uint32_t af[4][4];
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt) {
+        const int tok = 16 * kk + (lane & 7) + 8 * ((lane >> 4) & 1);
+        const int f = 64 * wm + 16 * mt + 8 * ((lane >> 3) & 1);
+        ldsm_x4_t(sa + wg_off(tok, f >> 3), af[mt]);
+      }
+      // G fragments (k = tokens, columns = features of G), two 8-column tiles per load
+      uint32_t bf[4][2];
+#pragma unroll
+      for (int np = 0; np < 2; ++np) {
+        const int tok = 16 * kk + (lane & 7) + 8 * ((lane >> 3) & 1);
+        const int f = 32 * wn + 16 * np + 8 * (lane >> 4);
+        uint32_t r[4];
+        ldsm_x4_t(sg + wg_off(tok, f >> 3), r);
+        bf[2 * np][0] = r[0];
+        bf[2 * np][1] = r[1];
+        bf[2 * np + 1][0] = r[2];
+        bf[2 * np + 1][1] = r[3];
+      }
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) mma_bf16_16816(acc[mt][nt], af[mt], bf[nt][0], bf[nt][1]);
+    }
+  }
+  cp_async_wait_all();
+  griddep_launch();
+  // partial tile of this token slice: part[sl][K][N]
+  float* out = part + int64_t(sl) * K * N;
+  const int g = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int r = k0 + 64 * wm + 16 * mt + g, c = n0 + 32 * wn + 8 * nt + 2 * tq;
+      *reinterpret_cast<float2*>(out + int64_t(r) * N + c) = make_float2(acc[mt][nt][0], acc[mt][nt][1]);
+      *reinterpret_cast<float2*>(out + int64_t(r + 8) * N + c) = make_float2(acc[mt][nt][2], acc[mt][nt][3]);
+    }
+}
+
+// C[k][n] (+)= sum over slices s in order of part[s][k][n]; four columns per thread
+__global__ void wgrad_reduce_kernel(const float* __restrict__ part, int splits, int K, int N, float* __restrict__ C,
+                                    int64_t ldc, int accumulate) {
+  griddep_wait();
+  const int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i >= int64_t(K) * N) return;
+  const int r = int(i / N), c = int(i % N);
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < splits; ++s) {
+    const float4 p = *reinterpret_cast<const float4*>(part + int64_t(s) * K * N + i);
+    v.x += p.x;
+    v.y += p.y;
+    v.z += p.z;
+    v.w += p.w;
+  }
+  float4* dst = reinterpret_cast<float4*>(C + int64_t(r) * ldc + c);
+  if (accumulate) {
+    const float4 o = *dst;
+    v.x += o.x;
+    v.y += o.y;
+    v.z += o.z;
+    v.w += o.w;
+  }
+  *dst = v;
+}
+
+// token slices: enough CTAs for two per SM, each slice at least 256 tokens
+int wgrad_splits(int M, int K, int N) {
+  const int tiles = (K / WG_T) * (N / WG_T);
+  const int by_sm = std::max(1, (2 * sm_count() + tiles - 1) / tiles);
+  const int by_rows = std::max(1, M / 256);
+  return std::min(by_sm, by_rows);
+}
+
+// ------------------------------------------------------------------ LayerNorm backward
+// One warp per row (d = 32 DPL columns, lane l holds columns l + 32 i).  With
+// xhat = (y - mean) rstd and g = dxt * gamma:
+//   dy = rstd (g - mean(g) - xhat mean(g xhat)),  xt = xhat gamma + beta,
+//   dgamma += dxt xhat,  dbeta += dxt  (over the rows; per block, then added in order).
+template <int DPL>
+__global__ void __launch_bounds__(256) ln_bwd_kernel(const bf16* __restrict__ y, const bf16* __restrict__ dxt, int M,
+                                                     const float* __restrict__ gamma, const float* __restrict__ beta,
+                                                     float eps, bf16* __restrict__ dy, bf16* __restrict__ xt,
+                                                     float* __restrict__ part) {
+  griddep_wait();
+  constexpr int D = 32 * DPL;
+  __shared__ float red[8][2][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float gm[DPL], bt[DPL], sg[DPL], sb[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    gm[i] = gamma[lane + 32 * i];
+    bt[i] = beta ? beta[lane + 32 * i] : 0.f;
+    sg[i] = 0.f;
+    sb[i] = 0.f;
+  }
+  const int rows_per_block = (M + gridDim.x - 1) / gridDim.x;
+  const int r0 = blockIdx.x * rows_per_block, r1 = min(M, r0 + rows_per_block);
+  for (int r = r0 + warp; r < r1; r += 8) {
+    float v[DPL], gv[DPL], dv[DPL];
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      v[i] = __bfloat162float(y[int64_t(r) * D + lane + 32 * i]);
+      dv[i] = __bfloat162float(dxt[int64_t(r) * D + lane + 32 * i]);
+      s += v[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / D;
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      v[i] -= mean;
+      q += v[i] * v[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    const float rstd = rsqrtf(q / D + eps);
+    float m1 = 0.f, m2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      v[i] *= rstd;  // xhat
+      gv[i] = dv[i] * gm[i];
+      m1 += gv[i];
+      m2 += gv[i] * v[i];
+      sg[i] += dv[i] * v[i];
+      sb[i] += dv[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      m1 += __shfl_xor_sync(0xffffffffu, m1, o);
+      m2 += __shfl_xor_sync(0xffffffffu, m2, o);
+    }
+    m1 /= D;
+    m2 /= D;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      dy[int64_t(r) * D + lane + 32 * i] = __float2bfloat16(rstd * (gv[i] - m1 - v[i] * m2));
+      if (xt) xt[int64_t(r) * D + lane + 32 * i] = __float2bfloat16(v[i] * gm[i] + bt[i]);
+    }
+  }
+  griddep_launch();
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    red[warp][0][lane + 32 * i] = sg[i];
+    red[warp][1][lane + 32 * i] = sb[i];
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < 2 * D; c += blockDim.x) {
+    const int which = c / D, col = c % D;
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) t += red[w][which][col];
+    part[(int64_t(blockIdx.x) * 2 + which) * D + col] = t;
+  }
+}
+
+// dgamma[c] = sum_b part[b][0][c], dbeta[c] = sum_b part[b][1][c] (blocks in order)
+__global__ void ln_bwd_reduce_kernel(const float* __restrict__ part, int blocks, int D, float* __restrict__ dgamma,
+                                     float* __restrict__ dbeta, int accumulate) {
+  griddep_wait();
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= 2 * D) return;
+  const int which = c / D, col = c % D;
+  float t = 0.f;
+  for (int b = 0; b < blocks; ++b) t += part[(int64_t(b) * 2 + which) * D + col];
+  float* dst = which == 0 ? dgamma : dbeta;
+  dst[col] = accumulate ? dst[col] + t : t;
+}
+
+// ------------------------------------------------------------------ SwiGLU backward
+// A = SiLU(P1) * P3 with P = [P1 | P3] ([M, 2h] bf16) and dA [M, h] bf16:
+//   dP1 = dA P3 SiLU'(P1),  dP3 = dA SiLU(P1),  SiLU'(x) = s (1 + x (1 - s)), s = sigma(x)
+// written to dP = [dP1 | dP3] ([M, 2h] bf16); optionally A itself (a_out [M, h]).
+__global__ void swiglu_bwd_kernel(const bf16* __restrict__ P, const bf16* __restrict__ dA, int64_t M, int h,
+                                  bf16* __restrict__ dP, bf16* __restrict__ a_out) {
+  griddep_wait();
+  const int64_t n8 = M * h / 8;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n8; i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t e = i * 8, r = e / h, c = e % h;
+    const uint4 p1 = *reinterpret_cast<const uint4*>(P + r * 2 * h + c);
+    const uint4 p3 = *reinterpret_cast<const uint4*>(P + r * 2 * h + h + c);
+    const uint4 da = *reinterpret_cast<const uint4*>(dA + e);
+    const __nv_bfloat162* x1 = reinterpret_cast<const __nv_bfloat162*>(&p1);
+    const __nv_bfloat162* x3 = reinterpret_cast<const __nv_bfloat162*>(&p3);
+    const __nv_bfloat162* g = reinterpret_cast<const __nv_bfloat162*>(&da);
+    uint4 o1, o3, oa;
+    __nv_bfloat162* w1 = reinterpret_cast<__nv_bfloat162*>(&o1);
+    __nv_bfloat162* w3 = reinterpret_cast<__nv_bfloat162*>(&o3);
+    __nv_bfloat162* wa = reinterpret_cast<__nv_bfloat162*>(&oa);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 a = __bfloat1622float2(x1[j]), b = __bfloat1622float2(x3[j]), d = __bfloat1622float2(g[j]);
+      const float sa = 1.f / (1.f + __expf(-a.x)), sb = 1.f / (1.f + __expf(-a.y));
+      const float fa = a.x * sa, fb = a.y * sb;  // SiLU
+      w1[j] = __floats2bfloat162_rn(d.x * b.x * sa * (1.f + a.x * (1.f - sa)), d.y * b.y * sb * (1.f + a.y * (1.f - sb)));
+      w3[j] = __floats2bfloat162_rn(d.x * fa, d.y * fb);
+      wa[j] = __floats2bfloat162_rn(fa * b.x, fb * b.y);
+    }
+    *reinterpret_cast<uint4*>(dP + r * 2 * h + c) = o1;
+    *reinterpret_cast<uint4*>(dP + r * 2 * h + h + c) = o3;
+    if (a_out) *reinterpret_cast<uint4*>(a_out + e) = oa;
+  }
+}
+
+// ------------------------------------------------------------------ lookup backward
+// dtable[ids[n]] += dX[n] (fp32 atomics, one warp per token, 8 values per lane per pass);
+// with dt, dt_table[bucket(dt[n])] += dX[n] through a per-block [16, d] shared
+// accumulator, so that the 16 bucket rows take one atomic per block and column.
+__global__ void __launch_bounds__(256) table_rows_bwd_kernel(const bf16* __restrict__ dX, int M, int d,
+                                                             const int32_t* __restrict__ ids,
+                                                             const int32_t* __restrict__ dt, int64_t n_items,
+                                                             float* __restrict__ dtable,
+                                                             float* __restrict__ ddt_table, int32_t* err) {
+  griddep_wait();
+  extern __shared__ float bucket_acc[];  // [16][d] when ddt_table
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool with_dt = dt && ddt_table;
+  if (with_dt)
+    for (int i = threadIdx.x; i < 16 * d; i += blockDim.x) bucket_acc[i] = 0.f;
+  __syncthreads();
+  const int per_block = (M + gridDim.x - 1) / gridDim.x;
+  const int r0 = blockIdx.x * per_block, r1 = min(M, r0 + per_block);
+  for (int r = r0 + warp; r < r1; r += 8) {
+    const int64_t id = ids[r];
+    const bool ok = id >= 0 && id < n_items;
+    if (!ok && lane == 0) set_error(err, STCA_ERR_ID_OUT_OF_RANGE);
+    const int b = with_dt ? dt_bucket(dt[r]) : 0;
+    for (int c = lane * 8; c < d; c += 256) {
+      const uint4 u = *reinterpret_cast<const uint4*>(dX + int64_t(r) * d + c);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(h2[j]);
+        if (ok) {
+          atomicAdd(dtable + id * d + c + 2 * j, f.x);
+          atomicAdd(dtable + id * d + c + 2 * j + 1, f.y);
+        }
+        if (with_dt) {
+          atomicAdd(bucket_acc + b * d + c + 2 * j, f.x);
+          atomicAdd(bucket_acc + b * d + c + 2 * j + 1, f.y);
+        }
+      }
+    }
+  }
+  griddep_launch();
+  if (!with_dt) return;
+  __syncthreads();
+  for (int i = threadIdx.x; i < 16 * d; i += blockDim.x)
+    if (bucket_acc[i] != 0.f) atomicAdd(ddt_table + i, bucket_acc[i]);
+}
+
+// dst [K, 2N] from W [K, N] without transposing: mode 3 puts column n of W at column
+// 128 (n / 64) + off + n % 64 (the head-interleaved [K_h | V_h] layout, d_h = 64), mode 4
+// at column off + n (two blocks side by side)
+__global__ void place_cols_kernel(const bf16* __restrict__ W, int K, int N, bf16* __restrict__ dst, int mode,
+                                  int off) {
+  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= int64_t(K) * N) return;
+  const int k = int(i / N), n = int(i % N);
+  const int col = mode == 3 ? 128 * (n / 64) + off + n % 64 : off + n;
+  dst[int64_t(k) * 2 * N + col] = W[i];
+}
+
+}  // namespace
+
+size_t gemm_wgrad_workspace_bytes(int M, int K, int N) {
+  if (M <= 0 || K <= 0 || N <= 0 || K % WG_T || N % WG_T) return 0;
+  return size_t(wgrad_splits(M, K, N)) * K * N * 4;
+}
+
+int gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, int M, int K, int N, float* C, int64_t ldc,
+               int accumulate, void* ws, size_t ws_bytes, cudaStream_t s) {
+  if (M < 0 || K <= 0 || N <= 0 || K % WG_T || N % WG_T || lda % 8 || ldg % 8 || ldc % 4) return STCA_ERR_UNSUPPORTED;
+  if (lda < K || ldg < N || ldc < N) return STCA_ERR_INVALID_ARG;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(G) |
+                       reinterpret_cast<uintptr_t>(C) | reinterpret_cast<uintptr_t>(ws);
+  if (al & 15) return STCA_ERR_INVALID_ARG;
+  const int splits = M > 0 ? wgrad_splits(M, K, N) : 1;
+  if (M > 0 && ws_bytes < size_t(splits) * K * N * 4) return STCA_ERR_CAPACITY;
+  float* part = static_cast<float*>(ws);
+  if (M > 0) {
+    cudaFuncSetAttribute(gemm_wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
+    if (launch_dep(gemm_wgrad_kernel, dim3(N / WG_T, K / WG_T, splits), dim3(256), WG_SMEM, s,
+                   static_cast<const bf16*>(A), lda, static_cast<const bf16*>(G), ldg, M, K, N, splits,
+                   part) != cudaSuccess)
+      return STCA_ERR_CUDA;
+    note_launch();
+  } else if (!accumulate) {
+    return cudaMemset2DAsync(C, size_t(ldc) * 4, 0, size_t(N) * 4, K, s) == cudaSuccess ? STCA_OK : STCA_ERR_CUDA;
+  } else {
+    return STCA_OK;
+  }
+  const int64_t n4 = int64_t(K) * N / 4;
+  if (launch_dep(wgrad_reduce_kernel, dim3(unsigned((n4 + 255) / 256)), dim3(256), 0, s,
+                 static_cast<const float*>(part), splits, K, N, C, ldc, accumulate) != cudaSuccess)
+    return STCA_ERR_CUDA;
+  note_launch();
+  return STCA_OK;
+}
+
+int ln_bwd_blocks(int M) { return std::max(1, std::min(2 * sm_count(), (M + 31) / 32)); }
+
+size_t layer_norm_bwd_workspace_bytes(int M, int d) { return size_t(ln_bwd_blocks(M)) * 2 * d * 4; }
+
+int layer_norm_bwd(const void* y, const void* dxt, int M, int d, const float* gamma, const float* beta, float eps,
+                   void* dy, void* xt, float* dgamma, float* dbeta, int accumulate, void* ws, size_t ws_bytes,
+                   cudaStream_t s) {
+  if (M < 0 || (d != 256 && d != 512)) return STCA_ERR_UNSUPPORTED;
+  if (!gamma || !dgamma || !dbeta || (M > 0 && (!y || !dxt || !dy))) return STCA_ERR_INVALID_ARG;
+  const int blocks = ln_bwd_blocks(M);
+  if (ws_bytes < size_t(blocks) * 2 * d * 4 || !ws) return STCA_ERR_CAPACITY;
+  float* part = static_cast<float*>(ws);
+  auto kern = d == 256 ? ln_bwd_kernel<8> : ln_bwd_kernel<16>;
+  if (launch_dep(kern, dim3(blocks), dim3(256), 0, s, static_cast<const bf16*>(y), static_cast<const bf16*>(dxt), M,
+                 gamma, beta, eps, static_cast<bf16*>(dy), static_cast<bf16*>(xt), part) != cudaSuccess)
+    return STCA_ERR_CUDA;
+  note_launch();
+  if (launch_dep(ln_bwd_reduce_kernel, dim3((2 * d + 255) / 256), dim3(256), 0, s, static_cast<const float*>(part),
+                 blocks, d, dgamma, dbeta, accumulate) != cudaSuccess)
+    return STCA_ERR_CUDA;
+  note_launch();
+  return STCA_OK;
+}
+
+int swiglu_bwd(const void* P, const void* dA, int M, int h, void* dP, void* a_out, cudaStream_t s) {
+  if (M < 0 || h <= 0 || h % 8) return STCA_ERR_UNSUPPORTED;
+  if (M == 0) return STCA_OK;
+  if (!P || !dA || !dP) return STCA_ERR_INVALID_ARG;
+  const uintptr_t al = reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(dA) |
+                       reinterpret_cast<uintptr_t>(dP) | reinterpret_cast<uintptr_t>(a_out);
+  if (al & 15) return STCA_ERR_INVALID_ARG;
+  const int64_t n8 = int64_t(M) * h / 8;
+  const int blocks = int(std::min<int64_t>((n8 + 255) / 256, int64_t(8) * sm_count()));
+  if (launch_dep(swiglu_bwd_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const bf16*>(P),
+                 static_cast<const bf16*>(dA), int64_t(M), h, static_cast<bf16*>(dP), static_cast<bf16*>(a_out)) !=
+      cudaSuccess)
+    return STCA_ERR_CUDA;
+  note_launch();
+  return STCA_OK;
+}
+
+int table_rows_bwd(const void* dX, int M, int d, const int32_t* ids, const int32_t* dt, int64_t n_items,
+                   float* dtable, float* ddt_table, int32_t* err, cudaStream_t s) {
+  if (M < 0 || d <= 0 || d % 8 || n_items <= 0) return STCA_ERR_INVALID_ARG;
+  if (M == 0) return STCA_OK;
+  if (!dX || !ids || !dtable || (reinterpret_cast<uintptr_t>(dX) & 15)) return STCA_ERR_INVALID_ARG;
+  const bool with_dt = dt && ddt_table;
+  const size_t smem = with_dt ? size_t(16) * d * 4 : 0;
+  if (smem > 48 * 1024) return STCA_ERR_UNSUPPORTED;
+  const int blocks = std::max(1, std::min(4 * sm_count(), (M + 7) / 8));
+  if (launch_dep(table_rows_bwd_kernel, dim3(blocks), dim3(256), smem, s, static_cast<const bf16*>(dX), M, d, ids,
+                 with_dt ? dt : nullptr, n_items, dtable, with_dt ? ddt_table : nullptr, err) != cudaSuccess)
+    return STCA_ERR_CUDA;
+  note_launch();
+  return STCA_OK;
+}
+
+int place_cols(const void* W, int K, int N, void* dst, int mode, int off, cudaStream_t s) {
+  if (!W || !dst || K <= 0 || N <= 0 || (mode != 3 && mode != 4)) return STCA_ERR_INVALID_ARG;
+  if (mode == 3 && (N % 64 || (off != 0 && off != 64))) return STCA_ERR_INVALID_ARG;
+  if (mode == 4 && off != 0 && off != N) return STCA_ERR_INVALID_ARG;
+  const int64_t n = int64_t(K) * N;
+  place_cols_kernel<<<unsigned((n + 255) / 256), 256, 0, s>>>(static_cast<const bf16*>(W), K, N,
+                                                              static_cast<bf16*>(dst), mode, off);
+  note_launch();
+  return cudaGetLastError() == cudaSuccess ? STCA_OK : STCA_ERR_CUDA;
+}
+
+}  // namespace stca

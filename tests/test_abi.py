@@ -110,6 +110,22 @@ def test_null_arguments_rejected_on_host():
     assert L.stca_k_attention_rows(0, 16, 16, 16, 16, 16, None, 16, 1, 1, 64, 1, 1, 0, 16, 16, 16, None, None) \
         == B.ERR_UNSUPPORTED                          # key weights with fp32 K/V
     assert L.stca_k_pack_weight(None, 4, 4, None, 0, 0, None) == B.ERR_INVALID_ARG
+    assert L.stca_k_pack_weight(16, 64, 100, 16, 3, 0, None) == B.ERR_INVALID_ARG   # mode 3 needs N % 64
+    assert L.stca_k_pack_weight(16, 64, 64, 16, 3, 32, None) == B.ERR_INVALID_ARG   # ... and the K or V half
+    assert L.stca_k_pack_weight(16, 64, 64, 16, 5, 0, None) == B.ERR_INVALID_ARG
+    # training entries: shapes the kernels do not take, workspace too small, missing buffers
+    assert L.stca_k_gemm_wgrad(16, 128, 16, 128, 100, 96, 128, 16, 128, 0, 16, 1 << 30, None) == B.ERR_UNSUPPORTED
+    assert L.stca_k_gemm_wgrad(16, 128, 16, 128, 100, 128, 128, 16, 128, 0, 16, 16, None) == B.ERR_CAPACITY
+    assert L.stca_k_gemm_wgrad(16, 120, 16, 128, 100, 128, 128, 16, 128, 0, 16, 1 << 30, None) == B.ERR_INVALID_ARG
+    assert L.stca_k_gemm_wgrad(None, 128, 16, 128, 100, 128, 128, 16, 128, 0, 16, 1 << 30, None) == B.ERR_INVALID_ARG
+    assert L.stca_k_layer_norm_bwd(16, 16, 10, 384, 16, None, 1e-5, 16, None, 16, 16, 0, 16, 1 << 20, None) \
+        == B.ERR_UNSUPPORTED
+    assert L.stca_k_layer_norm_bwd(16, 16, 10, 256, 16, None, 1e-5, 16, None, 16, 16, 0, 16, 4, None) \
+        == B.ERR_CAPACITY
+    assert L.stca_k_swiglu_bwd(16, 16, 10, 12, 16, None, None) == B.ERR_UNSUPPORTED        # h % 8
+    assert L.stca_k_swiglu_bwd(16, 16, 10, 16, 24, None, None) == B.ERR_INVALID_ARG        # alignment
+    assert L.stca_k_table_rows_bwd(16, 10, 12, 16, None, 100, 16, None, None, None) == B.ERR_INVALID_ARG
+    assert L.stca_k_table_rows_bwd(16, 10, 256, None, None, 100, 16, None, None, None) == B.ERR_INVALID_ARG
     assert L.stca_k_gemm_resident(1, 1, None, None, None, None, None, 0, 5, 256, None, 128, None, 128, None, None,
                                   None) == B.ERR_INVALID_ARG
     # x_out only with the gather

@@ -1,0 +1,179 @@
+"""Backward of one layer's history side on the GPU (X -> LN(SwiGLU(X)) -> [K | V], then the
+lookup), composed from the library's kernel-level entries, against the fp64 oracle
+(``stca_grad.history_layer_bwd`` and ``table_rows_bwd``) on the same bf16 inputs.
+
+The forward values the backward needs are recomputed on the GPU the way a training step
+would (the gathered rows X, x W1 | x W3, the SwiGLU output A and y = A W2); the upstream
+dK, dV are random, rounded to bf16 as the attention backward would hand them over.
+Gradients are compared normwise per tensor: max |g - r| / max |r| <= 2e-2 (bf16 operands
+and intermediates, fp32 accumulation).  The weight-gradient GEMM and the LayerNorm
+backward are also checked alone against float64 on their exact bf16 inputs."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import stca_grad as G
+from oracle import stca_ref as R
+from target_attention_b200 import binding as B
+from tests._util import bf16_to_f64, zeros_err
+from workloads import make_stca
+
+pytestmark = pytest.mark.gpu
+dev = "cuda"
+TOL = 2e-2
+
+
+def up16(bits):
+    """bf16 bit patterns (uint16) -> device bf16 tensor."""
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+
+def to_bf16(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).to(dev)
+
+
+def ws(nbytes):
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=dev)
+
+
+def normwise(got, ref):
+    ref = np.asarray(ref, np.float64)
+    return float(np.abs(np.asarray(got, np.float64) - ref).max() / max(np.abs(ref).max(), 1e-30))
+
+
+@pytest.mark.parametrize("M, K, N, lda_pad", [(1000, 128, 128, 0), (5003, 256, 512, 8), (77, 512, 256, 0)])
+def test_gemm_wgrad_matches_float64(M, K, N, lda_pad):
+    """C = A^T G over ragged token counts (a partial last stage, several token slices),
+    padded leading dimensions, and C += A^T G with accumulate."""
+    g = np.random.default_rng(M)
+    A = to_bf16(g.standard_normal((M, K + lda_pad)))
+    Gm = to_bf16(g.standard_normal((M, N)))
+    C = torch.full((K, N), float("nan"), device=dev)
+    w = ws(B.stca_k_gemm_wgrad_workspace_bytes(M, K, N))
+    B.check(B.stca_k_gemm_wgrad(A, K + lda_pad, Gm, N, M, K, N, C, N, 0, w, w.numel()))
+    ref = bf16_to_f64(A)[:, :K].T @ bf16_to_f64(Gm)
+    got = C.cpu().numpy()
+    assert normwise(got, ref) < 1e-5
+    B.check(B.stca_k_gemm_wgrad(A, K + lda_pad, Gm, N, M, K, N, C, N, 1, w, w.numel()))
+    assert normwise(C.cpu().numpy(), 2 * ref) < 1e-5
+    # the partials are added in a fixed order: the same bits every run
+    C2 = torch.empty_like(C)
+    B.check(B.stca_k_gemm_wgrad(A, K + lda_pad, Gm, N, M, K, N, C2, N, 0, w, w.numel()))
+    assert torch.equal(C2.cpu(), torch.from_numpy(got))
+
+
+@pytest.mark.parametrize("d", [256, 512])
+def test_layer_norm_bwd_matches_oracle(d):
+    g = np.random.default_rng(d)
+    M, eps = 333, 1e-5
+    y = to_bf16(g.standard_normal((M, d)) * 2 + 0.5)
+    dxt = to_bf16(g.standard_normal((M, d)))
+    gamma = torch.from_numpy(g.standard_normal(d).astype(np.float32)).to(dev)
+    beta = torch.from_numpy(g.standard_normal(d).astype(np.float32)).to(dev)
+    dy = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+    xt = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+    dg = torch.empty(d, device=dev)
+    db = torch.empty(d, device=dev)
+    w = ws(B.stca_k_layer_norm_bwd_workspace_bytes(M, d))
+    B.check(B.stca_k_layer_norm_bwd(y, dxt, M, d, gamma, beta, eps, dy, xt, dg, db, 0, w, w.numel()))
+    y64, dxt64 = bf16_to_f64(y), bf16_to_f64(dxt)
+    rdy, rdg, rdb = G.layer_norm_bwd(y64, gamma.cpu().numpy(), beta.cpu().numpy(), eps, dxt64)
+    assert normwise(bf16_to_f64(dy), rdy) < 1e-2
+    assert normwise(dg.cpu().numpy(), rdg) < 1e-4 and normwise(db.cpu().numpy(), rdb) < 1e-4
+    rxt = R.layer_norm(y64, gamma.cpu().numpy(), beta.cpu().numpy(), eps)
+    assert normwise(bf16_to_f64(xt), rxt) < 1e-2
+
+
+@pytest.mark.parametrize("config", [2, 3])
+def test_history_layer_backward_matches_oracle(config):
+    """config 2's shape (d = 256, h = 512, no time feature) and config 3's (d = 512,
+    h = 1024, 16 time buckets), two users of ragged length, layer 0's weights."""
+    wl = make_stca(config, users=2, L=1500 if config == 2 else 900, n_items=3000)
+    cfg = wl["cfg"]
+    d, h, eps = cfg["d"], cfg["hidden"], 1e-5
+    w = wl["weights"]
+    ffn, WK, WV = w["hist"][0], w["WK"][0], w["WV"][0]
+    ids, dt = wl["ids"], wl["dt"]
+    M = len(ids)
+    g = np.random.default_rng(5)
+    bf16_round = lambda x: torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    dK, dV = bf16_round(g.standard_normal((M, d))), bf16_round(g.standard_normal((M, d)))
+    # device inputs
+    table, W1, W3, W2 = up16(wl["table"]), up16(ffn["W1"]), up16(ffn["W3"]), up16(ffn["W2"])
+    dtab = up16(wl["dt_table"]) if dt is not None else None
+    ids_t = torch.from_numpy(ids.astype(np.int32)).to(dev)
+    dt_t = torch.from_numpy(dt.astype(np.int32)).to(dev) if dt is not None else None
+    gamma = torch.from_numpy(R.to_f64(ffn["gamma"]).astype(np.float32)).to(dev)
+    beta = torch.from_numpy(R.to_f64(ffn["beta"]).astype(np.float32)).to(dev)
+    err = zeros_err()
+    n_items = int(wl["table"].shape[0])
+    bf = lambda *shape: torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    # ---- forward values, recomputed
+    W13p = bf(2 * h, d)                                   # SwiGLU operand (packed modes 1 + 2)
+    B.check(B.stca_k_pack_weight(W1, d, h, W13p, 1, 0))
+    B.check(B.stca_k_pack_weight(W3, d, h, W13p, 2, 0))
+    X, A = bf(M, d), bf(M, h)
+    B.check(B.stca_k_gemm_resident(1, 1, None, ids_t, dt_t, table, dtab, n_items, M, d, W13p, h, A, h, err, x_out=X))
+    Pp = bf(2 * h, d)                                     # [x W1 | x W3] operand (mode 0)
+    B.check(B.stca_k_pack_weight(W1, d, h, Pp, 0, 0))
+    B.check(B.stca_k_pack_weight(W3, d, h, Pp, 0, h))
+    P = bf(M, 2 * h)
+    B.check(B.stca_k_gemm_resident(0, 0, X, None, None, None, None, 0, M, d, Pp, 2 * h, P, 2 * h, err))
+    W2p = bf(d, h)
+    B.check(B.stca_k_pack_weight(W2, h, d, W2p, 0, 0))
+    y = bf(M, d)
+    B.check(B.stca_k_gemm_rowwise(0, A, M, h, W2p, d, None, None, eps, y, d, err))
+    # ---- backward
+    dKV = np.zeros((M, 2 * d))
+    for hh in range(d // 64):                            # the K/V rows' [K_h | V_h] columns
+        dKV[:, 128 * hh:128 * hh + 64] = dK[:, 64 * hh:64 * hh + 64]
+        dKV[:, 128 * hh + 64:128 * hh + 128] = dV[:, 64 * hh:64 * hh + 64]
+    dKV_t = to_bf16(dKV)
+    WKVi = bf(d, 2 * d)
+    B.check(B.stca_k_pack_weight(up16(WK), d, d, WKVi, 3, 0))
+    B.check(B.stca_k_pack_weight(up16(WV), d, d, WKVi, 3, 64))
+    dXt = bf(M, d)
+    B.check(B.stca_k_gemm_rowwise(0, dKV_t, M, 2 * d, WKVi, d, None, None, eps, dXt, d, err))
+    dy, Xt = bf(M, d), bf(M, d)
+    dgamma, dbeta = torch.empty(d, device=dev), torch.empty(d, device=dev)
+    wln = ws(B.stca_k_layer_norm_bwd_workspace_bytes(M, d))
+    B.check(B.stca_k_layer_norm_bwd(y, dXt, M, d, gamma, beta, eps, dy, Xt, dgamma, dbeta, 0, wln, wln.numel()))
+    dWKV = torch.empty((d, 2 * d), device=dev)
+    wg = ws(max(B.stca_k_gemm_wgrad_workspace_bytes(M, K, N) for K, N in ((d, 2 * d), (h, d), (d, 2 * h))))
+    B.check(B.stca_k_gemm_wgrad(Xt, d, dKV_t, 2 * d, M, d, 2 * d, dWKV, 2 * d, 0, wg, wg.numel()))
+    dA = bf(M, h)                                        # dy W2^T: W2 itself is the operand
+    B.check(B.stca_k_gemm_resident(0, 0, dy, None, None, None, None, 0, M, d, W2, h, dA, h, err))
+    dW2 = torch.empty((h, d), device=dev)
+    B.check(B.stca_k_gemm_wgrad(A, h, dy, d, M, h, d, dW2, d, 0, wg, wg.numel()))
+    dP = bf(M, 2 * h)
+    B.check(B.stca_k_swiglu_bwd(P, dA, M, h, dP, None))
+    W13c = bf(d, 2 * h)                                  # [W1 | W3] side by side
+    B.check(B.stca_k_pack_weight(W1, d, h, W13c, 4, 0))
+    B.check(B.stca_k_pack_weight(W3, d, h, W13c, 4, h))
+    dX = bf(M, d)
+    B.check(B.stca_k_gemm_rowwise(0, dP, M, 2 * h, W13c, d, None, None, eps, dX, d, err))
+    dW13 = torch.empty((d, 2 * h), device=dev)
+    B.check(B.stca_k_gemm_wgrad(X, d, dP, 2 * h, M, d, 2 * h, dW13, 2 * h, 0, wg, wg.numel()))
+    dtable = torch.zeros((n_items, d), device=dev)
+    ddt = torch.zeros((16, d), device=dev) if dt is not None else None
+    B.check(B.stca_k_table_rows_bwd(dX, M, d, ids_t, dt_t, n_items, dtable, ddt, err))
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    # ---- oracle on the same stored values
+    X64 = R.gather_history(wl["table"], ids, dt, wl.get("dt_table"))
+    rdX, rg = G.history_layer_bwd(X64, ffn, WK, WV, eps, dK, dV)
+    rtab = np.zeros((n_items, d))
+    rdt = np.zeros((16, d)) if dt is not None else None
+    G.table_rows_bwd(rtab, rdt, ids, dt, rdX)
+    gKV = dWKV.cpu().numpy()
+    gWK = np.concatenate([gKV[:, 128 * hh:128 * hh + 64] for hh in range(d // 64)], axis=1)
+    gWV = np.concatenate([gKV[:, 128 * hh + 64:128 * hh + 128] for hh in range(d // 64)], axis=1)
+    got = {"WK": gWK, "WV": gWV, "W2": dW2.cpu().numpy(), "W1": dW13.cpu().numpy()[:, :h],
+           "W3": dW13.cpu().numpy()[:, h:], "gamma": dgamma.cpu().numpy(), "beta": dbeta.cpu().numpy()}
+    errs = {k: normwise(got[k], rg[k]) for k in got}
+    errs["X"] = normwise(bf16_to_f64(dX), rdX)
+    errs["table"] = normwise(dtable.cpu().numpy(), rtab)
+    if dt is not None:
+        errs["dt_table"] = normwise(ddt.cpu().numpy(), rdt)
+    print("history-side backward, normwise errors:", {k: f"{v:.1e}" for k, v in errs.items()})
+    assert max(errs.values()) <= TOL, errs
