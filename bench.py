@@ -61,10 +61,11 @@ def parse():
                     help="control run: history ids uniform over the table instead of Zipf")
     ap.add_argument("--kv-fold", action="store_true",
                     help="fold W_K / W_V into the queries (d = 256 STCA workloads only)")
-    ap.add_argument("--probe", choices=["attention"], default=None,
-                    help="instead of the step: time one kernel alone on the workload's shapes and print "
-                         "one JSON line per input form (attention: contiguous keys, and the compacted "
-                         "per-user key lists of the workload's ids, through the kernel-level entries)")
+    ap.add_argument("--probe", choices=["attention", "history-backward"], default=None,
+                    help="instead of the step: time kernels alone on the workload's shapes and print one "
+                         "JSON line per kernel or input form (attention: contiguous keys and the compacted "
+                         "per-user key lists of the workload's ids; history-backward: every step of one "
+                         "layer's history-side backward at the workload's d, h and history tokens)")
     return ap.parse_args()
 
 
@@ -829,10 +830,88 @@ def run_probe_attention(args):
                           "frac": round(gbs / peaks["hbm_gbs"], 4)}), flush=True)
 
 
+def run_probe_history_backward(args):
+    """One layer's history-side backward (target_attention_b200.training) on the workload's
+    shapes (--workload 2 or 3; every history token, no distinct-key compaction): the forward
+    recompute and the backward, each step bracketed by CUDA events, median over 3 x steps
+    runs after warm-up.  GEMMs are charged 2 M K N flop against the measured sustained bf16
+    rate; the LayerNorm / SwiGLU backward and the lookup scatter their bytes against the
+    measured HBM rate."""
+    import statistics
+    import numpy as np
+    import torch
+    from target_attention_b200.training import HistoryLayerBackward
+    wl = make_workload(args, data_seed=rank_data_seed(args.workload, 0))
+    assert wl["cfg"]["kind"] == "stca", "history-backward probes an STCA workload (2 or 3)"
+    cfg, w = wl["cfg"], wl["weights"]
+    d, h = cfg["d"], cfg["hidden"]
+    ids, dt = wl["ids"], wl["dt"]
+    M, n_items = len(ids), int(wl["table"].shape[0])
+    dev = "cuda"
+    up16 = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)
+    f32 = lambda a: torch.from_numpy(np.asarray(a, np.float32)).to(dev)
+    ffn = w["hist"][0]  # LayerNorm parameters are stored as float32
+    layer = HistoryLayerBackward(M, d, h, up16(ffn["W1"]), up16(ffn["W3"]), up16(ffn["W2"]), up16(w["WK"][0]),
+                                 up16(w["WV"][0]), f32(ffn["gamma"]), f32(ffn["beta"]))
+    ids_t = torch.from_numpy(ids.astype(np.int32)).to(dev)
+    dt_t = torch.from_numpy(dt.astype(np.int32)).to(dev) if dt is not None else None
+    table = up16(wl["table"])
+    dtab = up16(wl["dt_table"]) if dt is not None else None
+    g = torch.Generator(device=dev)
+    g.manual_seed(3)
+    dKV = torch.randn((M, 2 * d), device=dev, generator=g).to(torch.bfloat16)
+    dtable = torch.zeros((n_items, d), device=dev)
+    ddt = torch.zeros((16, d), device=dev) if dt is not None else None
+
+    times = {}
+    def run(record):
+        marks = []
+        on_step = (lambda name: (marks.append((name, torch.cuda.Event(enable_timing=True))), marks[-1][1].record())) \
+            if record else None
+        start = torch.cuda.Event(enable_timing=True)
+        start.record()
+        layer.recompute(ids_t, dt_t, table, dtab, n_items, on_step=on_step)
+        layer.backward(dKV, ids_t, dt_t, n_items, dtable, ddt, on_step=on_step)
+        return start, marks
+
+    for _ in range(max(args.warmup, 1)):
+        run(False)
+    torch.cuda.synchronize()
+    for _ in range(3 * args.steps):
+        start, marks = run(True)
+        torch.cuda.synchronize()
+        prev = start
+        for name, ev in marks:
+            times.setdefault(name, []).append(prev.elapsed_time(ev))
+            prev = ev
+        times.setdefault("layer", []).append(start.elapsed_time(marks[-1][1]))
+    assert int(layer.err.item()) == 0
+    peaks = load_peaks()
+    flops = layer.flops()
+    bytes_ = {"LN backward": M * d * 2 * 4, "SwiGLU backward": M * h * 2 * 5, "table rows": M * d * (2 + 2 * 4)}
+    total_flop = sum(flops.values())
+    for name, ts in times.items():
+        ms = statistics.median(ts)
+        line = {"probe": "history-backward", "step": name, "workload": args.workload, "history_tokens": M, "d": d,
+                "hidden": h, "median_ms": round(ms, 4), "runs": len(ts)}
+        if name in flops or name == "layer":
+            f = total_flop if name == "layer" else flops[name]
+            tf = f / ms / 1e9
+            line.update(flop=f, achieved_tflops=round(tf, 1), peak_tflops=peaks["bf16_tflops_sustained"],
+                        frac=round(tf / peaks["bf16_tflops_sustained"], 4))
+        elif name in bytes_:
+            gbs = bytes_[name] / ms / 1e6
+            line.update(bytes=bytes_[name], achieved_gbs=round(gbs, 1), peak_gbs=peaks["hbm_gbs"],
+                        frac=round(gbs / peaks["hbm_gbs"], 4))
+        print(json.dumps(line), flush=True)
+
+
 if __name__ == "__main__":
     a = parse()
     if a.probe == "attention":
         run_probe_attention(a)
+    elif a.probe == "history-backward":
+        run_probe_history_backward(a)
     elif a.impl == "reference":
         run_reference(a)
     else:

@@ -140,9 +140,9 @@ int stca_k_swiglu_bwd(const void* P, const void* dA, int M, int h, void* dP, voi
 
 /* The lookup's backward: dtable[ids[n]] += dX[n] for n < M (dX [M, d] bf16, dtable
  * [n_items, d] fp32) and, with dt and ddt_table, ddt_table[b(dt[n])] += dX[n] ([16, d] fp32,
- * b as in stca_k_gemm_resident).  fp32 atomic adds: the order of the additions into a row
- * varies between runs.  An id outside [0, n_items) is skipped and records
- * STCA_ERR_ID_OUT_OF_RANGE in err. */
+ * b as in stca_k_gemm_resident).  d % 8 == 0 (at most 768 with dt), dX and dtable 16-byte
+ * aligned.  fp32 atomic adds: the order of the additions into a row varies between runs.
+ * An id outside [0, n_items) is skipped and records STCA_ERR_ID_OUT_OF_RANGE in err. */
 int stca_k_table_rows_bwd(const void* dX, int M, int d, const int32_t* ids, const int32_t* dt, int64_t n_items,
                           float* dtable, float* ddt_table, int32_t* err, void* stream);
 

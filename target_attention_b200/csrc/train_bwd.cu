@@ -24,13 +24,13 @@ namespace {
 // accumulating in registers with mma.sync m16n8k16 (both operands come out of the
 // token-major tiles through ldmatrix.trans); slices write their partial tiles to a
 // workspace that a second kernel adds up in a fixed order, so the result does not depend
-// on scheduling.  Tokens stream through a 4-stage cp.async ring of 32-token stages
-// (8 KB of A and 8 KB of G, 256-byte rows with the 16-byte chunks XOR-swizzled by row).
+// on scheduling.  Tokens stream through a 3-stage cp.async ring of 64-token stages
+// (16 KB of A and 16 KB of G, 256-byte rows with the 16-byte chunks XOR-swizzled by row).
 constexpr int WG_T = 128;       // C tile (K and N)
-constexpr int WG_TK = 32;       // tokens per stage
-constexpr int WG_STAGES = 4;
-constexpr int WG_TILE_BYTES = WG_TK * WG_T * 2;  // 8 KB
-constexpr int WG_SMEM = WG_STAGES * 2 * WG_TILE_BYTES;  // 64 KB
+constexpr int WG_TK = 64;       // tokens per stage
+constexpr int WG_STAGES = 3;
+constexpr int WG_TILE_BYTES = WG_TK * WG_T * 2;  // 16 KB
+constexpr int WG_SMEM = WG_STAGES * 2 * WG_TILE_BYTES;  // 96 KB: two CTAs per SM
 
 __device__ __forceinline__ uint32_t wg_off(int tok, int chunk) {  // byte offset in a tile
   return uint32_t(tok * 256 + ((chunk ^ (tok & 7)) << 4));
@@ -49,14 +49,14 @@ __global__ void __launch_bounds__(256, 2) gemm_wgrad_kernel(const bf16* __restri
   const uint32_t base = smem_u32(wg_smem);
 
   // stage s: A tile at base + s * 2 * TILE, G tile right after; thread t copies chunks
-  // t and t + 256 of each (token = chunk / 16, 16-byte chunk = chunk % 16)
+  // t, t + 256, ... of each (token = chunk / 16, 16-byte chunk = chunk % 16)
   auto load = [&](int st, int slot) {
     if (st >= n_st) return;
     const int t0 = m_lo + st * WG_TK;
     uint8_t* sa = wg_smem + slot * 2 * WG_TILE_BYTES;
     uint8_t* sg = sa + WG_TILE_BYTES;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < WG_TK * 16 / 256; ++i) {
       const int c = tid + 256 * i, tok = c >> 4, ch = c & 15;
       const int m = t0 + tok;
       const bool ok = m < m_hi;
@@ -297,7 +297,8 @@ __global__ void swiglu_bwd_kernel(const bf16* __restrict__ P, const bf16* __rest
 }
 
 // ------------------------------------------------------------------ lookup backward
-// dtable[ids[n]] += dX[n] (fp32 atomics, one warp per token, 8 values per lane per pass);
+// dtable[ids[n]] += dX[n] (16-byte fp32 vector atomics, one warp per token, 8 values per
+// lane per pass);
 // with dt, dt_table[bucket(dt[n])] += dX[n] through a per-block [16, d] shared
 // accumulator, so that the 16 bucket rows take one atomic per block and column.
 __global__ void __launch_bounds__(256) table_rows_bwd_kernel(const bf16* __restrict__ dX, int M, int d,
@@ -322,17 +323,21 @@ __global__ void __launch_bounds__(256) table_rows_bwd_kernel(const bf16* __restr
     for (int c = lane * 8; c < d; c += 256) {
       const uint4 u = *reinterpret_cast<const uint4*>(dX + int64_t(r) * d + c);
       const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+      float f[8];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float2 f = __bfloat1622float2(h2[j]);
-        if (ok) {
-          atomicAdd(dtable + id * d + c + 2 * j, f.x);
-          atomicAdd(dtable + id * d + c + 2 * j + 1, f.y);
-        }
-        if (with_dt) {
-          atomicAdd(bucket_acc + b * d + c + 2 * j, f.x);
-          atomicAdd(bucket_acc + b * d + c + 2 * j + 1, f.y);
-        }
+        const float2 t = __bfloat1622float2(h2[j]);
+        f[2 * j] = t.x;
+        f[2 * j + 1] = t.y;
+      }
+      if (ok) {  // 16-byte vector reductions: a quarter of the atomic operations on hot rows
+        float4* row = reinterpret_cast<float4*>(dtable + id * d + c);
+        atomicAdd(row, make_float4(f[0], f[1], f[2], f[3]));
+        atomicAdd(row + 1, make_float4(f[4], f[5], f[6], f[7]));
+      }
+      if (with_dt) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) atomicAdd(bucket_acc + b * d + c + j, f[j]);
       }
     }
   }
@@ -437,7 +442,8 @@ int table_rows_bwd(const void* dX, int M, int d, const int32_t* ids, const int32
                    float* dtable, float* ddt_table, int32_t* err, cudaStream_t s) {
   if (M < 0 || d <= 0 || d % 8 || n_items <= 0) return STCA_ERR_INVALID_ARG;
   if (M == 0) return STCA_OK;
-  if (!dX || !ids || !dtable || (reinterpret_cast<uintptr_t>(dX) & 15)) return STCA_ERR_INVALID_ARG;
+  if (!dX || !ids || !dtable || ((reinterpret_cast<uintptr_t>(dX) | reinterpret_cast<uintptr_t>(dtable)) & 15))
+    return STCA_ERR_INVALID_ARG;
   const bool with_dt = dt && ddt_table;
   const size_t smem = with_dt ? size_t(16) * d * 4 : 0;
   if (smem > 48 * 1024) return STCA_ERR_UNSUPPORTED;

@@ -1,5 +1,6 @@
 """Backward of one layer's history side on the GPU (X -> LN(SwiGLU(X)) -> [K | V], then the
-lookup), composed from the library's kernel-level entries, against the fp64 oracle
+lookup), as ``target_attention_b200.training.HistoryLayerBackward`` composes it from the
+library's kernel-level entries, against the fp64 oracle
 (``stca_grad.history_layer_bwd`` and ``table_rows_bwd``) on the same bf16 inputs.
 
 The forward values the backward needs are recomputed on the GPU the way a training step
@@ -15,7 +16,8 @@ import torch
 from oracle import stca_grad as G
 from oracle import stca_ref as R
 from target_attention_b200 import binding as B
-from tests._util import bf16_to_f64, zeros_err
+from target_attention_b200.training import HistoryLayerBackward
+from tests._util import bf16_to_f64
 from workloads import make_stca
 
 pytestmark = pytest.mark.gpu
@@ -105,60 +107,20 @@ def test_history_layer_backward_matches_oracle(config):
     dt_t = torch.from_numpy(dt.astype(np.int32)).to(dev) if dt is not None else None
     gamma = torch.from_numpy(R.to_f64(ffn["gamma"]).astype(np.float32)).to(dev)
     beta = torch.from_numpy(R.to_f64(ffn["beta"]).astype(np.float32)).to(dev)
-    err = zeros_err()
     n_items = int(wl["table"].shape[0])
-    bf = lambda *shape: torch.empty(shape, dtype=torch.bfloat16, device=dev)
-    # ---- forward values, recomputed
-    W13p = bf(2 * h, d)                                   # SwiGLU operand (packed modes 1 + 2)
-    B.check(B.stca_k_pack_weight(W1, d, h, W13p, 1, 0))
-    B.check(B.stca_k_pack_weight(W3, d, h, W13p, 2, 0))
-    X, A = bf(M, d), bf(M, h)
-    B.check(B.stca_k_gemm_resident(1, 1, None, ids_t, dt_t, table, dtab, n_items, M, d, W13p, h, A, h, err, x_out=X))
-    Pp = bf(2 * h, d)                                     # [x W1 | x W3] operand (mode 0)
-    B.check(B.stca_k_pack_weight(W1, d, h, Pp, 0, 0))
-    B.check(B.stca_k_pack_weight(W3, d, h, Pp, 0, h))
-    P = bf(M, 2 * h)
-    B.check(B.stca_k_gemm_resident(0, 0, X, None, None, None, None, 0, M, d, Pp, 2 * h, P, 2 * h, err))
-    W2p = bf(d, h)
-    B.check(B.stca_k_pack_weight(W2, h, d, W2p, 0, 0))
-    y = bf(M, d)
-    B.check(B.stca_k_gemm_rowwise(0, A, M, h, W2p, d, None, None, eps, y, d, err))
-    # ---- backward
+    # ---- forward values recomputed, then the backward (target_attention_b200.training)
+    layer = HistoryLayerBackward(M, d, h, W1, W3, W2, up16(WK), up16(WV), gamma, beta, eps)
+    layer.recompute(ids_t, dt_t, table, dtab, n_items)
     dKV = np.zeros((M, 2 * d))
     for hh in range(d // 64):                            # the K/V rows' [K_h | V_h] columns
         dKV[:, 128 * hh:128 * hh + 64] = dK[:, 64 * hh:64 * hh + 64]
         dKV[:, 128 * hh + 64:128 * hh + 128] = dV[:, 64 * hh:64 * hh + 64]
-    dKV_t = to_bf16(dKV)
-    WKVi = bf(d, 2 * d)
-    B.check(B.stca_k_pack_weight(up16(WK), d, d, WKVi, 3, 0))
-    B.check(B.stca_k_pack_weight(up16(WV), d, d, WKVi, 3, 64))
-    dXt = bf(M, d)
-    B.check(B.stca_k_gemm_rowwise(0, dKV_t, M, 2 * d, WKVi, d, None, None, eps, dXt, d, err))
-    dy, Xt = bf(M, d), bf(M, d)
-    dgamma, dbeta = torch.empty(d, device=dev), torch.empty(d, device=dev)
-    wln = ws(B.stca_k_layer_norm_bwd_workspace_bytes(M, d))
-    B.check(B.stca_k_layer_norm_bwd(y, dXt, M, d, gamma, beta, eps, dy, Xt, dgamma, dbeta, 0, wln, wln.numel()))
-    dWKV = torch.empty((d, 2 * d), device=dev)
-    wg = ws(max(B.stca_k_gemm_wgrad_workspace_bytes(M, K, N) for K, N in ((d, 2 * d), (h, d), (d, 2 * h))))
-    B.check(B.stca_k_gemm_wgrad(Xt, d, dKV_t, 2 * d, M, d, 2 * d, dWKV, 2 * d, 0, wg, wg.numel()))
-    dA = bf(M, h)                                        # dy W2^T: W2 itself is the operand
-    B.check(B.stca_k_gemm_resident(0, 0, dy, None, None, None, None, 0, M, d, W2, h, dA, h, err))
-    dW2 = torch.empty((h, d), device=dev)
-    B.check(B.stca_k_gemm_wgrad(A, h, dy, d, M, h, d, dW2, d, 0, wg, wg.numel()))
-    dP = bf(M, 2 * h)
-    B.check(B.stca_k_swiglu_bwd(P, dA, M, h, dP, None))
-    W13c = bf(d, 2 * h)                                  # [W1 | W3] side by side
-    B.check(B.stca_k_pack_weight(W1, d, h, W13c, 4, 0))
-    B.check(B.stca_k_pack_weight(W3, d, h, W13c, 4, h))
-    dX = bf(M, d)
-    B.check(B.stca_k_gemm_rowwise(0, dP, M, 2 * h, W13c, d, None, None, eps, dX, d, err))
-    dW13 = torch.empty((d, 2 * h), device=dev)
-    B.check(B.stca_k_gemm_wgrad(X, d, dP, 2 * h, M, d, 2 * h, dW13, 2 * h, 0, wg, wg.numel()))
     dtable = torch.zeros((n_items, d), device=dev)
     ddt = torch.zeros((16, d), device=dev) if dt is not None else None
-    B.check(B.stca_k_table_rows_bwd(dX, M, d, ids_t, dt_t, n_items, dtable, ddt, err))
+    layer.backward(to_bf16(dKV), ids_t, dt_t, n_items, dtable, ddt)
     torch.cuda.synchronize()
-    assert err.item() == 0
+    assert layer.err.item() == 0
+    dWKV, dW2, dW13, dgamma, dbeta, dX = layer.dWKV, layer.dW2, layer.dW13, layer.dgamma, layer.dbeta, layer.dX
     # ---- oracle on the same stored values
     X64 = R.gather_history(wl["table"], ids, dt, wl.get("dt_table"))
     rdX, rg = G.history_layer_bwd(X64, ffn, WK, WV, eps, dK, dV)
