@@ -43,7 +43,8 @@ def normwise(got, ref):
     return float(np.abs(np.asarray(got, np.float64) - ref).max() / max(np.abs(ref).max(), 1e-30))
 
 
-@pytest.mark.parametrize("M, K, N, lda_pad", [(1000, 128, 128, 0), (5003, 256, 512, 8), (77, 512, 256, 0)])
+@pytest.mark.parametrize("M, K, N, lda_pad", [(1000, 128, 128, 0), (5003, 256, 512, 8), (77, 512, 256, 0),
+                                               (40_000, 128, 768, 0), (300, 384, 256, 16)])
 def test_gemm_wgrad_matches_float64(M, K, N, lda_pad):
     """C = A^T G over ragged token counts (a partial last stage, several token slices),
     padded leading dimensions, and C += A^T G with accumulate."""
