@@ -122,21 +122,32 @@ size_t stca_k_gemm_wgrad_workspace_bytes(int M, int K, int N);
 int stca_k_gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, int M, int K, int N, float* C,
                       int64_t ldc, int accumulate, void* ws, size_t ws_bytes, void* stream);
 
-/* LayerNorm backward over rows of d = 256 or 512 (biased variance, eps): y [M, d] bf16 the
- * LayerNorm's input, dxt [M, d] bf16 the gradient of its output, gamma (beta may be NULL)
- * [d] fp32.  Writes dy [M, d] bf16 and, when xt is not NULL, the output xt = LN(y) [M, d]
- * bf16 (for the K/V weight gradients); dgamma, dbeta [d] fp32 are set (accumulate: added
- * to).  ws: at least stca_k_layer_norm_bwd_workspace_bytes(M, d) bytes. */
+/* LayerNorm backward over rows of d = 256 or 512 (biased variance, eps): y [M, d] the
+ * LayerNorm's input, dxt [M, d] the gradient of its output (bf16, or fp32 when fp32 != 0:
+ * the target side keeps fp32 rows), gamma (beta may be NULL) [d] fp32.  Writes dy [M, d]
+ * and, when xt is not NULL, the output xt = LN(y) [M, d] in the same type (for the K/V
+ * weight gradients); dgamma, dbeta [d] fp32 are set (accumulate: added to).  Rows dense.
+ * ws: at least stca_k_layer_norm_bwd_workspace_bytes(M, d) bytes. */
 size_t stca_k_layer_norm_bwd_workspace_bytes(int M, int d);
-int stca_k_layer_norm_bwd(const void* y, const void* dxt, int M, int d, const float* gamma, const float* beta,
-                          float eps, void* dy, void* xt, float* dgamma, float* dbeta, int accumulate, void* ws,
-                          size_t ws_bytes, void* stream);
+int stca_k_layer_norm_bwd(const void* y, const void* dxt, int M, int d, int fp32, const float* gamma,
+                          const float* beta, float eps, void* dy, void* xt, float* dgamma, float* dbeta,
+                          int accumulate, void* ws, size_t ws_bytes, void* stream);
 
-/* SwiGLU backward: A = SiLU(P1) * P3 with P = [P1 | P3] [M, 2h] bf16 (x W1 and x W3 side by
- * side) and dA [M, h] bf16.  Writes dP = [dP1 | dP3] [M, 2h] bf16 with dP1 = dA P3 SiLU'(P1),
- * dP3 = dA SiLU(P1), and A [M, h] bf16 into a_out when not NULL.  h % 8 == 0, pointers
- * 16-byte aligned. */
-int stca_k_swiglu_bwd(const void* P, const void* dA, int M, int h, void* dP, void* a_out, void* stream);
+/* LayerNorm forward (biased variance, eps) of rows x [M, ldx] -> y [M, ldy], d = 256 or
+ * 512, both bf16 or both fp32 (x_fp32 = y_fp32; else STCA_ERR_UNSUPPORTED): the training
+ * step recomputes the forward's LayerNorm outputs with it. */
+int stca_k_layer_norm(const void* x, int64_t ldx, int x_fp32, int M, int d, const float* gamma, const float* beta,
+                      float eps, void* y, int64_t ldy, int y_fp32, void* stream);
+
+/* dst [rows, ldd] bf16 = src [rows, lds] fp32 rounded to nearest even (operands of the
+ * weight-gradient GEMM from the target side's fp32 rows). */
+int stca_k_f32_to_bf16(const float* src, int64_t lds, int rows, int cols, void* dst, int64_t ldd, void* stream);
+
+/* SwiGLU backward: A = SiLU(P1) * P3 with P = [P1 | P3] [M, 2h] (x W1 and x W3 side by side)
+ * and dA [M, h], bf16 (fp32 when fp32 != 0).  Writes dP = [dP1 | dP3] [M, 2h] with
+ * dP1 = dA P3 SiLU'(P1), dP3 = dA SiLU(P1), and A [M, h] into a_out when not NULL, in the
+ * same type.  h % 8 == 0; bf16 pointers 16-byte aligned. */
+int stca_k_swiglu_bwd(const void* P, const void* dA, int M, int h, int fp32, void* dP, void* a_out, void* stream);
 
 /* The lookup's backward: dtable[ids[n]] += dX[n] for n < M (dX [M, d] bf16, dtable
  * [n_items, d] fp32) and, with dt and ddt_table, ddt_table[b(dt[n])] += dX[n] ([16, d] fp32,

@@ -113,9 +113,11 @@ _SIGS = [
     ("stca_k_gemm_wgrad_workspace_bytes", ctypes.c_size_t, [_i32, _i32, _i32]),
     ("stca_k_gemm_wgrad", _i32, [_vp, _i64, _vp, _i64, _i32, _i32, _i32, _vp, _i64, _i32, _vp, ctypes.c_size_t, _vp]),
     ("stca_k_layer_norm_bwd_workspace_bytes", ctypes.c_size_t, [_i32, _i32]),
-    ("stca_k_layer_norm_bwd", _i32, [_vp, _vp, _i32, _i32, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _i32, _vp,
-                                     ctypes.c_size_t, _vp]),
-    ("stca_k_swiglu_bwd", _i32, [_vp, _vp, _i32, _i32, _vp, _vp, _vp]),
+    ("stca_k_layer_norm_bwd", _i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _i32,
+                                     _vp, ctypes.c_size_t, _vp]),
+    ("stca_k_layer_norm", _i32, [_vp, _i64, _i32, _i32, _i32, _vp, _vp, ctypes.c_float, _vp, _i64, _i32, _vp]),
+    ("stca_k_f32_to_bf16", _i32, [_vp, _i64, _i32, _i32, _vp, _i64, _vp]),
+    ("stca_k_swiglu_bwd", _i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     ("stca_k_table_rows_bwd", _i32, [_vp, _i32, _i32, _vp, _vp, _i64, _vp, _vp, _vp, _vp]),
     ("stca_k_dedup_workspace_bytes", ctypes.c_size_t, [_i32]),
     ("stca_k_dedup", _i32, [_vp, _vp, _i32, _vp, ctypes.c_size_t, _vp, _vp, _vp, _vp, _vp]),
@@ -355,13 +357,22 @@ def stca_k_layer_norm_bwd_workspace_bytes(M, d) -> int:
 
 
 def stca_k_layer_norm_bwd(y, dxt, M, d, gamma, beta, eps, dy, xt, dgamma, dbeta, accumulate, ws, ws_bytes,
-                          stream=None) -> int:
-    return lib().stca_k_layer_norm_bwd(ptr(y), ptr(dxt), M, d, ptr(gamma), ptr(beta), eps, ptr(dy), ptr(xt),
+                          stream=None, fp32=0) -> int:
+    return lib().stca_k_layer_norm_bwd(ptr(y), ptr(dxt), M, d, fp32, ptr(gamma), ptr(beta), eps, ptr(dy), ptr(xt),
                                        ptr(dgamma), ptr(dbeta), accumulate, ptr(ws), ws_bytes, stream_ptr(stream))
 
 
-def stca_k_swiglu_bwd(P, dA, M, h, dP, a_out, stream=None) -> int:
-    return lib().stca_k_swiglu_bwd(ptr(P), ptr(dA), M, h, ptr(dP), ptr(a_out), stream_ptr(stream))
+def stca_k_layer_norm(x, ldx, x_fp32, M, d, gamma, beta, eps, y, ldy, y_fp32, stream=None) -> int:
+    return lib().stca_k_layer_norm(ptr(x), ldx, x_fp32, M, d, ptr(gamma), ptr(beta), eps, ptr(y), ldy, y_fp32,
+                                   stream_ptr(stream))
+
+
+def stca_k_f32_to_bf16(src, lds, rows, cols, dst, ldd, stream=None) -> int:
+    return lib().stca_k_f32_to_bf16(ptr(src), lds, rows, cols, ptr(dst), ldd, stream_ptr(stream))
+
+
+def stca_k_swiglu_bwd(P, dA, M, h, dP, a_out, stream=None, fp32=0) -> int:
+    return lib().stca_k_swiglu_bwd(ptr(P), ptr(dA), M, h, fp32, ptr(dP), ptr(a_out), stream_ptr(stream))
 
 
 def stca_k_table_rows_bwd(dX, M, d, ids, dt, n_items, dtable, ddt_table, err, stream=None) -> int:

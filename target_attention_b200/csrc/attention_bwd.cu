@@ -17,7 +17,8 @@
 // kernel (one slice writes dQ directly).
 //
 // A CTA of 4 warps serves one (user, slice, head).  Queries go in chunks of 16: Q (scaled
-// by c) and dO of the chunk sit in shared memory as bf16 tiles.  Each warp streams its own
+// by c), the scores' query operand (formed as the forward forms it) and dO of the chunk
+// sit in shared memory as bf16 tiles.  Each warp streams its own
 // 16-key tiles (keys w, w + 4, ... of the slice) through a 3-stage cp.async ring and, with
 // the keys as the MMA row dimension (mma.sync m16n8k16, fp32 accumulation):
 //   S^T = K Q^T, dP^T = V dO^T   ->  P^T, dS^T in registers
@@ -48,7 +49,8 @@ constexpr int OFF_DO = OFF_Q + BQBYTES;
 constexpr int OFF_DS = OFF_DO + BQBYTES;
 constexpr int OFF_D = OFF_DS + BW * BDS;
 constexpr int OFF_L = OFF_D + BQ * 4;
-constexpr int BWD_SMEM = OFF_L + BQ * 4;
+constexpr int OFF_Q2 = OFF_L + BQ * 4;          // the scores' own query tile (see the fill below)
+constexpr int BWD_SMEM = OFF_Q2 + BQBYTES;
 static_assert(BW * BQ * BD * 4 <= BRING, "the dQ combine reuses the ring");
 
 // Byte offset of 16-byte chunk ch (0..7) of row r in a tile of 128-byte rows (64 bf16),
@@ -96,7 +98,7 @@ __global__ void __launch_bounds__(B_THREADS, 4) attn_bwd_kernel(BwdArgs a) {
   const int n_tiles = (nk + BKT - 1) / BKT;
   const int n_local = n_tiles > warp ? (n_tiles - warp + BW - 1) / BW : 0;
   uint8_t* ring = smem + warp * BSTAGES * BSTAGE;
-  const uint32_t sQ = smem_u32(smem + OFF_Q), sO = smem_u32(smem + OFF_DO);
+  const uint32_t sQ = smem_u32(smem + OFF_Q), sO = smem_u32(smem + OFF_DO), sQ2 = smem_u32(smem + OFF_Q2);
   uint8_t* dS_tile = smem + OFF_DS + warp * BDS;
   float* Ds = reinterpret_cast<float*>(smem + OFF_D);
   float* Ls = reinterpret_cast<float*>(smem + OFF_L);
@@ -122,29 +124,56 @@ __global__ void __launch_bounds__(B_THREADS, 4) attn_bwd_kernel(BwdArgs a) {
   for (int qp = 0; qp < m; qp += BQ) {
     const int mq = min(BQ, m - qp);
     __syncthreads();  // the previous chunk is done with every shared buffer
-    // ---- Q (scaled by c) and dO of the chunk as bf16 tiles; D = dO . O; lse in log2 units
+    // ---- Q and dO of the chunk as bf16 tiles; D = dO . O; lse in log2 units.  The scores
+    // are recomputed exactly as the forward formed them, so that the forward's lse
+    // normalises these weights (softmax) and the mask [s > 0] is the forward's (ReLU): Q2
+    // holds bf16(q c log2e) for the softmax (the forward's query operand), and for the ReLU
+    // the low terms bf16(q c - bf16(q c)) that the forward adds to Q = bf16(q c).  dK takes Q.
+    const float qs2 = B_LOG2E * c;
     for (int i = threadIdx.x; i < BQ * 8; i += B_THREADS) {
       const int r = i >> 3, ch = i & 7;
-      uint4 qv = make_uint4(0, 0, 0, 0), ov = qv;
+      uint4 qv = make_uint4(0, 0, 0, 0), ov = qv, q2 = qv;
       if (r < mq) {
         const int64_t off = int64_t(t0 + qp + r) * d + qcol + ch * 8;
         const float4 q0 = *reinterpret_cast<const float4*>(a.Q + off);
         const float4 q1 = *reinterpret_cast<const float4*>(a.Q + off + 4);
         const float4 o0 = *reinterpret_cast<const float4*>(a.dO + off);
         const float4 o1 = *reinterpret_cast<const float4*>(a.dO + off + 4);
-        qv = make_uint4(pack_bf16x2(q0.x * c, q0.y * c), pack_bf16x2(q0.z * c, q0.w * c),
-                        pack_bf16x2(q1.x * c, q1.y * c), pack_bf16x2(q1.z * c, q1.w * c));
+        const float x[8] = {q0.x * c, q0.y * c, q0.z * c, q0.w * c, q1.x * c, q1.y * c, q1.z * c, q1.w * c};
+        qv = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                        pack_bf16x2(x[6], x[7]));
+        if (SCORE == 0) {
+          const float y[8] = {q0.x * qs2, q0.y * qs2, q0.z * qs2, q0.w * qs2,
+                              q1.x * qs2, q1.y * qs2, q1.z * qs2, q1.w * qs2};
+          q2 = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                          pack_bf16x2(y[6], y[7]));
+        } else {
+          const uint32_t hw[4] = {qv.x, qv.y, qv.z, qv.w};
+          uint32_t lw[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 hf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[k]));
+            lw[k] = pack_bf16x2(x[2 * k] - hf.x, x[2 * k + 1] - hf.y);
+          }
+          q2 = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
         ov = make_uint4(pack_bf16x2(o0.x, o0.y), pack_bf16x2(o0.z, o0.w), pack_bf16x2(o1.x, o1.y),
                         pack_bf16x2(o1.z, o1.w));
       }
       *reinterpret_cast<uint4*>(smem + OFF_Q + sw128(r, ch)) = qv;
+      *reinterpret_cast<uint4*>(smem + OFF_Q2 + sw128(r, ch)) = q2;
       *reinterpret_cast<uint4*>(smem + OFF_DO + sw128(r, ch)) = ov;
     }
     for (int r = warp; r < BQ; r += BW) {
       float dsum = 0.f;
       if (r < mq) {
         const int64_t off = int64_t(t0 + qp + r) * d + qcol;
-        dsum = a.dO[off + lane] * a.O[off + lane] + a.dO[off + lane + 32] * a.O[off + lane + 32];
+        // dO rounded to bf16 as the dP^T MMA sees it: with D and dP from the same dO, ds is
+        // the softmax Jacobian applied to that dO.  (With fp32 dO here and bf16 dO in dP the
+        // rounding error times the values' common offset no longer cancels in dp - D.)
+        const float g0 = __bfloat162float(__float2bfloat16_rn(a.dO[off + lane]));
+        const float g1 = __bfloat162float(__float2bfloat16_rn(a.dO[off + lane + 32]));
+        dsum = g0 * a.O[off + lane] + g1 * a.O[off + lane + 32];
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
@@ -201,10 +230,15 @@ __global__ void __launch_bounds__(B_THREADS, 4) attn_bwd_kernel(BwdArgs a) {
         uint32_t ka[4], va[4], qb[4], ob[4];
         ldsm_x4(sK + sw128(ar, 2 * kk + (lane >> 4)), ka);
         ldsm_x4(sV + sw128(ar, 2 * kk + (lane >> 4)), va);
-        ldsm_x4(sQ + sw128(br, 2 * kk + ((lane >> 3) & 1)), qb);
+        ldsm_x4(sQ2 + sw128(br, 2 * kk + ((lane >> 3) & 1)), qb);
         ldsm_x4(sO + sw128(br, 2 * kk + ((lane >> 3) & 1)), ob);
         mma_bf16_16816(sT[0], ka, qb[0], qb[1]);
         mma_bf16_16816(sT[1], ka, qb[2], qb[3]);
+        if (SCORE == 1) {  // + the high terms: s = K (Q + Q2)
+          ldsm_x4(sQ + sw128(br, 2 * kk + ((lane >> 3) & 1)), qb);
+          mma_bf16_16816(sT[0], ka, qb[0], qb[1]);
+          mma_bf16_16816(sT[1], ka, qb[2], qb[3]);
+        }
         mma_bf16_16816(dpT[0], va, ob[0], ob[1]);
         mma_bf16_16816(dpT[1], va, ob[2], ob[3]);
       }
@@ -217,7 +251,7 @@ __global__ void __launch_bounds__(B_THREADS, 4) attn_bwd_kernel(BwdArgs a) {
           const bool kok = g + (e >> 1) * 8 < valid;
           const int qi = nt * 2 + (e & 1);
           if (SCORE == 0) {
-            const float p = kok ? exp2_approx(sT[nt][e] * B_LOG2E - lse2[qi]) : 0.f;
+            const float p = kok ? exp2_approx(sT[nt][e] - lse2[qi]) : 0.f;  // scores in log2 units
             pT[nt][e] = p;
             dsT[nt][e] = p * (dpT[nt][e] - Dq[qi]);
           } else {

@@ -286,10 +286,13 @@ size_t gemm_wgrad_workspace_bytes(int M, int K, int N);
 int gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, int M, int K, int N, float* C, int64_t ldc,
                int accumulate, void* ws, size_t ws_bytes, cudaStream_t s);
 size_t layer_norm_bwd_workspace_bytes(int M, int d);
-int layer_norm_bwd(const void* y, const void* dxt, int M, int d, const float* gamma, const float* beta, float eps,
-                   void* dy, void* xt, float* dgamma, float* dbeta, int accumulate, void* ws, size_t ws_bytes,
-                   cudaStream_t s);
-int swiglu_bwd(const void* P, const void* dA, int M, int h, void* dP, void* a_out, cudaStream_t s);
+int layer_norm_bwd(const void* y, const void* dxt, int M, int d, int fp32, const float* gamma, const float* beta,
+                   float eps, void* dy, void* xt, float* dgamma, float* dbeta, int accumulate, void* ws,
+                   size_t ws_bytes, cudaStream_t s);
+int swiglu_bwd(const void* P, const void* dA, int M, int h, int fp32, void* dP, void* a_out, cudaStream_t s);
+int layer_norm_fwd(const void* x, int64_t ldx, int x_fp32, int M, int d, const float* gamma, const float* beta,
+                   float eps, void* y, int64_t ldy, int y_fp32, cudaStream_t s);
+int f32_to_bf16(const float* src, int64_t lds, int rows, int cols, void* dst, int64_t ldd, cudaStream_t s);
 int table_rows_bwd(const void* dX, int M, int d, const int32_t* ids, const int32_t* dt, int64_t n_items,
                    float* dtable, float* ddt_table, int32_t* err, cudaStream_t s);
 int place_cols(const void* W, int K, int N, void* dst, int mode, int off, cudaStream_t s);

@@ -55,15 +55,24 @@ int stca_k_gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, in
 
 size_t stca_k_layer_norm_bwd_workspace_bytes(int M, int d) { return M < 0 ? 0 : layer_norm_bwd_workspace_bytes(M, d); }
 
-int stca_k_layer_norm_bwd(const void* y, const void* dxt, int M, int d, const float* gamma, const float* beta,
-                          float eps, void* dy, void* xt, float* dgamma, float* dbeta, int accumulate, void* ws,
-                          size_t ws_bytes, void* stream) {
-  return layer_norm_bwd(y, dxt, M, d, gamma, beta, eps, dy, xt, dgamma, dbeta, accumulate, ws, ws_bytes,
+int stca_k_layer_norm_bwd(const void* y, const void* dxt, int M, int d, int fp32, const float* gamma,
+                          const float* beta, float eps, void* dy, void* xt, float* dgamma, float* dbeta,
+                          int accumulate, void* ws, size_t ws_bytes, void* stream) {
+  return layer_norm_bwd(y, dxt, M, d, fp32, gamma, beta, eps, dy, xt, dgamma, dbeta, accumulate, ws, ws_bytes,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
-int stca_k_swiglu_bwd(const void* P, const void* dA, int M, int h, void* dP, void* a_out, void* stream) {
-  return swiglu_bwd(P, dA, M, h, dP, a_out, reinterpret_cast<cudaStream_t>(stream));
+int stca_k_layer_norm(const void* x, int64_t ldx, int x_fp32, int M, int d, const float* gamma, const float* beta,
+                      float eps, void* y, int64_t ldy, int y_fp32, void* stream) {
+  return layer_norm_fwd(x, ldx, x_fp32, M, d, gamma, beta, eps, y, ldy, y_fp32, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int stca_k_swiglu_bwd(const void* P, const void* dA, int M, int h, int fp32, void* dP, void* a_out, void* stream) {
+  return swiglu_bwd(P, dA, M, h, fp32, dP, a_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int stca_k_f32_to_bf16(const float* src, int64_t lds, int rows, int cols, void* dst, int64_t ldd, void* stream) {
+  return f32_to_bf16(src, lds, rows, cols, dst, ldd, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int stca_k_table_rows_bwd(const void* dX, int M, int d, const int32_t* ids, const int32_t* dt, int64_t n_items,

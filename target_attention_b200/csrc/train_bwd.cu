@@ -169,10 +169,16 @@ int wgrad_splits(int M, int K, int N) {
 // xhat = (y - mean) rstd and g = dxt * gamma:
 //   dy = rstd (g - mean(g) - xhat mean(g xhat)),  xt = xhat gamma + beta,
 //   dgamma += dxt xhat,  dbeta += dxt  (over the rows; per block, then added in order).
-template <int DPL>
-__global__ void __launch_bounds__(256) ln_bwd_kernel(const bf16* __restrict__ y, const bf16* __restrict__ dxt, int M,
+__device__ __forceinline__ float ld_f(const bf16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ float ld_f(const float* p) { return *p; }
+__device__ __forceinline__ void st_f(bf16* p, float v) { *p = __float2bfloat16(v); }
+__device__ __forceinline__ void st_f(float* p, float v) { *p = v; }
+
+// rows of bf16 (the history side) or fp32 (the target side, which keeps fp32 activations)
+template <int DPL, typename T>
+__global__ void __launch_bounds__(256) ln_bwd_kernel(const T* __restrict__ y, const T* __restrict__ dxt, int M,
                                                      const float* __restrict__ gamma, const float* __restrict__ beta,
-                                                     float eps, bf16* __restrict__ dy, bf16* __restrict__ xt,
+                                                     float eps, T* __restrict__ dy, T* __restrict__ xt,
                                                      float* __restrict__ part) {
   griddep_wait();
   constexpr int D = 32 * DPL;
@@ -193,8 +199,8 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const bf16* __restrict__ y,
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < DPL; ++i) {
-      v[i] = __bfloat162float(y[int64_t(r) * D + lane + 32 * i]);
-      dv[i] = __bfloat162float(dxt[int64_t(r) * D + lane + 32 * i]);
+      v[i] = ld_f(y + int64_t(r) * D + lane + 32 * i);
+      dv[i] = ld_f(dxt + int64_t(r) * D + lane + 32 * i);
       s += v[i];
     }
 #pragma unroll
@@ -228,8 +234,8 @@ __global__ void __launch_bounds__(256) ln_bwd_kernel(const bf16* __restrict__ y,
     m2 /= D;
 #pragma unroll
     for (int i = 0; i < DPL; ++i) {
-      dy[int64_t(r) * D + lane + 32 * i] = __float2bfloat16(rstd * (gv[i] - m1 - v[i] * m2));
-      if (xt) xt[int64_t(r) * D + lane + 32 * i] = __float2bfloat16(v[i] * gm[i] + bt[i]);
+      st_f(dy + int64_t(r) * D + lane + 32 * i, rstd * (gv[i] - m1 - v[i] * m2));
+      if (xt) st_f(xt + int64_t(r) * D + lane + 32 * i, v[i] * gm[i] + bt[i]);
     }
   }
   griddep_launch();
@@ -293,6 +299,69 @@ __global__ void swiglu_bwd_kernel(const bf16* __restrict__ P, const bf16* __rest
     *reinterpret_cast<uint4*>(dP + r * 2 * h + c) = o1;
     *reinterpret_cast<uint4*>(dP + r * 2 * h + h + c) = o3;
     if (a_out) *reinterpret_cast<uint4*>(a_out + e) = oa;
+  }
+}
+
+// LayerNorm forward, one warp per row of d = 32 DPL (biased variance): the training step
+// recomputes the forward's LayerNorm outputs with it (bf16 history rows, fp32 target rows).
+template <int DPL, typename TI, typename TO>
+__global__ void __launch_bounds__(256) ln_fwd_kernel(const TI* __restrict__ x, int64_t ldx, int M,
+                                                     const float* __restrict__ gamma, const float* __restrict__ beta,
+                                                     float eps, TO* __restrict__ y, int64_t ldy) {
+  griddep_wait();
+  constexpr int D = 32 * DPL;
+  const int lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r < M) {
+    float v[DPL];
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      v[i] = ld_f(x + int64_t(r) * ldx + lane + 32 * i);
+      s += v[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / D;
+    float q = 0.f;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      v[i] -= mean;
+      q += v[i] * v[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+    const float rstd = rsqrtf(q / D + eps);
+#pragma unroll
+    for (int i = 0; i < DPL; ++i)
+      st_f(y + int64_t(r) * ldy + lane + 32 * i, v[i] * rstd * gamma[lane + 32 * i] + (beta ? beta[lane + 32 * i] : 0.f));
+  }
+  griddep_launch();
+}
+
+// SwiGLU backward on fp32 rows (the target side): as swiglu_bwd_kernel, one value per thread
+__global__ void swiglu_bwd_f32_kernel(const float* __restrict__ P, const float* __restrict__ dA, int64_t M, int h,
+                                      float* __restrict__ dP, float* __restrict__ a_out) {
+  griddep_wait();
+  const int64_t n = M * h;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = e / h, c = e % h;
+    const float a = P[r * 2 * h + c], b = P[r * 2 * h + h + c], d = dA[e];
+    const float sg = 1.f / (1.f + __expf(-a)), f = a * sg;
+    dP[r * 2 * h + c] = d * b * sg * (1.f + a * (1.f - sg));
+    dP[r * 2 * h + h + c] = d * f;
+    if (a_out) a_out[e] = f * b;
+  }
+}
+
+// dst [rows, cols] bf16 (ld ldd) = round-to-nearest-even of src [rows, cols] fp32 (ld lds)
+__global__ void f32_to_bf16_kernel(const float* __restrict__ src, int64_t lds, int rows, int cols,
+                                   bf16* __restrict__ dst, int64_t ldd) {
+  griddep_wait();
+  const int64_t n = int64_t(rows) * cols;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = e / cols, c = e % cols;
+    dst[r * ldd + c] = __float2bfloat16(src[r * lds + c]);
   }
 }
 
@@ -401,18 +470,25 @@ int ln_bwd_blocks(int M) { return std::max(1, std::min(2 * sm_count(), (M + 31) 
 
 size_t layer_norm_bwd_workspace_bytes(int M, int d) { return size_t(ln_bwd_blocks(M)) * 2 * d * 4; }
 
-int layer_norm_bwd(const void* y, const void* dxt, int M, int d, const float* gamma, const float* beta, float eps,
-                   void* dy, void* xt, float* dgamma, float* dbeta, int accumulate, void* ws, size_t ws_bytes,
-                   cudaStream_t s) {
+template <typename T>
+static cudaError_t launch_ln_bwd(int d, int blocks, cudaStream_t s, const void* y, const void* dxt, int M,
+                                 const float* gamma, const float* beta, float eps, void* dy, void* xt, float* part) {
+  auto kern = d == 256 ? ln_bwd_kernel<8, T> : ln_bwd_kernel<16, T>;
+  return launch_dep(kern, dim3(blocks), dim3(256), 0, s, static_cast<const T*>(y), static_cast<const T*>(dxt), M,
+                    gamma, beta, eps, static_cast<T*>(dy), static_cast<T*>(xt), part);
+}
+
+int layer_norm_bwd(const void* y, const void* dxt, int M, int d, int fp32, const float* gamma, const float* beta,
+                   float eps, void* dy, void* xt, float* dgamma, float* dbeta, int accumulate, void* ws,
+                   size_t ws_bytes, cudaStream_t s) {
   if (M < 0 || (d != 256 && d != 512)) return STCA_ERR_UNSUPPORTED;
   if (!gamma || !dgamma || !dbeta || (M > 0 && (!y || !dxt || !dy))) return STCA_ERR_INVALID_ARG;
   const int blocks = ln_bwd_blocks(M);
   if (ws_bytes < size_t(blocks) * 2 * d * 4 || !ws) return STCA_ERR_CAPACITY;
   float* part = static_cast<float*>(ws);
-  auto kern = d == 256 ? ln_bwd_kernel<8> : ln_bwd_kernel<16>;
-  if (launch_dep(kern, dim3(blocks), dim3(256), 0, s, static_cast<const bf16*>(y), static_cast<const bf16*>(dxt), M,
-                 gamma, beta, eps, static_cast<bf16*>(dy), static_cast<bf16*>(xt), part) != cudaSuccess)
-    return STCA_ERR_CUDA;
+  const cudaError_t e = fp32 ? launch_ln_bwd<float>(d, blocks, s, y, dxt, M, gamma, beta, eps, dy, xt, part)
+                             : launch_ln_bwd<bf16>(d, blocks, s, y, dxt, M, gamma, beta, eps, dy, xt, part);
+  if (e != cudaSuccess) return STCA_ERR_CUDA;
   note_launch();
   if (launch_dep(ln_bwd_reduce_kernel, dim3((2 * d + 255) / 256), dim3(256), 0, s, static_cast<const float*>(part),
                  blocks, d, dgamma, dbeta, accumulate) != cudaSuccess)
@@ -421,10 +497,20 @@ int layer_norm_bwd(const void* y, const void* dxt, int M, int d, const float* ga
   return STCA_OK;
 }
 
-int swiglu_bwd(const void* P, const void* dA, int M, int h, void* dP, void* a_out, cudaStream_t s) {
+int swiglu_bwd(const void* P, const void* dA, int M, int h, int fp32, void* dP, void* a_out, cudaStream_t s) {
   if (M < 0 || h <= 0 || h % 8) return STCA_ERR_UNSUPPORTED;
   if (M == 0) return STCA_OK;
   if (!P || !dA || !dP) return STCA_ERR_INVALID_ARG;
+  if (fp32) {
+    const int64_t n = int64_t(M) * h;
+    const int blocks = int(std::min<int64_t>((n + 255) / 256, int64_t(8) * sm_count()));
+    if (launch_dep(swiglu_bwd_f32_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const float*>(P),
+                   static_cast<const float*>(dA), int64_t(M), h, static_cast<float*>(dP), static_cast<float*>(a_out)) !=
+        cudaSuccess)
+      return STCA_ERR_CUDA;
+    note_launch();
+    return STCA_OK;
+  }
   const uintptr_t al = reinterpret_cast<uintptr_t>(P) | reinterpret_cast<uintptr_t>(dA) |
                        reinterpret_cast<uintptr_t>(dP) | reinterpret_cast<uintptr_t>(a_out);
   if (al & 15) return STCA_ERR_INVALID_ARG;
@@ -433,6 +519,39 @@ int swiglu_bwd(const void* P, const void* dA, int M, int h, void* dP, void* a_ou
   if (launch_dep(swiglu_bwd_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const bf16*>(P),
                  static_cast<const bf16*>(dA), int64_t(M), h, static_cast<bf16*>(dP), static_cast<bf16*>(a_out)) !=
       cudaSuccess)
+    return STCA_ERR_CUDA;
+  note_launch();
+  return STCA_OK;
+}
+
+int layer_norm_fwd(const void* x, int64_t ldx, int x_fp32, int M, int d, const float* gamma, const float* beta,
+                   float eps, void* y, int64_t ldy, int y_fp32, cudaStream_t s) {
+  if (M < 0 || (d != 256 && d != 512)) return STCA_ERR_UNSUPPORTED;
+  if (M == 0) return STCA_OK;
+  if (!x || !y || !gamma || ldx < d || ldy < d) return STCA_ERR_INVALID_ARG;
+  const dim3 grid((M + 7) / 8), block(256);
+  cudaError_t e;
+  if (x_fp32 && y_fp32)
+    e = launch_dep(d == 256 ? ln_fwd_kernel<8, float, float> : ln_fwd_kernel<16, float, float>, grid, block, 0, s,
+                   static_cast<const float*>(x), ldx, M, gamma, beta, eps, static_cast<float*>(y), ldy);
+  else if (!x_fp32 && !y_fp32)
+    e = launch_dep(d == 256 ? ln_fwd_kernel<8, bf16, bf16> : ln_fwd_kernel<16, bf16, bf16>, grid, block, 0, s,
+                   static_cast<const bf16*>(x), ldx, M, gamma, beta, eps, static_cast<bf16*>(y), ldy);
+  else
+    return STCA_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return STCA_ERR_CUDA;
+  note_launch();
+  return STCA_OK;
+}
+
+int f32_to_bf16(const float* src, int64_t lds, int rows, int cols, void* dst, int64_t ldd, cudaStream_t s) {
+  if (rows < 0 || cols < 0 || lds < cols || ldd < cols) return STCA_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return STCA_OK;
+  if (!src || !dst) return STCA_ERR_INVALID_ARG;
+  const int64_t n = int64_t(rows) * cols;
+  const int blocks = int(std::min<int64_t>((n + 255) / 256, int64_t(8) * sm_count()));
+  if (launch_dep(f32_to_bf16_kernel, dim3(blocks), dim3(256), 0, s, src, lds, rows, cols, static_cast<bf16*>(dst),
+                 ldd) != cudaSuccess)
     return STCA_ERR_CUDA;
   note_launch();
   return STCA_OK;

@@ -97,3 +97,258 @@ def _stepper(on_step):
         if on_step is not None:
             on_step(what)
     return check
+
+
+class _Ffn:
+    """One fp32-activation SwiGLU FFN of the target side (y = (SiLU(x W1) * (x W3)) W2, then
+    an optional LayerNorm): the operand layouts its forward and backward GEMMs take."""
+
+    def __init__(self, f, d, h, device):
+        bf = lambda *s: torch.empty(s, dtype=torch.bfloat16, device=device)
+        self.f, self.d, self.h = f, d, h
+        self.P0, self.P12, self.W2p, self.W13c = bf(2 * h, d), bf(2 * h, d), bf(d, h), bf(d, 2 * h)
+        for args in ((f["W1"], d, h, self.P0, 0, 0), (f["W3"], d, h, self.P0, 0, h), (f["W1"], d, h, self.P12, 1, 0),
+                     (f["W3"], d, h, self.P12, 2, 0), (f["W2"], h, d, self.W2p, 0, 0),
+                     (f["W1"], d, h, self.W13c, 4, 0), (f["W3"], d, h, self.W13c, 4, h)):
+            B.check(B.stca_k_pack_weight(*args), "pack")
+
+
+class StcaTrainingStep:
+    """Gradients of L = sum_t dZ[t] . z[t] through the whole STCA forward (the pages train
+    it at about 2K-long histories: STCA notes, "短序列训练，长序列推理"), every step on the
+    library's kernels, one history row per token.
+
+    Forward values are recomputed: the history side per layer (HistoryLayerBackward's
+    recompute, then Xt = LN(y) and the K/V rows), the target side in fp32 rows (q^(1) =
+    LN(SwiGLU_t(x_t)); per layer Q = q W_Q, the attention with its log-sum-exp, o = obar W_O
+    written into the concatenation [o^(1) .. o^(M) | x_t]; q^(i+1) = LN(SwiGLU(cat W_C));
+    z = SwiGLU_Z(cat W_Z)).  The backward then runs in reverse: the z FFN, W_Z, per layer
+    W_O, the attention backward (dQ and the K/V rows' gradients), W_Q, the fusion FFN and W_C
+    or the layer-1 target FFN, and the history side of the layer.  The target side's
+    weight gradients reduce over the T target rows with the weight-gradient GEMM on bf16
+    copies of the fp32 rows.
+
+    w: the weights as device tensors in the structure of the workload's weights (bf16
+    matrices, fp32 LayerNorm parameters).  The caller writes x_t (fp32 [T, d]) into
+    ``x_t_slot()`` before ``run``.
+    """
+
+    def __init__(self, cfg, w, B_users, n_tok, T, device="cuda"):
+        d, h, M, H = cfg["d"], cfg["hidden"], cfg["M"], cfg["H"]
+        self.cfg, self.w, self.dev = cfg, w, device
+        self.d, self.h, self.M, self.H, self.B, self.N, self.T = d, h, M, H, B_users, n_tok, T
+        self.eps = float(cfg.get("ln_eps", 1e-5))
+        self.score = 0 if cfg["score"] == "softmax" else 1
+        f32 = lambda *s: torch.zeros(s, dtype=torch.float32, device=device)
+        bf = lambda *s: torch.empty(s, dtype=torch.bfloat16, device=device)
+        self.f32, self.bf = f32, bf
+        pk = lambda W, K, N: self._pack0(W, K, N)
+        # target side operands
+        self.WQp = [pk(w["WQ"][i], d, d) for i in range(M)]
+        self.WOp = [pk(w["WO"][i], d, d) for i in range(M)]
+        self.WCp = [None] + [pk(w["WC"][i], (i + 1) * d, d) for i in range(1, M)]
+        self.WZp = pk(w["WZ"], (M + 1) * d, d)
+        self.tgt = _Ffn(w["tgt"], d, h, device)
+        self.fuse = [None] + [_Ffn(w["fuse"][i], d, h, device) for i in range(1, M)]
+        self.zffn = _Ffn(w["zffn"], d, h, device)
+        # history side, one per layer, and the K/V rows' forward operand
+        self.hist = [HistoryLayerBackward(n_tok, d, h, w["hist"][i]["W1"], w["hist"][i]["W3"], w["hist"][i]["W2"],
+                                          w["WK"][i], w["WV"][i], w["hist"][i]["gamma"], w["hist"][i]["beta"],
+                                          self.eps, device) for i in range(M)]
+        self.KVp = [self._pack0(self.hist[i].WKVi, d, 2 * d) for i in range(M)]
+        self.KV = [bf(max(n_tok, 1), 2 * d) for _ in range(M)]
+        # target-side activations (fp32 rows) and their bf16 copies for the weight gradients
+        C = (M + 1) * d
+        self.cat, self.dcat = f32(max(T, 1), C), f32(max(T, 1), C)
+        self.q = []  # q^(1) .. q^(M), set by run()
+        self.Qp = [f32(max(T, 1), d) for _ in range(M)]
+        self.obar = [f32(max(T, 1), d) for _ in range(M)]
+        self.lse = [f32(max(T, 1), H) for _ in range(M)]
+        self.u = [None] + [f32(max(T, 1), d) for _ in range(1, M)]
+        self.zin = f32(max(T, 1), d)
+        self.z = None  # z [T, d], set by run()
+        self.ffn_state = {}
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def x_t_slot(self):
+        """The fp32 [T, d] block of the concatenation where x_t goes (written by the caller)."""
+        return self.cat[:, self.M * self.d:]
+
+    # ---------------------------------------------------------------- helpers
+    def _pack0(self, W, K, N):
+        dst = self.bf(N, K)
+        B.check(B.stca_k_pack_weight(W, K, N, dst, 0, 0), "pack")
+        return dst
+
+    def _gq(self, A, lda, K, Wp, N, C, ldc, dual=0, ksplit=None, kshift=0, R=None, ldr=0):
+        """C [T, N] = A W (+ R) with A fp32 rows (lda), Wp the K-major operand [N(or 2N), K]."""
+        B.check(B.stca_k_gemm_query(A, lda, self.T, K, K if ksplit is None else ksplit, kshift, Wp, N, dual, R, ldr,
+                                    C, ldc, self.err), "target-side GEMM")
+
+    def _to_bf16(self, X, ld, cols):
+        out = self.bf(max(self.T, 1), cols)
+        B.check(B.stca_k_f32_to_bf16(X, ld, self.T, cols, out, cols), "bf16 copy")
+        return out
+
+    def _wgrad(self, A16, lda, G16, ldg, K, N, out=None):
+        out = self.f32(K, N) if out is None else out
+        wsz = B.stca_k_gemm_wgrad_workspace_bytes(self.T, K, N)
+        ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=self.dev)
+        B.check(B.stca_k_gemm_wgrad(A16, lda, G16, ldg, self.T, K, N, out, N, 0, ws, ws.numel()), "weight gradient")
+        return out
+
+    # ---------------------------------------------------------------- target-side FFNs
+    def _ffn_fwd(self, key, ffn, x, ldx, K, ln):
+        """y = SwiGLU(x) (then LN when ln): keeps x, P = [x W1 | x W3], A and y for the backward.
+        x: fp32 rows [T, ldx] of which the first K columns are the input (K = d)."""
+        d, h, T = self.d, self.h, self.T
+        st = {"x": x, "ldx": ldx, "P": self.f32(max(T, 1), 2 * h), "A": self.f32(max(T, 1), h),
+              "y": self.f32(max(T, 1), d), "out": self.f32(max(T, 1), d) if ln is not None else None}
+        self._gq(x, ldx, K, ffn.P0, 2 * h, st["P"], 2 * h)
+        self._gq(x, ldx, K, ffn.P12, h, st["A"], h, dual=1)
+        self._gq(st["A"], h, h, ffn.W2p, d, st["y"], d)
+        if ln is not None:
+            B.check(B.stca_k_layer_norm(st["y"], d, 1, T, d, ln["gamma"], ln["beta"], self.eps, st["out"], d, 1),
+                    "LayerNorm")
+        self.ffn_state[key] = st
+        return st["out"] if ln is not None else st["y"]
+
+    def _ffn_bwd(self, key, ffn, ln, dout, ld_dout, dx, ld_dx, R=None, ldr=0):
+        """Backward of _ffn_fwd[key] from dout [T, d]: writes dx (= dP [W1 | W3]^T (+ R)) and
+        returns the FFN's weight gradients."""
+        d, h, T = self.d, self.h, self.T
+        st = self.ffn_state[key]
+        g = {}
+        dy = dout
+        if ln is not None:
+            dy = self.f32(max(T, 1), d)
+            g["gamma"], g["beta"] = self.f32(d), self.f32(d)
+            wsz = B.stca_k_layer_norm_bwd_workspace_bytes(T, d)
+            ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=self.dev)
+            assert ld_dout == d, "the LayerNorm backward takes dense rows"
+            B.check(B.stca_k_layer_norm_bwd(st["y"], dout, T, d, ln["gamma"], ln["beta"], self.eps, dy, None,
+                                            g["gamma"], g["beta"], 0, ws, ws.numel(), fp32=1), "LayerNorm backward")
+            ld_dout = d
+        dA = self.f32(max(T, 1), h)
+        self._gq(dy, ld_dout, d, ffn.f["W2"], h, dA, h)               # dA = dy W2^T (W2 itself)
+        g["W2"] = self._wgrad(self._to_bf16(st["A"], h, h), h, self._to_bf16(dy, ld_dout, d), d, h, d)
+        dP = self.f32(max(T, 1), 2 * h)
+        B.check(B.stca_k_swiglu_bwd(st["P"], dA, T, h, dP, None, fp32=1), "SwiGLU backward")
+        W13 = self._wgrad(self._to_bf16(st["x"], st["ldx"], d), d, self._to_bf16(dP, 2 * h, 2 * h), 2 * h, d, 2 * h)
+        g["W1"], g["W3"] = W13[:, :h], W13[:, h:]
+        self._gq(dP, 2 * h, 2 * h, ffn.W13c, d, dx, ld_dx, R=R, ldr=ldr)  # dx = dP [W1 | W3]^T (+ R)
+        return g
+
+    # ---------------------------------------------------------------- the step
+    def run(self, ids, dt, hoff, toff, table, dt_table, n_items, dZ, dtable, ddt_table=None):
+        """Forward recompute and backward for upstream dZ [T, d] (fp32).  Returns the weight
+        gradients in the workload's structure (fp32 device tensors), except that W_K and W_V
+        of layer i come as one [d, 2d] matrix "WKV_interleaved"[i] in the K/V rows' column
+        order (head j's W_K columns at 128 j, its W_V columns at 128 j + 64); the table rows'
+        gradients are added into dtable (and ddt_table); d x_t is ``dx_t()``."""
+        d, h, M, H, T, N = self.d, self.h, self.M, self.H, self.T, self.N
+        C = (M + 1) * d
+        w, sc = self.w, self.score
+        pa = self.f32(1, max(T, 1), d)
+        pm = self.f32(1, max(T, 1), H, 2)
+        # ---- forward: history side per layer, then the target side
+        for i in range(M):
+            L = self.hist[i]
+            L.recompute(ids, dt, table, dt_table, n_items)
+            B.check(B.stca_k_layer_norm(L.y, d, 0, N, d, w["hist"][i]["gamma"], w["hist"][i]["beta"], self.eps, L.Xt,
+                                        d, 0), "history LayerNorm")
+            B.check(B.stca_k_gemm_resident(0, 0, L.Xt, None, None, None, None, 0, N, d, self.KVp[i], 2 * d, self.KV[i],
+                                           2 * d, self.err), "K/V rows")
+        xt = self.x_t_slot()
+        q0 = self._ffn_fwd("tgt", self.tgt, xt, C, d, w["tgt"])
+        q = [q0]
+        for i in range(M):
+            self._gq(q[i], d, d, self.WQp[i], d, self.Qp[i], d)
+            B.check(B.stca_attention_train_forward(self.Qp[i], self.KV[i], hoff, toff, self.B, T, d, H, 1, sc, pa, pm,
+                                                   self.obar[i], self.lse[i] if sc == 0 else None, self.err),
+                    "attention")
+            self._gq(self.obar[i], d, d, self.WOp[i], d, self.cat[:, i * d:], C)  # o^(i+1) into the concatenation
+            if i + 1 < M:
+                # u = [o^(1) .. o^(i+1) | x_t] W_C^(i+2): two column blocks of the concatenation
+                self._gq(self.cat, C, (i + 2) * d, self.WCp[i + 1], d, self.u[i + 1], d, ksplit=(i + 1) * d,
+                         kshift=(M - i - 1) * d)
+                q.append(self._ffn_fwd(("fuse", i + 1), self.fuse[i + 1], self.u[i + 1], d, d, w["fuse"][i + 1]))
+        self.q = q
+        self._gq(self.cat, C, C, self.WZp, d, self.zin, d)
+        self.z = self._ffn_fwd("z", self.zffn, self.zin, d, d, None)
+        return self._backward(ids, dt, hoff, toff, n_items, dZ, dtable, ddt_table)
+
+    def _backward(self, ids, dt, hoff, toff, n_items, dZ, dtable, ddt_table):
+        d, h, M, H, T, N = self.d, self.h, self.M, self.H, self.T, self.N
+        C = (M + 1) * d
+        w, sc = self.w, self.score
+        g = {"hist": [None] * M, "WQ": [None] * M, "WKV_interleaved": [None] * M, "WO": [None] * M,
+             "WC": [None] * M, "fuse": [None] * M}
+        # z = SwiGLU_Z(cat W_Z)
+        dzin = self.f32(max(T, 1), d)
+        g["zffn"] = self._ffn_bwd("z", self.zffn, None, dZ, d, dzin, d)
+        cat16 = self._to_bf16(self.cat, C, C)
+        g["WZ"] = self._wgrad(cat16, C, self._to_bf16(dzin, d, d), d, C, d)
+        self._gq(dzin, d, d, w["WZ"], C, self.dcat, C)                    # d cat = dzin W_Z^T (every block)
+        dobar, dQ, dq = self.f32(max(T, 1), d), self.f32(max(T, 1), d), self.f32(max(T, 1), d)
+        dKV = self.f32(max(N, 1), 2 * d)
+        dKV16 = self.bf(max(N, 1), 2 * d)
+        for i in reversed(range(M)):
+            dout = self.dcat[:, i * d:]
+            g["WO"][i] = self._wgrad(self._to_bf16(self.obar[i], d, d), d, self._to_bf16(dout, C, d), d, d, d)
+            self._gq(dout, C, d, w["WO"][i], d, dobar, d)                 # d obar = d o W_O^T
+            B.check(B.stca_attention_backward(self.Qp[i], self.KV[i], hoff, toff, self.B, T, d, H, 1, sc, self.obar[i],
+                                              self.lse[i] if sc == 0 else None, dobar, dQ, dKV, None),
+                    "attention backward")
+            g["WQ"][i] = self._wgrad(self._to_bf16(self.q[i], d, d), d, self._to_bf16(dQ, d, d), d, d, d)
+            self._gq(dQ, d, d, w["WQ"][i], d, dq, d)                      # dq = dQ W_Q^T
+            xt_blk = self.dcat[:, M * d:]
+            if i == 0:   # q^(1) = LN(SwiGLU_t(x_t)): d x_t gathers into the concatenation's x_t block
+                g["tgt"] = self._ffn_bwd("tgt", self.tgt, w["tgt"], dq, d, xt_blk, C, R=xt_blk, ldr=C)
+            else:        # q^(i+1) = LN(SwiGLU(u)), u = [o^(1) .. o^(i) | x_t] W_C^(i+1)
+                du = self.f32(max(T, 1), d)
+                g["fuse"][i] = self._ffn_bwd(("fuse", i), self.fuse[i], w["fuse"][i], dq, d, du, d)
+                du16 = self._to_bf16(du, d, d)
+                gWC = self.f32((i + 1) * d, d)
+                self._wgrad(cat16, C, du16, d, i * d, d, out=gWC[:i * d])
+                self._wgrad(cat16[:, M * d:], C, du16, d, d, d, out=gWC[i * d:])
+                g["WC"][i] = gWC
+                # the o^(j) blocks and x_t take du W_C^T (added to what they already hold)
+                self._gq(du, d, d, w["WC"][i][:i * d], i * d, self.dcat, C, R=self.dcat, ldr=C)
+                self._gq(du, d, d, w["WC"][i][i * d:], d, xt_blk, C, R=xt_blk, ldr=C)
+            # the history side of layer i from its K/V rows' gradients
+            B.check(B.stca_k_f32_to_bf16(dKV, 2 * d, N, 2 * d, dKV16, 2 * d), "bf16 copy")
+            L = self.hist[i]
+            L.backward(dKV16, ids, dt, n_items, dtable, ddt_table)
+            # [dW_K | dW_V] in the K/V rows' head-interleaved columns: head j's K at 128 j, V at 128 j + 64
+            g["WKV_interleaved"][i] = L.dWKV
+            g["hist"][i] = {"W1": L.dW13[:, :h], "W3": L.dW13[:, h:], "W2": L.dW2, "gamma": L.dgamma,
+                            "beta": L.dbeta}
+        return g
+
+    def dx_t(self):
+        """d x_t [T, d] fp32 (a view of the concatenation's gradient) after ``run``."""
+        return self.dcat[:, self.M * self.d:]
+
+
+def device_weights(w, device="cuda"):
+    """The workload's weights (bf16 bit patterns as uint16, fp32 LayerNorm parameters) as
+    device tensors in the same structure (bf16 and fp32), for StcaTrainingStep."""
+    import numpy as np
+
+    def up(a):
+        if a is None:
+            return None
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(a.astype(np.float32)).to(device)
+
+    def walk(x):
+        if isinstance(x, dict):
+            return {k: walk(v) for k, v in x.items()}
+        if isinstance(x, list):
+            return [walk(v) for v in x]
+        return up(x)
+
+    return walk(w)

@@ -118,13 +118,16 @@ def test_null_arguments_rejected_on_host():
     assert L.stca_k_gemm_wgrad(16, 128, 16, 128, 100, 128, 128, 16, 128, 0, 16, 16, None) == B.ERR_CAPACITY
     assert L.stca_k_gemm_wgrad(16, 120, 16, 128, 100, 128, 128, 16, 128, 0, 16, 1 << 30, None) == B.ERR_INVALID_ARG
     assert L.stca_k_gemm_wgrad(None, 128, 16, 128, 100, 128, 128, 16, 128, 0, 16, 1 << 30, None) == B.ERR_INVALID_ARG
-    assert L.stca_k_layer_norm_bwd(16, 16, 10, 384, 16, None, 1e-5, 16, None, 16, 16, 0, 16, 1 << 20, None) \
+    assert L.stca_k_layer_norm_bwd(16, 16, 10, 384, 0, 16, None, 1e-5, 16, None, 16, 16, 0, 16, 1 << 20, None) \
         == B.ERR_UNSUPPORTED
-    assert L.stca_k_layer_norm_bwd(16, 16, 10, 256, 16, None, 1e-5, 16, None, 16, 16, 0, 16, 4, None) \
+    assert L.stca_k_layer_norm_bwd(16, 16, 10, 256, 0, 16, None, 1e-5, 16, None, 16, 16, 0, 16, 4, None) \
         == B.ERR_CAPACITY
-    assert L.stca_k_swiglu_bwd(16, 16, 10, 12, 16, None, None) == B.ERR_UNSUPPORTED        # h % 8
-    assert L.stca_k_swiglu_bwd(16, 16, 10, 16, 24, None, None) == B.ERR_INVALID_ARG        # alignment
+    assert L.stca_k_swiglu_bwd(16, 16, 10, 12, 0, 16, None, None) == B.ERR_UNSUPPORTED        # h % 8
+    assert L.stca_k_swiglu_bwd(16, 16, 10, 16, 0, 24, None, None) == B.ERR_INVALID_ARG        # alignment
     assert L.stca_k_table_rows_bwd(16, 10, 12, 16, None, 100, 16, None, None, None) == B.ERR_INVALID_ARG
+    assert L.stca_k_layer_norm(16, 256, 1, 10, 256, 16, None, 1e-5, 16, 256, 0, None) == B.ERR_UNSUPPORTED  # fp32 -> bf16
+    assert L.stca_k_layer_norm(16, 100, 1, 10, 256, 16, None, 1e-5, 16, 256, 1, None) == B.ERR_INVALID_ARG  # ldx < d
+    assert L.stca_k_f32_to_bf16(16, 8, 4, 16, 16, 16, None) == B.ERR_INVALID_ARG                           # lds < cols
     assert L.stca_k_table_rows_bwd(16, 10, 256, None, None, 100, 16, None, None, None) == B.ERR_INVALID_ARG
     assert L.stca_k_gemm_resident(1, 1, None, None, None, None, None, 0, 5, 256, None, 128, None, 128, None, None,
                                   None) == B.ERR_INVALID_ARG

@@ -66,25 +66,49 @@ def test_gemm_wgrad_matches_float64(M, K, N, lda_pad):
 
 
 @pytest.mark.parametrize("d", [256, 512])
-def test_layer_norm_bwd_matches_oracle(d):
-    g = np.random.default_rng(d)
+@pytest.mark.parametrize("fp32", [0, 1])
+def test_layer_norm_bwd_and_fwd_match_oracle(d, fp32):
+    """LayerNorm backward (bf16 history rows, fp32 target rows) and the forward the training
+    step recomputes with."""
+    g = np.random.default_rng(d + fp32)
     M, eps = 333, 1e-5
-    y = to_bf16(g.standard_normal((M, d)) * 2 + 0.5)
-    dxt = to_bf16(g.standard_normal((M, d)))
+    cast = (lambda x: torch.from_numpy(np.asarray(x, np.float32)).to(dev)) if fp32 else to_bf16
+    y = cast(g.standard_normal((M, d)) * 2 + 0.5)
+    dxt = cast(g.standard_normal((M, d)))
     gamma = torch.from_numpy(g.standard_normal(d).astype(np.float32)).to(dev)
     beta = torch.from_numpy(g.standard_normal(d).astype(np.float32)).to(dev)
-    dy = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
-    xt = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+    dy, xt, xf = torch.empty_like(y), torch.empty_like(y), torch.empty_like(y)
     dg = torch.empty(d, device=dev)
     db = torch.empty(d, device=dev)
     w = ws(B.stca_k_layer_norm_bwd_workspace_bytes(M, d))
-    B.check(B.stca_k_layer_norm_bwd(y, dxt, M, d, gamma, beta, eps, dy, xt, dg, db, 0, w, w.numel()))
+    B.check(B.stca_k_layer_norm_bwd(y, dxt, M, d, gamma, beta, eps, dy, xt, dg, db, 0, w, w.numel(), fp32=fp32))
+    B.check(B.stca_k_layer_norm(y, d, fp32, M, d, gamma, beta, eps, xf, d, fp32))
     y64, dxt64 = bf16_to_f64(y), bf16_to_f64(dxt)
     rdy, rdg, rdb = G.layer_norm_bwd(y64, gamma.cpu().numpy(), beta.cpu().numpy(), eps, dxt64)
-    assert normwise(bf16_to_f64(dy), rdy) < 1e-2
+    bar = 1e-5 if fp32 else 1e-2
+    assert normwise(bf16_to_f64(dy), rdy) < bar
     assert normwise(dg.cpu().numpy(), rdg) < 1e-4 and normwise(db.cpu().numpy(), rdb) < 1e-4
     rxt = R.layer_norm(y64, gamma.cpu().numpy(), beta.cpu().numpy(), eps)
-    assert normwise(bf16_to_f64(xt), rxt) < 1e-2
+    assert normwise(bf16_to_f64(xt), rxt) < bar
+    assert normwise(bf16_to_f64(xf), rxt) < bar
+
+
+def test_swiglu_bwd_fp32_and_bf16_copy():
+    g = np.random.default_rng(9)
+    M, h = 77, 64
+    P = torch.from_numpy(g.standard_normal((M, 2 * h)).astype(np.float32)).to(dev)
+    dA = torch.from_numpy(g.standard_normal((M, h)).astype(np.float32)).to(dev)
+    dP, A = torch.empty_like(P), torch.empty_like(dA)
+    B.check(B.stca_k_swiglu_bwd(P, dA, M, h, dP, A, fp32=1))
+    p, da = P.cpu().double().numpy(), dA.cpu().double().numpy()
+    a, b = p[:, :h], p[:, h:]
+    sig = 1 / (1 + np.exp(-a))
+    assert normwise(A.cpu().numpy(), a * sig * b) < 1e-5
+    assert normwise(dP.cpu().numpy()[:, :h], da * b * G.silu_grad(a)) < 1e-5
+    assert normwise(dP.cpu().numpy()[:, h:], da * a * sig) < 1e-5
+    out = torch.empty((M, h), dtype=torch.bfloat16, device=dev)
+    B.check(B.stca_k_f32_to_bf16(P, 2 * h, M, h, out, h))       # a strided block, rounded to bf16
+    assert torch.equal(out, P[:, :h].to(torch.bfloat16))
 
 
 @pytest.mark.parametrize("config", [2, 3])
