@@ -61,7 +61,7 @@ def parse():
                     help="control run: history ids uniform over the table instead of Zipf")
     ap.add_argument("--kv-fold", action="store_true",
                     help="fold W_K / W_V into the queries (d = 256 STCA workloads only)")
-    ap.add_argument("--probe", choices=["attention", "history-backward"], default=None,
+    ap.add_argument("--probe", choices=["attention", "history-backward", "train-step"], default=None,
                     help="instead of the step: time kernels alone on the workload's shapes and print one "
                          "JSON line per kernel or input form (attention: contiguous keys and the compacted "
                          "per-user key lists of the workload's ids; history-backward: every step of one "
@@ -906,12 +906,90 @@ def run_probe_history_backward(args):
         print(json.dumps(line), flush=True)
 
 
+def run_probe_train_step(args):
+    """The whole training step (target_attention_b200.training.StcaTrainingStep: every
+    layer's history side recomputed, the target side, then the backward into every weight,
+    the table rows and x_t) on the workload's batch (--workload 2 or 3), three phases
+    bracketed by CUDA events, median over 3 x steps runs after warm-up.  The flop rate
+    counts the history GEMMs and the attention products against the measured sustained
+    bf16 rate."""
+    import statistics
+    import numpy as np
+    import torch
+    from target_attention_b200 import binding as B
+    from target_attention_b200.training import StcaTrainingStep, device_weights
+    wl = make_workload(args, data_seed=rank_data_seed(args.workload, 0))
+    assert wl["cfg"]["kind"] == "stca", "train-step probes an STCA workload (2 or 3)"
+    cfg = wl["cfg"]
+    d = cfg["d"]
+    dev = "cuda"
+    lengths, tpu = wl["lengths"], wl["targets_per_user"]
+    Bu, N, T = len(lengths), int(lengths.sum()), int(tpu.sum())
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).to(dev)
+    up16 = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    hoff = torch.empty(Bu + 1, dtype=torch.int32, device=dev)
+    toff = torch.empty(Bu + 1, dtype=torch.int32, device=dev)
+    B.check(B.stca_k_offsets(i32(lengths), Bu, hoff, N, err))
+    B.check(B.stca_k_offsets(i32(tpu), Bu, toff, T, err))
+    step = StcaTrainingStep(cfg, device_weights(wl["weights"]), Bu, N, T)
+    step.x_t_slot().copy_(up16(wl["x_t"]).float())
+    ids = i32(wl["ids"])
+    dt = i32(wl["dt"]) if wl["dt"] is not None else None
+    table = up16(wl["table"])
+    dt_table = up16(wl["dt_table"]) if wl["dt"] is not None else None
+    n_items = int(wl["table"].shape[0])
+    g = torch.Generator(device=dev)
+    g.manual_seed(3)
+    dZ = torch.randn((T, d), device=dev, generator=g)
+    dtable = torch.zeros((n_items, d), device=dev)
+    ddt = torch.zeros((16, d), device=dev) if dt is not None else None
+
+    def once():
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        ev[0].record()
+        step.forward_history(ids, dt, table, dt_table, n_items)
+        ev[1].record()
+        step.forward_target(hoff, toff)
+        ev[2].record()
+        step.backward(ids, dt, hoff, toff, n_items, dZ, dtable, ddt)
+        ev[3].record()
+        return ev
+
+    for _ in range(max(args.warmup, 1)):
+        once()
+    torch.cuda.synchronize()
+    times = {k: [] for k in ("history forward", "target forward", "backward", "step")}
+    for _ in range(3 * args.steps):
+        ev = once()
+        torch.cuda.synchronize()
+        for k, (a, b) in zip(times, ((0, 1), (1, 2), (2, 3), (0, 3))):
+            times[k].append(ev[a].elapsed_time(ev[b]))
+    assert int(err.item()) == 0 and int(step.err.item()) == 0
+    flops = step.flops(lengths, tpu)
+    peak = load_peaks()["bf16_tflops_sustained"]
+    for name, ts in times.items():
+        ms = statistics.median(ts)
+        line = {"probe": "train-step", "phase": name, "workload": args.workload, "users": Bu, "history_tokens": N,
+                "targets": T, "d": d, "layers": cfg["M"], "score": cfg["score"], "median_ms": round(ms, 4),
+                "runs": len(ts)}
+        if name == "step":
+            f = sum(flops.values())
+            tf = f / ms / 1e9
+            line.update(flop=f, flop_attention=flops["attention"], achieved_tflops=round(tf, 1), peak_tflops=peak,
+                        frac=round(tf / peak, 4), history_tokens_per_s=round(N / ms * 1e3),
+                        targets_per_s=round(T / ms * 1e3))
+        print(json.dumps(line), flush=True)
+
+
 if __name__ == "__main__":
     a = parse()
     if a.probe == "attention":
         run_probe_attention(a)
     elif a.probe == "history-backward":
         run_probe_history_backward(a)
+    elif a.probe == "train-step":
+        run_probe_train_step(a)
     elif a.impl == "reference":
         run_reference(a)
     else:

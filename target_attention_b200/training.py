@@ -58,17 +58,19 @@ class HistoryLayerBackward:
         step(B.stca_k_gemm_rowwise(0, self.A, M, h, self.W2p, d, None, None, self.eps, self.y, d, e, stream),
                 "A W2")
 
-    def backward(self, dKV, ids, dt, n_items, dtable, ddt_table=None, stream=None, on_step=None):
+    def backward(self, dKV, ids, dt, n_items, dtable, ddt_table=None, stream=None, on_step=None, xt_ready=False):
         """dKV [M, 2d] bf16 (head-interleaved K | V columns).  Weight gradients land in
         dWKV (head-interleaved columns), dW2, dW13 ([dW1 | dW3]), dgamma, dbeta; the table
         rows' gradients are added into dtable (and ddt_table).  on_step(name), when given, is
-        called after each step is enqueued (a profiler records events there)."""
+        called after each step is enqueued (a profiler records events there).  xt_ready: Xt =
+        LN(y) is already in ``Xt`` (the LayerNorm backward then does not write it again)."""
         M, d, h, e = self.M, self.d, self.h, self.err
         step = _stepper(on_step)
         step(B.stca_k_gemm_rowwise(0, dKV, M, 2 * d, self.WKVi, d, None, None, self.eps, self.dXt, d, e, stream),
                 "dKV [W_K | W_V]^T")
-        step(B.stca_k_layer_norm_bwd(self.y, self.dXt, M, d, self.gamma, self.beta, self.eps, self.dy, self.Xt,
-                                        self.dgamma, self.dbeta, 0, self.wln, self.wln.numel(), stream), "LN backward")
+        step(B.stca_k_layer_norm_bwd(self.y, self.dXt, M, d, self.gamma, self.beta, self.eps, self.dy,
+                                        None if xt_ready else self.Xt, self.dgamma, self.dbeta, 0, self.wln,
+                                        self.wln.numel(), stream), "LN backward")
         step(B.stca_k_gemm_wgrad(self.Xt, d, dKV, 2 * d, M, d, 2 * d, self.dWKV, 2 * d, 0, self.wg, self.wg.numel(),
                                     stream), "Xt^T dKV")
         step(B.stca_k_gemm_resident(0, 0, self.dy, None, None, None, None, 0, M, d, self.W2, h, self.dA, h, e,
@@ -246,12 +248,13 @@ class StcaTrainingStep:
         of layer i come as one [d, 2d] matrix "WKV_interleaved"[i] in the K/V rows' column
         order (head j's W_K columns at 128 j, its W_V columns at 128 j + 64); the table rows'
         gradients are added into dtable (and ddt_table); d x_t is ``dx_t()``."""
-        d, h, M, H, T, N = self.d, self.h, self.M, self.H, self.T, self.N
-        C = (M + 1) * d
-        w, sc = self.w, self.score
-        pa = self.f32(1, max(T, 1), d)
-        pm = self.f32(1, max(T, 1), H, 2)
-        # ---- forward: history side per layer, then the target side
+        self.forward_history(ids, dt, table, dt_table, n_items)
+        self.forward_target(hoff, toff)
+        return self.backward(ids, dt, hoff, toff, n_items, dZ, dtable, ddt_table)
+
+    def forward_history(self, ids, dt, table, dt_table, n_items):
+        """Every layer's history side recomputed: the rows X, A, P, y, Xt = LN(y) and the K/V rows."""
+        d, M, N, w = self.d, self.M, self.N, self.w
         for i in range(M):
             L = self.hist[i]
             L.recompute(ids, dt, table, dt_table, n_items)
@@ -259,6 +262,14 @@ class StcaTrainingStep:
                                         d, 0), "history LayerNorm")
             B.check(B.stca_k_gemm_resident(0, 0, L.Xt, None, None, None, None, 0, N, d, self.KVp[i], 2 * d, self.KV[i],
                                            2 * d, self.err), "K/V rows")
+
+    def forward_target(self, hoff, toff):
+        """The target side in fp32 rows, from x_t (in ``x_t_slot()``) and the K/V rows."""
+        d, M, H, T = self.d, self.M, self.H, self.T
+        C = (M + 1) * d
+        w, sc = self.w, self.score
+        pa = self.f32(1, max(T, 1), d)
+        pm = self.f32(1, max(T, 1), H, 2)
         xt = self.x_t_slot()
         q0 = self._ffn_fwd("tgt", self.tgt, xt, C, d, w["tgt"])
         q = [q0]
@@ -276,9 +287,9 @@ class StcaTrainingStep:
         self.q = q
         self._gq(self.cat, C, C, self.WZp, d, self.zin, d)
         self.z = self._ffn_fwd("z", self.zffn, self.zin, d, d, None)
-        return self._backward(ids, dt, hoff, toff, n_items, dZ, dtable, ddt_table)
 
-    def _backward(self, ids, dt, hoff, toff, n_items, dZ, dtable, ddt_table):
+    def backward(self, ids, dt, hoff, toff, n_items, dZ, dtable, ddt_table=None):
+        """The backward after forward_history and forward_target (see ``run``)."""
         d, h, M, H, T, N = self.d, self.h, self.M, self.H, self.T, self.N
         C = (M + 1) * d
         w, sc = self.w, self.score
@@ -319,12 +330,22 @@ class StcaTrainingStep:
             # the history side of layer i from its K/V rows' gradients
             B.check(B.stca_k_f32_to_bf16(dKV, 2 * d, N, 2 * d, dKV16, 2 * d), "bf16 copy")
             L = self.hist[i]
-            L.backward(dKV16, ids, dt, n_items, dtable, ddt_table)
+            L.backward(dKV16, ids, dt, n_items, dtable, ddt_table, xt_ready=True)
             # [dW_K | dW_V] in the K/V rows' head-interleaved columns: head j's K at 128 j, V at 128 j + 64
             g["WKV_interleaved"][i] = L.dWKV
             g["hist"][i] = {"W1": L.dW13[:, :h], "W3": L.dW13[:, h:], "W2": L.dW2, "gamma": L.dgamma,
                             "beta": L.dbeta}
         return g
+
+    def flops(self, lengths, targets_per_user):
+        """Multiply-add work of one step in flop: every history-side GEMM (recompute, the K/V
+        rows and the backward) and the attention products (forward q.k and p v; backward the
+        scores again, dP, dV, dK and dQ: 14 d flop per (target, key) pair).  The target
+        side's T-row GEMMs are not counted."""
+        import numpy as np
+        pairs = float(np.dot(np.asarray(lengths, np.float64), np.asarray(targets_per_user, np.float64)))
+        hist = sum(self.hist[0].flops().values()) + 2 * self.N * self.d * 2 * self.d
+        return {"history": self.M * hist, "attention": self.M * 14 * self.d * pairs}
 
     def dx_t(self):
         """d x_t [T, d] fp32 (a view of the concatenation's gradient) after ``run``."""
