@@ -117,10 +117,13 @@ int stca_k_attention_rows(int kv_bf16, const float* Q, const void* KV, const int
  * multiples of 128, lda and ldg multiples of 8, ldc of 4, pointers 16-byte aligned (else
  * STCA_ERR_UNSUPPORTED / STCA_ERR_INVALID_ARG).  ws: device scratch of at least
  * stca_k_gemm_wgrad_workspace_bytes(M, K, N) bytes (else STCA_ERR_CAPACITY): the token
- * slices' partial tiles, added in a fixed order, so the result is the same every run. */
+ * slices' partial tiles, added in a fixed order, so the result is the same every run.
+ * impl: 0 the tcgen05 kernel (both operands read MN-major from their token-major rows by
+ * TMA), 1 the mma.sync kernel; other values STCA_ERR_INVALID_ARG.  err (device, may be
+ * NULL) receives STCA_ERR_TIMEOUT if a bounded wait of the tcgen05 kernel ran out. */
 size_t stca_k_gemm_wgrad_workspace_bytes(int M, int K, int N);
 int stca_k_gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, int M, int K, int N, float* C,
-                      int64_t ldc, int accumulate, void* ws, size_t ws_bytes, void* stream);
+                      int64_t ldc, int accumulate, int impl, void* ws, size_t ws_bytes, int32_t* err, void* stream);
 
 /* LayerNorm backward over rows of d = 256 or 512 (biased variance, eps): y [M, d] the
  * LayerNorm's input, dxt [M, d] the gradient of its output (bf16, or fp32 when fp32 != 0:

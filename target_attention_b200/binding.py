@@ -111,7 +111,8 @@ _SIGS = [
     ("stca_k_attention_rows", _i32, [_i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                      _vp, _vp, _vp, _vp, _vp]),
     ("stca_k_gemm_wgrad_workspace_bytes", ctypes.c_size_t, [_i32, _i32, _i32]),
-    ("stca_k_gemm_wgrad", _i32, [_vp, _i64, _vp, _i64, _i32, _i32, _i32, _vp, _i64, _i32, _vp, ctypes.c_size_t, _vp]),
+    ("stca_k_gemm_wgrad", _i32, [_vp, _i64, _vp, _i64, _i32, _i32, _i32, _vp, _i64, _i32, _i32, _vp, ctypes.c_size_t,
+                                 _vp, _vp]),
     ("stca_k_layer_norm_bwd_workspace_bytes", ctypes.c_size_t, [_i32, _i32]),
     ("stca_k_layer_norm_bwd", _i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, ctypes.c_float, _vp, _vp, _vp, _vp, _i32,
                                      _vp, ctypes.c_size_t, _vp]),
@@ -347,9 +348,10 @@ def stca_k_gemm_wgrad_workspace_bytes(M, K, N) -> int:
     return lib().stca_k_gemm_wgrad_workspace_bytes(M, K, N)
 
 
-def stca_k_gemm_wgrad(A, lda, G, ldg, M, K, N, C, ldc, accumulate, ws, ws_bytes, stream=None) -> int:
-    return lib().stca_k_gemm_wgrad(ptr(A), lda, ptr(G), ldg, M, K, N, ptr(C), ldc, accumulate, ptr(ws), ws_bytes,
-                                   stream_ptr(stream))
+def stca_k_gemm_wgrad(A, lda, G, ldg, M, K, N, C, ldc, accumulate, ws, ws_bytes, stream=None, impl=0,
+                      err=None) -> int:
+    return lib().stca_k_gemm_wgrad(ptr(A), lda, ptr(G), ldg, M, K, N, ptr(C), ldc, accumulate, impl, ptr(ws),
+                                   ws_bytes, ptr(err), stream_ptr(stream))
 
 
 def stca_k_layer_norm_bwd_workspace_bytes(M, d) -> int:

@@ -281,10 +281,15 @@ int compact_user_rows(const int32_t* hoff, int B, const int32_t* rows, int32_t* 
 
 // ---------------------------------------------------------------- training: history side
 // C [K, N] (+)= A^T G over M tokens (A [M, K], G [M, N] bf16, C fp32); K, N % 128 == 0;
-// ws: gemm_wgrad_workspace_bytes(M, K, N) bytes (per-slice partial tiles).
+// ws: gemm_wgrad_workspace_bytes(M, K, N) bytes (per-slice partial tiles).  impl: 0 the
+// tcgen05 kernel (tc_wgrad.cu), 1 the mma.sync kernel; err: timeouts (may be null).
 size_t gemm_wgrad_workspace_bytes(int M, int K, int N);
 int gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, int M, int K, int N, float* C, int64_t ldc,
-               int accumulate, void* ws, size_t ws_bytes, cudaStream_t s);
+               int accumulate, int impl, void* ws, size_t ws_bytes, int32_t* err, cudaStream_t s);
+// the tcgen05 kernel alone: per-slice partial tiles part [splits, K, N]
+int tc_wgrad_splits(int M, int K, int N);
+int tc_wgrad_partials(const void* A, int64_t lda, const void* G, int64_t ldg, int M, int K, int N, int splits,
+                      float* part, int32_t* err, cudaStream_t s);
 size_t layer_norm_bwd_workspace_bytes(int M, int d);
 int layer_norm_bwd(const void* y, const void* dxt, int M, int d, int fp32, const float* gamma, const float* beta,
                    float eps, void* dy, void* xt, float* dgamma, float* dbeta, int accumulate, void* ws,

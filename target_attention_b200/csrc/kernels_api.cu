@@ -48,9 +48,10 @@ int stca_k_pack_weight(const void* W, int K, int N, void* dst, int mode, int row
 size_t stca_k_gemm_wgrad_workspace_bytes(int M, int K, int N) { return gemm_wgrad_workspace_bytes(M, K, N); }
 
 int stca_k_gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, int M, int K, int N, float* C,
-                      int64_t ldc, int accumulate, void* ws, size_t ws_bytes, void* stream) {
+                      int64_t ldc, int accumulate, int impl, void* ws, size_t ws_bytes, int32_t* err, void* stream) {
   if (M < 0 || (M > 0 && (!A || !G || !ws)) || !C) return STCA_ERR_INVALID_ARG;
-  return gemm_wgrad(A, lda, G, ldg, M, K, N, C, ldc, accumulate, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+  return gemm_wgrad(A, lda, G, ldg, M, K, N, C, ldc, accumulate, impl, ws, ws_bytes, err,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t stca_k_layer_norm_bwd_workspace_bytes(int M, int d) { return M < 0 ? 0 : layer_norm_bwd_workspace_bytes(M, d); }

@@ -433,20 +433,25 @@ __global__ void place_cols_kernel(const bf16* __restrict__ W, int K, int N, bf16
 
 size_t gemm_wgrad_workspace_bytes(int M, int K, int N) {
   if (M <= 0 || K <= 0 || N <= 0 || K % WG_T || N % WG_T) return 0;
-  return size_t(wgrad_splits(M, K, N)) * K * N * 4;
+  return size_t(std::max(wgrad_splits(M, K, N), tc_wgrad_splits(M, K, N))) * K * N * 4;
 }
 
 int gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, int M, int K, int N, float* C, int64_t ldc,
-               int accumulate, void* ws, size_t ws_bytes, cudaStream_t s) {
+               int accumulate, int impl, void* ws, size_t ws_bytes, int32_t* err, cudaStream_t s) {
   if (M < 0 || K <= 0 || N <= 0 || K % WG_T || N % WG_T || lda % 8 || ldg % 8 || ldc % 4) return STCA_ERR_UNSUPPORTED;
-  if (lda < K || ldg < N || ldc < N) return STCA_ERR_INVALID_ARG;
+  if (lda < K || ldg < N || ldc < N || impl < 0 || impl > 1) return STCA_ERR_INVALID_ARG;
   const uintptr_t al = reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(G) |
                        reinterpret_cast<uintptr_t>(C) | reinterpret_cast<uintptr_t>(ws);
   if (al & 15) return STCA_ERR_INVALID_ARG;
-  const int splits = M > 0 ? wgrad_splits(M, K, N) : 1;
+  // 0: the tensor-core (tcgen05) kernel; 1: the mma.sync kernel (both kept under test)
+  const bool tc = impl != 1;
+  const int splits = M > 0 ? (tc ? tc_wgrad_splits(M, K, N) : wgrad_splits(M, K, N)) : 1;
   if (M > 0 && ws_bytes < size_t(splits) * K * N * 4) return STCA_ERR_CAPACITY;
   float* part = static_cast<float*>(ws);
-  if (M > 0) {
+  if (M > 0 && tc) {
+    const int rc = tc_wgrad_partials(A, lda, G, ldg, M, K, N, splits, part, err, s);
+    if (rc != STCA_OK) return rc;
+  } else if (M > 0) {
     cudaFuncSetAttribute(gemm_wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, WG_SMEM);
     if (launch_dep(gemm_wgrad_kernel, dim3(N / WG_T, K / WG_T, splits), dim3(256), WG_SMEM, s,
                    static_cast<const bf16*>(A), lda, static_cast<const bf16*>(G), ldg, M, K, N, splits,

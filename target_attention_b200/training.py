@@ -72,16 +72,16 @@ class HistoryLayerBackward:
                                         None if xt_ready else self.Xt, self.dgamma, self.dbeta, 0, self.wln,
                                         self.wln.numel(), stream), "LN backward")
         step(B.stca_k_gemm_wgrad(self.Xt, d, dKV, 2 * d, M, d, 2 * d, self.dWKV, 2 * d, 0, self.wg, self.wg.numel(),
-                                    stream), "Xt^T dKV")
+                                    stream, err=e), "Xt^T dKV")
         step(B.stca_k_gemm_resident(0, 0, self.dy, None, None, None, None, 0, M, d, self.W2, h, self.dA, h, e,
                                        stream), "dy W2^T")
-        step(B.stca_k_gemm_wgrad(self.A, h, self.dy, d, M, h, d, self.dW2, d, 0, self.wg, self.wg.numel(), stream),
-                "A^T dy")
+        step(B.stca_k_gemm_wgrad(self.A, h, self.dy, d, M, h, d, self.dW2, d, 0, self.wg, self.wg.numel(), stream,
+                                    err=e), "A^T dy")
         step(B.stca_k_swiglu_bwd(self.P, self.dA, M, h, self.dP, None, stream), "SwiGLU backward")
         step(B.stca_k_gemm_rowwise(0, self.dP, M, 2 * h, self.W13c, d, None, None, self.eps, self.dX, d, e, stream),
                 "dP [W1 | W3]^T")
         step(B.stca_k_gemm_wgrad(self.X, d, self.dP, 2 * h, M, d, 2 * h, self.dW13, 2 * h, 0, self.wg,
-                                    self.wg.numel(), stream), "X^T dP")
+                                    self.wg.numel(), stream, err=e), "X^T dP")
         step(B.stca_k_table_rows_bwd(self.dX, M, d, ids, dt, n_items, dtable, ddt_table, e, stream),
                 "table rows")
 
@@ -196,7 +196,8 @@ class StcaTrainingStep:
         out = self.f32(K, N) if out is None else out
         wsz = B.stca_k_gemm_wgrad_workspace_bytes(self.T, K, N)
         ws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=self.dev)
-        B.check(B.stca_k_gemm_wgrad(A16, lda, G16, ldg, self.T, K, N, out, N, 0, ws, ws.numel()), "weight gradient")
+        B.check(B.stca_k_gemm_wgrad(A16, lda, G16, ldg, self.T, K, N, out, N, 0, ws, ws.numel(), err=self.err),
+                "weight gradient")
         return out
 
     # ---------------------------------------------------------------- target-side FFNs

@@ -114,10 +114,17 @@ def test_null_arguments_rejected_on_host():
     assert L.stca_k_pack_weight(16, 64, 64, 16, 3, 32, None) == B.ERR_INVALID_ARG   # ... and the K or V half
     assert L.stca_k_pack_weight(16, 64, 64, 16, 5, 0, None) == B.ERR_INVALID_ARG
     # training entries: shapes the kernels do not take, workspace too small, missing buffers
-    assert L.stca_k_gemm_wgrad(16, 128, 16, 128, 100, 96, 128, 16, 128, 0, 16, 1 << 30, None) == B.ERR_UNSUPPORTED
-    assert L.stca_k_gemm_wgrad(16, 128, 16, 128, 100, 128, 128, 16, 128, 0, 16, 16, None) == B.ERR_CAPACITY
-    assert L.stca_k_gemm_wgrad(16, 120, 16, 128, 100, 128, 128, 16, 128, 0, 16, 1 << 30, None) == B.ERR_INVALID_ARG
-    assert L.stca_k_gemm_wgrad(None, 128, 16, 128, 100, 128, 128, 16, 128, 0, 16, 1 << 30, None) == B.ERR_INVALID_ARG
+    assert L.stca_k_gemm_wgrad(16, 128, 16, 128, 100, 96, 128, 16, 128, 0, 0, 16, 1 << 30, None, None) == \
+        B.ERR_UNSUPPORTED
+    for impl in (0, 1):
+        assert L.stca_k_gemm_wgrad(16, 128, 16, 128, 100, 128, 128, 16, 128, 0, impl, 16, 16, None, None) == \
+            B.ERR_CAPACITY
+    assert L.stca_k_gemm_wgrad(16, 120, 16, 128, 100, 128, 128, 16, 128, 0, 0, 16, 1 << 30, None, None) == \
+        B.ERR_INVALID_ARG
+    assert L.stca_k_gemm_wgrad(None, 128, 16, 128, 100, 128, 128, 16, 128, 0, 0, 16, 1 << 30, None, None) == \
+        B.ERR_INVALID_ARG
+    assert L.stca_k_gemm_wgrad(16, 128, 16, 128, 100, 128, 128, 16, 128, 0, 3, 16, 1 << 30, None, None) == \
+        B.ERR_INVALID_ARG
     assert L.stca_k_layer_norm_bwd(16, 16, 10, 384, 0, 16, None, 1e-5, 16, None, 16, 16, 0, 16, 1 << 20, None) \
         == B.ERR_UNSUPPORTED
     assert L.stca_k_layer_norm_bwd(16, 16, 10, 256, 0, 16, None, 1e-5, 16, None, 16, 16, 0, 16, 4, None) \
