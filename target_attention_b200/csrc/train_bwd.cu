@@ -417,6 +417,177 @@ __global__ void __launch_bounds__(256) table_rows_bwd_kernel(const bf16* __restr
     if (bucket_acc[i] != 0.f) atomicAdd(ddt_table + i, bucket_acc[i]);
 }
 
+// The same scatter with the tokens of each 1024-token chunk grouped by id first, for d a
+// multiple of 256: a shared-memory hash table (2048 slots, linear probing, at most 1024
+// keys) gives each token its group; a scan lays the groups' members out contiguously;
+// then one warp per group sums the members' rows in registers (four rows in flight) and
+// adds the sum to the id's row with one set of vector atomics.  A Zipf-popular id that
+// appears 100 times in a chunk costs one row of atomics there instead of 100, which is
+// what the atomics on hot rows were waiting on.
+constexpr int TR_CH = 1024, TR_HS = 2048, TR_THREADS = 256;
+constexpr size_t TR_SMEM_INT = size_t(4 * TR_HS + 3 * TR_CH + 4) * 4;  // keys cnt start fill | slot order gslot | misc
+
+template <int DV>
+__global__ void __launch_bounds__(TR_THREADS) table_rows_grouped_kernel(const bf16* __restrict__ dX, int M,
+                                                                        const int32_t* __restrict__ ids,
+                                                                        const int32_t* __restrict__ dt,
+                                                                        int64_t n_items, float* __restrict__ dtable,
+                                                                        float* __restrict__ ddt_table, int32_t* err) {
+  constexpr int d = 256 * DV;
+  griddep_wait();
+  extern __shared__ __align__(16) int tr_smem[];
+  int* keys = tr_smem;                // [TR_HS] id, -1 empty
+  int* cnt = keys + TR_HS;            // [TR_HS] members per slot
+  int* start = cnt + TR_HS;           // [TR_HS] first member position
+  int* fill = start + TR_HS;          // [TR_HS] members placed so far
+  int* slot_of = fill + TR_HS;        // [TR_CH] token -> slot (-1: skipped)
+  int* order = slot_of + TR_CH;       // [TR_CH] tokens grouped by slot
+  int* gslot = order + TR_CH;         // [TR_CH] slot of group g
+  int* misc = gslot + TR_CH;          // [0] groups, [1] next group, [2..3] scan scratch
+  float* bucket_acc = reinterpret_cast<float*>(misc + 4);  // [16][d] when ddt_table
+  __shared__ int warp_sum[TR_THREADS / 32], warp_ne[TR_THREADS / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool with_dt = dt && ddt_table;
+  if (with_dt)
+    for (int i = threadIdx.x; i < 16 * d; i += TR_THREADS) bucket_acc[i] = 0.f;
+  const int nchunks = (M + TR_CH - 1) / TR_CH;
+  for (int chunk = blockIdx.x; chunk < nchunks; chunk += gridDim.x) {
+    const int c0 = chunk * TR_CH;
+    for (int i = threadIdx.x; i < TR_HS; i += TR_THREADS) {
+      keys[i] = -1;
+      cnt[i] = 0;
+      fill[i] = 0;
+    }
+    if (threadIdx.x == 0) misc[1] = 0;
+    __syncthreads();
+    // ---- groups: insert each token's id (bounded probing; at most TR_CH < TR_HS keys)
+    for (int t = threadIdx.x; t < TR_CH; t += TR_THREADS) {
+      const int r = c0 + t;
+      int slot = -1;
+      if (r < M) {
+        const int id = ids[r];
+        if (id < 0 || int64_t(id) >= n_items) {
+          set_error(err, STCA_ERR_ID_OUT_OF_RANGE);
+        } else {
+          uint32_t h = (uint32_t(id) * 2654435761u) >> (32 - 11);
+          for (int p = 0; p < TR_HS; ++p, h = (h + 1) & (TR_HS - 1)) {
+            const int k = atomicCAS(&keys[h], -1, id);
+            if (k == -1 || k == id) {
+              slot = int(h);
+              break;
+            }
+          }
+          if (slot >= 0) atomicAdd(&cnt[slot], 1);
+          else set_error(err, STCA_ERR_CAPACITY);
+        }
+      }
+      slot_of[t] = slot;
+    }
+    __syncthreads();
+    // ---- exclusive scans of the member counts and of the non-empty slots (8 slots a thread)
+    {
+      const int s0 = threadIdx.x * (TR_HS / TR_THREADS);
+      int sum = 0, ne = 0;
+#pragma unroll
+      for (int i = 0; i < TR_HS / TR_THREADS; ++i) {
+        sum += cnt[s0 + i];
+        ne += cnt[s0 + i] > 0;
+      }
+      int isum = sum, ine = ne;  // inclusive warp scans
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int a = __shfl_up_sync(0xffffffffu, isum, o), b = __shfl_up_sync(0xffffffffu, ine, o);
+        if (lane >= o) {
+          isum += a;
+          ine += b;
+        }
+      }
+      if (lane == 31) {
+        warp_sum[warp] = isum;
+        warp_ne[warp] = ine;
+      }
+      __syncthreads();
+      int base = isum - sum, gbase = ine - ne;
+      for (int w = 0; w < warp; ++w) {
+        base += warp_sum[w];
+        gbase += warp_ne[w];
+      }
+      if (threadIdx.x == TR_THREADS - 1) misc[0] = gbase + ne;
+#pragma unroll
+      for (int i = 0; i < TR_HS / TR_THREADS; ++i) {
+        const int c = cnt[s0 + i];
+        start[s0 + i] = base;
+        base += c;
+        if (c > 0) gslot[gbase++] = s0 + i;
+      }
+    }
+    __syncthreads();
+    for (int t = threadIdx.x; t < TR_CH; t += TR_THREADS) {
+      const int slot = slot_of[t];
+      if (slot >= 0) order[start[slot] + atomicAdd(&fill[slot], 1)] = t;
+    }
+    __syncthreads();
+    // ---- one warp per group (taken in turn): sum the members' rows, then one add per id
+    const int ngroups = misc[0];
+    while (true) {
+      int g = 0;
+      if (lane == 0) g = atomicAdd(&misc[1], 1);
+      g = __shfl_sync(0xffffffffu, g, 0);
+      if (g >= ngroups) break;
+      const int slot = gslot[g];
+      const int64_t id = keys[slot];
+      const int beg = start[slot], n = cnt[slot];
+      float acc[DV][8];
+#pragma unroll
+      for (int v = 0; v < DV; ++v)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[v][j] = 0.f;
+      for (int m = 0; m < n; m += 4) {
+        uint4 u[4][DV];
+        int rr[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          rr[q] = m + q < n ? c0 + order[beg + m + q] : -1;
+#pragma unroll
+          for (int v = 0; v < DV; ++v)
+            u[q][v] = rr[q] >= 0 ? *reinterpret_cast<const uint4*>(dX + int64_t(rr[q]) * d + v * 256 + lane * 8)
+                                 : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int b = (with_dt && rr[q] >= 0) ? dt_bucket(dt[rr[q]]) : 0;
+#pragma unroll
+          for (int v = 0; v < DV; ++v) {
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u[q][v]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float2 f = __bfloat1622float2(h2[j]);
+              acc[v][2 * j] += f.x;
+              acc[v][2 * j + 1] += f.y;
+              if (with_dt && rr[q] >= 0) {
+                atomicAdd(bucket_acc + b * d + v * 256 + lane * 8 + 2 * j, f.x);
+                atomicAdd(bucket_acc + b * d + v * 256 + lane * 8 + 2 * j + 1, f.y);
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < DV; ++v) {
+        float4* row = reinterpret_cast<float4*>(dtable + id * d + v * 256 + lane * 8);
+        atomicAdd(row, make_float4(acc[v][0], acc[v][1], acc[v][2], acc[v][3]));
+        atomicAdd(row + 1, make_float4(acc[v][4], acc[v][5], acc[v][6], acc[v][7]));
+      }
+    }
+    __syncthreads();  // the chunk's tables are reset next
+  }
+  griddep_launch();
+  if (!with_dt) return;
+  __syncthreads();
+  for (int i = threadIdx.x; i < 16 * d; i += TR_THREADS)
+    if (bucket_acc[i] != 0.f) atomicAdd(ddt_table + i, bucket_acc[i]);
+}
+
 // dst [K, 2N] from W [K, N] without transposing: mode 3 puts column n of W at column
 // 128 (n / 64) + off + n % 64 (the head-interleaved [K_h | V_h] layout, d_h = 64), mode 4
 // at column off + n (two blocks side by side)
@@ -569,6 +740,18 @@ int table_rows_bwd(const void* dX, int M, int d, const int32_t* ids, const int32
   if (!dX || !ids || !dtable || ((reinterpret_cast<uintptr_t>(dX) | reinterpret_cast<uintptr_t>(dtable)) & 15))
     return STCA_ERR_INVALID_ARG;
   const bool with_dt = dt && ddt_table;
+  if (d == 256 || d == 512) {  // tokens grouped by id per chunk
+    const size_t smem = TR_SMEM_INT + (with_dt ? size_t(16) * d * 4 : 0);
+    const int blocks = std::max(1, std::min(4 * sm_count(), (M + TR_CH - 1) / TR_CH));
+    auto kern = d == 256 ? table_rows_grouped_kernel<1> : table_rows_grouped_kernel<2>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+      return STCA_ERR_CUDA;
+    if (launch_dep(kern, dim3(blocks), dim3(TR_THREADS), smem, s, static_cast<const bf16*>(dX), M, ids,
+                   with_dt ? dt : nullptr, n_items, dtable, with_dt ? ddt_table : nullptr, err) != cudaSuccess)
+      return STCA_ERR_CUDA;
+    note_launch();
+    return STCA_OK;
+  }
   const size_t smem = with_dt ? size_t(16) * d * 4 : 0;
   if (smem > 48 * 1024) return STCA_ERR_UNSUPPORTED;
   const int blocks = std::max(1, std::min(4 * sm_count(), (M + 7) / 8));

@@ -125,6 +125,46 @@ def test_swiglu_bwd_fp32_and_bf16_copy():
     assert torch.equal(out, P[:, :h].to(torch.bfloat16))
 
 
+@pytest.mark.parametrize("d", [128, 256, 512])
+@pytest.mark.parametrize("ids_kind", ["hot", "single", "uniform"])
+def test_table_rows_bwd_matches_oracle(d, ids_kind):
+    """The lookup's backward dE[ids] += dX, dT[bucket] += dX (stca_grad.table_rows_bwd) on
+    5003 tokens (ragged against the 1024-token groups): half the tokens on one id, or every
+    token on one id, or uniform ids; with time buckets.  d = 128 runs the per-token kernel,
+    256 and 512 the grouped one."""
+    g = np.random.default_rng(d)
+    M, n_items = 5003, 700
+    ids = g.integers(0, n_items, M)
+    if ids_kind == "hot":
+        ids[g.random(M) < 0.5] = 17
+    elif ids_kind == "single":
+        ids[:] = 3
+    dt = g.integers(0, 10 ** 6, M)
+    dX16 = to_bf16(g.standard_normal((M, d)))
+    ids_t = torch.from_numpy(ids.astype(np.int32)).to(dev)
+    dt_t = torch.from_numpy(dt.astype(np.int32)).to(dev)
+    dtab = torch.zeros((n_items, d), device=dev)
+    ddt = torch.zeros((16, d), device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    B.check(B.stca_k_table_rows_bwd(dX16, M, d, ids_t, dt_t, n_items, dtab, ddt, err))
+    rtab, rdt = np.zeros((n_items, d)), np.zeros((16, d))
+    G.table_rows_bwd(rtab, rdt, ids, dt, bf16_to_f64(dX16))
+    assert err.item() == 0
+    assert normwise(dtab.cpu().numpy(), rtab) < 1e-5
+    assert normwise(ddt.cpu().numpy(), rdt) < 1e-5
+    # an id outside the table is reported and its row is skipped
+    ids2 = ids.copy()
+    ids2[100] = n_items
+    B.check(B.stca_k_table_rows_bwd(dX16, M, d, torch.from_numpy(ids2.astype(np.int32)).to(dev), None, n_items,
+                                    dtab.zero_(), None, err))
+    assert err.item() == B.ERR_ID_OUT_OF_RANGE
+    keep = np.ones(M, bool)
+    keep[100] = False
+    rtab = np.zeros((n_items, d))
+    G.table_rows_bwd(rtab, None, ids[keep], None, bf16_to_f64(dX16)[keep])
+    assert normwise(dtab.cpu().numpy(), rtab) < 1e-5
+
+
 @pytest.mark.parametrize("config", [2, 3])
 def test_history_layer_backward_matches_oracle(config):
     """config 2's shape (d = 256, h = 512, no time feature) and config 3's (d = 512,
