@@ -378,10 +378,13 @@ int stca_attention_train_forward(const float* Q, const void* KV, const int32_t* 
  *   dV_j = sum_t p_tj dout_t, dK_j = sum_t ds_tj q_t / sqrt(d_h), dQ_t = sum_j ds_tj k_j / sqrt(d_h)
  * with s = q . k / sqrt(d_h) per head; a key's gradient sums over all of its user's
  * targets, and a key with no target of its user gets 0.  part_dq [splits, T, d] float32
- * scratch for splits > 1 (may be NULL when splits == 1).  Deterministic: no atomics. */
+ * scratch for splits > 1 (may be NULL when splits == 1).  dkv_bf16 (may be NULL): when
+ * given, the K/V gradients are written there as bf16 [N, H, 2 d_h] (rounded to nearest
+ * even from the same fp32 sums) and dKV only holds the fp32 partial sums of users with
+ * more than 16 targets; 16-byte aligned.  Deterministic: no atomics. */
 int stca_attention_backward(const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B, int T,
                             int d, int H, int splits, int score, const float* out, const float* lse,
-                            const float* dout, float* dQ, float* dKV, float* part_dq, void* stream);
+                            const float* dout, float* dQ, float* dKV, float* part_dq, void* dkv_bf16, void* stream);
 
 #ifdef __cplusplus
 }

@@ -86,7 +86,7 @@ _SIGS = [
     ("stca_attention_train_forward", _i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
                                             _vp, _vp, _vp]),
     ("stca_attention_backward", _i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
-                                       _vp, _vp, _vp]),
+                                       _vp, _vp, _vp, _vp]),
     ("hyformer_forward", _i32, [_vp, _vp, _vp, _i32, _vp, _vp, _i32, _vp, _i32, _i32, ctypes.POINTER(HyfWeights),
                                 _vp, _vp]),
     ("stca_sync_status", _i32, [_vp]),
@@ -291,10 +291,12 @@ def stca_attention_train_forward(Q, KV, hoff, toff, B, T, d, H, splits, score, p
 
 
 def stca_attention_backward(Q, KV, hoff, toff, B, T, d, H, splits, score, out, lse, dout, dQ, dKV, part_dq=None,
-                            stream=None) -> int:
-    """Backward of the attention step: dQ [T, d] and dKV [N, H, 2 d_h] (fp32)."""
+                            stream=None, dKV16=None) -> int:
+    """Backward of the attention step: dQ [T, d] and dKV [N, H, 2 d_h] (fp32; or bf16 into
+    dKV16 when given, dKV then holding only partial sums)."""
     return lib().stca_attention_backward(ptr(Q), ptr(KV), ptr(hoff), ptr(toff), B, T, d, H, splits, score, ptr(out),
-                                         ptr(lse), ptr(dout), ptr(dQ), ptr(dKV), ptr(part_dq), stream_ptr(stream))
+                                         ptr(lse), ptr(dout), ptr(dQ), ptr(dKV), ptr(part_dq), ptr(dKV16),
+                                         stream_ptr(stream))
 
 
 def hyformer_forward(h, ids_feed, len_feed, n_feed, ids_search, len_search, n_search, q0, B, n_query,

@@ -66,7 +66,8 @@ struct BwdArgs {
   const float* lse;   // [T, H] softmax log-sum-exp (natural log)
   const float* dO;    // [T, d]
   float* dQ;          // [T, d]
-  float* dKV;         // [N, H, 2 d_h] fp32: [dK_h | dV_h] per head
+  float* dKV;         // [N, H, 2 d_h] fp32: [dK_h | dV_h] per head (with dKV16: partial sums only)
+  bf16* dKV16;        // [N, H, 2 d_h] bf16 result, or null
   float* part_dq;     // [splits, T, d] when splits > 1
   int B, T, d, H, splits;
 };
@@ -90,7 +91,10 @@ __global__ void __launch_bounds__(B_THREADS, 4) attn_bwd_kernel(BwdArgs a) {
   if (m <= 0) {  // no target attends to these keys: zero gradients
     for (int64_t i = threadIdx.x; i < int64_t(nk) * (2 * BD / 4); i += B_THREADS) {
       const int64_t key = k0 + i / (2 * BD / 4);
-      reinterpret_cast<float4*>(a.dKV + key * ld + kvcol)[i % (2 * BD / 4)] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (a.dKV16)
+        reinterpret_cast<uint2*>(a.dKV16 + key * ld + kvcol)[i % (2 * BD / 4)] = make_uint2(0u, 0u);
+      else
+        reinterpret_cast<float4*>(a.dKV + key * ld + kvcol)[i % (2 * BD / 4)] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
     return;
   }
@@ -297,7 +301,11 @@ __global__ void __launch_bounds__(B_THREADS, 4) attn_bwd_kernel(BwdArgs a) {
         for (int hr = 0; hr < 2; ++hr) {
           const int key = g + 8 * hr;
           if (key < valid) {
-            float* dst = a.dKV + (row0 + key) * ld + kvcol + which * BD + 2 * tq;
+            const int64_t off = (row0 + key) * ld + kvcol + which * BD + 2 * tq;
+            float* dst = a.dKV + off;
+            // the last query chunk writes the bf16 result when one is asked for; earlier
+            // chunks keep fp32 partial sums
+            const bool to16 = a.dKV16 && qp + BQ >= m;
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
               float2 v = make_float2(acc[nt][2 * hr], acc[nt][2 * hr + 1]);
@@ -306,7 +314,10 @@ __global__ void __launch_bounds__(B_THREADS, 4) attn_bwd_kernel(BwdArgs a) {
                 v.x += prev.x;
                 v.y += prev.y;
               }
-              *reinterpret_cast<float2*>(dst + nt * 8) = v;
+              if (to16)
+                *reinterpret_cast<uint32_t*>(a.dKV16 + off + nt * 8) = pack_bf16x2(v.x, v.y);
+              else
+                *reinterpret_cast<float2*>(dst + nt * 8) = v;
             }
           }
         }
@@ -369,7 +380,7 @@ __global__ void sum_splits_kernel(const float* __restrict__ part, int splits, in
 
 int attention_bwd_bf16(const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B, int T, int d,
                        int H, int splits, int score, const float* O, const float* lse, const float* dO, float* dQ,
-                       float* dKV, float* part_dq, cudaStream_t s) {
+                       float* dKV, float* part_dq, void* dKV16, cudaStream_t s) {
   if (B == 0) return 0;
   if (d % H != 0 || d / H != BD) return STCA_ERR_UNSUPPORTED;
   BwdArgs a;
@@ -382,6 +393,7 @@ int attention_bwd_bf16(const float* Q, const void* KV, const int32_t* hoff, cons
   a.dO = dO;
   a.dQ = dQ;
   a.dKV = dKV;
+  a.dKV16 = reinterpret_cast<bf16*>(dKV16);
   a.part_dq = part_dq;
   a.B = B;
   a.T = T;
@@ -460,13 +472,14 @@ extern "C" int stca_attention_train_forward(const float* Q, const void* KV, cons
 extern "C" int stca_attention_backward(const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff,
                                        int B, int T, int d, int H, int splits, int score, const float* out,
                                        const float* lse, const float* dout, float* dQ, float* dKV, float* part_dq,
-                                       void* stream) {
+                                       void* dkv_bf16, void* stream) {
   int rc = train_args_ok(Q, KV, hoff, toff, B, T, d, H, splits, score);
   if (rc != STCA_OK) return rc;
   if (B == 0) return STCA_OK;
-  if (!dKV || (T > 0 && (!dout || !dQ || (score == 0 && (!out || !lse)))) || (splits > 1 && T > 0 && !part_dq))
+  if (!dKV || (T > 0 && (!dout || !dQ || (score == 0 && (!out || !lse)))) || (splits > 1 && T > 0 && !part_dq) ||
+      (reinterpret_cast<uintptr_t>(dkv_bf16) & 15))
     return STCA_ERR_INVALID_ARG;
   return stca::attention_bwd_bf16(Q, KV, hoff, toff, B, T, d, H, splits, score, out, lse, dout, dQ, dKV, part_dq,
-                                  reinterpret_cast<cudaStream_t>(stream));
+                                  dkv_bf16, reinterpret_cast<cudaStream_t>(stream));
 }
 

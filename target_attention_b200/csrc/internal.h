@@ -219,7 +219,7 @@ int attention_fold_bf16(const FoldArgs& a, cudaStream_t s);
 // Backward of the bf16 attention (per-token K/V rows, d_h = 64); see stca_attention_backward.
 int attention_bwd_bf16(const float* Q, const void* KV, const int32_t* hoff, const int32_t* toff, int B, int T, int d,
                        int H, int splits, int score, const float* O, const float* lse, const float* dO, float* dQ,
-                       float* dKV, float* part_dq, cudaStream_t s);
+                       float* dKV, float* part_dq, void* dKV16, cudaStream_t s);
 int attention_f32(const AttnArgs& a, cudaStream_t s);
 // combines the slices; not needed after attention_bf16 with splits == 1, which writes out
 int attention_merge(const AttnArgs& a, cudaStream_t s);

@@ -303,14 +303,14 @@ class StcaTrainingStep:
         g["WZ"] = self._wgrad(cat16, C, self._to_bf16(dzin, d, d), d, C, d)
         self._gq(dzin, d, d, w["WZ"], C, self.dcat, C)                    # d cat = dzin W_Z^T (every block)
         dobar, dQ, dq = self.f32(max(T, 1), d), self.f32(max(T, 1), d), self.f32(max(T, 1), d)
-        dKV = self.f32(max(N, 1), 2 * d)
+        dKV = self.f32(max(N, 1), 2 * d)        # fp32 partial sums of users with more than 16 targets
         dKV16 = self.bf(max(N, 1), 2 * d)
         for i in reversed(range(M)):
             dout = self.dcat[:, i * d:]
             g["WO"][i] = self._wgrad(self._to_bf16(self.obar[i], d, d), d, self._to_bf16(dout, C, d), d, d, d)
             self._gq(dout, C, d, w["WO"][i], d, dobar, d)                 # d obar = d o W_O^T
             B.check(B.stca_attention_backward(self.Qp[i], self.KV[i], hoff, toff, self.B, T, d, H, 1, sc, self.obar[i],
-                                              self.lse[i] if sc == 0 else None, dobar, dQ, dKV, None),
+                                              self.lse[i] if sc == 0 else None, dobar, dQ, dKV, None, dKV16=dKV16),
                     "attention backward")
             g["WQ"][i] = self._wgrad(self._to_bf16(self.q[i], d, d), d, self._to_bf16(dQ, d, d), d, d, d)
             self._gq(dQ, d, d, w["WQ"][i], d, dq, d)                      # dq = dQ W_Q^T
@@ -329,7 +329,6 @@ class StcaTrainingStep:
                 self._gq(du, d, d, w["WC"][i][:i * d], i * d, self.dcat, C, R=self.dcat, ldr=C)
                 self._gq(du, d, d, w["WC"][i][i * d:], d, xt_blk, C, R=xt_blk, ldr=C)
             # the history side of layer i from its K/V rows' gradients
-            B.check(B.stca_k_f32_to_bf16(dKV, 2 * d, N, 2 * d, dKV16, 2 * d), "bf16 copy")
             L = self.hist[i]
             L.backward(dKV16, ids, dt, n_items, dtable, ddt_table, xt_ready=True)
             # [dW_K | dW_V] in the K/V rows' head-interleaved columns: head j's K at 128 j, V at 128 j + 64

@@ -164,10 +164,11 @@ def test_training_entries_reject_bad_arguments_on_host():
     assert f(16, 16, 16, 16, 1, 1, 256, 4, 1, 0, None, None, 16, None, None, None) == B.ERR_INVALID_ARG  # lse
     assert f(16, 16, 16, 16, 1, 1, 256, 4, 2, 0, None, None, 16, 16, None, None) == B.ERR_INVALID_ARG  # scratch
     assert f(16, 16, 16, 16, 1, 1, 256, 8, 1, 0, None, None, 16, 16, None, None) == B.ERR_UNSUPPORTED  # d_h 32
-    assert b(16, 16, 16, 16, 1, 1, 256, 4, 1, 0, 16, 16, 16, 16, None, None, None) == B.ERR_INVALID_ARG  # dKV
-    assert b(16, 16, 16, 16, 1, 1, 256, 4, 2, 0, 16, 16, 16, 16, 16, None, None) == B.ERR_INVALID_ARG  # part_dq
-    assert b(16, 16, 16, 16, 1, 1, 256, 4, 1, 0, None, None, 16, 16, 16, None, None) == B.ERR_INVALID_ARG  # out
-    assert b(16, 16, 16, 16, 1, 1, 512, 4, 1, 0, 16, 16, 16, 16, 16, None, None) == B.ERR_UNSUPPORTED  # d_h 128
+    assert b(16, 16, 16, 16, 1, 1, 256, 4, 1, 0, 16, 16, 16, 16, None, None, None, None) == B.ERR_INVALID_ARG  # dKV
+    assert b(16, 16, 16, 16, 1, 1, 256, 4, 2, 0, 16, 16, 16, 16, 16, None, None, None) == B.ERR_INVALID_ARG  # part_dq
+    assert b(16, 16, 16, 16, 1, 1, 256, 4, 1, 0, None, None, 16, 16, 16, None, None, None) == B.ERR_INVALID_ARG  # out
+    assert b(16, 16, 16, 16, 1, 1, 512, 4, 1, 0, 16, 16, 16, 16, 16, None, None, None) == B.ERR_UNSUPPORTED  # d_h 128
+    assert b(16, 16, 16, 16, 1, 1, 256, 4, 1, 0, 16, 16, 16, 16, 16, None, 18, None) == B.ERR_INVALID_ARG  # bf16 out
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -63,7 +63,16 @@ def _backward(x, score, splits, out, lse):
     pdq = torch.empty((splits, max(x["T"], 1), D), device=dev)
     B.check(B.stca_attention_backward(x["Qt"], x["KVt"], x["hoff"], x["toff"], x["B"], x["T"], D, H, splits, score,
                                       out, lse, x["dOt"], dQ, dKV, pdq), "backward")
+    # the bf16 form: the same fp32 sums rounded to nearest even, dKV only as scratch
+    dQ2 = torch.empty_like(dQ)
+    scratch = torch.full_like(dKV, float("nan"))
+    dKV16 = torch.full(dKV.shape, float("nan"), dtype=torch.bfloat16, device=dev)
+    B.check(B.stca_attention_backward(x["Qt"], x["KVt"], x["hoff"], x["toff"], x["B"], x["T"], D, H, splits, score,
+                                      out, lse, x["dOt"], dQ2, scratch, pdq, dKV16=dKV16), "backward, bf16 K/V")
     torch.cuda.synchronize()
+    n = x["N"]
+    assert torch.equal(dKV16[:n], dKV[:n].to(torch.bfloat16))
+    assert torch.equal(dQ2, dQ)
     return dQ.cpu().numpy()[:x["T"]], dKV.cpu().numpy()[:x["N"]]
 
 
