@@ -44,10 +44,13 @@ int stca_k_pack_weight(const void* W, int K, int N, void* dst, int mode, int row
  * An id outside [0, n_items) reads as a zero row and records STCA_ERR_ID_OUT_OF_RANGE.
  * x_out (amode 1 only, else STCA_ERR_INVALID_ARG; may be null): bf16 [M, K], 16-byte
  * aligned, receives the gathered A rows exactly as the MMAs consumed them, so that later
- * GEMMs over the same rows can take them as a dense amode-0 operand. */
+ * GEMMs over the same rows can take them as a dense amode-0 operand.  p_out (epi 1 only,
+ * else STCA_ERR_INVALID_ARG; may be null): bf16 [M, 2 Nout], 16-byte aligned, receives the
+ * pre-activations [A W1 | A W3] rounded from the same fp32 accumulators (the training
+ * backward's SwiGLU derivative needs them). */
 int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, const int32_t* dt, const void* table,
                          const void* dt_table, int64_t n_items, int M, int K, const void* Wp, int Nout, void* C,
-                         int ldc, void* x_out, int32_t* err, void* stream);
+                         int ldc, void* x_out, void* p_out, int32_t* err, void* stream);
 
 /* Fused history FFN of `layers` layers for d = 256 ([notes] STCA: X~_l = LN_l(SwiGLU_l(X))
  * from the original X; [wechat] §1.1 lookup while computing).  Rows r < M of X are

@@ -100,7 +100,7 @@ _SIGS = [
     ("stca_k_offsets", _i32, [_vp, _i32, _vp, _i32, _vp, _vp]),
     ("stca_k_pack_weight", _i32, [_vp, _i32, _i32, _vp, _i32, _i32, _vp]),
     ("stca_k_gemm_resident", _i32, [_i32, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _vp, _i32, _vp, _i32, _vp,
-                                    _vp, _vp]),
+                                    _vp, _vp, _vp]),
     ("stca_k_ffn_fused", _i32, [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp, ctypes.c_float, _vp,
                           _i32, _vp, _vp, _vp]),
     ("stca_k_gemm_query", _i32, [_vp, _i64, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _vp, _i64, _vp, _i64, _vp,
@@ -318,9 +318,10 @@ def stca_k_pack_weight(W, K, N, dst, mode, row_offset, stream=None) -> int:
 
 
 def stca_k_gemm_resident(amode, epi, A, ids, dt, table, dt_table, n_items, M, K, Wp, Nout, C, ldc, err,
-                         stream=None, x_out=None) -> int:
+                         stream=None, x_out=None, p_out=None) -> int:
     return lib().stca_k_gemm_resident(amode, epi, ptr(A), ptr(ids), ptr(dt), ptr(table), ptr(dt_table), n_items, M,
-                                      K, ptr(Wp), Nout, ptr(C), ldc, ptr(x_out), ptr(err), stream_ptr(stream))
+                                      K, ptr(Wp), Nout, ptr(C), ldc, ptr(x_out), ptr(p_out), ptr(err),
+                                      stream_ptr(stream))
 
 
 def stca_k_gemm_query(A, lda, M, K, ksplit, kshift, Wp, N, dual, R, ldr, C, ldc, err, stream=None) -> int:

@@ -37,6 +37,9 @@ struct EpiFold {
   const float* stats;
   const float* cvec;
   const float* bvec;
+  // EPI_SWIGLU only: when set, bf16 [M, 2 Nout] receiving the pre-activations [A W1 | A W3]
+  // (rounded from the same fp32 accumulators), which the training backward needs
+  void* p_out;
 };
 // c and b of the fold for W = [WK | WV] ([d, d] bf16 each, row-major): out [2][2d] fp32,
 // in the K/V GEMM's output column order: head-interleaved [K_h | V_h] per head of width dh
@@ -77,11 +80,13 @@ int tc_pack_weights(const PackJob* jobs, int n, cudaStream_t s);
 // M_dev, when not null, is a device int holding the number of rows actually present
 // (<= M); M then only sizes the tensor maps and buffers.  x_out (A_GATHER only, may be
 // null): bf16 [M, K] receiving the gathered A rows (E[id] + T[bucket]) as the MMAs used them.
+// p_out (EPI_SWIGLU only, may be null): bf16 [M, 2 Nout] receiving [A W1 | A W3].
 // max_pairs > 0 caps the persistent grid at that many CTA pairs (leaving SMs to kernels that
 // run beside it on another stream).
 int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int K, const void* Wp,
                      int Nout, void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev = nullptr,
-                     void* x_out = nullptr, const EpiFold* fold = nullptr, int max_pairs = 0);
+                     void* x_out = nullptr, const EpiFold* fold = nullptr, int max_pairs = 0,
+                     void* p_out = nullptr);
 
 // C[M, N] (bf16) = epi(A Wp^T), A dense bf16 [M, K] streamed (K a multiple of 64),
 // N in {256, 512}; epi EPI_LN applies LayerNorm (gamma, beta, eps) over the full row.

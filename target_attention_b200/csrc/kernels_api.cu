@@ -83,9 +83,10 @@ int stca_k_table_rows_bwd(const void* dX, int M, int d, const int32_t* ids, cons
 
 int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, const int32_t* dt, const void* table,
                          const void* dt_table, int64_t n_items, int M, int K, const void* Wp, int Nout, void* C,
-                         int ldc, void* x_out, int32_t* err, void* stream) {
+                         int ldc, void* x_out, void* p_out, int32_t* err, void* stream) {
   if (M < 0 || !Wp || (M > 0 && !C)) return STCA_ERR_INVALID_ARG;
   if (x_out && amode != A_GATHER) return STCA_ERR_INVALID_ARG;
+  if (p_out && epi != EPI_SWIGLU) return STCA_ERR_INVALID_ARG;
   if (epi != EPI_PLAIN && epi != EPI_SWIGLU) return STCA_ERR_INVALID_ARG;
   GatherSrc g;
   memset(&g, 0, sizeof(g));
@@ -100,7 +101,7 @@ int stca_k_gemm_resident(int amode, int epi, const void* A, const int32_t* ids, 
     return STCA_ERR_INVALID_ARG;
   }
   return tc_gemm_resident(amode, epi, A, g, M, K, Wp, Nout, C, ldc, err, reinterpret_cast<cudaStream_t>(stream),
-                          nullptr, x_out);
+                          nullptr, x_out, nullptr, 0, p_out);
 }
 
 int stca_k_ffn_fused(const int32_t* ids, const int32_t* dt, const void* table, const void* dt_table, int64_t n_items,

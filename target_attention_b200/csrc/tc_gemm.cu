@@ -107,8 +107,8 @@ template <int AMODE, int EPI, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
     tc_gemm_resident_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmX,
-                            GatherSrc g, int M_max, int K, int NT, int store_x, int32_t* err, const int32_t* M_dev,
-                            EpiFold fold) {
+                            const __grid_constant__ CUtensorMap tmP, GatherSrc g, int M_max, int K, int NT,
+                            int store_x, int32_t* err, const int32_t* M_dev, EpiFold fold) {
   griddep_wait();
   griddep_launch();
   extern __shared__ uint8_t smem_raw[];
@@ -420,6 +420,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
             tmem_ld_32x32b_x32(tb + col, gv);
             tmem_ld_32x32b_x32(tb + 128 + col, uv);
             tmem_ld_wait();
+            if (fold.p_out) {  // the pre-activations [A W1 | A W3], tile stores like C's
+              epi_store(stage, gv, lane, &tmP, nt * 128 + col, y);
+              epi_store(stage, uv, lane, &tmP, NT * 128 + nt * 128 + col, y);
+            }
 #pragma unroll
             for (int e = 0; e < 32; ++e) gv[e] = silu_tanh(gv[e]) * uv[e];
             epi_store(stage, gv, lane, &tmC, nt * 128 + col, y);
@@ -843,8 +847,8 @@ size_t rowwise_smem(int nb, int stages) {
 
 template <int AMODE, int EPI, int STAGES>
 int run_resident(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const CUtensorMap& tx,
-                 int store_x, const GatherSrc& g, int M, int K, int NT, int32_t* err, cudaStream_t s,
-                 const int32_t* M_dev, const EpiFold& fold, int max_pairs) {
+                 const CUtensorMap& tp, int store_x, const GatherSrc& g, int M, int K, int NT, int32_t* err,
+                 cudaStream_t s, const int32_t* M_dev, const EpiFold& fold, int max_pairs) {
   auto kern = tc_gemm_resident_kernel<AMODE, EPI, STAGES>;
   const size_t smem = resident_smem(K, STAGES, AMODE == A_GATHER);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
@@ -852,7 +856,7 @@ int run_resident(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap
   int pairs = std::min((M + 2 * BM - 1) / (2 * BM), sm_count() / 2);
   if (max_pairs > 0) pairs = std::min(pairs, max_pairs);
   const int grid = 2 * pairs;
-  launch_dep(kern, dim3(grid), dim3(512), smem, s, ta, tb, tc, tx, g, M, K, NT, store_x, err, M_dev, fold);
+  launch_dep(kern, dim3(grid), dim3(512), smem, s, ta, tb, tc, tx, tp, g, M, K, NT, store_x, err, M_dev, fold);
   note_launch();
   return cudaGetLastError() == cudaSuccess ? 0 : STCA_ERR_CUDA;
 }
@@ -921,7 +925,7 @@ int tc_pack_weights(const PackJob* jobs, int n, cudaStream_t s) {
 
 int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int K, const void* Wp, int Nout,
                      void* C, int ldc, int32_t* err, cudaStream_t s, const int32_t* M_dev, void* x_out,
-                     const EpiFold* fold, int max_pairs) {
+                     const EpiFold* fold, int max_pairs, void* p_out) {
   if (M == 0) return 0;
   if (M < 0 || (K != 256 && K != 512) || Nout <= 0 || ldc % 8 != 0) return STCA_ERR_UNSUPPORTED;
   const int N = epi == EPI_SWIGLU ? 2 * Nout : Nout;
@@ -929,12 +933,14 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
   const int NT = N / 256;
   if (reinterpret_cast<uintptr_t>(C) % 16 != 0) return STCA_ERR_INVALID_ARG;
   if (x_out && (amode != A_GATHER || reinterpret_cast<uintptr_t>(x_out) % 16 != 0)) return STCA_ERR_INVALID_ARG;
+  if (p_out && (epi != EPI_SWIGLU || reinterpret_cast<uintptr_t>(p_out) % 16 != 0)) return STCA_ERR_INVALID_ARG;
   if (epi == EPI_LNFOLD && (!fold || !fold->stats || !fold->cvec || !fold->bvec || amode != A_TMA))
     return STCA_ERR_INVALID_ARG;
-  EpiFold fz;
-  memset(&fz, 0, sizeof(fz));
-  const EpiFold& fo = fold ? *fold : fz;
-  CUtensorMap ta, tb, tc, tx;
+  EpiFold fo;
+  memset(&fo, 0, sizeof(fo));
+  if (fold) fo = *fold;
+  fo.p_out = p_out;
+  CUtensorMap ta, tb, tc, tx, tp;
   memset(&ta, 0, sizeof(ta));
   if (!make_tmap(&tb, Wp, N, K, K, BM)) return STCA_ERR_CUDA;
   if (!make_tmap_out(&tc, C, M, Nout, ldc)) return STCA_ERR_CUDA;
@@ -950,10 +956,16 @@ int tc_gemm_resident(int amode, int epi, const void* A, GatherSrc g, int M, int 
     tx = tb;  // unused
   }
   const int sx = x_out != nullptr;
+  // P [M, 2 Nout] written by the SwiGLU epilogue: 32 x 32 boxes like C
+  if (p_out) {
+    if (!make_tmap_out(&tp, p_out, M, 2 * uint64_t(Nout), 2 * uint64_t(Nout))) return STCA_ERR_CUDA;
+  } else {
+    tp = tc;  // unused
+  }
   // stage counts fill the 227 KB of shared memory (see resident_smem)
 #define STCA_RES(AM, EP)                                                                                   \
-  (K == 512 ? run_resident<AM, EP, 5>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev, fo, max_pairs)     \
-            : run_resident<AM, EP, 9>(ta, tb, tc, tx, sx, g, M, K, NT, err, s, M_dev, fo, max_pairs))
+  (K == 512 ? run_resident<AM, EP, 5>(ta, tb, tc, tx, tp, sx, g, M, K, NT, err, s, M_dev, fo, max_pairs)     \
+            : run_resident<AM, EP, 9>(ta, tb, tc, tx, tp, sx, g, M, K, NT, err, s, M_dev, fo, max_pairs))
   if (amode == A_TMA && epi == EPI_PLAIN) return STCA_RES(A_TMA, EPI_PLAIN);
   if (amode == A_TMA && epi == EPI_LNFOLD) return STCA_RES(A_TMA, EPI_LNFOLD);
   if (amode == A_TMA && epi == EPI_SWIGLU) return STCA_RES(A_TMA, EPI_SWIGLU);

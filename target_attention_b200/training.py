@@ -29,10 +29,10 @@ class HistoryLayerBackward:
         self.W2 = W2
         # operand layouts: forward GEMMs take packed weights, backward GEMMs the weights
         # as they are or with their columns placed side by side / head-interleaved
-        self.W13p, self.Pp, self.W2p = bf(2 * h, d), bf(2 * h, d), bf(d, h)
+        self.W13p, self.W2p = bf(2 * h, d), bf(d, h)
         self.WKVi, self.W13c = bf(d, 2 * d), bf(d, 2 * h)
-        for args in ((W1, d, h, self.W13p, 1, 0), (W3, d, h, self.W13p, 2, 0), (W1, d, h, self.Pp, 0, 0),
-                     (W3, d, h, self.Pp, 0, h), (W2, h, d, self.W2p, 0, 0), (WK, d, d, self.WKVi, 3, 0),
+        for args in ((W1, d, h, self.W13p, 1, 0), (W3, d, h, self.W13p, 2, 0), (W2, h, d, self.W2p, 0, 0),
+                     (WK, d, d, self.WKVi, 3, 0),
                      (WV, d, d, self.WKVi, 3, 64), (W1, d, h, self.W13c, 4, 0), (W3, d, h, self.W13c, 4, h)):
             B.check(B.stca_k_pack_weight(*args), "pack")
         # activations and gradients of the rows
@@ -51,10 +51,10 @@ class HistoryLayerBackward:
     def recompute(self, ids, dt, table, dt_table, n_items, stream=None, on_step=None):
         M, d, h, e = self.M, self.d, self.h, self.err
         step = _stepper(on_step)
+        # A = SiLU(X W1) * (X W3), with the gathered X and the pre-activations P = [X W1 | X W3]
+        # written by the same GEMM
         step(B.stca_k_gemm_resident(1, 1, None, ids, dt, table, dt_table, n_items, M, d, self.W13p, h, self.A, h, e,
-                                       stream, x_out=self.X), "SwiGLU GEMM")
-        step(B.stca_k_gemm_resident(0, 0, self.X, None, None, None, None, 0, M, d, self.Pp, 2 * h, self.P, 2 * h, e,
-                                       stream), "X [W1 | W3]")
+                                       stream, x_out=self.X, p_out=self.P), "SwiGLU GEMM")
         step(B.stca_k_gemm_rowwise(0, self.A, M, h, self.W2p, d, None, None, self.eps, self.y, d, e, stream),
                 "A W2")
 
@@ -88,7 +88,7 @@ class HistoryLayerBackward:
     def flops(self):
         """Multiply-add work of each GEMM of recompute() + backward(), in flop."""
         M, d, h = self.M, self.d, self.h
-        return {"SwiGLU GEMM": 2 * M * d * 2 * h, "X [W1 | W3]": 2 * M * d * 2 * h, "A W2": 2 * M * h * d,
+        return {"SwiGLU GEMM": 2 * M * d * 2 * h, "A W2": 2 * M * h * d,
                 "dKV [W_K | W_V]^T": 2 * M * 2 * d * d, "Xt^T dKV": 2 * M * d * 2 * d, "dy W2^T": 2 * M * d * h,
                 "A^T dy": 2 * M * h * d, "dP [W1 | W3]^T": 2 * M * 2 * h * d, "X^T dP": 2 * M * d * 2 * h}
 

@@ -137,10 +137,12 @@ def test_null_arguments_rejected_on_host():
     assert L.stca_k_f32_to_bf16(16, 8, 4, 16, 16, 16, None) == B.ERR_INVALID_ARG                           # lds < cols
     assert L.stca_k_table_rows_bwd(16, 10, 256, None, None, 100, 16, None, None, None) == B.ERR_INVALID_ARG
     assert L.stca_k_gemm_resident(1, 1, None, None, None, None, None, 0, 5, 256, None, 128, None, 128, None, None,
-                                  None) == B.ERR_INVALID_ARG
-    # x_out only with the gather
+                                  None, None) == B.ERR_INVALID_ARG
+    # x_out only with the gather, p_out only with the SwiGLU epilogue
     assert L.stca_k_gemm_resident(0, 0, 16, None, None, None, None, 0, 5, 256, 16, 256, 16, 256, 16, None,
-                                  None) == B.ERR_INVALID_ARG
+                                  None, None) == B.ERR_INVALID_ARG
+    assert L.stca_k_gemm_resident(0, 0, 16, None, None, None, None, 0, 5, 256, 16, 256, 16, 256, None, 16,
+                                  None, None) == B.ERR_INVALID_ARG
     assert L.stca_k_attention(1, 16, 16, 16, 16, 1, 1, 256, 4, 33, 0, 16, 16, 16, None, None) == B.ERR_INVALID_ARG
     # target-side GEMM: missing operands, then shapes the tensor-core kernel does not take
     assert L.stca_k_gemm_query(None, 64, 1, 64, 64, 0, None, 32, 0, None, 0, None, 32, None, None) \

@@ -452,11 +452,20 @@ def test_gather_swiglu_many_tiles_per_pair(with_dt):
     C = torch.empty((M, hidden), dtype=torch.bfloat16, device=dev)
     Xw = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
     err = zeros_err()
+    P = torch.empty((M, 2 * hidden), dtype=torch.bfloat16, device=dev)
     B.check(B.stca_k_gemm_resident(1, 1, None, torch.from_numpy(ids).to(dev),
                                    torch.from_numpy(dt).to(dev) if with_dt else None, E, T, n_items, M, K, Wp,
-                                   hidden, C, hidden, err, x_out=Xw))
+                                   hidden, C, hidden, err, x_out=Xw, p_out=P))
     torch.cuda.synchronize()
     assert err.item() == 0
+    # the pre-activations [X W1 | X W3]: the plain GEMM over the written-through rows gives
+    # the same fp32 accumulators (same K order), so the same bits
+    Pp = _pack(W1, 0, 2 * hidden)
+    _pack(W3, 0, 2 * hidden, dst=Pp, row_offset=hidden)
+    P2 = torch.empty_like(P)
+    B.check(B.stca_k_gemm_resident(0, 0, Xw, None, None, None, None, 0, M, K, Pp, 2 * hidden, P2, 2 * hidden, err))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bits_of(P), bits_of(P2))
     # every written-through row, bit for bit (fp32 sum rounded once to bf16)
     Ef = E.float().cpu().numpy()[ids]
     if with_dt:
