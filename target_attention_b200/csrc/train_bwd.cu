@@ -642,9 +642,13 @@ int gemm_wgrad(const void* A, int64_t lda, const void* G, int64_t ldg, int M, in
   return STCA_OK;
 }
 
-int ln_bwd_blocks(int M) { return std::max(1, std::min(2 * sm_count(), (M + 31) / 32)); }
+// as many 256-thread blocks as fit on every SM at once (d = 256: 64 registers a thread, four
+// blocks; d = 512: 128 registers, two), so that more rows are in flight
+int ln_bwd_blocks(int M, int d) {
+  return std::max(1, std::min((d == 256 ? 4 : 2) * sm_count(), (M + 31) / 32));
+}
 
-size_t layer_norm_bwd_workspace_bytes(int M, int d) { return size_t(ln_bwd_blocks(M)) * 2 * d * 4; }
+size_t layer_norm_bwd_workspace_bytes(int M, int d) { return size_t(ln_bwd_blocks(M, d)) * 2 * d * 4; }
 
 template <typename T>
 static cudaError_t launch_ln_bwd(int d, int blocks, cudaStream_t s, const void* y, const void* dxt, int M,
@@ -659,7 +663,7 @@ int layer_norm_bwd(const void* y, const void* dxt, int M, int d, int fp32, const
                    size_t ws_bytes, cudaStream_t s) {
   if (M < 0 || (d != 256 && d != 512)) return STCA_ERR_UNSUPPORTED;
   if (!gamma || !dgamma || !dbeta || (M > 0 && (!y || !dxt || !dy))) return STCA_ERR_INVALID_ARG;
-  const int blocks = ln_bwd_blocks(M);
+  const int blocks = ln_bwd_blocks(M, d);
   if (ws_bytes < size_t(blocks) * 2 * d * 4 || !ws) return STCA_ERR_CAPACITY;
   float* part = static_cast<float*>(ws);
   const cudaError_t e = fp32 ? launch_ln_bwd<float>(d, blocks, s, y, dxt, M, gamma, beta, eps, dy, xt, part)
