@@ -65,7 +65,10 @@ def parse():
                     help="instead of the step: time kernels alone on the workload's shapes and print one "
                          "JSON line per kernel or input form (attention: contiguous keys and the compacted "
                          "per-user key lists of the workload's ids; history-backward: every step of one "
-                         "layer's history-side backward at the workload's d, h and history tokens)")
+                         "layer's history-side backward at the workload's d, h and history tokens; "
+                         "train-step: the whole training step by phase)")
+    ap.add_argument("--graph", action="store_true",
+                    help="train-step probe: time replays of the whole step captured as one CUDA graph")
     return ap.parse_args()
 
 
@@ -960,7 +963,20 @@ def run_probe_train_step(args):
         once()
     torch.cuda.synchronize()
     times = {k: [] for k in ("history forward", "target forward", "backward", "step")}
-    for _ in range(3 * args.steps):
+    if args.graph:  # the whole step as one CUDA graph: only the step's time
+        graph, _ = step.capture(ids, dt, hoff, toff, table, dt_table, n_items, dZ, dtable, ddt)
+        times = {"step (graph)": []}
+        for _ in range(max(args.warmup, 1)):
+            graph.replay()
+        torch.cuda.synchronize()
+        for _ in range(3 * args.steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            times["step (graph)"].append(e0.elapsed_time(e1))
+    for _ in range(0 if args.graph else 3 * args.steps):
         ev = once()
         torch.cuda.synchronize()
         for k, (a, b) in zip(times, ((0, 1), (1, 2), (2, 3), (0, 3))):
@@ -973,7 +989,7 @@ def run_probe_train_step(args):
         line = {"probe": "train-step", "phase": name, "workload": args.workload, "users": Bu, "history_tokens": N,
                 "targets": T, "d": d, "layers": cfg["M"], "score": cfg["score"], "median_ms": round(ms, 4),
                 "runs": len(ts)}
-        if name == "step":
+        if name.startswith("step"):
             f = sum(flops.values())
             tf = f / ms / 1e9
             line.update(flop=f, flop_attention=flops["attention"], achieved_tflops=round(tf, 1), peak_tflops=peak,

@@ -253,6 +253,23 @@ class StcaTrainingStep:
         self.forward_target(hoff, toff)
         return self.backward(ids, dt, hoff, toff, n_items, dZ, dtable, ddt_table)
 
+    def capture(self, ids, dt, hoff, toff, table, dt_table, n_items, dZ, dtable, ddt_table=None):
+        """Records one whole step (``run`` on the same buffers) as a CUDA graph: the step is a
+        few hundred launches, most of them small on the target side, and replaying them as
+        one graph removes the per-launch host work.  One eager step runs first, on the
+        capture stream (so the caching allocator has every buffer).  Returns (graph, grads):
+        ``graph.replay()`` recomputes ``grads`` in place; like ``run`` it adds the table rows'
+        gradients into dtable (and ddt_table) on every replay."""
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.run(ids, dt, hoff, toff, table, dt_table, n_items, dZ, dtable, ddt_table)
+        torch.cuda.current_stream().wait_stream(s)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            grads = self.run(ids, dt, hoff, toff, table, dt_table, n_items, dZ, dtable, ddt_table)
+        return graph, grads
+
     def forward_history(self, ids, dt, table, dt_table, n_items):
         """Every layer's history side recomputed: the rows X, A, P, y, Xt = LN(y) and the K/V rows."""
         d, M, N, w = self.d, self.M, self.N, self.w

@@ -85,3 +85,46 @@ def test_training_step_matches_oracle(config, kw):
     worst = max(errs, key=errs.get)
     print(f"training step: worst {worst} {errs[worst]:.2e};", {k: f"{v:.1e}" for k, v in errs.items()})
     assert errs[worst] <= TOL, errs
+
+
+def test_training_step_replays_as_one_cuda_graph():
+    """The whole step captured as a CUDA graph (StcaTrainingStep.capture) gives the eager
+    step's weight gradients bit for bit (every reduction runs in a fixed order) and its
+    table gradient up to the order of the lookup scatter's atomics."""
+    wl = make_stca(2, users=3, L=600, n_items=2000)
+    cfg = wl["cfg"]
+    d = cfg["d"]
+    lengths, tpu = wl["lengths"], wl["targets_per_user"]
+    Bu, N, T = len(lengths), int(lengths.sum()), int(tpu.sum())
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.int32)).to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    hoff, toff = torch.empty(Bu + 1, dtype=torch.int32, device=dev), torch.empty(Bu + 1, dtype=torch.int32, device=dev)
+    B.check(B.stca_k_offsets(i32(lengths), Bu, hoff, N, err))
+    B.check(B.stca_k_offsets(i32(tpu), Bu, toff, T, err))
+    up16 = lambda bits: torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+    table = up16(wl["table"])
+    n_items = int(wl["table"].shape[0])
+    step = StcaTrainingStep(cfg, device_weights(wl["weights"]), Bu, N, T)
+    step.x_t_slot().copy_(up16(wl["x_t"]).float())
+    ids = i32(wl["ids"])
+    dZ = torch.from_numpy(np.random.default_rng(4).standard_normal((T, d)).astype(np.float32)).to(dev)
+    dtab = torch.zeros((n_items, d), device=dev)
+    eager = step.run(ids, None, hoff, toff, table, None, n_items, dZ, dtab)
+    flat = lambda g: [t.clone() for t in _leaves(g)]
+    ref, ref_tab = flat(eager), dtab.clone()
+    graph, grads = step.capture(ids, None, hoff, toff, table, None, n_items, dZ, dtab)
+    dtab.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert step.err.item() == 0
+    for a, b in zip(flat(grads), ref):
+        assert torch.equal(a, b)
+    assert torch.allclose(dtab, ref_tab, rtol=0, atol=1e-6 * float(ref_tab.abs().max()))
+
+
+def _leaves(g):
+    if isinstance(g, dict):
+        return [t for k in sorted(g) for t in _leaves(g[k])]
+    if isinstance(g, (list, tuple)):
+        return [t for x in g for t in _leaves(x)]
+    return [] if g is None else [g]
