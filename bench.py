@@ -761,7 +761,10 @@ def run_probe_attention(args):
     values beyond the rare rescales), timed with CUDA events around each launch after
     warm-up; the median of 3 x steps launches.  "contiguous": every user's keys are its own
     consecutive K/V rows; "compacted": the per-user distinct keys of the workload's ids,
-    gathered by row from the call's distinct-key K/V matrix and weighted by their counts."""
+    gathered by row from the call's distinct-key K/V matrix and weighted by their counts.
+    "backward": the training backward (stca_attention_backward, bf16 K/V gradients) over the
+    contiguous keys, from the training forward's output and log-sum-exp; its bytes are the
+    K/V read and the K/V gradients written (8 d per key) plus the query-side rows."""
     import statistics
     import numpy as np
     import torch
@@ -801,10 +804,20 @@ def run_probe_attention(args):
     pm = torch.empty((1, T, H, 2), device=dev)
     out = torch.empty((T, d), device=dev)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
+    # the training backward over the contiguous keys: the forward's output and lse first
+    out_t = torch.empty((T, d), device=dev)
+    lse_t = torch.empty((T, H), device=dev)
+    B.check(B.stca_attention_train_forward(Q, KVc, hoff_c, toff_t, Bu, T, d, H, 1, 0, pa, pm, out_t, lse_t, err))
+    dO = torch.randn((T, d), device=dev, generator=g)
+    dQ = torch.empty((T, d), device=dev)
+    dKV = torch.empty((n_att, 2 * d), device=dev)
+    dKV16 = torch.empty((n_att, 2 * d), dtype=torch.bfloat16, device=dev)
     modes = {
         "contiguous": lambda: B.stca_k_attention(1, Q, KVc, hoff_c, toff_t, Bu, T, d, H, 1, 0, pa, pm, out, err),
         "compacted": lambda: B.stca_k_attention_rows(1, Q, KVu, hoff_t, toff_t, rows_t, lens_t, mult_t, Bu, T, d, H,
                                                      1, 0, pa, pm, out, err),
+        "backward": lambda: B.stca_attention_backward(Q, KVc, hoff_c, toff_t, Bu, T, d, H, 1, 0, out_t, lse_t, dO, dQ,
+                                                      dKV, None, dKV16=dKV16),
     }
     peaks = load_peaks()
     times = {k: [] for k in modes}
@@ -823,12 +836,15 @@ def run_probe_attention(args):
             times[k] += [e0.elapsed_time(e1) for e0, e1 in ev]
     assert int(err.item()) == 0
     work = n_att * H * 4 * (d // H) + 2 * T * d * 4  # attended K/V segments + queries and outputs
+    # backward: K/V read and their gradients written (bf16), Q, O, dO read and dQ written
+    work_bwd = n_att * 8 * d + 4 * T * d * 4
     for k in modes:
         ms = statistics.median(times[k])
-        gbs = work / ms / 1e6
+        w_k = work_bwd if k == "backward" else work
+        gbs = w_k / ms / 1e6
         print(json.dumps({"probe": "attention", "mode": k, "users": Bu, "attended_keys": n_att,
                           "distinct_keys": int(U), "ids": "uniform" if args.uniform_ids else "zipf",
-                          "median_ms": round(ms, 4), "launches": len(times[k]), "work_bytes": work,
+                          "median_ms": round(ms, 4), "launches": len(times[k]), "work_bytes": w_k,
                           "achieved_gbs": round(gbs, 1), "peak_gbs": peaks["hbm_gbs"],
                           "frac": round(gbs / peaks["hbm_gbs"], 4)}), flush=True)
 
