@@ -226,19 +226,22 @@ def _torch_mha(d, H, WQ, WK, WV, WO):
     return mha
 
 
-@pytest.mark.parametrize("score_layers", [1, 2])
+@pytest.mark.parametrize("score_layers", [1, 2, 3])
 def test_stca_score_path_vs_torch_multihead_attention(score_layers):
     """Each layer's o^(i) is standard multi-head attention of the one query q^(i) over the
     user's X~^(i) ([review] 核心公式: alpha = softmax(q W_Q (X~ W_K)^T / sqrt(d_h)),
     o = alpha X~ W_V, heads joined by W_O).  torch.nn.MultiheadAttention does the
     projections, the head split and the 1/sqrt(d_h) scale itself, so a wrong scale, a
     swapped W_Q/W_K or a wrong head slice in the oracle fails here.  LayerNorm and SiLU
-    come from torch's functional ops."""
+    come from torch's functional ops.  The chain is followed to the model's output z
+    ([review] architecture tree: z from [o^(1) | ... | o^(M) | x_t] W_Z through the z
+    SwiGLU), so with three layers the order of several o blocks in the concatenations,
+    the fusion of each layer and W_Z are pinned too."""
     d, H, L = 64, 4, 7
     wl = make_stca(2, users=1, lengths=np.array([L], np.int32), n_items=100, d=d, H=H, hidden=128, m=2,
                    M=score_layers)
     cfg, w = wl["cfg"], wl["weights"]
-    _, o = R.stca_forward(wl)
+    z, o = R.stca_forward(wl)
     t = lambda a: torch.from_numpy(_f64(a))
 
     def ln_swiglu(x, f, ln=True):
@@ -258,6 +261,8 @@ def test_stca_score_path_vs_torch_multihead_attention(score_layers):
             np.testing.assert_allclose(o[i, k], outs[-1].numpy(), rtol=1e-11, atol=1e-12)
             if i + 1 < score_layers:
                 q = ln_swiglu(torch.cat(outs + [x_t]) @ t(w["WC"][i + 1]), w["fuse"][i + 1])
+        zk = ln_swiglu(torch.cat(outs + [x_t]) @ t(w["WZ"]), w["zffn"], ln=False)
+        np.testing.assert_allclose(z[k], zk.numpy(), rtol=1e-11, atol=1e-12)
 
 
 def test_rlb_batched_equals_independent_targets():
